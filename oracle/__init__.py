@@ -1,0 +1,241 @@
+"""fp64 CPU oracle for RoPE + grouped-query KV-cache attention and the
+lightning-indexer sparse path.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may import this package.
+The CUDA product path never imports it, and it imports nothing from the
+product package: the two are independent statements of the same method.
+
+All arrays are numpy.  bf16 inputs are passed as ``np.uint16`` bit patterns
+(widened exactly inside the C code); fp64 inputs as ``np.float64``.  Results
+are fp64.  Each wrapper names the C function it calls; the C file cites the
+passage of the pages each one restates.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+NONE, PI, NTK, YARN, DYN_NTK = 0, 1, 2, 3, 4
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        i32, i64, dbl, vp = ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+        L.oracle_rope_freqs.argtypes = [i32, dbl, i32, dbl, dbl, dbl, dbl, dbl, vp, vp, vp]
+        L.oracle_yarn_gamma.argtypes = [i32, dbl, dbl, dbl, dbl, vp]
+        L.oracle_rope_table.argtypes = [i32, dbl, i32, dbl, dbl, dbl, dbl, dbl, i32, vp, vp]
+        L.oracle_rope_apply.argtypes = [i32, vp, i32, i32, i32, i64, i64, i64, vp, vp, vp, i32, i32,
+                                        i32, vp]
+        L.oracle_attn_decode.argtypes = [i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, dbl, i32, vp,
+                                         vp, vp, i32]
+        L.oracle_attn_prefill.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, dbl, i32, vp,
+                                          vp, vp, i32]
+        L.oracle_softmax_merge.argtypes = [i32, i32, vp, vp, vp, vp]
+        L.oracle_dsa_scores.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp, i32]
+        L.oracle_topk.argtypes = [vp, i32, i32, vp]
+        L.oracle_topk_rows.argtypes = [vp, vp, i32, i32, i32, vp, i32]
+        L.oracle_attn_sparse.argtypes = [i32, vp, vp, vp, i32, i32, i32, i32, i32, i32, dbl, vp, vp,
+                                         i32]
+        L.oracle_kv_cache_bytes_per_token.argtypes = [i32, i32, i32, i32]
+        L.oracle_kv_cache_bytes_per_token.restype = i64
+        L.oracle_latent_cache_bytes_per_token.argtypes = [i32, i32, i32, i32]
+        L.oracle_latent_cache_bytes_per_token.restype = i64
+        L.oracle_max_threads.restype = i32
+        _lib = L
+    return _lib
+
+
+def max_threads() -> int:
+    return lib().oracle_max_threads()
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _src(x):
+    """(dtype flag, contiguous array) for a bf16-bits or fp64 input."""
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        return 0, x
+    if x.dtype == np.float64:
+        return 1, x
+    raise TypeError(f"oracle inputs are uint16 (bf16 bits) or float64, got {x.dtype}")
+
+
+def _check(rc, fn):
+    if rc != 0:
+        raise ValueError(f"{fn} rejected its arguments (rc={rc})")
+
+
+def rope_freqs(d, base, scaling=NONE, s=1.0, L_train=0.0, alpha=1.0, beta=32.0, L_cur=0.0):
+    """-> (theta [d/2], position divisor, cos/sin magnitude).  oracle_rope_freqs."""
+    theta = np.zeros(d // 2, np.float64)
+    pos_div = np.zeros(1, np.float64)
+    mag = np.zeros(1, np.float64)
+    _check(lib().oracle_rope_freqs(d, base, scaling, s, L_train, alpha, beta, L_cur, _p(theta),
+                                   _p(pos_div), _p(mag)), "oracle_rope_freqs")
+    return theta, float(pos_div[0]), float(mag[0])
+
+
+def yarn_gamma(d, base, L_train, alpha=1.0, beta=32.0):
+    g = np.zeros(d // 2, np.float64)
+    _check(lib().oracle_yarn_gamma(d, base, L_train, alpha, beta, _p(g)), "oracle_yarn_gamma")
+    return g
+
+
+def rope_table(d, base, max_pos, scaling=NONE, s=1.0, L_train=0.0, alpha=1.0, beta=32.0, L_cur=0.0):
+    """-> (cos, sin), each [max_pos, d/2] fp64.  oracle_rope_table."""
+    c = np.zeros((max_pos, d // 2), np.float64)
+    sn = np.zeros((max_pos, d // 2), np.float64)
+    _check(lib().oracle_rope_table(d, base, scaling, s, L_train, alpha, beta, L_cur, max_pos, _p(c),
+                                   _p(sn)), "oracle_rope_table")
+    return c, sn
+
+
+def rope_apply(x, pos, cos, sin, pair_style=0, layout="bthd"):
+    """Rotate head vectors.  x: [B, T, H, d] (layout 'bthd') or [B, H, T, d]
+    (layout 'bhtd'); pos: [B, T] int32.  Returns fp64 in the same layout."""
+    flag, x = _src(x)
+    if layout == "bthd":
+        B, T, H, d = x.shape
+        sb, st, sh = T * H * d, H * d, d
+    elif layout == "bhtd":
+        B, H, T, d = x.shape
+        sb, st, sh = H * T * d, d, T * d
+    else:
+        raise ValueError(layout)
+    pos = np.ascontiguousarray(pos, dtype=np.int32).reshape(B, T)
+    cos = np.ascontiguousarray(cos, np.float64)
+    sin = np.ascontiguousarray(sin, np.float64)
+    y = np.zeros((B, T, H, d), np.float64)
+    _check(lib().oracle_rope_apply(flag, _p(x), B, T, H, sb, st, sh, _p(pos), _p(cos), _p(sin),
+                                   cos.shape[0], d, pair_style, _p(y)), "oracle_rope_apply")
+    return y if layout == "bthd" else np.ascontiguousarray(y.transpose(0, 2, 1, 3))
+
+
+def attn_decode(q, k, v, seq_lens, scale, sel=None, nthreads=0):
+    """q [B,H,d], k/v [B,Hk,T_max,d] -> (out, lse).  sel: optional [(b,h), ...]."""
+    fq, q = _src(q)
+    fk, k = _src(k)
+    fv, v = _src(v)
+    if not (fq == fk == fv):
+        raise TypeError("q, k, v must share a dtype")
+    B, H, d = q.shape
+    _, Hk, T_max, _ = k.shape
+    lens = np.ascontiguousarray(seq_lens, np.int32)
+    if sel is None:
+        out = np.zeros((B, H, d), np.float64)
+        lse = np.zeros((B, H), np.float64)
+        n_sel, selp = 0, None
+    else:
+        s = np.ascontiguousarray(np.asarray(sel, np.int32).reshape(-1, 2))
+        n_sel, selp = s.shape[0], _p(s)
+        out = np.zeros((n_sel, d), np.float64)
+        lse = np.zeros(n_sel, np.float64)
+    _check(lib().oracle_attn_decode(fq, _p(q), _p(k), _p(v), _p(lens), B, H, Hk, d, T_max, scale,
+                                    n_sel, selp, _p(out), _p(lse), nthreads), "oracle_attn_decode")
+    return out, lse
+
+
+def attn_prefill(q, k, v, scale, sel=None, nthreads=0):
+    """q [B,T,H,d], k/v [B,Hk,T,d] -> (out [B,T,H,d], lse [B,H,T]) or, with
+    sel = [(b,h,i), ...], (out [n,d], lse [n])."""
+    fq, q = _src(q)
+    fk, k = _src(k)
+    fv, v = _src(v)
+    if not (fq == fk == fv):
+        raise TypeError("q, k, v must share a dtype")
+    B, T, H, d = q.shape
+    Hk = k.shape[1]
+    if sel is None:
+        out = np.zeros((B, T, H, d), np.float64)
+        lse = np.zeros((B, H, T), np.float64)
+        n_sel, selp = 0, None
+    else:
+        s = np.ascontiguousarray(np.asarray(sel, np.int32).reshape(-1, 3))
+        n_sel, selp = s.shape[0], _p(s)
+        out = np.zeros((n_sel, d), np.float64)
+        lse = np.zeros(n_sel, np.float64)
+    _check(lib().oracle_attn_prefill(fq, _p(q), _p(k), _p(v), B, T, H, Hk, d, scale, n_sel, selp,
+                                     _p(out), _p(lse), nthreads), "oracle_attn_prefill")
+    return out, lse
+
+
+def softmax_merge(o, lse):
+    o = np.ascontiguousarray(o, np.float64)
+    lse = np.ascontiguousarray(lse, np.float64)
+    n, d = o.shape
+    out = np.zeros(d, np.float64)
+    ol = np.zeros(1, np.float64)
+    _check(lib().oracle_softmax_merge(n, d, _p(o), _p(lse), _p(out), _p(ol)), "oracle_softmax_merge")
+    return out, float(ol[0])
+
+
+def dsa_scores(q_idx, w, k_idx, lens, nthreads=0):
+    """q_idx [B,H_I,d_I] uint16, w [B,H_I] float32, k_idx [B,L_max,d_I] uint16
+    -> scores [B, L_max] fp64 (-inf past each length)."""
+    q_idx = np.ascontiguousarray(q_idx, np.uint16)
+    k_idx = np.ascontiguousarray(k_idx, np.uint16)
+    w = np.ascontiguousarray(w, np.float32)
+    B, HI, dI = q_idx.shape
+    L_max = k_idx.shape[1]
+    lens = np.ascontiguousarray(lens, np.int32)
+    sc = np.zeros((B, L_max), np.float64)
+    _check(lib().oracle_dsa_scores(_p(q_idx), _p(w), _p(k_idx), _p(lens), B, HI, dI, L_max, _p(sc),
+                                   nthreads), "oracle_dsa_scores")
+    return sc
+
+
+def topk(scores, k, lens=None, nthreads=0):
+    """Row-wise top-k of scores [B, L_max] (fp32 or fp64, widened exactly):
+    (score desc, index asc), -1 padded.  -> int32 [B, k]."""
+    sc = np.ascontiguousarray(np.asarray(scores).astype(np.float64))
+    if sc.ndim == 1:
+        sc = sc[None]
+    B, L_max = sc.shape
+    lens = np.full(B, L_max, np.int32) if lens is None else np.ascontiguousarray(lens, np.int32)
+    idx = np.zeros((B, k), np.int32)
+    _check(lib().oracle_topk_rows(_p(sc), _p(lens), B, L_max, k, _p(idx), nthreads),
+           "oracle_topk_rows")
+    return idx
+
+
+def attn_sparse(q, latent, idx, Dv, scale, nthreads=0):
+    """q [B,Hq,Dk], latent [B,L_max,Dk], idx [B,k] int32 (-1 skipped)
+    -> (out [B,Hq,Dv], lse [B,Hq])."""
+    fq, q = _src(q)
+    fc, latent = _src(latent)
+    if fq != fc:
+        raise TypeError("q and latent must share a dtype")
+    B, Hq, Dk = q.shape
+    L_max = latent.shape[1]
+    idx = np.ascontiguousarray(idx, np.int32)
+    k = idx.shape[1]
+    out = np.zeros((B, Hq, Dv), np.float64)
+    lse = np.zeros((B, Hq), np.float64)
+    _check(lib().oracle_attn_sparse(fq, _p(q), _p(latent), _p(idx), B, Hq, Dk, Dv, L_max, k, scale,
+                                    _p(out), _p(lse), nthreads), "oracle_attn_sparse")
+    return out, lse
+
+
+def kv_cache_bytes_per_token(n_layer, n_kv_head, d_head, bytes_per_elem=2):
+    return int(lib().oracle_kv_cache_bytes_per_token(n_layer, n_kv_head, d_head, bytes_per_elem))
+
+
+def latent_cache_bytes_per_token(n_layer, d_c, d_rope, bytes_per_elem=2):
+    return int(lib().oracle_latent_cache_bytes_per_token(n_layer, d_c, d_rope, bytes_per_elem))
+
+
+def bf16_bits_to_f64(bits):
+    """Exact widening of bf16 bit patterns (uint16) to float64."""
+    bits = np.ascontiguousarray(bits, np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
