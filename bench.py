@@ -1,0 +1,393 @@
+#!/usr/bin/env python3
+"""Benchmark of the RoPE + grouped-query KV-cache decode path on B200.
+
+Headline workload: the Llama-3-8B-shaped single-layer decode (B=16, n_head=32,
+n_kv_head=8, d=128, ragged cache lengths uniform in [1024, 8192], RoPE base
+500000).  One step = rope_apply_qk on the batch's new queries (each at
+position len_b; cached keys were rotated when written) + attn_decode_gqa.
+Metric: effective HBM GB/s = algorithmic bytes (K/V rows read once, q read,
+out and lse written) / step time; also tokens/s (= B / step time).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvattn|reference]
+With --gpus N > 1 (launched by torch.distributed.run) every rank decodes its
+own batch (weak scaling, no collective on the data path); value = bytes of
+all ranks / max-over-ranks time.  --impl reference times the fp64 CPU oracle
+on the host cores on a bounded sample of the same workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mqa_kv_cache_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode-attn effective HBM GB/s (% of peak) & tok/s; prefill TFLOP/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def decode_bytes(w, lens):
+    """Algorithmic bytes of one decode over the batch: every valid K and V row
+    once, the queries, the outputs and the lse values."""
+    kv = int(lens.sum()) * w.Hk * w.d * 2 * 2
+    return kv + w.B * w.H * w.d * 2 * 2 + w.B * w.H * 4
+
+
+# ---------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index, period=0.005):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------- GPU arm
+
+class DecodeStep:
+    """Device-resident decode workload; step() = rope on q + decode."""
+
+    def __init__(self, K, w, device, seed):
+        self.K, self.w = K, w
+        inp = W.decode_inputs(w, device=device, seed=seed, lens=W.lengths(w.B, w.T_lo, w.T_hi, seed))
+        r = w.rope
+        p = K.rope_params(w.d, base=r.base, scaling=r.scaling, s=r.s, L_train=r.L_train, alpha=r.alpha,
+                          beta=r.beta)
+        self.cos, self.sin = K.rope_table_build(p, w.T_max + 1, device=device)
+        self.k, self.v = inp["k"], inp["v"]
+        # cached keys are rotated once, when they are written to the cache
+        K.rope_apply_qk(None, None, self.k, inp["k_pos"].to(device), self.cos, self.sin, k_layout="bhtd")
+        self.q_raw = inp["q"]
+        self.q = inp["q"].clone()
+        self.lens = inp["seq_lens"].to(device)
+        self.lens_host = inp["seq_lens"].clone()
+        self.q_pos = inp["q_pos"].to(device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((w.B, w.H), dtype=torch.float32, device=device)
+        self.ws = K.workspace(K.attn_decode_gqa_workspace_bytes(w.B, w.H, w.Hk, w.d, w.T_max), device)
+        self.bytes = decode_bytes(w, inp["seq_lens"])
+        self.launches_per_step = 3  # rope_apply, decode, merge
+
+    def reset_q(self):
+        self.q.copy_(self.q_raw)
+
+    def rope(self):
+        self.K.rope_apply_qk(self.q, self.q_pos, None, None, self.cos, self.sin, q_layout="bhd")
+
+    def attn(self):
+        self.K.attn_decode_gqa(self.q, self.k, self.v, self.lens, self.w.scale, out=self.out, lse=self.lse,
+                               ws=self.ws)
+
+    def step(self):
+        self.rope()
+        self.attn()
+
+
+def capture(fn):
+    """Capture fn() (launches on the current stream) as a CUDA graph."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_steps(fn, steps, flush, before=None):
+    """Per-step CUDA-event times (ms) on the current stream, L2 flushed between steps."""
+    st = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        if before is not None:
+            before()
+        flush.zero_()
+        a.record(st)
+        fn()
+        b.record(st)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def run_gpu(args, rank, world, device):
+    from mqa_kv_cache_b200 import kvattn as K
+    peaks = load_peaks()
+    w = W.LLAMA3_8B_DECODE
+    seed = W.SEED_BASE + w.index + rank
+    job = DecodeStep(K, w, device, seed)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    for _ in range(args.warmup):
+        job.reset_q()
+        job.step()
+    torch.cuda.synchronize()
+    # the step and the attention alone, captured once as CUDA graphs
+    step_graph = capture(job.step)
+    attn_graph = capture(job.attn)
+    for _ in range(args.warmup):
+        job.reset_q()
+        step_graph.replay()
+        attn_graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K whole steps (graph replays, L2 flushed in between) ----
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device() if device.index is None else device.index)
+    with sampler:
+        step_ms = time_steps(step_graph.replay, args.steps, flush, before=job.reset_q)
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(float(np.mean(step_ms)), world, device)
+
+    # ---- dominant kernel alone (decode + merge launches), same stream ----
+    attn_ms = max_over_ranks(float(np.mean(time_steps(attn_graph.replay, args.steps, flush))), world, device)
+    # the same step launched eagerly from Python (host launch path included)
+    eager_ms = max_over_ranks(float(np.mean(time_steps(job.step, args.steps, flush, before=job.reset_q))),
+                              world, device)
+
+    # ---- end to end through the public API with host buffers ----
+    q_host = job.q_raw.cpu().pin_memory()
+    pos_host = job.q_pos.cpu().pin_memory()
+    lens_host = job.lens_host.pin_memory()
+    out_host = torch.empty(job.out.shape, dtype=torch.bfloat16).pin_memory()
+    lse_host = torch.empty(job.lse.shape, dtype=torch.float32).pin_memory()
+
+    def e2e():
+        job.q.copy_(q_host, non_blocking=True)
+        job.q_pos.copy_(pos_host, non_blocking=True)
+        job.lens.copy_(lens_host, non_blocking=True)
+        job.step()
+        out_host.copy_(job.out, non_blocking=True)
+        lse_host.copy_(job.lse, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e()
+    e2e_ms = max_over_ranks(float(np.mean(time_steps(e2e, args.steps, flush))), world, device)
+    h2d = q_host.numel() * 2 + pos_host.numel() * 4 + lens_host.numel() * 4
+    d2h = out_host.numel() * 2 + lse_host.numel() * 4
+
+    total_bytes = job.bytes * world
+    gbs = total_bytes / (ms * 1e-3) / 1e9
+    attn_gbs = job.bytes / (attn_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": round(gbs, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 q/k/v, ragged lengths U[1024,8192])",
+        "config": {"workload": w.name, "B": w.B, "n_head": w.H, "n_kv_head": w.Hk, "head_dim": w.d,
+                   "T_max": w.T_max, "mean_len": float(job.lens_host.float().mean()), "rope_base": w.rope.base,
+                   "parallelism": f"dp{world} (independent batches)",
+                   "l2": "flushed between timed steps (256 MB write), and inputs exceed L2"},
+        "tok_per_s": round(w.B * world / (ms * 1e-3), 1),
+        "step_launch": "CUDA graph replay (eager Python launch: %.4f ms/step)" % eager_ms,
+        "pct_of_hbm_peak": round(100.0 * gbs / world / peaks["hbm_gbs"], 2),
+        "pct_of_nominal_8tbs": round(100.0 * gbs / world / 8000.0, 2),
+        "roofline": {"kernel": "attn_decode_gqa (split-K decode + merge)", "bound": "hbm",
+                     "achieved": round(attn_gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(attn_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "peak_source": peaks["source"], "algorithmic_bytes": job.bytes},
+        "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": job.launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    return line
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def oracle_decode_sample(w, n_units, seed, nthreads):
+    """(seconds, algorithmic bytes) of the fp64 oracle on the first n_units
+    (batch, head) pairs of the workload."""
+    import oracle
+    inp = W.decode_inputs(w, seed=seed, lens=W.lengths(w.B, w.T_lo, w.T_hi, seed))
+    qb, kb, vb = W.bf16_bits(inp["q"]), W.bf16_bits(inp["k"]), W.bf16_bits(inp["v"])
+    lens = inp["seq_lens"].numpy()
+    sel = [(u // w.H, u % w.H) for u in range(n_units)]
+    t0 = time.perf_counter()
+    oracle.attn_decode(qb, kb, vb, lens, w.scale, sel=sel, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    nbytes = sum(int(lens[b]) * w.d * 2 * 2 + w.d * 2 * 2 + 4 for b, _ in sel)
+    return dt, nbytes, (qb, kb, vb, lens, sel)
+
+
+def cpu_baseline(budget_s=20.0):
+    import oracle
+    w = W.LLAMA3_8B_DECODE
+    nthreads = oracle.max_threads()
+    seed = W.SEED_BASE + w.index
+    dt, nbytes, (qb, kb, vb, lens, sel) = oracle_decode_sample(w, w.B * w.H, seed, nthreads)
+    reps, total_t = 1, dt
+    while total_t < min(budget_s, 10.0) and reps < 50:
+        t0 = time.perf_counter()
+        oracle.attn_decode(qb, kb, vb, lens, w.scale, sel=sel, nthreads=nthreads)
+        total_t += time.perf_counter() - t0
+        reps += 1
+    return {"value": round(nbytes * reps / total_t / 1e9, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+            "sample": f"full {w.name} batch ({w.B * w.H} (batch, head) outputs), {reps} passes, fp64"}
+
+
+def run_reference(args):
+    import oracle
+    w = W.LLAMA3_8B_DECODE
+    nthreads = oracle.max_threads()
+    seed = W.SEED_BASE + w.index
+    # size one step so that warmup + steps fit in about two minutes
+    dt_full, _, _ = oracle_decode_sample(w, w.B * w.H, seed, nthreads)
+    frac = min(1.0, 120.0 / max(1, args.steps + args.warmup) / max(dt_full, 1e-6))
+    n_units = max(1, int(frac * w.B * w.H))
+    inp = W.decode_inputs(w, seed=seed, lens=W.lengths(w.B, w.T_lo, w.T_hi, seed))
+    qb, kb, vb = W.bf16_bits(inp["q"]), W.bf16_bits(inp["k"]), W.bf16_bits(inp["v"])
+    lens = inp["seq_lens"].numpy()
+    sel = [(u // w.H, u % w.H) for u in range(n_units)]
+    nbytes = sum(int(lens[b]) * w.d * 2 * 2 + w.d * 2 * 2 + 4 for b, _ in sel)
+    for _ in range(args.warmup):
+        oracle.attn_decode(qb, kb, vb, lens, w.scale, sel=sel, nthreads=nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attn_decode(qb, kb, vb, lens, w.scale, sel=sel, nthreads=nthreads)
+    dt = (time.perf_counter() - t0) / max(1, args.steps)
+    val = nbytes / dt / 1e9
+    sample = f"{n_units} of {w.B * w.H} (batch, head) outputs of {w.name} per step, fp64"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (same seeded workload)",
+        "config": {"workload": w.name, "B": w.B, "n_head": w.H, "n_kv_head": w.Hk, "head_dim": w.d,
+                   "T_max": w.T_max, "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------------- distributed plumbing
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, world, device):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="kvattn", choices=["kvattn", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    line = run_gpu(args, rank, world, device)
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

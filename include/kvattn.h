@@ -1,0 +1,204 @@
+/*
+ * kvattn.h -- C ABI of the B200 (sm_100a) RoPE + grouped-query KV-cache
+ * attention library (libkvattn.so).
+ *
+ * Scope: causal attention of new queries over a KV cache, with RoPE applied
+ * to q and k only (plain, PI, NTK, YaRN and dynamic-NTK frequency scaling and
+ * the YaRN cos/sin temperature), MHA / GQA / MQA head grouping, and the
+ * lightning-indexer top-k + sparse latent-row decode.  Sources are cited per
+ * entry point by page title and section:
+ *   "Agentic RL 入门3：transformer 架构"        (RoPE §1.1-1.2, GQA §2.1, DSA §2.2, MLA §2.3)
+ *   "注意力变体与 MoE"                         (KV cache, decode roofline, GQA attention())
+ *   "attention"                               (GroupQueryAttention; DSA ①②③)
+ *   "注意力机制进化史：从MHA、MQA、GQA、MLA到NSA、MoBA！" (KV cache append, layer_past)
+ *
+ * Conventions (all entry points):
+ *  - Tensors are caller-owned DEVICE memory unless stated otherwise.  The
+ *    library never allocates or frees device memory; scratch space is the
+ *    caller's `workspace`, sized by the matching *_workspace_bytes() query.
+ *  - bf16 values are passed as their 16-bit patterns (kvattn_bf16).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and never synchronises the host.
+ *  - Every pointer to a tensor must be 16-byte aligned; the innermost
+ *    dimension is contiguous.  Shapes are in elements.
+ *  - Return value: KVATTN_OK (0) or a negative KVATTN_ERR_* code, with a
+ *    message in kvattn_last_error_string() (thread-local).  Argument errors
+ *    are detected on the host before anything is launched; on error nothing
+ *    is written.
+ *  - Values that only the device can see (positions, sequence lengths, top-k
+ *    indices) are range-checked inside the kernels: an out-of-range value is
+ *    never dereferenced; it is clamped or skipped as each entry point states,
+ *    and, when `dev_status` is non-NULL, the matching KVATTN_STATUS_* bit is
+ *    OR-ed into *dev_status (a device int32 the caller zeroes).
+ *  - Inputs are read-only unless the entry point says it writes them.
+ */
+#ifndef KVATTN_H
+#define KVATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t kvattn_bf16; /* bf16 bit pattern */
+
+/* ---- status ------------------------------------------------------------ */
+#define KVATTN_OK 0
+#define KVATTN_ERR_NULL (-1)        /* a required pointer is NULL */
+#define KVATTN_ERR_ALIGN (-2)       /* a pointer or stride breaks the 16-byte rule */
+#define KVATTN_ERR_SHAPE (-3)       /* inconsistent or out-of-range sizes */
+#define KVATTN_ERR_UNSUPPORTED (-4) /* valid but not implemented (e.g. head_dim) */
+#define KVATTN_ERR_CUDA (-5)        /* a CUDA runtime/driver call failed */
+#define KVATTN_ERR_WORKSPACE (-6)   /* workspace NULL or smaller than required */
+
+/* Device-side status bits (OR-ed into *dev_status). */
+#define KVATTN_STATUS_BAD_POSITION 0x1 /* a RoPE position outside [0, max_pos) */
+#define KVATTN_STATUS_BAD_LENGTH 0x2   /* a sequence length outside [0, T_max] */
+#define KVATTN_STATUS_BAD_INDEX 0x4    /* a top-k index outside [-1, L_max) */
+#define KVATTN_STATUS_NAN_SCORE 0x8    /* an indexer score was NaN */
+#define KVATTN_STATUS_TIMEOUT 0x10     /* a pipeline wait ran out of time; outputs are invalid */
+
+/* Message for the last error on the calling thread ("" when none). */
+const char* kvattn_last_error_string(void);
+
+/* Library version string. */
+const char* kvattn_version(void);
+
+/* ---- RoPE ----------------------------------------------------------------
+ * "Agentic RL 入门3：transformer 架构" §1.1 (rotation R(m, theta_i),
+ * theta_i = base^(-2i/d)), §1.2 ① PI, ② NTK-aware, ③ YaRN (NTK-by-parts
+ * ramp and attention temperature), ④ dynamic NTK.
+ */
+#define KVATTN_ROPE_NONE 0    /* theta_i = base^(-2i/d) */
+#define KVATTN_ROPE_PI 1      /* position m -> m / s */
+#define KVATTN_ROPE_NTK 2     /* base -> base * s^(d/(d-2)) */
+#define KVATTN_ROPE_YARN 3    /* ramp-blended theta, cos/sin x (0.1 ln s + 1) */
+#define KVATTN_ROPE_DYN_NTK 4 /* NTK with s = max(1, L_cur / L_train) */
+
+typedef struct kvattn_rope_params {
+    int head_dim;   /* d: even, 4 .. 256 */
+    int scaling;    /* KVATTN_ROPE_* */
+    int pair_style; /* 0: pairs (2i, 2i+1) (default); 1: pairs (i, i + d/2) */
+    int reserved;   /* must be 0 */
+    double base;    /* RoPE base b (10000, 500000, ...) */
+    double s;       /* extension factor s = L_new / L_train (PI, NTK, YaRN); >= 1 */
+    double L_train; /* training length (YaRN ramp, dynamic NTK) */
+    double alpha;   /* YaRN ramp lower edge (default 1): gamma = 0 for r <= alpha */
+    double beta;    /* YaRN ramp upper edge (default 32): gamma = 1 for r > beta */
+    double L_cur;   /* current length (dynamic NTK only) */
+} kvattn_rope_params;
+
+/*
+ * Build the cos/sin table: cos_out[m*(d/2) + i] = mag * cos((m/pdiv) * theta_i),
+ * sin_out likewise, for m in [0, max_pos), i in [0, d/2).  theta_i, the
+ * position divisor pdiv (s for PI, else 1) and the magnitude mag
+ * (0.1 ln s + 1 for YaRN, else 1) follow the scaling mode.  Angles are formed
+ * and evaluated in fp64 on the device; the table is stored as fp32.
+ * cos_out, sin_out: device fp32 [max_pos][d/2], written.  Errors:
+ * KVATTN_ERR_NULL, _SHAPE (max_pos < 1, bad d, s < 1, beta <= alpha,
+ * L_train <= 0 where needed), _UNSUPPORTED (unknown scaling or pair_style).
+ */
+int rope_table_build(const kvattn_rope_params* params, int max_pos, float* cos_out, float* sin_out,
+                     void* stream);
+
+/*
+ * Rotate q and k IN PLACE with a table from rope_table_build (v is never
+ * rotated: position enters only the score, §1.1 last paragraph).
+ * Each of q and k is a 4-D view [nb][nt][nh][d] with element (b,t,h,j) at
+ * x[b*sb + t*st + h*sh + j] (strides in elements, multiples of 8), and
+ * positions pos[b*nt + t] (device int32).  Examples: decode queries
+ * [B][H][d] -> (B, 1, H, d, H*d, 0, d); a cache [B][Hk][T][d] ->
+ * (B, T, Hk, d, Hk*T*d, d, T*d); prefill queries [B][T][H][d] ->
+ * (B, T, H, d, T*H*d, H*d, d).  Either of q or k may be NULL (skipped).
+ * For pair (a, b) with table entries (c, s): (x_a, x_b) ->
+ * (x_a c - x_b s, x_a s + x_b c), computed in fp32, stored as bf16 (RNE).
+ * A position outside [0, max_pos) leaves that vector unchanged and sets
+ * KVATTN_STATUS_BAD_POSITION.  head_dim: multiple of 16, <= 256.
+ */
+int rope_apply_qk(kvattn_bf16* q, int q_nb, int q_nt, int q_nh, int64_t q_sb, int64_t q_st,
+                  int64_t q_sh, const int32_t* q_pos, kvattn_bf16* k, int k_nb, int k_nt, int k_nh,
+                  int64_t k_sb, int64_t k_st, int64_t k_sh, const int32_t* k_pos,
+                  const float* cos_tab, const float* sin_tab, int max_pos, int head_dim,
+                  int pair_style, int32_t* dev_status, void* stream);
+
+/* ---- decode over a KV cache -----------------------------------------------
+ * One new query per sequence attends to every cached row: "注意力变体与 MoE"
+ * (decode reads all cached K/V; GQA attention()), "注意力机制进化史" (KV cache
+ * layer_past append), "attention" GroupQueryAttention (query head h uses KV
+ * head h / g, g = n_head / n_kv_head; n_kv_head = n_head is MHA, 1 is MQA).
+ *
+ * q [B][n_head][d]; k_cache, v_cache [B][n_kv_head][T_max][d] with rows
+ * 0 .. seq_lens[b]-1 valid (rows past the length are never used, whatever
+ * they hold); seq_lens device int32 [B].
+ * out [B][n_head][d] bf16 = softmax(scale * q k^T) v;
+ * lse [B][n_head] fp32 (natural log of the sum of exp(scale * q.k)), or NULL.
+ * A sequence of length 0 gives out = 0 and lse = -inf.  A length outside
+ * [0, T_max] is clamped into it and sets KVATTN_STATUS_BAD_LENGTH.
+ * workspace: device scratch of attn_decode_gqa_workspace_bytes(...) bytes
+ * (256-byte aligned); its contents need no initialisation.
+ * Supported: head_dim in {64, 128}; n_head % n_kv_head == 0 with
+ * g = n_head / n_kv_head in {1, 2, 4, 8, 16, 32, 64}; T_max >= 1.
+ */
+size_t attn_decode_gqa_workspace_bytes(int B, int n_head, int n_kv_head, int head_dim, int T_max);
+
+int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
+                    const int32_t* seq_lens, int B, int n_head, int n_kv_head, int head_dim,
+                    int T_max, float scale, kvattn_bf16* out, float* lse, void* workspace,
+                    size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ---- causal prefill ---------------------------------------------------------
+ * softmax(scale * q k^T + M) v with the lower-triangular mask M (key j is
+ * visible to query i iff j <= i): "注意力变体与 MoE" attention() (triu(1)
+ * filled with -inf), grouped as in decode.
+ * q [B][T][n_head][d]; k, v [B][n_kv_head][T][d]; out [B][T][n_head][d] bf16;
+ * lse [B][n_head][T] fp32 or NULL.  Supported: head_dim 128; g as in decode.
+ */
+int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B,
+                        int T, int n_head, int n_kv_head, int head_dim, float scale,
+                        kvattn_bf16* out, float* lse, void* stream);
+
+/* ---- lightning indexer + top-k ---------------------------------------------
+ * "Agentic RL 入门3" §2.2 (1): s_{b,t} = sum_{j < H_I} w[b][j] *
+ * ReLU(q_idx[b][j] . k_idx[b][t]) (no scale, no RoPE); §2.2 (2): S_b =
+ * TopK_t(s_{b,t}); "attention" DSA ① (64 heads, one key shared by all heads).
+ * q_idx [B][H_I][d_I] bf16; w [B][H_I] fp32; k_idx [B][L_max][d_I] bf16;
+ * seq_lens device int32 [B] or NULL (= L_max for every row).
+ * topk_idx [B][k] int32: the k largest scores of row b under the order
+ * (score descending, index ascending) -- ties go to the lower index -- listed
+ * in that order; min(k, len) entries, then -1.  The selection is made on the
+ * fp32 scores the kernel computed; scores_out [B][L_max] fp32 receives them
+ * (-inf past each length) when non-NULL.
+ * Supported: H_I = 64, d_I = 128, 1 <= k <= 2048, L_max >= 1.
+ */
+size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k);
+
+int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* k_idx,
+                   const int32_t* seq_lens, int B, int n_idx_head, int idx_dim, int L_max, int k,
+                   int32_t* topk_idx, float* scores_out, void* workspace, size_t workspace_bytes,
+                   int32_t* dev_status, void* stream);
+
+/* ---- sparse latent-row decode -------------------------------------------------
+ * "Agentic RL 入门3" §2.2 (2) o = MLA(q, {k_j, v_j : j in S}); "attention"
+ * DSA ② (after weight absorption every query head reads the same single-head
+ * latent rows: MQA over the selected rows) and the "乘法结合律" note
+ * ([1,128,576] queries).  Key row j = latent[b][j][0 .. Dk-1]; value row
+ * j = latent[b][j][0 .. Dv-1] (K and V share the latent, §2.3.5).
+ * q [B][Hq][Dk] bf16; latent [B][L_max][Dk] bf16; topk_idx [B][k] int32
+ * (-1 = unused slot; other values outside [0, L_max) are skipped and set
+ * KVATTN_STATUS_BAD_INDEX).  out [B][Hq][Dv] bf16; lse [B][Hq] fp32 or NULL.
+ * A row with no valid index gives out = 0, lse = -inf.
+ * Supported: Dk = 576, Dv = 512, Hq in {16, 32, 64, 128}, 1 <= k <= 2048.
+ */
+size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k);
+
+int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const int32_t* topk_idx,
+                       int B, int Hq, int Dk, int Dv, int L_max, int k, float scale,
+                       kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
+                       int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVATTN_H */

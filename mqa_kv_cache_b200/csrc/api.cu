@@ -1,0 +1,319 @@
+// api.cu -- the extern "C" boundary of libkvattn.so.
+//
+// Every entry point validates its arguments on the host (returning a
+// KVATTN_ERR_* code and a thread-local message before anything is launched),
+// lays out the caller's workspace, encodes TMA tensor maps where a kernel
+// streams through one, and launches on the caller's stream.  Nothing here
+// allocates device memory or synchronises the host.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok()
+{
+    g_err[0] = '\0';
+    return KVATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kWsAlign = 256;
+size_t align_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+// Per-device SM count, queried once.
+int num_sms_current(int* out)
+{
+    static std::mutex mu;
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 64) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        *out = n;
+        return 0;
+    }
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+        cache[dev] = n;
+    }
+    *out = cache[dev];
+    return 0;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor map over [z][y][x] (x innermost) with a {64, box_y, 1} box and
+// 128-byte swizzle; out-of-range rows read as zero.
+int make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint32_t box_y)
+{
+    auto fn = encode_fn();
+    if (!fn) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[3] = {x, y, z};
+    cuuint64_t strides[2] = {x * 2, x * y * 2};
+    cuuint32_t box[3] = {64, box_y, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return KVATTN_OK;
+}
+
+int cuda_status(cudaError_t e, const char* what)
+{
+    if (e != cudaSuccess) return fail(KVATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+bool g_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16 || g == 32 || g == 64; }
+
+// Decode workspace layout for a given grid.
+struct DecodeWs {
+    size_t off_o, off_ml, off_info, total;
+};
+
+DecodeWs decode_ws(int B, int n_head, int n_kv_head, int head_dim, int grid)
+{
+    const long long slots = kvattn::decode_max_slots(B, n_kv_head, grid);
+    const int g = n_head / n_kv_head;
+    DecodeWs w;
+    w.off_o = 0;
+    w.off_ml = align_up(static_cast<size_t>(slots) * g * head_dim * sizeof(float));
+    w.off_info = w.off_ml + align_up(static_cast<size_t>(slots) * g * 2 * sizeof(float));
+    w.total = w.off_info + align_up(static_cast<size_t>(B) * n_kv_head * sizeof(int2));
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvattn_last_error_string(void) { return g_err; }
+
+const char* kvattn_version(void) { return "kvattn 0.1.0 (sm_100a)"; }
+
+// ---------------------------------------------------------------------------
+int rope_table_build(const kvattn_rope_params* p, int max_pos, float* cos_out, float* sin_out, void* stream)
+{
+    if (!p || !cos_out || !sin_out) return fail(KVATTN_ERR_NULL, "rope_table_build: NULL argument");
+    if (p->reserved != 0) return fail(KVATTN_ERR_SHAPE, "rope_table_build: reserved must be 0");
+    if (p->head_dim < 4 || p->head_dim > 256 || (p->head_dim & 1))
+        return fail(KVATTN_ERR_SHAPE, "rope_table_build: head_dim %d must be even, 4..256", p->head_dim);
+    if (max_pos < 1) return fail(KVATTN_ERR_SHAPE, "rope_table_build: max_pos %d < 1", max_pos);
+    if (p->scaling < KVATTN_ROPE_NONE || p->scaling > KVATTN_ROPE_DYN_NTK)
+        return fail(KVATTN_ERR_UNSUPPORTED, "rope_table_build: unknown scaling %d", p->scaling);
+    if (p->pair_style != 0 && p->pair_style != 1)
+        return fail(KVATTN_ERR_UNSUPPORTED, "rope_table_build: pair_style %d", p->pair_style);
+    if (!(p->base > 0.0) || !std::isfinite(p->base)) return fail(KVATTN_ERR_SHAPE, "rope_table_build: base must be > 0");
+    const bool uses_s = p->scaling == KVATTN_ROPE_PI || p->scaling == KVATTN_ROPE_NTK || p->scaling == KVATTN_ROPE_YARN;
+    if (uses_s && !(p->s >= 1.0 && std::isfinite(p->s)))
+        return fail(KVATTN_ERR_SHAPE, "rope_table_build: s must be >= 1");
+    if ((p->scaling == KVATTN_ROPE_YARN || p->scaling == KVATTN_ROPE_DYN_NTK) && !(p->L_train > 0.0))
+        return fail(KVATTN_ERR_SHAPE, "rope_table_build: L_train must be > 0");
+    if (p->scaling == KVATTN_ROPE_YARN && !(p->beta > p->alpha))
+        return fail(KVATTN_ERR_SHAPE, "rope_table_build: beta must exceed alpha");
+    if (p->scaling == KVATTN_ROPE_DYN_NTK && !(p->L_cur >= 0.0))
+        return fail(KVATTN_ERR_SHAPE, "rope_table_build: L_cur must be >= 0");
+    if (static_cast<long long>(max_pos) * (p->head_dim / 2) > (1ll << 40))
+        return fail(KVATTN_ERR_SHAPE, "rope_table_build: table too large");
+    return cuda_status(kvattn::launch_rope_table(*p, max_pos, cos_out, sin_out, static_cast<cudaStream_t>(stream)),
+                       "rope_table_build launch");
+}
+
+// ---------------------------------------------------------------------------
+int rope_apply_qk(kvattn_bf16* q, int q_nb, int q_nt, int q_nh, int64_t q_sb, int64_t q_st, int64_t q_sh,
+                  const int32_t* q_pos, kvattn_bf16* k, int k_nb, int k_nt, int k_nh, int64_t k_sb, int64_t k_st,
+                  int64_t k_sh, const int32_t* k_pos, const float* cos_tab, const float* sin_tab, int max_pos,
+                  int head_dim, int pair_style, int32_t* dev_status, void* stream)
+{
+    if (!cos_tab || !sin_tab) return fail(KVATTN_ERR_NULL, "rope_apply_qk: NULL table");
+    if (head_dim < 16 || head_dim > 256 || head_dim % 16)
+        return fail(KVATTN_ERR_UNSUPPORTED, "rope_apply_qk: head_dim %d must be a multiple of 16, <= 256", head_dim);
+    if (pair_style != 0 && pair_style != 1) return fail(KVATTN_ERR_UNSUPPORTED, "rope_apply_qk: pair_style");
+    if (max_pos < 1) return fail(KVATTN_ERR_SHAPE, "rope_apply_qk: max_pos < 1");
+    if (!aligned16(cos_tab) || !aligned16(sin_tab)) return fail(KVATTN_ERR_ALIGN, "rope_apply_qk: table alignment");
+    struct V {
+        kvattn_bf16* x;
+        int nb, nt, nh;
+        int64_t sb, st, sh;
+        const int32_t* pos;
+        const char* name;
+    } views[2] = {{q, q_nb, q_nt, q_nh, q_sb, q_st, q_sh, q_pos, "q"}, {k, k_nb, k_nt, k_nh, k_sb, k_st, k_sh, k_pos, "k"}};
+    for (auto& v : views) {
+        if (!v.x) continue;
+        if (!v.pos) return fail(KVATTN_ERR_NULL, "rope_apply_qk: %s positions NULL", v.name);
+        if (v.nb < 0 || v.nt < 0 || v.nh < 0) return fail(KVATTN_ERR_SHAPE, "rope_apply_qk: negative %s size", v.name);
+        if (!aligned16(v.x)) return fail(KVATTN_ERR_ALIGN, "rope_apply_qk: %s not 16-byte aligned", v.name);
+        if (v.sb % 8 || v.st % 8 || v.sh % 8 || v.sb < 0 || v.st < 0 || v.sh < 0)
+            return fail(KVATTN_ERR_ALIGN, "rope_apply_qk: %s strides must be non-negative multiples of 8", v.name);
+        if (static_cast<long long>(v.nb) * v.nt * v.nh > (1ll << 40))
+            return fail(KVATTN_ERR_SHAPE, "rope_apply_qk: %s too large", v.name);
+    }
+    int sms = 0;
+    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "rope_apply_qk: no CUDA device");
+    kvattn::RopeApplyArgs a{};
+    a.q = q;
+    a.q_nb = q ? q_nb : 0;
+    a.q_nt = q_nt;
+    a.q_nh = q_nh;
+    a.q_sb = q_sb;
+    a.q_st = q_st;
+    a.q_sh = q_sh;
+    a.q_pos = q_pos;
+    a.k = k;
+    a.k_nb = k ? k_nb : 0;
+    a.k_nt = k_nt;
+    a.k_nh = k_nh;
+    a.k_sb = k_sb;
+    a.k_st = k_st;
+    a.k_sh = k_sh;
+    a.k_pos = k_pos;
+    a.cos_tab = cos_tab;
+    a.sin_tab = sin_tab;
+    a.max_pos = max_pos;
+    a.head_dim = head_dim;
+    a.pair_style = pair_style;
+    a.dev_status = dev_status;
+    a.num_sms = sms;
+    return cuda_status(kvattn::launch_rope_apply(a, static_cast<cudaStream_t>(stream)), "rope_apply_qk launch");
+}
+
+// ---------------------------------------------------------------------------
+size_t attn_decode_gqa_workspace_bytes(int B, int n_head, int n_kv_head, int head_dim, int T_max)
+{
+    (void)T_max;
+    if (B < 1 || n_head < 1 || n_kv_head < 1 || n_head % n_kv_head || head_dim < 1) return 0;
+    int sms = 0;
+    if (num_sms_current(&sms) != 0) return 0;
+    return decode_ws(B, n_head, n_kv_head, head_dim, kvattn::decode_grid(sms)).total;
+}
+
+int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
+                    const int32_t* seq_lens, int B, int n_head, int n_kv_head, int head_dim, int T_max, float scale,
+                    kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                    void* stream)
+{
+    if (!q || !k_cache || !v_cache || !seq_lens || !out)
+        return fail(KVATTN_ERR_NULL, "attn_decode_gqa: NULL argument");
+    if (B < 1 || B > kvattn::DECODE_MAX_B) return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: B %d outside 1..%d", B, kvattn::DECODE_MAX_B);
+    if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head)
+        return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: n_head %d not a multiple of n_kv_head %d", n_head, n_kv_head);
+    const int g = n_head / n_kv_head;
+    if (!g_supported(g)) return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: group size %d", g);
+    if (head_dim != 64 && head_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: head_dim %d", head_dim);
+    if (T_max < 1 || static_cast<long long>(B) * n_kv_head > (1ll << 31) - 1)
+        return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: T_max %d / batch too large", T_max);
+    if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: scale must be finite > 0");
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return fail(KVATTN_ERR_ALIGN, "attn_decode_gqa: tensors must be 16-byte aligned");
+    int sms = 0;
+    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "attn_decode_gqa: no CUDA device");
+    const int grid = kvattn::decode_grid(sms);
+    const DecodeWs ws = decode_ws(B, n_head, n_kv_head, head_dim, grid);
+    if (!workspace || workspace_bytes < ws.total)
+        return fail(KVATTN_ERR_WORKSPACE, "attn_decode_gqa: workspace needs %zu bytes", ws.total);
+    if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
+        return fail(KVATTN_ERR_ALIGN, "attn_decode_gqa: workspace must be 256-byte aligned");
+
+    CUtensorMap tm_k, tm_v;
+    const uint64_t units = static_cast<uint64_t>(B) * n_kv_head;
+    if (make_map_3d(&tm_k, k_cache, head_dim, T_max, units, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_3d(&tm_v, v_cache, head_dim, T_max, units, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
+
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    kvattn::DecodeArgs a{};
+    a.q = q;
+    a.seq_lens = seq_lens;
+    a.out = out;
+    a.lse = lse;
+    a.part_o = reinterpret_cast<float*>(w + ws.off_o);
+    a.part_ml = reinterpret_cast<float*>(w + ws.off_ml);
+    a.unit_info = reinterpret_cast<int2*>(w + ws.off_info);
+    a.dev_status = dev_status;
+    a.B = B;
+    a.H = n_head;
+    a.Hk = n_kv_head;
+    a.g = g;
+    a.d = head_dim;
+    a.T_max = T_max;
+    a.scale = scale;
+    a.grid = grid;
+    return cuda_status(kvattn::launch_decode(a, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
+                       "attn_decode_gqa launch");
+}
+
+// ---------------------------------------------------------------------------
+int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B, int T, int n_head,
+                        int n_kv_head, int head_dim, float scale, kvattn_bf16* out, float* lse, void* stream)
+{
+    (void)q, (void)k, (void)v, (void)B, (void)T, (void)n_head, (void)n_kv_head, (void)head_dim, (void)scale;
+    (void)out, (void)lse, (void)stream;
+    return fail(KVATTN_ERR_UNSUPPORTED, "attn_prefill_causal: not built yet");
+}
+
+size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k)
+{
+    (void)B, (void)L_max, (void)k;
+    return 0;
+}
+
+int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* k_idx, const int32_t* seq_lens, int B,
+                   int n_idx_head, int idx_dim, int L_max, int k, int32_t* topk_idx, float* scores_out,
+                   void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    (void)q_idx, (void)w, (void)k_idx, (void)seq_lens, (void)B, (void)n_idx_head, (void)idx_dim, (void)L_max, (void)k;
+    (void)topk_idx, (void)scores_out, (void)workspace, (void)workspace_bytes, (void)dev_status, (void)stream;
+    return fail(KVATTN_ERR_UNSUPPORTED, "dsa_index_topk: not built yet");
+}
+
+size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k)
+{
+    (void)B, (void)Hq, (void)Dv, (void)k;
+    return 0;
+}
+
+int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const int32_t* topk_idx, int B, int Hq, int Dk,
+                       int Dv, int L_max, int k, float scale, kvattn_bf16* out, float* lse, void* workspace,
+                       size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    (void)q, (void)latent, (void)topk_idx, (void)B, (void)Hq, (void)Dk, (void)Dv, (void)L_max, (void)k, (void)scale;
+    (void)out, (void)lse, (void)workspace, (void)workspace_bytes, (void)dev_status, (void)stream;
+    return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_sparse: not built yet");
+}
+
+}  // extern "C"

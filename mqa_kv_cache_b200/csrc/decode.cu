@@ -1,0 +1,579 @@
+// decode.cu -- one new query per sequence over a bf16 KV cache, all query
+// heads of a KV group served by a single read of each K/V tile.
+//
+// Method: softmax(scale q k^T) v per query head, query head h reading KV head
+// h / g ("注意力变体与 MoE", GQA attention(): the g heads of a group share one
+// K/V and a real kernel reads the shared block once; "attention",
+// GroupQueryAttention).  The cache is read exactly once: decode is bound by
+// HBM, with g FLOP per byte (same page, decode roofline).
+//
+// Work split (ragged, balanced by tiles, computed on the device from the
+// lengths): the cache rows of every (batch, kv-head) unit are cut into tiles
+// of 64 rows; all tiles of all units form one ordered list of N tiles; CTA c
+// of G = min(grid, N) CTAs owns tiles x with floor(x G / N) == c, a
+// contiguous range.  Where a range crosses units it produces one "piece" per
+// unit.  A unit that lies inside one CTA is finished there; otherwise every
+// piece writes an unnormalised partial (O, running max, sum) and a second
+// kernel merges the partials of the unit (the split-softmax identity).
+//
+// CTA: 4 consumer warps + 1 TMA producer warp.  K and V tiles [64 x d] land in
+// shared memory through a 3-D tensor map (d, T_max, B*Hk) with 128-byte
+// swizzle, STAGES deep, one mbarrier pair per stage.  Consumers run bf16
+// mma.sync m16n8k16 with the query heads of the group as the M rows (a group
+// of g <= 16 heads is one M tile, zero-padded; g = 32/64 use 2/4 M tiles),
+// fp32 accumulation, online softmax in base 2 with quad shuffles.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvattn {
+
+namespace {
+
+constexpr int TILE = 64;   // cache rows per pipeline stage
+constexpr int CWARPS = 4;  // consumer warps
+constexpr int THREADS = 32 * (CWARPS + 1);
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
+
+template <int D>
+struct Cfg {
+    static constexpr int STAGES = D == 128 ? 5 : 8;
+    static constexpr int HALVES = D / 64;  // 128-byte column blocks per row
+    static constexpr int TILE_BYTES = TILE * D * 2;
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K tile + V tile
+    static constexpr int SCR_STRIDE = D + 8;            // floats per scratch row
+    static constexpr int OFF_SCR_O = STAGES * STAGE_BYTES;
+    static constexpr int OFF_SCR_ML = OFF_SCR_O + CWARPS * 16 * SCR_STRIDE * 4;
+    static constexpr int OFF_N = OFF_SCR_ML + CWARPS * 16 * 2 * 4;
+    static constexpr int OFF_UB = OFF_N + DECODE_MAX_B * 4;
+    static constexpr int OFF_LEN = OFF_UB + (DECODE_MAX_B + 1) * 4;
+    static constexpr int OFF_BAR = ((OFF_LEN + DECODE_MAX_B * 4) + 7) / 8 * 8;
+    static constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+};
+
+// ---- work plan ------------------------------------------------------------------
+
+__device__ __forceinline__ int owner_of(long long x, long long N, int G)
+{
+    return static_cast<int>((x * G) / N);
+}
+
+__device__ __forceinline__ long long range_start(int c, long long N, int G)
+{
+    return (static_cast<long long>(c) * N + G - 1) / G;
+}
+
+__device__ __forceinline__ int unit_count(long long U, int n, long long N, int G)
+{
+    return n ? owner_of(U + n - 1, N, G) - owner_of(U, N, G) + 1 : 0;
+}
+
+// Block-wide.  s_len[b] = clamped length, s_n[b] = tiles per unit of batch b,
+// s_Ub[b] = tiles of one kv-head slice before batch b (s_Ub[B] = total).
+// Returns N = Hk * s_Ub[B].
+__device__ long long plan_prefix(const int32_t* __restrict__ seq_lens, int B, int Hk, int T_max, int* s_len,
+                                 int* s_n, int* s_Ub, int32_t* dev_status, bool report)
+{
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const int len = seq_lens[b];
+        const int lc = min(max(len, 0), T_max);
+        if (lc != len && report) report_status(dev_status, KVATTN_STATUS_BAD_LENGTH);
+        s_len[b] = lc;
+        s_n[b] = (lc + TILE - 1) / TILE;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int per = (B + 31) / 32;
+        const int beg = min(lane * per, B), end = min(beg + per, B);
+        int sum = 0;
+        for (int b = beg; b < end; ++b) sum += s_n[b];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int b = beg; b < end; ++b) {
+            s_Ub[b] = run;
+            run += s_n[b];
+        }
+        if (lane == 31) s_Ub[B] = incl;
+    }
+    __syncthreads();
+    return static_cast<long long>(Hk) * s_Ub[B];
+}
+
+// Block-wide: number of partial slots used by units 0 .. u_end-1.
+__device__ int slots_before(int u_end, int Hk, const int* s_n, const int* s_Ub, long long N, int G, int* s_acc)
+{
+    if (threadIdx.x == 0) *s_acc = 0;
+    __syncthreads();
+    int local = 0;
+    for (int u = threadIdx.x; u < u_end; u += blockDim.x) {
+        const int b = u / Hk, kvh = u - b * Hk;
+        const int n = s_n[b];
+        const long long U = static_cast<long long>(Hk) * s_Ub[b] + static_cast<long long>(kvh) * n;
+        local += unit_count(U, n, N, G);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+    if ((threadIdx.x & 31) == 0 && local) atomicAdd(s_acc, local);
+    __syncthreads();
+    const int r = *s_acc;
+    __syncthreads();
+    return r;
+}
+
+// Position in the unit walk of one CTA.
+struct Walk {
+    int b, kvh;
+    long long U;  // first global tile of the unit
+    int S;        // first partial slot of the unit
+};
+
+__device__ __forceinline__ void walk_next(Walk& w, int B, int Hk, const int* s_n, long long N, int G)
+{
+    const int n = s_n[w.b];
+    w.S += unit_count(w.U, n, N, G);
+    w.U += n;
+    if (++w.kvh == Hk) {
+        w.kvh = 0;
+        ++w.b;
+        while (w.b < B && s_n[w.b] == 0) ++w.b;
+    }
+}
+
+__device__ __forceinline__ uint32_t ld_u32(const kvattn_bf16* p)
+{
+    return *reinterpret_cast<const uint32_t*>(p);
+}
+
+// ---- the decode kernel ---------------------------------------------------------
+
+template <int D, int NMT>
+__global__ void __launch_bounds__(THREADS, 1)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, DecodeArgs a)
+{
+    using C = Cfg<D>;
+    constexpr int WPM = CWARPS / NMT;  // warps sharing one M tile (split the tile's rows)
+    constexpr int TPW = TILE / WPM;    // cache rows per warp per tile
+    constexpr int NT = TPW / 8;        // score n-tiles per warp
+    constexpr int KS = D / 16;         // k-steps of q.k
+    constexpr int DT = D / 8;          // output n-tiles
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* scr_o = reinterpret_cast<float*>(smem + C::OFF_SCR_O);
+    float* scr_ml = reinterpret_cast<float*>(smem + C::OFF_SCR_ML);
+    int* s_n = reinterpret_cast<int*>(smem + C::OFF_N);
+    int* s_Ub = reinterpret_cast<int*>(smem + C::OFF_UB);
+    int* s_len = reinterpret_cast<int*>(smem + C::OFF_LEN);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + C::STAGES;
+    int* s_misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
+    volatile int* s_abort = s_misc + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], CWARPS);
+        }
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == CWARPS && lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    // everything above overlaps the previous kernel of the stream
+    pdl_wait();
+    pdl_trigger();
+    const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
+                                    blockIdx.x == 0);
+    if (N == 0) return;
+    // With fewer tiles than CTAs only the first N CTAs take part, so that every
+    // participating CTA owns at least one tile and the CTAs owning a unit's
+    // tiles are consecutive (the piece count of a unit is then exact).
+    const int G = static_cast<int>(N < a.grid ? N : a.grid), c = blockIdx.x;
+    if (c >= G) return;
+    const long long lo = range_start(c, N, G), hi = range_start(c + 1, N, G);
+
+    // unit holding tile `lo`: the last batch entry whose first tile is <= lo
+    int b0 = 0;
+    {
+        int lo_b = 0, hi_b = a.B - 1;
+        while (lo_b < hi_b) {
+            const int mid = (lo_b + hi_b + 1) >> 1;
+            if (static_cast<long long>(a.Hk) * s_Ub[mid] <= lo) lo_b = mid;
+            else hi_b = mid - 1;
+        }
+        b0 = lo_b;
+    }
+    const int n0 = s_n[b0];
+    const int kvh0 = static_cast<int>((lo - static_cast<long long>(a.Hk) * s_Ub[b0]) / n0);
+    const int S0 = slots_before(b0 * a.Hk + kvh0, a.Hk, s_n, s_Ub, N, G, s_misc + 2);
+    const Walk w_start{b0, kvh0, static_cast<long long>(a.Hk) * s_Ub[b0] + static_cast<long long>(kvh0) * n0, S0};
+
+    if (warp == CWARPS) {
+        // ===== producer: one thread streams K/V tiles of every piece in order =====
+        if (lane != 0) return;
+        Walk w = w_start;
+        int it = 0;
+        bool ok = true;
+        while (ok && w.U < hi && w.b < a.B) {
+            const int n = s_n[w.b];
+            const long long tb = (lo > w.U ? lo : w.U) - w.U;
+            const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+            const int z = w.b * a.Hk + w.kvh;
+            for (long long t = tb; t < te; ++t, ++it) {
+                const int s = it % C::STAGES;
+                const uint32_t ph = (it / C::STAGES) & 1;
+                if (it >= C::STAGES) {
+                    if (*s_abort || !mbar_wait(&empty[s], ph ^ 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                uint8_t* kd = smem + s * C::STAGE_BYTES;
+                uint8_t* vd = kd + C::TILE_BYTES;
+#pragma unroll
+                for (int h = 0; h < C::HALVES; ++h) {
+                    tma_load_3d(kd + h * (TILE * 128), &tm_k, &full[s], h * 64, static_cast<int>(t * TILE), z);
+                    tma_load_3d(vd + h * (TILE * 128), &tm_v, &full[s], h * 64, static_cast<int>(t * TILE), z);
+                }
+            }
+            walk_next(w, a.B, a.Hk, s_n, N, G);
+        }
+        if (!ok) {
+            *s_abort = 1;
+            report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+        }
+        // copies still in flight complete before the CTA leaves (bounded waits)
+        for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
+            mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
+        return;
+    }
+
+    // ===== consumers =====
+    const int mt = warp / WPM, sub = warp % WPM;
+    const int tok0 = sub * TPW;
+    const int r0 = lane >> 2, cq = lane & 3;
+    const int g = a.g;
+    const float sl2 = a.scale * kLog2e;
+    const int ctid = threadIdx.x;  // 0 .. 127
+    const int rows_out = g < NMT * 16 ? g : NMT * 16;
+
+    Walk w = w_start;
+    int it = 0;
+    while (w.U < hi && w.b < a.B) {
+        const int n = s_n[w.b];
+        const int len = s_len[w.b];
+        const long long tb = (lo > w.U ? lo : w.U) - w.U;
+        const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+        const int count = unit_count(w.U, n, N, G);
+        const int slot = w.S + (c - owner_of(w.U, N, G));
+
+        // query fragments (A operand): rows = heads of the group, zero beyond g
+        uint32_t qa[KS][4];
+        {
+            const kvattn_bf16* qg = a.q + (static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * g) * D;
+            const int ra = mt * 16 + r0, rb = ra + 8;
+#pragma unroll
+            for (int kk = 0; kk < KS; ++kk) {
+                const int col = kk * 16 + 2 * cq;
+                qa[kk][0] = ra < g ? ld_u32(qg + ra * D + col) : 0u;
+                qa[kk][1] = rb < g ? ld_u32(qg + rb * D + col) : 0u;
+                qa[kk][2] = ra < g ? ld_u32(qg + ra * D + col + 8) : 0u;
+                qa[kk][3] = rb < g ? ld_u32(qg + rb * D + col + 8) : 0u;
+            }
+        }
+        float o[DT][4];
+#pragma unroll
+        for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+        for (long long t = tb; t < te; ++t, ++it) {
+            const int s = it % C::STAGES;
+            const uint32_t ph = (it / C::STAGES) & 1;
+            bool have = false;
+            if (!*s_abort) {
+                have = mbar_wait(&full[s], ph);
+                if (!have) {
+                    *s_abort = 1;
+                    report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+                }
+            }
+            if (have) {
+                const uint32_t sK = smem_u32(smem + s * C::STAGE_BYTES);
+                const uint32_t sV = sK + C::TILE_BYTES;
+                const int n_valid = len - static_cast<int>(t) * TILE;  // >= 1
+
+                // ---- S = Q K^T over this warp's rows of the tile ----
+                float sc[NT][4];
+#pragma unroll
+                for (int i = 0; i < NT; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
+                const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+                for (int kk = 0; kk < KS; ++kk) {
+                    const int dim = kk * 16 + ((mi & 1) << 3);
+                    const uint32_t dbase = sK + (dim >> 6) * (TILE * 128);
+                    const int chunk = (dim & 63) >> 3;
+#pragma unroll
+                    for (int np = 0; np < NT / 2; ++np) {
+                        const int tok = tok0 + np * 16 + rr + ((mi >> 1) << 3);
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(dbase + swz128(tok, chunk), b0, b1, b2, b3);
+                        mma_bf16_16816(sc[2 * np], qa[kk], b0, b1);
+                        mma_bf16_16816(sc[2 * np + 1], qa[kk], b2, b3);
+                    }
+                }
+                // ---- online softmax (base 2) ----
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < NT; ++i) {
+                    const int tk = tok0 + i * 8 + 2 * cq;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float v = sc[i][e] * sl2;
+                        if (tk + (e & 1) >= n_valid) v = -INFINITY;
+                        sc[i][e] = v;
+                    }
+                    mx0 = fmaxf(mx0, fmaxf(sc[i][0], sc[i][1]));
+                    mx1 = fmaxf(mx1, fmaxf(sc[i][2], sc[i][3]));
+                }
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+                const float mu0 = mn0 == -INFINITY ? 0.f : mn0;
+                const float mu1 = mn1 == -INFINITY ? 0.f : mn1;
+                const float al0 = fast_exp2(m0 - mu0), al1 = fast_exp2(m1 - mu1);
+                m0 = mn0;
+                m1 = mn1;
+                float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+                for (int i = 0; i < NT; ++i) {
+                    sc[i][0] = fast_exp2(sc[i][0] - mu0);
+                    sc[i][1] = fast_exp2(sc[i][1] - mu0);
+                    sc[i][2] = fast_exp2(sc[i][2] - mu1);
+                    sc[i][3] = fast_exp2(sc[i][3] - mu1);
+                    ps0 += sc[i][0] + sc[i][1];
+                    ps1 += sc[i][2] + sc[i][3];
+                }
+                l0 = l0 * al0 + ps0;
+                l1 = l1 * al1 + ps1;
+#pragma unroll
+                for (int i = 0; i < DT; ++i) {
+                    o[i][0] *= al0;
+                    o[i][1] *= al0;
+                    o[i][2] *= al1;
+                    o[i][3] *= al1;
+                }
+                // ---- O += P V ----
+                const bool tail = n_valid < TILE;
+#pragma unroll
+                for (int j = 0; j < TPW / 16; ++j) {
+                    uint32_t pa[4];
+                    pa[0] = pack_bf16x2(sc[2 * j][0], sc[2 * j][1]);
+                    pa[1] = pack_bf16x2(sc[2 * j][2], sc[2 * j][3]);
+                    pa[2] = pack_bf16x2(sc[2 * j + 1][0], sc[2 * j + 1][1]);
+                    pa[3] = pack_bf16x2(sc[2 * j + 1][2], sc[2 * j + 1][3]);
+                    const int tok = tok0 + j * 16 + rr + ((mi & 1) << 3);
+                    // rows this thread's V fragments hold (for the tail mask)
+                    const int vt = tok0 + j * 16 + 2 * cq;
+#pragma unroll
+                    for (int dp = 0; dp < D / 16; ++dp) {
+                        const int dim = dp * 16 + ((mi >> 1) << 3);
+                        uint32_t v0, v1, v2, v3;
+                        ldsm_x4_t(sV + (dim >> 6) * (TILE * 128) + swz128(tok, (dim & 63) >> 3), v0, v1, v2, v3);
+                        if (tail) {
+                            // rows past the length may hold anything (NaN included):
+                            // zero them so that 0 * garbage cannot reach the sum
+                            const uint32_t k0 = (vt < n_valid ? 0x0000ffffu : 0u) | (vt + 1 < n_valid ? 0xffff0000u : 0u);
+                            const uint32_t k1 =
+                                (vt + 8 < n_valid ? 0x0000ffffu : 0u) | (vt + 9 < n_valid ? 0xffff0000u : 0u);
+                            v0 &= k0;
+                            v2 &= k0;
+                            v1 &= k1;
+                            v3 &= k1;
+                        }
+                        mma_bf16_16816(o[2 * dp], pa, v0, v1);
+                        mma_bf16_16816(o[2 * dp + 1], pa, v2, v3);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+
+        // ---- finish the piece: merge the warps of each M tile, then write ----
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+        {
+            float* so = scr_o + warp * 16 * C::SCR_STRIDE;
+#pragma unroll
+            for (int i = 0; i < DT; ++i) {
+                const int col = i * 8 + 2 * cq;
+                *reinterpret_cast<float2*>(so + r0 * C::SCR_STRIDE + col) = make_float2(o[i][0], o[i][1]);
+                *reinterpret_cast<float2*>(so + (r0 + 8) * C::SCR_STRIDE + col) = make_float2(o[i][2], o[i][3]);
+            }
+            if (cq == 0) {
+                float* ml = scr_ml + warp * 32;
+                ml[r0] = m0;
+                ml[r0 + 8] = m1;
+                ml[16 + r0] = l0;
+                ml[16 + r0 + 8] = l1;
+            }
+        }
+        named_bar_sync(1, CWARPS * 32);
+        {
+            const bool fin = count == 1;
+            const long long bh = static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * g;
+            for (int idx = ctid; idx < rows_out * D; idx += CWARPS * 32) {
+                const int row = idx / D, dim = idx - row * D;
+                const int mtile = row >> 4, lr = row & 15;
+                float M = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < WPM; ++j) M = fmaxf(M, scr_ml[(mtile * WPM + j) * 32 + lr]);
+                const float Mu = M == -INFINITY ? 0.f : M;
+                float acc = 0.f, L = 0.f;
+#pragma unroll
+                for (int j = 0; j < WPM; ++j) {
+                    const int wj = mtile * WPM + j;
+                    const float wgt = fast_exp2(scr_ml[wj * 32 + lr] - Mu);
+                    acc += wgt * scr_o[(wj * 16 + lr) * C::SCR_STRIDE + dim];
+                    L += wgt * scr_ml[wj * 32 + 16 + lr];
+                }
+                if (fin) {
+                    const long long oi = (bh + row) * D + dim;
+                    reinterpret_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+                    if (dim == 0 && a.lse) a.lse[bh + row] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+                } else {
+                    const long long pi = static_cast<long long>(slot) * g + row;
+                    a.part_o[pi * D + dim] = acc;
+                    if (dim == 0) {
+                        a.part_ml[pi * 2] = Mu;
+                        a.part_ml[pi * 2 + 1] = L;
+                    }
+                }
+            }
+            // the unit's first piece records its slot range for the merge kernel
+            if (tb == 0 && ctid == 0) a.unit_info[w.b * a.Hk + w.kvh] = make_int2(w.S, count);
+        }
+        named_bar_sync(1, CWARPS * 32);
+        walk_next(w, a.B, a.Hk, s_n, N, G);
+    }
+}
+
+// ---- merge of split units --------------------------------------------------------
+// One CTA per (unit, block of 8 heads), one warp per head.  With weights
+// w_j = 2^(m_j - M) / sum_i 2^(m_i - M) l_i:  out = sum_j w_j O_j  and
+// lse = ln 2 * (M + log2 sum_j 2^(m_j - M) l_j): the softmax over a union of
+// key sets is the max-shifted mix of the parts.
+constexpr int MERGE_WARPS = 8;
+
+template <int D>
+__global__ void __launch_bounds__(MERGE_WARPS * 32) decode_combine_kernel(DecodeArgs a)
+{
+    extern __shared__ float s_w[];  // [MERGE_WARPS][max pieces]
+    pdl_wait();
+    pdl_trigger();
+    const int u = blockIdx.x;
+    const int b = u / a.Hk, kvh = u - b * a.Hk;
+    const int g = a.g;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.y * MERGE_WARPS + warp;
+    if (row >= g) return;
+    const long long bh = static_cast<long long>(b) * a.H + static_cast<long long>(kvh) * g + row;
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * D;
+    const int len = min(max(a.seq_lens[b], 0), a.T_max);
+    if (len == 0) {
+        for (int dim = lane; dim < D; dim += 32) out[dim] = __float2bfloat16_rn(0.f);
+        if (lane == 0 && a.lse) a.lse[bh] = -INFINITY;
+        return;
+    }
+    const int2 info = a.unit_info[u];
+    if (info.y <= 1) return;  // finished inside one CTA
+    const long long base = static_cast<long long>(info.x) * g + row;
+    float M = -INFINITY;
+    for (int j = lane; j < info.y; j += 32) M = fmaxf(M, a.part_ml[(base + static_cast<long long>(j) * g) * 2]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float* w = s_w + warp * a.grid;
+    float L = 0.f;
+    for (int j = lane; j < info.y; j += 32) {
+        const long long pj = (base + static_cast<long long>(j) * g) * 2;
+        const float e = fast_exp2(a.part_ml[pj] - M);
+        w[j] = e;
+        L += e * a.part_ml[pj + 1];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    __syncwarp();
+    const float inv = 1.f / L;
+    float acc[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
+    for (int j = 0; j < info.y; ++j) {
+        const float wj = w[j] * inv;
+        const float* o = a.part_o + (base + static_cast<long long>(j) * g) * D;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) acc[i] += wj * o[lane + 32 * i];
+    }
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) out[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
+    if (lane == 0 && a.lse) a.lse[bh] = (M + __log2f(L)) * kLn2;
+}
+
+template <int D, int NMT>
+cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                         cudaStream_t stream)
+{
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(decode_kernel<D, NMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    e = launch_pdl(decode_kernel<D, NMT>, dim3(a.grid), dim3(THREADS), Cfg<D>::SMEM, stream, tm_k, tm_v, a);
+    if (e != cudaSuccess) return e;
+    const dim3 cgrid(a.B * a.Hk, (a.g + MERGE_WARPS - 1) / MERGE_WARPS);
+    return launch_pdl(decode_combine_kernel<D>, cgrid, dim3(MERGE_WARPS * 32),
+                      static_cast<size_t>(MERGE_WARPS) * a.grid * sizeof(float), stream, a);
+}
+
+}  // namespace
+
+long long decode_max_slots(int B, int Hk, int grid)
+{
+    return static_cast<long long>(grid) + static_cast<long long>(B) * Hk;
+}
+
+int decode_grid(int num_sms) { return num_sms; }
+
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          cudaStream_t stream)
+{
+    const int nmt = a.g <= 16 ? 1 : (a.g <= 32 ? 2 : 4);
+    if (a.d == 128) {
+        if (nmt == 1) return launch_typed<128, 1>(a, tm_k, tm_v, stream);
+        if (nmt == 2) return launch_typed<128, 2>(a, tm_k, tm_v, stream);
+        return launch_typed<128, 4>(a, tm_k, tm_v, stream);
+    }
+    if (nmt == 1) return launch_typed<64, 1>(a, tm_k, tm_v, stream);
+    if (nmt == 2) return launch_typed<64, 2>(a, tm_k, tm_v, stream);
+    return launch_typed<64, 4>(a, tm_k, tm_v, stream);
+}
+
+}  // namespace kvattn

@@ -1,0 +1,77 @@
+// kernels.h -- internal launch interface between the C-ABI layer (api.cu)
+// and the kernel files.  Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/kvattn.h"
+
+namespace kvattn {
+
+// Launch `kernel` on `stream` with programmatic stream serialisation (the
+// kernel calls pdl_wait() before reading what earlier kernels wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// ---- RoPE ----
+cudaError_t launch_rope_table(const kvattn_rope_params& p, int max_pos, float* cos_out, float* sin_out,
+                              cudaStream_t stream);
+
+struct RopeApplyArgs {
+    kvattn_bf16* q;
+    int q_nb, q_nt, q_nh;
+    int64_t q_sb, q_st, q_sh;
+    const int32_t* q_pos;
+    kvattn_bf16* k;
+    int k_nb, k_nt, k_nh;
+    int64_t k_sb, k_st, k_sh;
+    const int32_t* k_pos;
+    const float* cos_tab;
+    const float* sin_tab;
+    int max_pos, head_dim, pair_style;
+    int32_t* dev_status;
+    int num_sms;
+};
+cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t stream);
+
+// ---- split-K decode ----
+constexpr int DECODE_MAX_B = 1024;
+
+struct DecodeArgs {
+    const kvattn_bf16* q;
+    const int32_t* seq_lens;
+    kvattn_bf16* out;
+    float* lse;
+    float* part_o;   // [slots][g][d]  unnormalised partial outputs
+    float* part_ml;  // [slots][g][2]  (running max in log2 units, sum of exponentials)
+    int2* unit_info; // [B*Hk]         (first slot, number of pieces) of every non-empty unit
+    int32_t* dev_status;
+    int B, H, Hk, g, d, T_max;
+    float scale;
+    int grid;        // persistent CTAs (also the number of tile ranges)
+};
+// Number of partial slots the decode kernel may write for a given grid.
+long long decode_max_slots(int B, int Hk, int grid);
+// Persistent CTAs per launch for this device.
+int decode_grid(int num_sms);
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
+                          cudaStream_t stream);
+
+}  // namespace kvattn

@@ -1,0 +1,181 @@
+// rope.cu -- RoPE cos/sin table construction and in-place rotation of q and k.
+//
+// Table: "Agentic RL 入门3：transformer 架构" §1.1 (theta_i = base^(-2i/d),
+// rotation R(m, theta_i)) and §1.2 ① PI, ② NTK-aware base, ③ YaRN ramp and
+// attention temperature, ④ dynamic NTK.  Angles are formed and evaluated in
+// fp64 (m * theta reaches ~3e4 rad at the 32K configurations, where an fp32
+// angle would already be off by ~2e-3 rad) and stored as fp32.
+//
+// Rotation: memory-bound.  One thread owns one 16-byte chunk (8 bf16) of a
+// head vector; for adjacent pairs that is 4 whole pairs, for half-split pairs
+// the thread also owns the partner chunk d/2 further on.  Math in fp32,
+// bf16 round-to-nearest-even on store.  v is never passed here.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvattn {
+
+namespace {
+
+constexpr double kTwoPi = 6.283185307179586476925286766559;
+
+__global__ void rope_table_kernel(kvattn_rope_params p, int max_pos, float* __restrict__ cos_out,
+                                  float* __restrict__ sin_out)
+{
+    const int half = p.head_dim / 2;
+    const long long total = static_cast<long long>(max_pos) * half;
+    for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const int m = static_cast<int>(idx / half);
+        const int i = static_cast<int>(idx - static_cast<long long>(m) * half);
+        const double d = static_cast<double>(p.head_dim);
+
+        double base = p.base;
+        if (p.scaling == KVATTN_ROPE_NTK) {
+            base = p.base * pow(p.s, d / (d - 2.0));
+        } else if (p.scaling == KVATTN_ROPE_DYN_NTK) {
+            const double s_dyn = fmax(1.0, p.L_cur / p.L_train);
+            base = p.base * pow(s_dyn, d / (d - 2.0));
+        }
+        // theta_i = base^(-2i/d)
+        double theta = exp(-(2.0 * i / d) * log(base));
+        double pos = static_cast<double>(m);
+        double mag = 1.0;
+        if (p.scaling == KVATTN_ROPE_PI) {
+            pos = pos / p.s;
+        } else if (p.scaling == KVATTN_ROPE_YARN) {
+            // turns completed inside the training window decide the blend
+            const double r = p.L_train * theta / kTwoPi;
+            const double gamma =
+                r > p.beta ? 1.0 : (r <= p.alpha ? 0.0 : (r - p.alpha) / (p.beta - p.alpha));
+            theta = gamma * theta + (1.0 - gamma) * (theta / p.s);
+            mag = 1.0 + 0.1 * log(p.s);
+        }
+        double sv, cv;
+        sincos(pos * theta, &sv, &cv);
+        cos_out[idx] = static_cast<float>(mag * cv);
+        sin_out[idx] = static_cast<float>(mag * sv);
+    }
+}
+
+struct RopeView {
+    __nv_bfloat16* x;
+    const int32_t* pos;
+    long long n_vec;  // nb * nt * nh
+    int nt, nh;
+    long long sb, st, sh;
+};
+
+// Rotate one 8-element chunk pair-wise with table row `m`.
+template <int PAIR_STYLE>
+__device__ __forceinline__ void rotate_chunk(__nv_bfloat16* vec, int chunk, int half, const float* cos_row,
+                                             const float* sin_row)
+{
+    if (PAIR_STYLE == 0) {
+        // elements 8c .. 8c+7 = pairs 4c .. 4c+3
+        uint4 raw = *reinterpret_cast<const uint4*>(vec + chunk * 8);
+        const float4 c = *reinterpret_cast<const float4*>(cos_row + chunk * 4);
+        const float4 s = *reinterpret_cast<const float4*>(sin_row + chunk * 4);
+        uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        const float cc[4] = {c.x, c.y, c.z, c.w};
+        const float ss[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a = bf16_lo(w[j]), b = bf16_hi(w[j]);
+            w[j] = pack_bf16x2(a * cc[j] - b * ss[j], a * ss[j] + b * cc[j]);
+        }
+        *reinterpret_cast<uint4*>(vec + chunk * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else {
+        // element 8c + j pairs with 8c + j + d/2; pair index 8c + j
+        uint4 ra = *reinterpret_cast<const uint4*>(vec + chunk * 8);
+        uint4 rb = *reinterpret_cast<const uint4*>(vec + half + chunk * 8);
+        const float4 c0 = *reinterpret_cast<const float4*>(cos_row + chunk * 8);
+        const float4 c1 = *reinterpret_cast<const float4*>(cos_row + chunk * 8 + 4);
+        const float4 s0 = *reinterpret_cast<const float4*>(sin_row + chunk * 8);
+        const float4 s1 = *reinterpret_cast<const float4*>(sin_row + chunk * 8 + 4);
+        uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+        uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+        const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a0 = bf16_lo(wa[j]), a1 = bf16_hi(wa[j]);
+            const float b0 = bf16_lo(wb[j]), b1 = bf16_hi(wb[j]);
+            const int i0 = 2 * j, i1 = 2 * j + 1;
+            wa[j] = pack_bf16x2(a0 * cc[i0] - b0 * ss[i0], a1 * cc[i1] - b1 * ss[i1]);
+            wb[j] = pack_bf16x2(a0 * ss[i0] + b0 * cc[i0], a1 * ss[i1] + b1 * cc[i1]);
+        }
+        *reinterpret_cast<uint4*>(vec + chunk * 8) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        *reinterpret_cast<uint4*>(vec + half + chunk * 8) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    }
+}
+
+template <int PAIR_STYLE>
+__global__ void rope_apply_kernel(RopeView qv, RopeView kv, const float* __restrict__ cos_tab,
+                                  const float* __restrict__ sin_tab, int max_pos, int head_dim,
+                                  int32_t* dev_status)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int half = head_dim / 2;
+    // threads per head vector: one per chunk of 8 elements (adjacent pairs) or
+    // per chunk of the first half (half-split pairs)
+    const int per_vec = PAIR_STYLE == 0 ? head_dim / 8 : head_dim / 16;
+    const long long q_threads = qv.n_vec * per_vec;
+    const long long total = q_threads + kv.n_vec * per_vec;
+    for (long long tid = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; tid < total;
+         tid += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const bool is_q = tid < q_threads;
+        const RopeView& v = is_q ? qv : kv;
+        const long long local = is_q ? tid : tid - q_threads;
+        const long long vec = local / per_vec;
+        const int chunk = static_cast<int>(local - vec * per_vec);
+        const int h = static_cast<int>(vec % v.nh);
+        const long long bt = vec / v.nh;
+        const int t = static_cast<int>(bt % v.nt);
+        const long long b = bt / v.nt;
+        const int m = v.pos[bt];
+        if (m < 0 || m >= max_pos) {
+            if (chunk == 0) report_status(dev_status, KVATTN_STATUS_BAD_POSITION);
+            continue;
+        }
+        __nv_bfloat16* base = v.x + b * v.sb + static_cast<long long>(t) * v.st + static_cast<long long>(h) * v.sh;
+        rotate_chunk<PAIR_STYLE>(base, chunk, half, cos_tab + static_cast<long long>(m) * half,
+                                 sin_tab + static_cast<long long>(m) * half);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_rope_table(const kvattn_rope_params& p, int max_pos, float* cos_out, float* sin_out,
+                              cudaStream_t stream)
+{
+    const long long total = static_cast<long long>(max_pos) * (p.head_dim / 2);
+    const int threads = 256;
+    const long long blocks = (total + threads - 1) / threads;
+    const int grid = static_cast<int>(blocks < 65535 ? blocks : 65535);
+    rope_table_kernel<<<grid, threads, 0, stream>>>(p, max_pos, cos_out, sin_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t stream)
+{
+    RopeView qv{reinterpret_cast<__nv_bfloat16*>(a.q), a.q_pos,
+                a.q ? static_cast<long long>(a.q_nb) * a.q_nt * a.q_nh : 0, a.q_nt > 0 ? a.q_nt : 1,
+                a.q_nh > 0 ? a.q_nh : 1, a.q_sb, a.q_st, a.q_sh};
+    RopeView kv{reinterpret_cast<__nv_bfloat16*>(a.k), a.k_pos,
+                a.k ? static_cast<long long>(a.k_nb) * a.k_nt * a.k_nh : 0, a.k_nt > 0 ? a.k_nt : 1,
+                a.k_nh > 0 ? a.k_nh : 1, a.k_sb, a.k_st, a.k_sh};
+    const int per_vec = a.pair_style == 0 ? a.head_dim / 8 : a.head_dim / 16;
+    const long long total = (qv.n_vec + kv.n_vec) * per_vec;
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    long long blocks = (total + threads - 1) / threads;
+    const long long cap = static_cast<long long>(a.num_sms) * 16;
+    if (blocks > cap) blocks = cap;
+    auto kern = a.pair_style == 0 ? rope_apply_kernel<0> : rope_apply_kernel<1>;
+    return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, qv, kv, a.cos_tab,
+                      a.sin_tab, a.max_pos, a.head_dim, a.dev_status);
+}
+
+}  // namespace kvattn

@@ -1,0 +1,264 @@
+"""Thin Python binding of libkvattn.so (the C ABI declared in include/kvattn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch provides device memory and the current stream; tensors must
+be CUDA tensors of the documented dtype and layout.  There is no CPU
+fallback: if the shared library is missing this module raises ImportError.
+Function names match the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m mqa_kv_cache_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_i32, _i64, _f32, _vp, _sz = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class RopeParams(ctypes.Structure):
+    _fields_ = [("head_dim", ctypes.c_int), ("scaling", ctypes.c_int), ("pair_style", ctypes.c_int),
+                ("reserved", ctypes.c_int), ("base", ctypes.c_double), ("s", ctypes.c_double),
+                ("L_train", ctypes.c_double), ("alpha", ctypes.c_double), ("beta", ctypes.c_double),
+                ("L_cur", ctypes.c_double)]
+
+
+_lib.kvattn_last_error_string.restype = ctypes.c_char_p
+_lib.kvattn_version.restype = ctypes.c_char_p
+_lib.rope_table_build.argtypes = [ctypes.POINTER(RopeParams), _i32, _vp, _vp, _vp]
+_lib.rope_apply_qk.argtypes = [_vp, _i32, _i32, _i32, _i64, _i64, _i64, _vp,
+                               _vp, _i32, _i32, _i32, _i64, _i64, _i64, _vp,
+                               _vp, _vp, _i32, _i32, _i32, _vp, _vp]
+_lib.attn_decode_gqa_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32]
+_lib.attn_decode_gqa_workspace_bytes.restype = _sz
+_lib.attn_decode_gqa.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
+                                 _vp, _vp]
+_lib.attn_prefill_causal.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]
+_lib.dsa_index_topk_workspace_bytes.argtypes = [_i32, _i32, _i32]
+_lib.dsa_index_topk_workspace_bytes.restype = _sz
+_lib.dsa_index_topk.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]
+_lib.attn_decode_sparse_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32]
+_lib.attn_decode_sparse_workspace_bytes.restype = _sz
+_lib.attn_decode_sparse.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
+                                    _vp, _vp]
+
+ROPE_NONE, ROPE_PI, ROPE_NTK, ROPE_YARN, ROPE_DYN_NTK = 0, 1, 2, 3, 4
+STATUS_BAD_POSITION, STATUS_BAD_LENGTH, STATUS_BAD_INDEX, STATUS_NAN_SCORE, STATUS_TIMEOUT = 1, 2, 4, 8, 16
+
+
+class KvattnError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"kvattn error {code}: {msg}")
+        self.code = code
+
+
+def library():
+    """The loaded ctypes.CDLL (for direct C-ABI calls)."""
+    return _lib
+
+
+def version() -> str:
+    return _lib.kvattn_version().decode()
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise KvattnError(rc, _lib.kvattn_last_error_string().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _contig(t, name):
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def rope_params(head_dim, base, scaling=ROPE_NONE, s=1.0, L_train=0.0, alpha=1.0, beta=32.0, L_cur=0.0,
+                pair_style=0) -> RopeParams:
+    return RopeParams(head_dim, scaling, pair_style, 0, base, s, L_train, alpha, beta, L_cur)
+
+
+def rope_table_build(params: RopeParams, max_pos: int, device=None):
+    """-> (cos, sin) fp32 [max_pos, head_dim/2] on `device` (default: current)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    half = params.head_dim // 2
+    cos = torch.empty((max_pos, half), dtype=torch.float32, device=dev)
+    sin = torch.empty((max_pos, half), dtype=torch.float32, device=dev)
+    _check(_lib.rope_table_build(ctypes.byref(params), max_pos, _ptr(cos), _ptr(sin), _stream()))
+    return cos, sin
+
+
+def _view(x, layout):
+    """(nb, nt, nh, sb, st, sh) of a head-vector tensor for rope_apply_qk."""
+    if x.stride(-1) != 1:
+        raise ValueError("innermost dimension must be contiguous")
+    if layout == "bhd":      # [B, H, d], one token per batch entry
+        B, H, _ = x.shape
+        return B, 1, H, x.stride(0), 0, x.stride(1)
+    if layout == "bthd":     # [B, T, H, d]
+        B, T, H, _ = x.shape
+        return B, T, H, x.stride(0), x.stride(1), x.stride(2)
+    if layout == "bhtd":     # [B, H, T, d] (the cache layout)
+        B, H, T, _ = x.shape
+        return B, T, H, x.stride(0), x.stride(2), x.stride(1)
+    raise ValueError(layout)
+
+
+def rope_apply_qk(q, q_pos, k, k_pos, cos, sin, q_layout="bthd", k_layout="bhtd", pair_style=0,
+                  dev_status=None):
+    """Rotate q and/or k in place.  Positions are int32 CUDA tensors with one
+    entry per (batch, token): q_pos [B, T_q] (T_q = 1 for 'bhd'), k_pos [B, T]."""
+    _need(cos, torch.float32, "cos")
+    _need(sin, torch.float32, "sin")
+    head_dim = 2 * cos.shape[1]
+    qv = (0, 0, 0, 0, 0, 0)
+    kv = (0, 0, 0, 0, 0, 0)
+    if q is not None:
+        _need(q, torch.bfloat16, "q")
+        _need(q_pos, torch.int32, "q_pos")
+        _contig(q_pos, "q_pos")
+        qv = _view(q, q_layout)
+        if q_pos.numel() != qv[0] * qv[1]:
+            raise ValueError("q_pos must hold one position per (batch, token)")
+    if k is not None:
+        _need(k, torch.bfloat16, "k")
+        _need(k_pos, torch.int32, "k_pos")
+        _contig(k_pos, "k_pos")
+        kv = _view(k, k_layout)
+        if k_pos.numel() != kv[0] * kv[1]:
+            raise ValueError("k_pos must hold one position per (batch, token)")
+    _check(_lib.rope_apply_qk(_ptr(q), *qv, _ptr(q_pos) if q is not None else None,
+                              _ptr(k), *kv, _ptr(k_pos) if k is not None else None,
+                              _ptr(cos), _ptr(sin), cos.shape[0], head_dim, pair_style, _ptr(dev_status),
+                              _stream()))
+
+
+def attn_decode_gqa_workspace_bytes(B, n_head, n_kv_head, head_dim, T_max) -> int:
+    return int(_lib.attn_decode_gqa_workspace_bytes(B, n_head, n_kv_head, head_dim, T_max))
+
+
+def workspace(nbytes: int, device=None):
+    """A 256-byte aligned uint8 CUDA buffer of at least `nbytes` bytes."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+
+
+def attn_decode_gqa(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, ws=None, dev_status=None,
+                    want_lse=True):
+    """q [B, H, d] bf16, k_cache/v_cache [B, Hk, T_max, d] bf16, seq_lens int32 [B]
+    -> (out [B, H, d] bf16, lse [B, H] fp32 or None)."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    _need(seq_lens, torch.int32, "seq_lens")
+    _contig(seq_lens, "seq_lens")
+    B, H, d = q.shape
+    Bk, Hk, T_max, dk = k_cache.shape
+    if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seq_lens.numel() != B:
+        raise ValueError("inconsistent decode shapes")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = attn_decode_gqa_workspace_bytes(B, H, Hk, d, T_max)
+    if ws is None:
+        ws = workspace(need, q.device)
+    _check(_lib.attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H, Hk, d, T_max,
+                                float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status),
+                                _stream()))
+    return out, lse
+
+
+def attn_prefill_causal(q, k, v, scale, out=None, lse=None, want_lse=True):
+    """q [B, T, H, d] bf16, k/v [B, Hk, T, d] bf16 -> (out [B, T, H, d] bf16, lse [B, H, T] fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    B, T, H, d = q.shape
+    Hk = k.shape[1]
+    if k.shape != (B, Hk, T, d) or v.shape != k.shape:
+        raise ValueError("inconsistent prefill shapes")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check(_lib.attn_prefill_causal(_ptr(q), _ptr(k), _ptr(v), B, T, H, Hk, d, float(scale), _ptr(out), _ptr(lse),
+                                    _stream()))
+    return out, lse
+
+
+def dsa_index_topk_workspace_bytes(B, L_max, k) -> int:
+    return int(_lib.dsa_index_topk_workspace_bytes(B, L_max, k))
+
+
+def dsa_index_topk(q_idx, w, k_idx, k, seq_lens=None, topk_idx=None, scores_out=None, ws=None, dev_status=None,
+                   want_scores=True):
+    """q_idx [B, H_I, d_I] bf16, w [B, H_I] fp32, k_idx [B, L_max, d_I] bf16
+    -> (topk_idx int32 [B, k], scores fp32 [B, L_max] or None)."""
+    _need(q_idx, torch.bfloat16, "q_idx")
+    _need(k_idx, torch.bfloat16, "k_idx")
+    _need(w, torch.float32, "w")
+    for t, n in ((q_idx, "q_idx"), (k_idx, "k_idx"), (w, "w")):
+        _contig(t, n)
+    B, HI, dI = q_idx.shape
+    L_max = k_idx.shape[1]
+    if seq_lens is not None:
+        _need(seq_lens, torch.int32, "seq_lens")
+    if topk_idx is None:
+        topk_idx = torch.empty((B, k), dtype=torch.int32, device=q_idx.device)
+    if scores_out is None and want_scores:
+        scores_out = torch.empty((B, L_max), dtype=torch.float32, device=q_idx.device)
+    if ws is None:
+        ws = workspace(dsa_index_topk_workspace_bytes(B, L_max, k), q_idx.device)
+    _check(_lib.dsa_index_topk(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(seq_lens), B, HI, dI, L_max, k,
+                               _ptr(topk_idx), _ptr(scores_out), _ptr(ws), ws.numel(), _ptr(dev_status),
+                               _stream()))
+    return topk_idx, scores_out
+
+
+def attn_decode_sparse_workspace_bytes(B, Hq, Dv, k) -> int:
+    return int(_lib.attn_decode_sparse_workspace_bytes(B, Hq, Dv, k))
+
+
+def attn_decode_sparse(q, latent, topk_idx, Dv, scale, out=None, lse=None, ws=None, dev_status=None,
+                       want_lse=True):
+    """q [B, Hq, Dk] bf16, latent [B, L_max, Dk] bf16, topk_idx int32 [B, k]
+    -> (out [B, Hq, Dv] bf16, lse [B, Hq] fp32)."""
+    _need(q, torch.bfloat16, "q")
+    _need(latent, torch.bfloat16, "latent")
+    _need(topk_idx, torch.int32, "topk_idx")
+    for t, n in ((q, "q"), (latent, "latent"), (topk_idx, "topk_idx")):
+        _contig(t, n)
+    B, Hq, Dk = q.shape
+    L_max = latent.shape[1]
+    k = topk_idx.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, Dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(attn_decode_sparse_workspace_bytes(B, Hq, Dv, k), q.device)
+    _check(_lib.attn_decode_sparse(_ptr(q), _ptr(latent), _ptr(topk_idx), B, Hq, Dk, Dv, L_max, k, float(scale),
+                                   _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status), _stream()))
+    return out, lse
