@@ -121,6 +121,15 @@ DecodeWs decode_ws(int B, int n_head, int n_kv_head, int head_dim, int grid)
 
 }  // namespace
 
+int kvattn::record_error(int code, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
 extern "C" {
 
 const char* kvattn_last_error_string(void) { return g_err; }

@@ -30,6 +30,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Record an error message for kvattn_last_error_string() and return `code`.
+int record_error(int code, const char* fmt, ...);
+
 // ---- RoPE ----
 cudaError_t launch_rope_table(const kvattn_rope_params& p, int max_pos, float* cos_out, float* sin_out,
                               cudaStream_t stream);
