@@ -148,6 +148,33 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
                     int T_max, float scale, kvattn_bf16* out, float* lse, void* workspace,
                     size_t workspace_bytes, int32_t* dev_status, void* stream);
 
+/*
+ * attn_decode_gqa for callers that cannot allocate device memory.  The pages
+ * have no counterpart to this entry point; it exists for callers that cannot
+ * give the library a workspace: code running inside another runtime's fixed
+ * memory pool (which owns the device and forbids cudaMalloc behind its back),
+ * code on a latency-critical path where cudaMalloc would implicitly
+ * synchronise the device, and plain C callers with no allocator of their own.
+ * Same arguments, layout and results as attn_decode_gqa, minus the workspace:
+ * the scratch lives in a file-scope device array of
+ * KVATTN_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.  The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).  A shape whose scratch need
+ * (attn_decode_gqa_workspace_bytes) exceeds the array is rejected with
+ * KVATTN_ERR_WORKSPACE.  The first call on a device looks the array's device
+ * address up (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls on a device share the one array and it keeps the last
+ * call's contents (the kernels write every entry before reading it, so none
+ * needs clearing): calls that can overlap on the GPU -- different streams, or
+ * graphs replayed concurrently -- race and corrupt each other's results.
+ */
+#define KVATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+int attn_decode_gqa_noalloc(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
+                            const int32_t* seq_lens, int B, int n_head, int n_kv_head, int head_dim,
+                            int T_max, float scale, kvattn_bf16* out, float* lse, int32_t* dev_status,
+                            void* stream);
+
 /* ---- causal prefill ---------------------------------------------------------
  * softmax(scale * q k^T + M) v with the lower-triangular mask M (key j is
  * visible to query i iff j <= i): "注意力变体与 MoE" attention() (triu(1)

@@ -41,6 +41,8 @@ _lib.attn_decode_gqa_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.attn_decode_gqa_workspace_bytes.restype = _sz
 _lib.attn_decode_gqa.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
                                  _vp, _vp]
+_lib.attn_decode_gqa_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
+                                         _vp]
 _lib.attn_prefill_causal.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]
 _lib.dsa_index_topk_workspace_bytes.argtypes = [_i32, _i32, _i32]
 _lib.dsa_index_topk_workspace_bytes.restype = _sz
@@ -187,6 +189,25 @@ def attn_decode_gqa(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, ws
     _check(_lib.attn_decode_gqa(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H, Hk, d, T_max,
                                 float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status),
                                 _stream()))
+    return out, lse
+
+
+def attn_decode_gqa_noalloc(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, dev_status=None,
+                            want_lse=True):
+    """attn_decode_gqa without a workspace: the library's static device scratch
+    is used (shared by every call on the device; see include/kvattn.h)."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    _need(seq_lens, torch.int32, "seq_lens")
+    B, H, d = q.shape
+    _, Hk, T_max, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    _check(_lib.attn_decode_gqa_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H, Hk, d, T_max,
+                                        float(scale), _ptr(out), _ptr(lse), _ptr(dev_status), _stream()))
     return out, lse
 
 
