@@ -216,7 +216,7 @@ int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* 
  * (-1 = unused slot; other values outside [0, L_max) are skipped and set
  * KVATTN_STATUS_BAD_INDEX).  out [B][Hq][Dv] bf16; lse [B][Hq] fp32 or NULL.
  * A row with no valid index gives out = 0, lse = -inf.
- * Supported: Dk = 576, Dv = 512, Hq in {16, 32, 64, 128}, 1 <= k <= 2048.
+ * Supported: Dk = 576, Dv = 512, Hq in {64, 128}, 1 <= k <= 2048.
  */
 size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k);
 

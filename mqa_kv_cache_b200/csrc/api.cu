@@ -297,32 +297,75 @@ int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn
 
 size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k)
 {
-    (void)B, (void)L_max, (void)k;
-    return 0;
+    (void)k;
+    if (B < 1 || L_max < 1) return 0;
+    return align_up(kvattn::dsa_scores_bytes(B, L_max));
 }
 
 int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* k_idx, const int32_t* seq_lens, int B,
                    int n_idx_head, int idx_dim, int L_max, int k, int32_t* topk_idx, float* scores_out,
                    void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
 {
-    (void)q_idx, (void)w, (void)k_idx, (void)seq_lens, (void)B, (void)n_idx_head, (void)idx_dim, (void)L_max, (void)k;
-    (void)topk_idx, (void)scores_out, (void)workspace, (void)workspace_bytes, (void)dev_status, (void)stream;
-    return fail(KVATTN_ERR_UNSUPPORTED, "dsa_index_topk: not built yet");
+    if (!q_idx || !w || !k_idx || !topk_idx) return fail(KVATTN_ERR_NULL, "dsa_index_topk: NULL argument");
+    if (n_idx_head != 64 || idx_dim != 128)
+        return fail(KVATTN_ERR_UNSUPPORTED, "dsa_index_topk: needs 64 indexer heads of width 128 (got %d x %d)",
+                    n_idx_head, idx_dim);
+    if (B < 1 || L_max < 1 || k < 1 || k > 2048)
+        return fail(KVATTN_ERR_SHAPE, "dsa_index_topk: B %d, L_max %d, k %d (k must be 1..2048)", B, L_max, k);
+    if (static_cast<long long>(B) * L_max > (1ll << 31))
+        return fail(KVATTN_ERR_SHAPE, "dsa_index_topk: B * L_max too large");
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(topk_idx) ||
+        (scores_out && !aligned16(scores_out)))
+        return fail(KVATTN_ERR_ALIGN, "dsa_index_topk: tensors must be 16-byte aligned");
+    float* scores = scores_out;
+    if (!scores) {
+        const size_t need = align_up(kvattn::dsa_scores_bytes(B, L_max));
+        if (!workspace || workspace_bytes < need)
+            return fail(KVATTN_ERR_WORKSPACE, "dsa_index_topk: workspace needs %zu bytes when scores_out is NULL",
+                        need);
+        if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
+            return fail(KVATTN_ERR_ALIGN, "dsa_index_topk: workspace must be 256-byte aligned");
+        scores = static_cast<float*>(workspace);
+    }
+    int sms = 0;
+    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "dsa_index_topk: no CUDA device");
+    CUtensorMap tm_k, tm_q;
+    if (make_map_3d(&tm_k, k_idx, 128, L_max, B, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_3d(&tm_q, q_idx, 128, 64, B, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    kvattn::DsaIndexArgs a{w, seq_lens, scores, topk_idx, dev_status, B, L_max, k, sms};
+    return cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, static_cast<cudaStream_t>(stream)),
+                       "dsa_index_topk launch");
 }
 
 size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k)
 {
-    (void)B, (void)Hq, (void)Dv, (void)k;
-    return 0;
+    if (B < 1 || Hq < 1 || Dv != 512 || k < 1) return 0;
+    return align_up(kvattn::sparse_partial_bytes(B, Hq, k));
 }
 
 int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const int32_t* topk_idx, int B, int Hq, int Dk,
                        int Dv, int L_max, int k, float scale, kvattn_bf16* out, float* lse, void* workspace,
                        size_t workspace_bytes, int32_t* dev_status, void* stream)
 {
-    (void)q, (void)latent, (void)topk_idx, (void)B, (void)Hq, (void)Dk, (void)Dv, (void)L_max, (void)k, (void)scale;
-    (void)out, (void)lse, (void)workspace, (void)workspace_bytes, (void)dev_status, (void)stream;
-    return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_sparse: not built yet");
+    if (!q || !latent || !topk_idx || !out) return fail(KVATTN_ERR_NULL, "attn_decode_sparse: NULL argument");
+    if (Dk != 576 || Dv != 512)
+        return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_sparse: needs Dk 576, Dv 512 (got %d, %d)", Dk, Dv);
+    if (Hq != 64 && Hq != 128)
+        return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_sparse: Hq must be 64 or 128 (got %d)", Hq);
+    if (B < 1 || L_max < 1 || k < 1 || k > 2048)
+        return fail(KVATTN_ERR_SHAPE, "attn_decode_sparse: B %d, L_max %d, k %d (k must be 1..2048)", B, L_max, k);
+    if (!(scale > 0.0f) || !std::isfinite(scale))
+        return fail(KVATTN_ERR_SHAPE, "attn_decode_sparse: scale must be finite > 0");
+    if (!aligned16(q) || !aligned16(latent) || !aligned16(out) || !aligned16(topk_idx))
+        return fail(KVATTN_ERR_ALIGN, "attn_decode_sparse: tensors must be 16-byte aligned");
+    const size_t need = align_up(kvattn::sparse_partial_bytes(B, Hq, k));
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return fail(KVATTN_ERR_WORKSPACE, "attn_decode_sparse: workspace needs %zu bytes", need);
+    if (need > 0 && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
+        return fail(KVATTN_ERR_ALIGN, "attn_decode_sparse: workspace must be 256-byte aligned");
+    kvattn::SparseLaunch l{q, latent, topk_idx, out, lse, need > 0 ? static_cast<float*>(workspace) : nullptr,
+                           dev_status, B, Hq, L_max, k, scale};
+    return cuda_status(kvattn::launch_sparse_attn(l, static_cast<cudaStream_t>(stream)), "attn_decode_sparse launch");
 }
 
 }  // extern "C"

@@ -300,14 +300,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (long long t = tb; t < te; ++t, ++it) {
             const int s = it % C::STAGES;
             const uint32_t ph = (it / C::STAGES) & 1;
-            bool have = false;
-            if (!*s_abort) {
-                have = mbar_wait(&full[s], ph);
-                if (!have) {
-                    *s_abort = 1;
-                    report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
-                }
-            }
+            const bool have = warp_wait(&full[s], ph, s_abort);
+            if (!have && lane == 0) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
             if (have) {
                 const uint32_t sK = smem_u32(smem + s * C::STAGE_BYTES);
                 const uint32_t sV = sK + C::TILE_BYTES;

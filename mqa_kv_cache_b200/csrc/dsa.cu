@@ -1,0 +1,500 @@
+// dsa.cu -- DeepSeek-V3.2-style lightning indexer and top-k selection.
+//
+// Indexer ("Agentic RL 入门3：transformer 架构" §2.2 (1); "attention", DSA ①):
+//   s_{b,t} = sum_{j<64} w[b][j] * ReLU(q_idx[b][j] . k_idx[b][t])
+// with 64 indexer heads sharing one 128-wide key per token.  Per batch row this
+// is a [L x 128] x [128 x 64] contraction followed by a ReLU-weighted reduction
+// over the 64 heads, so it runs on the tensor cores: tcgen05.mma with the 128
+// tokens of a tile as M, the 64 heads as N and K = 128, the fp32 accumulator
+// in TMEM (two 64-column buffers so the epilogue of one tile overlaps the MMA
+// of the next), and the head reduction fused into the TMEM read-out.  It is
+// bound by the one read of k_idx from HBM (intensity ~63 FLOP/byte).
+//
+// Top-k (§2.2 (2): S = TopK_t(s_t), ties to the lower index): one cluster of
+// 8 CTAs per batch row runs an exact 3-digit (11/11/10-bit) radix select on
+// order-preserving 32-bit keys of the fp32 scores, with the histograms summed
+// through distributed shared memory; the selected (key, index) pairs are then
+// sorted by (score desc, index asc) in the cluster's first CTA.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace kvattn {
+
+namespace {
+
+// ---- indexer ------------------------------------------------------------------
+
+constexpr int IX_TOK = 128;   // tokens per tile (MMA M)
+constexpr int IX_HEADS = 64;  // indexer heads (MMA N)
+constexpr int IX_DIM = 128;   // key width (MMA K)
+constexpr int IX_STAGES = 6;
+constexpr int IX_BOX = IX_TOK * 128;          // one 64-column SW128 box of a k tile (bytes)
+constexpr int IX_TILE = 2 * IX_BOX;           // k tile [128 x 128] bf16
+constexpr int IX_QBOX = IX_HEADS * 128;       // one 64-column box of q [64 x 64]
+constexpr int IX_QBYTES = 2 * IX_QBOX;
+constexpr int IX_THREADS = 192;               // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 epilogue
+constexpr int IX_TMEM_COLS = 128;             // two 64-column accumulators
+constexpr uint32_t IX_IDESC = umma_idesc_bf16(IX_TOK, IX_HEADS);
+
+constexpr int IX_OFF_Q = IX_STAGES * IX_TILE;
+constexpr int IX_OFF_W = IX_OFF_Q + IX_QBYTES;
+constexpr int IX_OFF_BAR = IX_OFF_W + IX_HEADS * 4;
+// full[S], empty[S], q_full, q_empty, acc_full[2], acc_empty[2], mma_done
+constexpr int IX_NBAR = 2 * IX_STAGES + 7;
+constexpr int IX_OFF_MISC = IX_OFF_BAR + IX_NBAR * 8;
+constexpr int IX_SMEM = IX_OFF_MISC + 32 + 1024;
+
+struct IndexerArgs {
+    const float* w;
+    const int32_t* seq_lens;
+    float* scores;
+    int32_t* dev_status;
+    int B, L_max, tiles_per_b, chunks_per_b;
+};
+
+__device__ __forceinline__ void ix_item(const IndexerArgs& a, int item, int& b, int& t0, int& t1)
+{
+    b = item / a.chunks_per_b;
+    const int c = item - b * a.chunks_per_b;
+    t0 = static_cast<int>(static_cast<long long>(c) * a.tiles_per_b / a.chunks_per_b);
+    t1 = static_cast<int>(static_cast<long long>(c + 1) * a.tiles_per_b / a.chunks_per_b);
+}
+
+__global__ void __launch_bounds__(IX_THREADS, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, IndexerArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + IX_OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + IX_STAGES;
+    uint64_t* q_full = bars + 2 * IX_STAGES;
+    uint64_t* q_empty = q_full + 1;
+    uint64_t* acc_full = q_full + 2;
+    uint64_t* acc_empty = q_full + 4;
+    uint64_t* mma_done = q_full + 6;
+    float* s_w = reinterpret_cast<float*>(smem + IX_OFF_W);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + IX_OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + IX_OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_items = a.B * a.chunks_per_b;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < IX_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
+        mbar_init(mma_done, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem, IX_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ===== TMA producer =====
+        if (lane == 0) {
+            int it = 0, n = 0;
+            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
+                int b, t0, t1;
+                ix_item(a, item, b, t0, t1);
+                if (n > 0 && !mbar_wait(q_empty, (n - 1) & 1)) {
+                    *s_abort = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(q_full, IX_QBYTES);
+                tma_load_3d(smem + IX_OFF_Q, &tm_q, q_full, 0, 0, b);
+                tma_load_3d(smem + IX_OFF_Q + IX_QBOX, &tm_q, q_full, 64, 0, b);
+                for (int t = t0; t < t1; ++t, ++it) {
+                    const int s = it % IX_STAGES;
+                    if (it >= IX_STAGES && (*s_abort || !mbar_wait(&empty[s], ((it / IX_STAGES) - 1) & 1))) {
+                        *s_abort = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], IX_TILE);
+                    uint8_t* dst = smem + s * IX_TILE;
+                    tma_load_3d(dst, &tm_k, &full[s], 0, t * IX_TOK, b);
+                    tma_load_3d(dst + IX_BOX, &tm_k, &full[s], 64, t * IX_TOK, b);
+                }
+            }
+            if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            for (int j = it - IX_STAGES > 0 ? it - IX_STAGES : 0; j < it; ++j)
+                mbar_wait(&full[j % IX_STAGES], (j / IX_STAGES) & 1);
+        }
+    } else if (warp == 1) {
+        // ===== MMA issuer (one thread) =====
+        if (lane == 0) {
+            const uint32_t q_addr = smem_u32(smem + IX_OFF_Q);
+            int it = 0, tc = 0, n = 0;
+            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
+                int b, t0, t1;
+                ix_item(a, item, b, t0, t1);
+                if (!mbar_wait(q_full, n & 1)) {
+                    *s_abort = 1;
+                    break;
+                }
+                for (int t = t0; t < t1; ++t, ++it, ++tc) {
+                    const int s = it % IX_STAGES;
+                    const int buf = tc & 1;
+                    if (*s_abort || !mbar_wait(&full[s], (it / IX_STAGES) & 1) ||
+                        (tc >= 2 && !mbar_wait(&acc_empty[buf], ((tc >> 1) - 1) & 1))) {
+                        *s_abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(smem + s * IX_TILE);
+                    const uint32_t d_addr = tmem + buf * IX_HEADS;
+#pragma unroll
+                    for (int ks = 0; ks < IX_DIM / 16; ++ks) {
+                        const uint32_t off = (ks & 3) * 32;
+                        const uint64_t ad = umma_desc_k_sw128(k_addr + (ks >> 2) * IX_BOX + off);
+                        const uint64_t bd = umma_desc_k_sw128(q_addr + (ks >> 2) * IX_QBOX + off);
+                        tc_mma_bf16(d_addr, ad, bd, IX_IDESC, ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[s]);
+                    tc_commit(&acc_full[buf]);
+                }
+                tc_commit(q_empty);
+            }
+            // every issued MMA has finished before the accumulators are released
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
+            if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+        }
+    } else {
+        // ===== epilogue: TMEM -> ReLU, weight, sum over heads -> scores =====
+        const int quarter = warp & 3;  // TMEM lanes this warp may read
+        const int row = quarter * 32 + lane;
+        const int ep = threadIdx.x - 64;
+        int tc = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+            int b, t0, t1;
+            ix_item(a, item, b, t0, t1);
+            const int len_raw = a.seq_lens ? a.seq_lens[b] : a.L_max;
+            const int len = min(max(len_raw, 0), a.L_max);
+            if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
+            named_bar_sync(2, 128);
+            if (ep < IX_HEADS) s_w[ep] = a.w[static_cast<long long>(b) * IX_HEADS + ep];
+            named_bar_sync(2, 128);
+            float* out = a.scores + static_cast<long long>(b) * a.L_max;
+            for (int t = t0; t < t1; ++t, ++tc) {
+                const int buf = tc & 1;
+                // on an abort the loops still run to the end (without waiting or
+                // working) so that all four warps meet at the same named barriers
+                if (!warp_wait(&acc_full[buf], (tc >> 1) & 1, s_abort)) continue;
+                tc_fence_after();
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_HEADS;
+                uint32_t v0[32], v1[32];
+                tmem_ld32(taddr, v0);
+                tmem_ld32(taddr + 32, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[j], fmaxf(__uint_as_float(v0[j]), 0.f), acc);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), acc);
+                const int tok = t * IX_TOK + row;
+                if (acc != acc) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
+                if (tok < a.L_max) out[tok] = tok < len ? acc : -INFINITY;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, IX_TMEM_COLS);
+    }
+}
+
+// ---- top-k --------------------------------------------------------------------
+
+constexpr int TK_CL = 8;  // CTAs per batch row (one cluster)
+constexpr int TK_THREADS = 1024;
+
+// Order-preserving 32-bit key of an fp32 score (larger score, larger key);
+// -0 is first made +0 so that it ties with +0; NaN maps to 0 (never selected
+// ahead of a number) and is reported.
+__device__ __forceinline__ uint32_t score_key(float f, bool& nan)
+{
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) {
+        nan = true;
+        return 0u;
+    }
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Block-wide inclusive scan (sum) of one value per thread; TK_THREADS threads.
+__device__ __forceinline__ int block_incl_scan(int v, int* s_warp)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    if (lane == 31) s_warp[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = s_warp[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += t;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int r = v + (warp > 0 ? s_warp[warp - 1] : 0);
+    __syncthreads();
+    return r;
+}
+
+struct TopkArgs {
+    const float* scores;
+    const int32_t* seq_lens;
+    int32_t* out;
+    int32_t* dev_status;
+    int L_max, k;
+};
+
+__global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
+{
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int row = blockIdx.x / TK_CL;
+    const int tid = threadIdx.x;
+
+    __shared__ uint32_t hist[2048];
+    __shared__ uint32_t tot[2048];
+    __shared__ unsigned long long sel[2048];
+    __shared__ int s_warp[32];
+    __shared__ uint32_t s_state[2];  // prefix, k_rem (written by rank 0 into every CTA)
+    __shared__ int s_counts[2];      // this CTA's (#key > T, #key == T)
+    __shared__ int s_nan;
+
+    pdl_wait();
+    pdl_trigger();
+
+    const int len_raw = a.seq_lens ? a.seq_lens[row] : a.L_max;
+    const int len = min(max(len_raw, 0), a.L_max);
+    if (len != len_raw && rank == 0 && tid == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
+    const int kk = min(a.k, len);
+    const int slice = (len + TK_CL - 1) / TK_CL;
+    const int lo = min(rank * slice, len), hi = min(lo + slice, len);
+    const float* sc = a.scores + static_cast<long long>(row) * a.L_max;
+    if (tid == 0) s_nan = 0;
+    bool nan = false;
+
+    uint32_t prefix = 0u, k_rem = static_cast<uint32_t>(kk);
+    uint32_t known = 0u;  // mask of key bits already fixed
+    if (len > a.k) {
+        const int shifts[3] = {21, 10, 0};
+        const int widths[3] = {11, 11, 10};
+        for (int p = 0; p < 3; ++p) {
+            const int sh = shifts[p], nb = 1 << widths[p];
+            for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
+            __syncthreads();
+            for (int i = lo + tid; i < hi; i += TK_THREADS) {
+                const uint32_t key = score_key(sc[i], nan);
+                if ((key & known) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+            }
+            cluster.sync();
+            // rank r sums bins [r nb/8, (r+1) nb/8) over the cluster into rank 0's `tot`
+            const int per = nb / TK_CL;
+            uint32_t* tot0 = cluster.map_shared_rank(tot, 0);
+            for (int bin = rank * per + tid; bin < (rank + 1) * per; bin += TK_THREADS) {
+                uint32_t v = 0u;
+#pragma unroll
+                for (int q = 0; q < TK_CL; ++q) v += cluster.map_shared_rank(hist, q)[bin];
+                tot0[bin] = v;
+            }
+            cluster.sync();
+            if (rank == 0) {
+                // suffix sums over bins (from the largest digit down): each thread owns 2 bins
+                const int b0 = nb - 1 - 2 * tid, b1 = b0 - 1;
+                const int c0 = (2 * tid < nb) ? static_cast<int>(tot[b0]) : 0;
+                const int c1 = (2 * tid + 1 < nb) ? static_cast<int>(tot[b1]) : 0;
+                const int incl = block_incl_scan(c0 + c1, s_warp);
+                const int before = incl - c0 - c1;  // keys in digits above b0
+                const int kr = static_cast<int>(k_rem);
+                if (2 * tid < nb && before < kr && before + c0 >= kr) {
+                    s_state[0] = prefix | (static_cast<uint32_t>(b0) << sh);
+                    s_state[1] = static_cast<uint32_t>(kr - before);
+                } else if (2 * tid + 1 < nb && before + c0 < kr && before + c0 + c1 >= kr) {
+                    s_state[0] = prefix | (static_cast<uint32_t>(b1) << sh);
+                    s_state[1] = static_cast<uint32_t>(kr - before - c0);
+                }
+                __syncthreads();
+                if (tid < TK_CL) {
+                    uint32_t* st = cluster.map_shared_rank(s_state, tid);
+                    st[0] = s_state[0];
+                    st[1] = s_state[1];
+                }
+            }
+            cluster.sync();
+            prefix = s_state[0];
+            k_rem = s_state[1];
+            known |= static_cast<uint32_t>(nb - 1) << sh;
+        }
+    } else {
+        prefix = 0u;  // every number has a key above 0: all of them are taken
+        known = 0xffffffffu;
+    }
+    const uint32_t T = prefix;
+
+    // ---- ordered compaction: each thread owns a contiguous run of the slice ----
+    const int run = (hi - lo + TK_THREADS - 1) / TK_THREADS;
+    const int r0 = min(lo + tid * run, hi), r1 = min(r0 + run, hi);
+    int n_gt = 0, n_eq = 0;
+    for (int i = r0; i < r1; ++i) {
+        const uint32_t key = score_key(sc[i], nan);
+        n_gt += key > T;
+        n_eq += key == T && T != 0u;
+    }
+    const int inc_gt = block_incl_scan(n_gt, s_warp);
+    const int inc_eq = block_incl_scan(n_eq, s_warp);
+    if (tid == TK_THREADS - 1) {
+        s_counts[0] = inc_gt;
+        s_counts[1] = inc_eq;
+    }
+    cluster.sync();
+    int gt_off = 0, eq_off = 0, gt_total = 0, eq_total = 0;
+    for (int q = 0; q < TK_CL; ++q) {
+        const int* c = cluster.map_shared_rank(s_counts, q);
+        if (q < rank) {
+            gt_off += c[0];
+            eq_off += c[1];
+        }
+        gt_total += c[0];
+        eq_total += c[1];
+    }
+    const int take_eq = kk - gt_total;  // keys equal to T that are still needed
+    unsigned long long* sel0 = cluster.map_shared_rank(sel, 0);
+    int pg = gt_off + inc_gt - n_gt, pe = eq_off + inc_eq - n_eq;
+    for (int i = r0; i < r1; ++i) {
+        const uint32_t key = score_key(sc[i], nan);
+        const unsigned long long comp =
+            (static_cast<unsigned long long>(0xffffffffu - key) << 32) | static_cast<uint32_t>(i);
+        if (key > T) {
+            sel0[pg++] = comp;
+        } else if (key == T && T != 0u) {
+            if (pe < take_eq) sel0[gt_total + pe] = comp;
+            ++pe;
+        }
+    }
+    if (nan) s_nan = 1;
+    cluster.sync();
+    if (rank == 0) {
+        // sort the k selected entries by (score desc, index asc)
+        // entries actually selected (fewer than kk only when NaN scores were skipped)
+        const int n_sel = gt_total + min(take_eq, eq_total);
+        int n = 1;
+        while (n < kk) n <<= 1;
+        for (int i = n_sel + tid; i < n; i += TK_THREADS) sel[i] = ~0ull;
+        __syncthreads();
+        for (int size = 2; size <= n; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int i = tid; i < (n >> 1); i += TK_THREADS) {
+                    const int x = 2 * stride * (i / stride) + (i % stride);
+                    const int y = x + stride;
+                    const bool asc = (x & size) == 0;
+                    const unsigned long long u = sel[x], v = sel[y];
+                    if ((u > v) == asc) {
+                        sel[x] = v;
+                        sel[y] = u;
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        int32_t* out = a.out + static_cast<long long>(row) * a.k;
+        for (int j = tid; j < a.k; j += TK_THREADS)
+            out[j] = j < kk ? static_cast<int32_t>(sel[j] & 0xffffffffull) : -1;
+    }
+    __syncthreads();
+    if (s_nan && tid == 0) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
+    cluster.sync();  // no CTA leaves while others may still touch its shared memory
+}
+
+}  // namespace
+
+size_t dsa_scores_bytes(int B, int L_max) { return static_cast<size_t>(B) * L_max * sizeof(float); }
+
+cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
+                                  cudaStream_t stream)
+{
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX_SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    IndexerArgs ia{};
+    ia.w = a.w;
+    ia.seq_lens = a.seq_lens;
+    ia.scores = a.scores;
+    ia.dev_status = a.dev_status;
+    ia.B = a.B;
+    ia.L_max = a.L_max;
+    ia.tiles_per_b = (a.L_max + IX_TOK - 1) / IX_TOK;
+    // about two contiguous chunks per CTA, never more chunks than tiles
+    int chunks = (2 * a.num_sms + a.B - 1) / a.B;
+    if (chunks > ia.tiles_per_b) chunks = ia.tiles_per_b;
+    if (chunks < 1) chunks = 1;
+    ia.chunks_per_b = chunks;
+    const int items = a.B * chunks;
+    const int grid = items < a.num_sms ? items : a.num_sms;
+    e = launch_pdl(indexer_kernel, dim3(grid), dim3(IX_THREADS), IX_SMEM, stream, tm_k, tm_q, ia);
+    if (e != cudaSuccess) return e;
+
+    TopkArgs ta{a.scores, a.seq_lens, a.topk_idx, a.dev_status, a.L_max, a.k};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * TK_CL);
+    cfg.blockDim = dim3(TK_THREADS);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = TK_CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, topk_kernel, ta);
+}
+
+}  // namespace kvattn

@@ -77,4 +77,33 @@ int decode_grid(int num_sms);
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                           cudaStream_t stream);
 
+// ---- lightning indexer + top-k ----
+struct DsaIndexArgs {
+    const float* w;
+    const int32_t* seq_lens;
+    float* scores;      // [B][L_max] fp32 (caller's scores_out or workspace)
+    int32_t* topk_idx;  // [B][k]
+    int32_t* dev_status;
+    int B, L_max, k, num_sms;
+};
+size_t dsa_scores_bytes(int B, int L_max);
+cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
+                                  cudaStream_t stream);
+
+// ---- sparse latent attention ----
+struct SparseLaunch {
+    const kvattn_bf16* q;
+    const kvattn_bf16* latent;
+    const int32_t* idx;
+    kvattn_bf16* out;
+    float* lse;
+    float* workspace;  // chunk partials (null when one chunk)
+    int32_t* dev_status;
+    int B, Hq, L_max, k;
+    float scale;
+};
+int sparse_chunks(int k);
+size_t sparse_partial_bytes(int B, int Hq, int k);
+cudaError_t launch_sparse_attn(const SparseLaunch& l, cudaStream_t stream);
+
 }  // namespace kvattn
