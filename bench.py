@@ -162,6 +162,12 @@ def capture(fn):
     return g
 
 
+def flush_l2(buf):
+    """Evict L2 by reading a buffer twice its size (clean lines: no write-back
+    of flush data can land inside the next timed step)."""
+    torch.sum(buf, dtype=torch.int32)
+
+
 def time_steps(fn, steps, flush, before=None):
     """Per-step CUDA-event times (ms) on the current stream, L2 flushed between steps."""
     st = torch.cuda.current_stream()
@@ -169,7 +175,7 @@ def time_steps(fn, steps, flush, before=None):
     for a, b in evs:
         if before is not None:
             before()
-        flush.zero_()
+        flush_l2(flush)
         a.record(st)
         fn()
         b.record(st)
@@ -254,7 +260,7 @@ def run_gpu(args, rank, world, device):
         "config": {"workload": w.name, "B": w.B, "n_head": w.H, "n_kv_head": w.Hk, "head_dim": w.d,
                    "T_max": w.T_max, "mean_len": float(job.lens_host.float().mean()), "rope_base": w.rope.base,
                    "parallelism": f"dp{world} (independent batches)",
-                   "l2": "flushed between timed steps (256 MB write), and inputs exceed L2"},
+                   "l2": "flushed between timed steps (read of a 256 MB buffer), and inputs exceed L2"},
         "tok_per_s": round(w.B * world / (ms * 1e-3), 1),
         "step_launch": "CUDA graph replay (eager Python launch: %.4f ms/step)" % eager_ms,
         "pct_of_hbm_peak": round(100.0 * gbs / world / peaks["hbm_gbs"], 2),
@@ -269,6 +275,121 @@ def run_gpu(args, rank, world, device):
         "clocks": sampler.summary(),
     }
     return line
+
+
+# ---------------------------------------------------------------------------- other configurations
+
+def _graph_ms(fn, steps, flush, warmup=3, before=None):
+    for _ in range(warmup):
+        if before is not None:
+            before()
+        fn()
+    torch.cuda.synchronize()
+    g = capture(fn)
+    return float(np.median(time_steps(g.replay, steps, flush, before=before)))
+
+
+def measure_decode_config(K, w, device, steps, flush, peaks):
+    job = DecodeStep(K, w, device, W.SEED_BASE + w.index)
+    ms = _graph_ms(job.step, steps, flush, before=job.reset_q)
+    attn_ms = _graph_ms(job.attn, steps, flush)
+    out = {"workload": w.name, "ms_per_step": round(ms, 5), "attn_ms": round(attn_ms, 5),
+           "algorithmic_bytes": job.bytes, "GB_s": round(job.bytes / (ms * 1e-3) / 1e9, 1),
+           "attn_GB_s": round(job.bytes / (attn_ms * 1e-3) / 1e9, 1),
+           "attn_pct_of_hbm_peak": round(100 * job.bytes / (attn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 1),
+           "tok_per_s": round(w.B / (ms * 1e-3), 1)}
+    del job
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_prefill(K, device, steps, flush, peaks):
+    w = W.PREFILL_8K
+    gen = W.generator(W.SEED_BASE + w.index, device)
+    q_raw = W.normal_bf16((w.B, w.T, w.H, w.d), gen, device)
+    k_raw = W.normal_bf16((w.B, w.Hk, w.T, w.d), gen, device)
+    v = W.normal_bf16((w.B, w.Hk, w.T, w.d), gen, device)
+    q, k = q_raw.clone(), k_raw.clone()
+    pos = torch.arange(w.T, dtype=torch.int32, device=device).repeat(w.B, 1)
+    cos, sin = K.rope_table_build(K.rope_params(w.d, base=w.rope.base), w.T, device=device)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=device)
+
+    def reset():
+        q.copy_(q_raw)
+        k.copy_(k_raw)
+
+    def rope():
+        K.rope_apply_qk(q, pos, k, pos, cos, sin, q_layout="bthd", k_layout="bhtd")
+
+    def attn():
+        K.attn_prefill_causal(q, k, v, w.scale, out=out, lse=lse)
+
+    def step():
+        rope()
+        attn()
+
+    flops = 4.0 * w.B * w.H * w.d * w.T * (w.T + 1) / 2
+    attn_ms = _graph_ms(attn, max(10, steps // 10), flush)
+    step_ms = _graph_ms(step, max(10, steps // 10), flush, before=reset)
+    rope_ms = _graph_ms(rope, max(10, steps // 10), flush, before=reset)
+    rope_bytes = 2 * 2 * (q.numel() + k.numel())
+    tf = flops / (attn_ms * 1e-3) / 1e12
+    return {"workload": w.name, "attn_ms": round(attn_ms, 4), "step_ms": round(step_ms, 4),
+            "causal_flops": flops, "attn_TFLOP_s": round(tf, 1),
+            "pct_of_bf16_peak_burst": round(100 * tf / peaks["bf16_tflops"], 1),
+            "pct_of_bf16_peak_sustained": round(100 * tf / peaks["bf16_tflops_sustained"], 1),
+            "rope_apply_ms": round(rope_ms, 4), "rope_apply_GB_s": round(rope_bytes / (rope_ms * 1e-3) / 1e9, 1),
+            "tok_per_s": round(w.B * w.T / (step_ms * 1e-3), 1)}
+
+
+def measure_dsa(K, device, steps, flush, peaks):
+    w = W.DSA_128K
+    gen = W.generator(W.SEED_BASE + w.index, device)
+    q_idx = W.normal_bf16((w.B, w.HI, w.dI), gen, device)
+    wt = W.uniform_f32((w.B, w.HI), gen, device)
+    k_idx = W.normal_bf16((w.B, w.L, w.dI), gen, device)
+    q = W.normal_bf16((w.B, w.Hq, w.Dk), gen, device)
+    latent = W.normal_bf16((w.B, w.L, w.Dk), gen, device)
+    idx = torch.empty((w.B, w.k), dtype=torch.int32, device=device)
+    scores = torch.empty((w.B, w.L), dtype=torch.float32, device=device)
+    out = torch.empty((w.B, w.Hq, w.Dv), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
+    ws1 = K.workspace(K.dsa_index_topk_workspace_bytes(w.B, w.L, w.k), device)
+    ws2 = K.workspace(K.attn_decode_sparse_workspace_bytes(w.B, w.Hq, w.Dv, w.k), device)
+
+    def index():
+        K.dsa_index_topk(q_idx, wt, k_idx, w.k, topk_idx=idx, scores_out=scores, ws=ws1)
+
+    def sparse():
+        K.attn_decode_sparse(q, latent, idx, w.Dv, w.sparse_scale, out=out, lse=lse, ws=ws2)
+
+    def step():
+        index()
+        sparse()
+
+    n = max(10, steps // 5)
+    index_ms = _graph_ms(index, n, flush)
+    sparse_ms = _graph_ms(sparse, n, flush)
+    step_ms = _graph_ms(step, n, flush)
+    idx_bytes = w.B * w.L * w.dI * 2
+    sp_bytes = w.B * w.k * w.Dk * 2
+    sp_flops = 2.0 * w.B * w.Hq * w.k * (w.Dk + w.Dv)
+    return {"workload": w.name, "step_ms": round(step_ms, 4), "tok_per_s": round(w.B / (step_ms * 1e-3), 1),
+            "index_topk_ms": round(index_ms, 4),
+            "indexer_GB_s_incl_topk": round(idx_bytes / (index_ms * 1e-3) / 1e9, 1),
+            "sparse_ms": round(sparse_ms, 4), "sparse_TFLOP_s": round(sp_flops / (sparse_ms * 1e-3) / 1e12, 1),
+            "sparse_gathered_bytes": sp_bytes}
+
+
+def measure_others(K, device, steps, flush, peaks):
+    res = {}
+    for w in (W.TINY_GQA, W.LLAMA2_70B_GQA_32K, W.LLAMA2_70B_MQA_32K, W.LLAMA2_70B_MHA_32K):
+        res[w.name] = measure_decode_config(K, w, device, steps, flush, peaks)
+    res[W.PREFILL_8K.name] = measure_prefill(K, device, steps, flush, peaks)
+    res[W.DSA_128K.name] = measure_dsa(K, device, steps, flush, peaks)
+    torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------------------- CPU oracle
@@ -360,6 +481,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="kvattn", choices=["kvattn", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true", help="skip the other configurations")
+    ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "prefill", "dsa"],
+                    help="time one other configuration alone and print its JSON")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -372,6 +496,24 @@ def main():
             print(json.dumps(run_reference(args)), flush=True)
         return 0
 
+    if args.only:
+        from mqa_kv_cache_b200 import kvattn as K
+        device = torch.device("cuda", local_rank)
+        torch.cuda.set_device(device)
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        peaks = load_peaks()
+        decode = {"tiny": W.TINY_GQA, "gqa32k": W.LLAMA2_70B_GQA_32K, "mqa32k": W.LLAMA2_70B_MQA_32K,
+                  "mha32k": W.LLAMA2_70B_MHA_32K}
+        if args.only in decode:
+            res = measure_decode_config(K, decode[args.only], device, args.steps, flush, peaks)
+        elif args.only == "prefill":
+            res = measure_prefill(K, device, args.steps, flush, peaks)
+        else:
+            res = measure_dsa(K, device, args.steps, flush, peaks)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return 0
+
     if world > 1:
         import datetime
         torch.cuda.set_device(local_rank)
@@ -380,6 +522,10 @@ def main():
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     line = run_gpu(args, rank, world, device)
+    if not args.headline_only:
+        from mqa_kv_cache_b200 import kvattn as K
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+        line["other_configs"] = measure_others(K, device, args.steps, flush, load_peaks())
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if world > 1:

@@ -94,6 +94,24 @@ int make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint
     return KVATTN_OK;
 }
 
+// 4-D bf16 tensor map over [w][z][y][x] with a {64, 1, box_z, 1} box and
+// 128-byte swizzle (one head's rows of a [B][T][H][d] tensor).
+int make_map_4d_rows(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint64_t w,
+                     uint32_t box_z)
+{
+    auto fn = encode_fn();
+    if (!fn) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[4] = {x, y, z, w};
+    cuuint64_t strides[3] = {x * 2, x * y * 2, x * y * z * 2};
+    cuuint32_t box[4] = {64, 1, box_z, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return KVATTN_OK;
+}
+
 int cuda_status(cudaError_t e, const char* what)
 {
     if (e != cudaSuccess) return fail(KVATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
@@ -290,9 +308,27 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
 int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B, int T, int n_head,
                         int n_kv_head, int head_dim, float scale, kvattn_bf16* out, float* lse, void* stream)
 {
-    (void)q, (void)k, (void)v, (void)B, (void)T, (void)n_head, (void)n_kv_head, (void)head_dim, (void)scale;
-    (void)out, (void)lse, (void)stream;
-    return fail(KVATTN_ERR_UNSUPPORTED, "attn_prefill_causal: not built yet");
+    if (!q || !k || !v || !out) return fail(KVATTN_ERR_NULL, "attn_prefill_causal: NULL argument");
+    if (head_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "attn_prefill_causal: head_dim %d (needs 128)", head_dim);
+    if (B < 1 || T < 1 || n_head < 1 || n_kv_head < 1 || n_head % n_kv_head)
+        return fail(KVATTN_ERR_SHAPE, "attn_prefill_causal: B %d T %d n_head %d n_kv_head %d", B, T, n_head, n_kv_head);
+    if (!g_supported(n_head / n_kv_head))
+        return fail(KVATTN_ERR_UNSUPPORTED, "attn_prefill_causal: group size %d", n_head / n_kv_head);
+    if (static_cast<long long>(B) * n_kv_head > (1ll << 31) - 1 || T > (1 << 30) ||
+        static_cast<long long>((T + 255) / 256) * B * n_head > (1ll << 31) - 1)
+        return fail(KVATTN_ERR_SHAPE, "attn_prefill_causal: problem too large");
+    if (!(scale > 0.0f) || !std::isfinite(scale))
+        return fail(KVATTN_ERR_SHAPE, "attn_prefill_causal: scale must be finite > 0");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(KVATTN_ERR_ALIGN, "attn_prefill_causal: tensors must be 16-byte aligned");
+    CUtensorMap tm_q, tm_k, tm_v;
+    if (make_map_4d_rows(&tm_q, q, head_dim, n_head, T, B, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    const uint64_t units = static_cast<uint64_t>(B) * n_kv_head;
+    if (make_map_3d(&tm_k, k, head_dim, T, units, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_3d(&tm_v, v, head_dim, T, units, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    kvattn::PrefillLaunch l{out, lse, nullptr, B, T, n_head, n_kv_head, scale};
+    return cuda_status(kvattn::launch_prefill(l, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
+                       "attn_prefill_causal launch");
 }
 
 size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k)

@@ -106,4 +106,15 @@ int sparse_chunks(int k);
 size_t sparse_partial_bytes(int B, int Hq, int k);
 cudaError_t launch_sparse_attn(const SparseLaunch& l, cudaStream_t stream);
 
+// ---- causal prefill ----
+struct PrefillLaunch {
+    kvattn_bf16* out;
+    float* lse;
+    int32_t* dev_status;
+    int B, T, H, Hk;
+    float scale;
+};
+cudaError_t launch_prefill(const PrefillLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                           const CUtensorMap& tm_v, cudaStream_t stream);
+
 }  // namespace kvattn

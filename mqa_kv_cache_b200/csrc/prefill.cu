@@ -1,0 +1,376 @@
+// prefill.cu -- causal attention over a whole prompt on the tcgen05 tensor cores.
+//
+// Method: O_i = sum_{j <= i} softmax_j(scale q_i . k_j) v_j per query head,
+// query head h reading KV head h / g ("注意力变体与 MoE", attention(): the
+// lower-triangular mask fills triu(1) with -inf; "attention",
+// GroupQueryAttention).  Both contractions (Q K^T and P V) are dense, so they
+// run on tcgen05 with fp32 accumulators in tensor memory, FlashAttention-style
+// (scores never leave the SM; "Agentic RL 入门3" §2.4: the matmul parts on tensor
+// cores, the sequential softmax parts between chunks).
+//
+// CTA = (batch, query head, block of 256 query rows) = two 128-row Q tiles that
+// share every K/V tile, so the softmax of one tile overlaps the MMAs of the
+// other.  Warps 0-3 / 4-7: softmax of Q tile 0 / 1, one thread per query row
+// (a full score row per thread: row max and sum need no shuffles); warp 8: the
+// single MMA-issuing thread; warp 9: TMA loads (Q once, then K_j, V_j through a
+// 4-slot ring).  TMEM (512 columns): S0 | S1 | O0 | O1, 128 columns each.
+// The softmax writes P (bf16, two per 32-bit column) over the first 64 columns
+// of its S buffer and the P V product takes P straight from TMEM.  The running
+// max is only moved (and O rescaled) when it grows by more than 2^8, so most
+// tiles never touch O.  Blocks of the longest query rows launch first.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvattn {
+
+namespace {
+
+constexpr int PF_D = 128;     // head dim
+constexpr int PF_BM = 128;    // query rows per Q tile
+constexpr int PF_BN = 128;    // keys per K/V tile
+constexpr int PF_SLOTS = 4;   // K/V ring slots (one tile each)
+constexpr int PF_THREADS = 320;
+constexpr int PF_TILE = PF_BN * PF_D * 2;  // 32 KB: one K or V tile, two 64-column SW128 boxes
+constexpr int PF_BOX = PF_BN * 128;        // 16 KB
+constexpr int PF_OFF_Q = 0;                // two Q tiles
+constexpr int PF_OFF_KV = 2 * PF_TILE;
+constexpr int PF_OFF_BAR = PF_OFF_KV + PF_SLOTS * PF_TILE;
+// kv_full[4], kv_empty[4], q_full, s_full[2], p_full[2], pv_done[2], mma_done
+constexpr int PF_NBAR = 2 * PF_SLOTS + 8;
+constexpr int PF_OFF_MISC = PF_OFF_BAR + PF_NBAR * 8;
+constexpr int PF_SMEM = PF_OFF_MISC + 32 + 1024;
+constexpr uint32_t PF_IDESC_S = umma_idesc_bf16(PF_BM, PF_BN);             // Q (K-major) x K (K-major)
+constexpr uint32_t PF_IDESC_O = umma_idesc_bf16(PF_BM, PF_D, false, true);  // P (tmem) x V (MN-major)
+constexpr float kLog2e = 1.44269504088896340736f;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+struct PrefillArgs {
+    kvattn_bf16* out;  // [B][T][H][d]
+    float* lse;        // [B][H][T] or null
+    int32_t* dev_status;
+    int B, T, H, Hk, g, n_qblk;
+    float scale;
+};
+
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, PrefillArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + PF_OFF_BAR);
+    uint64_t* kv_full = bars;
+    uint64_t* kv_empty = bars + PF_SLOTS;
+    uint64_t* q_full = bars + 2 * PF_SLOTS;
+    uint64_t* s_full = q_full + 1;
+    uint64_t* p_full = q_full + 3;
+    uint64_t* pv_done = q_full + 5;
+    uint64_t* mma_done = q_full + 7;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + PF_OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + PF_OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // work item: longest query blocks first
+    const int bh_count = a.B * a.H;
+    const int qblk = a.n_qblk - 1 - static_cast<int>(blockIdx.x) / bh_count;
+    const int bh = static_cast<int>(blockIdx.x) % bh_count;
+    const int b = bh / a.H, h = bh - b * a.H;
+    const int kvh = h / a.g;
+    const int q0 = qblk * 2 * PF_BM;
+    const int n_qt = (a.T - q0) > PF_BM ? 2 : 1;   // Q tiles in this block
+    // K/V tiles seen by Q tile t: keys 0 .. q0 + 128 t + 127 (the last one on the diagonal)
+    const int n_kv0 = q0 / PF_BN + 1;
+    const int n_kv = n_kv0 + (n_qt - 1);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < PF_SLOTS; ++i) {
+            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_empty[i], 1);
+        }
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&pv_done[i], 1);
+        }
+        mbar_init(mma_done, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 9 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 8) {
+        tmem_alloc(s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 9) {
+        // ===== TMA loads =====
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, n_qt * PF_TILE);
+            for (int t = 0; t < n_qt; ++t) {
+                uint8_t* dst = smem + PF_OFF_Q + t * PF_TILE;
+                tma_load_4d(dst, &tm_q, q_full, 0, h, q0 + t * PF_BM, b);
+                tma_load_4d(dst + PF_BOX, &tm_q, q_full, 64, h, q0 + t * PF_BM, b);
+            }
+            const int z = b * a.Hk + kvh;
+            int u = 0;  // ring sequence: K_0, V_0, K_1, V_1, ...
+            for (int j = 0; j < n_kv && !*s_abort; ++j) {
+                for (int kv = 0; kv < 2; ++kv, ++u) {
+                    const int slot = u % PF_SLOTS;
+                    if (u >= PF_SLOTS && !mbar_wait(&kv_empty[slot], ((u / PF_SLOTS) - 1) & 1)) {
+                        *s_abort = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&kv_full[slot], PF_TILE);
+                    uint8_t* dst = smem + PF_OFF_KV + slot * PF_TILE;
+                    const CUtensorMap* m = kv == 0 ? &tm_k : &tm_v;
+                    tma_load_3d(dst, m, &kv_full[slot], 0, j * PF_BN, z);
+                    tma_load_3d(dst + PF_BOX, m, &kv_full[slot], 64, j * PF_BN, z);
+                }
+            }
+            if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            for (int x = u - PF_SLOTS > 0 ? u - PF_SLOTS : 0; x < u; ++x)
+                mbar_wait(&kv_full[x % PF_SLOTS], (x / PF_SLOTS) & 1);
+        }
+    } else if (warp == 8) {
+        // ===== MMA issue (one thread) =====
+        if (lane == 0) {
+            const uint32_t sq = smem_u32(smem + PF_OFF_Q);
+            const uint32_t skv = smem_u32(smem + PF_OFF_KV);
+            bool ok = mbar_wait(q_full, 0);
+            int u = 0;
+            auto issue_s = [&](int t, uint32_t kslot_addr) {
+                const uint32_t d = tmem + t * PF_BN;  // S_t
+                const uint32_t qa = sq + t * PF_TILE;
+#pragma unroll
+                for (int ks = 0; ks < PF_D / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * PF_BOX + (ks & 3) * 32;
+                    tc_mma_bf16(d, umma_desc_k_sw128(qa + off), umma_desc_k_sw128(kslot_addr + off), PF_IDESC_S,
+                                ks > 0 ? 1u : 0u);
+                }
+                tc_commit(&s_full[t]);
+            };
+            auto issue_pv = [&](int t, int j, uint32_t vslot_addr) {
+                const uint32_t d = tmem + 256 + t * PF_D;  // O_t
+                const uint32_t pa = tmem + t * PF_BN;      // P_t over S_t, bf16 pairs
+#pragma unroll
+                for (int ks = 0; ks < PF_BN / 16; ++ks) {
+                    // V tile [keys][d]: 16 keys = 2 eight-row atoms (2 KB); the two 64-wide d blocks 16 KB apart
+                    const uint64_t bd = umma_desc_mn_sw128(vslot_addr + ks * 2048, PF_BOX, 1024);
+                    tc_mma_bf16_ts(d, pa + ks * 8, bd, PF_IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+                }
+                tc_commit(&pv_done[t]);
+            };
+            // S for tile 0 of every Q tile
+            int kslot = 0;
+            if (ok) {
+                kslot = u % PF_SLOTS;
+                ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
+                ++u;
+            }
+            if (ok) {
+                tc_fence_after();
+                const uint32_t ka = skv + kslot * PF_TILE;
+                if (n_kv0 > 0) issue_s(0, ka);
+                if (n_qt > 1) issue_s(1, ka);
+                tc_commit(&kv_empty[kslot]);
+            }
+            for (int j = 0; j < n_kv && ok; ++j) {
+                const int vslot = u % PF_SLOTS;
+                ok = mbar_wait(&kv_full[vslot], (u / PF_SLOTS) & 1);
+                ++u;
+                if (!ok) break;
+                const uint32_t va = skv + vslot * PF_TILE;
+                for (int t = 0; t < n_qt && ok; ++t) {
+                    if (j >= n_kv0 + t) continue;  // Q tile 0 stops one tile earlier
+                    ok = mbar_wait(&p_full[t], j & 1);
+                    if (!ok) break;
+                    tc_fence_after();
+                    issue_pv(t, j, va);
+                }
+                if (!ok) break;
+                tc_commit(&kv_empty[vslot]);
+                if (j + 1 < n_kv) {
+                    kslot = u % PF_SLOTS;
+                    ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
+                    ++u;
+                    if (!ok) break;
+                    const uint32_t ka = skv + kslot * PF_TILE;
+                    for (int t = 0; t < n_qt && ok; ++t) {
+                        if (j + 1 >= n_kv0 + t) continue;
+                        // P_t (read by the P V just issued) shares columns with S_t: wait for it
+                        ok = mbar_wait(&pv_done[t], j & 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_s(t, ka);
+                    }
+                    tc_commit(&kv_empty[kslot]);
+                }
+            }
+            if (!ok) {
+                *s_abort = 1;
+                report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            }
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+    } else {
+        // ===== softmax + epilogue: warps 0-3 -> Q tile 0, warps 4-7 -> Q tile 1 =====
+        const int t = warp >> 2;
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;  // query row in the tile = TMEM lane
+        const int qrow = q0 + t * PF_BM + row;
+        const int n_tiles = n_kv0 + t;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + t * PF_BN;
+        const uint32_t o_addr = tmem + lane_off + 256 + t * PF_D;
+        const float sl2 = a.scale * kLog2e;
+        float m_run = -INFINITY, l_run = 0.f;
+        if (t < n_qt) {
+            for (int j = 0; j < n_tiles; ++j) {
+                if (!warp_wait(&s_full[t], j & 1, s_abort)) continue;
+                tc_fence_after();
+                uint32_t sv[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sv[c]);
+                tmem_wait_ld();
+                const bool diag = j == n_tiles - 1;  // keys j*128 .. : the diagonal tile
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        float v = __uint_as_float(sv[c][i]) * sl2;
+                        if (diag && c * 32 + i > row) v = -INFINITY;
+                        sv[c][i] = __float_as_uint(v);
+                        mx = fmaxf(mx, v);
+                    }
+                }
+                // Move this row's reference max only when it grows by more than 2^8.
+                // The O rescale uses warp-collective TMEM loads/stores, so the
+                // warp takes that path together (alpha = 1 for rows that keep
+                // their reference).
+                const bool move = mx > m_run + kRescaleThreshold || m_run == -INFINITY;
+                const float m_new = move ? fmaxf(mx, m_run) : m_run;
+                const bool rescale = move && m_run != -INFINITY && j > 0;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.f;
+                    l_run *= alpha;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(o_addr + c * 32, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                        tmem_st32(o_addr + c * 32, ov);
+                    }
+                }
+                m_run = m_new;
+                const float mu = m_run == -INFINITY ? 0.f : m_run;
+                float ls = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = fast_exp2(__uint_as_float(sv[c][2 * i]) - mu);
+                        const float p1 = fast_exp2(__uint_as_float(sv[c][2 * i + 1]) - mu);
+                        ls += p0 + p1;
+                        pk[i] = pack_bf16x2(p0, p1);
+                    }
+                    // P columns 16c .. 16c+15 hold keys 32c .. 32c+31, two per column
+                    asm volatile(
+                        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(
+                            s_addr + c * 16),
+                        "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3]), "r"(pk[4]), "r"(pk[5]), "r"(pk[6]),
+                        "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]), "r"(pk[13]),
+                        "r"(pk[14]), "r"(pk[15])
+                        : "memory");
+                }
+                l_run += ls;
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[t]);
+            }
+            // ---- epilogue: O / l -> bf16 rows, lse ----
+            if (warp_wait(&pv_done[t], (n_tiles - 1) & 1, s_abort)) {
+                tc_fence_after();
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
+                                      ((static_cast<long long>(b) * a.T + qrow) * a.H + h) * PF_D;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(o_addr + c * 32, ov);
+                    tmem_wait_ld();
+                    if (qrow < a.T) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
+                            w.y = pack_bf16x2(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
+                            w.z = pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv);
+                            w.w = pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv);
+                            *reinterpret_cast<uint4*>(orow + c * 32 + i) = w;
+                        }
+                    }
+                }
+                if (a.lse && qrow < a.T)
+                    a.lse[(static_cast<long long>(b) * a.H + h) * a.T + qrow] =
+                        l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                           const CUtensorMap& tm_v, cudaStream_t stream)
+{
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    PrefillArgs a{};
+    a.out = l.out;
+    a.lse = l.lse;
+    a.dev_status = l.dev_status;
+    a.B = l.B;
+    a.T = l.T;
+    a.H = l.H;
+    a.Hk = l.Hk;
+    a.g = l.H / l.Hk;
+    a.n_qblk = (l.T + 2 * PF_BM - 1) / (2 * PF_BM);
+    a.scale = l.scale;
+    const long long grid = static_cast<long long>(a.n_qblk) * l.B * l.H;
+    return launch_pdl(prefill_kernel, dim3(static_cast<unsigned>(grid)), dim3(PF_THREADS), PF_SMEM, stream, tm_q,
+                      tm_k, tm_v, a);
+}
+
+}  // namespace kvattn

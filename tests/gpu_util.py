@@ -19,7 +19,15 @@ def rel_l2(got: np.ndarray, ref: np.ndarray) -> float:
     return float(num / den) if den > 0 else float(num)
 
 
-def assert_attn_close(out, ref_out, lse=None, ref_lse=None, what=""):
+def chain_lse_tol(q_norm, k_norm_max, scale):
+    """LSE tolerance for chains that round rotated q and k to bf16 before the
+    attention kernel: each factor carries a relative error <= 2^-9, so every
+    score moves by at most 2^-8 * scale * |q| |k| (Cauchy-Schwarz), and a
+    log-sum-exp moves by at most the largest score change."""
+    return 2.0 ** -8 * scale * q_norm * k_norm_max + LSE_ABS
+
+
+def assert_attn_close(out, ref_out, lse=None, ref_lse=None, what="", lse_tol=None):
     got = to_np_f64(out) if isinstance(out, torch.Tensor) else out
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     err = np.abs(got - ref_out)
@@ -31,8 +39,9 @@ def assert_attn_close(out, ref_out, lse=None, ref_lse=None, what=""):
         fin = np.isfinite(ref_lse)
         assert np.array_equal(np.isfinite(gl), fin), f"{what}: lse finiteness differs"
         if fin.any():
-            e = np.abs(gl[fin] - ref_lse[fin]).max()
-            assert e <= LSE_ABS, f"{what}: lse max-abs {e:.3e}"
+            tol = np.broadcast_to(LSE_ABS if lse_tol is None else lse_tol, ref_lse.shape)[fin]
+            e = np.abs(gl[fin] - ref_lse[fin])
+            assert np.all(e <= tol), f"{what}: lse error {e.max():.3e} above its bound"
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
