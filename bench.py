@@ -31,6 +31,10 @@ sys.path.insert(0, ROOT)
 from mqa_kv_cache_b200 import workloads as W  # noqa: E402
 
 METRIC = "decode-attn effective HBM GB/s (% of peak) & tok/s; prefill TFLOP/s"
+# DRAM bytes (read + write) of one decode_kernel launch on the headline workload, from the
+# ncu capture summarised in profiles/decode_kernel_llama3_8b_ragged_B16_H32_Hk8.md; None once
+# the kernel changes after that capture.
+DECODE_TRAFFIC_BYTES = 294_912_000 + 5_736_192
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -267,7 +271,7 @@ def run_gpu(args, rank, world, device):
         "pct_of_nominal_8tbs": round(100.0 * gbs / world / 8000.0, 2),
         "roofline": {"kernel": "attn_decode_gqa (split-K decode + merge)", "bound": "hbm",
                      "achieved": round(attn_gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(attn_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "frac": round(attn_gbs / peaks["hbm_gbs"], 4), "traffic": DECODE_TRAFFIC_BYTES,
                      "peak_source": peaks["source"], "algorithmic_bytes": job.bytes},
         "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
