@@ -45,6 +45,35 @@ constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
+// Degree-3 polynomial for 2^f on [-1/2, 1/2], minimax in relative error
+// (max 7.5e-5), produced by fit_exp2_poly.py in this directory.
+constexpr float kP0 = 0.99992806f, kP1 = 0.69326097f, kP2 = 0.24261113f, kP3 = 0.05517167f;
+constexpr float kShifter = 12582912.0f;  // 1.5 * 2^23: x + shifter rounds x to an integer in the low bits
+
+// 2^x for two values on the FMA pipe (Cody-Waite split x = n + f, n = rint(x)):
+// 2^x = 2^n * p(f), with 2^n applied by adding n to the exponent field.  Inputs
+// below -125 are raised to -125 (the result, ~2e-38, is zero for every use here).
+__device__ __forceinline__ float2 exp2_fma2(float2 x)
+{
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = __fadd2_rn(x, make_float2(kShifter, kShifter));
+    const float2 n = __fadd2_rn(t, make_float2(-kShifter, -kShifter));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+    float2 p = __ffma2_rn(make_float2(kP3, kP3), f, make_float2(kP2, kP2));
+    p = __ffma2_rn(p, f, make_float2(kP1, kP1));
+    p = __ffma2_rn(p, f, make_float2(kP0, kP0));
+    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 struct PrefillArgs {
     kvattn_bf16* out;  // [B][T][H][d]
     float* lse;        // [B][H][T] or null
@@ -241,22 +270,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             for (int j = 0; j < n_tiles; ++j) {
                 if (!warp_wait(&s_full[t], j & 1, s_abort)) continue;
                 tc_fence_after();
-                uint32_t sv[4][32];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sv[c]);
-                tmem_wait_ld();
                 const bool diag = j == n_tiles - 1;  // keys j*128 .. : the diagonal tile
+                // Pass 1: row max of the raw scores (scale > 0 commutes with the max),
+                // one 32-column chunk in registers at a time.
                 float mx = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    uint32_t sv[32];
+                    tmem_ld32(s_addr + c * 32, sv);
+                    tmem_wait_ld();
+                    if (diag) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        float v = __uint_as_float(sv[c][i]) * sl2;
-                        if (diag && c * 32 + i > row) v = -INFINITY;
-                        sv[c][i] = __float_as_uint(v);
-                        mx = fmaxf(mx, v);
+                        for (int i = 0; i < 32; ++i)
+                            if (c * 32 + i > row) sv[i] = 0xff800000u;  // -inf: key after the query
                     }
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
                 }
+                mx *= sl2;
                 // Move this row's reference max only when it grows by more than 2^8.
                 // The O rescale uses warp-collective TMEM loads/stores, so the
                 // warp takes that path together (alpha = 1 for rows that keep
@@ -279,18 +310,35 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 }
                 m_run = m_new;
                 const float mu = m_run == -INFINITY ? 0.f : m_run;
-                float ls = 0.f;
+                const float2 sc2 = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
+                float2 acc = make_float2(0.f, 0.f);
+                // Pass 2: p = 2^(s * scale * log2 e - m) -> bf16 P over the first 64 S
+                // columns (chunk c's P lands in columns 16c..16c+15, all already read).
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
+                    uint32_t sv[32];
+                    tmem_ld32(s_addr + c * 32, sv);
+                    tmem_wait_ld();
+                    if (diag) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (c * 32 + i > row) sv[i] = 0xff800000u;
+                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float p0 = fast_exp2(__uint_as_float(sv[c][2 * i]) - mu);
-                        const float p1 = fast_exp2(__uint_as_float(sv[c][2 * i + 1]) - mu);
-                        ls += p0 + p1;
-                        pk[i] = pack_bf16x2(p0, p1);
+                        const float2 x =
+                            __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nmu);
+                        float2 pr;
+                        if ((i & 3) == 0) {
+                            pr = exp2_fma2(x);  // a quarter of the exponentials off the MUFU pipe
+                        } else {
+                            pr.x = fast_exp2(x.x);
+                            pr.y = fast_exp2(x.y);
+                        }
+                        acc = __fadd2_rn(acc, pr);
+                        pk[i] = pack_bf16x2(pr.x, pr.y);
                     }
-                    // P columns 16c .. 16c+15 hold keys 32c .. 32c+31, two per column
                     asm volatile(
                         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
                         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(
@@ -300,6 +348,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         "r"(pk[14]), "r"(pk[15])
                         : "memory");
                 }
+                const float ls = acc.x + acc.y;
                 l_run += ls;
                 tmem_wait_st();
                 tc_fence_before();
