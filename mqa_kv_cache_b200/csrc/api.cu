@@ -277,10 +277,14 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
     if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
         return fail(KVATTN_ERR_ALIGN, "attn_decode_gqa: workspace must be 256-byte aligned");
 
-    CUtensorMap tm_k, tm_v;
+    CUtensorMap tm_q, tm_k, tm_v;
     const uint64_t units = static_cast<uint64_t>(B) * n_kv_head;
     if (make_map_3d(&tm_k, k_cache, head_dim, T_max, units, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
     if (make_map_3d(&tm_v, v_cache, head_dim, T_max, units, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    // the tensor-core path reads the queries of one KV group as a [B*Hk][g][d] box
+    memset(&tm_q, 0, sizeof tm_q);
+    if (kvattn::decode_tc_supported(head_dim, g) && make_map_3d(&tm_q, q, head_dim, g, units, 64) != KVATTN_OK)
+        return KVATTN_ERR_CUDA;
 
     uint8_t* w = static_cast<uint8_t*>(workspace);
     kvattn::DecodeArgs a{};
@@ -300,7 +304,7 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
     a.T_max = T_max;
     a.scale = scale;
     a.grid = grid;
-    return cuda_status(kvattn::launch_decode(a, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
+    return cuda_status(kvattn::launch_decode(a, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
                        "attn_decode_gqa launch");
 }
 

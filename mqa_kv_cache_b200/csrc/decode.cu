@@ -23,13 +23,14 @@
 // of g <= 16 heads is one M tile, zero-padded; g = 32/64 use 2/4 M tiles),
 // fp32 accumulation, online softmax in base 2 with quad shuffles.
 #include "common.cuh"
+#include "decode_plan.cuh"
 #include "kernels.h"
 
 namespace kvattn {
 
 namespace {
 
-constexpr int TILE = 64;   // cache rows per pipeline stage
+constexpr int TILE = DEC_TILE;  // cache rows per pipeline stage
 constexpr int CWARPS = 4;  // consumer warps
 constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr float kLn2 = 0.69314718055994530942f;
@@ -51,100 +52,6 @@ struct Cfg {
     static constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
 };
-
-// ---- work plan ------------------------------------------------------------------
-
-__device__ __forceinline__ int owner_of(long long x, long long N, int G)
-{
-    return static_cast<int>((x * G) / N);
-}
-
-__device__ __forceinline__ long long range_start(int c, long long N, int G)
-{
-    return (static_cast<long long>(c) * N + G - 1) / G;
-}
-
-__device__ __forceinline__ int unit_count(long long U, int n, long long N, int G)
-{
-    return n ? owner_of(U + n - 1, N, G) - owner_of(U, N, G) + 1 : 0;
-}
-
-// Block-wide.  s_len[b] = clamped length, s_n[b] = tiles per unit of batch b,
-// s_Ub[b] = tiles of one kv-head slice before batch b (s_Ub[B] = total).
-// Returns N = Hk * s_Ub[B].
-__device__ long long plan_prefix(const int32_t* __restrict__ seq_lens, int B, int Hk, int T_max, int* s_len,
-                                 int* s_n, int* s_Ub, int32_t* dev_status, bool report)
-{
-    for (int b = threadIdx.x; b < B; b += blockDim.x) {
-        const int len = seq_lens[b];
-        const int lc = min(max(len, 0), T_max);
-        if (lc != len && report) report_status(dev_status, KVATTN_STATUS_BAD_LENGTH);
-        s_len[b] = lc;
-        s_n[b] = (lc + TILE - 1) / TILE;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        const int per = (B + 31) / 32;
-        const int beg = min(lane * per, B), end = min(beg + per, B);
-        int sum = 0;
-        for (int b = beg; b < end; ++b) sum += s_n[b];
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - sum;
-        for (int b = beg; b < end; ++b) {
-            s_Ub[b] = run;
-            run += s_n[b];
-        }
-        if (lane == 31) s_Ub[B] = incl;
-    }
-    __syncthreads();
-    return static_cast<long long>(Hk) * s_Ub[B];
-}
-
-// Block-wide: number of partial slots used by units 0 .. u_end-1.
-__device__ int slots_before(int u_end, int Hk, const int* s_n, const int* s_Ub, long long N, int G, int* s_acc)
-{
-    if (threadIdx.x == 0) *s_acc = 0;
-    __syncthreads();
-    int local = 0;
-    for (int u = threadIdx.x; u < u_end; u += blockDim.x) {
-        const int b = u / Hk, kvh = u - b * Hk;
-        const int n = s_n[b];
-        const long long U = static_cast<long long>(Hk) * s_Ub[b] + static_cast<long long>(kvh) * n;
-        local += unit_count(U, n, N, G);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
-    if ((threadIdx.x & 31) == 0 && local) atomicAdd(s_acc, local);
-    __syncthreads();
-    const int r = *s_acc;
-    __syncthreads();
-    return r;
-}
-
-// Position in the unit walk of one CTA.
-struct Walk {
-    int b, kvh;
-    long long U;  // first global tile of the unit
-    int S;        // first partial slot of the unit
-};
-
-__device__ __forceinline__ void walk_next(Walk& w, int B, int Hk, const int* s_n, long long N, int G)
-{
-    const int n = s_n[w.b];
-    w.S += unit_count(w.U, n, N, G);
-    w.U += n;
-    if (++w.kvh == Hk) {
-        w.kvh = 0;
-        ++w.b;
-        while (w.b < B && s_n[w.b] == 0) ++w.b;
-    }
-}
 
 __device__ __forceinline__ uint32_t ld_u32(const kvattn_bf16* p)
 {
@@ -542,12 +449,18 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tm_k, const CUt
     }
     e = launch_pdl(decode_kernel<D, NMT>, dim3(a.grid), dim3(THREADS), Cfg<D>::SMEM, stream, tm_k, tm_v, a);
     if (e != cudaSuccess) return e;
-    const dim3 cgrid(a.B * a.Hk, (a.g + MERGE_WARPS - 1) / MERGE_WARPS);
-    return launch_pdl(decode_combine_kernel<D>, cgrid, dim3(MERGE_WARPS * 32),
-                      static_cast<size_t>(MERGE_WARPS) * a.grid * sizeof(float), stream, a);
+    return launch_decode_merge(a, stream);
 }
 
 }  // namespace
+
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream)
+{
+    const dim3 cgrid(a.B * a.Hk, (a.g + MERGE_WARPS - 1) / MERGE_WARPS);
+    const size_t smem = static_cast<size_t>(MERGE_WARPS) * a.grid * sizeof(float);
+    if (a.d == 128) return launch_pdl(decode_combine_kernel<128>, cgrid, dim3(MERGE_WARPS * 32), smem, stream, a);
+    return launch_pdl(decode_combine_kernel<64>, cgrid, dim3(MERGE_WARPS * 32), smem, stream, a);
+}
 
 long long decode_max_slots(int B, int Hk, int grid)
 {
@@ -556,9 +469,10 @@ long long decode_max_slots(int B, int Hk, int grid)
 
 int decode_grid(int num_sms) { return num_sms; }
 
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                          cudaStream_t stream)
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                          const CUtensorMap& tm_v, cudaStream_t stream)
 {
+    if (decode_tc_supported(a.d, a.g)) return launch_decode_tc(a, tm_q, tm_k, tm_v, stream);
     const int nmt = a.g <= 16 ? 1 : (a.g <= 32 ? 2 : 4);
     if (a.d == 128) {
         if (nmt == 1) return launch_typed<128, 1>(a, tm_k, tm_v, stream);

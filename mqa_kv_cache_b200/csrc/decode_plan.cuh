@@ -1,0 +1,115 @@
+// decode_plan.cuh -- the ragged split-K work plan shared by the decode kernels.
+//
+// The cache rows of every (batch, kv-head) unit are cut into tiles of
+// DEC_TILE rows; the tiles of all units, in unit order, form one list of N
+// tiles; CTA c of the G = min(grid, N) participating CTAs owns the tiles x with
+// floor(x G / N) == c.  Where a CTA's range crosses units it makes one piece per
+// unit; the pieces of a unit get consecutive partial slots.  Everything is
+// computed on the device from the lengths, so the host never waits for them.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace kvattn {
+
+constexpr int DEC_TILE = 64;  // cache rows per tile
+
+namespace {
+
+
+__device__ __forceinline__ int owner_of(long long x, long long N, int G)
+{
+    return static_cast<int>((x * G) / N);
+}
+
+__device__ __forceinline__ long long range_start(int c, long long N, int G)
+{
+    return (static_cast<long long>(c) * N + G - 1) / G;
+}
+
+__device__ __forceinline__ int unit_count(long long U, int n, long long N, int G)
+{
+    return n ? owner_of(U + n - 1, N, G) - owner_of(U, N, G) + 1 : 0;
+}
+
+// Block-wide.  s_len[b] = clamped length, s_n[b] = tiles per unit of batch b,
+// s_Ub[b] = tiles of one kv-head slice before batch b (s_Ub[B] = total).
+// Returns N = Hk * s_Ub[B].
+__device__ long long plan_prefix(const int32_t* __restrict__ seq_lens, int B, int Hk, int T_max, int* s_len,
+                                 int* s_n, int* s_Ub, int32_t* dev_status, bool report)
+{
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+        const int len = seq_lens[b];
+        const int lc = min(max(len, 0), T_max);
+        if (lc != len && report) report_status(dev_status, KVATTN_STATUS_BAD_LENGTH);
+        s_len[b] = lc;
+        s_n[b] = (lc + DEC_TILE - 1) / DEC_TILE;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        const int per = (B + 31) / 32;
+        const int beg = min(lane * per, B), end = min(beg + per, B);
+        int sum = 0;
+        for (int b = beg; b < end; ++b) sum += s_n[b];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int b = beg; b < end; ++b) {
+            s_Ub[b] = run;
+            run += s_n[b];
+        }
+        if (lane == 31) s_Ub[B] = incl;
+    }
+    __syncthreads();
+    return static_cast<long long>(Hk) * s_Ub[B];
+}
+
+// Block-wide: number of partial slots used by units 0 .. u_end-1.
+__device__ int slots_before(int u_end, int Hk, const int* s_n, const int* s_Ub, long long N, int G, int* s_acc)
+{
+    if (threadIdx.x == 0) *s_acc = 0;
+    __syncthreads();
+    int local = 0;
+    for (int u = threadIdx.x; u < u_end; u += blockDim.x) {
+        const int b = u / Hk, kvh = u - b * Hk;
+        const int n = s_n[b];
+        const long long U = static_cast<long long>(Hk) * s_Ub[b] + static_cast<long long>(kvh) * n;
+        local += unit_count(U, n, N, G);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(0xffffffffu, local, o);
+    if ((threadIdx.x & 31) == 0 && local) atomicAdd(s_acc, local);
+    __syncthreads();
+    const int r = *s_acc;
+    __syncthreads();
+    return r;
+}
+
+// Position in the unit walk of one CTA.
+struct Walk {
+    int b, kvh;
+    long long U;  // first global tile of the unit
+    int S;        // first partial slot of the unit
+};
+
+__device__ __forceinline__ void walk_next(Walk& w, int B, int Hk, const int* s_n, long long N, int G)
+{
+    const int n = s_n[w.b];
+    w.S += unit_count(w.U, n, N, G);
+    w.U += n;
+    if (++w.kvh == Hk) {
+        w.kvh = 0;
+        ++w.b;
+        while (w.b < B && s_n[w.b] == 0) ++w.b;
+    }
+}
+
+}  // namespace
+
+}  // namespace kvattn

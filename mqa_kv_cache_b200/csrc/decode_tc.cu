@@ -1,0 +1,472 @@
+// decode_tc.cu -- decode over a KV cache for groups of 64 query heads (MQA at
+// n_head = 64) on the tcgen05 tensor cores.
+//
+// Same method, plan and merge as decode.cu (softmax(scale q k^T) v, query head
+// h reading KV head h / g; "注意力变体与 MoE": each K/V tile read once for the
+// whole group).  With g = 64 (MQA at n_head = 64) every byte of K/V feeds 64
+// heads, 64 FLOP/byte: streaming at HBM speed needs ~0.3 PFLOP/s of bf16 MMA,
+// which is the tcgen05 rate, not the mma.sync one.
+//
+// Per 64-key tile: S = Q K^T with M = 64 heads (rows in TMEM lanes 0-15 of
+// each 32-lane quarter), N = 64 keys, K = 128, double-buffered in TMEM so
+// the next tile's scores are computed while this one's softmax runs; the
+// softmax (one thread per head, lanes 0-15 of four warps) writes P as bf16
+// into a swizzled shared-memory tile and O += P V runs as a second MMA into a
+// 128-column TMEM accumulator.  Warp 0 streams Q (per piece) and the K and V
+// tiles through separate TMA rings (a K slot is released as soon as its S MMA
+// is done, a V slot after its P V); warp 1 issues the S MMAs (and owns TMEM),
+// warp 6 the P V MMAs, so neither waits for the other's operands.
+#include "common.cuh"
+#include "decode_plan.cuh"
+#include "kernels.h"
+
+namespace kvattn {
+
+namespace {
+
+constexpr int TC_T = DEC_TILE;            // keys per tile (64)
+constexpr int TC_D = 128;                 // head dim
+constexpr int TC_M = 64;                  // query heads per MMA
+constexpr int TC_KS = 4;                  // K ring slots
+constexpr int TC_VS = 6;                  // V ring slots
+constexpr int TC_BOX = TC_T * 128;        // 8 KB: 64 rows x one 64-wide d block
+constexpr int TC_TILE = 2 * TC_BOX;       // 16 KB: a K or V tile [64 x 128]
+constexpr int TC_QBOX = TC_M * 128;       // 8 KB
+constexpr int TC_PBYTES = TC_M * 128;     // 8 KB: P tile [64 heads x 64 keys] bf16
+constexpr int TC_THREADS = 224;           // w0 TMA, w1 S MMAs + TMEM, w2-5 softmax, w6 P V MMAs
+constexpr int TC_TMEM_COLS = 256;         // S0 | S1 (64 columns each) | O (128)
+constexpr int TC_OCOL = 2 * TC_T;
+constexpr uint32_t TC_IDESC_S = umma_idesc_bf16(TC_M, TC_T);             // Q x K^T
+constexpr uint32_t TC_IDESC_O = umma_idesc_bf16(TC_M, TC_D, false, true);  // P x V (V MN-major)
+constexpr float kLog2e = 1.44269504088896340736f;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kRescaleThreshold = 8.0f;
+
+constexpr int TC_OFF_K = 0;
+constexpr int TC_OFF_V = TC_OFF_K + TC_KS * TC_TILE;
+constexpr int TC_OFF_Q = TC_OFF_V + TC_VS * TC_TILE;
+constexpr int TC_OFF_P = TC_OFF_Q + 2 * TC_QBOX;                  // two P tiles
+constexpr int TC_OFF_N = TC_OFF_P + 2 * TC_PBYTES;
+constexpr int TC_OFF_UB = TC_OFF_N + DECODE_MAX_B * 4;
+constexpr int TC_OFF_LEN = TC_OFF_UB + (DECODE_MAX_B + 1) * 4;
+constexpr int TC_OFF_BAR = (TC_OFF_LEN + DECODE_MAX_B * 4 + 7) / 8 * 8;
+// kfull[KS], kempty[KS], vfull[VS], vempty[VS], q_full, q_empty, s_full[2], p_full[2], pv_done[2], done[2]
+constexpr int TC_NBAR = 2 * TC_KS + 2 * TC_VS + 10;
+constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
+constexpr int TC_SMEM = TC_OFF_MISC + 32 + 1024;
+
+// The tiles of one CTA in stream order, with the piece they belong to.
+struct TileStream {
+    Walk w;
+    long long t_cur = 0, t_end = 0;
+    int piece = -1;
+    __device__ bool next(long long lo, long long hi, int B, int Hk, const int* s_n, long long N, int G,
+                         bool& first)
+    {
+        if (t_cur >= t_end) {
+            if (piece >= 0) walk_next(w, B, Hk, s_n, N, G);
+            if (!(w.U < hi && w.b < B)) return false;
+            const int n = s_n[w.b];
+            t_cur = (lo > w.U ? lo : w.U) - w.U;
+            t_end = (hi < w.U + n ? hi : w.U + n) - w.U;
+            ++piece;
+            first = true;
+        } else {
+            first = false;
+        }
+        ++t_cur;
+        return true;
+    }
+};
+
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, DecodeArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    int* s_n = reinterpret_cast<int*>(smem + TC_OFF_N);
+    int* s_Ub = reinterpret_cast<int*>(smem + TC_OFF_UB);
+    int* s_len = reinterpret_cast<int*>(smem + TC_OFF_LEN);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TC_OFF_BAR);
+    uint64_t* kfull = bars;
+    uint64_t* kempty = kfull + TC_KS;
+    uint64_t* vfull = kempty + TC_KS;
+    uint64_t* vempty = vfull + TC_VS;
+    uint64_t* q_full = vempty + TC_VS;
+    uint64_t* q_empty = q_full + 1;
+    // Every barrier below is indexed by tile parity (i & 1), so that no waiter is ever
+    // more than one phase behind it (the P and S double buffers bound the lag).
+    uint64_t* s_full = q_full + 2;   // [2]: S of tile i ready in S buffer i & 1
+    uint64_t* p_full = q_full + 4;   // [2]: P of tile i ready in P buffer i & 1 (S buffer i & 1 read)
+    uint64_t* pv_done = q_full + 6;  // [2]: P V of tile i finished (P buffer i & 1 free, O updated)
+    uint64_t* done = q_full + 8;     // [2]: all S MMAs / all P V MMAs finished
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + TC_OFF_MISC + 4);
+    int* s_acc = reinterpret_cast<int*>(smem + TC_OFF_MISC + 8);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < TC_KS; ++s) {
+            mbar_init(&kfull[s], 1);
+            mbar_init(&kempty[s], 1);
+        }
+        for (int s = 0; s < TC_VS; ++s) {
+            mbar_init(&vfull[s], 1);
+            mbar_init(&vempty[s], 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(&s_full[x], 1);
+            mbar_init(&p_full[x], 4);
+            mbar_init(&pv_done[x], 1);
+            mbar_init(&done[x], 1);
+        }
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem, TC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    pdl_wait();
+    pdl_trigger();
+
+    const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
+                                    blockIdx.x == 0);
+    const int G = static_cast<int>(N < a.grid ? N : a.grid), c = blockIdx.x;
+    const bool active = N > 0 && c < G;
+    long long lo = 0, hi = 0;
+    Walk w_start{0, 0, 0, 0};
+    if (active) {
+        lo = range_start(c, N, G);
+        hi = range_start(c + 1, N, G);
+        int lo_b = 0, hi_b = a.B - 1;
+        while (lo_b < hi_b) {
+            const int mid = (lo_b + hi_b + 1) >> 1;
+            if (static_cast<long long>(a.Hk) * s_Ub[mid] <= lo) lo_b = mid;
+            else hi_b = mid - 1;
+        }
+        const int n0 = s_n[lo_b];
+        const int kvh0 = static_cast<int>((lo - static_cast<long long>(a.Hk) * s_Ub[lo_b]) / n0);
+        w_start = Walk{lo_b, kvh0, static_cast<long long>(a.Hk) * s_Ub[lo_b] + static_cast<long long>(kvh0) * n0, 0};
+    }
+    // slots_before synchronises the whole CTA: every thread takes part
+    const int S0 = slots_before(active ? w_start.b * a.Hk + w_start.kvh : 0, a.Hk, s_n, s_Ub, N > 0 ? N : 1,
+                                G > 0 ? G : 1, s_acc);
+    w_start.S = S0;
+
+    if (active && warp == 0) {
+        // ===== TMA producer: Q of each piece, then K and V of each tile =====
+        if (lane == 0) {
+            Walk w = w_start;
+            int it = 0, np = 0;
+            bool ok = true;
+            while (ok && w.U < hi && w.b < a.B) {
+                const int n = s_n[w.b];
+                const long long tb = (lo > w.U ? lo : w.U) - w.U;
+                const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+                const int z = w.b * a.Hk + w.kvh;
+                if (np > 0 && !mbar_wait(q_empty, (np - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(q_full, 2 * TC_QBOX);
+                tma_load_3d(smem + TC_OFF_Q, &tm_q, q_full, 0, 0, z);
+                tma_load_3d(smem + TC_OFF_Q + TC_QBOX, &tm_q, q_full, 64, 0, z);
+                for (long long t = tb; t < te; ++t, ++it) {
+                    const int ks = it % TC_KS, vs = it % TC_VS;
+                    const int row = static_cast<int>(t * TC_T);
+                    if (it >= TC_KS && (*s_abort || !mbar_wait(&kempty[ks], ((it / TC_KS) - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&kfull[ks], TC_TILE);
+                    uint8_t* kd = smem + TC_OFF_K + ks * TC_TILE;
+                    tma_load_3d(kd, &tm_k, &kfull[ks], 0, row, z);
+                    tma_load_3d(kd + TC_BOX, &tm_k, &kfull[ks], 64, row, z);
+                    if (it >= TC_VS && (*s_abort || !mbar_wait(&vempty[vs], ((it / TC_VS) - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&vfull[vs], TC_TILE);
+                    uint8_t* vd = smem + TC_OFF_V + vs * TC_TILE;
+                    tma_load_3d(vd, &tm_v, &vfull[vs], 0, row, z);
+                    tma_load_3d(vd + TC_BOX, &tm_v, &vfull[vs], 64, row, z);
+                }
+                ++np;
+                walk_next(w, a.B, a.Hk, s_n, N, G);
+            }
+            if (!ok) {
+                *s_abort = 1;
+                report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            }
+            // copies still in flight complete before the CTA leaves (bounded waits)
+            for (int j = it - TC_KS > 0 ? it - TC_KS : 0; j < it; ++j) mbar_wait(&kfull[j % TC_KS], (j / TC_KS) & 1);
+            for (int j = it - TC_VS > 0 ? it - TC_VS : 0; j < it; ++j) mbar_wait(&vfull[j % TC_VS], (j / TC_VS) & 1);
+        }
+    } else if (active && warp == 1) {
+        // ===== S = Q K^T issuer =====
+        if (lane == 0) {
+            const uint32_t sq = smem_u32(smem + TC_OFF_Q);
+            TileStream ts{w_start};
+            bool ok = true, first = false;
+            int piece_s = -1;
+            for (int i = 0; ok && ts.next(lo, hi, a.B, a.Hk, s_n, N, G, first); ++i) {
+                if (ts.piece != piece_s) {
+                    if (piece_s >= 0) tc_commit(q_empty);  // every S of the previous piece is issued
+                    if (!(ok = mbar_wait(q_full, ts.piece & 1))) break;
+                    piece_s = ts.piece;
+                }
+                const int ks = i % TC_KS;
+                // S buffer i & 1 was read by the softmax of tile i - 2
+                if (i >= 2 && !(ok = mbar_wait(&p_full[i & 1], ((i >> 1) - 1) & 1))) break;
+                if (!(ok = mbar_wait(&kfull[ks], (i / TC_KS) & 1))) break;
+                tc_fence_after();
+                const uint32_t kt = smem_u32(smem + TC_OFF_K + ks * TC_TILE);
+                const uint32_t d = tmem + (i & 1) * TC_T;
+#pragma unroll
+                for (int kk = 0; kk < TC_D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * TC_BOX + (kk & 3) * 32;
+                    tc_mma_bf16(d, umma_desc_k_sw128(sq + off), umma_desc_k_sw128(kt + off), TC_IDESC_S,
+                                kk > 0 ? 1u : 0u);
+                }
+                tc_commit(&kempty[ks]);
+                tc_commit(&s_full[i & 1]);
+            }
+            if (!ok) {
+                *s_abort = 1;
+                report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            }
+            tc_commit(&done[0]);
+            mbar_wait(&done[0], 0);
+        }
+    } else if (active && warp == 6) {
+        // ===== O += P V issuer =====
+        if (lane == 0) {
+            const uint32_t sp = smem_u32(smem + TC_OFF_P);
+            TileStream ts{w_start};
+            bool ok = true, first = false;
+            for (int i = 0; ok && ts.next(lo, hi, a.B, a.Hk, s_n, N, G, first); ++i) {
+                const int vs = i % TC_VS;
+                if (!(ok = mbar_wait(&p_full[i & 1], (i >> 1) & 1))) break;
+                if (!(ok = mbar_wait(&vfull[vs], (i / TC_VS) & 1))) break;
+                tc_fence_after();
+                const uint32_t vt = smem_u32(smem + TC_OFF_V + vs * TC_TILE);
+                const uint32_t pa = sp + (i & 1) * TC_PBYTES;
+#pragma unroll
+                for (int kk = 0; kk < TC_T / 16; ++kk) {
+                    const uint64_t bd = umma_desc_mn_sw128(vt + kk * 2048, TC_BOX, 1024);
+                    tc_mma_bf16(tmem + TC_OCOL, umma_desc_k_sw128(pa + kk * 32), bd, TC_IDESC_O,
+                                (!first || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&vempty[vs]);
+                tc_commit(&pv_done[i & 1]);
+            }
+            if (!ok) {
+                *s_abort = 1;
+                report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            }
+            tc_commit(&done[1]);
+            mbar_wait(&done[1], 0);
+        }
+    } else if (active && warp >= 2 && warp <= 5) {
+        // ===== softmax + epilogue: one thread per head (lanes 0-15 of warps 2-5) =====
+        const int quarter = warp & 3;
+        const int hrow = quarter * 16 + lane;       // head row of the group (valid for lane < 16)
+        const bool live = lane < 16 && hrow < a.g;  // this lane owns a real head
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t o_addr = tmem + lane_off + TC_OCOL;
+        const float sl2 = a.scale * kLog2e;
+        uint8_t* sP0 = smem + TC_OFF_P;
+        Walk w = w_start;
+        int i = 0;
+        while (w.U < hi && w.b < a.B) {
+            const int n = s_n[w.b];
+            const int len = s_len[w.b];
+            const long long tb = (lo > w.U ? lo : w.U) - w.U;
+            const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+            const int count = unit_count(w.U, n, N, G);
+            const int slot = w.S + (c - owner_of(w.U, N, G));
+            float m_run = -INFINITY, l_run = 0.f;
+            for (long long t = tb; t < te; ++t, ++i) {
+                const bool first = t == tb;
+                if (!warp_wait(&s_full[i & 1], (i >> 1) & 1, s_abort)) continue;
+                // P buffer i & 1 is free once the P V of tile i - 2 has finished
+                if (t - tb >= 2 && !warp_wait(&pv_done[i & 1], ((i >> 1) - 1) & 1, s_abort)) continue;
+                tc_fence_after();
+                const int n_valid = len - static_cast<int>(t) * TC_T;  // >= 1
+                uint32_t sv[2][32];
+                tmem_ld32(tmem + lane_off + (i & 1) * TC_T, sv[0]);
+                tmem_ld32(tmem + lane_off + (i & 1) * TC_T + 32, sv[1]);
+                tmem_wait_ld();
+                if (n_valid < TC_T) {  // tail tile (warp-uniform): keys past the length -> -inf
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (cc * 32 + j >= n_valid) sv[cc][j] = 0xff800000u;
+                }
+                // row max in four independent 3-input chains
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int j = 0; j < 64; j += 8)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        m4[q] = fmax3(m4[q], __uint_as_float(sv[(j + 2 * q) >> 5][(j + 2 * q) & 31]),
+                                      __uint_as_float(sv[(j + 2 * q + 1) >> 5][(j + 2 * q + 1) & 31]));
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+                const bool move = live && (mx > m_run + kRescaleThreshold || m_run == -INFINITY);
+                const float m_new = move ? fmaxf(mx, m_run) : m_run;
+                const bool rescale = move && m_run != -INFINITY && !first;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O must be stable: wait for the P V of the previous tile
+                    if (!warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, s_abort)) continue;
+                    tc_fence_after();
+                    const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.f;
+                    l_run *= alpha;
+#pragma unroll
+                    for (int cc = 0; cc < 4; ++cc) {
+                        uint32_t ov[32];
+                        tmem_ld32(o_addr + cc * 32, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
+                        tmem_st32(o_addr + cc * 32, ov);
+                    }
+                    tmem_wait_st();
+                }
+                m_run = m_new;
+                const float mu = m_run == -INFINITY ? 0.f : m_run;
+                // a tail tile's V rows are zeroed below: its load must have landed first
+                if (n_valid < TC_T && !warp_wait(&vfull[i % TC_VS], (i / TC_VS) & 1, s_abort)) continue;
+                if (lane < 16) {
+                    // P row -> 128-byte swizzled row of P tile i & 1 (zero rows for padding heads)
+                    const float2 sc2 = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
+                    float2 acc = make_float2(0.f, 0.f);
+                    uint8_t* prow = sP0 + (i & 1) * TC_PBYTES;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int k0 = ch * 8 + 2 * e;
+                            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[k0 >> 5][k0 & 31]),
+                                                                    __uint_as_float(sv[k0 >> 5][(k0 + 1) & 31])),
+                                                        sc2, nmu);
+                            float2 pr;
+                            if (e == 0) {
+                                pr = exp2_fma2(x);  // a quarter of the exponentials off the MUFU pipe
+                            } else {
+                                pr.x = fast_exp2(x.x);
+                                pr.y = fast_exp2(x.y);
+                            }
+                            if (!live) pr = make_float2(0.f, 0.f);
+                            acc = __fadd2_rn(acc, pr);
+                            pk[e] = pack_bf16x2(pr.x, pr.y);
+                        }
+                        *reinterpret_cast<uint4*>(prow + swz128(hrow, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                    l_run += acc.x + acc.y;
+                    // rows of a tail tile past the length may hold anything: zero them in V so
+                    // that 0 * garbage cannot reach O (the V slot is not read before p_full)
+                    if (n_valid < TC_T && hrow >= n_valid) {
+                        uint8_t* vrow = smem + TC_OFF_V + (i % TC_VS) * TC_TILE + hrow * 128;
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) {
+                            *reinterpret_cast<uint4*>(vrow + ch * 16) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(vrow + TC_BOX + ch * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                }
+                // make the shared-memory writes visible to the tensor cores
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[i & 1]);
+            }
+            // ---- end of the piece: O (and m, l) out once its last P V has finished ----
+            if (warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, s_abort)) {
+                tc_fence_after();
+                const bool fin = count == 1;
+                const long long bh = static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g + hrow;
+                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    uint32_t ov[16];
+                    tmem_ld16(o_addr + cc * 16, ov);
+                    tmem_wait_ld();
+                    if (live) {
+                        if (fin) {
+                            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * TC_D + cc * 16;
+#pragma unroll
+                            for (int j = 0; j < 16; j += 8)
+                                *reinterpret_cast<uint4*>(orow + j) = make_uint4(
+                                    pack_bf16x2(__uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv),
+                                    pack_bf16x2(__uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv),
+                                    pack_bf16x2(__uint_as_float(ov[j + 4]) * inv, __uint_as_float(ov[j + 5]) * inv),
+                                    pack_bf16x2(__uint_as_float(ov[j + 6]) * inv, __uint_as_float(ov[j + 7]) * inv));
+                        } else {
+                            float* po = a.part_o + (static_cast<long long>(slot) * a.g + hrow) * TC_D + cc * 16;
+#pragma unroll
+                            for (int j = 0; j < 16; j += 4)
+                                *reinterpret_cast<float4*>(po + j) =
+                                    make_float4(__uint_as_float(ov[j]), __uint_as_float(ov[j + 1]),
+                                                __uint_as_float(ov[j + 2]), __uint_as_float(ov[j + 3]));
+                        }
+                    }
+                }
+                if (live) {
+                    if (fin) {
+                        if (a.lse) a.lse[bh] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+                    } else {
+                        const long long pi = static_cast<long long>(slot) * a.g + hrow;
+                        a.part_ml[pi * 2] = m_run == -INFINITY ? 0.f : m_run;
+                        a.part_ml[pi * 2 + 1] = l_run;
+                    }
+                }
+                if (tb == 0 && warp == 2 && lane == 0) a.unit_info[w.b * a.Hk + w.kvh] = make_int2(w.S, count);
+            }
+            walk_next(w, a.B, a.Hk, s_n, N, G);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TC_TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+bool decode_tc_supported(int d, int g) { return d == TC_D && g == TC_M; }
+
+cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, cudaStream_t stream)
+{
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr_set[dev]) {
+        e = cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM);
+        if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
+    }
+    e = launch_pdl(decode_tc_kernel, dim3(a.grid), dim3(TC_THREADS), TC_SMEM, stream, tm_q, tm_k, tm_v, a);
+    if (e != cudaSuccess) return e;
+    return launch_decode_merge(a, stream);
+}
+
+}  // namespace kvattn

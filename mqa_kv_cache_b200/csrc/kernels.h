@@ -74,8 +74,14 @@ struct DecodeArgs {
 long long decode_max_slots(int B, int Hk, int grid);
 // Persistent CTAs per launch for this device.
 int decode_grid(int num_sms);
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
-                          cudaStream_t stream);
+// Runs the tcgen05 kernel for the groups decode_tc_supported() accepts, the
+// mma.sync kernel otherwise, then the merge of split units.
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                          const CUtensorMap& tm_v, cudaStream_t stream);
+bool decode_tc_supported(int d, int g);
+cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                             const CUtensorMap& tm_v, cudaStream_t stream);
+cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
 
 // ---- lightning indexer + top-k ----
 struct DsaIndexArgs {

@@ -45,35 +45,6 @@ constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-// Degree-3 polynomial for 2^f on [-1/2, 1/2], minimax in relative error
-// (max 7.5e-5), produced by fit_exp2_poly.py in this directory.
-constexpr float kP0 = 0.99992806f, kP1 = 0.69326097f, kP2 = 0.24261113f, kP3 = 0.05517167f;
-constexpr float kShifter = 12582912.0f;  // 1.5 * 2^23: x + shifter rounds x to an integer in the low bits
-
-// 2^x for two values on the FMA pipe (Cody-Waite split x = n + f, n = rint(x)):
-// 2^x = 2^n * p(f), with 2^n applied by adding n to the exponent field.  Inputs
-// below -125 are raised to -125 (the result, ~2e-38, is zero for every use here).
-__device__ __forceinline__ float2 exp2_fma2(float2 x)
-{
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 t = __fadd2_rn(x, make_float2(kShifter, kShifter));
-    const float2 n = __fadd2_rn(t, make_float2(-kShifter, -kShifter));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-    float2 p = __ffma2_rn(make_float2(kP3, kP3), f, make_float2(kP2, kP2));
-    p = __ffma2_rn(p, f, make_float2(kP1, kP1));
-    p = __ffma2_rn(p, f, make_float2(kP0, kP0));
-    return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
-__device__ __forceinline__ float fmax3(float a, float b, float c)
-{
-    float r;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-    return r;
-}
-
 struct PrefillArgs {
     kvattn_bf16* out;  // [B][T][H][d]
     float* lse;        // [B][H][T] or null

@@ -1,4 +1,4 @@
-"""The FMA-pipe exponential used for part of the softmax in prefill.cu: the
+"""The FMA-pipe exponential used for part of the softmax (common.cuh): the
 coefficients are read out of the kernel source and the whole algorithm
 (shifter rounding x = n + f, degree-3 polynomial, n added to the exponent
 field) is emulated step by step in fp32 and compared with the exact 2^x.
@@ -9,7 +9,7 @@ import re
 import numpy as np
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "mqa_kv_cache_b200", "csrc",
-                   "prefill.cu")
+                   "common.cuh")
 
 
 def _coeffs():
