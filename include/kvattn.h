@@ -193,11 +193,11 @@ int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn
  * q_idx [B][H_I][d_I] bf16; w [B][H_I] fp32; k_idx [B][L_max][d_I] bf16;
  * seq_lens device int32 [B] or NULL (= L_max for every row).
  * topk_idx [B][k] int32: the k largest scores of row b under the order
- * (score descending, index ascending) -- ties go to the lower index -- listed
- * in that order; min(k, len) entries, then -1.  The selection is made on the
- * fp32 scores the kernel computed; scores_out [B][L_max] fp32 receives them
- * (-inf past each length) when non-NULL.
- * Supported: H_I = 64, d_I = 128, 1 <= k <= 2048, L_max >= 1.
+ * (score descending, index ascending) -- ties go to the lower index --
+ * listed in increasing index order; min(k, len) entries, then -1.  The
+ * selection is made on the fp32 scores the kernel computed; scores_out
+ * [B][L_max] fp32 receives them (-inf past each length) when non-NULL.
+ * Supported: H_I = 64, d_I = 128, 1 <= k <= 2048, 1 <= L_max <= 131072.
  */
 size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k);
 

@@ -352,6 +352,8 @@ int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* 
                     n_idx_head, idx_dim);
     if (B < 1 || L_max < 1 || k < 1 || k > 2048)
         return fail(KVATTN_ERR_SHAPE, "dsa_index_topk: B %d, L_max %d, k %d (k must be 1..2048)", B, L_max, k);
+    if (L_max > 131072)
+        return fail(KVATTN_ERR_UNSUPPORTED, "dsa_index_topk: L_max %d above 131072", L_max);
     if (static_cast<long long>(B) * L_max > (1ll << 31))
         return fail(KVATTN_ERR_SHAPE, "dsa_index_topk: B * L_max too large");
     if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(topk_idx) ||

@@ -11,10 +11,11 @@
 // bound by the one read of k_idx from HBM (intensity ~63 FLOP/byte).
 //
 // Top-k (§2.2 (2): S = TopK_t(s_t), ties to the lower index): one cluster of
-// 8 CTAs per batch row runs an exact 3-digit (11/11/10-bit) radix select on
-// order-preserving 32-bit keys of the fp32 scores, with the histograms summed
-// through distributed shared memory; the selected (key, index) pairs are then
-// sorted by (score desc, index asc) in the cluster's first CTA.
+// 8 CTAs per batch row, each holding its slice of order-preserving 32-bit keys
+// of the fp32 scores in shared memory, runs an exact 3-digit (11/11/10-bit)
+// radix select; every CTA sums the cluster's histograms through distributed
+// shared memory and finds the digit itself.  An ordered compaction then writes
+// the selected indices straight out in increasing index order.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -286,6 +287,8 @@ struct TopkArgs {
     int L_max, k;
 };
 
+constexpr int TK_SLICE_MAX = 16384;  // keys per CTA held in shared memory
+
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
 {
     cg::cluster_group cluster = cg::this_cluster();
@@ -293,11 +296,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     const int row = blockIdx.x / TK_CL;
     const int tid = threadIdx.x;
 
+    extern __shared__ uint32_t s_keys[];  // this CTA's slice as keys (TK_SLICE_MAX at most)
     __shared__ uint32_t hist[2048];
-    __shared__ uint32_t tot[2048];
-    __shared__ unsigned long long sel[2048];
     __shared__ int s_warp[32];
-    __shared__ uint32_t s_state[2];  // prefix, k_rem (written by rank 0 into every CTA)
+    __shared__ uint32_t s_sel[2];    // threshold digit, keys still needed from it
     __shared__ int s_counts[2];      // this CTA's (#key > T, #key == T)
     __shared__ int s_nan;
 
@@ -310,12 +312,17 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     const int kk = min(a.k, len);
     const int slice = (len + TK_CL - 1) / TK_CL;
     const int lo = min(rank * slice, len), hi = min(lo + slice, len);
+    const int n_mine = hi - lo;
     const float* sc = a.scores + static_cast<long long>(row) * a.L_max;
     if (tid == 0) s_nan = 0;
     bool nan = false;
+    // keys of the slice -> shared memory (one read of the scores)
+    for (int i = tid; i < n_mine; i += TK_THREADS) s_keys[i] = score_key(sc[lo + i], nan);
+    __syncthreads();
 
-    uint32_t prefix = 0u, k_rem = static_cast<uint32_t>(kk);
-    uint32_t known = 0u;  // mask of key bits already fixed
+    // ---- radix select: the (k)-th largest key T, and how many keys equal to T to take ----
+    uint32_t prefix = 0u, known = 0u;
+    int k_rem = kk;
     if (len > a.k) {
         const int shifts[3] = {21, 10, 0};
         const int widths[3] = {11, 11, 10};
@@ -323,60 +330,47 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
             const int sh = shifts[p], nb = 1 << widths[p];
             for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
             __syncthreads();
-            for (int i = lo + tid; i < hi; i += TK_THREADS) {
-                const uint32_t key = score_key(sc[i], nan);
+            for (int i = tid; i < n_mine; i += TK_THREADS) {
+                const uint32_t key = s_keys[i];
                 if ((key & known) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
             }
             cluster.sync();
-            // rank r sums bins [r nb/8, (r+1) nb/8) over the cluster into rank 0's `tot`
-            const int per = nb / TK_CL;
-            uint32_t* tot0 = cluster.map_shared_rank(tot, 0);
-            for (int bin = rank * per + tid; bin < (rank + 1) * per; bin += TK_THREADS) {
-                uint32_t v = 0u;
+            // every CTA sums the cluster's histograms and finds the digit itself:
+            // thread t owns digits nb-1-2t and nb-2-2t (largest first)
+            const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
+            int c0 = 0, c1 = 0;
+            if (d0 >= 0) {
 #pragma unroll
-                for (int q = 0; q < TK_CL; ++q) v += cluster.map_shared_rank(hist, q)[bin];
-                tot0[bin] = v;
-            }
-            cluster.sync();
-            if (rank == 0) {
-                // suffix sums over bins (from the largest digit down): each thread owns 2 bins
-                const int b0 = nb - 1 - 2 * tid, b1 = b0 - 1;
-                const int c0 = (2 * tid < nb) ? static_cast<int>(tot[b0]) : 0;
-                const int c1 = (2 * tid + 1 < nb) ? static_cast<int>(tot[b1]) : 0;
-                const int incl = block_incl_scan(c0 + c1, s_warp);
-                const int before = incl - c0 - c1;  // keys in digits above b0
-                const int kr = static_cast<int>(k_rem);
-                if (2 * tid < nb && before < kr && before + c0 >= kr) {
-                    s_state[0] = prefix | (static_cast<uint32_t>(b0) << sh);
-                    s_state[1] = static_cast<uint32_t>(kr - before);
-                } else if (2 * tid + 1 < nb && before + c0 < kr && before + c0 + c1 >= kr) {
-                    s_state[0] = prefix | (static_cast<uint32_t>(b1) << sh);
-                    s_state[1] = static_cast<uint32_t>(kr - before - c0);
-                }
-                __syncthreads();
-                if (tid < TK_CL) {
-                    uint32_t* st = cluster.map_shared_rank(s_state, tid);
-                    st[0] = s_state[0];
-                    st[1] = s_state[1];
+                for (int q = 0; q < TK_CL; ++q) {
+                    const uint32_t* hq = cluster.map_shared_rank(hist, q);
+                    c0 += static_cast<int>(hq[d0]);
+                    if (d1 >= 0) c1 += static_cast<int>(hq[d1]);
                 }
             }
-            cluster.sync();
-            prefix = s_state[0];
-            k_rem = s_state[1];
+            const int incl = block_incl_scan(c0 + c1, s_warp);
+            const int before = incl - c0 - c1;
+            if (d0 >= 0 && before < k_rem && before + c0 >= k_rem) {
+                s_sel[0] = static_cast<uint32_t>(d0);
+                s_sel[1] = static_cast<uint32_t>(k_rem - before);
+            } else if (d1 >= 0 && before + c0 < k_rem && before + c0 + c1 >= k_rem) {
+                s_sel[0] = static_cast<uint32_t>(d1);
+                s_sel[1] = static_cast<uint32_t>(k_rem - before - c0);
+            }
+            cluster.sync();  // every CTA has read every histogram before any is cleared
+            prefix |= s_sel[0] << sh;
+            k_rem = static_cast<int>(s_sel[1]);
             known |= static_cast<uint32_t>(nb - 1) << sh;
         }
-    } else {
-        prefix = 0u;  // every number has a key above 0: all of them are taken
-        known = 0xffffffffu;
     }
-    const uint32_t T = prefix;
+    // With len <= k everything is taken: T = 0 selects every number (NaN keys are 0).
+    const uint32_t T = len > a.k ? prefix : 0u;
 
     // ---- ordered compaction: each thread owns a contiguous run of the slice ----
-    const int run = (hi - lo + TK_THREADS - 1) / TK_THREADS;
-    const int r0 = min(lo + tid * run, hi), r1 = min(r0 + run, hi);
+    const int run = (n_mine + TK_THREADS - 1) / TK_THREADS;
+    const int r0 = min(tid * run, n_mine), r1 = min(r0 + run, n_mine);
     int n_gt = 0, n_eq = 0;
     for (int i = r0; i < r1; ++i) {
-        const uint32_t key = score_key(sc[i], nan);
+        const uint32_t key = s_keys[i];
         n_gt += key > T;
         n_eq += key == T && T != 0u;
     }
@@ -387,62 +381,40 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
         s_counts[1] = inc_eq;
     }
     cluster.sync();
-    int gt_off = 0, eq_off = 0, gt_total = 0, eq_total = 0;
+    int gt_before = 0, eq_before = 0, gt_total = 0, eq_total = 0;
+#pragma unroll
     for (int q = 0; q < TK_CL; ++q) {
-        const int* c = cluster.map_shared_rank(s_counts, q);
+        const int* cq = cluster.map_shared_rank(s_counts, q);
         if (q < rank) {
-            gt_off += c[0];
-            eq_off += c[1];
+            gt_before += cq[0];
+            eq_before += cq[1];
         }
-        gt_total += c[0];
-        eq_total += c[1];
+        gt_total += cq[0];
+        eq_total += cq[1];
     }
-    const int take_eq = kk - gt_total;  // keys equal to T that are still needed
-    unsigned long long* sel0 = cluster.map_shared_rank(sel, 0);
-    int pg = gt_off + inc_gt - n_gt, pe = eq_off + inc_eq - n_eq;
+    const int take_eq = kk - gt_total;  // keys equal to T still needed (lowest indices first)
+    // selected entries before this thread's run, in index order
+    int g_rank = gt_before + inc_gt - n_gt;
+    int e_rank = eq_before + inc_eq - n_eq;
+    int pos = g_rank + min(e_rank, max(take_eq, 0));
+    int32_t* out = a.out + static_cast<long long>(row) * a.k;
     for (int i = r0; i < r1; ++i) {
-        const uint32_t key = score_key(sc[i], nan);
-        const unsigned long long comp =
-            (static_cast<unsigned long long>(0xffffffffu - key) << 32) | static_cast<uint32_t>(i);
-        if (key > T) {
-            sel0[pg++] = comp;
-        } else if (key == T && T != 0u) {
-            if (pe < take_eq) sel0[gt_total + pe] = comp;
-            ++pe;
+        const uint32_t key = s_keys[i];
+        bool take = key > T;
+        if (key == T && T != 0u) {
+            take = e_rank < take_eq;
+            ++e_rank;
         }
+        if (take) out[pos++] = lo + i;
     }
+    // -1 after the selected entries (fewer than kk only when NaN scores were skipped)
+    const int n_sel = gt_total + min(max(take_eq, 0), eq_total);
+    if (rank == 0)
+        for (int j = n_sel + tid; j < a.k; j += TK_THREADS) out[j] = -1;
     if (nan) s_nan = 1;
-    cluster.sync();
-    if (rank == 0) {
-        // sort the k selected entries by (score desc, index asc)
-        // entries actually selected (fewer than kk only when NaN scores were skipped)
-        const int n_sel = gt_total + min(take_eq, eq_total);
-        int n = 1;
-        while (n < kk) n <<= 1;
-        for (int i = n_sel + tid; i < n; i += TK_THREADS) sel[i] = ~0ull;
-        __syncthreads();
-        for (int size = 2; size <= n; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                for (int i = tid; i < (n >> 1); i += TK_THREADS) {
-                    const int x = 2 * stride * (i / stride) + (i % stride);
-                    const int y = x + stride;
-                    const bool asc = (x & size) == 0;
-                    const unsigned long long u = sel[x], v = sel[y];
-                    if ((u > v) == asc) {
-                        sel[x] = v;
-                        sel[y] = u;
-                    }
-                }
-                __syncthreads();
-            }
-        }
-        int32_t* out = a.out + static_cast<long long>(row) * a.k;
-        for (int j = tid; j < a.k; j += TK_THREADS)
-            out[j] = j < kk ? static_cast<int32_t>(sel[j] & 0xffffffffull) : -1;
-    }
     __syncthreads();
     if (s_nan && tid == 0) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
-    cluster.sync();  // no CTA leaves while others may still touch its shared memory
+    cluster.sync();  // no CTA leaves while others may still read its shared memory
 }
 
 }  // namespace
@@ -480,10 +452,18 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     if (e != cudaSuccess) return e;
 
     TopkArgs ta{a.scores, a.seq_lens, a.topk_idx, a.dev_status, a.L_max, a.k};
+    const size_t key_bytes = static_cast<size_t>((a.L_max + TK_CL - 1) / TK_CL) * sizeof(uint32_t);
+    static bool tk_attr[64] = {};
+    if (dev < 64 && !tk_attr[dev]) {
+        e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 TK_SLICE_MAX * static_cast<int>(sizeof(uint32_t)));
+        if (e != cudaSuccess) return e;
+        tk_attr[dev] = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * TK_CL);
     cfg.blockDim = dim3(TK_THREADS);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = key_bytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
