@@ -191,8 +191,7 @@ def run_gpu(args, rank, world, device):
     from mqa_kv_cache_b200 import kvattn as K
     peaks = load_peaks()
     w = W.LLAMA3_8B_DECODE
-    seed = W.SEED_BASE + w.index + rank
-    job = DecodeStep(K, w, device, seed)
+    job = DecodeStep(K, w, device, rank_seed(w, rank))
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     for _ in range(args.warmup):
@@ -216,7 +215,7 @@ def run_gpu(args, rank, world, device):
         step_ms = time_steps(step_graph.replay, args.steps, flush, before=job.reset_q)
     barrier(world)
     torch.cuda.synchronize()
-    ms = max_over_ranks(float(np.mean(step_ms)), world, device)
+    total_bytes, ms = whole_job(job.bytes, float(np.mean(step_ms)), world, device)
 
     # ---- dominant kernel alone (decode + merge launches), same stream ----
     attn_ms = max_over_ranks(float(np.mean(time_steps(attn_graph.replay, args.steps, flush))), world, device)
@@ -245,7 +244,6 @@ def run_gpu(args, rank, world, device):
     h2d = q_host.numel() * 2 + pos_host.numel() * 4 + lens_host.numel() * 4
     d2h = out_host.numel() * 2 + lse_host.numel() * 4
 
-    total_bytes = job.bytes * world
     gbs = total_bytes / (ms * 1e-3) / 1e9
     attn_gbs = job.bytes / (attn_ms * 1e-3) / 1e9
     line = {
@@ -261,8 +259,9 @@ def run_gpu(args, rank, world, device):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q/k/v, ragged lengths U[1024,8192])",
-        "config": {"workload": w.name, "B": w.B, "n_head": w.H, "n_kv_head": w.Hk, "head_dim": w.d,
-                   "T_max": w.T_max, "mean_len": float(job.lens_host.float().mean()), "rope_base": w.rope.base,
+        "config": {"workload": w.name, "B": w.B, "global_batch": w.B * world, "n_head": w.H, "n_kv_head": w.Hk,
+                   "head_dim": w.d, "T_max": w.T_max, "mean_len": float(job.lens_host.float().mean()),
+                   "rope_base": w.rope.base,
                    "parallelism": f"dp{world} (independent batches)",
                    "l2": "flushed between timed steps (read of a 256 MB buffer), and inputs exceed L2"},
         "tok_per_s": round(w.B * world / (ms * 1e-3), 1),
@@ -470,12 +469,31 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def max_over_ranks(x, world, device):
+def _reduce(x, world, device, op):
     if world == 1:
         return x
     t = torch.tensor([x], dtype=torch.float64, device=device)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x, world, device):
+    return _reduce(x, world, device, torch.distributed.ReduceOp.MAX if world > 1 else None)
+
+
+def sum_over_ranks(x, world, device):
+    return _reduce(x, world, device, torch.distributed.ReduceOp.SUM if world > 1 else None)
+
+
+def rank_seed(w, rank):
+    """Every rank draws its own batch (own ragged lengths) of the workload."""
+    return W.SEED_BASE + w.index + rank
+
+
+def whole_job(local_bytes, local_ms, world, device):
+    """(bytes all ranks processed, max-over-ranks step time): the weak-scaling
+    throughput is their ratio."""
+    return sum_over_ranks(float(local_bytes), world, device), max_over_ranks(local_ms, world, device)
 
 
 def main():
@@ -530,10 +548,11 @@ def main():
         from mqa_kv_cache_b200 import kvattn as K
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
         line["other_configs"] = measure_others(K, device, args.steps, flush, load_peaks())
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline()
     if world > 1:
         torch.distributed.destroy_process_group()
+    # the oracle on the host cores: rank 0 of a single-GPU run only
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
