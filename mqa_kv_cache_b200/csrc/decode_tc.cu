@@ -10,8 +10,9 @@
 // Per 64-key tile: S = Q K^T with M = 64 heads (rows in TMEM lanes 0-15 of
 // each 32-lane quarter), N = 64 keys, K = 128, double-buffered in TMEM so
 // the next tile's scores are computed while this one's softmax runs; the
-// softmax (one thread per head, lanes 0-15 of four warps) writes P as bf16
-// into a swizzled shared-memory tile and O += P V runs as a second MMA into a
+// softmax (four warps reading their 16 lanes with the 16x256b shape, so that
+// all 32 threads work: a head's keys spread over a lane quad, two heads per
+// thread) writes P as bf16 into a swizzled shared-memory tile and O += P V runs as a second MMA into a
 // 128-column TMEM accumulator.  Warp 0 streams Q (per piece) and the K and V
 // tiles through separate TMA rings (a K slot is released as soon as its S MMA
 // is done, a V slot after its P V); warp 1 issues the S MMAs (and owns TMEM),
@@ -281,13 +282,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             mbar_wait(&done[1], 0);
         }
     } else if (active && warp >= 2 && warp <= 5) {
-        // ===== softmax + epilogue: one thread per head (lanes 0-15 of warps 2-5) =====
+        // ===== softmax + epilogue: 16 heads per warp, read with the 16-lane TMEM shape =====
+        // Thread t of quarter q holds heads h0 = 16q + t/4 and h1 = h0 + 8 (g = 64: every
+        // row is a head) and, of each 8-key chunk j, keys 8j + cq and 8j + cq + 1 with
+        // cq = 2 (t % 4); a head's 64 scores are spread over one lane quad.
         const int quarter = warp & 3;
-        const int hrow = quarter * 16 + lane;       // head row of the group (valid for lane < 16)
-        const bool live = lane < 16 && hrow < a.g;  // this lane owns a real head
+        const int h0 = quarter * 16 + (lane >> 2), h1 = h0 + 8;
+        const int cq = 2 * (lane & 3);
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t o_addr = tmem + lane_off + TC_OCOL;
         const float sl2 = a.scale * kLog2e;
+        const float2 sc2 = make_float2(sl2, sl2);
         uint8_t* sP0 = smem + TC_OFF_P;
         Walk w = w_start;
         int i = 0;
@@ -298,7 +303,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
             const int count = unit_count(w.U, n, N, G);
             const int slot = w.S + (c - owner_of(w.U, N, G));
-            float m_run = -INFINITY, l_run = 0.f;
+            float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of h0, h1
+            float2 l2 = make_float2(0.f, 0.f);      // this thread's share of their sums
             for (long long t = tb; t < te; ++t, ++i) {
                 const bool first = t == tb;
                 if (!warp_wait(&s_full[i & 1], (i >> 1) & 1, s_abort)) continue;
@@ -306,87 +312,87 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 if (t - tb >= 2 && !warp_wait(&pv_done[i & 1], ((i >> 1) - 1) & 1, s_abort)) continue;
                 tc_fence_after();
                 const int n_valid = len - static_cast<int>(t) * TC_T;  // >= 1
-                uint32_t sv[2][32];
-                tmem_ld32(tmem + lane_off + (i & 1) * TC_T, sv[0]);
-                tmem_ld32(tmem + lane_off + (i & 1) * TC_T + 32, sv[1]);
+                uint32_t sv[32];
+                tmem_ld_16x256b_x8(tmem + lane_off + (i & 1) * TC_T, sv);
                 tmem_wait_ld();
                 if (n_valid < TC_T) {  // tail tile (warp-uniform): keys past the length -> -inf
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (cc * 32 + j >= n_valid) sv[cc][j] = 0xff800000u;
+                    for (int x = 0; x < 32; ++x)
+                        if (8 * (x >> 2) + cq + (x & 1) >= n_valid) sv[x] = 0xff800000u;
                 }
-                // row max in four independent 3-input chains
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                // row maxima: two 3-input chains per head, then across the quad
+                float ma0 = -INFINITY, mb0 = -INFINITY, ma1 = -INFINITY, mb1 = -INFINITY;
 #pragma unroll
-                for (int j = 0; j < 64; j += 8)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        m4[q] = fmax3(m4[q], __uint_as_float(sv[(j + 2 * q) >> 5][(j + 2 * q) & 31]),
-                                      __uint_as_float(sv[(j + 2 * q + 1) >> 5][(j + 2 * q + 1) & 31]));
-                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
-                const bool move = live && (mx > m_run + kRescaleThreshold || m_run == -INFINITY);
-                const float m_new = move ? fmaxf(mx, m_run) : m_run;
-                const bool rescale = move && m_run != -INFINITY && !first;
-                if (__any_sync(0xffffffffu, rescale)) {
+                for (int j = 0; j < 8; j += 2) {
+                    ma0 = fmax3(ma0, __uint_as_float(sv[4 * j]), __uint_as_float(sv[4 * j + 1]));
+                    mb0 = fmax3(mb0, __uint_as_float(sv[4 * j + 4]), __uint_as_float(sv[4 * j + 5]));
+                    ma1 = fmax3(ma1, __uint_as_float(sv[4 * j + 2]), __uint_as_float(sv[4 * j + 3]));
+                    mb1 = fmax3(mb1, __uint_as_float(sv[4 * j + 6]), __uint_as_float(sv[4 * j + 7]));
+                }
+                float mx0 = fmaxf(ma0, mb0), mx1 = fmaxf(ma1, mb1);
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2)) * sl2;
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2)) * sl2;
+                const bool mv0 = mx0 > m0 + kRescaleThreshold || m0 == -INFINITY;
+                const bool mv1 = mx1 > m1 + kRescaleThreshold || m1 == -INFINITY;
+                const float n0 = mv0 ? fmaxf(mx0, m0) : m0, n1 = mv1 ? fmaxf(mx1, m1) : m1;
+                const bool rs0 = mv0 && m0 != -INFINITY && !first, rs1 = mv1 && m1 != -INFINITY && !first;
+                if (__any_sync(0xffffffffu, rs0 || rs1)) {
                     // O must be stable: wait for the P V of the previous tile
                     if (!warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, s_abort)) continue;
                     tc_fence_after();
-                    const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.f;
-                    l_run *= alpha;
+                    const float al0 = rs0 ? fast_exp2(m0 - n0) : 1.f, al1 = rs1 ? fast_exp2(m1 - n1) : 1.f;
+                    l2.x *= al0;
+                    l2.y *= al1;
 #pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int half = 0; half < 2; ++half) {
                         uint32_t ov[32];
-                        tmem_ld32(o_addr + cc * 32, ov);
+                        tmem_ld_16x256b_x8(o_addr + half * 64, ov);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha);
-                        tmem_st32(o_addr + cc * 32, ov);
+                        for (int x = 0; x < 32; ++x)
+                            ov[x] = __float_as_uint(__uint_as_float(ov[x]) * ((x & 2) ? al1 : al0));
+                        tmem_st_16x256b_x8(o_addr + half * 64, ov);
                     }
                     tmem_wait_st();
                 }
-                m_run = m_new;
-                const float mu = m_run == -INFINITY ? 0.f : m_run;
+                m0 = n0;
+                m1 = n1;
+                const float2 nmu0 = make_float2(m0 == -INFINITY ? 0.f : -m0, m0 == -INFINITY ? 0.f : -m0);
+                const float2 nmu1 = make_float2(m1 == -INFINITY ? 0.f : -m1, m1 == -INFINITY ? 0.f : -m1);
                 // a tail tile's V rows are zeroed below: its load must have landed first
                 if (n_valid < TC_T && !warp_wait(&vfull[i % TC_VS], (i / TC_VS) & 1, s_abort)) continue;
-                if (lane < 16) {
-                    // P row -> 128-byte swizzled row of P tile i & 1 (zero rows for padding heads)
-                    const float2 sc2 = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
-                    float2 acc = make_float2(0.f, 0.f);
-                    uint8_t* prow = sP0 + (i & 1) * TC_PBYTES;
+                // P -> 128-byte swizzled rows h0, h1 of P tile i & 1 (4 bytes per chunk and head)
+                uint8_t* pt = sP0 + (i & 1) * TC_PBYTES + cq * 2;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int k0 = ch * 8 + 2 * e;
-                            const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[k0 >> 5][k0 & 31]),
-                                                                    __uint_as_float(sv[k0 >> 5][(k0 + 1) & 31])),
-                                                        sc2, nmu);
-                            float2 pr;
-                            if (e == 0) {
-                                pr = exp2_fma2(x);  // a quarter of the exponentials off the MUFU pipe
-                            } else {
-                                pr.x = fast_exp2(x.x);
-                                pr.y = fast_exp2(x.y);
-                            }
-                            if (!live) pr = make_float2(0.f, 0.f);
-                            acc = __fadd2_rn(acc, pr);
-                            pk[e] = pack_bf16x2(pr.x, pr.y);
-                        }
-                        *reinterpret_cast<uint4*>(prow + swz128(hrow, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                for (int j = 0; j < 8; ++j) {
+                    const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * j]), __uint_as_float(sv[4 * j + 1])),
+                                                 sc2, nmu0);
+                    const float2 x1 = __ffma2_rn(
+                        make_float2(__uint_as_float(sv[4 * j + 2]), __uint_as_float(sv[4 * j + 3])), sc2, nmu1);
+                    const float2 p0 = make_float2(fast_exp2(x0.x), fast_exp2(x0.y));
+                    float2 p1;
+                    if ((j & 1) == 0) {
+                        p1 = exp2_fma2(x1);  // a quarter of the exponentials off the MUFU pipe
+                    } else {
+                        p1.x = fast_exp2(x1.x);
+                        p1.y = fast_exp2(x1.y);
                     }
-                    l_run += acc.x + acc.y;
-                    // rows of a tail tile past the length may hold anything: zero them in V so
-                    // that 0 * garbage cannot reach O (the V slot is not read before p_full)
-                    if (n_valid < TC_T && hrow >= n_valid) {
-                        uint8_t* vrow = smem + TC_OFF_V + (i % TC_VS) * TC_TILE + hrow * 128;
+                    l2.x += p0.x + p0.y;
+                    l2.y += p1.x + p1.y;
+                    *reinterpret_cast<uint32_t*>(pt + swz128(h0, j)) = pack_bf16x2(p0.x, p0.y);
+                    *reinterpret_cast<uint32_t*>(pt + swz128(h1, j)) = pack_bf16x2(p1.x, p1.y);
+                }
+                // rows of a tail tile past the length may hold anything: zero them in V so
+                // that 0 * garbage cannot reach O (the V slot is not read before p_full);
+                // thread (q, t) clears half (t % 2) of key row 16q + t/2
+                if (n_valid < TC_T) {
+                    const int vr = quarter * 16 + (lane >> 1);
+                    if (vr >= n_valid) {
+                        uint8_t* vrow = smem + TC_OFF_V + (i % TC_VS) * TC_TILE + (lane & 1) * TC_BOX + vr * 128;
 #pragma unroll
-                        for (int ch = 0; ch < 8; ++ch) {
-                            *reinterpret_cast<uint4*>(vrow + ch * 16) = make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4*>(vrow + TC_BOX + ch * 16) = make_uint4(0, 0, 0, 0);
-                        }
+                        for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4*>(vrow + ch * 16) = make_uint4(0, 0, 0, 0);
                     }
                 }
                 // make the shared-memory writes visible to the tensor cores
@@ -396,43 +402,49 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 if (lane == 0) mbar_arrive(&p_full[i & 1]);
             }
             // ---- end of the piece: O (and m, l) out once its last P V has finished ----
+            float l0 = l2.x, l1 = l2.y;
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
             if (warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, s_abort)) {
                 tc_fence_after();
                 const bool fin = count == 1;
-                const long long bh = static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g + hrow;
-                const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+                const long long bh0 = static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g + h0;
+                const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    uint32_t ov[16];
-                    tmem_ld16(o_addr + cc * 16, ov);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t ov[32];
+                    tmem_ld_16x256b_x8(o_addr + half * 64, ov);
                     tmem_wait_ld();
-                    if (live) {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int col = half * 64 + 8 * j + cq;
+                        const float o00 = __uint_as_float(ov[4 * j]), o01 = __uint_as_float(ov[4 * j + 1]);
+                        const float o10 = __uint_as_float(ov[4 * j + 2]), o11 = __uint_as_float(ov[4 * j + 3]);
                         if (fin) {
-                            __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * TC_D + cc * 16;
-#pragma unroll
-                            for (int j = 0; j < 16; j += 8)
-                                *reinterpret_cast<uint4*>(orow + j) = make_uint4(
-                                    pack_bf16x2(__uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv),
-                                    pack_bf16x2(__uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv),
-                                    pack_bf16x2(__uint_as_float(ov[j + 4]) * inv, __uint_as_float(ov[j + 5]) * inv),
-                                    pack_bf16x2(__uint_as_float(ov[j + 6]) * inv, __uint_as_float(ov[j + 7]) * inv));
+                            __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + bh0 * TC_D + col;
+                            *reinterpret_cast<uint32_t*>(o) = pack_bf16x2(o00 * inv0, o01 * inv0);
+                            *reinterpret_cast<uint32_t*>(o + 8 * TC_D) = pack_bf16x2(o10 * inv1, o11 * inv1);
                         } else {
-                            float* po = a.part_o + (static_cast<long long>(slot) * a.g + hrow) * TC_D + cc * 16;
-#pragma unroll
-                            for (int j = 0; j < 16; j += 4)
-                                *reinterpret_cast<float4*>(po + j) =
-                                    make_float4(__uint_as_float(ov[j]), __uint_as_float(ov[j + 1]),
-                                                __uint_as_float(ov[j + 2]), __uint_as_float(ov[j + 3]));
+                            float* po = a.part_o + (static_cast<long long>(slot) * a.g + h0) * TC_D + col;
+                            *reinterpret_cast<float2*>(po) = make_float2(o00, o01);
+                            *reinterpret_cast<float2*>(po + 8 * TC_D) = make_float2(o10, o11);
                         }
                     }
                 }
-                if (live) {
+                if ((lane & 3) == 0) {
                     if (fin) {
-                        if (a.lse) a.lse[bh] = l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+                        if (a.lse) {
+                            a.lse[bh0] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
+                            a.lse[bh0 + 8] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
+                        }
                     } else {
-                        const long long pi = static_cast<long long>(slot) * a.g + hrow;
-                        a.part_ml[pi * 2] = m_run == -INFINITY ? 0.f : m_run;
-                        a.part_ml[pi * 2 + 1] = l_run;
+                        const long long pi = static_cast<long long>(slot) * a.g + h0;
+                        a.part_ml[pi * 2] = m0 == -INFINITY ? 0.f : m0;
+                        a.part_ml[pi * 2 + 1] = l0;
+                        a.part_ml[(pi + 8) * 2] = m1 == -INFINITY ? 0.f : m1;
+                        a.part_ml[(pi + 8) * 2 + 1] = l1;
                     }
                 }
                 if (tb == 0 && warp == 2 && lane == 0) a.unit_info[w.b * a.Hk + w.kvh] = make_int2(w.S, count);
