@@ -137,10 +137,19 @@ int rope_apply_qk(kvattn_bf16* q, int q_nb, int q_nt, int q_nh, int64_t q_sb, in
  * A sequence of length 0 gives out = 0 and lse = -inf.  A length outside
  * [0, T_max] is clamped into it and sets KVATTN_STATUS_BAD_LENGTH.
  * workspace: device scratch of attn_decode_gqa_workspace_bytes(...) bytes
- * (256-byte aligned); its contents need no initialisation.
+ * (256-byte aligned).  Its first KVATTN_DECODE_WS_ZERO_BYTES bytes hold one
+ * counter per (batch, KV head) pair -- how many pieces of a split pair have
+ * finished, so that the CTA finishing the last one merges the pair -- and
+ * must be zero before the first call on the workspace (cudaMemsetAsync once);
+ * every call leaves them zero again, except one that sets
+ * KVATTN_STATUS_TIMEOUT, after which they must be cleared before reuse.  The
+ * rest of the workspace needs no initialisation.  Calls that share a
+ * workspace must be ordered (one stream, or events).
  * Supported: head_dim in {64, 128}; n_head % n_kv_head == 0 with
- * g = n_head / n_kv_head in {1, 2, 4, 8, 16, 32, 64}; T_max >= 1.
+ * g = n_head / n_kv_head in {1, 2, 4, 8, 16, 32, 64}; T_max >= 1;
+ * B * n_kv_head <= KVATTN_DECODE_WS_ZERO_BYTES / 4.
  */
+#define KVATTN_DECODE_WS_ZERO_BYTES (64u << 10)
 size_t attn_decode_gqa_workspace_bytes(int B, int n_head, int n_kv_head, int head_dim, int T_max);
 
 int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
@@ -163,9 +172,10 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
  * (attn_decode_gqa_workspace_bytes) exceeds the array is rejected with
  * KVATTN_ERR_WORKSPACE.  The first call on a device looks the array's device
  * address up (cudaGetSymbolAddress); make that first call before any stream
- * capture.  All calls on a device share the one array and it keeps the last
- * call's contents (the kernels write every entry before reading it, so none
- * needs clearing): calls that can overlap on the GPU -- different streams, or
+ * capture.  All calls on a device share the one array: it starts zeroed, as
+ * the counter region at its start requires, and every call leaves that region
+ * zero (after a KVATTN_STATUS_TIMEOUT the results of later calls on the device
+ * are undefined).  Calls that can overlap on the GPU -- different streams, or
  * graphs replayed concurrently -- race and corrupt each other's results.
  */
 #define KVATTN_NOALLOC_SCRATCH_BYTES (8u << 20)

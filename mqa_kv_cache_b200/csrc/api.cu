@@ -121,6 +121,8 @@ int cuda_status(cudaError_t e, const char* what)
 bool g_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16 || g == 32 || g == 64; }
 
 // Decode workspace layout for a given grid.
+// [0, KVATTN_DECODE_WS_ZERO_BYTES): per-unit piece counters (zero between calls, at a
+// fixed place so that calls of any shape agree on it); then the partials.
 struct DecodeWs {
     size_t off_o, off_ml, off_info, total;
 };
@@ -130,8 +132,8 @@ DecodeWs decode_ws(int B, int n_head, int n_kv_head, int head_dim, int grid)
     const long long slots = kvattn::decode_max_slots(B, n_kv_head, grid);
     const int g = n_head / n_kv_head;
     DecodeWs w;
-    w.off_o = 0;
-    w.off_ml = align_up(static_cast<size_t>(slots) * g * head_dim * sizeof(float));
+    w.off_o = KVATTN_DECODE_WS_ZERO_BYTES;
+    w.off_ml = w.off_o + align_up(static_cast<size_t>(slots) * g * head_dim * sizeof(float));
     w.off_info = w.off_ml + align_up(static_cast<size_t>(slots) * g * 2 * sizeof(float));
     w.total = w.off_info + align_up(static_cast<size_t>(B) * n_kv_head * sizeof(int2));
     return w;
@@ -263,8 +265,10 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
     const int g = n_head / n_kv_head;
     if (!g_supported(g)) return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: group size %d", g);
     if (head_dim != 64 && head_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: head_dim %d", head_dim);
-    if (T_max < 1 || static_cast<long long>(B) * n_kv_head > (1ll << 31) - 1)
-        return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: T_max %d / batch too large", T_max);
+    if (T_max < 1) return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: T_max %d", T_max);
+    if (static_cast<long long>(B) * n_kv_head > KVATTN_DECODE_WS_ZERO_BYTES / 4)
+        return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: B * n_kv_head = %lld above %u",
+                    static_cast<long long>(B) * n_kv_head, KVATTN_DECODE_WS_ZERO_BYTES / 4);
     if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: scale must be finite > 0");
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return fail(KVATTN_ERR_ALIGN, "attn_decode_gqa: tensors must be 16-byte aligned");
@@ -295,6 +299,7 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
     a.part_o = reinterpret_cast<float*>(w + ws.off_o);
     a.part_ml = reinterpret_cast<float*>(w + ws.off_ml);
     a.unit_info = reinterpret_cast<int2*>(w + ws.off_info);
+    a.unit_cnt = reinterpret_cast<int*>(w);
     a.dev_status = dev_status;
     a.B = B;
     a.H = n_head;

@@ -22,6 +22,8 @@
 // mma.sync m16n8k16 with the query heads of the group as the M rows (a group
 // of g <= 16 heads is one M tile, zero-padded; g = 32/64 use 2/4 M tiles),
 // fp32 accumulation, online softmax in base 2 with quad shuffles.
+#include <type_traits>
+
 #include "common.cuh"
 #include "decode_plan.cuh"
 #include "kernels.h"
@@ -36,7 +38,7 @@ constexpr int THREADS = 32 * (CWARPS + 1);
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
-template <int D>
+template <int D, int NMT>
 struct Cfg {
     static constexpr int STAGES = D == 128 ? 5 : 8;
     static constexpr int HALVES = D / 64;  // 128-byte column blocks per row
@@ -45,17 +47,69 @@ struct Cfg {
     static constexpr int SCR_STRIDE = D + 8;            // floats per scratch row
     static constexpr int OFF_SCR_O = STAGES * STAGE_BYTES;
     static constexpr int OFF_SCR_ML = OFF_SCR_O + CWARPS * 16 * SCR_STRIDE * 4;
-    static constexpr int OFF_N = OFF_SCR_ML + CWARPS * 16 * 2 * 4;
+    static constexpr int OFF_Q = OFF_SCR_ML + CWARPS * 16 * 2 * 4;  // q rows of the next piece
+    static constexpr int Q_BYTES = NMT * 16 * D * 2;
+    static constexpr int OFF_N = OFF_Q + Q_BYTES;
     static constexpr int OFF_UB = OFF_N + DECODE_MAX_B * 4;
     static constexpr int OFF_LEN = OFF_UB + (DECODE_MAX_B + 1) * 4;
     static constexpr int OFF_BAR = ((OFF_LEN + DECODE_MAX_B * 4) + 7) / 8 * 8;
-    static constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
-    static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
+    static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
+    static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
+    static_assert(SMEM <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ uint32_t ld_u32(const kvattn_bf16* p)
 {
     return *reinterpret_cast<const uint32_t*>(p);
+}
+
+// ---- merge of a split unit ------------------------------------------------------
+// The softmax over a union of key sets is the max-shifted mix of its parts: with
+// M = max_j m_j, L = sum_j 2^(m_j - M) l_j and w_j = 2^(m_j - M) / L,
+// out = sum_j w_j O_j and lse = ln 2 (M + log2 L).  nthr threads of the CTA run it
+// (named barrier 1); s_w holds g x count weights.
+template <int D>
+__device__ void merge_unit(const DecodeArgs& a, int u, int S, int count, float* s_w, int tid, int nthr)
+{
+    const int g = a.g;
+    const int b = u / a.Hk, kvh = u - b * a.Hk;
+    const long long bh0 = static_cast<long long>(b) * a.H + static_cast<long long>(kvh) * g;
+    for (int h = tid; h < g; h += nthr) {
+        const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + static_cast<long long>(S) * g + h;
+        float M = -INFINITY;
+#pragma unroll 4
+        for (int j = 0; j < count; ++j) M = fmaxf(M, __ldcg(ml + static_cast<long long>(j) * g).x);
+        float L = 0.f;
+#pragma unroll 4
+        for (int j = 0; j < count; ++j) {
+            const float2 v = __ldcg(ml + static_cast<long long>(j) * g);
+            const float e = fast_exp2(v.x - M);
+            s_w[h * count + j] = e;
+            L += e * v.y;
+        }
+        const float inv = 1.f / L;
+        for (int j = 0; j < count; ++j) s_w[h * count + j] *= inv;
+        if (a.lse) a.lse[bh0 + h] = (M + __log2f(L)) * kLn2;
+    }
+    named_bar_sync(1, nthr);
+    constexpr int Q4 = D / 4;
+    for (int idx = tid; idx < g * Q4; idx += nthr) {
+        const int h = idx / Q4, q4 = idx - h * Q4;
+        const float4* o = reinterpret_cast<const float4*>(a.part_o + (static_cast<long long>(S) * g + h) * D) + q4;
+        const long long step = static_cast<long long>(g) * Q4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int j = 0; j < count; ++j) {
+            const float4 v = __ldcg(o + j * step);
+            const float wj = s_w[h * count + j];
+            acc.x += wj * v.x;
+            acc.y += wj * v.y;
+            acc.z += wj * v.z;
+            acc.w += wj * v.w;
+        }
+        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (bh0 + h) * D + 4 * q4) =
+            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+    }
 }
 
 // ---- the decode kernel ---------------------------------------------------------
@@ -64,7 +118,7 @@ template <int D, int NMT>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, DecodeArgs a)
 {
-    using C = Cfg<D>;
+    using C = Cfg<D, NMT>;
     constexpr int WPM = CWARPS / NMT;  // warps sharing one M tile (split the tile's rows)
     constexpr int TPW = TILE / WPM;    // cache rows per warp per tile
     constexpr int NT = TPW / 8;        // score n-tiles per warp
@@ -80,8 +134,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     int* s_len = reinterpret_cast<int*>(smem + C::OFF_LEN);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + C::STAGES;
+    uint64_t* q_full = empty + C::STAGES;
+    uint64_t* q_empty = q_full + 1;
+    uint8_t* sQ = smem + C::OFF_Q;
     int* s_misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     volatile int* s_abort = s_misc + 1;
+    int* s_merge = s_misc + 4;  // [0] = count of units to merge here, then (unit, first slot, pieces) x 2
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -89,7 +147,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], CWARPS);
         }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, CWARPS);
         *s_abort = 0;
+        s_merge[0] = 0;
         fence_barrier_init();
     }
     if (warp == CWARPS && lane == 0) {
@@ -101,6 +162,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     pdl_trigger();
     const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
                                     blockIdx.x == 0);
+    // empty sequences have no tiles: their heads get zeros and lse = -inf here
+    for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+        if (s_len[b] != 0) continue;
+        __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(a.out) + static_cast<long long>(b) * a.H * D;
+        for (int i = threadIdx.x; i < a.H * D; i += blockDim.x) ob[i] = __float2bfloat16_rn(0.f);
+        if (a.lse)
+            for (int h = threadIdx.x; h < a.H; h += blockDim.x) a.lse[static_cast<long long>(b) * a.H + h] = -INFINITY;
+    }
     if (N == 0) return;
     // With fewer tiles than CTAs only the first N CTAs take part, so that every
     // participating CTA owns at least one tile and the CTAs owning a unit's
@@ -129,13 +198,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ===== producer: one thread streams K/V tiles of every piece in order =====
         if (lane != 0) return;
         Walk w = w_start;
-        int it = 0;
+        int it = 0, np = 0;
         bool ok = true;
+        const uint32_t q_bytes = static_cast<uint32_t>(a.g) * D * 2;
         while (ok && w.U < hi && w.b < a.B) {
             const int n = s_n[w.b];
             const long long tb = (lo > w.U ? lo : w.U) - w.U;
             const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
             const int z = w.b * a.Hk + w.kvh;
+            // the piece's g query rows (contiguous), once the consumers hold the previous ones
+            if (np > 0 && (*s_abort || !mbar_wait(q_empty, (np - 1) & 1))) {
+                ok = false;
+                break;
+            }
+            mbar_arrive_expect_tx(q_full, q_bytes);
+            bulk_load(sQ, a.q + (static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g) * D, q_bytes,
+                      q_full);
+            ++np;
             for (long long t = tb; t < te; ++t, ++it) {
                 const int s = it % C::STAGES;
                 const uint32_t ph = (it / C::STAGES) & 1;
@@ -163,6 +242,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // copies still in flight complete before the CTA leaves (bounded waits)
         for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
             mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
+        if (np > 0) mbar_wait(q_full, (np - 1) & 1);
         return;
     }
 
@@ -176,7 +256,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int rows_out = g < NMT * 16 ? g : NMT * 16;
 
     Walk w = w_start;
-    int it = 0;
+    int it = 0, piece = 0;
     while (w.U < hi && w.b < a.B) {
         const int n = s_n[w.b];
         const int len = s_len[w.b];
@@ -185,19 +265,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int count = unit_count(w.U, n, N, G);
         const int slot = w.S + (c - owner_of(w.U, N, G));
 
-        // query fragments (A operand): rows = heads of the group, zero beyond g
+        // query fragments (A operand) from the prefetched rows: heads of the group, zero beyond g
         uint32_t qa[KS][4];
         {
-            const kvattn_bf16* qg = a.q + (static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * g) * D;
+            const bool have_q = warp_wait(q_full, piece & 1, s_abort);
+            const uint8_t* qg = sQ;
             const int ra = mt * 16 + r0, rb = ra + 8;
+            const bool va = have_q && ra < g, vb = have_q && rb < g;
 #pragma unroll
             for (int kk = 0; kk < KS; ++kk) {
                 const int col = kk * 16 + 2 * cq;
-                qa[kk][0] = ra < g ? ld_u32(qg + ra * D + col) : 0u;
-                qa[kk][1] = rb < g ? ld_u32(qg + rb * D + col) : 0u;
-                qa[kk][2] = ra < g ? ld_u32(qg + ra * D + col + 8) : 0u;
-                qa[kk][3] = rb < g ? ld_u32(qg + rb * D + col + 8) : 0u;
+                qa[kk][0] = va ? *reinterpret_cast<const uint32_t*>(qg + (ra * D + col) * 2) : 0u;
+                qa[kk][1] = vb ? *reinterpret_cast<const uint32_t*>(qg + (rb * D + col) * 2) : 0u;
+                qa[kk][2] = va ? *reinterpret_cast<const uint32_t*>(qg + (ra * D + col + 8) * 2) : 0u;
+                qa[kk][3] = vb ? *reinterpret_cast<const uint32_t*>(qg + (rb * D + col + 8) * 2) : 0u;
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_empty);
+            ++piece;
         }
         float o[DT][4];
 #pragma unroll
@@ -366,25 +451,50 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
             }
-            // the unit's first piece records its slot range for the merge kernel
-            if (tb == 0 && ctid == 0) a.unit_info[w.b * a.Hk + w.kvh] = make_int2(w.S, count);
         }
         named_bar_sync(1, CWARPS * 32);
+        if (count > 1 && ctid == 0) {
+            // every thread's partial is written (barrier above); publish, then count the piece
+            const int u = w.b * a.Hk + w.kvh;
+            __threadfence();
+            if (atomicAdd(&a.unit_cnt[u], 1) == count - 1) {
+                __threadfence();
+                a.unit_cnt[u] = 0;  // the unit is complete: leave the counter as found
+                const int k = s_merge[0]++;
+                s_merge[1 + 3 * k] = u;
+                s_merge[2 + 3 * k] = w.S;
+                s_merge[3 + 3 * k] = count;
+            }
+        }
         walk_next(w, a.B, a.Hk, s_n, N, G);
+    }
+
+    // ---- the last piece of a split unit merges it (a CTA's range is contiguous, so
+    // at most its first and last units are split: two merges at most) ----
+    if (ctid == 0 && *s_abort) s_merge[0] = 0;  // after a timeout nothing is merged
+    named_bar_sync(1, CWARPS * 32);
+    float* s_w = reinterpret_cast<float*>(smem);  // the K/V stages are idle now
+    for (int k = 0; k < s_merge[0]; ++k) {
+        const int u = s_merge[1 + 3 * k], S = s_merge[2 + 3 * k], cnt = s_merge[3 + 3 * k];
+        merge_unit<D>(a, u, S, cnt, s_w, ctid, CWARPS * 32);
+        named_bar_sync(1, CWARPS * 32);
     }
 }
 
 // ---- merge of split units --------------------------------------------------------
-// One CTA per (unit, block of 8 heads), one warp per head.  With weights
-// w_j = 2^(m_j - M) / sum_i 2^(m_i - M) l_i:  out = sum_j w_j O_j  and
-// lse = ln 2 * (M + log2 sum_j 2^(m_j - M) l_j): the softmax over a union of
-// key sets is the max-shifted mix of the parts.
+// One warp per query head.  With weights w_j = 2^(m_j - M) / sum_i 2^(m_i - M) l_i:
+// out = sum_j w_j O_j and lse = ln 2 * (M + log2 sum_j 2^(m_j - M) l_j): the softmax
+// over a union of key sets is the max-shifted mix of the parts.  Lane j holds
+// (m_j, l_j) of slot j, and every slot's O row is requested together with them, so
+// the merge costs two dependent memory round trips after the slot range is known.
 constexpr int MERGE_WARPS = 8;
+constexpr int MERGE_BATCH = 16;  // slots whose O rows are in flight together
 
 template <int D>
 __global__ void __launch_bounds__(MERGE_WARPS * 32) decode_combine_kernel(DecodeArgs a)
 {
-    extern __shared__ float s_w[];  // [MERGE_WARPS][max pieces]
+    constexpr int PL = D / 32;  // dims per lane
+    using VecF = typename std::conditional<PL == 4, float4, float2>::type;
     pdl_wait();
     pdl_trigger();
     const int u = blockIdx.x;
@@ -393,44 +503,75 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) decode_combine_kernel(Decode
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.y * MERGE_WARPS + warp;
     if (row >= g) return;
+    const int len_raw = a.seq_lens[b];
+    const int2 info = a.unit_info[u];
     const long long bh = static_cast<long long>(b) * a.H + static_cast<long long>(kvh) * g + row;
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * D;
-    const int len = min(max(a.seq_lens[b], 0), a.T_max);
-    if (len == 0) {
-        for (int dim = lane; dim < D; dim += 32) out[dim] = __float2bfloat16_rn(0.f);
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * D + lane * PL;
+    if (min(max(len_raw, 0), a.T_max) == 0) {
+#pragma unroll
+        for (int i = 0; i < PL; ++i) out[i] = __float2bfloat16_rn(0.f);
         if (lane == 0 && a.lse) a.lse[bh] = -INFINITY;
         return;
     }
-    const int2 info = a.unit_info[u];
     if (info.y <= 1) return;  // finished inside one CTA
-    const long long base = static_cast<long long>(info.x) * g + row;
-    float M = -INFINITY;
-    for (int j = lane; j < info.y; j += 32) M = fmaxf(M, a.part_ml[(base + static_cast<long long>(j) * g) * 2]);
+    const int count = info.y;
+    const long long base = static_cast<long long>(info.x) * g + row;  // row of slot 0
+    float M = -INFINITY, L = 0.f;
+    float acc[PL];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float* w = s_w + warp * a.grid;
-    float L = 0.f;
-    for (int j = lane; j < info.y; j += 32) {
-        const long long pj = (base + static_cast<long long>(j) * g) * 2;
-        const float e = fast_exp2(a.part_ml[pj] - M);
-        w[j] = e;
-        L += e * a.part_ml[pj + 1];
+    for (int i = 0; i < PL; ++i) acc[i] = 0.f;
+    for (int j0 = 0; j0 < count; j0 += 32) {
+        // (m, l) of slots j0 + lane, and the O rows of the first MERGE_BATCH of them
+        const int jl = j0 + lane;
+        float2 ml = make_float2(-INFINITY, 0.f);
+        if (jl < count) ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + base + static_cast<long long>(jl) * g);
+        const int nj = min(32, count - j0);
+        VecF ov[MERGE_BATCH];
+#pragma unroll
+        for (int j = 0; j < MERGE_BATCH; ++j)
+            if (j < nj)
+                ov[j] = __ldcg(reinterpret_cast<const VecF*>(a.part_o + (base + static_cast<long long>(j0 + j) * g) * D) +
+                               lane);
+        // rescale what is accumulated so far to the new maximum
+        float Mc = ml.x;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Mc = fmaxf(Mc, __shfl_xor_sync(0xffffffffu, Mc, o));
+        const float Mn = fmaxf(M, Mc);
+        const float r = M == -INFINITY ? 0.f : fast_exp2(M - Mn);
+        L *= r;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) acc[i] *= r;
+        M = Mn;
+        const float wl = jl < count ? fast_exp2(ml.x - M) : 0.f;
+        float Ls = wl * ml.y;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+        L += Ls;
+#pragma unroll
+        for (int j = 0; j < MERGE_BATCH; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, wl, j);
+            if (j < nj) {
+                const float* v = reinterpret_cast<const float*>(&ov[j]);
+#pragma unroll
+                for (int i = 0; i < PL; ++i) acc[i] += wj * v[i];
+            }
+        }
+        for (int j = MERGE_BATCH; j < nj; ++j) {
+            const float wj = __shfl_sync(0xffffffffu, wl, j);
+            const VecF x = __ldcg(reinterpret_cast<const VecF*>(a.part_o + (base + static_cast<long long>(j0 + j) * g) * D) +
+                                  lane);
+            const float* v = reinterpret_cast<const float*>(&x);
+#pragma unroll
+            for (int i = 0; i < PL; ++i) acc[i] += wj * v[i];
+        }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    __syncwarp();
     const float inv = 1.f / L;
-    float acc[D / 32];
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) acc[i] = 0.f;
-    for (int j = 0; j < info.y; ++j) {
-        const float wj = w[j] * inv;
-        const float* o = a.part_o + (base + static_cast<long long>(j) * g) * D;
-#pragma unroll
-        for (int i = 0; i < D / 32; ++i) acc[i] += wj * o[lane + 32 * i];
+    if (PL == 4) {
+        *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
+                                                    pack_bf16x2(acc[PL - 2] * inv, acc[PL - 1] * inv));
+    } else {
+        *reinterpret_cast<uint32_t*>(out) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
     }
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) out[lane + 32 * i] = __float2bfloat16_rn(acc[i]);
     if (lane == 0 && a.lse) a.lse[bh] = (M + __log2f(L)) * kLn2;
 }
 
@@ -443,13 +584,13 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tm_k, const CUt
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(decode_kernel<D, NMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
+        e = cudaFuncSetAttribute(decode_kernel<D, NMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<D, NMT>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    e = launch_pdl(decode_kernel<D, NMT>, dim3(a.grid), dim3(THREADS), Cfg<D>::SMEM, stream, tm_k, tm_v, a);
-    if (e != cudaSuccess) return e;
-    return launch_decode_merge(a, stream);
+    // split units are merged inside the kernel, by the CTA that finishes their last piece
+    return launch_pdl(decode_kernel<D, NMT>, dim3(a.grid), dim3(THREADS), Cfg<D, NMT>::SMEM, stream, tm_k, tm_v, a);
 }
 
 }  // namespace
@@ -457,9 +598,8 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tm_k, const CUt
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream)
 {
     const dim3 cgrid(a.B * a.Hk, (a.g + MERGE_WARPS - 1) / MERGE_WARPS);
-    const size_t smem = static_cast<size_t>(MERGE_WARPS) * a.grid * sizeof(float);
-    if (a.d == 128) return launch_pdl(decode_combine_kernel<128>, cgrid, dim3(MERGE_WARPS * 32), smem, stream, a);
-    return launch_pdl(decode_combine_kernel<64>, cgrid, dim3(MERGE_WARPS * 32), smem, stream, a);
+    if (a.d == 128) return launch_pdl(decode_combine_kernel<128>, cgrid, dim3(MERGE_WARPS * 32), 0, stream, a);
+    return launch_pdl(decode_combine_kernel<64>, cgrid, dim3(MERGE_WARPS * 32), 0, stream, a);
 }
 
 long long decode_max_slots(int B, int Hk, int grid)

@@ -65,6 +65,7 @@ struct DecodeArgs {
     float* part_o;   // [slots][g][d]  unnormalised partial outputs
     float* part_ml;  // [slots][g][2]  (running max in log2 units, sum of exponentials)
     int2* unit_info; // [B*Hk]         (first slot, number of pieces) of every non-empty unit
+    int* unit_cnt;   // [B*Hk]         pieces of a split unit finished so far (zero between calls)
     int32_t* dev_status;
     int B, H, Hk, g, d, T_max;
     float scale;

@@ -161,9 +161,10 @@ def attn_decode_gqa_workspace_bytes(B, n_head, n_kv_head, head_dim, T_max) -> in
 
 
 def workspace(nbytes: int, device=None):
-    """A 256-byte aligned uint8 CUDA buffer of at least `nbytes` bytes."""
+    """A zero-filled, 256-byte aligned uint8 CUDA buffer of at least `nbytes`
+    bytes (the decode workspace wants its counter region zero before first use)."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
 
 
 def attn_decode_gqa(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, ws=None, dev_status=None,

@@ -165,20 +165,47 @@ def test_chain_rope_then_decode(K, wl, T_max):
     assert_attn_close(out, ro, lse, rl, f"chain {wl.name}", lse_tol=chain_lse_tol(qn, kmax_h, wl.scale))
 
 
-def test_workspace_contents_do_not_matter(K):
-    """The workspace needs no initialisation: NaN-filled scratch gives the same result."""
+ZERO_BYTES = 64 << 10  # KVATTN_DECODE_WS_ZERO_BYTES: the per-unit counters at the start of the workspace
+
+
+def test_workspace_partials_need_no_initialisation(K):
+    """Only the counter region must start zero: NaN-filled partials give the
+    same result, and the call leaves the counters zero."""
     B, H, Hk, d, T_max = 3, 4, 2, 64, 300
-    lens = torch.tensor([300, 1, 129], dtype=torch.int32)
+    lens = torch.tensor([300, 1, 129], dtype=torch.int32)  # 18 tiles: units split over up to 5 CTAs
     gen = W.generator(77)
     q = W.normal_bf16((B, H, d), gen).cuda()
     k = W.normal_bf16((B, Hk, T_max, d), gen).cuda()
     v = W.normal_bf16((B, Hk, T_max, d), gen).cuda()
     ws = K.workspace(K.attn_decode_gqa_workspace_bytes(B, H, Hk, d, T_max))
     ws.fill_(0xFF)
+    ws[:ZERO_BYTES].zero_()
     o1, l1 = K.attn_decode_gqa(q, k, v, lens.cuda(), d ** -0.5, ws=ws)
-    ws.fill_(0x00)
+    torch.cuda.synchronize()
+    assert int(ws[:ZERO_BYTES].count_nonzero()) == 0
+    ws.zero_()
     o2, l2 = K.attn_decode_gqa(q, k, v, lens.cuda(), d ** -0.5, ws=ws)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     ro, rl = _oracle(q.cpu(), k.cpu(), v.cpu(), lens, d ** -0.5)
     assert_attn_close(o1, ro, l1, rl, "nan workspace")
+
+
+def test_one_workspace_serves_calls_of_every_shape(K):
+    """Calls of different shapes (both kernels, split and unsplit units) share one
+    workspace: each finds the counters zero and leaves them zero."""
+    shapes = [(2, 8, 2, 128, 5000, 31), (16, 64, 1, 128, 3000, 32), (5, 4, 4, 64, 700, 33),
+              (1, 16, 1, 128, 9000, 34), (7, 32, 8, 128, 2000, 35)]
+    need = max(K.attn_decode_gqa_workspace_bytes(B, H, Hk, d, T) for B, H, Hk, d, T, _ in shapes)
+    ws = K.workspace(need)
+    for B, H, Hk, d, T, seed in shapes:
+        gen = W.generator(seed)
+        q = W.normal_bf16((B, H, d), gen).cuda()
+        k = W.normal_bf16((B, Hk, T, d), gen).cuda()
+        v = W.normal_bf16((B, Hk, T, d), gen).cuda()
+        lens = torch.randint(1, T + 1, (B,), generator=torch.Generator().manual_seed(seed), dtype=torch.int32)
+        out, lse = K.attn_decode_gqa(q, k, v, lens.cuda(), d ** -0.5, ws=ws)
+        torch.cuda.synchronize()
+        assert int(ws[:ZERO_BYTES].count_nonzero()) == 0, (B, H, Hk, d, T)
+        ro, rl = _oracle(q.cpu(), k.cpu(), v.cpu(), lens, d ** -0.5)
+        assert_attn_close(out, ro, lse, rl, f"shared workspace {(B, H, Hk, d, T)}")
