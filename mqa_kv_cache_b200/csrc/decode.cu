@@ -66,49 +66,63 @@ __device__ __forceinline__ uint32_t ld_u32(const kvattn_bf16* p)
 // ---- merge of a split unit ------------------------------------------------------
 // The softmax over a union of key sets is the max-shifted mix of its parts: with
 // M = max_j m_j, L = sum_j 2^(m_j - M) l_j and w_j = 2^(m_j - M) / L,
-// out = sum_j w_j O_j and lse = ln 2 (M + log2 L).  nthr threads of the CTA run it
-// (named barrier 1); s_w holds g x count weights.
+// out = sum_j w_j O_j and lse = ln 2 (M + log2 L).  Thread items are (head,
+// 4 dims); an item requests every slot's (m, l) and O chunk at once, so the merge
+// costs one memory round trip (the weights are recomputed per item).
+constexpr int MERGE_MAX_BATCH = 8;
+
 template <int D>
-__device__ void merge_unit(const DecodeArgs& a, int u, int S, int count, float* s_w, int tid, int nthr)
+__device__ void merge_unit(const DecodeArgs& a, int u, int S, int count, int tid, int nthr)
 {
     const int g = a.g;
     const int b = u / a.Hk, kvh = u - b * a.Hk;
     const long long bh0 = static_cast<long long>(b) * a.H + static_cast<long long>(kvh) * g;
-    for (int h = tid; h < g; h += nthr) {
-        const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + static_cast<long long>(S) * g + h;
-        float M = -INFINITY;
-#pragma unroll 4
-        for (int j = 0; j < count; ++j) M = fmaxf(M, __ldcg(ml + static_cast<long long>(j) * g).x);
-        float L = 0.f;
-#pragma unroll 4
-        for (int j = 0; j < count; ++j) {
-            const float2 v = __ldcg(ml + static_cast<long long>(j) * g);
-            const float e = fast_exp2(v.x - M);
-            s_w[h * count + j] = e;
-            L += e * v.y;
-        }
-        const float inv = 1.f / L;
-        for (int j = 0; j < count; ++j) s_w[h * count + j] *= inv;
-        if (a.lse) a.lse[bh0 + h] = (M + __log2f(L)) * kLn2;
-    }
-    named_bar_sync(1, nthr);
     constexpr int Q4 = D / 4;
+    const long long ml_step = g;                              // float2 per slot
+    const long long o_step = static_cast<long long>(g) * Q4;  // float4 per slot
     for (int idx = tid; idx < g * Q4; idx += nthr) {
         const int h = idx / Q4, q4 = idx - h * Q4;
+        const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + static_cast<long long>(S) * g + h;
         const float4* o = reinterpret_cast<const float4*>(a.part_o + (static_cast<long long>(S) * g + h) * D) + q4;
-        const long long step = static_cast<long long>(g) * Q4;
+        float M = -INFINITY, L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-        for (int j = 0; j < count; ++j) {
-            const float4 v = __ldcg(o + j * step);
-            const float wj = s_w[h * count + j];
-            acc.x += wj * v.x;
-            acc.y += wj * v.y;
-            acc.z += wj * v.z;
-            acc.w += wj * v.w;
+        for (int j0 = 0; j0 < count; j0 += MERGE_MAX_BATCH) {
+            float2 mlv[MERGE_MAX_BATCH];
+            float4 ov[MERGE_MAX_BATCH];
+#pragma unroll
+            for (int j = 0; j < MERGE_MAX_BATCH; ++j) {
+                if (j0 + j < count) {
+                    mlv[j] = __ldcg(ml + (j0 + j) * ml_step);
+                    ov[j] = __ldcg(o + (j0 + j) * o_step);
+                }
+            }
+            float Mb = M;
+#pragma unroll
+            for (int j = 0; j < MERGE_MAX_BATCH; ++j)
+                if (j0 + j < count) Mb = fmaxf(Mb, mlv[j].x);
+            const float r = M == -INFINITY ? 0.f : fast_exp2(M - Mb);
+            L *= r;
+            acc.x *= r;
+            acc.y *= r;
+            acc.z *= r;
+            acc.w *= r;
+            M = Mb;
+#pragma unroll
+            for (int j = 0; j < MERGE_MAX_BATCH; ++j) {
+                if (j0 + j < count) {
+                    const float e = fast_exp2(mlv[j].x - M);
+                    L += e * mlv[j].y;
+                    acc.x += e * ov[j].x;
+                    acc.y += e * ov[j].y;
+                    acc.z += e * ov[j].z;
+                    acc.w += e * ov[j].w;
+                }
+            }
         }
+        const float inv = 1.f / L;
         *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (bh0 + h) * D + 4 * q4) =
-            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+            make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+        if (q4 == 0 && a.lse) a.lse[bh0 + h] = (M + __log2f(L)) * kLn2;
     }
 }
 
@@ -139,7 +153,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* sQ = smem + C::OFF_Q;
     int* s_misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     volatile int* s_abort = s_misc + 1;
-    int* s_merge = s_misc + 4;  // [0] = count of units to merge here, then (unit, first slot, pieces) x 2
+    int* s_merge = s_misc + 4;  // [0] = split pieces made here, then (unit, first slot, pieces) x 2
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -453,32 +467,40 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
         named_bar_sync(1, CWARPS * 32);
-        if (count > 1 && ctid == 0) {
-            // every thread's partial is written (barrier above); publish, then count the piece
-            const int u = w.b * a.Hk + w.kvh;
-            __threadfence();
-            if (atomicAdd(&a.unit_cnt[u], 1) == count - 1) {
-                __threadfence();
-                a.unit_cnt[u] = 0;  // the unit is complete: leave the counter as found
-                const int k = s_merge[0]++;
-                s_merge[1 + 3 * k] = u;
-                s_merge[2 + 3 * k] = w.S;
-                s_merge[3 + 3 * k] = count;
-            }
+        if (count > 1 && ctid == 0 && s_merge[0] < 2) {  // a split piece: counted once the CTA is done
+            const int k = s_merge[0]++;
+            s_merge[1 + 3 * k] = w.b * a.Hk + w.kvh;
+            s_merge[2 + 3 * k] = w.S;
+            s_merge[3 + 3 * k] = count;
         }
         walk_next(w, a.B, a.Hk, s_n, N, G);
     }
 
-    // ---- the last piece of a split unit merges it (a CTA's range is contiguous, so
-    // at most its first and last units are split: two merges at most) ----
-    if (ctid == 0 && *s_abort) s_merge[0] = 0;  // after a timeout nothing is merged
-    named_bar_sync(1, CWARPS * 32);
-    float* s_w = reinterpret_cast<float*>(smem);  // the K/V stages are idle now
-    for (int k = 0; k < s_merge[0]; ++k) {
-        const int u = s_merge[1 + 3 * k], S = s_merge[2 + 3 * k], cnt = s_merge[3 + 3 * k];
-        merge_unit<D>(a, u, S, cnt, s_w, ctid, CWARPS * 32);
-        named_bar_sync(1, CWARPS * 32);
+    // ---- count this CTA's split pieces (its range is contiguous: at most its first and
+    // last units are split); the piece that completes a unit merges it ----
+    if (ctid == 0) {
+        int nm = 0;
+        if (!*s_abort) {  // after a timeout nothing is counted or merged
+            const int np = s_merge[0];
+            __threadfence();  // every partial written here (barrier above) before the counts
+            const int old0 = np > 0 ? atomicAdd(&a.unit_cnt[s_merge[1]], 1) : 0;
+            const int old1 = np > 1 ? atomicAdd(&a.unit_cnt[s_merge[4]], 1) : 0;
+            for (int k = 0; k < np; ++k) {
+                if ((k == 0 ? old0 : old1) == s_merge[3 + 3 * k] - 1) {
+                    a.unit_cnt[s_merge[1 + 3 * k]] = 0;  // complete: leave the counter as found
+                    s_merge[1 + 3 * nm] = s_merge[1 + 3 * k];
+                    s_merge[2 + 3 * nm] = s_merge[2 + 3 * k];
+                    s_merge[3 + 3 * nm] = s_merge[3 + 3 * k];
+                    ++nm;
+                }
+            }
+            if (nm) __threadfence();
+        }
+        s_merge[0] = nm;
     }
+    named_bar_sync(1, CWARPS * 32);
+    for (int k = 0; k < s_merge[0]; ++k)
+        merge_unit<D>(a, s_merge[1 + 3 * k], s_merge[2 + 3 * k], s_merge[3 + 3 * k], ctid, CWARPS * 32);
 }
 
 // ---- merge of split units --------------------------------------------------------
