@@ -34,7 +34,7 @@ METRIC = "decode-attn effective HBM GB/s (% of peak) & tok/s; prefill TFLOP/s"
 # DRAM bytes (read + write) of one decode_kernel launch on the headline workload, from the
 # ncu capture summarised in profiles/decode_kernel_llama3_8b_ragged_B16_H32_Hk8.md; None once
 # the kernel changes after that capture.
-DECODE_TRAFFIC_BYTES = 294_912_000 + 5_736_192
+DECODE_TRAFFIC_BYTES = 295_062_272 + 4_179_712
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -112,8 +112,26 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------- GPU arm
 
+def packed(specs, device):
+    """One uint8 buffer holding tensors of the given (shape, dtype) at 256-byte
+    aligned offsets, and views of them: a step's inputs (or outputs) then cross
+    the PCIe link as one copy."""
+    offs, total = [], 0
+    for shape, dt in specs:
+        offs.append(total)
+        nbytes = int(np.prod(shape)) * torch.tensor([], dtype=dt).element_size()
+        total += (nbytes + 255) // 256 * 256
+    buf = torch.zeros(total, dtype=torch.uint8, device=device)
+    views = []
+    for (shape, dt), o in zip(specs, offs):
+        nbytes = int(np.prod(shape)) * torch.tensor([], dtype=dt).element_size()
+        views.append(buf[o:o + nbytes].view(dt).view(shape))
+    return buf, views
+
+
 class DecodeStep:
-    """Device-resident decode workload; step() = rope on q + decode."""
+    """Device-resident decode workload; step() = rope on q + decode.  The step's
+    inputs (q, positions, lengths) and outputs (out, lse) each live in one buffer."""
 
     def __init__(self, K, w, device, seed):
         self.K, self.w = K, w
@@ -126,15 +144,20 @@ class DecodeStep:
         # cached keys are rotated once, when they are written to the cache
         K.rope_apply_qk(None, None, self.k, inp["k_pos"].to(device), self.cos, self.sin, k_layout="bhtd")
         self.q_raw = inp["q"]
-        self.q = inp["q"].clone()
-        self.lens = inp["seq_lens"].to(device)
+        self.inbuf, (self.q, self.q_pos, self.lens) = packed(
+            [(tuple(inp["q"].shape), torch.bfloat16), (tuple(inp["q_pos"].shape), torch.int32),
+             (tuple(inp["seq_lens"].shape), torch.int32)], device)
+        self.q.copy_(inp["q"])
+        self.q_pos.copy_(inp["q_pos"])
+        self.lens.copy_(inp["seq_lens"])
         self.lens_host = inp["seq_lens"].clone()
-        self.q_pos = inp["q_pos"].to(device)
-        self.out = torch.empty_like(self.q)
-        self.lse = torch.empty((w.B, w.H), dtype=torch.float32, device=device)
+        self.outbuf, (self.out, self.lse) = packed(
+            [(tuple(inp["q"].shape), torch.bfloat16), ((w.B, w.H), torch.float32)], device)
         self.ws = K.workspace(K.attn_decode_gqa_workspace_bytes(w.B, w.H, w.Hk, w.d, w.T_max), device)
         self.bytes = decode_bytes(w, inp["seq_lens"])
-        self.launches_per_step = 3  # rope_apply, decode, merge
+        # rope_apply and the decode kernel; the tcgen05 path (d = 128 with 64 query heads per
+        # KV head) adds its merge kernel, the mma.sync path merges inside the decode kernel
+        self.launches_per_step = 3 if (w.d == 128 and w.g == 64) else 2
 
     def reset_q(self):
         self.q.copy_(self.q_raw)
@@ -223,26 +246,22 @@ def run_gpu(args, rank, world, device):
     eager_ms = max_over_ranks(float(np.mean(time_steps(job.step, args.steps, flush, before=job.reset_q))),
                               world, device)
 
-    # ---- end to end through the public API with host buffers ----
-    q_host = job.q_raw.cpu().pin_memory()
-    pos_host = job.q_pos.cpu().pin_memory()
-    lens_host = job.lens_host.pin_memory()
-    out_host = torch.empty(job.out.shape, dtype=torch.bfloat16).pin_memory()
-    lse_host = torch.empty(job.lse.shape, dtype=torch.float32).pin_memory()
+    # ---- end to end through the public API with host buffers: the step's packed
+    # inputs (raw q, positions, lengths) in, rope + decode, packed (out, lse) back ----
+    job.reset_q()
+    in_host = job.inbuf.cpu().pin_memory()
+    out_host = torch.empty(job.outbuf.shape, dtype=torch.uint8).pin_memory()
 
     def e2e():
-        job.q.copy_(q_host, non_blocking=True)
-        job.q_pos.copy_(pos_host, non_blocking=True)
-        job.lens.copy_(lens_host, non_blocking=True)
+        job.inbuf.copy_(in_host, non_blocking=True)
         job.step()
-        out_host.copy_(job.out, non_blocking=True)
-        lse_host.copy_(job.lse, non_blocking=True)
+        out_host.copy_(job.outbuf, non_blocking=True)
 
     for _ in range(args.warmup):
         e2e()
     e2e_ms = max_over_ranks(float(np.mean(time_steps(e2e, args.steps, flush))), world, device)
-    h2d = q_host.numel() * 2 + pos_host.numel() * 4 + lens_host.numel() * 4
-    d2h = out_host.numel() * 2 + lse_host.numel() * 4
+    h2d = in_host.numel()
+    d2h = out_host.numel()
 
     gbs = total_bytes / (ms * 1e-3) / 1e9
     attn_gbs = job.bytes / (attn_ms * 1e-3) / 1e9

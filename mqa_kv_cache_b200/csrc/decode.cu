@@ -192,21 +192,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (c >= G) return;
     const long long lo = range_start(c, N, G), hi = range_start(c + 1, N, G);
 
-    // unit holding tile `lo`: the last batch entry whose first tile is <= lo
-    int b0 = 0;
-    {
-        int lo_b = 0, hi_b = a.B - 1;
-        while (lo_b < hi_b) {
-            const int mid = (lo_b + hi_b + 1) >> 1;
-            if (static_cast<long long>(a.Hk) * s_Ub[mid] <= lo) lo_b = mid;
-            else hi_b = mid - 1;
-        }
-        b0 = lo_b;
-    }
-    const int n0 = s_n[b0];
-    const int kvh0 = static_cast<int>((lo - static_cast<long long>(a.Hk) * s_Ub[b0]) / n0);
-    const int S0 = slots_before(b0 * a.Hk + kvh0, a.Hk, s_n, s_Ub, N, G, s_misc + 2);
-    const Walk w_start{b0, kvh0, static_cast<long long>(a.Hk) * s_Ub[b0] + static_cast<long long>(kvh0) * n0, S0};
+    // the unit holding tile `lo`, and the partial slots of the units before it
+    Walk w_start = walk_from(lo, a.B, a.Hk, s_n, s_Ub, 0);
+    w_start.S = slots_before(w_start.b * a.Hk + w_start.kvh, a.Hk, s_n, s_Ub, N, G, s_misc + 2);
 
     if (warp == CWARPS) {
         // ===== producer: one thread streams K/V tiles of every piece in order =====
@@ -215,10 +203,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         int it = 0, np = 0;
         bool ok = true;
         const uint32_t q_bytes = static_cast<uint32_t>(a.g) * D * 2;
-        while (ok && w.U < hi && w.b < a.B) {
-            const int n = s_n[w.b];
-            const long long tb = (lo > w.U ? lo : w.U) - w.U;
-            const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+        for (; ok && w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
+            long long tb, te;
+            if (!piece_tiles(w, s_n[w.b], lo, hi, tb, te)) continue;
             const int z = w.b * a.Hk + w.kvh;
             // the piece's g query rows (contiguous), once the consumers hold the previous ones
             if (np > 0 && (*s_abort || !mbar_wait(q_empty, (np - 1) & 1))) {
@@ -247,7 +234,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma_load_3d(vd + h * (TILE * 128), &tm_v, &full[s], h * 64, static_cast<int>(t * TILE), z);
                 }
             }
-            walk_next(w, a.B, a.Hk, s_n, N, G);
         }
         if (!ok) {
             *s_abort = 1;
@@ -271,13 +257,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     Walk w = w_start;
     int it = 0, piece = 0;
-    while (w.U < hi && w.b < a.B) {
+    for (; w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
         const int n = s_n[w.b];
         const int len = s_len[w.b];
-        const long long tb = (lo > w.U ? lo : w.U) - w.U;
-        const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+        long long tb, te;
+        if (!piece_tiles(w, n, lo, hi, tb, te)) continue;
         const int count = unit_count(w.U, n, N, G);
-        const int slot = w.S + (c - owner_of(w.U, N, G));
+        const int slot = w.S + (c - unit_first_owner(w.U, N, G));
 
         // query fragments (A operand) from the prefetched rows: heads of the group, zero beyond g
         uint32_t qa[KS][4];
@@ -473,7 +459,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             s_merge[2 + 3 * k] = w.S;
             s_merge[3 + 3 * k] = count;
         }
-        walk_next(w, a.B, a.Hk, s_n, N, G);
     }
 
     // ---- count this CTA's split pieces (its range is contiguous: at most its first and

@@ -28,6 +28,7 @@ __device__ __forceinline__ long long range_start(int c, long long N, int G)
     return (static_cast<long long>(c) * N + G - 1) / G;
 }
 
+// Pieces of the unit whose first tile is U: the CTAs owning any of its n tiles.
 __device__ __forceinline__ int unit_count(long long U, int n, long long N, int G)
 {
     return n ? owner_of(U + n - 1, N, G) - owner_of(U, N, G) + 1 : 0;
@@ -97,6 +98,34 @@ struct Walk {
     long long U;  // first global tile of the unit
     int S;        // first partial slot of the unit
 };
+
+// Tiles [tb, te) of the unit at w (n tiles) that lie in the range [lo, hi) of
+// global tiles; false when there are none.
+__device__ __forceinline__ bool piece_tiles(const Walk& w, int n, long long lo, long long hi, long long& tb,
+                                            long long& te)
+{
+    tb = (lo > w.U ? lo : w.U) - w.U;
+    te = (hi < w.U + n ? hi : w.U + n) - w.U;
+    return tb < te;
+}
+
+// The CTA owning the unit's first tile (its piece takes the unit's first slot).
+__device__ __forceinline__ int unit_first_owner(long long U, long long N, int G) { return owner_of(U, N, G); }
+
+// The unit holding global tile lo: b = the last batch entry starting at or before lo.
+__device__ __forceinline__ Walk walk_from(long long lo, int B, int Hk, const int* s_n, const int* s_Ub, int S)
+{
+    int lo_b = 0, hi_b = B - 1;
+    while (lo_b < hi_b) {
+        const int mid = (lo_b + hi_b + 1) >> 1;
+        if (static_cast<long long>(Hk) * s_Ub[mid] <= lo) lo_b = mid;
+        else hi_b = mid - 1;
+    }
+    const long long Ub = static_cast<long long>(Hk) * s_Ub[lo_b];
+    const int n = s_n[lo_b];
+    const int kvh = static_cast<int>((lo - Ub) / n);
+    return Walk{lo_b, kvh, Ub + static_cast<long long>(kvh) * n, S};
+}
 
 __device__ __forceinline__ void walk_next(Walk& w, int B, int Hk, const int* s_n, long long N, int G)
 {

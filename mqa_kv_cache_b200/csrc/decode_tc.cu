@@ -65,11 +65,12 @@ struct TileStream {
                          bool& first)
     {
         if (t_cur >= t_end) {
-            if (piece >= 0) walk_next(w, B, Hk, s_n, N, G);
-            if (!(w.U < hi && w.b < B)) return false;
-            const int n = s_n[w.b];
-            t_cur = (lo > w.U ? lo : w.U) - w.U;
-            t_end = (hi < w.U + n ? hi : w.U + n) - w.U;
+            // the next unit holding tiles of the range
+            for (bool moved = piece < 0;; moved = false) {
+                if (!moved) walk_next(w, B, Hk, s_n, N, G);
+                if (!(w.U < hi && w.b < B)) return false;
+                if (piece_tiles(w, s_n[w.b], lo, hi, t_cur, t_end)) break;
+            }
             ++piece;
             first = true;
         } else {
@@ -152,15 +153,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (active) {
         lo = range_start(c, N, G);
         hi = range_start(c + 1, N, G);
-        int lo_b = 0, hi_b = a.B - 1;
-        while (lo_b < hi_b) {
-            const int mid = (lo_b + hi_b + 1) >> 1;
-            if (static_cast<long long>(a.Hk) * s_Ub[mid] <= lo) lo_b = mid;
-            else hi_b = mid - 1;
-        }
-        const int n0 = s_n[lo_b];
-        const int kvh0 = static_cast<int>((lo - static_cast<long long>(a.Hk) * s_Ub[lo_b]) / n0);
-        w_start = Walk{lo_b, kvh0, static_cast<long long>(a.Hk) * s_Ub[lo_b] + static_cast<long long>(kvh0) * n0, 0};
+        w_start = walk_from(lo, a.B, a.Hk, s_n, s_Ub, 0);
     }
     // slots_before synchronises the whole CTA: every thread takes part
     const int S0 = slots_before(active ? w_start.b * a.Hk + w_start.kvh : 0, a.Hk, s_n, s_Ub, N > 0 ? N : 1,
@@ -173,10 +166,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             Walk w = w_start;
             int it = 0, np = 0;
             bool ok = true;
-            while (ok && w.U < hi && w.b < a.B) {
-                const int n = s_n[w.b];
-                const long long tb = (lo > w.U ? lo : w.U) - w.U;
-                const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+            for (; ok && w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
+                long long tb, te;
+                if (!piece_tiles(w, s_n[w.b], lo, hi, tb, te)) continue;
                 const int z = w.b * a.Hk + w.kvh;
                 if (np > 0 && !mbar_wait(q_empty, (np - 1) & 1)) {
                     ok = false;
@@ -206,7 +198,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     tma_load_3d(vd + TC_BOX, &tm_v, &vfull[vs], 64, row, z);
                 }
                 ++np;
-                walk_next(w, a.B, a.Hk, s_n, N, G);
             }
             if (!ok) {
                 *s_abort = 1;
@@ -296,13 +287,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         uint8_t* sP0 = smem + TC_OFF_P;
         Walk w = w_start;
         int i = 0;
-        while (w.U < hi && w.b < a.B) {
+        for (; w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
             const int n = s_n[w.b];
             const int len = s_len[w.b];
-            const long long tb = (lo > w.U ? lo : w.U) - w.U;
-            const long long te = (hi < w.U + n ? hi : w.U + n) - w.U;
+            long long tb, te;
+            if (!piece_tiles(w, n, lo, hi, tb, te)) continue;
             const int count = unit_count(w.U, n, N, G);
-            const int slot = w.S + (c - owner_of(w.U, N, G));
+            const int slot = w.S + (c - unit_first_owner(w.U, N, G));
             float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of h0, h1
             float2 l2 = make_float2(0.f, 0.f);      // this thread's share of their sums
             for (long long t = tb; t < te; ++t, ++i) {
@@ -449,7 +440,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 }
                 if (tb == 0 && warp == 2 && lane == 0) a.unit_info[w.b * a.Hk + w.kvh] = make_int2(w.S, count);
             }
-            walk_next(w, a.B, a.Hk, s_n, N, G);
         }
     }
     tc_fence_before();
