@@ -31,9 +31,9 @@ sys.path.insert(0, ROOT)
 from mqa_kv_cache_b200 import workloads as W  # noqa: E402
 
 METRIC = "decode-attn effective HBM GB/s (% of peak) & tok/s; prefill TFLOP/s"
-# DRAM bytes (read + write) of one decode_kernel launch on the headline workload, from the
-# ncu capture summarised in profiles/decode_kernel_llama3_8b_ragged_B16_H32_Hk8.md; None once
-# the kernel changes after that capture.
+# DRAM bytes (read + write) of one decode_kernel launch on the headline workload, from an ncu
+# capture of the current kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the
+# kernel changes after that capture.
 DECODE_TRAFFIC_BYTES = 295_062_272 + 4_179_712
 L2_FLUSH_BYTES = 256 << 20
 
