@@ -410,9 +410,12 @@ int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const in
         return fail(KVATTN_ERR_WORKSPACE, "attn_decode_sparse: workspace needs %zu bytes", need);
     if (need > 0 && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
         return fail(KVATTN_ERR_ALIGN, "attn_decode_sparse: workspace must be 256-byte aligned");
+    CUtensorMap tm_q;
+    if (make_map_3d(&tm_q, q, Dk, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
     kvattn::SparseLaunch l{q, latent, topk_idx, out, lse, need > 0 ? static_cast<float*>(workspace) : nullptr,
                            dev_status, B, Hq, L_max, k, scale};
-    return cuda_status(kvattn::launch_sparse_attn(l, static_cast<cudaStream_t>(stream)), "attn_decode_sparse launch");
+    return cuda_status(kvattn::launch_sparse_attn(l, tm_q, static_cast<cudaStream_t>(stream)),
+                       "attn_decode_sparse launch");
 }
 
 }  // extern "C"

@@ -111,7 +111,8 @@ struct SparseLaunch {
 };
 int sparse_chunks(int k);
 size_t sparse_partial_bytes(int B, int Hq, int k);
-cudaError_t launch_sparse_attn(const SparseLaunch& l, cudaStream_t stream);
+// tm_q: 3-D map over q [B][Hq][576] with a {64, Hq, 1} box (128-byte swizzle).
+cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, cudaStream_t stream);
 
 // ---- causal prefill ----
 struct PrefillLaunch {

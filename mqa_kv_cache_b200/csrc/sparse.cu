@@ -6,13 +6,22 @@
 // the step is multi-query attention over the selected rows, with the 576-wide
 // row as key and its first 512 columns as value (§2.3.3, §2.3.5).
 //
-// Kernel: one CTA per (batch row, block of 64 heads, chunk of 256 selected
-// rows).  The chunk's rows are gathered 64 at a time with 16-byte cp.async
-// (double-buffered, XOR-swizzled 16-byte chunks so that ldmatrix is
-// conflict-free; invalid indices are zero-filled and masked).  Eight warps:
-// warp w owns 16 heads (w / 2) and half of the 512 value columns (w % 2); the
-// scores S = Q K^T (K = 576) and the online softmax are computed by both warps
-// of a pair, P V by each for its half.  bf16 mma.sync, fp32 accumulation.
+// Kernel (tcgen05): one CTA per (batch row, chunk of 128 selected rows), all
+// query heads as the M = 128 rows of both MMAs.
+//   - warps 0-3 gather the chunk's 128 latent rows (cp.async, 16 bytes at a
+//     time) into nine 64-column blocks laid out as the tensor cores read them
+//     (128-byte rows, 128-byte swizzle); each block is signalled as it lands.
+//     Invalid indices are zero-filled and their columns masked.
+//   - warp 4 streams the queries through a two-slot TMA ring, 64 columns at a
+//     time; warp 5 issues S = Q C^T (M = 128 heads, N = 128 rows, K = 576) into
+//     TMEM, block by block as the gather lands.
+//   - warps 0-3 (thread = head = TMEM lane) take the row softmax of S in base 2
+//     and write P as bf16 into shared memory; warp 5 then issues O = P V with
+//     V = the same resident rows read as an MN-major operand, N = 256 twice,
+//     into all 512 TMEM columns (S's columns are free by then).
+//   - warps 0-3 write O (normalised when the row has one chunk, else the
+//     unnormalised partial with its running max and sum); the first half is
+//     written while the second half's MMAs run.
 // Chunks of one row are merged by a second kernel (the split-softmax identity).
 #include "common.cuh"
 #include "kernels.h"
@@ -23,29 +32,28 @@ namespace {
 
 constexpr int SP_DK = 576;
 constexpr int SP_DV = 512;
-constexpr int SP_ROWS = 64;                     // gathered rows per tile
-constexpr int SP_CHUNK = 256;                   // selected rows per CTA
-constexpr int SP_HB = 64;                       // query heads per CTA
-constexpr int SP_WARPS = 8;
-constexpr int SP_THREADS = SP_WARPS * 32;
-constexpr int SP_RB = SP_DK * 2;                // bytes per row (1152)
-constexpr int SP_CPR = SP_RB / 16;              // 16-byte chunks per row (72)
-constexpr int SP_TILE_BYTES = SP_ROWS * SP_RB;  // 73728
-constexpr int SP_Q_BYTES = SP_HB * SP_RB;       // 73728
-constexpr int SP_OFF_TILE = SP_Q_BYTES;
-constexpr int SP_OFF_IDX = SP_OFF_TILE + 2 * SP_TILE_BYTES;
-constexpr int SP_SMEM = SP_OFF_IDX + 2 * SP_ROWS * 4 + 128;
+constexpr int SP_ROWS = 128;                   // selected rows per CTA (N of S, K of P V)
+constexpr int SP_M = 128;                      // query heads per MMA (rows past Hq are discarded)
+constexpr int SP_KB = SP_DK / 64;              // 64-column blocks of a latent row (9)
+constexpr int SP_BLOCK = SP_ROWS * 128;        // 16 KB: 128 rows x 64 columns
+constexpr int SP_QBLOCK = SP_M * 128;          // 16 KB: 128 heads x 64 columns
+constexpr int SP_THREADS = 192;                // w0-3 gather/softmax/epilogue, w4 TMA, w5 MMA + TMEM
+constexpr int SP_OFF_C = 0;                              // 9 blocks of gathered rows
+constexpr int SP_OFF_Q = SP_OFF_C + SP_KB * SP_BLOCK;    // 2 query slots
+constexpr int SP_OFF_P = SP_OFF_Q + 2 * SP_QBLOCK;       // P: 2 blocks of 64 rows
+constexpr int SP_OFF_VALID = SP_OFF_P + 2 * SP_BLOCK;    // [128] row valid flags
+constexpr int SP_OFF_BAR = SP_OFF_VALID + SP_ROWS * 4;
+// c_full[9], q_full[2], q_empty[2], s_full, p_full, o_full[2], done
+constexpr int SP_NBAR = SP_KB + 2 + 2 + 1 + 1 + 2 + 1;
+constexpr int SP_OFF_MISC = SP_OFF_BAR + SP_NBAR * 8;
+constexpr int SP_SMEM = SP_OFF_MISC + 16 + 1024;  // + alignment slack
+static_assert(SP_SMEM <= 232448, "shared memory");
+constexpr uint32_t SP_IDESC_S = umma_idesc_bf16(SP_M, SP_ROWS);              // Q x C^T, both K-major
+constexpr uint32_t SP_IDESC_O = umma_idesc_bf16(SP_M, 256, false, true);     // P x V, V MN-major
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
-// Byte offset of 16-byte chunk c of row r: chunks XOR-swizzled in groups of 8.
-__device__ __forceinline__ uint32_t sp_off(int r, int c)
-{
-    return static_cast<uint32_t>(r * SP_RB + (((c & ~7) | ((c & 7) ^ (r & 7))) << 4));
-}
-
 struct SparseArgs {
-    const kvattn_bf16* q;       // [B][Hq][576]
     const kvattn_bf16* latent;  // [B][L_max][576]
     const int32_t* idx;         // [B][k]
     kvattn_bf16* out;           // [B][Hq][512]
@@ -57,225 +65,318 @@ struct SparseArgs {
     float scale;
 };
 
-__global__ void __launch_bounds__(SP_THREADS, 1) sparse_attn_kernel(SparseArgs a)
+// cp.async groups still pending after block kb's group may be at most 8 - kb.
+__device__ __forceinline__ void wait_block_groups(int kb)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    const uint32_t sQ = smem_u32(smem);
-    int* s_idx = reinterpret_cast<int*>(smem + SP_OFF_IDX);  // [2][SP_ROWS] validated row numbers (-1 = none)
-
-    const int chunk = blockIdx.x, hblk = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int hg = warp >> 1, vh = warp & 1;
-    const int r0 = lane >> 2, cq = lane & 3;
-    const int row_lo = chunk * SP_CHUNK;
-    const int row_hi = min(row_lo + SP_CHUNK, a.k);
-    const int n_tiles = (row_hi - row_lo + SP_ROWS - 1) / SP_ROWS;
-    const int h_base = hblk * SP_HB;
-    const kvattn_bf16* lat = a.latent + static_cast<long long>(b) * a.L_max * SP_DK;
-    pdl_wait();
-    pdl_trigger();
-
-    // queries of this head block -> shared memory (group 0)
-    const kvattn_bf16* qb = a.q + (static_cast<long long>(b) * a.Hq + h_base) * SP_DK;
-    for (int i = tid; i < SP_HB * SP_CPR; i += SP_THREADS) {
-        const int r = i / SP_CPR, c = i - r * SP_CPR;
-        cp_async16(sQ + sp_off(r, c), qb + r * SP_DK + c * 8, 16);
-    }
-    auto gather = [&](int t, int buf) {
-        const uint32_t dst = smem_u32(smem + SP_OFF_TILE + buf * SP_TILE_BYTES);
-        const int base = row_lo + t * SP_ROWS;
-        if (tid < SP_ROWS) {
-            int j = base + tid < row_hi ? a.idx[static_cast<long long>(b) * a.k + base + tid] : -1;
-            if (j < -1 || j >= a.L_max) {
-                report_status(a.dev_status, KVATTN_STATUS_BAD_INDEX);
-                j = -1;
-            }
-            s_idx[buf * SP_ROWS + tid] = j;
-        }
-        __syncthreads();
-        for (int i = tid; i < SP_ROWS * SP_CPR; i += SP_THREADS) {
-            const int r = i / SP_CPR, c = i - r * SP_CPR;
-            const int j = s_idx[buf * SP_ROWS + r];
-            const kvattn_bf16* src = lat + static_cast<long long>(j < 0 ? 0 : j) * SP_DK + c * 8;
-            cp_async16(dst + sp_off(r, c), src, j < 0 ? 0u : 16u);
-        }
-    };
-    gather(0, 0);
-    cp_async_commit();
-
-    float o[SP_DV / 2 / 8][4];  // 16 heads x 256 value columns
-#pragma unroll
-    for (int i = 0; i < SP_DV / 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    const float sl2 = a.scale * kLog2e;
-    const int mi = lane >> 3, rr = lane & 7;
-
-    for (int t = 0; t < n_tiles; ++t) {
-        const int buf = t & 1;
-        if (t + 1 < n_tiles) gather(t + 1, buf ^ 1);
-        cp_async_commit();
-        cp_async_wait<1>();
-        __syncthreads();
-        const uint32_t sT = smem_u32(smem + SP_OFF_TILE + buf * SP_TILE_BYTES);
-        // ---- S = Q K^T over the tile's 64 rows (K = 576) ----
-        float sc[SP_ROWS / 8][4];
-#pragma unroll
-        for (int i = 0; i < SP_ROWS / 8; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
-#pragma unroll 4
-        for (int kk = 0; kk < SP_DK / 16; ++kk) {
-            uint32_t qa[4];
-            {
-                const int r = hg * 16 + rr + ((mi & 1) << 3);
-                const int c = kk * 2 + (mi >> 1);
-                ldsm_x4(sQ + sp_off(r, c), qa[0], qa[1], qa[2], qa[3]);
-            }
-#pragma unroll
-            for (int np = 0; np < SP_ROWS / 16; ++np) {
-                const int r = np * 16 + rr + ((mi >> 1) << 3);
-                const int c = kk * 2 + (mi & 1);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(sT + sp_off(r, c), b0, b1, b2, b3);
-                mma_bf16_16816(sc[2 * np], qa, b0, b1);
-                mma_bf16_16816(sc[2 * np + 1], qa, b2, b3);
-            }
-        }
-        // ---- online softmax over the 64 rows ----
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < SP_ROWS / 8; ++i) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int r = i * 8 + 2 * cq + (e & 1);
-                float v = sc[i][e] * sl2;
-                if (s_idx[buf * SP_ROWS + r] < 0) v = -INFINITY;
-                sc[i][e] = v;
-            }
-            mx0 = fmaxf(mx0, fmaxf(sc[i][0], sc[i][1]));
-            mx1 = fmaxf(mx1, fmaxf(sc[i][2], sc[i][3]));
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float mu0 = mn0 == -INFINITY ? 0.f : mn0, mu1 = mn1 == -INFINITY ? 0.f : mn1;
-        const float al0 = fast_exp2(m0 - mu0), al1 = fast_exp2(m1 - mu1);
-        m0 = mn0;
-        m1 = mn1;
-        float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < SP_ROWS / 8; ++i) {
-            sc[i][0] = fast_exp2(sc[i][0] - mu0);
-            sc[i][1] = fast_exp2(sc[i][1] - mu0);
-            sc[i][2] = fast_exp2(sc[i][2] - mu1);
-            sc[i][3] = fast_exp2(sc[i][3] - mu1);
-            ps0 += sc[i][0] + sc[i][1];
-            ps1 += sc[i][2] + sc[i][3];
-        }
-        l0 = l0 * al0 + ps0;
-        l1 = l1 * al1 + ps1;
-#pragma unroll
-        for (int i = 0; i < SP_DV / 16; ++i) {
-            o[i][0] *= al0;
-            o[i][1] *= al0;
-            o[i][2] *= al1;
-            o[i][3] *= al1;
-        }
-        // ---- O += P V for this warp's 256 value columns ----
-#pragma unroll
-        for (int j = 0; j < SP_ROWS / 16; ++j) {
-            uint32_t pa[4];
-            pa[0] = pack_bf16x2(sc[2 * j][0], sc[2 * j][1]);
-            pa[1] = pack_bf16x2(sc[2 * j][2], sc[2 * j][3]);
-            pa[2] = pack_bf16x2(sc[2 * j + 1][0], sc[2 * j + 1][1]);
-            pa[3] = pack_bf16x2(sc[2 * j + 1][2], sc[2 * j + 1][3]);
-            const int r = j * 16 + rr + ((mi & 1) << 3);
-#pragma unroll
-            for (int dp = 0; dp < SP_DV / 2 / 16; ++dp) {
-                const int c = (vh * (SP_DV / 2) + dp * 16) / 8 + (mi >> 1);
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_t(sT + sp_off(r, c), v0, v1, v2, v3);
-                mma_bf16_16816(o[2 * dp], pa, v0, v1);
-                mma_bf16_16816(o[2 * dp + 1], pa, v2, v3);
-            }
-        }
-        __syncthreads();  // the buffer is refilled by the next iteration's gather
-    }
-    cp_async_wait<0>();
-
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    const int ha = h_base + hg * 16 + r0, hb = ha + 8;
-    if (a.chunks == 1) {
-        const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + static_cast<long long>(b) * a.Hq * SP_DV;
-#pragma unroll
-        for (int i = 0; i < SP_DV / 16; ++i) {
-            const int col = vh * (SP_DV / 2) + i * 8 + 2 * cq;
-            *reinterpret_cast<uint32_t*>(out + static_cast<long long>(ha) * SP_DV + col) =
-                pack_bf16x2(o[i][0] * i0, o[i][1] * i0);
-            *reinterpret_cast<uint32_t*>(out + static_cast<long long>(hb) * SP_DV + col) =
-                pack_bf16x2(o[i][2] * i1, o[i][3] * i1);
-        }
-        if (a.lse && vh == 0 && cq == 0) {
-            const long long bh = static_cast<long long>(b) * a.Hq;
-            a.lse[bh + ha] = l0 > 0.f ? (m0 + __log2f(l0)) * kLn2 : -INFINITY;
-            a.lse[bh + hb] = l1 > 0.f ? (m1 + __log2f(l1)) * kLn2 : -INFINITY;
-        }
-    } else {
-        const long long pbase = (static_cast<long long>(b) * a.chunks + chunk) * a.Hq;
-        float* po = a.part_o + pbase * SP_DV;
-#pragma unroll
-        for (int i = 0; i < SP_DV / 16; ++i) {
-            const int col = vh * (SP_DV / 2) + i * 8 + 2 * cq;
-            *reinterpret_cast<float2*>(po + static_cast<long long>(ha) * SP_DV + col) = make_float2(o[i][0], o[i][1]);
-            *reinterpret_cast<float2*>(po + static_cast<long long>(hb) * SP_DV + col) = make_float2(o[i][2], o[i][3]);
-        }
-        if (vh == 0 && cq == 0) {
-            a.part_ml[(pbase + ha) * 2] = m0;
-            a.part_ml[(pbase + ha) * 2 + 1] = l0;
-            a.part_ml[(pbase + hb) * 2] = m1;
-            a.part_ml[(pbase + hb) * 2 + 1] = l1;
-        }
+    switch (kb) {
+    case 0: cp_async_wait<8>(); break;
+    case 1: cp_async_wait<7>(); break;
+    case 2: cp_async_wait<6>(); break;
+    case 3: cp_async_wait<5>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 5: cp_async_wait<3>(); break;
+    case 6: cp_async_wait<2>(); break;
+    case 7: cp_async_wait<1>(); break;
+    default: cp_async_wait<0>(); break;
     }
 }
 
-// One warp per (batch row, head): merge the chunk partials.
-__global__ void __launch_bounds__(256) sparse_merge_kernel(SparseArgs a)
+__global__ void __launch_bounds__(SP_THREADS, 1)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, SparseArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    int* s_valid = reinterpret_cast<int*>(smem + SP_OFF_VALID);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SP_OFF_BAR);
+    uint64_t* c_full = bars;                 // [9]: block kb of the rows landed (128 arrivals)
+    uint64_t* q_full = c_full + SP_KB;       // [2]
+    uint64_t* q_empty = q_full + 2;          // [2]
+    uint64_t* s_full = q_empty + 2;          // S complete in TMEM
+    uint64_t* p_full = s_full + 1;           // P written (S read), 128 arrivals
+    uint64_t* o_full = p_full + 1;           // [2]: O columns 0-255 / 256-511 complete
+    uint64_t* done = o_full + 2;             // every MMA finished
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SP_OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SP_OFF_MISC + 4);
+
+    const int chunk = blockIdx.x, b = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int i = 0; i < SP_KB; ++i) mbar_init(&c_full[i], 128);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1);
+            mbar_init(&q_empty[i], 1);
+            mbar_init(&o_full[i], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(done, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 4 && lane == 0) tma_prefetch_desc(&tm_q);
+    if (warp == 5) {
+        tmem_alloc(s_tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp < 4) {
+        // ===== gather: thread t brings selected row t of the chunk =====
+        const int t = tid;
+        const int slot = chunk * SP_ROWS + t;
+        int j = slot < a.k ? a.idx[static_cast<long long>(b) * a.k + slot] : -1;
+        if (j < -1 || j >= a.L_max) {
+            report_status(a.dev_status, KVATTN_STATUS_BAD_INDEX);
+            j = -1;
+        }
+        s_valid[t] = j >= 0;
+        const kvattn_bf16* src = a.latent + (static_cast<long long>(b) * a.L_max + (j < 0 ? 0 : j)) * SP_DK;
+        const uint32_t bytes = j < 0 ? 0u : 16u;  // 0: zero-fill
+        const uint32_t c0 = smem_u32(smem + SP_OFF_C);
+#pragma unroll
+        for (int kb = 0; kb < SP_KB; ++kb) {
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) cp_async16(c0 + kb * SP_BLOCK + swz128(t, ch), src + kb * 64 + ch * 8, bytes);
+            cp_async_commit();
+        }
+#pragma unroll
+        for (int kb = 0; kb < SP_KB; ++kb) {
+            wait_block_groups(kb);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(&c_full[kb]);
+        }
+        named_bar_sync(1, 128);  // every row's valid flag is written
+
+        // ===== softmax of head row t (TMEM lane t) =====
+        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        const bool live = t < a.Hq;
+        const float sl2 = a.scale * kLog2e;
+        float m = -INFINITY, l = 0.f;
+        if (warp_wait(s_full, 0, s_abort)) {
+            tc_fence_after();
+            uint32_t sv[4][32];
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_off + cc * 32, sv[cc]);
+            tmem_wait_ld();
+            float mx = -INFINITY;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    if (!s_valid[cc * 32 + i]) sv[cc][i] = 0xff800000u;  // -inf: not a selected row
+                    mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
+                }
+            }
+            m = mx * sl2;
+            const float mu = m == -INFINITY ? 0.f : m;
+            const float2 sc2 = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
+            float2 acc = make_float2(0.f, 0.f);
+            uint8_t* prow = smem + SP_OFF_P;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {  // 8-row chunk (16 bytes of P) q of this 32-row group
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = q * 8 + 2 * e;
+                        const float2 x = __ffma2_rn(
+                            make_float2(__uint_as_float(sv[cc][i]), __uint_as_float(sv[cc][i + 1])), sc2, nmu);
+                        float2 p;
+                        if (e == 0) {
+                            p = exp2_fma2(x);  // a quarter of the exponentials off the MUFU pipe
+                        } else {
+                            p.x = fast_exp2(x.x);
+                            p.y = fast_exp2(x.y);
+                        }
+                        if (!live) p = make_float2(0.f, 0.f);
+                        acc = __fadd2_rn(acc, p);
+                        pk[e] = pack_bf16x2(p.x, p.y);
+                    }
+                    const int col = cc * 32 + q * 8;  // first selected row of the 16-byte chunk
+                    *reinterpret_cast<uint4*>(prow + (col >> 6) * SP_BLOCK + swz128(t, (col & 63) >> 3)) =
+                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            l = acc.x + acc.y;
+        }
+        // S is read and P is written: the P V MMAs may reuse S's columns
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(p_full);
+
+        // ===== epilogue: O row t, half by half =====
+        const bool one = a.chunks == 1;
+        const long long bh = static_cast<long long>(b) * a.Hq + t;
+        const long long pr = (static_cast<long long>(b) * a.chunks + chunk) * a.Hq + t;  // partial row
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            if (!warp_wait(&o_full[half], 0, s_abort)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+                uint32_t ov[32];
+                tmem_ld32(tmem + lane_off + half * 256 + cc * 32, ov);
+                tmem_wait_ld();
+                if (!live) continue;
+                const int col = half * 256 + cc * 32;
+                if (one) {
+                    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * SP_DV + col;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8)
+                        *reinterpret_cast<uint4*>(o + i) = make_uint4(
+                            pack_bf16x2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv));
+                } else {
+                    float* po = a.part_o + pr * SP_DV + col;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(po + i) =
+                            make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]),
+                                        __uint_as_float(ov[i + 2]), __uint_as_float(ov[i + 3]));
+                }
+            }
+        }
+        if (live) {
+            if (one) {
+                if (a.lse) a.lse[bh] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+            } else {
+                a.part_ml[pr * 2] = m;  // log2 units; -inf when the chunk holds no valid row
+                a.part_ml[pr * 2 + 1] = l;
+            }
+        }
+    } else if (warp == 4) {
+        // ===== queries: 64 columns at a time through two slots =====
+        if (lane == 0) {
+            bool ok = true;
+            const uint32_t q_bytes = static_cast<uint32_t>(a.Hq) * 128;
+            int kb = 0;
+            for (; kb < SP_KB; ++kb) {
+                const int s = kb & 1;
+                if (kb >= 2 && !(ok = mbar_wait(&q_empty[s], ((kb >> 1) - 1) & 1))) break;
+                mbar_arrive_expect_tx(&q_full[s], q_bytes);
+                tma_load_3d(smem + SP_OFF_Q + s * SP_QBLOCK, &tm_q, &q_full[s], kb * 64, 0, b);
+            }
+            if (!ok) {
+                *s_abort = 1;
+                report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            }
+            // copies in flight complete before the CTA leaves (bounded waits)
+            for (int j = kb - 2 > 0 ? kb - 2 : 0; j < kb; ++j) mbar_wait(&q_full[j & 1], (j >> 1) & 1);
+        }
+    } else {
+        // ===== MMA issuer =====
+        if (lane == 0) {
+            bool ok = true;
+            const uint32_t c0 = smem_u32(smem + SP_OFF_C), q0 = smem_u32(smem + SP_OFF_Q);
+            const uint32_t p0 = smem_u32(smem + SP_OFF_P);
+            for (int kb = 0; kb < SP_KB && ok; ++kb) {
+                if (!(ok = mbar_wait(&c_full[kb], 0))) break;
+                if (!(ok = mbar_wait(&q_full[kb & 1], (kb >> 1) & 1))) break;
+                tc_fence_after();
+                const uint32_t qs = q0 + (kb & 1) * SP_QBLOCK, cs = c0 + kb * SP_BLOCK;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    tc_mma_bf16(tmem, umma_desc_k_sw128(qs + kk * 32), umma_desc_k_sw128(cs + kk * 32), SP_IDESC_S,
+                                (kb | kk) ? 1u : 0u);
+                tc_commit(&q_empty[kb & 1]);
+            }
+            if (ok) {
+                tc_commit(s_full);
+                ok = mbar_wait(p_full, 0);
+            }
+            if (ok) {
+                tc_fence_after();
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    // V rows = the chunk's first 512 columns, blocks 4*half .. 4*half+3
+#pragma unroll
+                    for (int kk = 0; kk < SP_ROWS / 16; ++kk) {
+                        const uint64_t ad = umma_desc_k_sw128(p0 + (kk >> 2) * SP_BLOCK + (kk & 3) * 32);
+                        const uint64_t bd = umma_desc_mn_sw128(c0 + 4 * half * SP_BLOCK + kk * 2048, SP_BLOCK, 1024);
+                        tc_mma_bf16(tmem + half * 256, ad, bd, SP_IDESC_O, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&o_full[half]);
+                }
+            }
+            if (!ok) {
+                *s_abort = 1;
+                report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            }
+            tc_commit(done);
+            mbar_wait(done, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---- merge of the chunk partials ------------------------------------------------
+// One CTA of four warps per (batch row, head); warp w merges value columns
+// 128w .. 128w+127, four per lane.  Lane j holds chunk j's (m, l), and every
+// chunk's columns are requested together with them: one memory round trip.
+constexpr int SPM_MAX_CHUNKS = 16;  // k <= 2048 in chunks of 128
+
+__global__ void __launch_bounds__(128) sparse_merge_kernel(SparseArgs a)
 {
     pdl_wait();
     pdl_trigger();
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    if (warp >= a.B * a.Hq) return;
-    const int b = warp / a.Hq, h = warp - b * a.Hq;
-    float M = -INFINITY;
-    for (int c = 0; c < a.chunks; ++c) M = fmaxf(M, a.part_ml[((static_cast<long long>(b) * a.chunks + c) * a.Hq + h) * 2]);
+    const int bh = blockIdx.x;
+    const int b = bh / a.Hq, h = bh - b * a.Hq;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int C = a.chunks;
+    const long long p0 = static_cast<long long>(b) * C * a.Hq + h;  // partial row of chunk 0
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (lane < C) ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + p0 + static_cast<long long>(lane) * a.Hq);
+    float4 ov[SPM_MAX_CHUNKS];
+#pragma unroll
+    for (int c = 0; c < SPM_MAX_CHUNKS; ++c)
+        if (c < C)
+            ov[c] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (p0 + static_cast<long long>(c) * a.Hq) * SP_DV +
+                                                           warp * 128) + lane);
+    float M = ml.x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const float Mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f;
-    float acc[SP_DV / 32];
+    const float wl = lane < C ? fast_exp2(ml.x - Mu) : 0.f;
+    float L = wl * ml.y;
 #pragma unroll
-    for (int i = 0; i < SP_DV / 32; ++i) acc[i] = 0.f;
-    for (int c = 0; c < a.chunks; ++c) {
-        const long long p = (static_cast<long long>(b) * a.chunks + c) * a.Hq + h;
-        const float wgt = fast_exp2(a.part_ml[p * 2] - Mu);
-        L += wgt * a.part_ml[p * 2 + 1];
-        const float* po = a.part_o + p * SP_DV;
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int i = 0; i < SP_DV / 32; ++i) acc[i] += wgt * po[lane + 32 * i];
+    for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
+        const float w = __shfl_sync(0xffffffffu, wl, c);
+        if (c < C) {
+            acc.x += w * ov[c].x;
+            acc.y += w * ov[c].y;
+            acc.z += w * ov[c].z;
+            acc.w += w * ov[c].w;
+        }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<long long>(b) * a.Hq + h) * SP_DV;
-#pragma unroll
-    for (int i = 0; i < SP_DV / 32; ++i) out[lane + 32 * i] = __float2bfloat16_rn(acc[i] * inv);
-    if (lane == 0 && a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<long long>(b) * a.Hq + h) * SP_DV +
+                         warp * 128 + lane * 4;
+    *reinterpret_cast<uint2*>(out) =
+        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+    if (warp == 0 && lane == 0 && a.lse)
+        a.lse[static_cast<long long>(b) * a.Hq + h] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
 }
 
 }  // namespace
 
-int sparse_chunks(int k) { return (k + SP_CHUNK - 1) / SP_CHUNK; }
+int sparse_chunks(int k) { return (k + SP_ROWS - 1) / SP_ROWS; }
 
 size_t sparse_partial_bytes(int B, int Hq, int k)
 {
@@ -284,7 +385,7 @@ size_t sparse_partial_bytes(int B, int Hq, int k)
     return static_cast<size_t>(B) * c * Hq * (SP_DV + 2) * sizeof(float);
 }
 
-cudaError_t launch_sparse_attn(const SparseLaunch& l, cudaStream_t stream)
+cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, cudaStream_t stream)
 {
     static bool attr_set[64] = {};
     int dev = 0;
@@ -296,7 +397,6 @@ cudaError_t launch_sparse_attn(const SparseLaunch& l, cudaStream_t stream)
         attr_set[dev] = true;
     }
     SparseArgs a{};
-    a.q = l.q;
     a.latent = l.latent;
     a.idx = l.idx;
     a.out = l.out;
@@ -310,10 +410,9 @@ cudaError_t launch_sparse_attn(const SparseLaunch& l, cudaStream_t stream)
     a.dev_status = l.dev_status;
     a.part_o = l.workspace;
     a.part_ml = l.workspace ? l.workspace + static_cast<size_t>(l.B) * a.chunks * l.Hq * SP_DV : nullptr;
-    e = launch_pdl(sparse_attn_kernel, dim3(a.chunks, l.Hq / SP_HB, l.B), dim3(SP_THREADS), SP_SMEM, stream, a);
+    e = launch_pdl(sparse_attn_kernel, dim3(a.chunks, l.B), dim3(SP_THREADS), SP_SMEM, stream, tm_q, a);
     if (e != cudaSuccess || a.chunks == 1) return e;
-    const int warps = l.B * l.Hq;
-    return launch_pdl(sparse_merge_kernel, dim3((warps * 32 + 255) / 256), dim3(256), 0, stream, a);
+    return launch_pdl(sparse_merge_kernel, dim3(l.B * l.Hq), dim3(128), 0, stream, a);
 }
 
 }  // namespace kvattn

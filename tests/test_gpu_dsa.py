@@ -135,7 +135,8 @@ def _sparse_ref(q, lat, idx, Dv, scale):
     return oracle.attn_sparse(W.bf16_bits(q), W.bf16_bits(lat), idx.numpy(), Dv, scale)
 
 
-@pytest.mark.parametrize("Hq,L,k", [(128, 3000, 700), (64, 600, 2048), (128, 5000, 256), (128, 2100, 2048)])
+@pytest.mark.parametrize("Hq,L,k", [(128, 3000, 700), (64, 600, 2048), (128, 5000, 256), (128, 2100, 2048),
+                                    (128, 300, 128), (64, 50, 1), (128, 1000, 129)])
 def test_sparse_attention(K, Hq, L, k):
     wl = W.DSA_128K
     B = 2
@@ -189,3 +190,19 @@ def test_sparse_bad_index_is_skipped_and_flagged(K):
     ok[0, 9] = -1
     ro, rl = _sparse_ref(q, lat, ok, wl.Dv, 0.07)
     assert_attn_close(out, ro, lse, rl, "bad index")
+
+
+def test_sparse_row_without_valid_index(K):
+    """A row whose selection is all -1 gives out = 0 and lse = -inf; the other row is unaffected."""
+    wl = W.DSA_128K
+    B, Hq, L, k = 2, 128, 400, 300
+    gen = W.generator(17)
+    q = W.normal_bf16((B, Hq, wl.Dk), gen)
+    lat = W.normal_bf16((B, L, wl.Dk), gen)
+    idx = torch.stack([torch.randperm(L, generator=gen)[:k] for _ in range(B)]).to(torch.int32)
+    idx[0] = -1
+    out, lse = K.attn_decode_sparse(q.cuda(), lat.cuda(), idx.cuda(), wl.Dv, wl.sparse_scale)
+    torch.cuda.synchronize()
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+    ro, rl = _sparse_ref(q[1:], lat[1:], idx[1:], wl.Dv, wl.sparse_scale)
+    assert_attn_close(out[1:], ro, lse[1:], rl, "row 1 next to an empty row")
