@@ -9,9 +9,10 @@
 // Kernel (tcgen05): one CTA per (batch row, chunk of 128 selected rows), all
 // query heads as the M = 128 rows of both MMAs.
 //   - warps 0-3 gather the chunk's 128 latent rows (cp.async, 16 bytes at a
-//     time) into nine 64-column blocks laid out as the tensor cores read them
-//     (128-byte rows, 128-byte swizzle); each block is signalled as it lands.
-//     Invalid indices are zero-filled and their columns masked.
+//     time, eight lanes per 128-byte line so that every warp request covers
+//     four whole lines) into nine 64-column blocks laid out as the tensor cores
+//     read them (128-byte rows, 128-byte swizzle); each block is signalled as it
+//     lands.  Invalid indices are zero-filled and their columns masked.
 //   - warp 4 streams the queries through a two-slot TMA ring, 64 columns at a
 //     time; warp 5 issues S = Q C^T (M = 128 heads, N = 128 rows, K = 576) into
 //     TMEM, block by block as the gather lands.
@@ -20,8 +21,9 @@
 //     V = the same resident rows read as an MN-major operand, N = 256 twice,
 //     into all 512 TMEM columns (S's columns are free by then).
 //   - warps 0-3 write O (normalised when the row has one chunk, else the
-//     unnormalised partial with its running max and sum); the first half is
-//     written while the second half's MMAs run.
+//     unnormalised partial with its running max and sum, stored column-major
+//     [column][head] so that a warp's 32 heads fill one 128-byte line); the
+//     first half is written while the second half's MMAs run.
 // Chunks of one row are merged by a second kernel (the split-softmax identity).
 #include "common.cuh"
 #include "kernels.h"
@@ -42,7 +44,8 @@ constexpr int SP_OFF_C = 0;                              // 9 blocks of gathered
 constexpr int SP_OFF_Q = SP_OFF_C + SP_KB * SP_BLOCK;    // 2 query slots
 constexpr int SP_OFF_P = SP_OFF_Q + 2 * SP_QBLOCK;       // P: 2 blocks of 64 rows
 constexpr int SP_OFF_VALID = SP_OFF_P + 2 * SP_BLOCK;    // [128] row valid flags
-constexpr int SP_OFF_BAR = SP_OFF_VALID + SP_ROWS * 4;
+constexpr int SP_OFF_ROW = SP_OFF_VALID + SP_ROWS * 4;   // [128] latent row of each slot (-1: none)
+constexpr int SP_OFF_BAR = SP_OFF_ROW + SP_ROWS * 4;
 // c_full[9], q_full[2], q_empty[2], s_full, p_full, o_full[2], done
 constexpr int SP_NBAR = SP_KB + 2 + 2 + 1 + 1 + 2 + 1;
 constexpr int SP_OFF_MISC = SP_OFF_BAR + SP_NBAR * 8;
@@ -58,7 +61,7 @@ struct SparseArgs {
     const int32_t* idx;         // [B][k]
     kvattn_bf16* out;           // [B][Hq][512]
     float* lse;                 // [B][Hq] or null
-    float* part_o;              // [B][chunks][Hq][512]
+    float* part_o;              // [B][chunks][512][Hq] (head fastest)
     float* part_ml;             // [B][chunks][Hq][2]
     int32_t* dev_status;
     int B, Hq, L_max, k, chunks;
@@ -87,6 +90,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     int* s_valid = reinterpret_cast<int*>(smem + SP_OFF_VALID);
+    int* s_row = reinterpret_cast<int*>(smem + SP_OFF_ROW);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SP_OFF_BAR);
     uint64_t* c_full = bars;                 // [9]: block kb of the rows landed (128 arrivals)
     uint64_t* q_full = c_full + SP_KB;       // [2]
@@ -126,22 +130,34 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     pdl_trigger();
 
     if (warp < 4) {
-        // ===== gather: thread t brings selected row t of the chunk =====
+        // ===== gather: the chunk's selected rows, block by block =====
         const int t = tid;
-        const int slot = chunk * SP_ROWS + t;
-        int j = slot < a.k ? a.idx[static_cast<long long>(b) * a.k + slot] : -1;
-        if (j < -1 || j >= a.L_max) {
-            report_status(a.dev_status, KVATTN_STATUS_BAD_INDEX);
-            j = -1;
+        {
+            const int slot = chunk * SP_ROWS + t;
+            int j = slot < a.k ? a.idx[static_cast<long long>(b) * a.k + slot] : -1;
+            if (j < -1 || j >= a.L_max) {
+                report_status(a.dev_status, KVATTN_STATUS_BAD_INDEX);
+                j = -1;
+            }
+            s_valid[t] = j >= 0;
+            s_row[t] = j;
         }
-        s_valid[t] = j >= 0;
-        const kvattn_bf16* src = a.latent + (static_cast<long long>(b) * a.L_max + (j < 0 ? 0 : j)) * SP_DK;
-        const uint32_t bytes = j < 0 ? 0u : 16u;  // 0: zero-fill
+        named_bar_sync(1, 128);  // every slot's row is known
+        // copy job i of a block: row i / 8, 16-byte chunk i % 8 (eight lanes per line)
+        const kvattn_bf16* lat = a.latent + static_cast<long long>(b) * a.L_max * SP_DK;
         const uint32_t c0 = smem_u32(smem + SP_OFF_C);
+        int jr[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) jr[u] = s_row[(t >> 3) + 16 * u];
 #pragma unroll
         for (int kb = 0; kb < SP_KB; ++kb) {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) cp_async16(c0 + kb * SP_BLOCK + swz128(t, ch), src + kb * 64 + ch * 8, bytes);
+            for (int u = 0; u < 8; ++u) {
+                const int r = (t >> 3) + 16 * u, ch = t & 7;
+                const int j = jr[u];
+                cp_async16(c0 + kb * SP_BLOCK + swz128(r, ch),
+                           lat + static_cast<long long>(j < 0 ? 0 : j) * SP_DK + kb * 64 + ch * 8, j < 0 ? 0u : 16u);
+            }
             cp_async_commit();
         }
 #pragma unroll
@@ -150,7 +166,6 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_arrive(&c_full[kb]);
         }
-        named_bar_sync(1, 128);  // every row's valid flag is written
 
         // ===== softmax of head row t (TMEM lane t) =====
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
@@ -213,7 +228,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
         // ===== epilogue: O row t, half by half =====
         const bool one = a.chunks == 1;
         const long long bh = static_cast<long long>(b) * a.Hq + t;
-        const long long pr = (static_cast<long long>(b) * a.chunks + chunk) * a.Hq + t;  // partial row
+        const long long pc = (static_cast<long long>(b) * a.chunks + chunk) * SP_DV;  // partial column 0
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
         for (int half = 0; half < 2; ++half) {
@@ -236,12 +251,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                             pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv),
                             pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv));
                 } else {
-                    float* po = a.part_o + pr * SP_DV + col;
+                    // [column][head]: the warp's 32 heads of one column are one 128-byte line
+                    float* po = a.part_o + (pc + col) * a.Hq + t;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(po + i) =
-                            make_float4(__uint_as_float(ov[i]), __uint_as_float(ov[i + 1]),
-                                        __uint_as_float(ov[i + 2]), __uint_as_float(ov[i + 3]));
+                    for (int i = 0; i < 32; ++i) po[static_cast<long long>(i) * a.Hq] = __uint_as_float(ov[i]);
                 }
             }
         }
@@ -249,6 +262,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             if (one) {
                 if (a.lse) a.lse[bh] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
             } else {
+                const long long pr = (static_cast<long long>(b) * a.chunks + chunk) * a.Hq + t;
                 a.part_ml[pr * 2] = m;  // log2 units; -inf when the chunk holds no valid row
                 a.part_ml[pr * 2 + 1] = l;
             }
@@ -324,54 +338,64 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
 }
 
 // ---- merge of the chunk partials ------------------------------------------------
-// One CTA of four warps per (batch row, head); warp w merges value columns
-// 128w .. 128w+127, four per lane.  Lane j holds chunk j's (m, l), and every
-// chunk's columns are requested together with them: one memory round trip.
+// CTA = (batch row, 32 heads, 32 value columns), 256 threads: lane = head, warp w
+// = columns 4w .. 4w+3.  Every thread derives its head's chunk weights from the
+// (m, l) pairs and requests all chunks' values at once (one round trip); the
+// 32 x 32 result is transposed through shared memory so that each head's 32
+// columns are written as one 64-byte run.
 constexpr int SPM_MAX_CHUNKS = 16;  // k <= 2048 in chunks of 128
+constexpr int SPM_HEADS = 32, SPM_COLS = 32;
 
-__global__ void __launch_bounds__(128) sparse_merge_kernel(SparseArgs a)
+__global__ void __launch_bounds__(256) sparse_merge_kernel(SparseArgs a)
 {
+    __shared__ float s_o[SPM_HEADS][SPM_COLS + 1];
+    __shared__ float s_lse[SPM_HEADS];
     pdl_wait();
     pdl_trigger();
-    const int bh = blockIdx.x;
-    const int b = bh / a.Hq, h = bh - b * a.Hq;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int C = a.chunks;
-    const long long p0 = static_cast<long long>(b) * C * a.Hq + h;  // partial row of chunk 0
-    float2 ml = make_float2(-INFINITY, 0.f);
-    if (lane < C) ml = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + p0 + static_cast<long long>(lane) * a.Hq);
-    float4 ov[SPM_MAX_CHUNKS];
-#pragma unroll
-    for (int c = 0; c < SPM_MAX_CHUNKS; ++c)
-        if (c < C)
-            ov[c] = __ldcg(reinterpret_cast<const float4*>(a.part_o + (p0 + static_cast<long long>(c) * a.Hq) * SP_DV +
-                                                           warp * 128) + lane);
-    float M = ml.x;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float Mu = M == -INFINITY ? 0.f : M;
-    const float wl = lane < C ? fast_exp2(ml.x - Mu) : 0.f;
-    float L = wl * ml.y;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int col0 = blockIdx.x * SPM_COLS, h0 = blockIdx.y * SPM_HEADS, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = h0 + lane;
+    const long long mlrow = static_cast<long long>(b) * C * a.Hq + h;  // (m, l) row of chunk 0
+    float2 ml[SPM_MAX_CHUNKS];
+    float ov[SPM_MAX_CHUNKS][4];
 #pragma unroll
     for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
-        const float w = __shfl_sync(0xffffffffu, wl, c);
         if (c < C) {
-            acc.x += w * ov[c].x;
-            acc.y += w * ov[c].y;
-            acc.z += w * ov[c].z;
-            acc.w += w * ov[c].w;
+            ml[c] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + mlrow + static_cast<long long>(c) * a.Hq);
+            const float* po = a.part_o + ((static_cast<long long>(b) * C + c) * SP_DV + col0 + 4 * warp) * a.Hq + h;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) ov[c][i] = __ldcg(po + static_cast<long long>(i) * a.Hq);
+        }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < SPM_MAX_CHUNKS; ++c)
+        if (c < C) M = fmaxf(M, ml[c].x);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
+        if (c < C) {
+            const float w = fast_exp2(ml[c].x - Mu);
+            L += w * ml[c].y;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] += w * ov[c][i];
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<long long>(b) * a.Hq + h) * SP_DV +
-                         warp * 128 + lane * 4;
-    *reinterpret_cast<uint2*>(out) =
-        make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-    if (warp == 0 && lane == 0 && a.lse)
-        a.lse[static_cast<long long>(b) * a.Hq + h] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s_o[lane][4 * warp + i] = acc[i] * inv;
+    if (warp == 0) s_lse[lane] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+    __syncthreads();
+    // thread -> (head tid / 8, columns 4 (tid % 8) .. +3): eight threads per head's 64 bytes
+    const int hh = threadIdx.x >> 3, cc = (threadIdx.x & 7) * 4;
+    __nv_bfloat16* out =
+        reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<long long>(b) * a.Hq + h0 + hh) * SP_DV + col0 + cc;
+    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(s_o[hh][cc], s_o[hh][cc + 1]),
+                                                pack_bf16x2(s_o[hh][cc + 2], s_o[hh][cc + 3]));
+    if (blockIdx.x == 0 && threadIdx.x < SPM_HEADS && a.lse)
+        a.lse[static_cast<long long>(b) * a.Hq + h0 + threadIdx.x] = s_lse[threadIdx.x];
 }
 
 }  // namespace
@@ -412,7 +436,7 @@ cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, c
     a.part_ml = l.workspace ? l.workspace + static_cast<size_t>(l.B) * a.chunks * l.Hq * SP_DV : nullptr;
     e = launch_pdl(sparse_attn_kernel, dim3(a.chunks, l.B), dim3(SP_THREADS), SP_SMEM, stream, tm_q, a);
     if (e != cudaSuccess || a.chunks == 1) return e;
-    return launch_pdl(sparse_merge_kernel, dim3(l.B * l.Hq), dim3(128), 0, stream, a);
+    return launch_pdl(sparse_merge_kernel, dim3(SP_DV / SPM_COLS, l.Hq / SPM_HEADS, l.B), dim3(256), 0, stream, a);
 }
 
 }  // namespace kvattn
