@@ -8,8 +8,8 @@
 // which is the tcgen05 rate, not the mma.sync one.
 //
 // Per 64-key tile: S = Q K^T with M = 64 heads (rows in TMEM lanes 0-15 of
-// each 32-lane quarter), N = 64 keys, K = 128, double-buffered in TMEM so
-// the next tile's scores are computed while this one's softmax runs; the
+// each 32-lane quarter), N = 64 keys, K = 128, double-buffered in TMEM so the
+// next tile's scores are computed while this one's softmax runs; the
 // softmax (four warps reading their 16 lanes with the 16x256b shape, so that
 // all 32 threads work: a head's keys spread over a lane quad, two heads per
 // thread) writes P as bf16 into a swizzled shared-memory tile and O += P V runs as a second MMA into a
@@ -35,8 +35,9 @@ constexpr int TC_TILE = 2 * TC_BOX;       // 16 KB: a K or V tile [64 x 128]
 constexpr int TC_QBOX = TC_M * 128;       // 8 KB
 constexpr int TC_PBYTES = TC_M * 128;     // 8 KB: P tile [64 heads x 64 keys] bf16
 constexpr int TC_THREADS = 224;           // w0 TMA, w1 S MMAs + TMEM, w2-5 softmax, w6 P V MMAs
+constexpr int TC_NB = 2;                  // S and P buffers (a third one measured no faster)
 constexpr int TC_TMEM_COLS = 256;         // S0 | S1 (64 columns each) | O (128)
-constexpr int TC_OCOL = 2 * TC_T;
+constexpr int TC_OCOL = TC_NB * TC_T;
 constexpr uint32_t TC_IDESC_S = umma_idesc_bf16(TC_M, TC_T);             // Q x K^T
 constexpr uint32_t TC_IDESC_O = umma_idesc_bf16(TC_M, TC_D, false, true);  // P x V (V MN-major)
 constexpr float kLog2e = 1.44269504088896340736f;
@@ -46,15 +47,16 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int TC_OFF_K = 0;
 constexpr int TC_OFF_V = TC_OFF_K + TC_KS * TC_TILE;
 constexpr int TC_OFF_Q = TC_OFF_V + TC_VS * TC_TILE;
-constexpr int TC_OFF_P = TC_OFF_Q + 2 * TC_QBOX;                  // two P tiles
-constexpr int TC_OFF_N = TC_OFF_P + 2 * TC_PBYTES;
+constexpr int TC_OFF_P = TC_OFF_Q + 2 * TC_QBOX;                  // TC_NB P tiles
+constexpr int TC_OFF_N = TC_OFF_P + TC_NB * TC_PBYTES;
 constexpr int TC_OFF_UB = TC_OFF_N + DECODE_MAX_B * 4;
 constexpr int TC_OFF_LEN = TC_OFF_UB + (DECODE_MAX_B + 1) * 4;
 constexpr int TC_OFF_BAR = (TC_OFF_LEN + DECODE_MAX_B * 4 + 7) / 8 * 8;
-// kfull[KS], kempty[KS], vfull[VS], vempty[VS], q_full, q_empty, s_full[2], p_full[2], pv_done[2], done[2]
-constexpr int TC_NBAR = 2 * TC_KS + 2 * TC_VS + 10;
+// kfull[KS], kempty[KS], vfull[VS], vempty[VS], q_full, q_empty, s_full[NB], p_full[NB], pv_done[NB], done[2]
+constexpr int TC_NBAR = 2 * TC_KS + 2 * TC_VS + 2 + 3 * TC_NB + 2;
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_SMEM = TC_OFF_MISC + 32 + 1024;
+static_assert(TC_SMEM <= 232448, "shared memory");
 
 // The tiles of one CTA in stream order, with the piece they belong to.
 struct TileStream {
@@ -97,12 +99,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint64_t* vempty = vfull + TC_VS;
     uint64_t* q_full = vempty + TC_VS;
     uint64_t* q_empty = q_full + 1;
-    // Every barrier below is indexed by tile parity (i & 1), so that no waiter is ever
-    // more than one phase behind it (the P and S double buffers bound the lag).
-    uint64_t* s_full = q_full + 2;   // [2]: S of tile i ready in S buffer i & 1
-    uint64_t* p_full = q_full + 4;   // [2]: P of tile i ready in P buffer i & 1 (S buffer i & 1 read)
-    uint64_t* pv_done = q_full + 6;  // [2]: P V of tile i finished (P buffer i & 1 free, O updated)
-    uint64_t* done = q_full + 8;     // [2]: all S MMAs / all P V MMAs finished
+    // Every barrier below is indexed by the tile's buffer i % TC_NB and waited with
+    // phase (i / TC_NB) & 1, so that no waiter is ever more than one phase behind it
+    // (the S and P buffers bound the lag).
+    uint64_t* s_full = q_full + 2;               // [NB]: S of tile i ready in S buffer i % NB
+    uint64_t* p_full = s_full + TC_NB;           // [NB]: P of tile i ready (S buffer i % NB read)
+    uint64_t* pv_done = p_full + TC_NB;          // [NB]: P V of tile i finished (P buffer free, O updated)
+    uint64_t* done = pv_done + TC_NB;            // [2]: all S MMAs / all P V MMAs finished
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + TC_OFF_MISC + 4);
     int* s_acc = reinterpret_cast<int*>(smem + TC_OFF_MISC + 8);
@@ -119,12 +122,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int x = 0; x < 2; ++x) {
+        for (int x = 0; x < TC_NB; ++x) {
             mbar_init(&s_full[x], 1);
             mbar_init(&p_full[x], 4);
             mbar_init(&pv_done[x], 1);
-            mbar_init(&done[x], 1);
         }
+        for (int x = 0; x < 2; ++x) mbar_init(&done[x], 1);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -221,12 +224,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     piece_s = ts.piece;
                 }
                 const int ks = i % TC_KS;
-                // S buffer i & 1 was read by the softmax of tile i - 2
-                if (i >= 2 && !(ok = mbar_wait(&p_full[i & 1], ((i >> 1) - 1) & 1))) break;
+                // S buffer i % NB was read by the softmax of tile i - NB
+                if (i >= TC_NB && !(ok = mbar_wait(&p_full[i % TC_NB], ((i / TC_NB) - 1) & 1))) break;
                 if (!(ok = mbar_wait(&kfull[ks], (i / TC_KS) & 1))) break;
                 tc_fence_after();
                 const uint32_t kt = smem_u32(smem + TC_OFF_K + ks * TC_TILE);
-                const uint32_t d = tmem + (i & 1) * TC_T;
+                const uint32_t d = tmem + (i % TC_NB) * TC_T;
 #pragma unroll
                 for (int kk = 0; kk < TC_D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * TC_BOX + (kk & 3) * 32;
@@ -234,7 +237,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                 kk > 0 ? 1u : 0u);
                 }
                 tc_commit(&kempty[ks]);
-                tc_commit(&s_full[i & 1]);
+                tc_commit(&s_full[i % TC_NB]);
             }
             if (!ok) {
                 *s_abort = 1;
@@ -251,11 +254,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             bool ok = true, first = false;
             for (int i = 0; ok && ts.next(lo, hi, a.B, a.Hk, s_n, N, G, first); ++i) {
                 const int vs = i % TC_VS;
-                if (!(ok = mbar_wait(&p_full[i & 1], (i >> 1) & 1))) break;
+                if (!(ok = mbar_wait(&p_full[i % TC_NB], (i / TC_NB) & 1))) break;
                 if (!(ok = mbar_wait(&vfull[vs], (i / TC_VS) & 1))) break;
                 tc_fence_after();
                 const uint32_t vt = smem_u32(smem + TC_OFF_V + vs * TC_TILE);
-                const uint32_t pa = sp + (i & 1) * TC_PBYTES;
+                const uint32_t pa = sp + (i % TC_NB) * TC_PBYTES;
 #pragma unroll
                 for (int kk = 0; kk < TC_T / 16; ++kk) {
                     const uint64_t bd = umma_desc_mn_sw128(vt + kk * 2048, TC_BOX, 1024);
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                                 (!first || kk > 0) ? 1u : 0u);
                 }
                 tc_commit(&vempty[vs]);
-                tc_commit(&pv_done[i & 1]);
+                tc_commit(&pv_done[i % TC_NB]);
             }
             if (!ok) {
                 *s_abort = 1;
@@ -298,13 +301,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             float2 l2 = make_float2(0.f, 0.f);      // this thread's share of their sums
             for (long long t = tb; t < te; ++t, ++i) {
                 const bool first = t == tb;
-                if (!warp_wait(&s_full[i & 1], (i >> 1) & 1, s_abort)) continue;
-                // P buffer i & 1 is free once the P V of tile i - 2 has finished
-                if (t - tb >= 2 && !warp_wait(&pv_done[i & 1], ((i >> 1) - 1) & 1, s_abort)) continue;
+                if (!warp_wait(&s_full[i % TC_NB], (i / TC_NB) & 1, s_abort)) continue;
+                // P buffer i % NB is free once the P V of tile i - NB has finished (the
+                // previous piece's epilogue waited for all of its P V)
+                if (t - tb >= TC_NB && !warp_wait(&pv_done[i % TC_NB], ((i / TC_NB) - 1) & 1, s_abort)) continue;
                 tc_fence_after();
                 const int n_valid = len - static_cast<int>(t) * TC_T;  // >= 1
                 uint32_t sv[32];
-                tmem_ld_16x256b_x8(tmem + lane_off + (i & 1) * TC_T, sv);
+                tmem_ld_16x256b_x8(tmem + lane_off + (i % TC_NB) * TC_T, sv);
                 tmem_wait_ld();
                 if (n_valid < TC_T) {  // tail tile (warp-uniform): keys past the length -> -inf
 #pragma unroll
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const bool rs0 = mv0 && m0 != -INFINITY && !first, rs1 = mv1 && m1 != -INFINITY && !first;
                 if (__any_sync(0xffffffffu, rs0 || rs1)) {
                     // O must be stable: wait for the P V of the previous tile
-                    if (!warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, s_abort)) continue;
+                    if (!warp_wait(&pv_done[(i - 1) % TC_NB], ((i - 1) / TC_NB) & 1, s_abort)) continue;
                     tc_fence_after();
                     const float al0 = rs0 ? fast_exp2(m0 - n0) : 1.f, al1 = rs1 ? fast_exp2(m1 - n1) : 1.f;
                     l2.x *= al0;
@@ -354,8 +358,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 const float2 nmu1 = make_float2(m1 == -INFINITY ? 0.f : -m1, m1 == -INFINITY ? 0.f : -m1);
                 // a tail tile's V rows are zeroed below: its load must have landed first
                 if (n_valid < TC_T && !warp_wait(&vfull[i % TC_VS], (i / TC_VS) & 1, s_abort)) continue;
-                // P -> 128-byte swizzled rows h0, h1 of P tile i & 1 (4 bytes per chunk and head)
-                uint8_t* pt = sP0 + (i & 1) * TC_PBYTES + cq * 2;
+                // P -> 128-byte swizzled rows h0, h1 of P tile i % NB (4 bytes per chunk and head)
+                uint8_t* pt = sP0 + (i % TC_NB) * TC_PBYTES + cq * 2;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float2 x0 = __ffma2_rn(make_float2(__uint_as_float(sv[4 * j]), __uint_as_float(sv[4 * j + 1])),
@@ -390,7 +394,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[i & 1]);
+                if (lane == 0) mbar_arrive(&p_full[i % TC_NB]);
             }
             // ---- end of the piece: O (and m, l) out once its last P V has finished ----
             float l0 = l2.x, l1 = l2.y;
@@ -398,7 +402,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
             l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
             l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-            if (warp_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, s_abort)) {
+            if (warp_wait(&pv_done[(i - 1) % TC_NB], ((i - 1) / TC_NB) & 1, s_abort)) {
                 tc_fence_after();
                 const bool fin = count == 1;
                 const long long bh0 = static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g + h0;

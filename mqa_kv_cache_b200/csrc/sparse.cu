@@ -13,11 +13,12 @@
 //     four whole lines) into nine 64-column blocks laid out as the tensor cores
 //     read them (128-byte rows, 128-byte swizzle); each block is signalled as it
 //     lands.  Invalid indices are zero-filled and their columns masked.
-//   - warp 4 streams the queries through a two-slot TMA ring, 64 columns at a
+//   - warp 4 streams the queries through a four-slot TMA ring, 64 columns at a
 //     time; warp 5 issues S = Q C^T (M = 128 heads, N = 128 rows, K = 576) into
 //     TMEM, block by block as the gather lands.
 //   - warps 0-3 (thread = head = TMEM lane) take the row softmax of S in base 2
-//     and write P as bf16 into shared memory; warp 5 then issues O = P V with
+//     and write P as bf16 into shared memory (over two query slots, free once S
+//     is complete); warp 5 then issues O = P V with
 //     V = the same resident rows read as an MN-major operand, N = 256 twice,
 //     into all 512 TMEM columns (S's columns are free by then).
 //   - warps 0-3 write O (normalised when the row has one chunk, else the
@@ -41,13 +42,14 @@ constexpr int SP_BLOCK = SP_ROWS * 128;        // 16 KB: 128 rows x 64 columns
 constexpr int SP_QBLOCK = SP_M * 128;          // 16 KB: 128 heads x 64 columns
 constexpr int SP_THREADS = 192;                // w0-3 gather/softmax/epilogue, w4 TMA, w5 MMA + TMEM
 constexpr int SP_OFF_C = 0;                              // 9 blocks of gathered rows
-constexpr int SP_OFF_Q = SP_OFF_C + SP_KB * SP_BLOCK;    // 2 query slots
-constexpr int SP_OFF_P = SP_OFF_Q + 2 * SP_QBLOCK;       // P: 2 blocks of 64 rows
-constexpr int SP_OFF_VALID = SP_OFF_P + 2 * SP_BLOCK;    // [128] row valid flags
-constexpr int SP_OFF_ROW = SP_OFF_VALID + SP_ROWS * 4;   // [128] latent row of each slot (-1: none)
+constexpr int SP_QS = 4;                                 // query slots
+constexpr int SP_OFF_Q = SP_OFF_C + SP_KB * SP_BLOCK;    // SP_QS query slots
+constexpr int SP_OFF_P = SP_OFF_Q;                       // P: 2 blocks of 64 rows, over slots 0-1 after S
+constexpr int SP_OFF_VALID = SP_OFF_Q + SP_QS * SP_QBLOCK;  // [4] bit masks: slot row holds a valid index
+constexpr int SP_OFF_ROW = SP_OFF_VALID + 16;            // [128] latent row of each slot (-1: none)
 constexpr int SP_OFF_BAR = SP_OFF_ROW + SP_ROWS * 4;
-// c_full[9], q_full[2], q_empty[2], s_full, p_full, o_full[2], done
-constexpr int SP_NBAR = SP_KB + 2 + 2 + 1 + 1 + 2 + 1;
+// c_full[9], q_full[4], q_empty[4], s_full, p_full, o_full[2], done
+constexpr int SP_NBAR = SP_KB + SP_QS + SP_QS + 1 + 1 + 2 + 1;
 constexpr int SP_OFF_MISC = SP_OFF_BAR + SP_NBAR * 8;
 constexpr int SP_SMEM = SP_OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(SP_SMEM <= 232448, "shared memory");
@@ -89,13 +91,13 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    int* s_valid = reinterpret_cast<int*>(smem + SP_OFF_VALID);
+    uint32_t* s_vmask = reinterpret_cast<uint32_t*>(smem + SP_OFF_VALID);
     int* s_row = reinterpret_cast<int*>(smem + SP_OFF_ROW);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SP_OFF_BAR);
     uint64_t* c_full = bars;                 // [9]: block kb of the rows landed (128 arrivals)
-    uint64_t* q_full = c_full + SP_KB;       // [2]
-    uint64_t* q_empty = q_full + 2;          // [2]
-    uint64_t* s_full = q_empty + 2;          // S complete in TMEM
+    uint64_t* q_full = c_full + SP_KB;       // [SP_QS]
+    uint64_t* q_empty = q_full + SP_QS;      // [SP_QS]
+    uint64_t* s_full = q_empty + SP_QS;      // S complete in TMEM
     uint64_t* p_full = s_full + 1;           // P written (S read), 128 arrivals
     uint64_t* o_full = p_full + 1;           // [2]: O columns 0-255 / 256-511 complete
     uint64_t* done = o_full + 2;             // every MMA finished
@@ -106,11 +108,11 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < SP_KB; ++i) mbar_init(&c_full[i], 128);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < SP_QS; ++i) {
             mbar_init(&q_full[i], 1);
             mbar_init(&q_empty[i], 1);
-            mbar_init(&o_full[i], 1);
         }
+        for (int i = 0; i < 2; ++i) mbar_init(&o_full[i], 1);
         mbar_init(s_full, 1);
         mbar_init(p_full, 128);
         mbar_init(done, 1);
@@ -139,7 +141,8 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                 report_status(a.dev_status, KVATTN_STATUS_BAD_INDEX);
                 j = -1;
             }
-            s_valid[t] = j >= 0;
+            const uint32_t vm = __ballot_sync(0xffffffffu, j >= 0);
+            if (lane == 0) s_vmask[warp] = vm;
             s_row[t] = j;
         }
         named_bar_sync(1, 128);  // every slot's row is known
@@ -181,9 +184,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             float mx = -INFINITY;
 #pragma unroll
             for (int cc = 0; cc < 4; ++cc) {
+                const uint32_t vm = s_vmask[cc];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    if (!s_valid[cc * 32 + i]) sv[cc][i] = 0xff800000u;  // -inf: not a selected row
+                    if (!((vm >> i) & 1u)) sv[cc][i] = 0xff800000u;  // -inf: not a selected row
                     mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
                 }
             }
@@ -268,14 +272,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             }
         }
     } else if (warp == 4) {
-        // ===== queries: 64 columns at a time through two slots =====
+        // ===== queries: 64 columns at a time through SP_QS slots =====
         if (lane == 0) {
             bool ok = true;
             const uint32_t q_bytes = static_cast<uint32_t>(a.Hq) * 128;
             int kb = 0;
             for (; kb < SP_KB; ++kb) {
-                const int s = kb & 1;
-                if (kb >= 2 && !(ok = mbar_wait(&q_empty[s], ((kb >> 1) - 1) & 1))) break;
+                const int s = kb % SP_QS;
+                if (kb >= SP_QS && !(ok = mbar_wait(&q_empty[s], ((kb / SP_QS) - 1) & 1))) break;
                 mbar_arrive_expect_tx(&q_full[s], q_bytes);
                 tma_load_3d(smem + SP_OFF_Q + s * SP_QBLOCK, &tm_q, &q_full[s], kb * 64, 0, b);
             }
@@ -284,7 +288,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                 report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
             }
             // copies in flight complete before the CTA leaves (bounded waits)
-            for (int j = kb - 2 > 0 ? kb - 2 : 0; j < kb; ++j) mbar_wait(&q_full[j & 1], (j >> 1) & 1);
+            for (int j = kb - SP_QS > 0 ? kb - SP_QS : 0; j < kb; ++j) mbar_wait(&q_full[j % SP_QS], (j / SP_QS) & 1);
         }
     } else {
         // ===== MMA issuer =====
@@ -294,14 +298,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             const uint32_t p0 = smem_u32(smem + SP_OFF_P);
             for (int kb = 0; kb < SP_KB && ok; ++kb) {
                 if (!(ok = mbar_wait(&c_full[kb], 0))) break;
-                if (!(ok = mbar_wait(&q_full[kb & 1], (kb >> 1) & 1))) break;
+                if (!(ok = mbar_wait(&q_full[kb % SP_QS], (kb / SP_QS) & 1))) break;
                 tc_fence_after();
-                const uint32_t qs = q0 + (kb & 1) * SP_QBLOCK, cs = c0 + kb * SP_BLOCK;
+                const uint32_t qs = q0 + (kb % SP_QS) * SP_QBLOCK, cs = c0 + kb * SP_BLOCK;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc_mma_bf16(tmem, umma_desc_k_sw128(qs + kk * 32), umma_desc_k_sw128(cs + kk * 32), SP_IDESC_S,
                                 (kb | kk) ? 1u : 0u);
-                tc_commit(&q_empty[kb & 1]);
+                tc_commit(&q_empty[kb % SP_QS]);
             }
             if (ok) {
                 tc_commit(s_full);
