@@ -3,8 +3,10 @@
 
 Headline workload: the Llama-3-8B-shaped single-layer decode (B=16, n_head=32,
 n_kv_head=8, d=128, ragged cache lengths uniform in [1024, 8192], RoPE base
-500000).  One step = rope_apply_qk on the batch's new queries (each at
-position len_b; cached keys were rotated when written) + attn_decode_gqa.
+500000).  One step = attn_decode_gqa_rope: the batch's new queries rotated
+at position len_b inside the decode kernel (cached keys were rotated when
+written), then attention over the cache.  The same work as two launches
+(rope_apply_qk, then attn_decode_gqa) is reported beside it.
 Metric: effective HBM GB/s = algorithmic bytes (K/V rows read once, q read,
 out and lse written) / step time; also tokens/s (= B / step time).
 
@@ -34,7 +36,7 @@ METRIC = "decode-attn effective HBM GB/s (% of peak) & tok/s; prefill TFLOP/s"
 # DRAM bytes (read + write) of one decode_kernel launch on the headline workload, from an ncu
 # capture of the current kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the
 # kernel changes after that capture.
-DECODE_TRAFFIC_BYTES = 295_062_272 + 4_179_712
+DECODE_TRAFFIC_BYTES = 295_059_200 + 3_644_416
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -143,7 +145,6 @@ class DecodeStep:
         self.k, self.v = inp["k"], inp["v"]
         # cached keys are rotated once, when they are written to the cache
         K.rope_apply_qk(None, None, self.k, inp["k_pos"].to(device), self.cos, self.sin, k_layout="bhtd")
-        self.q_raw = inp["q"]
         self.inbuf, (self.q, self.q_pos, self.lens) = packed(
             [(tuple(inp["q"].shape), torch.bfloat16), (tuple(inp["q_pos"].shape), torch.int32),
              (tuple(inp["seq_lens"].shape), torch.int32)], device)
@@ -155,23 +156,32 @@ class DecodeStep:
             [(tuple(inp["q"].shape), torch.bfloat16), ((w.B, w.H), torch.float32)], device)
         self.ws = K.workspace(K.attn_decode_gqa_workspace_bytes(w.B, w.H, w.Hk, w.d, w.T_max), device)
         self.bytes = decode_bytes(w, inp["seq_lens"])
-        # rope_apply and the decode kernel; the tcgen05 path (d = 128 with 64 query heads per
-        # KV head) adds its merge kernel, the mma.sync path merges inside the decode kernel
-        self.launches_per_step = 3 if (w.d == 128 and w.g == 64) else 2
-
-    def reset_q(self):
-        self.q.copy_(self.q_raw)
-
-    def rope(self):
-        self.K.rope_apply_qk(self.q, self.q_pos, None, None, self.cos, self.sin, q_layout="bhd")
-
-    def attn(self):
-        self.K.attn_decode_gqa(self.q, self.k, self.v, self.lens, self.w.scale, out=self.out, lse=self.lse,
-                               ws=self.ws)
+        # the decode kernel (RoPE of q inside); the tcgen05 path (d = 128 with 64 query heads
+        # per KV head) adds its merge kernel, the mma.sync path merges inside the decode kernel
+        self.launches_per_step = 2 if (w.d == 128 and w.g == 64) else 1
+        self.q_work = self.q.clone()  # the unfused variant rotates a copy in place
+        # queries rotated once, for the attention kernel alone (attn_decode_gqa)
+        self.q_rot = self.q.clone()
+        K.rope_apply_qk(self.q_rot, self.q_pos, None, None, self.cos, self.sin, q_layout="bhd")
 
     def step(self):
-        self.rope()
-        self.attn()
+        """The fused step: queries rotated inside the decode kernel (q is not modified)."""
+        self.K.attn_decode_gqa_rope(self.q, self.q_pos, self.cos, self.sin, self.k, self.v, self.lens,
+                                    self.w.scale, out=self.out, lse=self.lse, ws=self.ws)
+
+    def attn(self):
+        """Attention alone on pre-rotated queries (attn_decode_gqa)."""
+        self.K.attn_decode_gqa(self.q_rot, self.k, self.v, self.lens, self.w.scale, out=self.out, lse=self.lse,
+                               ws=self.ws)
+
+    def reset_work(self):
+        self.q_work.copy_(self.q)
+
+    def unfused(self):
+        """The same work as two launches: rope_apply_qk on a copy, then attn_decode_gqa."""
+        self.K.rope_apply_qk(self.q_work, self.q_pos, None, None, self.cos, self.sin, q_layout="bhd")
+        self.K.attn_decode_gqa(self.q_work, self.k, self.v, self.lens, self.w.scale, out=self.out, lse=self.lse,
+                               ws=self.ws)
 
 
 def capture(fn):
@@ -218,16 +228,17 @@ def run_gpu(args, rank, world, device):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     for _ in range(args.warmup):
-        job.reset_q()
         job.step()
+        job.reset_work()
+        job.unfused()
     torch.cuda.synchronize()
-    # the step and the attention alone, captured once as CUDA graphs
+    # the fused step and the unfused pair, captured once as CUDA graphs
     step_graph = capture(job.step)
-    attn_graph = capture(job.attn)
+    unfused_graph = capture(job.unfused)
     for _ in range(args.warmup):
-        job.reset_q()
         step_graph.replay()
-        attn_graph.replay()
+        job.reset_work()
+        unfused_graph.replay()
     torch.cuda.synchronize()
 
     # ---- timed region: K whole steps (graph replays, L2 flushed in between) ----
@@ -235,20 +246,20 @@ def run_gpu(args, rank, world, device):
     torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device() if device.index is None else device.index)
     with sampler:
-        step_ms = time_steps(step_graph.replay, args.steps, flush, before=job.reset_q)
+        step_ms = time_steps(step_graph.replay, args.steps, flush)
     barrier(world)
     torch.cuda.synchronize()
     total_bytes, ms = whole_job(job.bytes, float(np.mean(step_ms)), world, device)
 
-    # ---- dominant kernel alone (decode + merge launches), same stream ----
-    attn_ms = max_over_ranks(float(np.mean(time_steps(attn_graph.replay, args.steps, flush))), world, device)
-    # the same step launched eagerly from Python (host launch path included)
-    eager_ms = max_over_ranks(float(np.mean(time_steps(job.step, args.steps, flush, before=job.reset_q))),
-                              world, device)
+    # ---- the step is one kernel: it is also the roofline's kernel.  For context: the same
+    # work as two launches, and the fused step launched eagerly from Python ----
+    attn_ms = ms
+    unfused_ms = max_over_ranks(float(np.mean(time_steps(unfused_graph.replay, args.steps, flush,
+                                                          before=job.reset_work))), world, device)
+    eager_ms = max_over_ranks(float(np.mean(time_steps(job.step, args.steps, flush))), world, device)
 
     # ---- end to end through the public API with host buffers: the step's packed
     # inputs (raw q, positions, lengths) in, rope + decode, packed (out, lse) back ----
-    job.reset_q()
     in_host = job.inbuf.cpu().pin_memory()
     out_host = torch.empty(job.outbuf.shape, dtype=torch.uint8).pin_memory()
 
@@ -285,9 +296,11 @@ def run_gpu(args, rank, world, device):
                    "l2": "flushed between timed steps (read of a 256 MB buffer), and inputs exceed L2"},
         "tok_per_s": round(w.B * world / (ms * 1e-3), 1),
         "step_launch": "CUDA graph replay (eager Python launch: %.4f ms/step)" % eager_ms,
+        "unfused_ms_per_step": round(unfused_ms, 5),
         "pct_of_hbm_peak": round(100.0 * gbs / world / peaks["hbm_gbs"], 2),
         "pct_of_nominal_8tbs": round(100.0 * gbs / world / 8000.0, 2),
-        "roofline": {"kernel": "attn_decode_gqa (split-K decode + merge)", "bound": "hbm",
+        "roofline": {"kernel": "decode_kernel (attn_decode_gqa_rope: RoPE of q, split-K decode, merge)",
+                     "bound": "hbm",
                      "achieved": round(attn_gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(attn_gbs / peaks["hbm_gbs"], 4), "traffic": DECODE_TRAFFIC_BYTES,
                      "peak_source": peaks["source"], "algorithmic_bytes": job.bytes},
@@ -313,11 +326,13 @@ def _graph_ms(fn, steps, flush, warmup=3, before=None):
 
 def measure_decode_config(K, w, device, steps, flush, peaks):
     job = DecodeStep(K, w, device, W.SEED_BASE + w.index)
-    ms = _graph_ms(job.step, steps, flush, before=job.reset_q)
+    ms = _graph_ms(job.step, steps, flush)
+    unfused_ms = _graph_ms(job.unfused, steps, flush, before=job.reset_work)
     attn_ms = _graph_ms(job.attn, steps, flush)
-    out = {"workload": w.name, "ms_per_step": round(ms, 5), "attn_ms": round(attn_ms, 5),
-           "algorithmic_bytes": job.bytes, "GB_s": round(job.bytes / (ms * 1e-3) / 1e9, 1),
-           "attn_GB_s": round(job.bytes / (attn_ms * 1e-3) / 1e9, 1),
+    out = {"workload": w.name, "ms_per_step": round(ms, 5), "unfused_ms_per_step": round(unfused_ms, 5),
+           "attn_ms": round(attn_ms, 5), "algorithmic_bytes": job.bytes,
+           "GB_s": round(job.bytes / (ms * 1e-3) / 1e9, 1),
+           "pct_of_hbm_peak": round(100 * job.bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 1),
            "attn_pct_of_hbm_peak": round(100 * job.bytes / (attn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 1),
            "tok_per_s": round(w.B / (ms * 1e-3), 1)}
     del job

@@ -158,6 +158,45 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
                     size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * attn_decode_gqa on queries that are not yet rotated: q [B][n_head][d] holds
+ * the raw projections, and each sequence's query is rotated inside the decode
+ * kernel at position q_pos[b] (device int32 [B]) with the tables of
+ * rope_table_build (cos_tab, sin_tab [max_pos][d/2], pair_style as in
+ * rope_apply_qk) -- RoPE on q only, never on v ("Agentic RL 入门3" §1.1), the
+ * cached keys having been rotated when they were written.  q is not modified.
+ * The rotation is bit-identical to rope_apply_qk's, so the result equals
+ * rope_apply_qk on q followed by attn_decode_gqa, in one launch.  A position
+ * outside [0, max_pos) sets KVATTN_STATUS_BAD_POSITION and that sequence's
+ * query is used unrotated.  Workspace, outputs and limits as attn_decode_gqa;
+ * the tables must be 16-byte aligned.
+ */
+int attn_decode_gqa_rope(const kvattn_bf16* q, const int32_t* q_pos, const float* cos_tab,
+                         const float* sin_tab, int max_pos, int pair_style, const kvattn_bf16* k_cache,
+                         const kvattn_bf16* v_cache, const int32_t* seq_lens, int B, int n_head,
+                         int n_kv_head, int head_dim, int T_max, float scale, kvattn_bf16* out,
+                         float* lse, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                         void* stream);
+
+/*
+ * Append the new token's key and value to the cache: "注意力机制进化史" (KV
+ * cache: the new k, v are concatenated to layer_past) with the key rotated at
+ * its own position first ("Agentic RL 入门3" §1.1: RoPE on k, not on v).
+ * k_new, v_new [B][n_kv_head][d] bf16; pos device int32 [B]: the slot the
+ * token takes, which is also its rotation position (normally the length before
+ * the append).  Writes k_cache[b][h][pos[b]] = RoPE(k_new[b][h], pos[b]) and
+ * v_cache[b][h][pos[b]] = v_new[b][h] for every KV head; nothing else in the
+ * caches changes.  The rotation is bit-identical to rope_apply_qk's.  A slot
+ * outside [0, T_max) or a position outside [0, max_pos) sets
+ * KVATTN_STATUS_BAD_POSITION and that sequence is left as it was.  The caller
+ * advances its lengths.  head_dim a multiple of 16, at most 256; all pointers
+ * 16-byte aligned.
+ */
+int kv_append_rope(const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int32_t* pos, int B,
+                   int n_kv_head, int head_dim, kvattn_bf16* k_cache, kvattn_bf16* v_cache, int T_max,
+                   const float* cos_tab, const float* sin_tab, int max_pos, int pair_style,
+                   int32_t* dev_status, void* stream);
+
+/*
  * attn_decode_gqa for callers that cannot allocate device memory.  The pages
  * have no counterpart to this entry point; it exists for callers that cannot
  * give the library a workspace: code running inside another runtime's fixed

@@ -252,34 +252,49 @@ size_t attn_decode_gqa_workspace_bytes(int B, int n_head, int n_kv_head, int hea
     return decode_ws(B, n_head, n_kv_head, head_dim, kvattn::decode_grid(sms)).total;
 }
 
-int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
-                    const int32_t* seq_lens, int B, int n_head, int n_kv_head, int head_dim, int T_max, float scale,
-                    kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                    void* stream)
+// Shared by attn_decode_gqa (rope == nullptr) and attn_decode_gqa_rope.
+struct DecodeRope {
+    const int32_t* q_pos;
+    const float* cos_tab;
+    const float* sin_tab;
+    int max_pos, pair_style;
+};
+
+static int decode_call(const char* name, const kvattn_bf16* q, const kvattn_bf16* k_cache,
+                       const kvattn_bf16* v_cache, const int32_t* seq_lens, int B, int n_head, int n_kv_head,
+                       int head_dim, int T_max, float scale, kvattn_bf16* out, float* lse, void* workspace,
+                       size_t workspace_bytes, int32_t* dev_status, void* stream, const DecodeRope* rope)
 {
     if (!q || !k_cache || !v_cache || !seq_lens || !out)
-        return fail(KVATTN_ERR_NULL, "attn_decode_gqa: NULL argument");
-    if (B < 1 || B > kvattn::DECODE_MAX_B) return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: B %d outside 1..%d", B, kvattn::DECODE_MAX_B);
+        return fail(KVATTN_ERR_NULL, "%s: NULL argument", name);
+    if (B < 1 || B > kvattn::DECODE_MAX_B) return fail(KVATTN_ERR_SHAPE, "%s: B %d outside 1..%d", name, B, kvattn::DECODE_MAX_B);
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head)
-        return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: n_head %d not a multiple of n_kv_head %d", n_head, n_kv_head);
+        return fail(KVATTN_ERR_SHAPE, "%s: n_head %d not a multiple of n_kv_head %d", name, n_head, n_kv_head);
     const int g = n_head / n_kv_head;
-    if (!g_supported(g)) return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: group size %d", g);
-    if (head_dim != 64 && head_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: head_dim %d", head_dim);
-    if (T_max < 1) return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: T_max %d", T_max);
+    if (!g_supported(g)) return fail(KVATTN_ERR_UNSUPPORTED, "%s: group size %d", name, g);
+    if (head_dim != 64 && head_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "%s: head_dim %d", name, head_dim);
+    if (T_max < 1) return fail(KVATTN_ERR_SHAPE, "%s: T_max %d", name, T_max);
     if (static_cast<long long>(B) * n_kv_head > KVATTN_DECODE_WS_ZERO_BYTES / 4)
-        return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_gqa: B * n_kv_head = %lld above %u",
+        return fail(KVATTN_ERR_UNSUPPORTED, "%s: B * n_kv_head = %lld above %u", name,
                     static_cast<long long>(B) * n_kv_head, KVATTN_DECODE_WS_ZERO_BYTES / 4);
-    if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa: scale must be finite > 0");
+    if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(KVATTN_ERR_SHAPE, "%s: scale must be finite > 0", name);
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
-        return fail(KVATTN_ERR_ALIGN, "attn_decode_gqa: tensors must be 16-byte aligned");
+        return fail(KVATTN_ERR_ALIGN, "%s: tensors must be 16-byte aligned", name);
+    if (rope) {
+        if (!rope->q_pos || !rope->cos_tab || !rope->sin_tab) return fail(KVATTN_ERR_NULL, "%s: NULL RoPE argument", name);
+        if (rope->pair_style != 0 && rope->pair_style != 1) return fail(KVATTN_ERR_UNSUPPORTED, "%s: pair_style", name);
+        if (rope->max_pos < 1) return fail(KVATTN_ERR_SHAPE, "%s: max_pos < 1", name);
+        if (!aligned16(rope->cos_tab) || !aligned16(rope->sin_tab))
+            return fail(KVATTN_ERR_ALIGN, "%s: tables must be 16-byte aligned", name);
+    }
     int sms = 0;
-    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "attn_decode_gqa: no CUDA device");
+    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "%s: no CUDA device", name);
     const int grid = kvattn::decode_grid(sms);
     const DecodeWs ws = decode_ws(B, n_head, n_kv_head, head_dim, grid);
     if (!workspace || workspace_bytes < ws.total)
-        return fail(KVATTN_ERR_WORKSPACE, "attn_decode_gqa: workspace needs %zu bytes", ws.total);
+        return fail(KVATTN_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, ws.total);
     if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
-        return fail(KVATTN_ERR_ALIGN, "attn_decode_gqa: workspace must be 256-byte aligned");
+        return fail(KVATTN_ERR_ALIGN, "%s: workspace must be 256-byte aligned", name);
 
     CUtensorMap tm_q, tm_k, tm_v;
     const uint64_t units = static_cast<uint64_t>(B) * n_kv_head;
@@ -301,6 +316,13 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
     a.unit_info = reinterpret_cast<int2*>(w + ws.off_info);
     a.unit_cnt = reinterpret_cast<int*>(w);
     a.dev_status = dev_status;
+    if (rope) {
+        a.q_pos = rope->q_pos;
+        a.cos_tab = rope->cos_tab;
+        a.sin_tab = rope->sin_tab;
+        a.max_pos = rope->max_pos;
+        a.pair_style = rope->pair_style;
+    }
     a.B = B;
     a.H = n_head;
     a.Hk = n_kv_head;
@@ -310,7 +332,48 @@ int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvat
     a.scale = scale;
     a.grid = grid;
     return cuda_status(kvattn::launch_decode(a, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
-                       "attn_decode_gqa launch");
+                       name);
+}
+
+int attn_decode_gqa(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
+                    const int32_t* seq_lens, int B, int n_head, int n_kv_head, int head_dim, int T_max, float scale,
+                    kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                    void* stream)
+{
+    return decode_call("attn_decode_gqa", q, k_cache, v_cache, seq_lens, B, n_head, n_kv_head, head_dim, T_max,
+                       scale, out, lse, workspace, workspace_bytes, dev_status, stream, nullptr);
+}
+
+int attn_decode_gqa_rope(const kvattn_bf16* q, const int32_t* q_pos, const float* cos_tab, const float* sin_tab,
+                         int max_pos, int pair_style, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
+                         const int32_t* seq_lens, int B, int n_head, int n_kv_head, int head_dim, int T_max,
+                         float scale, kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, void* stream)
+{
+    const DecodeRope r{q_pos, cos_tab, sin_tab, max_pos, pair_style};
+    return decode_call("attn_decode_gqa_rope", q, k_cache, v_cache, seq_lens, B, n_head, n_kv_head, head_dim,
+                       T_max, scale, out, lse, workspace, workspace_bytes, dev_status, stream, &r);
+}
+
+// ---------------------------------------------------------------------------
+int kv_append_rope(const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int32_t* pos, int B, int n_kv_head,
+                   int head_dim, kvattn_bf16* k_cache, kvattn_bf16* v_cache, int T_max, const float* cos_tab,
+                   const float* sin_tab, int max_pos, int pair_style, int32_t* dev_status, void* stream)
+{
+    if (!k_new || !v_new || !pos || !k_cache || !v_cache || !cos_tab || !sin_tab)
+        return fail(KVATTN_ERR_NULL, "kv_append_rope: NULL argument");
+    if (B < 1 || n_kv_head < 1 || T_max < 1 || max_pos < 1)
+        return fail(KVATTN_ERR_SHAPE, "kv_append_rope: B %d, n_kv_head %d, T_max %d, max_pos %d", B, n_kv_head, T_max,
+                    max_pos);
+    if (head_dim < 16 || head_dim > 256 || head_dim % 16)
+        return fail(KVATTN_ERR_UNSUPPORTED, "kv_append_rope: head_dim %d must be a multiple of 16, <= 256", head_dim);
+    if (pair_style != 0 && pair_style != 1) return fail(KVATTN_ERR_UNSUPPORTED, "kv_append_rope: pair_style");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(cos_tab) ||
+        !aligned16(sin_tab))
+        return fail(KVATTN_ERR_ALIGN, "kv_append_rope: tensors must be 16-byte aligned");
+    kvattn::KvAppendArgs a{k_new, v_new, pos, k_cache, v_cache, cos_tab, sin_tab, B, n_kv_head, head_dim, T_max,
+                           max_pos, pair_style, dev_status};
+    return cuda_status(kvattn::launch_kv_append(a, static_cast<cudaStream_t>(stream)), "kv_append_rope launch");
 }
 
 // ---------------------------------------------------------------------------

@@ -431,6 +431,45 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
 
+// One RoPE pair rotation (a, b) -> (a cos - b sin, a sin + b cos) in fp32 with the
+// operations spelled out (no contraction left to the compiler), so that every
+// kernel that rotates -- in place, fused into decode, or on append -- produces
+// the same bits.
+__device__ __forceinline__ float2 rope_pair(float a, float b, float c, float s)
+{
+    return make_float2(__fmaf_rn(a, c, -__fmul_rn(b, s)), __fmaf_rn(a, s, __fmul_rn(b, c)));
+}
+
+// Rotate 8 bf16 elements (four packed pairs) of an adjacent-pair vector chunk:
+// pairs (2j, 2j+1) of the chunk with table entries c[j], s[j].
+__device__ __forceinline__ uint4 rope_chunk_adjacent(uint4 raw, const float (&c)[4], const float (&s)[4])
+{
+    uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 r = rope_pair(bf16_lo(w[j]), bf16_hi(w[j]), c[j], s[j]);
+        w[j] = pack_bf16x2(r.x, r.y);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Rotate two 8-element chunks of a half-split vector: element j of chunk `ra`
+// pairs with element j of chunk `rb` (d/2 further on), table entries c[j], s[j].
+__device__ __forceinline__ void rope_chunk_half(uint4& ra, uint4& rb, const float (&c)[8], const float (&s)[8])
+{
+    uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+    uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 r0 = rope_pair(bf16_lo(wa[j]), bf16_lo(wb[j]), c[2 * j], s[2 * j]);
+        const float2 r1 = rope_pair(bf16_hi(wa[j]), bf16_hi(wb[j]), c[2 * j + 1], s[2 * j + 1]);
+        wa[j] = pack_bf16x2(r0.x, r1.x);
+        wb[j] = pack_bf16x2(r0.y, r1.y);
+    }
+    ra = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+    rb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a TMA
 // SWIZZLE_128B tile whose rows are 128 bytes: chunk index XOR (row mod 8).
 __device__ __forceinline__ uint32_t swz128(int row, int chunk)

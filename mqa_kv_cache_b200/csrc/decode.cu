@@ -49,7 +49,9 @@ struct Cfg {
     static constexpr int OFF_SCR_ML = OFF_SCR_O + CWARPS * 16 * SCR_STRIDE * 4;
     static constexpr int OFF_Q = OFF_SCR_ML + CWARPS * 16 * 2 * 4;  // q rows of the next piece
     static constexpr int Q_BYTES = NMT * 16 * D * 2;
-    static constexpr int OFF_N = OFF_Q + Q_BYTES;
+    static constexpr int OFF_CS = OFF_Q + Q_BYTES;                   // cos row | sin row of its position
+    static constexpr int OFF_QPOS = OFF_CS + 2 * (D / 2) * 4;        // [DECODE_MAX_B] query positions
+    static constexpr int OFF_N = OFF_QPOS + DECODE_MAX_B * 4;
     static constexpr int OFF_UB = OFF_N + DECODE_MAX_B * 4;
     static constexpr int OFF_LEN = OFF_UB + (DECODE_MAX_B + 1) * 4;
     static constexpr int OFF_BAR = ((OFF_LEN + DECODE_MAX_B * 4) + 7) / 8 * 8;
@@ -61,6 +63,42 @@ struct Cfg {
 __device__ __forceinline__ uint32_t ld_u32(const kvattn_bf16* p)
 {
     return *reinterpret_cast<const uint32_t*>(p);
+}
+
+// ---- RoPE of query rows held in shared memory ------------------------------------
+// rows [rows][D] bf16, contiguous; cos/sin rows of D/2 entries.  nthr threads each
+// take 8-element chunks (adjacent pairs) or pairs of chunks d/2 apart (half-split).
+__device__ __forceinline__ void rope_rows_smem(uint8_t* rows, int nrows, int D, const float* cs, const float* sn,
+                                               int pair_style, int tid, int nthr)
+{
+    __nv_bfloat16* q = reinterpret_cast<__nv_bfloat16*>(rows);
+    if (pair_style == 0) {
+        const int per = D / 8;
+        for (int i = tid; i < nrows * per; i += nthr) {
+            const int r = i / per, ch = i - r * per;
+            const float cc[4] = {cs[4 * ch], cs[4 * ch + 1], cs[4 * ch + 2], cs[4 * ch + 3]};
+            const float ss[4] = {sn[4 * ch], sn[4 * ch + 1], sn[4 * ch + 2], sn[4 * ch + 3]};
+            uint4* p = reinterpret_cast<uint4*>(q + r * D + ch * 8);
+            *p = rope_chunk_adjacent(*p, cc, ss);
+        }
+    } else {
+        const int per = D / 16, half = D / 2;
+        for (int i = tid; i < nrows * per; i += nthr) {
+            const int r = i / per, ch = i - r * per;
+            float cc[8], ss[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                cc[j] = cs[8 * ch + j];
+                ss[j] = sn[8 * ch + j];
+            }
+            uint4* pa = reinterpret_cast<uint4*>(q + r * D + ch * 8);
+            uint4* pb = reinterpret_cast<uint4*>(q + r * D + half + ch * 8);
+            uint4 ra = *pa, rb = *pb;
+            rope_chunk_half(ra, rb, cc, ss);
+            *pa = ra;
+            *pb = rb;
+        }
+    }
 }
 
 // ---- merge of a split unit ------------------------------------------------------
@@ -151,6 +189,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint64_t* q_full = empty + C::STAGES;
     uint64_t* q_empty = q_full + 1;
     uint8_t* sQ = smem + C::OFF_Q;
+    float* sCos = reinterpret_cast<float*>(smem + C::OFF_CS);
+    float* sSin = sCos + D / 2;
+    int* s_qpos = reinterpret_cast<int*>(smem + C::OFF_QPOS);
+    const bool rope = a.cos_tab != nullptr;
     int* s_misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     volatile int* s_abort = s_misc + 1;
     int* s_merge = s_misc + 4;  // [0] = split pieces made here, then (unit, first slot, pieces) x 2
@@ -175,7 +217,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     pdl_wait();
     pdl_trigger();
     const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
-                                    blockIdx.x == 0);
+                                    blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos);
     // empty sequences have no tiles: their heads get zeros and lse = -inf here
     for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
         if (s_len[b] != 0) continue;
@@ -212,9 +254,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 ok = false;
                 break;
             }
-            mbar_arrive_expect_tx(q_full, q_bytes);
+            // with RoPE, the cos and sin rows of the query's position come along
+            const int qp = rope ? s_qpos[w.b] : -1;
+            const bool rot = rope && qp >= 0 && qp < a.max_pos;
+            mbar_arrive_expect_tx(q_full, q_bytes + (rot ? D * 4 : 0));
             bulk_load(sQ, a.q + (static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g) * D, q_bytes,
                       q_full);
+            if (rot) {
+                bulk_load(sCos, a.cos_tab + static_cast<long long>(qp) * (D / 2), D * 2, q_full);
+                bulk_load(sSin, a.sin_tab + static_cast<long long>(qp) * (D / 2), D * 2, q_full);
+            }
             ++np;
             for (long long t = tb; t < te; ++t, ++it) {
                 const int s = it % C::STAGES;
@@ -270,6 +319,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         {
             const bool have_q = warp_wait(q_full, piece & 1, s_abort);
             const uint8_t* qg = sQ;
+            if (rope) {
+                // rotate the piece's g query rows in place (bad positions: flagged, left as given)
+                const int qp = s_qpos[w.b];
+                if (qp >= 0 && qp < a.max_pos) {
+                    if (have_q) rope_rows_smem(sQ, g, D, sCos, sSin, a.pair_style, ctid, CWARPS * 32);
+                } else if (ctid == 0 && c == unit_first_owner(w.U, N, G)) {
+                    report_status(a.dev_status, KVATTN_STATUS_BAD_POSITION);
+                }
+                // the rows are read below, and rewritten by the next bulk copy after q_empty
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                named_bar_sync(1, CWARPS * 32);
+            }
             const int ra = mt * 16 + r0, rb = ra + 8;
             const bool va = have_q && ra < g, vb = have_q && rb < g;
 #pragma unroll
@@ -623,8 +684,8 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q, const CU
     const int nmt = a.g <= 16 ? 1 : (a.g <= 32 ? 2 : 4);
     if (a.d == 128) {
         if (nmt == 1) return launch_typed<128, 1>(a, tm_k, tm_v, stream);
-        if (nmt == 2) return launch_typed<128, 2>(a, tm_k, tm_v, stream);
-        return launch_typed<128, 4>(a, tm_k, tm_v, stream);
+        // g = 64 at d = 128 is the tcgen05 kernel's
+        return launch_typed<128, 2>(a, tm_k, tm_v, stream);
     }
     if (nmt == 1) return launch_typed<64, 1>(a, tm_k, tm_v, stream);
     if (nmt == 2) return launch_typed<64, 2>(a, tm_k, tm_v, stream);

@@ -48,12 +48,14 @@ constexpr int TC_OFF_K = 0;
 constexpr int TC_OFF_V = TC_OFF_K + TC_KS * TC_TILE;
 constexpr int TC_OFF_Q = TC_OFF_V + TC_VS * TC_TILE;
 constexpr int TC_OFF_P = TC_OFF_Q + 2 * TC_QBOX;                  // TC_NB P tiles
-constexpr int TC_OFF_N = TC_OFF_P + TC_NB * TC_PBYTES;
+constexpr int TC_OFF_CS = TC_OFF_P + TC_NB * TC_PBYTES;          // cos row | sin row of the query position
+constexpr int TC_OFF_QPOS = TC_OFF_CS + 2 * (TC_D / 2) * 4;       // [DECODE_MAX_B] query positions
+constexpr int TC_OFF_N = TC_OFF_QPOS + DECODE_MAX_B * 4;
 constexpr int TC_OFF_UB = TC_OFF_N + DECODE_MAX_B * 4;
 constexpr int TC_OFF_LEN = TC_OFF_UB + (DECODE_MAX_B + 1) * 4;
 constexpr int TC_OFF_BAR = (TC_OFF_LEN + DECODE_MAX_B * 4 + 7) / 8 * 8;
 // kfull[KS], kempty[KS], vfull[VS], vempty[VS], q_full, q_empty, s_full[NB], p_full[NB], pv_done[NB], done[2]
-constexpr int TC_NBAR = 2 * TC_KS + 2 * TC_VS + 2 + 3 * TC_NB + 2;
+constexpr int TC_NBAR = 2 * TC_KS + 2 * TC_VS + 2 + 3 * TC_NB + 2 + 1;  // + q_rot
 constexpr int TC_OFF_MISC = TC_OFF_BAR + TC_NBAR * 8;
 constexpr int TC_SMEM = TC_OFF_MISC + 32 + 1024;
 static_assert(TC_SMEM <= 232448, "shared memory");
@@ -83,6 +85,42 @@ struct TileStream {
     }
 };
 
+// RoPE of the 64 query rows of a piece in place, in their two 128-byte-swizzled
+// boxes (box k: dims 64k .. 64k+63, row h at h * 128 bytes, 16-byte chunk j of a
+// row at ((j ^ (h & 7)) << 4)).  nthr threads take chunks.
+__device__ __forceinline__ void rope_q_swizzled(uint8_t* q, const float* cs, const float* sn, int pair_style,
+                                                int tid, int nthr)
+{
+    if (pair_style == 0) {
+        // chunk (box k, j) holds pairs 32k + 4j .. 32k + 4j + 3
+        for (int i = tid; i < TC_M * 16; i += nthr) {
+            const int h = i >> 4, k = (i >> 3) & 1, j = i & 7;
+            const int p0 = 32 * k + 4 * j;
+            const float cc[4] = {cs[p0], cs[p0 + 1], cs[p0 + 2], cs[p0 + 3]};
+            const float ss[4] = {sn[p0], sn[p0 + 1], sn[p0 + 2], sn[p0 + 3]};
+            uint4* p = reinterpret_cast<uint4*>(q + k * TC_QBOX + swz128(h, j));
+            *p = rope_chunk_adjacent(*p, cc, ss);
+        }
+    } else {
+        // element e of chunk j in box 0 pairs with the same element in box 1: pair 8j + e
+        for (int i = tid; i < TC_M * 8; i += nthr) {
+            const int h = i >> 3, j = i & 7;
+            float cc[8], ss[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                cc[e] = cs[8 * j + e];
+                ss[e] = sn[8 * j + e];
+            }
+            uint4* pa = reinterpret_cast<uint4*>(q + swz128(h, j));
+            uint4* pb = reinterpret_cast<uint4*>(q + TC_QBOX + swz128(h, j));
+            uint4 ra = *pa, rb = *pb;
+            rope_chunk_half(ra, rb, cc, ss);
+            *pa = ra;
+            *pb = rb;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(TC_THREADS, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, DecodeArgs a)
@@ -106,6 +144,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint64_t* p_full = s_full + TC_NB;           // [NB]: P of tile i ready (S buffer i % NB read)
     uint64_t* pv_done = p_full + TC_NB;          // [NB]: P V of tile i finished (P buffer free, O updated)
     uint64_t* done = pv_done + TC_NB;            // [2]: all S MMAs / all P V MMAs finished
+    uint64_t* q_rot = done + 2;                  // with RoPE: the piece's Q rows rotated (4 warps)
+    float* sCos = reinterpret_cast<float*>(smem + TC_OFF_CS);
+    float* sSin = sCos + TC_D / 2;
+    int* s_qpos = reinterpret_cast<int*>(smem + TC_OFF_QPOS);
+    const bool rope = a.cos_tab != nullptr;
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + TC_OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + TC_OFF_MISC + 4);
     int* s_acc = reinterpret_cast<int*>(smem + TC_OFF_MISC + 8);
@@ -122,6 +165,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
+        mbar_init(q_rot, 4);
         for (int x = 0; x < TC_NB; ++x) {
             mbar_init(&s_full[x], 1);
             mbar_init(&p_full[x], 4);
@@ -148,7 +192,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     pdl_trigger();
 
     const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
-                                    blockIdx.x == 0);
+                                    blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos);
     const int G = static_cast<int>(N < a.grid ? N : a.grid), c = blockIdx.x;
     const bool active = N > 0 && c < G;
     long long lo = 0, hi = 0;
@@ -177,9 +221,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     ok = false;
                     break;
                 }
-                mbar_arrive_expect_tx(q_full, 2 * TC_QBOX);
+                // with RoPE, the cos and sin rows of the query's position come along
+                const int qp = rope ? s_qpos[w.b] : -1;
+                const bool rot = rope && qp >= 0 && qp < a.max_pos;
+                mbar_arrive_expect_tx(q_full, 2 * TC_QBOX + (rot ? TC_D * 4 : 0));
                 tma_load_3d(smem + TC_OFF_Q, &tm_q, q_full, 0, 0, z);
                 tma_load_3d(smem + TC_OFF_Q + TC_QBOX, &tm_q, q_full, 64, 0, z);
+                if (rot) {
+                    bulk_load(sCos, a.cos_tab + static_cast<long long>(qp) * (TC_D / 2), TC_D * 2, q_full);
+                    bulk_load(sSin, a.sin_tab + static_cast<long long>(qp) * (TC_D / 2), TC_D * 2, q_full);
+                }
                 for (long long t = tb; t < te; ++t, ++it) {
                     const int ks = it % TC_KS, vs = it % TC_VS;
                     const int row = static_cast<int>(t * TC_T);
@@ -220,7 +271,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int i = 0; ok && ts.next(lo, hi, a.B, a.Hk, s_n, N, G, first); ++i) {
                 if (ts.piece != piece_s) {
                     if (piece_s >= 0) tc_commit(q_empty);  // every S of the previous piece is issued
-                    if (!(ok = mbar_wait(q_full, ts.piece & 1))) break;
+                    // the piece's Q has landed (and, with RoPE, been rotated by the softmax warps)
+                    if (!(ok = mbar_wait(rope ? q_rot : q_full, ts.piece & 1))) break;
                     piece_s = ts.piece;
                 }
                 const int ks = i % TC_KS;
@@ -289,7 +341,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const float2 sc2 = make_float2(sl2, sl2);
         uint8_t* sP0 = smem + TC_OFF_P;
         Walk w = w_start;
-        int i = 0;
+        int i = 0, pc = 0;
         for (; w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
             const int n = s_n[w.b];
             const int len = s_len[w.b];
@@ -297,6 +349,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             if (!piece_tiles(w, n, lo, hi, tb, te)) continue;
             const int count = unit_count(w.U, n, N, G);
             const int slot = w.S + (c - unit_first_owner(w.U, N, G));
+            if (rope) {
+                // rotate the piece's 64 Q rows in their swizzled boxes, then release the S MMAs
+                // (bad positions: flagged, Q left as given)
+                const int qp = s_qpos[w.b];
+                if (warp_wait(q_full, pc & 1, s_abort)) {
+                    if (qp >= 0 && qp < a.max_pos)
+                        rope_q_swizzled(smem + TC_OFF_Q, sCos, sSin, a.pair_style, (warp - 2) * 32 + lane, 128);
+                    else if (tb == 0 && warp == 2 && lane == 0)
+                        report_status(a.dev_status, KVATTN_STATUS_BAD_POSITION);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_rot);
+            }
+            ++pc;
             float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of h0, h1
             float2 l2 = make_float2(0.f, 0.f);      // this thread's share of their sums
             for (long long t = tb; t < te; ++t, ++i) {

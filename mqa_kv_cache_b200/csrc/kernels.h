@@ -54,6 +54,19 @@ struct RopeApplyArgs {
 };
 cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t stream);
 
+struct KvAppendArgs {
+    const kvattn_bf16* k_new;  // [B][Hk][d]
+    const kvattn_bf16* v_new;  // [B][Hk][d]
+    const int32_t* pos;        // [B] cache slot = rotation position
+    kvattn_bf16* k_cache;      // [B][Hk][T_max][d]
+    kvattn_bf16* v_cache;
+    const float* cos_tab;
+    const float* sin_tab;
+    int B, Hk, head_dim, T_max, max_pos, pair_style;
+    int32_t* dev_status;
+};
+cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t stream);
+
 // ---- split-K decode ----
 constexpr int DECODE_MAX_B = 1024;
 
@@ -66,6 +79,11 @@ struct DecodeArgs {
     float* part_ml;  // [slots][g][2]  (running max in log2 units, sum of exponentials)
     int2* unit_info; // [B*Hk]         (first slot, number of pieces) of every non-empty unit
     int* unit_cnt;   // [B*Hk]         pieces of a split unit finished so far (zero between calls)
+    // RoPE of the queries inside the kernel (cos_tab null: q is used as given)
+    const int32_t* q_pos;  // [B] position of each sequence's query
+    const float* cos_tab;  // [max_pos][d/2]
+    const float* sin_tab;
+    int max_pos, pair_style;
     int32_t* dev_status;
     int B, H, Hk, g, d, T_max;
     float scale;

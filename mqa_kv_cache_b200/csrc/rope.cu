@@ -66,47 +66,36 @@ struct RopeView {
     long long sb, st, sh;
 };
 
-// Rotate one 8-element chunk pair-wise with table row `m`.
+// Rotate one 8-element chunk (adjacent pairs) or one pair of 8-element chunks
+// (half-split pairs) of vector `src` with table row cos_row / sin_row into `vec`
+// (the same vector for an in-place rotation).
 template <int PAIR_STYLE>
 __device__ __forceinline__ void rotate_chunk(__nv_bfloat16* vec, int chunk, int half, const float* cos_row,
-                                             const float* sin_row)
+                                             const float* sin_row, const __nv_bfloat16* src = nullptr)
 {
+    if (!src) src = vec;
     if (PAIR_STYLE == 0) {
         // elements 8c .. 8c+7 = pairs 4c .. 4c+3
-        uint4 raw = *reinterpret_cast<const uint4*>(vec + chunk * 8);
         const float4 c = *reinterpret_cast<const float4*>(cos_row + chunk * 4);
         const float4 s = *reinterpret_cast<const float4*>(sin_row + chunk * 4);
-        uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-        const float cc[4] = {c.x, c.y, c.z, c.w};
-        const float ss[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float a = bf16_lo(w[j]), b = bf16_hi(w[j]);
-            w[j] = pack_bf16x2(a * cc[j] - b * ss[j], a * ss[j] + b * cc[j]);
-        }
-        *reinterpret_cast<uint4*>(vec + chunk * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {s.x, s.y, s.z, s.w};
+        *reinterpret_cast<uint4*>(vec + chunk * 8) =
+            rope_chunk_adjacent(*reinterpret_cast<const uint4*>(src + chunk * 8), cc, ss);
     } else {
         // element 8c + j pairs with 8c + j + d/2; pair index 8c + j
-        uint4 ra = *reinterpret_cast<const uint4*>(vec + chunk * 8);
-        uint4 rb = *reinterpret_cast<const uint4*>(vec + half + chunk * 8);
+        uint4* pa = reinterpret_cast<uint4*>(vec + chunk * 8);
+        uint4* pb = reinterpret_cast<uint4*>(vec + half + chunk * 8);
         const float4 c0 = *reinterpret_cast<const float4*>(cos_row + chunk * 8);
         const float4 c1 = *reinterpret_cast<const float4*>(cos_row + chunk * 8 + 4);
         const float4 s0 = *reinterpret_cast<const float4*>(sin_row + chunk * 8);
         const float4 s1 = *reinterpret_cast<const float4*>(sin_row + chunk * 8 + 4);
-        uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
-        uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
         const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
         const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float a0 = bf16_lo(wa[j]), a1 = bf16_hi(wa[j]);
-            const float b0 = bf16_lo(wb[j]), b1 = bf16_hi(wb[j]);
-            const int i0 = 2 * j, i1 = 2 * j + 1;
-            wa[j] = pack_bf16x2(a0 * cc[i0] - b0 * ss[i0], a1 * cc[i1] - b1 * ss[i1]);
-            wb[j] = pack_bf16x2(a0 * ss[i0] + b0 * cc[i0], a1 * ss[i1] + b1 * cc[i1]);
-        }
-        *reinterpret_cast<uint4*>(vec + chunk * 8) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-        *reinterpret_cast<uint4*>(vec + half + chunk * 8) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+        uint4 ra = *reinterpret_cast<const uint4*>(src + chunk * 8);
+        uint4 rb = *reinterpret_cast<const uint4*>(src + half + chunk * 8);
+        rope_chunk_half(ra, rb, cc, ss);
+        *pa = ra;
+        *pb = rb;
     }
 }
 
@@ -145,6 +134,40 @@ __global__ void rope_apply_kernel(RopeView qv, RopeView kv, const float* __restr
     }
 }
 
+// New token's k rotated at its position into cache slot pos[b], v copied there.
+// One thread per 8-element chunk (adjacent pairs) or per pair of chunks
+// (half-split pairs) of every (batch, kv head) vector.
+template <int PAIR_STYLE>
+__global__ void kv_append_kernel(KvAppendArgs a)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int half = a.head_dim / 2;
+    const int per_vec = PAIR_STYLE == 0 ? a.head_dim / 8 : a.head_dim / 16;
+    const long long total = static_cast<long long>(a.B) * a.Hk * per_vec;
+    for (long long tid = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; tid < total;
+         tid += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long vec = tid / per_vec;  // b * Hk + h
+        const int chunk = static_cast<int>(tid - vec * per_vec);
+        const int b = static_cast<int>(vec / a.Hk);
+        const int m = a.pos[b];
+        if (m < 0 || m >= a.T_max || m >= a.max_pos) {
+            if (chunk == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_POSITION);
+            continue;
+        }
+        const long long row = (vec * a.T_max + m) * a.head_dim;
+        const __nv_bfloat16* kn = reinterpret_cast<const __nv_bfloat16*>(a.k_new) + vec * a.head_dim;
+        const __nv_bfloat16* vn = reinterpret_cast<const __nv_bfloat16*>(a.v_new) + vec * a.head_dim;
+        __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(a.k_cache) + row;
+        __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(a.v_cache) + row;
+        rotate_chunk<PAIR_STYLE>(kc, chunk, half, a.cos_tab + static_cast<long long>(m) * half,
+                                 a.sin_tab + static_cast<long long>(m) * half, kn);
+        *reinterpret_cast<uint4*>(vc + chunk * 8) = *reinterpret_cast<const uint4*>(vn + chunk * 8);
+        if (PAIR_STYLE == 1)
+            *reinterpret_cast<uint4*>(vc + half + chunk * 8) = *reinterpret_cast<const uint4*>(vn + half + chunk * 8);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_rope_table(const kvattn_rope_params& p, int max_pos, float* cos_out, float* sin_out,
@@ -176,6 +199,17 @@ cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t stream)
     auto kern = a.pair_style == 0 ? rope_apply_kernel<0> : rope_apply_kernel<1>;
     return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, qv, kv, a.cos_tab,
                       a.sin_tab, a.max_pos, a.head_dim, a.dev_status);
+}
+
+cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t stream)
+{
+    const int per_vec = a.pair_style == 0 ? a.head_dim / 8 : a.head_dim / 16;
+    const long long total = static_cast<long long>(a.B) * a.Hk * per_vec;
+    const int threads = 128;
+    long long blocks = (total + threads - 1) / threads;
+    if (blocks > 65535) blocks = 65535;
+    auto kern = a.pair_style == 0 ? kv_append_kernel<0> : kv_append_kernel<1>;
+    return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, a);
 }
 
 }  // namespace kvattn

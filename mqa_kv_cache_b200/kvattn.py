@@ -41,6 +41,9 @@ _lib.attn_decode_gqa_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32]
 _lib.attn_decode_gqa_workspace_bytes.restype = _sz
 _lib.attn_decode_gqa.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
                                  _vp, _vp]
+_lib.attn_decode_gqa_rope.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                      _f32, _vp, _vp, _vp, _sz, _vp, _vp]
+_lib.kv_append_rope.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp]
 _lib.attn_decode_gqa_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
                                          _vp]
 _lib.attn_prefill_causal.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]
@@ -191,6 +194,56 @@ def attn_decode_gqa(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, ws
                                 float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status),
                                 _stream()))
     return out, lse
+
+
+def attn_decode_gqa_rope(q, q_pos, cos, sin, k_cache, v_cache, seq_lens, scale, pair_style=0, out=None, lse=None,
+                         ws=None, dev_status=None, want_lse=True):
+    """attn_decode_gqa with the queries rotated inside the kernel: q [B, H, d] raw
+    (not modified), q_pos int32 [B] (or [B, 1]) their positions, cos/sin the
+    rope_table_build tables [max_pos, d/2]."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    for t, n in ((seq_lens, "seq_lens"), (q_pos, "q_pos")):
+        _need(t, torch.int32, n)
+        _contig(t, n)
+    _need(cos, torch.float32, "cos")
+    _need(sin, torch.float32, "sin")
+    B, H, d = q.shape
+    Bk, Hk, T_max, dk = k_cache.shape
+    if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seq_lens.numel() != B or q_pos.numel() != B:
+        raise ValueError("inconsistent decode shapes")
+    if cos.shape[1] * 2 != d or sin.shape != cos.shape:
+        raise ValueError("tables must be [max_pos, d/2]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    need = attn_decode_gqa_workspace_bytes(B, H, Hk, d, T_max)
+    if ws is None:
+        ws = workspace(need, q.device)
+    _check(_lib.attn_decode_gqa_rope(_ptr(q), _ptr(q_pos), _ptr(cos), _ptr(sin), cos.shape[0], pair_style,
+                                     _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), B, H, Hk, d, T_max, float(scale),
+                                     _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status), _stream()))
+    return out, lse
+
+
+def kv_append_rope(k_new, v_new, pos, k_cache, v_cache, cos, sin, pair_style=0, dev_status=None):
+    """Write RoPE(k_new) and v_new ([B, Hk, d]) into slot pos[b] (int32 [B]) of the
+    [B, Hk, T_max, d] caches."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    _need(pos, torch.int32, "pos")
+    _contig(pos, "pos")
+    _need(cos, torch.float32, "cos")
+    _need(sin, torch.float32, "sin")
+    B, Hk, d = k_new.shape
+    Bc, Hc, T_max, dc = k_cache.shape
+    if (Bc, Hc, dc) != (B, Hk, d) or v_cache.shape != k_cache.shape or v_new.shape != k_new.shape or pos.numel() != B:
+        raise ValueError("inconsistent append shapes")
+    _check(_lib.kv_append_rope(_ptr(k_new), _ptr(v_new), _ptr(pos), B, Hk, d, _ptr(k_cache), _ptr(v_cache), T_max,
+                               _ptr(cos), _ptr(sin), cos.shape[0], pair_style, _ptr(dev_status), _stream()))
 
 
 def attn_decode_gqa_noalloc(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, dev_status=None,
