@@ -288,6 +288,10 @@ struct TopkArgs {
 };
 
 constexpr int TK_SLICE_MAX = 16384;  // keys per CTA held in shared memory
+// Key i of the slice sits at word i + i / 16: a thread's run of 16 keys then
+// starts in its own bank, so the runs of a warp are read without conflicts.
+__device__ __forceinline__ int kpad(int i) { return i + (i >> 4); }
+constexpr int TK_SLICE_WORDS = TK_SLICE_MAX + TK_SLICE_MAX / 16;
 
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
 {
@@ -296,7 +300,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     const int row = blockIdx.x / TK_CL;
     const int tid = threadIdx.x;
 
-    extern __shared__ uint32_t s_keys[];  // this CTA's slice as keys (TK_SLICE_MAX at most)
+    extern __shared__ uint32_t s_keys[];  // this CTA's slice as keys (TK_SLICE_MAX at most), kpad layout
     __shared__ uint32_t hist[2048];
     __shared__ int s_warp[32];
     __shared__ uint32_t s_sel[2];    // threshold digit, keys still needed from it
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     if (tid == 0) s_nan = 0;
     bool nan = false;
     // keys of the slice -> shared memory (one read of the scores)
-    for (int i = tid; i < n_mine; i += TK_THREADS) s_keys[i] = score_key(sc[lo + i], nan);
+    for (int i = tid; i < n_mine; i += TK_THREADS) s_keys[kpad(i)] = score_key(sc[lo + i], nan);
     __syncthreads();
 
     // ---- radix select: the (k)-th largest key T, and how many keys equal to T to take ----
@@ -330,9 +334,14 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
             const int sh = shifts[p], nb = 1 << widths[p];
             for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
             __syncthreads();
-            for (int i = tid; i < n_mine; i += TK_THREADS) {
-                const uint32_t key = s_keys[i];
-                if ((key & known) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+            // scores bunch into few top digits: lanes with equal digits add once per warp
+            for (int base = 0; base < n_mine; base += TK_THREADS) {
+                const int i = base + tid;
+                const uint32_t key = i < n_mine ? s_keys[kpad(i)] : 0u;
+                const bool in = i < n_mine && (key & known) == prefix;
+                const uint32_t digit = in ? (key >> sh) & (nb - 1) : 0xffffffffu;
+                const uint32_t same = __match_any_sync(0xffffffffu, digit);
+                if (in && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[digit], static_cast<uint32_t>(__popc(same)));
             }
             cluster.sync();
             // every CTA sums the cluster's histograms and finds the digit itself:
@@ -370,7 +379,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     const int r0 = min(tid * run, n_mine), r1 = min(r0 + run, n_mine);
     int n_gt = 0, n_eq = 0;
     for (int i = r0; i < r1; ++i) {
-        const uint32_t key = s_keys[i];
+        const uint32_t key = s_keys[kpad(i)];
         n_gt += key > T;
         n_eq += key == T && T != 0u;
     }
@@ -399,7 +408,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     int pos = g_rank + min(e_rank, max(take_eq, 0));
     int32_t* out = a.out + static_cast<long long>(row) * a.k;
     for (int i = r0; i < r1; ++i) {
-        const uint32_t key = s_keys[i];
+        const uint32_t key = s_keys[kpad(i)];
         bool take = key > T;
         if (key == T && T != 0u) {
             take = e_rank < take_eq;
@@ -452,11 +461,12 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     if (e != cudaSuccess) return e;
 
     TopkArgs ta{a.scores, a.seq_lens, a.topk_idx, a.dev_status, a.L_max, a.k};
-    const size_t key_bytes = static_cast<size_t>((a.L_max + TK_CL - 1) / TK_CL) * sizeof(uint32_t);
+    const int slice_max = (a.L_max + TK_CL - 1) / TK_CL;
+    const size_t key_bytes = static_cast<size_t>(slice_max + (slice_max >> 4) + 1) * sizeof(uint32_t);
     static bool tk_attr[64] = {};
     if (dev < 64 && !tk_attr[dev]) {
         e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 TK_SLICE_MAX * static_cast<int>(sizeof(uint32_t)));
+                                 (TK_SLICE_WORDS + 1) * static_cast<int>(sizeof(uint32_t)));
         if (e != cudaSuccess) return e;
         tk_attr[dev] = true;
     }
