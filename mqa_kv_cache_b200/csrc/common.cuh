@@ -249,6 +249,15 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t tmem_d, uint64_t adesc, uin
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// After tmem_wait_ld: registers filled by an earlier tcgen05.ld may be read only
+// from here on.  The empty statement "redefines" them, so that the compiler cannot
+// move a read of them above the wait (it does not know that the load is async).
+template <int N>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[N])
+{
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 consecutive 32-bit columns of this thread's TMEM lane.

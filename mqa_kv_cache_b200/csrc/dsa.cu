@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     const int tid = threadIdx.x;
 
     extern __shared__ uint32_t s_keys[];  // this CTA's slice as keys (TK_SLICE_MAX at most), kpad layout
-    __shared__ uint32_t hist[2048];
+    __shared__ uint32_t hist2[2][2048];  // per-pass histograms, alternating (see below)
     __shared__ int s_warp[32];
     __shared__ uint32_t s_sel[2];    // threshold digit, keys still needed from it
     __shared__ int s_counts[2];      // this CTA's (#key > T, #key == T)
@@ -332,6 +332,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
         const int widths[3] = {11, 11, 10};
         for (int p = 0; p < 3; ++p) {
             const int sh = shifts[p], nb = 1 << widths[p];
+            // Pass p clears and fills buffer p & 1.  Buffer p & 1 was last read by the other CTAs in
+            // pass p - 2, before they reached pass p - 1's cluster barrier, which this CTA has passed:
+            // one cluster barrier per pass suffices.
+            uint32_t* hist = hist2[p & 1];
             for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
             __syncthreads();
             // scores bunch into few top digits: lanes with equal digits add once per warp
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
                 s_sel[0] = static_cast<uint32_t>(d1);
                 s_sel[1] = static_cast<uint32_t>(k_rem - before - c0);
             }
-            cluster.sync();  // every CTA has read every histogram before any is cleared
+            __syncthreads();  // s_sel is written
             prefix |= s_sel[0] << sh;
             k_rem = static_cast<int>(s_sel[1]);
             known |= static_cast<uint32_t>(nb - 1) << sh;

@@ -242,21 +242,26 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (!warp_wait(&s_full[t], j & 1, s_abort)) continue;
                 tc_fence_after();
                 const bool diag = j == n_tiles - 1;  // keys j*128 .. : the diagonal tile
-                // Pass 1: row max of the raw scores (scale > 0 commutes with the max),
-                // one 32-column chunk in registers at a time.
+                // Pass 1: row max of the raw scores (scale > 0 commutes with the max): the four
+                // 32-column loads are in flight together, one wait.
                 float mx = -INFINITY;
+                {
+                    uint32_t sv[4][32];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t sv[32];
-                    tmem_ld32(s_addr + c * 32, sv);
+                    for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sv[c]);
                     tmem_wait_ld();
-                    if (diag) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (c * 32 + i > row) sv[i] = 0xff800000u;  // -inf: key after the query
+                    for (int c = 0; c < 4; ++c) {
+                        tmem_regs_ready(sv[c]);
+                        if (diag) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (c * 32 + i > row) sv[c][i] = 0xff800000u;  // -inf: key after the query
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2)
+                            mx = fmax3(mx, __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
                     }
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(sv[i]), __uint_as_float(sv[i + 1]));
                 }
                 mx *= sl2;
                 // Move this row's reference max only when it grows by more than 2^8.
@@ -285,11 +290,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 float2 acc = make_float2(0.f, 0.f);
                 // Pass 2: p = 2^(s * scale * log2 e - m) -> bf16 P over the first 64 S
                 // columns (chunk c's P lands in columns 16c..16c+15, all already read).
+                // Chunk c + 1 is loaded while chunk c is processed.
+                uint32_t sb[2][32];
+                tmem_ld32(s_addr, sb[0]);
+                tmem_wait_ld();
+                tmem_regs_ready(sb[0]);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t sv[32];
-                    tmem_ld32(s_addr + c * 32, sv);
-                    tmem_wait_ld();
+                    uint32_t (&sv)[32] = sb[c & 1];
+                    if (c < 3) tmem_ld32(s_addr + (c + 1) * 32, sb[(c + 1) & 1]);
                     if (diag) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
@@ -318,6 +327,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]), "r"(pk[13]),
                         "r"(pk[14]), "r"(pk[15])
                         : "memory");
+                    if (c < 3) {
+                        tmem_wait_ld();
+                        tmem_regs_ready(sb[(c + 1) & 1]);
+                    }
                 }
                 const float ls = acc.x + acc.y;
                 l_run += ls;
