@@ -394,10 +394,11 @@ int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
         return fail(KVATTN_ERR_ALIGN, "attn_prefill_causal: tensors must be 16-byte aligned");
     CUtensorMap tm_q, tm_k, tm_v;
-    if (make_map_4d_rows(&tm_q, q, head_dim, n_head, T, B, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_4d_rows(&tm_q, q, head_dim, n_head, T, B, kvattn::PREFILL_Q_ROWS) != KVATTN_OK)
+        return KVATTN_ERR_CUDA;
     const uint64_t units = static_cast<uint64_t>(B) * n_kv_head;
-    if (make_map_3d(&tm_k, k, head_dim, T, units, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
-    if (make_map_3d(&tm_v, v, head_dim, T, units, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_3d(&tm_k, k, head_dim, T, units, kvattn::PREFILL_KV_ROWS) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_3d(&tm_v, v, head_dim, T, units, kvattn::PREFILL_KV_ROWS) != KVATTN_OK) return KVATTN_ERR_CUDA;
     kvattn::PrefillLaunch l{out, lse, nullptr, B, T, n_head, n_kv_head, scale};
     return cuda_status(kvattn::launch_prefill(l, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
                        "attn_prefill_causal launch");

@@ -133,6 +133,8 @@ size_t sparse_partial_bytes(int B, int Hq, int k);
 cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, cudaStream_t stream);
 
 // ---- causal prefill ----
+constexpr int PREFILL_Q_ROWS = 128;  // rows of a Q tile (box height of tm_q)
+constexpr int PREFILL_KV_ROWS = 128;  // keys of a K/V tile (box height of tm_k, tm_v)
 struct PrefillLaunch {
     kvattn_bf16* out;
     float* lse;

@@ -28,6 +28,7 @@ namespace {
 constexpr int PF_D = 128;     // head dim
 constexpr int PF_BM = 128;    // query rows per Q tile
 constexpr int PF_BN = 128;    // keys per K/V tile
+static_assert(PF_BM == PREFILL_Q_ROWS && PF_BN == PREFILL_KV_ROWS, "tensor map boxes");
 constexpr int PF_SLOTS = 4;   // K/V ring slots (one tile each)
 constexpr int PF_THREADS = 320;
 constexpr int PF_TILE = PF_BN * PF_D * 2;  // 32 KB: one K or V tile, two 64-column SW128 boxes
