@@ -419,10 +419,40 @@ def measure_dsa(K, device, steps, flush, peaks):
             "sparse_gathered_bytes": sp_bytes}
 
 
+def measure_window(K, device, steps, flush, peaks):
+    """Llama-3-8B-shaped decode at 32768 tokens over a rolling cache of 4 sinks +
+    a 4092-token window (attn_decode_gqa_rope_window): 4096 rows per KV head read."""
+    w = W.LLAMA3_8B_DECODE
+    n_sink, window, length = 4, 4092, 32768
+    cap = n_sink + window
+    gen = W.generator(W.SEED_BASE + w.index + 7, device)
+    q = W.normal_bf16((w.B, w.H, w.d), gen, device)
+    kc = W.normal_bf16((w.B, w.Hk, cap, w.d), gen, device)
+    vc = W.normal_bf16((w.B, w.Hk, cap, w.d), gen, device)
+    lens = torch.full((w.B,), length, dtype=torch.int32, device=device)
+    cos, sin = K.rope_table_build(K.rope_params(w.d, base=w.rope.base), length + 1, device=device)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H), dtype=torch.float32, device=device)
+    ws = K.workspace(K.attn_decode_gqa_workspace_bytes(w.B, w.H, w.Hk, w.d, cap), device)
+
+    def step():
+        K.attn_decode_gqa_rope_window(q, lens, cos, sin, kc, vc, lens, w.scale, n_sink, window, out=out, lse=lse, ws=ws)
+
+    ms = _graph_ms(step, steps, flush)
+    nbytes = w.B * w.Hk * cap * w.d * 2 * 2 + w.B * w.H * w.d * 2 * 2 + w.B * w.H * 4
+    return {"workload": f"llama3_8b_decode_B16_H32_Hk8_len{length}_sink{n_sink}_window{window}",
+            "ms_per_step": round(ms, 5), "algorithmic_bytes": nbytes,
+            "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "pct_of_hbm_peak": round(100 * nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 1),
+            "tok_per_s": round(w.B / (ms * 1e-3), 1)}
+
+
 def measure_others(K, device, steps, flush, peaks):
     res = {}
     for w in (W.TINY_GQA, W.LLAMA2_70B_GQA_32K, W.LLAMA2_70B_MQA_32K, W.LLAMA2_70B_MHA_32K):
         res[w.name] = measure_decode_config(K, w, device, steps, flush, peaks)
+    win = measure_window(K, device, steps, flush, peaks)
+    res[win["workload"]] = win
     res[W.PREFILL_8K.name] = measure_prefill(K, device, steps, flush, peaks)
     res[W.DSA_128K.name] = measure_dsa(K, device, steps, flush, peaks)
     torch.cuda.empty_cache()
@@ -538,7 +568,7 @@ def main():
     ap.add_argument("--impl", default="kvattn", choices=["kvattn", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", action="store_true", help="skip the other configurations")
-    ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "prefill", "dsa"],
+    ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "window", "prefill", "dsa"],
                     help="time one other configuration alone and print its JSON")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -564,6 +594,8 @@ def main():
             res = measure_decode_config(K, decode[args.only], device, args.steps, flush, peaks)
         elif args.only == "prefill":
             res = measure_prefill(K, device, args.steps, flush, peaks)
+        elif args.only == "window":
+            res = measure_window(K, device, args.steps, flush, peaks)
         else:
             res = measure_dsa(K, device, args.steps, flush, peaks)
         if rank == 0:

@@ -196,6 +196,37 @@ int kv_append_rope(const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int
                    const float* cos_tab, const float* sin_tab, int max_pos, int pair_style,
                    int32_t* dev_status, void* stream);
 
+/* ---- sliding window with attention sinks over a rolling cache ----------------
+ * "Agentic RL 入门3" §1 (sliding-window attention: a query sees the last w
+ * keys; the first s tokens kept as attention sinks), the band mask of the
+ * "attention" page: the query at position i sees keys j with i - w < j <= i
+ * and the s first tokens.  A rolling cache of capacity T_max >= n_sink + window
+ * rows per (batch, KV head) keeps the token at position p in slot p if
+ * p < n_sink, else in slot n_sink + (p - n_sink) mod window; after len tokens
+ * its first min(len, n_sink + window) slots hold tokens 0 .. n_sink-1 and the
+ * last window tokens (each key rotated at its own position, so slot order does
+ * not matter to attention).
+ *
+ * kv_append_rope_ring: kv_append_rope into that layout (pos[b] = the token's
+ * position; its slot follows from it).
+ * attn_decode_gqa_rope_window: attn_decode_gqa_rope over such a cache, with
+ * seq_lens[b] = tokens appended so far (any value >= 0, not limited by T_max):
+ * attention runs over the min(seq_lens[b], n_sink + window) filled slots.
+ * Both: n_sink >= 0, window >= 1, n_sink + window <= T_max; otherwise as their
+ * linear-cache counterparts.
+ */
+int kv_append_rope_ring(const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int32_t* pos, int n_sink,
+                        int window, int B, int n_kv_head, int head_dim, kvattn_bf16* k_cache,
+                        kvattn_bf16* v_cache, int T_max, const float* cos_tab, const float* sin_tab,
+                        int max_pos, int pair_style, int32_t* dev_status, void* stream);
+
+int attn_decode_gqa_rope_window(const kvattn_bf16* q, const int32_t* q_pos, const float* cos_tab,
+                                const float* sin_tab, int max_pos, int pair_style, const kvattn_bf16* k_cache,
+                                const kvattn_bf16* v_cache, const int32_t* seq_lens, int n_sink, int window,
+                                int B, int n_head, int n_kv_head, int head_dim, int T_max, float scale,
+                                kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, void* stream);
+
 /*
  * attn_decode_gqa for callers that cannot allocate device memory.  The pages
  * have no counterpart to this entry point; it exists for callers that cannot

@@ -263,7 +263,8 @@ struct DecodeRope {
 static int decode_call(const char* name, const kvattn_bf16* q, const kvattn_bf16* k_cache,
                        const kvattn_bf16* v_cache, const int32_t* seq_lens, int B, int n_head, int n_kv_head,
                        int head_dim, int T_max, float scale, kvattn_bf16* out, float* lse, void* workspace,
-                       size_t workspace_bytes, int32_t* dev_status, void* stream, const DecodeRope* rope)
+                       size_t workspace_bytes, int32_t* dev_status, void* stream, const DecodeRope* rope,
+                       int len_cap = 0)
 {
     if (!q || !k_cache || !v_cache || !seq_lens || !out)
         return fail(KVATTN_ERR_NULL, "%s: NULL argument", name);
@@ -316,6 +317,7 @@ static int decode_call(const char* name, const kvattn_bf16* q, const kvattn_bf16
     a.unit_info = reinterpret_cast<int2*>(w + ws.off_info);
     a.unit_cnt = reinterpret_cast<int*>(w);
     a.dev_status = dev_status;
+    a.len_cap = len_cap;
     if (rope) {
         a.q_pos = rope->q_pos;
         a.cos_tab = rope->cos_tab;
@@ -355,25 +357,61 @@ int attn_decode_gqa_rope(const kvattn_bf16* q, const int32_t* q_pos, const float
                        T_max, scale, out, lse, workspace, workspace_bytes, dev_status, stream, &r);
 }
 
+int attn_decode_gqa_rope_window(const kvattn_bf16* q, const int32_t* q_pos, const float* cos_tab,
+                                const float* sin_tab, int max_pos, int pair_style, const kvattn_bf16* k_cache,
+                                const kvattn_bf16* v_cache, const int32_t* seq_lens, int n_sink, int window, int B,
+                                int n_head, int n_kv_head, int head_dim, int T_max, float scale, kvattn_bf16* out,
+                                float* lse, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                                void* stream)
+{
+    if (n_sink < 0 || window < 1 || static_cast<long long>(n_sink) + window > T_max)
+        return fail(KVATTN_ERR_SHAPE, "attn_decode_gqa_rope_window: n_sink %d, window %d, capacity %d", n_sink, window,
+                    T_max);
+    const DecodeRope r{q_pos, cos_tab, sin_tab, max_pos, pair_style};
+    return decode_call("attn_decode_gqa_rope_window", q, k_cache, v_cache, seq_lens, B, n_head, n_kv_head, head_dim,
+                       T_max, scale, out, lse, workspace, workspace_bytes, dev_status, stream, &r, n_sink + window);
+}
+
+// ---------------------------------------------------------------------------
+static int kv_append_call(const char* name, const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int32_t* pos,
+                          int B, int n_kv_head, int head_dim, kvattn_bf16* k_cache, kvattn_bf16* v_cache, int T_max,
+                          const float* cos_tab, const float* sin_tab, int max_pos, int pair_style, int n_sink,
+                          int window, int32_t* dev_status, void* stream)
+{
+    if (!k_new || !v_new || !pos || !k_cache || !v_cache || !cos_tab || !sin_tab)
+        return fail(KVATTN_ERR_NULL, "%s: NULL argument", name);
+    if (B < 1 || n_kv_head < 1 || T_max < 1 || max_pos < 1)
+        return fail(KVATTN_ERR_SHAPE, "%s: B %d, n_kv_head %d, T_max %d, max_pos %d", name, B, n_kv_head, T_max,
+                    max_pos);
+    if (head_dim < 16 || head_dim > 256 || head_dim % 16)
+        return fail(KVATTN_ERR_UNSUPPORTED, "%s: head_dim %d must be a multiple of 16, <= 256", name, head_dim);
+    if (pair_style != 0 && pair_style != 1) return fail(KVATTN_ERR_UNSUPPORTED, "%s: pair_style", name);
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(cos_tab) ||
+        !aligned16(sin_tab))
+        return fail(KVATTN_ERR_ALIGN, "%s: tensors must be 16-byte aligned", name);
+    kvattn::KvAppendArgs a{k_new, v_new, pos, k_cache, v_cache, cos_tab, sin_tab, B, n_kv_head, head_dim, T_max,
+                           max_pos, pair_style, n_sink, window, dev_status};
+    return cuda_status(kvattn::launch_kv_append(a, static_cast<cudaStream_t>(stream)), name);
+}
+
+int kv_append_rope_ring(const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int32_t* pos, int n_sink,
+                        int window, int B, int n_kv_head, int head_dim, kvattn_bf16* k_cache, kvattn_bf16* v_cache,
+                        int T_max, const float* cos_tab, const float* sin_tab, int max_pos, int pair_style,
+                        int32_t* dev_status, void* stream)
+{
+    if (n_sink < 0 || window < 1 || static_cast<long long>(n_sink) + window > T_max)
+        return fail(KVATTN_ERR_SHAPE, "kv_append_rope_ring: n_sink %d, window %d, capacity %d", n_sink, window, T_max);
+    return kv_append_call("kv_append_rope_ring", k_new, v_new, pos, B, n_kv_head, head_dim, k_cache, v_cache, T_max,
+                          cos_tab, sin_tab, max_pos, pair_style, n_sink, window, dev_status, stream);
+}
+
 // ---------------------------------------------------------------------------
 int kv_append_rope(const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int32_t* pos, int B, int n_kv_head,
                    int head_dim, kvattn_bf16* k_cache, kvattn_bf16* v_cache, int T_max, const float* cos_tab,
                    const float* sin_tab, int max_pos, int pair_style, int32_t* dev_status, void* stream)
 {
-    if (!k_new || !v_new || !pos || !k_cache || !v_cache || !cos_tab || !sin_tab)
-        return fail(KVATTN_ERR_NULL, "kv_append_rope: NULL argument");
-    if (B < 1 || n_kv_head < 1 || T_max < 1 || max_pos < 1)
-        return fail(KVATTN_ERR_SHAPE, "kv_append_rope: B %d, n_kv_head %d, T_max %d, max_pos %d", B, n_kv_head, T_max,
-                    max_pos);
-    if (head_dim < 16 || head_dim > 256 || head_dim % 16)
-        return fail(KVATTN_ERR_UNSUPPORTED, "kv_append_rope: head_dim %d must be a multiple of 16, <= 256", head_dim);
-    if (pair_style != 0 && pair_style != 1) return fail(KVATTN_ERR_UNSUPPORTED, "kv_append_rope: pair_style");
-    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(cos_tab) ||
-        !aligned16(sin_tab))
-        return fail(KVATTN_ERR_ALIGN, "kv_append_rope: tensors must be 16-byte aligned");
-    kvattn::KvAppendArgs a{k_new, v_new, pos, k_cache, v_cache, cos_tab, sin_tab, B, n_kv_head, head_dim, T_max,
-                           max_pos, pair_style, dev_status};
-    return cuda_status(kvattn::launch_kv_append(a, static_cast<cudaStream_t>(stream)), "kv_append_rope launch");
+    return kv_append_call("kv_append_rope", k_new, v_new, pos, B, n_kv_head, head_dim, k_cache, v_cache, T_max,
+                          cos_tab, sin_tab, max_pos, pair_style, 0, 0, dev_status, stream);
 }
 
 // ---------------------------------------------------------------------------

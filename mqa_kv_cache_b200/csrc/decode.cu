@@ -217,7 +217,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     pdl_wait();
     pdl_trigger();
     const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
-                                    blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos);
+                                    blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos,
+                                    a.len_cap);
     // empty sequences have no tiles: their heads get zeros and lse = -inf here
     for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
         if (s_len[b] != 0) continue;
@@ -575,7 +576,7 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) decode_combine_kernel(Decode
     const int2 info = a.unit_info[u];
     const long long bh = static_cast<long long>(b) * a.H + static_cast<long long>(kvh) * g + row;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * D + lane * PL;
-    if (min(max(len_raw, 0), a.T_max) == 0) {
+    if (min(max(a.len_cap > 0 && len_raw > a.len_cap ? a.len_cap : len_raw, 0), a.T_max) == 0) {
 #pragma unroll
         for (int i = 0; i < PL; ++i) out[i] = __float2bfloat16_rn(0.f);
         if (lane == 0 && a.lse) a.lse[bh] = -INFINITY;

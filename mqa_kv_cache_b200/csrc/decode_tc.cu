@@ -192,7 +192,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     pdl_trigger();
 
     const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
-                                    blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos);
+                                    blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos,
+                                    a.len_cap);
     const int G = static_cast<int>(N < a.grid ? N : a.grid), c = blockIdx.x;
     const bool active = N > 0 && c < G;
     long long lo = 0, hi = 0;

@@ -63,6 +63,8 @@ struct KvAppendArgs {
     const float* cos_tab;
     const float* sin_tab;
     int B, Hk, head_dim, T_max, max_pos, pair_style;
+    int n_sink, window;        // window > 0: rolling cache, slot of position p >= n_sink is
+                               // n_sink + (p - n_sink) % window; window == 0: slot = position
     int32_t* dev_status;
 };
 cudaError_t launch_kv_append(const KvAppendArgs& a, cudaStream_t stream);
@@ -84,6 +86,8 @@ struct DecodeArgs {
     const float* cos_tab;  // [max_pos][d/2]
     const float* sin_tab;
     int max_pos, pair_style;
+    int len_cap;           // > 0: a sequence of length len uses min(len, len_cap) cache rows
+                           // (a rolling cache holding the sinks and the window)
     int32_t* dev_status;
     int B, H, Hk, g, d, T_max;
     float scale;

@@ -134,7 +134,8 @@ __global__ void rope_apply_kernel(RopeView qv, RopeView kv, const float* __restr
     }
 }
 
-// New token's k rotated at its position into cache slot pos[b], v copied there.
+// New token's k rotated at its position into its cache slot (the position, or its
+// place in a rolling cache of sinks + window), v copied there.
 // One thread per 8-element chunk (adjacent pairs) or per pair of chunks
 // (half-split pairs) of every (batch, kv head) vector.
 template <int PAIR_STYLE>
@@ -151,11 +152,12 @@ __global__ void kv_append_kernel(KvAppendArgs a)
         const int chunk = static_cast<int>(tid - vec * per_vec);
         const int b = static_cast<int>(vec / a.Hk);
         const int m = a.pos[b];
-        if (m < 0 || m >= a.T_max || m >= a.max_pos) {
+        const int slot = (a.window > 0 && m >= a.n_sink) ? a.n_sink + (m - a.n_sink) % a.window : m;
+        if (m < 0 || slot >= a.T_max || m >= a.max_pos) {
             if (chunk == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_POSITION);
             continue;
         }
-        const long long row = (vec * a.T_max + m) * a.head_dim;
+        const long long row = (vec * a.T_max + slot) * a.head_dim;
         const __nv_bfloat16* kn = reinterpret_cast<const __nv_bfloat16*>(a.k_new) + vec * a.head_dim;
         const __nv_bfloat16* vn = reinterpret_cast<const __nv_bfloat16*>(a.v_new) + vec * a.head_dim;
         __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(a.k_cache) + row;

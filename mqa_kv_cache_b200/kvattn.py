@@ -44,6 +44,10 @@ _lib.attn_decode_gqa.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i3
 _lib.attn_decode_gqa_rope.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                       _f32, _vp, _vp, _vp, _sz, _vp, _vp]
 _lib.kv_append_rope.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _i32, _i32, _vp, _vp]
+_lib.kv_append_rope_ring.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp, _i32, _i32,
+                                     _vp, _vp]
+_lib.attn_decode_gqa_rope_window.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                             _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp, _vp]
 _lib.attn_decode_gqa_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
                                          _vp]
 _lib.attn_prefill_causal.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]
@@ -244,6 +248,48 @@ def kv_append_rope(k_new, v_new, pos, k_cache, v_cache, cos, sin, pair_style=0, 
         raise ValueError("inconsistent append shapes")
     _check(_lib.kv_append_rope(_ptr(k_new), _ptr(v_new), _ptr(pos), B, Hk, d, _ptr(k_cache), _ptr(v_cache), T_max,
                                _ptr(cos), _ptr(sin), cos.shape[0], pair_style, _ptr(dev_status), _stream()))
+
+
+def kv_append_rope_ring(k_new, v_new, pos, k_cache, v_cache, cos, sin, n_sink, window, pair_style=0, dev_status=None):
+    """kv_append_rope into a rolling cache of n_sink + window slots (slot of position
+    p >= n_sink: n_sink + (p - n_sink) % window)."""
+    for t, n in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    _need(pos, torch.int32, "pos")
+    _contig(pos, "pos")
+    B, Hk, d = k_new.shape
+    Bc, Hc, T_max, dc = k_cache.shape
+    if (Bc, Hc, dc) != (B, Hk, d) or v_cache.shape != k_cache.shape or v_new.shape != k_new.shape or pos.numel() != B:
+        raise ValueError("inconsistent append shapes")
+    _check(_lib.kv_append_rope_ring(_ptr(k_new), _ptr(v_new), _ptr(pos), int(n_sink), int(window), B, Hk, d,
+                                    _ptr(k_cache), _ptr(v_cache), T_max, _ptr(cos), _ptr(sin), cos.shape[0],
+                                    pair_style, _ptr(dev_status), _stream()))
+
+
+def attn_decode_gqa_rope_window(q, q_pos, cos, sin, k_cache, v_cache, seq_lens, scale, n_sink, window, pair_style=0,
+                                out=None, lse=None, ws=None, dev_status=None, want_lse=True):
+    """attn_decode_gqa_rope over a rolling cache: seq_lens = tokens so far; attention over the
+    min(seq_lens, n_sink + window) filled slots (the sinks and the last `window` tokens)."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    for t, n in ((seq_lens, "seq_lens"), (q_pos, "q_pos")):
+        _need(t, torch.int32, n)
+        _contig(t, n)
+    B, H, d = q.shape
+    _, Hk, T_max, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(attn_decode_gqa_workspace_bytes(B, H, Hk, d, T_max), q.device)
+    _check(_lib.attn_decode_gqa_rope_window(_ptr(q), _ptr(q_pos), _ptr(cos), _ptr(sin), cos.shape[0], pair_style,
+                                            _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), int(n_sink), int(window), B,
+                                            H, Hk, d, T_max, float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                            _ptr(dev_status), _stream()))
+    return out, lse
 
 
 def attn_decode_gqa_noalloc(q, k_cache, v_cache, seq_lens, scale, out=None, lse=None, dev_status=None,

@@ -145,6 +145,35 @@ def attn_decode(q, k, v, seq_lens, scale, sel=None, nthreads=0):
     return out, lse
 
 
+def window_positions(length, n_sink, window):
+    """Token positions a query at position `length` attends to under a sliding
+    window with attention sinks ("Agentic RL 入门3" §1: the last w keys, the first
+    s tokens kept; the band i - w < j <= i of the "attention" page, with the query's
+    own token not yet in the cache): tokens 0 .. n_sink-1 and the last `window`
+    of the `length` cached tokens, each once, in increasing order."""
+    sinks = list(range(min(n_sink, length)))
+    return sinks + list(range(max(n_sink, length - window), length))
+
+
+def attn_decode_window(q, k, v, seq_lens, scale, n_sink, window):
+    """Decode over a linear cache (row t holds token t) restricted to the window
+    and the sinks: the plain decode definition over the gathered rows of each
+    sequence.  q [B,H,d], k/v [B,Hk,T,d] (bf16 bits or float64) -> (out, lse)."""
+    B, H, d = np.shape(q)
+    Hk = np.shape(k)[1]
+    out = np.zeros((B, H, d), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    for b in range(B):
+        idx = window_positions(int(seq_lens[b]), n_sink, window)
+        n = len(idx)
+        kb = np.asarray(k)[b:b + 1][:, :, idx] if n else np.asarray(k)[b:b + 1][:, :, :1]
+        vb = np.asarray(v)[b:b + 1][:, :, idx] if n else np.asarray(v)[b:b + 1][:, :, :1]
+        o, l = attn_decode(np.asarray(q)[b:b + 1], np.ascontiguousarray(kb), np.ascontiguousarray(vb),
+                           np.array([n], np.int32), scale)
+        out[b], lse[b] = o[0], l[0]
+    return out, lse
+
+
 def attn_prefill(q, k, v, scale, sel=None, nthreads=0):
     """q [B,T,H,d], k/v [B,Hk,T,d] -> (out [B,T,H,d], lse [B,H,T]) or, with
     sel = [(b,h,i), ...], (out [n,d], lse [n])."""

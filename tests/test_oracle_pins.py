@@ -502,3 +502,60 @@ def test_sparse_attention_equals_masked_dense():
     perm = np.array([[9, -1, 4, 17, 25, -1, 3]], np.int32)
     out2, _ = oracle.attn_sparse(q, C, perm, Dv, 0.5)
     np.testing.assert_allclose(out2, out, rtol=1e-13, atol=1e-15)
+
+
+# ---- sliding window with attention sinks ----------------------------------------
+
+def test_window_positions_small_cases():
+    assert oracle.window_positions(10, 2, 3) == [0, 1, 7, 8, 9]
+    assert oracle.window_positions(3, 4, 2) == [0, 1, 2]      # everything fits
+    assert oracle.window_positions(5, 0, 2) == [3, 4]         # no sinks
+    assert oracle.window_positions(6, 2, 4) == [0, 1, 2, 3, 4, 5]  # sinks and window meet
+    assert oracle.window_positions(7, 2, 4) == [0, 1, 3, 4, 5, 6]
+    assert oracle.window_positions(0, 3, 5) == []
+
+
+def _rand(shape, rng):
+    return rng.standard_normal(shape)
+
+
+def test_window_decode_against_masked_softmax():
+    """The windowed decode equals softmax over all rows with -inf outside the row set,
+    written out here in numpy (brute force, fp64)."""
+    rng = np.random.default_rng(3)
+    B, H, Hk, d, T = 3, 4, 2, 8, 40
+    q, k, v = _rand((B, H, d), rng), _rand((B, Hk, T, d), rng), _rand((B, Hk, T, d), rng)
+    lens = np.array([40, 9, 23], np.int32)
+    s_, w_, scale = 3, 7, 0.3
+    out, lse = oracle.attn_decode_window(q, k, v, lens, scale, s_, w_)
+    for b in range(B):
+        keep = np.zeros(T, bool)
+        keep[:min(s_, lens[b])] = True
+        keep[max(s_, lens[b] - w_):lens[b]] = True
+        for h in range(H):
+            sc = scale * k[b, h // (H // Hk)] @ q[b, h]
+            sc[~keep] = -np.inf
+            p = np.exp(sc - sc.max())
+            np.testing.assert_allclose(out[b, h], (p / p.sum()) @ v[b, h // (H // Hk)], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(lse[b, h], sc.max() + np.log(p.sum()), rtol=1e-12)
+
+
+def test_window_decode_special_cases():
+    rng = np.random.default_rng(4)
+    B, H, Hk, d, T = 2, 2, 1, 16, 30
+    q, k, v = _rand((B, H, d), rng), _rand((B, Hk, T, d), rng), _rand((B, Hk, T, d), rng)
+    lens = np.array([30, 12], np.int32)
+    full, full_l = oracle.attn_decode(q, k, v, lens, 0.25)
+    # a window (plus sinks) covering every cached token is the plain decode
+    for s_, w_ in ((0, 30), (5, 25), (2, 100)):
+        o, l = oracle.attn_decode_window(q, k, v, lens, 0.25, s_, w_)
+        np.testing.assert_array_equal(o, full)
+        np.testing.assert_array_equal(l, full_l)
+    # window 1, no sinks: the last cached token's value
+    o, l = oracle.attn_decode_window(q, k, v, lens, 0.25, 0, 1)
+    for b in range(B):
+        np.testing.assert_allclose(o[b], np.repeat(v[b, :, lens[b] - 1], H, axis=0), rtol=1e-14)
+        np.testing.assert_allclose(l[b], 0.25 * (q[b] @ k[b, 0, lens[b] - 1]), rtol=1e-12)
+    # an empty cache attends to nothing
+    o, l = oracle.attn_decode_window(q, k, v, np.array([0, 0], np.int32), 0.25, 2, 3)
+    assert np.all(o == 0) and np.all(np.isneginf(l))
