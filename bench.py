@@ -380,6 +380,32 @@ def measure_prefill(K, device, steps, flush, peaks):
             "tok_per_s": round(w.B * w.T / (step_ms * 1e-3), 1)}
 
 
+def measure_prefill_window(K, device, steps, flush, peaks):
+    """The prefill shape with a 2048-token window and 4 sink tokens
+    (attn_prefill_causal_window); FLOPs counted over the rows' actual key sets."""
+    w = W.PREFILL_8K
+    n_sink, window = 4, 2048
+    gen = W.generator(W.SEED_BASE + w.index + 9, device)
+    q = W.normal_bf16((w.B, w.T, w.H, w.d), gen, device)
+    k = W.normal_bf16((w.B, w.Hk, w.T, w.d), gen, device)
+    v = W.normal_bf16((w.B, w.Hk, w.T, w.d), gen, device)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.T), dtype=torch.float32, device=device)
+
+    def attn():
+        K.attn_prefill_causal_window(q, k, v, w.scale, n_sink, window, out=out, lse=lse)
+
+    ms = _graph_ms(attn, max(10, steps // 10), flush)
+    i = np.arange(w.T) + 1  # keys a row's query could see (causal), then the window and the sinks
+    seen = np.where(i > n_sink, np.minimum(i, n_sink) + i - np.maximum(n_sink, i - window), i)
+    flops = 4.0 * w.B * w.H * w.d * float(seen.sum())
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"causal_prefill_B2_T8192_H32_Hk8_d128_sink{n_sink}_window{window}", "attn_ms": round(ms, 4),
+            "flops": flops, "attn_TFLOP_s": round(tf, 1),
+            "pct_of_bf16_peak_burst": round(100 * tf / peaks["bf16_tflops"], 1),
+            "tok_per_s": round(w.B * w.T / (ms * 1e-3), 1)}
+
+
 def measure_dsa(K, device, steps, flush, peaks):
     w = W.DSA_128K
     gen = W.generator(W.SEED_BASE + w.index, device)
@@ -454,6 +480,8 @@ def measure_others(K, device, steps, flush, peaks):
     win = measure_window(K, device, steps, flush, peaks)
     res[win["workload"]] = win
     res[W.PREFILL_8K.name] = measure_prefill(K, device, steps, flush, peaks)
+    pw = measure_prefill_window(K, device, steps, flush, peaks)
+    res[pw["workload"]] = pw
     res[W.DSA_128K.name] = measure_dsa(K, device, steps, flush, peaks)
     torch.cuda.empty_cache()
     return res
@@ -568,7 +596,7 @@ def main():
     ap.add_argument("--impl", default="kvattn", choices=["kvattn", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", action="store_true", help="skip the other configurations")
-    ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "window", "prefill", "dsa"],
+    ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "window", "prefill", "prefill_window", "dsa"],
                     help="time one other configuration alone and print its JSON")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -596,6 +624,8 @@ def main():
             res = measure_prefill(K, device, args.steps, flush, peaks)
         elif args.only == "window":
             res = measure_window(K, device, args.steps, flush, peaks)
+        elif args.only == "prefill_window":
+            res = measure_prefill_window(K, device, args.steps, flush, peaks)
         else:
             res = measure_dsa(K, device, args.steps, flush, peaks)
         if rank == 0:

@@ -266,6 +266,17 @@ int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn
                         int T, int n_head, int n_kv_head, int head_dim, float scale,
                         kvattn_bf16* out, float* lse, void* stream);
 
+/*
+ * attn_prefill_causal with a sliding window and attention sinks (the band
+ * mask of the "attention" page, "Agentic RL 入门3" §1 sinks): query row i sees
+ * key j iff j <= i and (j > i - window or j < n_sink).  Key tiles entirely
+ * outside every row's set are skipped.  window >= 1, n_sink >= 0; otherwise as
+ * attn_prefill_causal.
+ */
+int attn_prefill_causal_window(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B,
+                               int T, int n_head, int n_kv_head, int head_dim, int n_sink, int window,
+                               float scale, kvattn_bf16* out, float* lse, void* stream);
+
 /* ---- lightning indexer + top-k ---------------------------------------------
  * "Agentic RL 入门3" §2.2 (1): s_{b,t} = sum_{j < H_I} w[b][j] *
  * ReLU(q_idx[b][j] . k_idx[b][t]) (no scale, no RoPE); §2.2 (2): S_b =

@@ -415,31 +415,49 @@ int kv_append_rope(const kvattn_bf16* k_new, const kvattn_bf16* v_new, const int
 }
 
 // ---------------------------------------------------------------------------
-int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B, int T, int n_head,
-                        int n_kv_head, int head_dim, float scale, kvattn_bf16* out, float* lse, void* stream)
+static int prefill_call(const char* name, const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B,
+                        int T, int n_head, int n_kv_head, int head_dim, float scale, kvattn_bf16* out, float* lse,
+                        int n_sink, int window, void* stream)
 {
-    if (!q || !k || !v || !out) return fail(KVATTN_ERR_NULL, "attn_prefill_causal: NULL argument");
-    if (head_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "attn_prefill_causal: head_dim %d (needs 128)", head_dim);
+    if (!q || !k || !v || !out) return fail(KVATTN_ERR_NULL, "%s: NULL argument", name);
+    if (head_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "%s: head_dim %d (needs 128)", name, head_dim);
     if (B < 1 || T < 1 || n_head < 1 || n_kv_head < 1 || n_head % n_kv_head)
-        return fail(KVATTN_ERR_SHAPE, "attn_prefill_causal: B %d T %d n_head %d n_kv_head %d", B, T, n_head, n_kv_head);
+        return fail(KVATTN_ERR_SHAPE, "%s: B %d T %d n_head %d n_kv_head %d", name, B, T, n_head, n_kv_head);
     if (!g_supported(n_head / n_kv_head))
-        return fail(KVATTN_ERR_UNSUPPORTED, "attn_prefill_causal: group size %d", n_head / n_kv_head);
+        return fail(KVATTN_ERR_UNSUPPORTED, "%s: group size %d", name, n_head / n_kv_head);
     if (static_cast<long long>(B) * n_kv_head > (1ll << 31) - 1 || T > (1 << 30) ||
         static_cast<long long>((T + 255) / 256) * B * n_head > (1ll << 31) - 1)
-        return fail(KVATTN_ERR_SHAPE, "attn_prefill_causal: problem too large");
+        return fail(KVATTN_ERR_SHAPE, "%s: problem too large", name);
     if (!(scale > 0.0f) || !std::isfinite(scale))
-        return fail(KVATTN_ERR_SHAPE, "attn_prefill_causal: scale must be finite > 0");
+        return fail(KVATTN_ERR_SHAPE, "%s: scale must be finite > 0", name);
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-        return fail(KVATTN_ERR_ALIGN, "attn_prefill_causal: tensors must be 16-byte aligned");
+        return fail(KVATTN_ERR_ALIGN, "%s: tensors must be 16-byte aligned", name);
     CUtensorMap tm_q, tm_k, tm_v;
     if (make_map_4d_rows(&tm_q, q, head_dim, n_head, T, B, kvattn::PREFILL_Q_ROWS) != KVATTN_OK)
         return KVATTN_ERR_CUDA;
     const uint64_t units = static_cast<uint64_t>(B) * n_kv_head;
     if (make_map_3d(&tm_k, k, head_dim, T, units, kvattn::PREFILL_KV_ROWS) != KVATTN_OK) return KVATTN_ERR_CUDA;
     if (make_map_3d(&tm_v, v, head_dim, T, units, kvattn::PREFILL_KV_ROWS) != KVATTN_OK) return KVATTN_ERR_CUDA;
-    kvattn::PrefillLaunch l{out, lse, nullptr, B, T, n_head, n_kv_head, scale};
+    kvattn::PrefillLaunch l{out, lse, nullptr, B, T, n_head, n_kv_head, scale, n_sink, window};
     return cuda_status(kvattn::launch_prefill(l, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
-                       "attn_prefill_causal launch");
+                       name);
+}
+
+int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B, int T, int n_head,
+                        int n_kv_head, int head_dim, float scale, kvattn_bf16* out, float* lse, void* stream)
+{
+    return prefill_call("attn_prefill_causal", q, k, v, B, T, n_head, n_kv_head, head_dim, scale, out, lse, 0, 0,
+                        stream);
+}
+
+int attn_prefill_causal_window(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn_bf16* v, int B, int T,
+                               int n_head, int n_kv_head, int head_dim, int n_sink, int window, float scale,
+                               kvattn_bf16* out, float* lse, void* stream)
+{
+    if (n_sink < 0 || window < 1)
+        return fail(KVATTN_ERR_SHAPE, "attn_prefill_causal_window: n_sink %d, window %d", n_sink, window);
+    return prefill_call("attn_prefill_causal_window", q, k, v, B, T, n_head, n_kv_head, head_dim, scale, out, lse,
+                        n_sink, window, stream);
 }
 
 size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k)

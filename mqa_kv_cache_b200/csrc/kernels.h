@@ -145,6 +145,7 @@ struct PrefillLaunch {
     int32_t* dev_status;
     int B, T, H, Hk;
     float scale;
+    int n_sink = 0, window = 0;  // window > 0: sliding window with n_sink sink tokens
 };
 cudaError_t launch_prefill(const PrefillLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                            const CUtensorMap& tm_v, cudaStream_t stream);

@@ -51,9 +51,13 @@ struct PrefillArgs {
     float* lse;        // [B][H][T] or null
     int32_t* dev_status;
     int B, T, H, Hk, g, n_qblk;
+    int n_sink, window;  // window > 0: query i sees keys j <= i with j > i - window or j < n_sink
     float scale;
 };
 
+// WINDOW: a sliding window with sinks is in effect (a.window > 0); the plain causal
+// kernel is compiled without the band test.
+template <bool WINDOW>
 __global__ void __launch_bounds__(PF_THREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, PrefillArgs a)
@@ -80,8 +84,21 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const int kvh = h / a.g;
     const int q0 = qblk * 2 * PF_BM;
     const int n_qt = (a.T - q0) > PF_BM ? 2 : 1;   // Q tiles in this block
-    // K/V tiles seen by Q tile t: keys 0 .. q0 + 128 t + 127 (the last one on the diagonal)
-    const int n_kv0 = q0 / PF_BN + 1;
+    // Key tiles.  Q tile t sees tiles 0 .. diag(t) (its diagonal tile); with a window, only the
+    // sink tiles [0, ns) and the band tiles [lo(t), diag(t)].  The CTA walks the union of its Q
+    // tiles' sets in increasing order (lo(0) <= lo(1), diag(1) = diag(0) + 1); each Q tile counts
+    // its own steps, which set its barrier phases.
+    const int ns = WINDOW ? (a.n_sink + PF_BN - 1) / PF_BN : 0;
+    auto diag_of = [&](int t) { return (q0 + t * PF_BM) / PF_BN; };
+    auto lo_of = [&](int t) {
+        const int first_key = q0 + t * PF_BM - a.window + 1;  // lowest band key of the tile's first row
+        return (WINDOW && first_key > 0) ? first_key / PF_BN : 0;
+    };
+    auto first_in = [&](int lo) { return (ns > 0 || lo == 0) ? 0 : lo; };
+    auto next_in = [&](int lo, int j) { return (j + 1 < ns || j + 1 >= lo) ? j + 1 : lo; };
+    auto in_t = [&](int t, int j) { return t < n_qt && j <= diag_of(t) && (j < ns || j >= lo_of(t)); };
+    const int lo_u = lo_of(0), d_u = diag_of(n_qt - 1);
+    const int n_kv0 = q0 / PF_BN + 1;  // plain causal: Q tile t sees tiles 0 .. n_kv0 - 1 + t
     const int n_kv = n_kv0 + (n_qt - 1);
 
     if (threadIdx.x == 0) {
@@ -125,19 +142,38 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 tma_load_4d(dst + PF_BOX, &tm_q, q_full, 64, h, q0 + t * PF_BM, b);
             }
             const int z = b * a.Hk + kvh;
-            int u = 0;  // ring sequence: K_0, V_0, K_1, V_1, ...
-            for (int j = 0; j < n_kv && !*s_abort; ++j) {
-                for (int kv = 0; kv < 2; ++kv, ++u) {
-                    const int slot = u % PF_SLOTS;
-                    if (u >= PF_SLOTS && !mbar_wait(&kv_empty[slot], ((u / PF_SLOTS) - 1) & 1)) {
-                        *s_abort = 1;
-                        break;
+            int u = 0;
+            if constexpr (WINDOW) {
+                // ring sequence: K_j, V_j for the CTA's key tiles j in increasing order
+                for (int j = first_in(lo_u); j <= d_u && !*s_abort; j = next_in(lo_u, j)) {
+                    for (int kv = 0; kv < 2; ++kv, ++u) {
+                        const int slot = u % PF_SLOTS;
+                        if (u >= PF_SLOTS && !mbar_wait(&kv_empty[slot], ((u / PF_SLOTS) - 1) & 1)) {
+                            *s_abort = 1;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&kv_full[slot], PF_TILE);
+                        uint8_t* dst = smem + PF_OFF_KV + slot * PF_TILE;
+                        const CUtensorMap* m = kv == 0 ? &tm_k : &tm_v;
+                        tma_load_3d(dst, m, &kv_full[slot], 0, j * PF_BN, z);
+                        tma_load_3d(dst + PF_BOX, m, &kv_full[slot], 64, j * PF_BN, z);
                     }
-                    mbar_arrive_expect_tx(&kv_full[slot], PF_TILE);
-                    uint8_t* dst = smem + PF_OFF_KV + slot * PF_TILE;
-                    const CUtensorMap* m = kv == 0 ? &tm_k : &tm_v;
-                    tma_load_3d(dst, m, &kv_full[slot], 0, j * PF_BN, z);
-                    tma_load_3d(dst + PF_BOX, m, &kv_full[slot], 64, j * PF_BN, z);
+                }
+            } else {
+                // ring sequence: K_0, V_0, K_1, V_1, ...
+                for (int j = 0; j < n_kv && !*s_abort; ++j) {
+                    for (int kv = 0; kv < 2; ++kv, ++u) {
+                        const int slot = u % PF_SLOTS;
+                        if (u >= PF_SLOTS && !mbar_wait(&kv_empty[slot], ((u / PF_SLOTS) - 1) & 1)) {
+                            *s_abort = 1;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&kv_full[slot], PF_TILE);
+                        uint8_t* dst = smem + PF_OFF_KV + slot * PF_TILE;
+                        const CUtensorMap* m = kv == 0 ? &tm_k : &tm_v;
+                        tma_load_3d(dst, m, &kv_full[slot], 0, j * PF_BN, z);
+                        tma_load_3d(dst + PF_BOX, m, &kv_full[slot], 64, j * PF_BN, z);
+                    }
                 }
             }
             if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
@@ -162,61 +198,117 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 }
                 tc_commit(&s_full[t]);
             };
-            auto issue_pv = [&](int t, int j, uint32_t vslot_addr) {
+            auto issue_pv = [&](int t, bool acc, uint32_t vslot_addr) {
                 const uint32_t d = tmem + 256 + t * PF_D;  // O_t
                 const uint32_t pa = tmem + t * PF_BN;      // P_t over S_t, bf16 pairs
 #pragma unroll
                 for (int ks = 0; ks < PF_BN / 16; ++ks) {
                     // V tile [keys][d]: 16 keys = 2 eight-row atoms (2 KB); the two 64-wide d blocks 16 KB apart
                     const uint64_t bd = umma_desc_mn_sw128(vslot_addr + ks * 2048, PF_BOX, 1024);
-                    tc_mma_bf16_ts(d, pa + ks * 8, bd, PF_IDESC_O, (j > 0 || ks > 0) ? 1u : 0u);
+                    tc_mma_bf16_ts(d, pa + ks * 8, bd, PF_IDESC_O, (acc || ks > 0) ? 1u : 0u);
                 }
                 tc_commit(&pv_done[t]);
             };
-            // S for tile 0 of every Q tile
-            int kslot = 0;
-            if (ok) {
-                kslot = u % PF_SLOTS;
-                ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
-                ++u;
-            }
-            if (ok) {
-                tc_fence_after();
-                const uint32_t ka = skv + kslot * PF_TILE;
-                if (n_kv0 > 0) issue_s(0, ka);
-                if (n_qt > 1) issue_s(1, ka);
-                tc_commit(&kv_empty[kslot]);
-            }
-            for (int j = 0; j < n_kv && ok; ++j) {
-                const int vslot = u % PF_SLOTS;
-                ok = mbar_wait(&kv_full[vslot], (u / PF_SLOTS) & 1);
-                ++u;
-                if (!ok) break;
-                const uint32_t va = skv + vslot * PF_TILE;
-                for (int t = 0; t < n_qt && ok; ++t) {
-                    if (j >= n_kv0 + t) continue;  // Q tile 0 stops one tile earlier
-                    ok = mbar_wait(&p_full[t], j & 1);
-                    if (!ok) break;
-                    tc_fence_after();
-                    issue_pv(t, j, va);
-                }
-                if (!ok) break;
-                tc_commit(&kv_empty[vslot]);
-                if (j + 1 < n_kv) {
+            if constexpr (WINDOW) {
+                // scores of the first key tile for the Q tiles that see it
+                int cnt[2] = {0, 0};  // P V products issued per Q tile
+                int kslot = 0;
+                int j = first_in(lo_u);
+                if (ok) {
                     kslot = u % PF_SLOTS;
                     ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
                     ++u;
-                    if (!ok) break;
+                }
+                if (ok) {
+                    tc_fence_after();
                     const uint32_t ka = skv + kslot * PF_TILE;
-                    for (int t = 0; t < n_qt && ok; ++t) {
-                        if (j + 1 >= n_kv0 + t) continue;
-                        // P_t (read by the P V just issued) shares columns with S_t: wait for it
-                        ok = mbar_wait(&pv_done[t], j & 1);
+                    for (int t = 0; t < 2; ++t)
+                        if (in_t(t, j)) issue_s(t, ka);
+                    tc_commit(&kv_empty[kslot]);
+                }
+                for (; j <= d_u && ok;) {
+                    const int jn = next_in(lo_u, j);
+                    const int vslot = u % PF_SLOTS;
+                    ok = mbar_wait(&kv_full[vslot], (u / PF_SLOTS) & 1);
+                    ++u;
+                    if (!ok) break;
+                    const uint32_t va = skv + vslot * PF_TILE;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (!in_t(t, j)) continue;
+                        ok = mbar_wait(&p_full[t], cnt[t] & 1);
                         if (!ok) break;
                         tc_fence_after();
-                        issue_s(t, ka);
+                        issue_pv(t, cnt[t] > 0, va);
+                        ++cnt[t];
                     }
+                    if (!ok) break;
+                    tc_commit(&kv_empty[vslot]);
+                    if (jn <= d_u) {
+                        kslot = u % PF_SLOTS;
+                        ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
+                        ++u;
+                        if (!ok) break;
+                        const uint32_t ka = skv + kslot * PF_TILE;
+                        for (int t = 0; t < 2 && ok; ++t) {
+                            if (!in_t(t, jn)) continue;
+                            // P_t (read by this Q tile's last P V) shares columns with S_t: wait for it
+                            if (cnt[t] > 0) {
+                                ok = mbar_wait(&pv_done[t], (cnt[t] - 1) & 1);
+                                if (!ok) break;
+                                tc_fence_after();
+                            }
+                            issue_s(t, ka);
+                        }
+                        tc_commit(&kv_empty[kslot]);
+                    }
+                    j = jn;
+                }
+            } else {
+                // S for tile 0 of every Q tile
+                int kslot = 0;
+                if (ok) {
+                    kslot = u % PF_SLOTS;
+                    ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
+                    ++u;
+                }
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t ka = skv + kslot * PF_TILE;
+                    if (n_kv0 > 0) issue_s(0, ka);
+                    if (n_qt > 1) issue_s(1, ka);
                     tc_commit(&kv_empty[kslot]);
+                }
+                for (int j = 0; j < n_kv && ok; ++j) {
+                    const int vslot = u % PF_SLOTS;
+                    ok = mbar_wait(&kv_full[vslot], (u / PF_SLOTS) & 1);
+                    ++u;
+                    if (!ok) break;
+                    const uint32_t va = skv + vslot * PF_TILE;
+                    for (int t = 0; t < n_qt && ok; ++t) {
+                        if (j >= n_kv0 + t) continue;  // Q tile 0 stops one tile earlier
+                        ok = mbar_wait(&p_full[t], j & 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_pv(t, j > 0, va);
+                    }
+                    if (!ok) break;
+                    tc_commit(&kv_empty[vslot]);
+                    if (j + 1 < n_kv) {
+                        kslot = u % PF_SLOTS;
+                        ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
+                        ++u;
+                        if (!ok) break;
+                        const uint32_t ka = skv + kslot * PF_TILE;
+                        for (int t = 0; t < n_qt && ok; ++t) {
+                            if (j + 1 >= n_kv0 + t) continue;
+                            // P_t (read by the P V just issued) shares columns with S_t: wait for it
+                            ok = mbar_wait(&pv_done[t], j & 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_s(t, ka);
+                        }
+                        tc_commit(&kv_empty[kslot]);
+                    }
                 }
             }
             if (!ok) {
@@ -232,17 +324,23 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;  // query row in the tile = TMEM lane
         const int qrow = q0 + t * PF_BM + row;
-        const int n_tiles = n_kv0 + t;
+        const int lo_t = lo_of(t), dg = diag_of(t);
+        // keys <= qrow - window (and not sinks) are outside the band; only tiles whose lowest key
+        // can fall that low for the tile's last row need the test
+        const int band_top = q0 + t * PF_BM + PF_BM - 1 - a.window;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + t * PF_BN;
         const uint32_t o_addr = tmem + lane_off + 256 + t * PF_D;
         const float sl2 = a.scale * kLog2e;
         float m_run = -INFINITY, l_run = 0.f;
         if (t < n_qt) {
-            for (int j = 0; j < n_tiles; ++j) {
-                if (!warp_wait(&s_full[t], j & 1, s_abort)) continue;
+            int k = 0;  // steps of this Q tile
+            for (int j = WINDOW ? first_in(lo_t) : 0; j <= dg; j = WINDOW ? next_in(lo_t, j) : j + 1, ++k) {
+                if (!warp_wait(&s_full[t], k & 1, s_abort)) continue;
                 tc_fence_after();
-                const bool diag = j == n_tiles - 1;  // keys j*128 .. : the diagonal tile
+                const bool diag = j == dg;  // keys j*128 .. : the diagonal tile
+                const bool band = WINDOW && j * PF_BN <= band_top;
+                const int kbase = j * PF_BN;
                 // Pass 1: row max of the raw scores (scale > 0 commutes with the max): the four
                 // 32-column loads are in flight together, one wait.
                 float mx = -INFINITY;
@@ -254,7 +352,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         tmem_regs_ready(sv[c]);
-                        if (diag) {
+                        if constexpr (WINDOW) {
+                            if (diag || band) {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) {
+                                    const int key = kbase + c * 32 + i;
+                                    // -inf: key after the query, or below its band and not a sink
+                                    if (key > qrow || (band && key <= qrow - a.window && key >= a.n_sink))
+                                        sv[c][i] = 0xff800000u;
+                                }
+                            }
+                        } else if (diag) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
                                 if (c * 32 + i > row) sv[c][i] = 0xff800000u;  // -inf: key after the query
@@ -271,7 +379,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 // their reference).
                 const bool move = mx > m_run + kRescaleThreshold || m_run == -INFINITY;
                 const float m_new = move ? fmaxf(mx, m_run) : m_run;
-                const bool rescale = move && m_run != -INFINITY && j > 0;
+                const bool rescale = move && m_run != -INFINITY && k > 0;
                 if (__any_sync(0xffffffffu, rescale)) {
                     const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.f;
                     l_run *= alpha;
@@ -300,7 +408,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 for (int c = 0; c < 4; ++c) {
                     uint32_t (&sv)[32] = sb[c & 1];
                     if (c < 3) tmem_ld32(s_addr + (c + 1) * 32, sb[(c + 1) & 1]);
-                    if (diag) {
+                    if constexpr (WINDOW) {
+                        if (diag || band) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const int key = kbase + c * 32 + i;
+                                if (key > qrow || (band && key <= qrow - a.window && key >= a.n_sink))
+                                    sv[i] = 0xff800000u;
+                            }
+                        }
+                    } else if (diag) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (c * 32 + i > row) sv[i] = 0xff800000u;
@@ -341,7 +458,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (lane == 0) mbar_arrive(&p_full[t]);
             }
             // ---- epilogue: O / l -> bf16 rows, lse ----
-            if (warp_wait(&pv_done[t], (n_tiles - 1) & 1, s_abort)) {
+            if (warp_wait(&pv_done[t], (k - 1) & 1, s_abort)) {
                 tc_fence_after();
                 const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
                 __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
@@ -387,7 +504,9 @@ cudaError_t launch_prefill(const PrefillLaunch& l, const CUtensorMap& tm_q, cons
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
+        e = cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
@@ -402,8 +521,10 @@ cudaError_t launch_prefill(const PrefillLaunch& l, const CUtensorMap& tm_q, cons
     a.g = l.H / l.Hk;
     a.n_qblk = (l.T + 2 * PF_BM - 1) / (2 * PF_BM);
     a.scale = l.scale;
+    a.n_sink = l.n_sink;
+    a.window = l.window;
     const long long grid = static_cast<long long>(a.n_qblk) * l.B * l.H;
-    return launch_pdl(prefill_kernel, dim3(static_cast<unsigned>(grid)), dim3(PF_THREADS), PF_SMEM, stream, tm_q,
+    return launch_pdl(a.window > 0 ? prefill_kernel<true> : prefill_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(PF_THREADS), PF_SMEM, stream, tm_q,
                       tm_k, tm_v, a);
 }
 

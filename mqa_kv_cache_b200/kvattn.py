@@ -51,6 +51,8 @@ _lib.attn_decode_gqa_rope_window.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _vp
 _lib.attn_decode_gqa_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
                                          _vp]
 _lib.attn_prefill_causal.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]
+_lib.attn_prefill_causal_window.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp,
+                                            _vp]
 _lib.dsa_index_topk_workspace_bytes.argtypes = [_i32, _i32, _i32]
 _lib.dsa_index_topk_workspace_bytes.restype = _sz
 _lib.dsa_index_topk.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp, _vp]
@@ -326,6 +328,24 @@ def attn_prefill_causal(q, k, v, scale, out=None, lse=None, want_lse=True):
         lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
     _check(_lib.attn_prefill_causal(_ptr(q), _ptr(k), _ptr(v), B, T, H, Hk, d, float(scale), _ptr(out), _ptr(lse),
                                     _stream()))
+    return out, lse
+
+
+def attn_prefill_causal_window(q, k, v, scale, n_sink, window, out=None, lse=None, want_lse=True):
+    """attn_prefill_causal where row i sees keys j <= i with j > i - window or j < n_sink."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, torch.bfloat16, n)
+        _contig(t, n)
+    B, T, H, d = q.shape
+    Hk = k.shape[1]
+    if k.shape != (B, Hk, T, d) or v.shape != k.shape:
+        raise ValueError("inconsistent prefill shapes")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check(_lib.attn_prefill_causal_window(_ptr(q), _ptr(k), _ptr(v), B, T, H, Hk, d, int(n_sink), int(window),
+                                           float(scale), _ptr(out), _ptr(lse), _stream()))
     return out, lse
 
 

@@ -174,6 +174,23 @@ def attn_decode_window(q, k, v, seq_lens, scale, n_sink, window):
     return out, lse
 
 
+def attn_prefill_window(q, k, v, scale, n_sink, window, sel):
+    """Causal prefill with a sliding window and sinks, row by row: row i of a prompt
+    is the decode of q_i over the prefix 0 .. i (its own token included, so the
+    band is i - window < j <= i) restricted to the sinks and the window.
+    q [B,T,H,d], k/v [B,Hk,T,d]; sel = [(b, h, i), ...] -> (out [n, d], lse [n])."""
+    q, k, v = np.asarray(q), np.asarray(k), np.asarray(v)
+    d = q.shape[-1]
+    out = np.zeros((len(sel), d), np.float64)
+    lse = np.zeros(len(sel), np.float64)
+    for n, (b, h, i) in enumerate(sel):
+        o, l = attn_decode_window(q[b:b + 1, i], np.ascontiguousarray(k[b:b + 1, :, :i + 1]),
+                                  np.ascontiguousarray(v[b:b + 1, :, :i + 1]), np.array([i + 1], np.int32), scale,
+                                  n_sink, window)
+        out[n], lse[n] = o[0, h], l[0, h]
+    return out, lse
+
+
 def attn_prefill(q, k, v, scale, sel=None, nthreads=0):
     """q [B,T,H,d], k/v [B,Hk,T,d] -> (out [B,T,H,d], lse [B,H,T]) or, with
     sel = [(b,h,i), ...], (out [n,d], lse [n])."""

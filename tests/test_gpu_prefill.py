@@ -109,3 +109,29 @@ def test_deterministic(K):
     a = _run(K, q, k, v, 0.1)
     b = _run(K, q, k, v, 0.1)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("T,n_sink,window", [(700, 4, 200), (513, 0, 128), (1000, 16, 300), (300, 3, 1),
+                                             (900, 130, 256), (385, 0, 129)])
+def test_window_prefill_against_oracle(K, T, n_sink, window):
+    """Row i sees keys j <= i with j > i - window or j < n_sink: sampled rows (every
+    third, plus the 128-row tile edges) against the row-by-row windowed decode."""
+    B, H, Hk = 1, 4, 2
+    q, k, v = _inputs(B, T, H, Hk, 300 + T + window)
+    out, lse = K.attn_prefill_causal_window(q.cuda(), k.cuda(), v.cuda(), 128 ** -0.5, n_sink, window)
+    torch.cuda.synchronize()
+    rows = sorted(set(range(0, T, 3)) | {r for r in (127, 128, 255, 256, 383, 384, 511, 512) if r < T} | {T - 1})
+    sel = [(0, h, i) for h in (0, 3) for i in rows]
+    ro, rl = oracle.attn_prefill_window(W.bf16_bits(q), W.bf16_bits(k), W.bf16_bits(v), 128 ** -0.5, n_sink, window,
+                                        sel)
+    got = torch.stack([out[b, i, h] for b, h, i in sel])
+    got_l = torch.stack([lse[b, h, i] for b, h, i in sel])
+    assert_attn_close(got, ro, got_l, rl, f"window prefill T={T} s={n_sink} w={window}")
+
+
+def test_window_longer_than_prompt_is_plain_causal(K):
+    q, k, v = _inputs(2, 600, 8, 2, 41)
+    a = K.attn_prefill_causal_window(q.cuda(), k.cuda(), v.cuda(), 0.1, 0, 600)
+    b = K.attn_prefill_causal(q.cuda(), k.cuda(), v.cuda(), 0.1)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])

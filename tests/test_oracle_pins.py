@@ -559,3 +559,24 @@ def test_window_decode_special_cases():
     # an empty cache attends to nothing
     o, l = oracle.attn_decode_window(q, k, v, np.array([0, 0], np.int32), 0.25, 2, 3)
     assert np.all(o == 0) and np.all(np.isneginf(l))
+
+
+def test_prefill_window_special_cases():
+    rng = np.random.default_rng(5)
+    B, T, H, Hk, d = 1, 24, 2, 1, 8
+    q, k, v = _rand((B, T, H, d), rng), _rand((B, Hk, T, d), rng), _rand((B, Hk, T, d), rng)
+    sel = [(0, h, i) for h in range(H) for i in (0, 1, 7, 23)]
+    full, full_l = oracle.attn_prefill(q, k, v, 0.5, sel=sel)
+    # a window as long as the prompt is the plain causal prefill
+    o, l = oracle.attn_prefill_window(q, k, v, 0.5, 0, T, sel)
+    np.testing.assert_allclose(o, full, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(l, full_l, rtol=1e-12)
+    # window 1, no sinks: every row sees only its own token
+    o, l = oracle.attn_prefill_window(q, k, v, 0.5, 0, 1, sel)
+    for n, (b, h, i) in enumerate(sel):
+        np.testing.assert_allclose(o[n], v[b, 0, i], rtol=1e-14)
+    # window 1 with 2 sinks: row 7 sees tokens 0, 1 and 7 only
+    o, l = oracle.attn_prefill_window(q, k, v, 0.5, 2, 1, [(0, 0, 7)])
+    sc = 0.5 * (k[0, 0, [0, 1, 7]] @ q[0, 7, 0])
+    p = np.exp(sc - sc.max())
+    np.testing.assert_allclose(o[0], (p / p.sum()) @ v[0, 0, [0, 1, 7]], rtol=1e-12)
