@@ -1,5 +1,5 @@
-"""fp64 CPU oracle for RoPE + grouped-query KV-cache attention and the
-lightning-indexer sparse path.
+"""fp64 CPU oracle for RoPE + grouped-query KV-cache attention, the
+lightning-indexer sparse path and the block-level (4-token group) indexer.
 
 TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / reference leg of ``bench.py`` may import this package.
@@ -285,3 +285,119 @@ def bf16_bits_to_f64(bits):
     bits = np.ascontiguousarray(bits, np.uint16)
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
+
+
+# ---------------------------------------------------------------------------
+# Block-level indexer ("attention" page, "Qwen Sparse Attention (QSA)" §3 ①–④)
+#
+# The visible prefix of a sequence of length L is cut into groups of 4 tokens;
+# each complete group becomes one block key: the mean of its 4 indexer keys,
+# normalised, then rotated at the position of the group's first token.  Blocks
+# are scored like the lightning indexer (a weighted sum over indexer heads of
+# ReLU(q . key)), the best n_top blocks are taken, every selected block is
+# unpacked back into its 4 token positions and the 0..3 tokens of the trailing
+# incomplete group are appended unconditionally; standard GQA attention then runs
+# over those tokens of the full-precision cache.
+#
+# Readings where the section leaves a step open:
+# * "normalise" = RMS normalisation without a learned gain,
+#   x / sqrt(mean(x^2) + eps) (the pages name RMS-style normalisation as their
+#   stabiliser elsewhere; no gain vector is given);
+# * the rotation is the model's RoPE table over all d_I dimensions at position 4j
+#   (the group's first token), with the same pair layout as every other rotation;
+# * the head weights w_j of the lightning indexer are kept (w_j = 1 gives the
+#   plain head sum of the section's sketch);
+# * one selection per sequence serves every KV head (the indexer has no KV-head
+#   axis);
+# * ties between block scores go to the lower block index, as in the top-k.
+# ---------------------------------------------------------------------------
+QSA_BLOCK = 4
+
+
+def qsa_block_keys(k_idx, lens, cos, sin, eps, pair_style=0):
+    """k_idx [B, L_max, d_I] (bf16 bits or float64), lens [B] -> block keys
+    [B, L_max // 4, d_I] fp64; rows j >= lens[b] // 4 are zero (no block)."""
+    _, k = _src(k_idx)
+    k = bf16_bits_to_f64(k) if k.dtype == np.uint16 else k
+    B, L_max, d = k.shape
+    nb_max = L_max // QSA_BLOCK
+    out = np.zeros((B, nb_max, d), np.float64)
+    for b in range(B):
+        nb = int(lens[b]) // QSA_BLOCK
+        if nb == 0:
+            continue
+        groups = k[b, :nb * QSA_BLOCK].reshape(nb, QSA_BLOCK, d)
+        mean = groups.sum(axis=1) / QSA_BLOCK
+        rms = np.sqrt((mean * mean).sum(axis=1) / d + eps)
+        normed = mean / rms[:, None]
+        pos = (np.arange(nb, dtype=np.int32) * QSA_BLOCK)[None]
+        out[b, :nb] = rope_apply(normed[None, :, None, :], pos, cos, sin, pair_style)[0, :, 0, :]
+    return out
+
+
+def qsa_scores(q_idx, w, block_keys, lens):
+    """Block scores s_j = sum_h w_h ReLU(q_h . key_j) over the complete blocks
+    j < lens[b] // 4; -inf elsewhere.  q_idx [B, H_I, d_I], w [B, H_I],
+    block_keys [B, NB, d_I] (bf16 bits or float64) -> [B, NB] fp64."""
+    q = np.asarray(q_idx)
+    q = bf16_bits_to_f64(q) if q.dtype == np.uint16 else q.astype(np.float64)
+    kb = np.asarray(block_keys)
+    kb = bf16_bits_to_f64(kb) if kb.dtype == np.uint16 else kb.astype(np.float64)
+    w = np.asarray(w, np.float64)
+    B, NB, _ = kb.shape
+    sc = np.full((B, NB), -np.inf)
+    for b in range(B):
+        nb = min(int(lens[b]) // QSA_BLOCK, NB)
+        dots = kb[b, :nb] @ q[b].T                      # [nb, H_I]
+        sc[b, :nb] = np.maximum(dots, 0.0) @ w[b]
+    return sc
+
+
+def qsa_expand(block_sel, lens, n_top):
+    """Selected blocks [B, n_top] (any order, -1 padded) -> (token positions
+    [B, 4 * n_top + 3] int32 in increasing order, -1 padded; counts [B]): every
+    selected block j gives 4j .. 4j+3, then the trailing tokens 4 * (L // 4) ..
+    L - 1 of the incomplete group."""
+    block_sel = np.asarray(block_sel, np.int64)
+    B = block_sel.shape[0]
+    width = QSA_BLOCK * n_top + QSA_BLOCK - 1
+    tok = np.full((B, width), -1, np.int32)
+    cnt = np.zeros(B, np.int32)
+    for b in range(B):
+        L = int(lens[b])
+        blocks = sorted(int(j) for j in block_sel[b] if j >= 0)
+        toks = [QSA_BLOCK * j + r for j in blocks for r in range(QSA_BLOCK)]
+        toks += list(range(QSA_BLOCK * (L // QSA_BLOCK), L))
+        tok[b, :len(toks)] = toks
+        cnt[b] = len(toks)
+    return tok, cnt
+
+
+def qsa_select(q_idx, w, block_keys, lens, n_top, scores=None):
+    """Score the complete blocks, keep the best n_top, expand with the tail.
+    With `scores` given (the kernel's own fp32 block scores), the selection is
+    taken on those, so that both sides decide in the same precision."""
+    nb_max = np.shape(block_keys)[1]
+    sc = qsa_scores(q_idx, w, block_keys, lens) if scores is None else np.asarray(scores, np.float64)
+    nb = np.array([min(int(x) // QSA_BLOCK, nb_max) for x in lens], np.int32)
+    sel = topk(sc, n_top, lens=nb)
+    return qsa_expand(sel, lens, n_top)
+
+
+def attn_decode_gqa_sparse(q, k, v, tok_idx, tok_count, scale):
+    """GQA decode over the listed tokens of a linear cache: the plain decode
+    definition over the gathered rows of each sequence (the first tok_count[b]
+    entries of tok_idx[b]).  q [B,H,d], k/v [B,Hk,T,d] -> (out, lse)."""
+    B, H, d = np.shape(q)
+    out = np.zeros((B, H, d), np.float64)
+    lse = np.zeros((B, H), np.float64)
+    k, v, q = np.asarray(k), np.asarray(v), np.asarray(q)
+    for b in range(B):
+        idx = [int(t) for t in tok_idx[b][:int(tok_count[b])]]
+        n = len(idx)
+        kb = k[b:b + 1][:, :, idx] if n else k[b:b + 1][:, :, :1]
+        vb = v[b:b + 1][:, :, idx] if n else v[b:b + 1][:, :, :1]
+        o, l = attn_decode(q[b:b + 1], np.ascontiguousarray(kb), np.ascontiguousarray(vb),
+                           np.array([n], np.int32), scale)
+        out[b], lse[b] = o[0], l[0]
+    return out, lse

@@ -98,6 +98,22 @@ def test_bad_length_is_clamped_and_flagged(K):
     assert_attn_close(out, ro, lse, rl, "clamped")
 
 
+@pytest.mark.parametrize("B,H,Hk,d,T", [(2, 8, 1, 128, 9000), (5, 64, 1, 128, 5000), (3, 16, 2, 64, 4000),
+                                        (16, 64, 1, 128, 3000), (7, 32, 1, 128, 2500)])
+def test_equal_lengths_split_into_whole_ranges(K, B, H, Hk, d, T):
+    """Units of one length: the plan may give each unit the same number of CTAs
+    (a multiple of the unit count), so that no CTA crosses into the next unit."""
+    gen = W.generator(300 + B + H + Hk + d)
+    q = W.normal_bf16((B, H, d), gen)
+    k = W.normal_bf16((B, Hk, T, d), gen)
+    v = W.normal_bf16((B, Hk, T, d), gen)
+    lens = torch.full((B,), T, dtype=torch.int32)
+    scale = d ** -0.5
+    out, lse = _run(K, q, k, v, lens, scale)
+    ro, rl = _oracle(q, k, v, lens, scale)
+    assert_attn_close(out, ro, lse, rl, f"equal B={B} H={H} Hk={Hk} d={d}")
+
+
 def test_deterministic(K):
     inp = W.decode_inputs(W.LLAMA3_8B_DECODE, B=4, T_max=2048)
     a = _run(K, inp["q"], inp["k"], inp["v"], inp["seq_lens"], 0.088)

@@ -580,3 +580,154 @@ def test_prefill_window_special_cases():
     sc = 0.5 * (k[0, 0, [0, 1, 7]] @ q[0, 7, 0])
     p = np.exp(sc - sc.max())
     np.testing.assert_allclose(o[0], (p / p.sum()) @ v[0, 0, [0, 1, 7]], rtol=1e-12)
+
+
+# ---- block-level indexer ("attention" page, "Qwen Sparse Attention (QSA)") -----------
+
+def _qsa_tables(d, n):
+    theta, _, _ = oracle.rope_freqs(d, 10000.0)
+    c, s = oracle.rope_table(d, 10000.0, n)
+    return theta, c, s
+
+
+def test_qsa_block_key_closed_form():
+    """A group of four equal keys u gives RMS-normalised u rotated by the angle
+    4j * theta_i at pair i: written with np.cos / np.sin from the frequencies, not
+    from the table, so a wrong rotation position (4j + 3, or j) fails."""
+    rng = np.random.default_rng(11)
+    d, eps = 16, 1e-6
+    theta, c, s = _qsa_tables(d, 64)
+    u = rng.standard_normal((5, d))
+    k = np.repeat(u, 4, axis=0)[None]                  # blocks 0..4, four equal rows each
+    kb = oracle.qsa_block_keys(k, np.array([20]), c, s, eps)
+    for j in range(5):
+        n = u[j] / math.sqrt((u[j] ** 2).mean() + eps)
+        ang = 4 * j * theta
+        x, y = n[0::2], n[1::2]
+        np.testing.assert_allclose(kb[0, j, 0::2], x * np.cos(ang) - y * np.sin(ang), rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(kb[0, j, 1::2], y * np.cos(ang) + x * np.sin(ang), rtol=1e-12, atol=1e-12)
+
+
+def test_qsa_block_key_is_the_mean_not_the_sum():
+    """Zero-sum offsets inside a group leave the block key unchanged, and with a
+    large eps the normalised magnitude is sqrt(d) * rms / sqrt(rms^2 + eps) of the
+    MEAN (a sum would carry rms 4x larger)."""
+    rng = np.random.default_rng(12)
+    d, eps = 8, 0.5
+    _, c, s = _qsa_tables(d, 16)
+    u = 0.1 * rng.standard_normal(d)
+    delta = rng.standard_normal((4, d))
+    delta -= delta.mean(axis=0)
+    k1 = np.repeat(u[None], 4, axis=0)[None]
+    k2 = (u[None] + delta)[None]
+    a = oracle.qsa_block_keys(k1, np.array([4]), c, s, eps)
+    b = oracle.qsa_block_keys(k2, np.array([4]), c, s, eps)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+    rms = math.sqrt((u ** 2).mean())
+    np.testing.assert_allclose(np.linalg.norm(a[0, 0]), math.sqrt(d) * rms / math.sqrt(rms * rms + eps), rtol=1e-12)
+
+
+def test_qsa_incomplete_group_makes_no_block():
+    rng = np.random.default_rng(13)
+    d = 8
+    _, c, s = _qsa_tables(d, 32)
+    k = rng.standard_normal((1, 12, d))
+    kb = oracle.qsa_block_keys(k, np.array([10]), c, s, 1e-6)
+    assert kb.shape == (1, 3, d)
+    assert np.all(kb[0, 2] == 0)                     # tokens 8, 9: no complete group
+    k2 = k.copy()
+    k2[0, 8:] = 1e3                                 # changing them changes no block key
+    np.testing.assert_array_equal(oracle.qsa_block_keys(k2, np.array([10]), c, s, 1e-6), kb)
+
+
+def test_qsa_scores_match_the_token_indexer_on_block_keys():
+    """Block scores are the lightning-indexer scores with blocks for tokens: the
+    numpy restatement agrees with the C indexer on bf16 block keys."""
+    gen = W.generator(14)
+    B, HI, dI, NB = 2, 4, 16, 30
+    q = W.bf16_bits(W.normal_bf16((B, HI, dI), gen))
+    kb = W.bf16_bits(W.normal_bf16((B, NB, dI), gen))
+    w = np.random.default_rng(14).uniform(0, 1, (B, HI)).astype(np.float32)
+    lens = np.array([4 * NB + 3, 4 * 7 + 1], np.int32)
+    sc = oracle.qsa_scores(q, w, kb, lens)
+    ref = oracle.dsa_scores(q, w, kb, np.array([NB, 7], np.int32))
+    np.testing.assert_allclose(sc, ref, rtol=1e-13, atol=0)
+    assert np.all(np.isneginf(sc[1, 7:]))
+
+
+def test_qsa_relu_drops_negative_heads():
+    q = np.array([[[1.0, 0.0], [0.0, 1.0]]])         # two indexer heads
+    kb = np.array([[[2.0, -3.0], [-1.0, -1.0]]])
+    w = np.array([[0.5, 2.0]])
+    sc = oracle.qsa_scores(q, w, kb, np.array([8]))
+    np.testing.assert_array_equal(sc, [[1.0, 0.0]])
+
+
+def test_qsa_expand_worked_example():
+    """Ten tokens: blocks 0 (0-3) and 1 (4-7) complete, tokens 8, 9 the tail.
+    With one block kept and block 1 the better, the set is 4..7 plus 8, 9."""
+    q = np.array([[[1.0, 0.0]]])
+    kb = np.array([[[0.1, 0.0], [0.9, 0.0]]])
+    tok, cnt = oracle.qsa_select(q, np.array([[1.0]]), kb, np.array([10]), n_top=1)
+    assert cnt[0] == 6
+    assert list(tok[0]) == [4, 5, 6, 7, 8, 9, -1]
+
+
+def test_qsa_budget_is_4k_plus_tail():
+    """512 blocks of 4 give 2048 tokens, plus 0..3 trailing ones: 2048..2051."""
+    rng = np.random.default_rng(15)
+    for L in (4 * 600, 4 * 600 + 1, 4 * 600 + 3, 4 * 512, 4 * 100 + 2):
+        sel = rng.permutation(L // 4)[:512]
+        tok, cnt = oracle.qsa_expand(sel[None], np.array([L]), 512)
+        nb = L // 4
+        assert cnt[0] == 4 * min(nb, 512) + L % 4 <= 2051
+        t = tok[0, :cnt[0]]
+        assert np.all(np.diff(t) > 0) and t[-1] < L and np.all(tok[0, cnt[0]:] == -1)
+        assert set(t[t >= 4 * nb]) == set(range(4 * nb, L))
+
+
+def test_qsa_ties_go_to_the_lower_block():
+    q = np.array([[[1.0]]])
+    kb = np.array([[[1.0], [2.0], [2.0], [2.0], [0.5]]])
+    tok, cnt = oracle.qsa_select(q, np.array([[1.0]]), kb, np.array([20]), n_top=2)
+    assert list(tok[0, :cnt[0]]) == [4, 5, 6, 7, 8, 9, 10, 11]
+
+
+def test_qsa_short_sequence_attends_to_everything():
+    """With at most n_top complete groups every token is selected, so the sparse
+    GQA decode is the plain decode."""
+    rng = np.random.default_rng(16)
+    B, H, Hk, d, T = 2, 4, 2, 8, 30
+    q, k, v = rng.standard_normal((B, H, d)), rng.standard_normal((B, Hk, T, d)), rng.standard_normal((B, Hk, T, d))
+    lens = np.array([30, 13], np.int32)
+    qi = rng.standard_normal((B, 3, d))
+    kb = rng.standard_normal((B, T // 4, d))
+    tok, cnt = oracle.qsa_select(qi, rng.uniform(0, 1, (B, 3)), kb, lens, n_top=8)
+    assert list(cnt) == [30, 13]
+    o, l = oracle.attn_decode_gqa_sparse(q, k, v, tok, cnt, 0.3)
+    ro, rl = oracle.attn_decode(q, k, v, lens, 0.3)
+    np.testing.assert_allclose(o, ro, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(l, rl, rtol=1e-13)
+
+
+def test_sparse_gqa_against_masked_softmax():
+    """Over any token list the sparse decode is softmax with -inf outside the list
+    (brute force in numpy); one listed token returns its value row."""
+    rng = np.random.default_rng(17)
+    B, H, Hk, d, T = 2, 6, 3, 8, 25
+    q, k, v = rng.standard_normal((B, H, d)), rng.standard_normal((B, Hk, T, d)), rng.standard_normal((B, Hk, T, d))
+    tok = np.full((B, 10), -1, np.int32)
+    tok[0, :5] = [0, 3, 4, 17, 24]
+    tok[1, :1] = [9]
+    cnt = np.array([5, 1], np.int32)
+    o, l = oracle.attn_decode_gqa_sparse(q, k, v, tok, cnt, 0.4)
+    for b in range(B):
+        keep = np.zeros(T, bool)
+        keep[tok[b, :cnt[b]]] = True
+        for h in range(H):
+            sc = 0.4 * k[b, h // 2] @ q[b, h]
+            sc[~keep] = -np.inf
+            p = np.exp(sc - sc.max())
+            np.testing.assert_allclose(o[b, h], (p / p.sum()) @ v[b, h // 2], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(l[b, h], sc.max() + np.log(p.sum()), rtol=1e-12)
+    np.testing.assert_allclose(o[1], v[1, np.arange(H) // 2, 9], rtol=1e-14)
