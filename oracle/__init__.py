@@ -387,13 +387,14 @@ def qsa_select(q_idx, w, block_keys, lens, n_top, scores=None):
 def attn_decode_gqa_sparse(q, k, v, tok_idx, tok_count, scale):
     """GQA decode over the listed tokens of a linear cache: the plain decode
     definition over the gathered rows of each sequence (the first tok_count[b]
-    entries of tok_idx[b]).  q [B,H,d], k/v [B,Hk,T,d] -> (out, lse)."""
+    entries of tok_idx[b]; an entry -1 marks an unused slot, as in the sparse
+    latent decode, and is skipped).  q [B,H,d], k/v [B,Hk,T,d] -> (out, lse)."""
     B, H, d = np.shape(q)
     out = np.zeros((B, H, d), np.float64)
     lse = np.zeros((B, H), np.float64)
     k, v, q = np.asarray(k), np.asarray(v), np.asarray(q)
     for b in range(B):
-        idx = [int(t) for t in tok_idx[b][:int(tok_count[b])]]
+        idx = [int(t) for t in tok_idx[b][:int(tok_count[b])] if t >= 0]
         n = len(idx)
         kb = k[b:b + 1][:, :, idx] if n else k[b:b + 1][:, :, :1]
         vb = v[b:b + 1][:, :, idx] if n else v[b:b + 1][:, :, :1]

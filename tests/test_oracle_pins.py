@@ -731,3 +731,10 @@ def test_sparse_gqa_against_masked_softmax():
             np.testing.assert_allclose(o[b, h], (p / p.sum()) @ v[b, h // 2], rtol=1e-12, atol=1e-13)
             np.testing.assert_allclose(l[b, h], sc.max() + np.log(p.sum()), rtol=1e-12)
     np.testing.assert_allclose(o[1], v[1, np.arange(H) // 2, 9], rtol=1e-14)
+    # -1 entries are unused slots: the same list with holes gives the same result
+    tok2 = np.full((B, 12), -1, np.int32)
+    tok2[0, :8] = [-1, 0, 3, -1, 4, 17, -1, 24]
+    tok2[1, :3] = [-1, 9, -1]
+    o2, l2 = oracle.attn_decode_gqa_sparse(q, k, v, tok2, np.array([8, 3], np.int32), 0.4)
+    np.testing.assert_array_equal(o2, o)
+    np.testing.assert_array_equal(l2, l)
