@@ -445,6 +445,68 @@ def measure_dsa(K, device, steps, flush, peaks):
             "sparse_gathered_bytes": sp_bytes}
 
 
+def measure_qsa(K, device, steps, flush, peaks):
+    """Block-level indexer decode step (B 8, ragged lengths up to 131072 tokens): the
+    key of the newest 4-token group (qsa_block_keys, one group per row), group scoring
+    + top-512 + expansion with the trailing partial group (qsa_select), then GQA
+    decode (H 32, Hk 8, d 128) over the <= 2051 selected tokens (attn_decode_gqa_sparse)."""
+    w = W.QSA_128K
+    inp = W.qsa_inputs(w, device=device)
+    lens = inp["seq_lens"].to(device)
+    cos, sin = K.rope_table_build(K.rope_params(w.dI, base=w.rope.base), w.L, device=device)
+    kb = K.qsa_block_keys(inp["k_idx"], lens, cos, sin)  # the stored keys of every complete group
+    newest = (lens // 4 - 1).clamp(min=0).to(torch.int32)
+    n_idx = 4 * w.n_top + 3
+    tok = torch.empty((w.B, n_idx), dtype=torch.int32, device=device)
+    cnt = torch.empty(w.B, dtype=torch.int32, device=device)
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty((w.B, w.H), dtype=torch.float32, device=device)
+    ws1 = K.workspace(K.qsa_select_workspace_bytes(w.B, w.L, w.n_top), device)
+    ws2 = K.workspace(K.attn_decode_gqa_sparse_workspace_bytes(w.B, w.H, w.Hk, w.d, n_idx), device)
+
+    def keys_new():
+        K.qsa_block_keys(inp["k_idx"], lens, cos, sin, block_keys=kb, block_from=newest, max_new=1)
+
+    def keys_all():
+        K.qsa_block_keys(inp["k_idx"], lens, cos, sin, block_keys=kb)
+
+    def select():
+        K.qsa_select(inp["q_idx"], inp["w"], kb, lens, n_top=w.n_top, tok_idx=tok, tok_count=cnt, ws=ws1)
+
+    def sparse():
+        K.attn_decode_gqa_sparse(inp["q"], inp["k"], inp["v"], tok, w.scale, tok_count=cnt, out=out, lse=lse, ws=ws2)
+
+    def step():
+        keys_new()
+        select()
+        sparse()
+
+    n = max(10, steps // 5)
+    step_ms = _graph_ms(step, n, flush)
+    select_ms = _graph_ms(select, n, flush)
+    sparse_ms = _graph_ms(sparse, n, flush)
+    keys_ms = _graph_ms(keys_all, n, flush)
+    L = [int(x) for x in inp["seq_lens"]]
+    nb = [x // 4 for x in L]
+    counts = [4 * min(g, w.n_top) + x % 4 for g, x in zip(nb, L)]
+    key_bytes = sum(nb) * w.dI * 2                                    # stored group keys read once
+    kv_bytes = sum(counts) * w.Hk * w.d * 2 * 2                        # gathered K and V rows
+    qo_bytes = w.B * w.H * w.d * 2 * 2 + w.B * w.H * 4
+    step_bytes = key_bytes + kv_bytes + qo_bytes + w.B * (w.HI * w.dI * 2 + w.HI * 4)
+    build_bytes = sum(L) * w.dI * 2 + key_bytes
+    hbm = peaks["hbm_gbs"]
+    return {"workload": w.name, "step_ms": round(step_ms, 4), "tok_per_s": round(w.B / (step_ms * 1e-3), 1),
+            "step_algorithmic_bytes": step_bytes,
+            "step_GB_s": round(step_bytes / (step_ms * 1e-3) / 1e9, 1),
+            "step_pct_of_hbm_peak": round(100 * step_bytes / (step_ms * 1e-3) / 1e9 / hbm, 1),
+            "select_ms": round(select_ms, 4), "group_key_bytes": key_bytes,
+            "sparse_ms": round(sparse_ms, 4), "sparse_gathered_bytes": kv_bytes,
+            "sparse_GB_s": round((kv_bytes + qo_bytes) / (sparse_ms * 1e-3) / 1e9, 1),
+            "sparse_pct_of_hbm_peak": round(100 * (kv_bytes + qo_bytes) / (sparse_ms * 1e-3) / 1e9 / hbm, 1),
+            "block_keys_full_build_ms": round(keys_ms, 4),
+            "block_keys_full_build_GB_s": round(build_bytes / (keys_ms * 1e-3) / 1e9, 1)}
+
+
 def measure_window(K, device, steps, flush, peaks):
     """Llama-3-8B-shaped decode at 32768 tokens over a rolling cache of 4 sinks +
     a 4092-token window (attn_decode_gqa_rope_window): 4096 rows per KV head read."""
@@ -483,6 +545,8 @@ def measure_others(K, device, steps, flush, peaks):
     pw = measure_prefill_window(K, device, steps, flush, peaks)
     res[pw["workload"]] = pw
     res[W.DSA_128K.name] = measure_dsa(K, device, steps, flush, peaks)
+    torch.cuda.empty_cache()
+    res[W.QSA_128K.name] = measure_qsa(K, device, steps, flush, peaks)
     torch.cuda.empty_cache()
     return res
 
@@ -596,7 +660,8 @@ def main():
     ap.add_argument("--impl", default="kvattn", choices=["kvattn", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", action="store_true", help="skip the other configurations")
-    ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "window", "prefill", "prefill_window", "dsa"],
+    ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "window", "prefill", "prefill_window", "dsa",
+                                       "qsa"],
                     help="time one other configuration alone and print its JSON")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -626,6 +691,8 @@ def main():
             res = measure_window(K, device, args.steps, flush, peaks)
         elif args.only == "prefill_window":
             res = measure_prefill_window(K, device, args.steps, flush, peaks)
+        elif args.only == "qsa":
+            res = measure_qsa(K, device, args.steps, flush, peaks)
         else:
             res = measure_dsa(K, device, args.steps, flush, peaks)
         if rank == 0:

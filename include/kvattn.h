@@ -4,12 +4,13 @@
  *
  * Scope: causal attention of new queries over a KV cache, with RoPE applied
  * to q and k only (plain, PI, NTK, YaRN and dynamic-NTK frequency scaling and
- * the YaRN cos/sin temperature), MHA / GQA / MQA head grouping, and the
- * lightning-indexer top-k + sparse latent-row decode.  Sources are cited per
+ * the YaRN cos/sin temperature), MHA / GQA / MQA head grouping, the
+ * lightning-indexer top-k + sparse latent-row decode, and the block-level
+ * (4-token group) indexer + sparse GQA decode.  Sources are cited per
  * entry point by page title and section:
  *   "Agentic RL 入门3：transformer 架构"        (RoPE §1.1-1.2, GQA §2.1, DSA §2.2, MLA §2.3)
  *   "注意力变体与 MoE"                         (KV cache, decode roofline, GQA attention())
- *   "attention"                               (GroupQueryAttention; DSA ①②③)
+ *   "attention"                               (GroupQueryAttention; DSA ①②③; QSA §3)
  *   "注意力机制进化史：从MHA、MQA、GQA、MLA到NSA、MoBA！" (KV cache append, layer_past)
  *
  * Conventions (all entry points):
@@ -315,6 +316,76 @@ int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const in
                        int B, int Hq, int Dk, int Dv, int L_max, int k, float scale,
                        kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
                        int32_t* dev_status, void* stream);
+
+/* ---- block-level indexer over 4-token groups ----------------------------------
+ * "attention" page, "Qwen Sparse Attention (QSA)" §3 ①–④: the visible prefix is
+ * cut into groups of 4 tokens; each complete group gets one block key (the mean of
+ * its 4 indexer keys, normalised, rotated at the group's first position); blocks
+ * are scored like the lightning indexer and the best n_top kept; the kept groups
+ * are unpacked into their 4 token positions and the 0..3 tokens of the trailing
+ * incomplete group are appended; standard GQA attention then runs over those
+ * tokens of the full-precision cache (at most 4 n_top + 3 of them: 2048..2051 for
+ * n_top = 512).  Readings where the section is silent: the normalisation is RMS
+ * without a gain, x / sqrt(mean(x^2) + eps); the rotation is RoPE over all 128
+ * dimensions with the caller's table at position 4j; the lightning indexer's head
+ * weights w are kept (all ones gives the section's plain head sum); one selection
+ * per sequence serves every KV head.
+ *
+ * qsa_block_keys: block key of group j of row b, for j in [block_from[b],
+ * min(seq_lens[b] / 4, block_from[b] + max_new)) -- a decode step that completes a
+ * group builds just that one (block_from = its index, max_new = 1); block_from
+ * NULL = 0; max_new <= 0 = no limit.  k_idx [B][L_max][128] bf16 (the indexer
+ * keys, unrotated); seq_lens device int32 [B] (tokens; outside [0, L_max]: clamped,
+ * KVATTN_STATUS_BAD_LENGTH); cos_tab / sin_tab [max_pos][64] fp32 from
+ * rope_table_build (position 4j >= max_pos: the key is stored unrotated and
+ * KVATTN_STATUS_BAD_POSITION set); pair_style as rope_apply_qk; eps >= 0.
+ * block_keys [B][L_max / 4][128] bf16 (written; other groups untouched).  The
+ * arithmetic is fp32, rounded once to bf16.  Supported: L_max a multiple of 4,
+ * B <= 65535.
+ */
+int qsa_block_keys(const kvattn_bf16* k_idx, const int32_t* seq_lens, const int32_t* block_from, int max_new, int B,
+                   int idx_dim, int L_max, const float* cos_tab, const float* sin_tab, int max_pos, int pair_style,
+                   float eps, kvattn_bf16* block_keys, int32_t* dev_status, void* stream);
+
+/*
+ * qsa_select: score the seq_lens[b] / 4 complete groups of row b, s_j = sum_h
+ * w[b][h] * ReLU(q_idx[b][h] . block_keys[b][j]) in fp32, keep the n_top best
+ * (ties to the lower group; the decision is taken on those fp32 scores) and expand.
+ * q_idx [B][64][128] bf16 (rotated at the query's position by the caller);
+ * w [B][64] fp32; block_keys [B][L_max / 4][128] bf16 (qsa_block_keys);
+ * seq_lens device int32 [B] (tokens).  tok_idx [B][4 n_top + 3] int32: the
+ * selected token positions in increasing order, -1 padded; tok_count [B] int32:
+ * how many (4 min(L / 4, n_top) + L mod 4).  scores_out [B][L_max / 4] fp32 (the
+ * group scores, -inf past each row's groups) or NULL.  workspace:
+ * qsa_select_workspace_bytes(...) bytes, 256-byte aligned, no initialisation.
+ * Supported: 64 indexer heads of width 128, L_max a multiple of 4 with
+ * L_max / 4 <= 131072, 1 <= n_top <= 2048.
+ */
+size_t qsa_select_workspace_bytes(int B, int L_max, int n_top);
+
+int qsa_select(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* block_keys, const int32_t* seq_lens, int B,
+               int n_idx_head, int idx_dim, int L_max, int n_top, int32_t* tok_idx, int32_t* tok_count,
+               float* scores_out, void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * attn_decode_gqa_sparse: attn_decode_gqa over a per-sequence list of cache rows
+ * ("Qwen Sparse Attention (QSA)" ③–④: the selected tokens' K and V are fetched
+ * from the full cache by index, then softmax(scale q K_sel^T) V_sel per query head,
+ * query head h reading KV head h / g).  tok_idx [B][n_idx] int32 cache rows (any
+ * order); the first tok_count[b] entries of row b are used (tok_count device int32
+ * [B], or NULL = all n_idx; a count outside [0, n_idx] is clamped and sets
+ * KVATTN_STATUS_BAD_LENGTH); an entry -1 is skipped, any other entry outside
+ * [0, T_max) is skipped and sets KVATTN_STATUS_BAD_INDEX.  A sequence with no used
+ * row gives out = 0, lse = -inf.  q, k_cache, v_cache, out, lse, workspace and its
+ * zero counter region as attn_decode_gqa (attn_decode_gqa_sparse_workspace_bytes).
+ * Supported: head_dim 64 (g <= 64) or 128 (g <= 32), g as attn_decode_gqa.
+ */
+size_t attn_decode_gqa_sparse_workspace_bytes(int B, int n_head, int n_kv_head, int head_dim, int n_idx);
+
+int attn_decode_gqa_sparse(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
+                           const int32_t* tok_idx, const int32_t* tok_count, int n_idx, int B, int n_head,
+                           int n_kv_head, int head_dim, int T_max, float scale, kvattn_bf16* out, float* lse,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -260,14 +260,27 @@ struct DecodeRope {
     int max_pos, pair_style;
 };
 
+struct DecodeGather {
+    const int32_t* idx;  // [B][n_idx] cache rows; the row counts come in seq_lens (may be NULL)
+    int n_idx;
+};
+
 static int decode_call(const char* name, const kvattn_bf16* q, const kvattn_bf16* k_cache,
                        const kvattn_bf16* v_cache, const int32_t* seq_lens, int B, int n_head, int n_kv_head,
                        int head_dim, int T_max, float scale, kvattn_bf16* out, float* lse, void* workspace,
                        size_t workspace_bytes, int32_t* dev_status, void* stream, const DecodeRope* rope,
-                       int len_cap = 0)
+                       int len_cap = 0, const DecodeGather* gather = nullptr)
 {
-    if (!q || !k_cache || !v_cache || !seq_lens || !out)
+    if (!q || !k_cache || !v_cache || (!seq_lens && !gather) || !out)
         return fail(KVATTN_ERR_NULL, "%s: NULL argument", name);
+    if (gather) {
+        if (!gather->idx) return fail(KVATTN_ERR_NULL, "%s: NULL index list", name);
+        if (gather->n_idx < 1) return fail(KVATTN_ERR_SHAPE, "%s: n_idx %d", name, gather->n_idx);
+        if (head_dim == 128 && n_head > 32 * n_kv_head)
+            return fail(KVATTN_ERR_UNSUPPORTED, "%s: group size above 32 at head_dim 128", name);
+        if (static_cast<long long>(B) * gather->n_idx > (1ll << 31))
+            return fail(KVATTN_ERR_SHAPE, "%s: B * n_idx too large", name);
+    }
     if (B < 1 || B > kvattn::DECODE_MAX_B) return fail(KVATTN_ERR_SHAPE, "%s: B %d outside 1..%d", name, B, kvattn::DECODE_MAX_B);
     if (n_head < 1 || n_kv_head < 1 || n_head % n_kv_head)
         return fail(KVATTN_ERR_SHAPE, "%s: n_head %d not a multiple of n_kv_head %d", name, n_head, n_kv_head);
@@ -318,6 +331,12 @@ static int decode_call(const char* name, const kvattn_bf16* q, const kvattn_bf16
     a.unit_cnt = reinterpret_cast<int*>(w);
     a.dev_status = dev_status;
     a.len_cap = len_cap;
+    if (gather) {
+        a.idx = gather->idx;
+        a.n_idx = gather->n_idx;
+        a.k_cache = k_cache;
+        a.v_cache = v_cache;
+    }
     if (rope) {
         a.q_pos = rope->q_pos;
         a.cos_tab = rope->cos_tab;
@@ -370,6 +389,21 @@ int attn_decode_gqa_rope_window(const kvattn_bf16* q, const int32_t* q_pos, cons
     const DecodeRope r{q_pos, cos_tab, sin_tab, max_pos, pair_style};
     return decode_call("attn_decode_gqa_rope_window", q, k_cache, v_cache, seq_lens, B, n_head, n_kv_head, head_dim,
                        T_max, scale, out, lse, workspace, workspace_bytes, dev_status, stream, &r, n_sink + window);
+}
+
+size_t attn_decode_gqa_sparse_workspace_bytes(int B, int n_head, int n_kv_head, int head_dim, int n_idx)
+{
+    return attn_decode_gqa_workspace_bytes(B, n_head, n_kv_head, head_dim, n_idx);
+}
+
+int attn_decode_gqa_sparse(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
+                           const int32_t* tok_idx, const int32_t* tok_count, int n_idx, int B, int n_head,
+                           int n_kv_head, int head_dim, int T_max, float scale, kvattn_bf16* out, float* lse,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    const DecodeGather gth{tok_idx, n_idx};
+    return decode_call("attn_decode_gqa_sparse", q, k_cache, v_cache, tok_count, B, n_head, n_kv_head, head_dim,
+                       T_max, scale, out, lse, workspace, workspace_bytes, dev_status, stream, nullptr, 0, &gth);
 }
 
 // ---------------------------------------------------------------------------
@@ -502,6 +536,89 @@ int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* 
     kvattn::DsaIndexArgs a{w, seq_lens, scores, topk_idx, dev_status, B, L_max, k, sms};
     return cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, static_cast<cudaStream_t>(stream)),
                        "dsa_index_topk launch");
+}
+
+// ---------------------------------------------------------------------------
+int qsa_block_keys(const kvattn_bf16* k_idx, const int32_t* seq_lens, const int32_t* block_from, int max_new, int B,
+                   int idx_dim, int L_max, const float* cos_tab, const float* sin_tab, int max_pos, int pair_style,
+                   float eps, kvattn_bf16* block_keys, int32_t* dev_status, void* stream)
+{
+    if (!k_idx || !seq_lens || !cos_tab || !sin_tab || !block_keys)
+        return fail(KVATTN_ERR_NULL, "qsa_block_keys: NULL argument");
+    if (idx_dim != 128) return fail(KVATTN_ERR_UNSUPPORTED, "qsa_block_keys: idx_dim %d (needs 128)", idx_dim);
+    if (B < 1 || L_max < kvattn::QSA_BLOCK || L_max % kvattn::QSA_BLOCK)
+        return fail(KVATTN_ERR_SHAPE, "qsa_block_keys: B %d, L_max %d (a positive multiple of 4)", B, L_max);
+    if (B > 65535) return fail(KVATTN_ERR_SHAPE, "qsa_block_keys: B %d above 65535", B);
+    if (max_pos < 1) return fail(KVATTN_ERR_SHAPE, "qsa_block_keys: max_pos < 1");
+    if (pair_style != 0 && pair_style != 1) return fail(KVATTN_ERR_UNSUPPORTED, "qsa_block_keys: pair_style");
+    if (!(eps >= 0.0f) || !std::isfinite(eps)) return fail(KVATTN_ERR_SHAPE, "qsa_block_keys: eps must be finite >= 0");
+    if (!aligned16(k_idx) || !aligned16(block_keys) || !aligned16(cos_tab) || !aligned16(sin_tab))
+        return fail(KVATTN_ERR_ALIGN, "qsa_block_keys: tensors must be 16-byte aligned");
+    kvattn::QsaKeysArgs a{};
+    a.k_idx = k_idx;
+    a.seq_lens = seq_lens;
+    a.block_from = block_from;
+    a.cos_tab = cos_tab;
+    a.sin_tab = sin_tab;
+    a.block_keys = block_keys;
+    a.dev_status = dev_status;
+    a.B = B;
+    a.L_max = L_max;
+    a.max_pos = max_pos;
+    a.pair_style = pair_style;
+    a.max_new = max_new > 0 ? max_new : L_max / kvattn::QSA_BLOCK;
+    a.eps = eps;
+    return cuda_status(kvattn::launch_qsa_block_keys(a, static_cast<cudaStream_t>(stream)), "qsa_block_keys launch");
+}
+
+static size_t qsa_scores_bytes(int B, int L_max) { return align_up(kvattn::dsa_scores_bytes(B, L_max / kvattn::QSA_BLOCK)); }
+static size_t qsa_blocks_bytes(int B, int n_top) { return align_up(static_cast<size_t>(B) * n_top * sizeof(int32_t)); }
+
+size_t qsa_select_workspace_bytes(int B, int L_max, int n_top)
+{
+    if (B < 1 || L_max < kvattn::QSA_BLOCK || n_top < 1) return 0;
+    return qsa_scores_bytes(B, L_max) + qsa_blocks_bytes(B, n_top);
+}
+
+int qsa_select(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* block_keys, const int32_t* seq_lens, int B,
+               int n_idx_head, int idx_dim, int L_max, int n_top, int32_t* tok_idx, int32_t* tok_count,
+               float* scores_out, void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    if (!q_idx || !w || !block_keys || !seq_lens || !tok_idx || !tok_count)
+        return fail(KVATTN_ERR_NULL, "qsa_select: NULL argument");
+    if (n_idx_head != 64 || idx_dim != 128)
+        return fail(KVATTN_ERR_UNSUPPORTED, "qsa_select: needs 64 indexer heads of width 128 (got %d x %d)", n_idx_head,
+                    idx_dim);
+    if (B < 1 || L_max < kvattn::QSA_BLOCK || L_max % kvattn::QSA_BLOCK || n_top < 1 || n_top > 2048)
+        return fail(KVATTN_ERR_SHAPE, "qsa_select: B %d, L_max %d (a positive multiple of 4), n_top %d (1..2048)", B,
+                    L_max, n_top);
+    const int nb_max = L_max / kvattn::QSA_BLOCK;
+    if (nb_max > 131072) return fail(KVATTN_ERR_UNSUPPORTED, "qsa_select: L_max %d above 4 * 131072", L_max);
+    if (static_cast<long long>(B) * L_max > (1ll << 31)) return fail(KVATTN_ERR_SHAPE, "qsa_select: B * L_max too large");
+    if (!aligned16(q_idx) || !aligned16(block_keys) || !aligned16(w) || !aligned16(tok_idx) ||
+        (scores_out && !aligned16(scores_out)))
+        return fail(KVATTN_ERR_ALIGN, "qsa_select: tensors must be 16-byte aligned");
+    const size_t need = qsa_select_workspace_bytes(B, L_max, n_top);
+    if (!workspace || workspace_bytes < need)
+        return fail(KVATTN_ERR_WORKSPACE, "qsa_select: workspace needs %zu bytes", need);
+    if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
+        return fail(KVATTN_ERR_ALIGN, "qsa_select: workspace must be 256-byte aligned");
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* scores = scores_out ? scores_out : reinterpret_cast<float*>(ws);
+    int32_t* blk = reinterpret_cast<int32_t*>(ws + qsa_scores_bytes(B, L_max));
+    int sms = 0;
+    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "qsa_select: no CUDA device");
+    CUtensorMap tm_k, tm_q;
+    if (make_map_3d(&tm_k, block_keys, 128, nb_max, B, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_3d(&tm_q, q_idx, 128, 64, B, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    kvattn::DsaIndexArgs a{w, seq_lens, scores, blk, dev_status, B, nb_max, n_top, sms};
+    static_assert(kvattn::QSA_BLOCK == 4, "len_shift below is log2 of the group size");
+    a.len_shift = 2;  // a row of L tokens has L / 4 complete groups
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int rc = cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, st), "qsa_select block scoring");
+    if (rc != KVATTN_OK) return rc;
+    kvattn::QsaExpandArgs e{blk, seq_lens, tok_idx, tok_count, dev_status, B, L_max, n_top};
+    return cuda_status(kvattn::launch_qsa_expand(e, st), "qsa_select expand");
 }
 
 size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k)

@@ -22,6 +22,14 @@
 // mma.sync m16n8k16 with the query heads of the group as the M rows (a group
 // of g <= 16 heads is one M tile, zero-padded; g = 32/64 use 2/4 M tiles),
 // fp32 accumulation, online softmax in base 2 with quad shuffles.
+//
+// Gather mode (a sparse token list per sequence, "attention" page, "Qwen Sparse
+// Attention (QSA)" ③–④: the selected tokens' full-precision K/V are fetched from
+// the cache by index and standard GQA attention runs over them): a unit's rows
+// are the listed cache rows.  The whole producer warp gathers each tile with
+// 16-byte cp.async (a 256-byte row = 16 lanes) into the same swizzled layout the
+// tensor map writes, with one asynchronous arrival per lane on the stage barrier,
+// and passes the tile's valid-row bitmask (skipped entries, the tail) along.
 #include <type_traits>
 
 #include "common.cuh"
@@ -56,7 +64,8 @@ struct Cfg {
     static constexpr int OFF_LEN = OFF_UB + (DECODE_MAX_B + 1) * 4;
     static constexpr int OFF_BAR = ((OFF_LEN + DECODE_MAX_B * 4) + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
-    static constexpr int SMEM = OFF_MISC + 64 + 1024;  // + alignment slack
+    static constexpr int OFF_MASK = OFF_MISC + 64;                  // [STAGES] valid rows (gather mode)
+    static constexpr int SMEM = OFF_MASK + STAGES * 8 + 1024;  // + alignment slack
     static_assert(SMEM <= 232448, "shared memory");
 };
 
@@ -148,7 +157,8 @@ __device__ void merge_unit(const DecodeArgs& a, int u, int S, int count, int tid
 #pragma unroll
             for (int j = 0; j < MERGE_MAX_BATCH; ++j) {
                 if (j0 + j < count) {
-                    const float e = fast_exp2(mlv[j].x - M);
+                    // a piece whose rows were all skipped (gather mode) has m = -inf, l = 0
+                    const float e = mlv[j].x == -INFINITY ? 0.f : fast_exp2(mlv[j].x - M);
                     L += e * mlv[j].y;
                     acc.x += e * ov[j].x;
                     acc.y += e * ov[j].y;
@@ -157,16 +167,18 @@ __device__ void merge_unit(const DecodeArgs& a, int u, int S, int count, int tid
                 }
             }
         }
-        const float inv = 1.f / L;
+        const float inv = L > 0.f ? 1.f / L : 0.f;
         *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(a.out) + (bh0 + h) * D + 4 * q4) =
             make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-        if (q4 == 0 && a.lse) a.lse[bh0 + h] = (M + __log2f(L)) * kLn2;
+        if (q4 == 0 && a.lse) a.lse[bh0 + h] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
     }
 }
 
 // ---- the decode kernel ---------------------------------------------------------
 
-template <int D, int NMT>
+static_assert(TILE == 64, "gather mode passes a tile's valid rows as one 64-bit mask");
+
+template <int D, int NMT, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, DecodeArgs a)
 {
@@ -196,11 +208,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     int* s_misc = reinterpret_cast<int*>(smem + C::OFF_MISC);
     volatile int* s_abort = s_misc + 1;
     int* s_merge = s_misc + 4;  // [0] = split pieces made here, then (unit, first slot, pieces) x 2
+    uint64_t* s_mask = reinterpret_cast<uint64_t*>(smem + C::OFF_MASK);  // valid rows of each stage (gather)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            // gather mode: one cp.async arrival per producer lane + the lane-0 arrival with the mask
+            mbar_init(&full[s], GATHER ? 33 : 1);
             mbar_init(&empty[s], CWARPS);
         }
         mbar_init(q_full, 1);
@@ -209,15 +223,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         s_merge[0] = 0;
         fence_barrier_init();
     }
-    if (warp == CWARPS && lane == 0) {
+    if (!GATHER && warp == CWARPS && lane == 0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
     // everything above overlaps the previous kernel of the stream
     pdl_wait();
     pdl_trigger();
-    const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, a.T_max, s_len, s_n, s_Ub, a.dev_status,
-                                    blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos,
+    const long long N = plan_prefix(a.seq_lens, a.B, a.Hk, GATHER ? a.n_idx : a.T_max, s_len, s_n, s_Ub,
+                                    a.dev_status, blockIdx.x == 0, rope ? a.q_pos : nullptr, s_qpos,
                                     a.len_cap);
     // empty sequences have no tiles: their heads get zeros and lse = -inf here
     for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
@@ -240,59 +254,117 @@ __global__ void __launch_bounds__(THREADS, 1)
     w_start.S = slots_before(w_start.b * a.Hk + w_start.kvh, a.Hk, s_n, s_Ub, N, G, s_misc + 2);
 
     if (warp == CWARPS) {
-        // ===== producer: one thread streams K/V tiles of every piece in order =====
-        if (lane != 0) return;
+        // ===== producer: streams K/V tiles of every piece in order (one thread with
+        // the tensor maps; the whole warp in gather mode) =====
+        if (!GATHER && lane != 0) return;
         Walk w = w_start;
         int it = 0, np = 0;
         bool ok = true;
         const uint32_t q_bytes = static_cast<uint32_t>(a.g) * D * 2;
+        constexpr int CPR = D / 8;     // 16-byte chunks of a row (gather mode)
+        constexpr int RPI = 32 / CPR;  // rows per warp-wide copy instruction
+        const int my_r = lane / CPR, my_ch = lane % CPR;
+        const uint32_t my_dst = (my_ch >> 3) * (TILE * 128);
         for (; ok && w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
             long long tb, te;
             if (!piece_tiles(w, s_n[w.b], lo, hi, tb, te)) continue;
             const int z = w.b * a.Hk + w.kvh;
             // the piece's g query rows (contiguous), once the consumers hold the previous ones
-            if (np > 0 && (*s_abort || !mbar_wait(q_empty, (np - 1) & 1))) {
-                ok = false;
-                break;
+            if (np > 0) {
+                const bool got = GATHER ? warp_wait(q_empty, (np - 1) & 1, s_abort)
+                                        : (!*s_abort && mbar_wait(q_empty, (np - 1) & 1));
+                if (!got) {
+                    ok = false;
+                    break;
+                }
             }
             // with RoPE, the cos and sin rows of the query's position come along
-            const int qp = rope ? s_qpos[w.b] : -1;
-            const bool rot = rope && qp >= 0 && qp < a.max_pos;
-            mbar_arrive_expect_tx(q_full, q_bytes + (rot ? D * 4 : 0));
-            bulk_load(sQ, a.q + (static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g) * D, q_bytes,
-                      q_full);
-            if (rot) {
-                bulk_load(sCos, a.cos_tab + static_cast<long long>(qp) * (D / 2), D * 2, q_full);
-                bulk_load(sSin, a.sin_tab + static_cast<long long>(qp) * (D / 2), D * 2, q_full);
+            if (lane == 0) {
+                const int qp = rope ? s_qpos[w.b] : -1;
+                const bool rot = rope && qp >= 0 && qp < a.max_pos;
+                mbar_arrive_expect_tx(q_full, q_bytes + (rot ? D * 4 : 0));
+                bulk_load(sQ, a.q + (static_cast<long long>(w.b) * a.H + static_cast<long long>(w.kvh) * a.g) * D,
+                          q_bytes, q_full);
+                if (rot) {
+                    bulk_load(sCos, a.cos_tab + static_cast<long long>(qp) * (D / 2), D * 2, q_full);
+                    bulk_load(sSin, a.sin_tab + static_cast<long long>(qp) * (D / 2), D * 2, q_full);
+                }
             }
             ++np;
+            // gather mode: this lane holds the row indices of rows `lane` and `lane + 32` of
+            // the next tile (-1 past the unit's count), loaded one tile ahead
+            const int cnt = s_len[w.b];
+            const int32_t* irow = GATHER ? a.idx + static_cast<long long>(w.b) * a.n_idx : nullptr;
+            int nia = -1, nib = -1;
+            if (GATHER) {
+                const int ra = static_cast<int>(tb) * TILE + lane;
+                nia = ra < cnt ? __ldg(irow + ra) : -1;
+                nib = ra + 32 < cnt ? __ldg(irow + ra + 32) : -1;
+            }
             for (long long t = tb; t < te; ++t, ++it) {
                 const int s = it % C::STAGES;
                 const uint32_t ph = (it / C::STAGES) & 1;
                 if (it >= C::STAGES) {
-                    if (*s_abort || !mbar_wait(&empty[s], ph ^ 1)) {
+                    const bool got = GATHER ? warp_wait(&empty[s], ph ^ 1, s_abort)
+                                            : (!*s_abort && mbar_wait(&empty[s], ph ^ 1));
+                    if (!got) {
                         ok = false;
                         break;
                     }
                 }
-                mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
                 uint8_t* kd = smem + s * C::STAGE_BYTES;
                 uint8_t* vd = kd + C::TILE_BYTES;
+                if constexpr (!GATHER) {
+                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
 #pragma unroll
-                for (int h = 0; h < C::HALVES; ++h) {
-                    tma_load_3d(kd + h * (TILE * 128), &tm_k, &full[s], h * 64, static_cast<int>(t * TILE), z);
-                    tma_load_3d(vd + h * (TILE * 128), &tm_v, &full[s], h * 64, static_cast<int>(t * TILE), z);
+                    for (int h = 0; h < C::HALVES; ++h) {
+                        tma_load_3d(kd + h * (TILE * 128), &tm_k, &full[s], h * 64, static_cast<int>(t * TILE), z);
+                        tma_load_3d(vd + h * (TILE * 128), &tm_v, &full[s], h * 64, static_cast<int>(t * TILE), z);
+                    }
+                } else {
+                    const int ia = nia, ib = nib;
+                    if (t + 1 < te) {
+                        const int ra = static_cast<int>(t + 1) * TILE + lane;
+                        nia = ra < cnt ? __ldg(irow + ra) : -1;
+                        nib = ra + 32 < cnt ? __ldg(irow + ra + 32) : -1;
+                    }
+                    const bool va = ia >= 0 && ia < a.T_max, vb = ib >= 0 && ib < a.T_max;
+                    if (ia < -1 || ia >= a.T_max || ib < -1 || ib >= a.T_max)
+                        report_status(a.dev_status, KVATTN_STATUS_BAD_INDEX);
+                    const uint32_t ma = __ballot_sync(0xffffffffu, va), mb = __ballot_sync(0xffffffffu, vb);
+                    const kvattn_bf16* kz = a.k_cache + static_cast<long long>(z) * a.T_max * D + my_ch * 8;
+                    const kvattn_bf16* vz = a.v_cache + static_cast<long long>(z) * a.T_max * D + my_ch * 8;
+                    const uint32_t sk = smem_u32(kd) + my_dst, sv = smem_u32(vd) + my_dst;
+#pragma unroll 8
+                    for (int i = 0; i < TILE / RPI; ++i) {
+                        const int r = i * RPI + my_r;  // row of the tile this lane copies a chunk of
+                        const int row = __shfl_sync(0xffffffffu, i * RPI < 32 ? ia : ib, r & 31);
+                        if (((r < 32 ? ma >> r : mb >> (r - 32)) & 1u) != 0u) {
+                            const long long off = static_cast<long long>(row) * D;
+                            const uint32_t so = swz128(r, my_ch & 7);
+                            cp_async16(sk + so, kz + off, 16);
+                            cp_async16(sv + so, vz + off, 16);
+                        }
+                    }
+                    cp_async_arrive_noinc(&full[s]);
+                    if (lane == 0) {
+                        s_mask[s] = (static_cast<uint64_t>(mb) << 32) | ma;
+                        mbar_arrive(&full[s]);
+                    }
                 }
             }
         }
-        if (!ok) {
+        if (!ok && lane == 0) {
             *s_abort = 1;
             report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
         }
         // copies still in flight complete before the CTA leaves (bounded waits)
-        for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
-            mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
-        if (np > 0) mbar_wait(q_full, (np - 1) & 1);
+        if (GATHER) cp_async_wait<0>();
+        if (lane == 0) {
+            for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
+                mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
+            if (np > 0) mbar_wait(q_full, (np - 1) & 1);
+        }
         return;
     }
 
@@ -360,6 +432,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t sK = smem_u32(smem + s * C::STAGE_BYTES);
                 const uint32_t sV = sK + C::TILE_BYTES;
                 const int n_valid = len - static_cast<int>(t) * TILE;  // >= 1
+                // gather mode: bit r set = row r of the tile holds a listed cache row
+                const uint64_t vm = GATHER ? s_mask[s] : ~0ull;
 
                 // ---- S = Q K^T over this warp's rows of the tile ----
                 float sc[NT][4];
@@ -388,7 +462,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         float v = sc[i][e] * sl2;
-                        if (tk + (e & 1) >= n_valid) v = -INFINITY;
+                        if (GATHER ? ((vm >> (tk + (e & 1))) & 1ull) == 0ull : tk + (e & 1) >= n_valid)
+                            v = -INFINITY;
                         sc[i][e] = v;
                     }
                     mx0 = fmaxf(mx0, fmaxf(sc[i][0], sc[i][1]));
@@ -424,7 +499,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     o[i][3] *= al1;
                 }
                 // ---- O += P V ----
-                const bool tail = n_valid < TILE;
+                const bool tail = GATHER ? vm != ~0ull : n_valid < TILE;
 #pragma unroll
                 for (int j = 0; j < TPW / 16; ++j) {
                     uint32_t pa[4];
@@ -443,9 +518,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                         if (tail) {
                             // rows past the length may hold anything (NaN included):
                             // zero them so that 0 * garbage cannot reach the sum
-                            const uint32_t k0 = (vt < n_valid ? 0x0000ffffu : 0u) | (vt + 1 < n_valid ? 0xffff0000u : 0u);
-                            const uint32_t k1 =
-                                (vt + 8 < n_valid ? 0x0000ffffu : 0u) | (vt + 9 < n_valid ? 0xffff0000u : 0u);
+                            uint32_t k0, k1;
+                            if constexpr (GATHER) {
+                                const uint32_t bits = static_cast<uint32_t>(vm >> vt);
+                                k0 = ((bits & 1u) ? 0x0000ffffu : 0u) | ((bits & 2u) ? 0xffff0000u : 0u);
+                                k1 = ((bits & 0x100u) ? 0x0000ffffu : 0u) | ((bits & 0x200u) ? 0xffff0000u : 0u);
+                            } else {
+                                k0 = (vt < n_valid ? 0x0000ffffu : 0u) | (vt + 1 < n_valid ? 0xffff0000u : 0u);
+                                k1 = (vt + 8 < n_valid ? 0x0000ffffu : 0u) | (vt + 9 < n_valid ? 0xffff0000u : 0u);
+                            }
                             v0 &= k0;
                             v2 &= k0;
                             v1 &= k1;
@@ -508,7 +589,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const long long pi = static_cast<long long>(slot) * g + row;
                     a.part_o[pi * D + dim] = acc;
                     if (dim == 0) {
-                        a.part_ml[pi * 2] = Mu;
+                        a.part_ml[pi * 2] = M;  // -inf only for a piece whose rows were all skipped
                         a.part_ml[pi * 2 + 1] = L;
                     }
                 }
@@ -644,7 +725,7 @@ __global__ void __launch_bounds__(MERGE_WARPS * 32) decode_combine_kernel(Decode
     if (lane == 0 && a.lse) a.lse[bh] = (M + __log2f(L)) * kLn2;
 }
 
-template <int D, int NMT>
+template <int D, int NMT, bool GATHER>
 cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_v,
                          cudaStream_t stream)
 {
@@ -653,13 +734,14 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tm_k, const CUt
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(decode_kernel<D, NMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(decode_kernel<D, NMT, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<D, NMT>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
     // split units are merged inside the kernel, by the CTA that finishes their last piece
-    return launch_pdl(decode_kernel<D, NMT>, dim3(a.grid), dim3(THREADS), Cfg<D, NMT>::SMEM, stream, tm_k, tm_v, a);
+    return launch_pdl(decode_kernel<D, NMT, GATHER>, dim3(a.grid), dim3(THREADS), Cfg<D, NMT>::SMEM, stream, tm_k,
+                      tm_v, a);
 }
 
 }  // namespace
@@ -681,16 +763,27 @@ int decode_grid(int num_sms) { return num_sms; }
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& tm_q, const CUtensorMap& tm_k,
                           const CUtensorMap& tm_v, cudaStream_t stream)
 {
-    if (decode_tc_supported(a.d, a.g)) return launch_decode_tc(a, tm_q, tm_k, tm_v, stream);
     const int nmt = a.g <= 16 ? 1 : (a.g <= 32 ? 2 : 4);
-    if (a.d == 128) {
-        if (nmt == 1) return launch_typed<128, 1>(a, tm_k, tm_v, stream);
-        // g = 64 at d = 128 is the tcgen05 kernel's
-        return launch_typed<128, 2>(a, tm_k, tm_v, stream);
+    if (a.idx) {
+        // gather mode: the mma.sync kernel (g <= 32 at d = 128)
+        if (a.d == 128) {
+            if (nmt == 1) return launch_typed<128, 1, true>(a, tm_k, tm_v, stream);
+            if (nmt == 2) return launch_typed<128, 2, true>(a, tm_k, tm_v, stream);
+            return cudaErrorInvalidValue;
+        }
+        if (nmt == 1) return launch_typed<64, 1, true>(a, tm_k, tm_v, stream);
+        if (nmt == 2) return launch_typed<64, 2, true>(a, tm_k, tm_v, stream);
+        return launch_typed<64, 4, true>(a, tm_k, tm_v, stream);
     }
-    if (nmt == 1) return launch_typed<64, 1>(a, tm_k, tm_v, stream);
-    if (nmt == 2) return launch_typed<64, 2>(a, tm_k, tm_v, stream);
-    return launch_typed<64, 4>(a, tm_k, tm_v, stream);
+    if (decode_tc_supported(a.d, a.g)) return launch_decode_tc(a, tm_q, tm_k, tm_v, stream);
+    if (a.d == 128) {
+        if (nmt == 1) return launch_typed<128, 1, false>(a, tm_k, tm_v, stream);
+        // g = 64 at d = 128 is the tcgen05 kernel's
+        return launch_typed<128, 2, false>(a, tm_k, tm_v, stream);
+    }
+    if (nmt == 1) return launch_typed<64, 1, false>(a, tm_k, tm_v, stream);
+    if (nmt == 2) return launch_typed<64, 2, false>(a, tm_k, tm_v, stream);
+    return launch_typed<64, 4, false>(a, tm_k, tm_v, stream);
 }
 
 }  // namespace kvattn

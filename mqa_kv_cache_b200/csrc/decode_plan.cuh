@@ -39,6 +39,7 @@ __device__ __forceinline__ int unit_count(long long U, int n, long long N, int G
 // Returns N = Hk * s_Ub[B].
 // With q_pos non-null, s_qpos[b] = q_pos[b] too (read in the same round trip).
 // With len_cap > 0 a length counts as min(len, len_cap) rows (a rolling cache).
+// With seq_lens null every row has T_max rows.
 __device__ long long plan_prefix(const int32_t* __restrict__ seq_lens, int B, int Hk, int T_max, int* s_len,
                                  int* s_n, int* s_Ub, int32_t* dev_status, bool report,
                                  const int32_t* __restrict__ q_pos = nullptr, int* s_qpos = nullptr,
@@ -46,7 +47,7 @@ __device__ long long plan_prefix(const int32_t* __restrict__ seq_lens, int B, in
 {
     for (int b = threadIdx.x; b < B; b += blockDim.x) {
         if (q_pos) s_qpos[b] = q_pos[b];
-        const int len_raw = seq_lens[b];
+        const int len_raw = seq_lens ? seq_lens[b] : T_max;
         const int len = (len_cap > 0 && len_raw > len_cap) ? len_cap : len_raw;
         const int lc = min(max(len, 0), T_max);
         if (lc != len && report) report_status(dev_status, KVATTN_STATUS_BAD_LENGTH);

@@ -55,6 +55,7 @@ struct IndexerArgs {
     float* scores;
     int32_t* dev_status;
     int B, L_max, tiles_per_b, chunks_per_b;
+    int len_shift;  // row b scores seq_lens[b] >> len_shift keys (2: 4-token groups)
 };
 
 __device__ __forceinline__ void ix_item(const IndexerArgs& a, int item, int& b, int& t0, int& t1)
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
             int b, t0, t1;
             ix_item(a, item, b, t0, t1);
-            const int len_raw = a.seq_lens ? a.seq_lens[b] : a.L_max;
+            const int len_raw = a.seq_lens ? (a.seq_lens[b] >> a.len_shift) : a.L_max;
             const int len = min(max(len_raw, 0), a.L_max);
             if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
             named_bar_sync(2, 128);
@@ -285,6 +286,7 @@ struct TopkArgs {
     int32_t* out;
     int32_t* dev_status;
     int L_max, k;
+    int len_shift;
 };
 
 constexpr int TK_SLICE_MAX = 16384;  // keys per CTA held in shared memory
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     pdl_wait();
     pdl_trigger();
 
-    const int len_raw = a.seq_lens ? a.seq_lens[row] : a.L_max;
+    const int len_raw = a.seq_lens ? (a.seq_lens[row] >> a.len_shift) : a.L_max;
     const int len = min(max(len_raw, 0), a.L_max);
     if (len != len_raw && rank == 0 && tid == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
     const int kk = min(a.k, len);
@@ -453,6 +455,7 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     ia.dev_status = a.dev_status;
     ia.B = a.B;
     ia.L_max = a.L_max;
+    ia.len_shift = a.len_shift;
     ia.tiles_per_b = (a.L_max + IX_TOK - 1) / IX_TOK;
     // about two contiguous chunks per CTA, never more chunks than tiles
     int chunks = (2 * a.num_sms + a.B - 1) / a.B;
@@ -464,7 +467,7 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     e = launch_pdl(indexer_kernel, dim3(grid), dim3(IX_THREADS), IX_SMEM, stream, tm_k, tm_q, ia);
     if (e != cudaSuccess) return e;
 
-    TopkArgs ta{a.scores, a.seq_lens, a.topk_idx, a.dev_status, a.L_max, a.k};
+    TopkArgs ta{a.scores, a.seq_lens, a.topk_idx, a.dev_status, a.L_max, a.k, a.len_shift};
     const int slice_max = (a.L_max + TK_CL - 1) / TK_CL;
     const size_t key_bytes = static_cast<size_t>(slice_max + (slice_max >> 4) + 1) * sizeof(uint32_t);
     static bool tk_attr[64] = {};

@@ -88,6 +88,13 @@ struct DecodeArgs {
     int max_pos, pair_style;
     int len_cap;           // > 0: a sequence of length len uses min(len, len_cap) cache rows
                            // (a rolling cache holding the sinks and the window)
+    // Gather mode (idx non-null): the rows of unit (b, kv-head) are the cache rows
+    // idx[b][0 .. n_b - 1], n_b = seq_lens[b] (n_idx when seq_lens is null); an
+    // entry outside [0, T_max) is skipped (-1 silently, any other value flagged).
+    const int32_t* idx;    // [B][n_idx]
+    int n_idx;
+    const kvattn_bf16* k_cache;  // [B][Hk][T_max][d], read by row in gather mode
+    const kvattn_bf16* v_cache;
     int32_t* dev_status;
     int B, H, Hk, g, d, T_max;
     float scale;
@@ -114,10 +121,35 @@ struct DsaIndexArgs {
     int32_t* topk_idx;  // [B][k]
     int32_t* dev_status;
     int B, L_max, k, num_sms;
+    int len_shift = 0;  // row b has seq_lens[b] >> len_shift keys (2: the 4-token block keys)
 };
 size_t dsa_scores_bytes(int B, int L_max);
 cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                                   cudaStream_t stream);
+
+// ---- block-level indexer (4-token groups) ----
+constexpr int QSA_BLOCK = 4;
+struct QsaKeysArgs {
+    const kvattn_bf16* k_idx;   // [B][L_max][128]
+    const int32_t* seq_lens;    // [B] tokens
+    const int32_t* block_from;  // [B] first block to build, or null (0)
+    const float* cos_tab;
+    const float* sin_tab;
+    kvattn_bf16* block_keys;    // [B][L_max / 4][128]
+    int32_t* dev_status;
+    int B, L_max, max_pos, pair_style, max_new;
+    float eps;
+};
+cudaError_t launch_qsa_block_keys(const QsaKeysArgs& a, cudaStream_t stream);
+struct QsaExpandArgs {
+    const int32_t* blk;   // [B][n_top] selected blocks, increasing, -1 padded
+    const int32_t* seq_lens;
+    int32_t* tok_idx;     // [B][4 n_top + 3]
+    int32_t* tok_count;   // [B]
+    int32_t* dev_status;
+    int B, L_max, n_top;
+};
+cudaError_t launch_qsa_expand(const QsaExpandArgs& a, cudaStream_t stream);
 
 // ---- sparse latent attention ----
 struct SparseLaunch {

@@ -60,6 +60,14 @@ _lib.attn_decode_sparse_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32]
 _lib.attn_decode_sparse_workspace_bytes.restype = _sz
 _lib.attn_decode_sparse.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
                                     _vp, _vp]
+_lib.qsa_block_keys.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32, _f32, _vp, _vp, _vp]
+_lib.qsa_select_workspace_bytes.argtypes = [_i32, _i32, _i32]
+_lib.qsa_select_workspace_bytes.restype = _sz
+_lib.qsa_select.argtypes = [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _sz, _vp, _vp]
+_lib.attn_decode_gqa_sparse_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, _i32]
+_lib.attn_decode_gqa_sparse_workspace_bytes.restype = _sz
+_lib.attn_decode_gqa_sparse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp,
+                                        _vp, _sz, _vp, _vp]
 
 ROPE_NONE, ROPE_PI, ROPE_NTK, ROPE_YARN, ROPE_DYN_NTK = 0, 1, 2, 3, 4
 STATUS_BAD_POSITION, STATUS_BAD_LENGTH, STATUS_BAD_INDEX, STATUS_NAN_SCORE, STATUS_TIMEOUT = 1, 2, 4, 8, 16
@@ -402,4 +410,91 @@ def attn_decode_sparse(q, latent, topk_idx, Dv, scale, out=None, lse=None, ws=No
         ws = workspace(attn_decode_sparse_workspace_bytes(B, Hq, Dv, k), q.device)
     _check(_lib.attn_decode_sparse(_ptr(q), _ptr(latent), _ptr(topk_idx), B, Hq, Dk, Dv, L_max, k, float(scale),
                                    _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status), _stream()))
+    return out, lse
+
+
+QSA_BLOCK = 4
+
+
+def qsa_block_keys(k_idx, seq_lens, cos, sin, block_keys=None, block_from=None, max_new=0, eps=1e-6, pair_style=0,
+                   dev_status=None):
+    """k_idx [B, L_max, 128] bf16 (L_max a multiple of 4), seq_lens int32 [B] (tokens)
+    -> block_keys [B, L_max // 4, 128] bf16 (groups [block_from, min(len // 4,
+    block_from + max_new)) written)."""
+    _need(k_idx, torch.bfloat16, "k_idx")
+    _contig(k_idx, "k_idx")
+    _need(seq_lens, torch.int32, "seq_lens")
+    B, L_max, dI = k_idx.shape
+    if block_keys is None:
+        block_keys = torch.zeros((B, L_max // QSA_BLOCK, dI), dtype=torch.bfloat16, device=k_idx.device)
+    _need(block_keys, torch.bfloat16, "block_keys")
+    if block_from is not None:
+        _need(block_from, torch.int32, "block_from")
+    _check(_lib.qsa_block_keys(_ptr(k_idx), _ptr(seq_lens), _ptr(block_from), int(max_new), B, dI, L_max, _ptr(cos),
+                               _ptr(sin), cos.shape[0], pair_style, float(eps), _ptr(block_keys), _ptr(dev_status),
+                               _stream()))
+    return block_keys
+
+
+def qsa_select_workspace_bytes(B, L_max, n_top) -> int:
+    return int(_lib.qsa_select_workspace_bytes(B, L_max, n_top))
+
+
+def qsa_select(q_idx, w, block_keys, seq_lens, n_top=512, tok_idx=None, tok_count=None, scores_out=None, ws=None,
+               dev_status=None, want_scores=False):
+    """q_idx [B, 64, 128] bf16, w [B, 64] fp32, block_keys [B, L_max // 4, 128] bf16,
+    seq_lens int32 [B] -> (tok_idx int32 [B, 4 n_top + 3], tok_count int32 [B],
+    group scores fp32 [B, L_max // 4] or None)."""
+    _need(q_idx, torch.bfloat16, "q_idx")
+    _need(block_keys, torch.bfloat16, "block_keys")
+    _need(w, torch.float32, "w")
+    _need(seq_lens, torch.int32, "seq_lens")
+    for t, n in ((q_idx, "q_idx"), (block_keys, "block_keys"), (w, "w")):
+        _contig(t, n)
+    B, HI, dI = q_idx.shape
+    L_max = block_keys.shape[1] * QSA_BLOCK
+    dev = q_idx.device
+    if tok_idx is None:
+        tok_idx = torch.empty((B, QSA_BLOCK * n_top + QSA_BLOCK - 1), dtype=torch.int32, device=dev)
+    if tok_count is None:
+        tok_count = torch.empty(B, dtype=torch.int32, device=dev)
+    if scores_out is None and want_scores:
+        scores_out = torch.empty((B, L_max // QSA_BLOCK), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(qsa_select_workspace_bytes(B, L_max, n_top), dev)
+    _check(_lib.qsa_select(_ptr(q_idx), _ptr(w), _ptr(block_keys), _ptr(seq_lens), B, HI, dI, L_max, n_top,
+                           _ptr(tok_idx), _ptr(tok_count), _ptr(scores_out), _ptr(ws), ws.numel(), _ptr(dev_status),
+                           _stream()))
+    return tok_idx, tok_count, scores_out
+
+
+def attn_decode_gqa_sparse_workspace_bytes(B, n_head, n_kv_head, head_dim, n_idx) -> int:
+    return int(_lib.attn_decode_gqa_sparse_workspace_bytes(B, n_head, n_kv_head, head_dim, n_idx))
+
+
+def attn_decode_gqa_sparse(q, k_cache, v_cache, tok_idx, scale, tok_count=None, out=None, lse=None, ws=None,
+                           dev_status=None, want_lse=True):
+    """q [B, H, d] bf16, k_cache/v_cache [B, Hk, T_max, d] bf16, tok_idx int32 [B, n_idx]
+    (the first tok_count[b] entries used; -1 skipped) -> (out [B, H, d], lse [B, H])."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (tok_idx, "tok_idx")):
+        _contig(t, n)
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, torch.bfloat16, n)
+    _need(tok_idx, torch.int32, "tok_idx")
+    if tok_count is not None:
+        _need(tok_count, torch.int32, "tok_count")
+    B, H, d = q.shape
+    Bk, Hk, T_max, dk = k_cache.shape
+    if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or tok_idx.shape[0] != B:
+        raise ValueError("inconsistent sparse decode shapes")
+    n_idx = tok_idx.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(attn_decode_gqa_sparse_workspace_bytes(B, H, Hk, d, n_idx), q.device)
+    _check(_lib.attn_decode_gqa_sparse(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(tok_idx), _ptr(tok_count), n_idx, B,
+                                       H, Hk, d, T_max, float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                       _ptr(dev_status), _stream()))
     return out, lse

@@ -1,4 +1,4 @@
-"""Seeded synthetic workloads for the five measured shapes.
+"""Seeded synthetic workloads for the measured shapes.
 
 This module only draws random numbers: it holds none of the method's
 arithmetic (no rotation, no softmax, no scoring).  Tests, the benchmark and
@@ -91,6 +91,27 @@ class DsaWorkload:
     sparse_scale: float = 192 ** -0.5  # 1/sqrt(d_h + d_h^R) with d_h = 128, d_h^R = 64
 
 
+@dataclass(frozen=True)
+class QsaWorkload:
+    """Block-level indexer over 4-token groups, then sparse GQA decode."""
+    name: str
+    index: int
+    B: int
+    L: int        # cache capacity (tokens); lengths are drawn in [L_lo, L]
+    L_lo: int
+    HI: int       # indexer heads
+    dI: int       # indexer key/query width
+    n_top: int    # groups kept
+    H: int        # attention heads
+    Hk: int       # KV heads
+    d: int        # head width
+    rope: RopeSpec = field(default_factory=lambda: RopeSpec(base=500000.0))
+
+    @property
+    def scale(self) -> float:
+        return self.d ** -0.5
+
+
 TINY_GQA = DecodeWorkload("tiny_gqa_decode_B2_H8_Hk2_d64_T256", 0, B=2, H=8, Hk=2, d=64, T_max=256,
                           T_lo=256, T_hi=256, rope=RopeSpec(base=10000.0))
 LLAMA3_8B_DECODE = DecodeWorkload("llama3_8b_decode_B16_H32_Hk8_d128_ragged1024-8192", 1, B=16, H=32,
@@ -110,6 +131,9 @@ PREFILL_8K = PrefillWorkload("causal_prefill_B2_T8192_H32_Hk8_d128", 3, B=2, T=8
                              d=128, rope=RopeSpec(base=500000.0))
 DSA_128K = DsaWorkload("dsa_sparse_decode_B8_L131072_HI64_dI128_k2048_Hq128_576-512", 4, B=8,
                        L=131072, HI=64, dI=128, k=2048, Hq=128, Dk=576, Dv=512)
+
+QSA_128K = QsaWorkload("qsa_block_sparse_decode_B8_L131072_HI64_dI128_top512x4_H32_Hk8_d128", 5, B=8, L=131072,
+                       L_lo=65536, HI=64, dI=128, n_top=512, H=32, Hk=8, d=128)
 
 DECODE_WORKLOADS = [TINY_GQA, LLAMA3_8B_DECODE, LLAMA2_70B_GQA_32K, LLAMA2_70B_MQA_32K,
                     LLAMA2_70B_MHA_32K]
@@ -190,6 +214,28 @@ def dsa_inputs(w: DsaWorkload, device="cpu", seed: int | None = None, B: int | N
         out["q"] = normal_bf16((B, w.Hq, w.Dk), gen, device)
         out["latent"] = normal_bf16((B, L, w.Dk), gen, device)
     out["seq_lens"] = torch.full((B,), L, dtype=torch.int32)
+    return out
+
+
+def qsa_inputs(w: QsaWorkload, device="cpu", seed: int | None = None, B: int | None = None,
+               L: int | None = None, L_lo: int | None = None, with_cache: bool = True) -> dict:
+    """q_idx [B, HI, dI] bf16, w [B, HI] fp32 U(0,1), k_idx [B, L, dI] bf16 (the
+    indexer keys), q [B, H, d], k/v [B, Hk, L, d] bf16, seq_lens int32 [B] drawn
+    uniformly in [L_lo, L] (every residue mod 4 occurs: the trailing partial group)."""
+    seed = SEED_BASE + w.index if seed is None else seed
+    B = w.B if B is None else B
+    if L_lo is None:
+        L_lo = w.L_lo if L is None else L // 2
+    L = w.L if L is None else L
+    gen = generator(seed, device)
+    out = dict(q_idx=normal_bf16((B, w.HI, w.dI), gen, device),
+               w=uniform_f32((B, w.HI), gen, device),
+               k_idx=normal_bf16((B, L, w.dI), gen, device))
+    if with_cache:
+        out["q"] = normal_bf16((B, w.H, w.d), gen, device)
+        out["k"] = normal_bf16((B, w.Hk, L, w.d), gen, device)
+        out["v"] = normal_bf16((B, w.Hk, L, w.d), gen, device)
+    out["seq_lens"] = lengths(B, L_lo, L, seed)
     return out
 
 
