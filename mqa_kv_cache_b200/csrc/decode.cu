@@ -26,10 +26,13 @@
 // Gather mode (a sparse token list per sequence, "attention" page, "Qwen Sparse
 // Attention (QSA)" ③–④: the selected tokens' full-precision K/V are fetched from
 // the cache by index and standard GQA attention runs over them): a unit's rows
-// are the listed cache rows.  The whole producer warp gathers each tile with
-// 16-byte cp.async (a 256-byte row = 16 lanes) into the same swizzled layout the
-// tensor map writes, with one asynchronous arrival per lane on the stage barrier,
-// and passes the tile's valid-row bitmask (skipped entries, the tail) along.
+// are the listed cache rows.  GATHER_WARPS producer warps copy each 64-row tile
+// with 16-byte cp.async (a 256-byte row = 16 lanes; each warp a quarter or half
+// of the rows) into the same swizzled layout as the tiled loads, each lane arriving
+// asynchronously on the stage barrier once its copies land, and the first one
+// passes the tile's valid-row bitmask (skipped entries, the tail) along.  Row
+// gathers through the copy engine (per-row bulk copies, tile::gather4) were
+// measured slower: the engine sustains few small copies in flight per SM.
 #include <type_traits>
 
 #include "common.cuh"
@@ -43,10 +46,13 @@ namespace {
 constexpr int TILE = DEC_TILE;  // cache rows per pipeline stage
 constexpr int CWARPS = 4;  // consumer warps
 constexpr int THREADS = 32 * (CWARPS + 1);
+constexpr int GATHER_WARPS = 2;  // gather mode: producer warps
+constexpr int IDX_TILES = GATHER_WARPS <= 2 ? 8 : 4;  // tiles whose row indices a producer warp stages at once
+constexpr int threads_of(bool gather) { return 32 * (CWARPS + (gather ? GATHER_WARPS : 1)); }
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
-template <int D, int NMT>
+template <int D, int NMT, bool GATHER>
 struct Cfg {
     static constexpr int STAGES = D == 128 ? 5 : 8;
     static constexpr int HALVES = D / 64;  // 128-byte column blocks per row
@@ -65,9 +71,17 @@ struct Cfg {
     static constexpr int OFF_BAR = ((OFF_LEN + DECODE_MAX_B * 4) + 7) / 8 * 8;
     static constexpr int OFF_MISC = OFF_BAR + (2 * STAGES + 2) * 8;
     static constexpr int OFF_MASK = OFF_MISC + 64;                  // [STAGES] valid rows (gather mode)
-    static constexpr int SMEM = OFF_MASK + STAGES * 8 + 1024;  // + alignment slack
+    static constexpr int OFF_IDX = (OFF_MASK + STAGES * 8 + 15) / 16 * 16;  // [GATHER_WARPS][IDX_TILES * TILE] rows
+    static constexpr int SMEM = OFF_IDX + (GATHER ? GATHER_WARPS * IDX_TILES * TILE * 4 : 0) + 1024;  // + slack
     static_assert(SMEM <= 232448, "shared memory");
 };
+
+// Byte offset of the 16-byte chunk holding dims dim .. dim+7 of row `tok` in a K or V
+// tile of 128-byte-swizzled 64-column blocks.
+__device__ __forceinline__ uint32_t tile_off(int tok, int dim)
+{
+    return static_cast<uint32_t>((dim >> 6) * (TILE * 128)) + swz128(tok, (dim & 63) >> 3);
+}
 
 __device__ __forceinline__ uint32_t ld_u32(const kvattn_bf16* p)
 {
@@ -179,10 +193,10 @@ __device__ void merge_unit(const DecodeArgs& a, int u, int S, int count, int tid
 static_assert(TILE == 64, "gather mode passes a tile's valid rows as one 64-bit mask");
 
 template <int D, int NMT, bool GATHER>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(threads_of(GATHER), 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, DecodeArgs a)
 {
-    using C = Cfg<D, NMT>;
+    using C = Cfg<D, NMT, GATHER>;
     constexpr int WPM = CWARPS / NMT;  // warps sharing one M tile (split the tile's rows)
     constexpr int TPW = TILE / WPM;    // cache rows per warp per tile
     constexpr int NT = TPW / 8;        // score n-tiles per warp
@@ -209,12 +223,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int* s_abort = s_misc + 1;
     int* s_merge = s_misc + 4;  // [0] = split pieces made here, then (unit, first slot, pieces) x 2
     uint64_t* s_mask = reinterpret_cast<uint64_t*>(smem + C::OFF_MASK);  // valid rows of each stage (gather)
+    int* s_idx = reinterpret_cast<int*>(smem + C::OFF_IDX);  // staged row indices, per producer warp (gather)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
-            // gather mode: one cp.async arrival per producer lane + the lane-0 arrival with the mask
-            mbar_init(&full[s], GATHER ? 33 : 1);
+            // gather mode: every producer lane arrives once its copies land, plus the mask arrival
+            mbar_init(&full[s], GATHER ? 32 * GATHER_WARPS + 1 : 1);
             mbar_init(&empty[s], CWARPS);
         }
         mbar_init(q_full, 1);
@@ -223,7 +238,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         s_merge[0] = 0;
         fence_barrier_init();
     }
-    if (!GATHER && warp == CWARPS && lane == 0) {
+    if (warp == CWARPS && lane == 0) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
@@ -253,24 +268,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     Walk w_start = walk_from(lo, a.B, a.Hk, s_n, s_Ub, 0);
     w_start.S = slots_before(w_start.b * a.Hk + w_start.kvh, a.Hk, s_n, s_Ub, N, G, s_misc + 2);
 
-    if (warp == CWARPS) {
+    if (warp >= CWARPS) {
         // ===== producer: streams K/V tiles of every piece in order (one thread with
-        // the tensor maps; the whole warp in gather mode) =====
+        // the tensor maps; GATHER_WARPS whole warps in gather mode) =====
         if (!GATHER && lane != 0) return;
+        const int pw = warp - CWARPS;  // producer warp (gather mode)
+        int* my_idx = s_idx + pw * (IDX_TILES * TILE);
+        // gather mode: a warp-wide copy instruction moves RPI rows (CPR lanes x 16 bytes
+        // each); lane group my_r copies rows my_r * NI .. my_r * NI + NI - 1 of a tile,
+        // producer warp pw the NIW of them starting at pw * NIW
+        constexpr int CPR = D / 8;
+        constexpr int RPI = 32 / CPR;
+        constexpr int NI = TILE / RPI;
+        constexpr int NIW = NI / GATHER_WARPS;
+        static_assert(NIW % 4 == 0, "row indices are read four at a time");
+        const int my_r = lane / CPR, my_ch = lane % CPR;
+        const uint32_t my_dst = (my_ch >> 3) * (TILE * 128);
         Walk w = w_start;
         int it = 0, np = 0;
         bool ok = true;
         const uint32_t q_bytes = static_cast<uint32_t>(a.g) * D * 2;
-        constexpr int CPR = D / 8;     // 16-byte chunks of a row (gather mode)
-        constexpr int RPI = 32 / CPR;  // rows per warp-wide copy instruction
-        const int my_r = lane / CPR, my_ch = lane % CPR;
-        const uint32_t my_dst = (my_ch >> 3) * (TILE * 128);
         for (; ok && w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
             long long tb, te;
             if (!piece_tiles(w, s_n[w.b], lo, hi, tb, te)) continue;
             const int z = w.b * a.Hk + w.kvh;
             // the piece's g query rows (contiguous), once the consumers hold the previous ones
-            if (np > 0) {
+            if (np > 0 && pw == 0) {
                 const bool got = GATHER ? warp_wait(q_empty, (np - 1) & 1, s_abort)
                                         : (!*s_abort && mbar_wait(q_empty, (np - 1) & 1));
                 if (!got) {
@@ -279,7 +302,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             // with RoPE, the cos and sin rows of the query's position come along
-            if (lane == 0) {
+            if (lane == 0 && pw == 0) {
                 const int qp = rope ? s_qpos[w.b] : -1;
                 const bool rot = rope && qp >= 0 && qp < a.max_pos;
                 mbar_arrive_expect_tx(q_full, q_bytes + (rot ? D * 4 : 0));
@@ -291,17 +314,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
             }
             ++np;
-            // gather mode: this lane holds the row indices of rows `lane` and `lane + 32` of
-            // the next tile (-1 past the unit's count), loaded one tile ahead
+            // gather mode: the row indices of up to IDX_TILES tiles at a time are staged in
+            // shared memory (all loads in flight together: one round trip per chunk)
             const int cnt = s_len[w.b];
             const int32_t* irow = GATHER ? a.idx + static_cast<long long>(w.b) * a.n_idx : nullptr;
-            int nia = -1, nib = -1;
-            if (GATHER) {
-                const int ra = static_cast<int>(tb) * TILE + lane;
-                nia = ra < cnt ? __ldg(irow + ra) : -1;
-                nib = ra + 32 < cnt ? __ldg(irow + ra + 32) : -1;
-            }
+            long long chunk_t0 = -IDX_TILES;
             for (long long t = tb; t < te; ++t, ++it) {
+                if (GATHER && t >= chunk_t0 + IDX_TILES) {
+                    chunk_t0 = t;
+                    const int e0 = static_cast<int>(t) * TILE;
+                    int v[IDX_TILES * TILE / 32];
+#pragma unroll
+                    for (int u = 0; u < IDX_TILES * TILE / 32; ++u) {
+                        const int e = e0 + u * 32 + lane;
+                        v[u] = e < cnt ? __ldg(irow + e) : -1;
+                    }
+                    __syncwarp();  // the previous chunk has been read by every lane
+#pragma unroll
+                    for (int u = 0; u < IDX_TILES * TILE / 32; ++u) my_idx[u * 32 + lane] = v[u];
+                    __syncwarp();
+                }
                 const int s = it % C::STAGES;
                 const uint32_t ph = (it / C::STAGES) & 1;
                 if (it >= C::STAGES) {
@@ -322,32 +354,36 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_3d(vd + h * (TILE * 128), &tm_v, &full[s], h * 64, static_cast<int>(t * TILE), z);
                     }
                 } else {
-                    const int ia = nia, ib = nib;
-                    if (t + 1 < te) {
-                        const int ra = static_cast<int>(t + 1) * TILE + lane;
-                        nia = ra < cnt ? __ldg(irow + ra) : -1;
-                        nib = ra + 32 < cnt ? __ldg(irow + ra + 32) : -1;
-                    }
+                    const int rb = static_cast<int>(t - chunk_t0) * TILE;
+                    const int ia = my_idx[rb + lane], ib = my_idx[rb + 32 + lane];
                     const bool va = ia >= 0 && ia < a.T_max, vb = ib >= 0 && ib < a.T_max;
-                    if (ia < -1 || ia >= a.T_max || ib < -1 || ib >= a.T_max)
+                    if (pw == 0 && (ia < -1 || ia >= a.T_max || ib < -1 || ib >= a.T_max))
                         report_status(a.dev_status, KVATTN_STATUS_BAD_INDEX);
                     const uint32_t ma = __ballot_sync(0xffffffffu, va), mb = __ballot_sync(0xffffffffu, vb);
                     const kvattn_bf16* kz = a.k_cache + static_cast<long long>(z) * a.T_max * D + my_ch * 8;
                     const kvattn_bf16* vz = a.v_cache + static_cast<long long>(z) * a.T_max * D + my_ch * 8;
                     const uint32_t sk = smem_u32(kd) + my_dst, sv = smem_u32(vd) + my_dst;
-#pragma unroll 8
-                    for (int i = 0; i < TILE / RPI; ++i) {
-                        const int r = i * RPI + my_r;  // row of the tile this lane copies a chunk of
-                        const int row = __shfl_sync(0xffffffffu, i * RPI < 32 ? ia : ib, r & 31);
-                        if (((r < 32 ? ma >> r : mb >> (r - 32)) & 1u) != 0u) {
-                            const long long off = static_cast<long long>(row) * D;
-                            const uint32_t so = swz128(r, my_ch & 7);
+                    const int r0 = my_r * NI + pw * NIW;  // first row of the tile this lane copies
+                    int rows[NIW];
+#pragma unroll
+                    for (int u = 0; u < NIW; u += 4) {
+                        const int4 x4 = *reinterpret_cast<const int4*>(my_idx + rb + r0 + u);
+                        rows[u] = x4.x;
+                        rows[u + 1] = x4.y;
+                        rows[u + 2] = x4.z;
+                        rows[u + 3] = x4.w;
+                    }
+#pragma unroll
+                    for (int u = 0; u < NIW; ++u) {
+                        if (rows[u] >= 0 && rows[u] < a.T_max) {  // the row's mask bit
+                            const long long off = static_cast<long long>(rows[u]) * D;
+                            const uint32_t so = swz128(r0 + u, my_ch & 7);
                             cp_async16(sk + so, kz + off, 16);
                             cp_async16(sv + so, vz + off, 16);
                         }
                     }
                     cp_async_arrive_noinc(&full[s]);
-                    if (lane == 0) {
+                    if (pw == 0 && lane == 0) {
                         s_mask[s] = (static_cast<uint64_t>(mb) << 32) | ma;
                         mbar_arrive(&full[s]);
                     }
@@ -360,7 +396,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         // copies still in flight complete before the CTA leaves (bounded waits)
         if (GATHER) cp_async_wait<0>();
-        if (lane == 0) {
+        if (lane == 0 && pw == 0) {
             for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
                 mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
             if (np > 0) mbar_wait(q_full, (np - 1) & 1);
@@ -443,13 +479,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < KS; ++kk) {
                     const int dim = kk * 16 + ((mi & 1) << 3);
-                    const uint32_t dbase = sK + (dim >> 6) * (TILE * 128);
-                    const int chunk = (dim & 63) >> 3;
 #pragma unroll
                     for (int np = 0; np < NT / 2; ++np) {
                         const int tok = tok0 + np * 16 + rr + ((mi >> 1) << 3);
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(dbase + swz128(tok, chunk), b0, b1, b2, b3);
+                        ldsm_x4(sK + tile_off(tok, dim), b0, b1, b2, b3);
                         mma_bf16_16816(sc[2 * np], qa[kk], b0, b1);
                         mma_bf16_16816(sc[2 * np + 1], qa[kk], b2, b3);
                     }
@@ -514,7 +548,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     for (int dp = 0; dp < D / 16; ++dp) {
                         const int dim = dp * 16 + ((mi >> 1) << 3);
                         uint32_t v0, v1, v2, v3;
-                        ldsm_x4_t(sV + (dim >> 6) * (TILE * 128) + swz128(tok, (dim & 63) >> 3), v0, v1, v2, v3);
+                        ldsm_x4_t(sV + tile_off(tok, dim), v0, v1, v2, v3);
                         if (tail) {
                             // rows past the length may hold anything (NaN included):
                             // zero them so that 0 * garbage cannot reach the sum
@@ -735,12 +769,13 @@ cudaError_t launch_typed(const DecodeArgs& a, const CUtensorMap& tm_k, const CUt
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_set[dev]) {
         e = cudaFuncSetAttribute(decode_kernel<D, NMT, GATHER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<D, NMT>::SMEM);
+                                 Cfg<D, NMT, GATHER>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
     // split units are merged inside the kernel, by the CTA that finishes their last piece
-    return launch_pdl(decode_kernel<D, NMT, GATHER>, dim3(a.grid), dim3(THREADS), Cfg<D, NMT>::SMEM, stream, tm_k,
+    return launch_pdl(decode_kernel<D, NMT, GATHER>, dim3(a.grid), dim3(threads_of(GATHER)), Cfg<D, NMT, GATHER>::SMEM,
+                      stream, tm_k,
                       tm_v, a);
 }
 
