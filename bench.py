@@ -17,6 +17,7 @@ all ranks / max-over-ranks time.  --impl reference times the fp64 CPU oracle
 on the host cores on a bounded sample of the same workload.
 """
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -445,12 +446,12 @@ def measure_dsa(K, device, steps, flush, peaks):
             "sparse_gathered_bytes": sp_bytes}
 
 
-def measure_qsa(K, device, steps, flush, peaks):
+def measure_qsa(K, device, steps, flush, peaks, B=None):
     """Block-level indexer decode step (B 8, ragged lengths up to 131072 tokens): the
     key of the newest 4-token group (qsa_block_keys, one group per row), group scoring
     + top-512 + expansion with the trailing partial group (qsa_select), then GQA
     decode (H 32, Hk 8, d 128) over the <= 2051 selected tokens (attn_decode_gqa_sparse)."""
-    w = W.QSA_128K
+    w = W.QSA_128K if B is None else dataclasses.replace(W.QSA_128K, B=B)
     inp = W.qsa_inputs(w, device=device)
     lens = inp["seq_lens"].to(device)
     cos, sin = K.rope_table_build(K.rope_params(w.dI, base=w.rope.base), w.L, device=device)
@@ -495,8 +496,8 @@ def measure_qsa(K, device, steps, flush, peaks):
     step_bytes = key_bytes + kv_bytes + qo_bytes + w.B * (w.HI * w.dI * 2 + w.HI * 4)
     build_bytes = sum(L) * w.dI * 2 + key_bytes
     hbm = peaks["hbm_gbs"]
-    return {"workload": w.name, "step_ms": round(step_ms, 4), "tok_per_s": round(w.B / (step_ms * 1e-3), 1),
-            "step_algorithmic_bytes": step_bytes,
+    return {"workload": w.name if B is None else w.name.replace("_B8_", f"_B{B}_"), "step_ms": round(step_ms, 4),
+            "tok_per_s": round(w.B / (step_ms * 1e-3), 1), "step_algorithmic_bytes": step_bytes,
             "step_GB_s": round(step_bytes / (step_ms * 1e-3) / 1e9, 1),
             "step_pct_of_hbm_peak": round(100 * step_bytes / (step_ms * 1e-3) / 1e9 / hbm, 1),
             "select_ms": round(select_ms, 4), "group_key_bytes": key_bytes,
@@ -663,6 +664,8 @@ def main():
     ap.add_argument("--only", choices=["tiny", "gqa32k", "mqa32k", "mha32k", "window", "prefill", "prefill_window", "dsa",
                                        "qsa"],
                     help="time one other configuration alone and print its JSON")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="with --only qsa: batch rows (default 8; a smaller case for profiler captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -692,7 +695,7 @@ def main():
         elif args.only == "prefill_window":
             res = measure_prefill_window(K, device, args.steps, flush, peaks)
         elif args.only == "qsa":
-            res = measure_qsa(K, device, args.steps, flush, peaks)
+            res = measure_qsa(K, device, args.steps, flush, peaks, B=args.batch)
         else:
             res = measure_dsa(K, device, args.steps, flush, peaks)
         if rank == 0:
