@@ -37,7 +37,7 @@ METRIC = "decode-attn effective HBM GB/s (% of peak) & tok/s; prefill TFLOP/s"
 # DRAM bytes (read + write) of one decode_kernel launch on the headline workload, from an ncu
 # capture of the current kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the
 # kernel changes after that capture.
-DECODE_TRAFFIC_BYTES = 295_059_200 + 3_644_416
+DECODE_TRAFFIC_BYTES = 295_056_640 + 4_192_768
 L2_FLUSH_BYTES = 256 << 20
 
 

@@ -572,12 +572,11 @@ int qsa_block_keys(const kvattn_bf16* k_idx, const int32_t* seq_lens, const int3
 }
 
 static size_t qsa_scores_bytes(int B, int L_max) { return align_up(kvattn::dsa_scores_bytes(B, L_max / kvattn::QSA_BLOCK)); }
-static size_t qsa_blocks_bytes(int B, int n_top) { return align_up(static_cast<size_t>(B) * n_top * sizeof(int32_t)); }
-
 size_t qsa_select_workspace_bytes(int B, int L_max, int n_top)
 {
     if (B < 1 || L_max < kvattn::QSA_BLOCK || n_top < 1) return 0;
-    return qsa_scores_bytes(B, L_max) + qsa_blocks_bytes(B, n_top);
+    (void)n_top;
+    return qsa_scores_bytes(B, L_max);
 }
 
 int qsa_select(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* block_keys, const int32_t* seq_lens, int B,
@@ -605,20 +604,19 @@ int qsa_select(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* bloc
         return fail(KVATTN_ERR_ALIGN, "qsa_select: workspace must be 256-byte aligned");
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     float* scores = scores_out ? scores_out : reinterpret_cast<float*>(ws);
-    int32_t* blk = reinterpret_cast<int32_t*>(ws + qsa_scores_bytes(B, L_max));
     int sms = 0;
     if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "qsa_select: no CUDA device");
     CUtensorMap tm_k, tm_q;
     if (make_map_3d(&tm_k, block_keys, 128, nb_max, B, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
     if (make_map_3d(&tm_q, q_idx, 128, 64, B, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
-    kvattn::DsaIndexArgs a{w, seq_lens, scores, blk, dev_status, B, nb_max, n_top, sms};
+    kvattn::DsaIndexArgs a{w, seq_lens, scores, nullptr, dev_status, B, nb_max, n_top, sms};
     static_assert(kvattn::QSA_BLOCK == 4, "len_shift below is log2 of the group size");
     a.len_shift = 2;  // a row of L tokens has L / 4 complete groups
-    const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int rc = cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, st), "qsa_select block scoring");
-    if (rc != KVATTN_OK) return rc;
-    kvattn::QsaExpandArgs e{blk, seq_lens, tok_idx, tok_count, dev_status, B, L_max, n_top};
-    return cuda_status(kvattn::launch_qsa_expand(e, st), "qsa_select expand");
+    a.tok_idx = tok_idx;  // the top-k writes the groups' tokens and the tail directly
+    a.tok_count = tok_count;
+    a.L_tok = L_max;
+    return cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, static_cast<cudaStream_t>(stream)),
+                       "qsa_select");
 }
 
 size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k)

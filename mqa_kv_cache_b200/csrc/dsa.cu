@@ -287,6 +287,9 @@ struct TopkArgs {
     int32_t* dev_status;
     int L_max, k;
     int len_shift;
+    int32_t* tok_out;    // groups mode (see DsaIndexArgs), else null
+    int32_t* tok_count;
+    int L_tok;
 };
 
 constexpr int TK_SLICE_MAX = 16384;  // keys per CTA held in shared memory
@@ -412,7 +415,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     int g_rank = gt_before + inc_gt - n_gt;
     int e_rank = eq_before + inc_eq - n_eq;
     int pos = g_rank + min(e_rank, max(take_eq, 0));
-    int32_t* out = a.out + static_cast<long long>(row) * a.k;
+    const int gs = 1 << a.len_shift;  // tokens per key in groups mode
+    const int width = a.k * gs + gs - 1;
+    int32_t* out = a.out ? a.out + static_cast<long long>(row) * a.k : nullptr;
+    int32_t* tout = a.tok_out ? a.tok_out + static_cast<long long>(row) * width : nullptr;
     for (int i = r0; i < r1; ++i) {
         const uint32_t key = s_keys[kpad(i)];
         bool take = key > T;
@@ -420,12 +426,30 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
             take = e_rank < take_eq;
             ++e_rank;
         }
-        if (take) out[pos++] = lo + i;
+        if (take) {
+            if (tout) {
+                for (int r = 0; r < gs; ++r) tout[pos * gs + r] = (lo + i) * gs + r;
+            } else {
+                out[pos] = lo + i;
+            }
+            ++pos;
+        }
     }
-    // -1 after the selected entries (fewer than kk only when NaN scores were skipped)
+    // -1 after the selected entries (fewer than kk only when NaN scores were skipped);
+    // in groups mode the row's trailing tokens come first
     const int n_sel = gt_total + min(max(take_eq, 0), eq_total);
-    if (rank == 0)
-        for (int j = n_sel + tid; j < a.k; j += TK_THREADS) out[j] = -1;
+    if (rank == 0) {
+        if (tout) {
+            const int tok_raw = a.seq_lens[row];
+            const int tok_len = min(max(tok_raw, 0), a.L_tok);
+            if (tok_len != tok_raw && tid == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
+            const int tail0 = len * gs, n_tail = max(tok_len - tail0, 0), first = n_sel * gs;
+            for (int j = first + tid; j < width; j += TK_THREADS) tout[j] = j - first < n_tail ? tail0 + (j - first) : -1;
+            if (tid == 0) a.tok_count[row] = first + n_tail;
+        } else {
+            for (int j = n_sel + tid; j < a.k; j += TK_THREADS) out[j] = -1;
+        }
+    }
     if (nan) s_nan = 1;
     __syncthreads();
     if (s_nan && tid == 0) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
@@ -467,7 +491,8 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     e = launch_pdl(indexer_kernel, dim3(grid), dim3(IX_THREADS), IX_SMEM, stream, tm_k, tm_q, ia);
     if (e != cudaSuccess) return e;
 
-    TopkArgs ta{a.scores, a.seq_lens, a.topk_idx, a.dev_status, a.L_max, a.k, a.len_shift};
+    TopkArgs ta{a.scores, a.seq_lens, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k, a.len_shift,
+                a.tok_idx, a.tok_count, a.L_tok};
     const int slice_max = (a.L_max + TK_CL - 1) / TK_CL;
     const size_t key_bytes = static_cast<size_t>(slice_max + (slice_max >> 4) + 1) * sizeof(uint32_t);
     static bool tk_attr[64] = {};

@@ -122,6 +122,13 @@ struct DsaIndexArgs {
     int32_t* dev_status;
     int B, L_max, k, num_sms;
     int len_shift = 0;  // row b has seq_lens[b] >> len_shift keys (2: the 4-token block keys)
+    // Groups mode (tok_idx non-null): key j stands for the 1 << len_shift tokens of group j;
+    // the selection is written as token positions (increasing) followed by the row's
+    // trailing tokens past its last complete group, -1 padded to (k << len_shift) +
+    // (1 << len_shift) - 1 entries, with the count in tok_count; topk_idx is not written.
+    int32_t* tok_idx = nullptr;
+    int32_t* tok_count = nullptr;
+    int L_tok = 0;  // token capacity of a row (seq_lens beyond it are clamped and flagged)
 };
 size_t dsa_scores_bytes(int B, int L_max);
 cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
@@ -141,15 +148,6 @@ struct QsaKeysArgs {
     float eps;
 };
 cudaError_t launch_qsa_block_keys(const QsaKeysArgs& a, cudaStream_t stream);
-struct QsaExpandArgs {
-    const int32_t* blk;   // [B][n_top] selected blocks, increasing, -1 padded
-    const int32_t* seq_lens;
-    int32_t* tok_idx;     // [B][4 n_top + 3]
-    int32_t* tok_count;   // [B]
-    int32_t* dev_status;
-    int B, L_max, n_top;
-};
-cudaError_t launch_qsa_expand(const QsaExpandArgs& a, cudaStream_t stream);
 
 // ---- sparse latent attention ----
 struct SparseLaunch {

@@ -1,6 +1,5 @@
-// qsa.cu -- the block-level indexer's two small kernels: building the keys of
-// complete 4-token groups, and unpacking selected groups back into token
-// positions ("attention" page, "Qwen Sparse Attention (QSA)" §3 ① and ②).
+// qsa.cu -- the block-level indexer's key builder: the keys of complete 4-token
+// groups ("attention" page, "Qwen Sparse Attention (QSA)" §3 ①).
 //
 // Block key of group j (tokens 4j .. 4j+3): the mean of the four indexer keys,
 // RMS-normalised (x / sqrt(mean(x^2) + eps), no gain), then rotated by RoPE at
@@ -9,9 +8,9 @@
 // stored keys instead of L token keys: the scoring and top-k are the lightning
 // indexer's kernels run over the block keys (dsa.cu, lengths shifted by 2).
 //
-// Expand: the n_top selected groups (listed in increasing order by the top-k)
-// become 4 n_top token positions, and the 0..3 tokens of the trailing
-// incomplete group follow unconditionally; the list stays increasing and is
+// Expand (written by the top-k kernel's compaction in its groups mode): the n_top
+// selected groups become 4 n_top token positions in increasing order, and the
+// 0..3 tokens of the trailing incomplete group follow unconditionally; the list is
 // -1 padded to 4 n_top + 3 entries.
 #include "common.cuh"
 #include "kernels.h"
@@ -110,37 +109,6 @@ __global__ void __launch_bounds__(QK_THREADS) qsa_block_keys_kernel(QsaKeysArgs 
     }
 }
 
-constexpr int QE_THREADS = 512;
-
-// grid (B).  tok[i] = 4 blk[i / 4] + i % 4 for i < 4 n_sel, then the tail.
-__global__ void __launch_bounds__(QE_THREADS) qsa_expand_kernel(QsaExpandArgs a)
-{
-    pdl_wait();
-    pdl_trigger();
-    const int b = blockIdx.x;
-    const int len_raw = a.seq_lens[b];
-    const int len = min(max(len_raw, 0), a.L_max);
-    if (len != len_raw && threadIdx.x == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
-    const int nb = len / QSA_BLOCK;
-    const int n_sel = min(nb, a.n_top);
-    const int n_blk_tok = QSA_BLOCK * n_sel;
-    const int count = n_blk_tok + (len - QSA_BLOCK * nb);
-    const int width = QSA_BLOCK * a.n_top + QSA_BLOCK - 1;
-    const int32_t* blk = a.blk + static_cast<long long>(b) * a.n_top;
-    int32_t* out = a.tok_idx + static_cast<long long>(b) * width;
-    for (int i = threadIdx.x; i < width; i += QE_THREADS) {
-        int t = -1;
-        if (i < n_blk_tok) {
-            const int j = blk[i / QSA_BLOCK];
-            t = j >= 0 ? j * QSA_BLOCK + (i % QSA_BLOCK) : -1;
-        } else if (i < count) {
-            t = QSA_BLOCK * nb + (i - n_blk_tok);
-        }
-        out[i] = t;
-    }
-    if (threadIdx.x == 0) a.tok_count[b] = count;
-}
-
 }  // namespace
 
 cudaError_t launch_qsa_block_keys(const QsaKeysArgs& a, cudaStream_t stream)
@@ -151,11 +119,6 @@ cudaError_t launch_qsa_block_keys(const QsaKeysArgs& a, cudaStream_t stream)
     if (gx > 4096) gx = 4096;  // grid-stride beyond
     if (gx < 1) gx = 1;
     return launch_pdl(qsa_block_keys_kernel, dim3(gx, a.B), dim3(QK_THREADS), 0, stream, a);
-}
-
-cudaError_t launch_qsa_expand(const QsaExpandArgs& a, cudaStream_t stream)
-{
-    return launch_pdl(qsa_expand_kernel, dim3(a.B), dim3(QE_THREADS), 0, stream, a);
 }
 
 }  // namespace kvattn
