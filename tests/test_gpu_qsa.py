@@ -312,3 +312,59 @@ def test_full_size_selection_properties_and_sampled_heads(K):
         ro, rl = oracle.attn_decode(W.bf16_bits(qs), W.bf16_bits(ks), W.bf16_bits(vs),
                                     np.array([len(rows)], np.int32), WL.scale)
         assert_attn_close(out[b:b + 1, h:h + 1], ro, lse[b:b + 1, h:h + 1], rl, f"qsa full b={b} h={h}")
+
+
+def test_select_nan_groups_are_never_taken(K):
+    """A group whose score is NaN is never selected (and flagged), so the list is
+    shorter than 4 n_top and the tail still follows.  (A NaN inside a key is not
+    enough: ReLU takes a NaN dot product to 0 on both sides.  A +inf key element met
+    by a head of weight 0 gives 0 * inf = NaN.)"""
+    B, L_max, n_top = 2, 4 * 400, 16
+    lens = [4 * 400, 4 * 20 + 3]
+    gen = W.generator(611)
+    q_idx = W.normal_bf16((B, 64, 128), gen)
+    w = W.uniform_f32((B, 64), gen)
+    kb = W.normal_bf16((B, L_max // 4, 128), gen)
+    q_idx[:, 0, 0] = 1.0
+    w[:, 0] = 0.0
+    kb[0, 7, 0] = float("inf")
+    for j in range(20):  # row 1: only 20 groups, 16 of them NaN -> 4 selectable
+        if j % 5:
+            kb[1, j, 0] = float("inf")
+    lens_t = torch.tensor(lens, dtype=torch.int32)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tok, cnt, sc = K.qsa_select(q_idx.cuda(), w.cuda(), kb.cuda(), lens_t.cuda(), n_top=n_top, want_scores=True,
+                                dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & K.STATUS_NAN_SCORE
+    g = sc.cpu().numpy().astype(np.float64)
+    # the oracle's top-k takes no NaN: select among each row's finite group scores
+    sel = np.full((B, n_top), -1, np.int64)
+    for b in range(B):
+        nb = lens[b] // 4
+        fin = np.flatnonzero(np.isfinite(g[b, :nb]))
+        assert len(fin) == nb - (1 if b == 0 else 16)
+        pick = oracle.topk(g[b, fin][None], n_top, lens=np.array([len(fin)], np.int32))[0]
+        sel[b, :np.count_nonzero(pick >= 0)] = fin[pick[pick >= 0]]
+    ref_tok, ref_cnt = oracle.qsa_expand(sel, lens_t.numpy(), n_top)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), ref_cnt)
+    np.testing.assert_array_equal(tok.cpu().numpy(), ref_tok)
+    assert ref_cnt[1] == 4 * 4 + 3
+
+
+def test_select_arguments_are_checked(K):
+    q_idx = torch.zeros((1, 64, 128), dtype=torch.bfloat16, device="cuda")
+    w = torch.ones((1, 64), dtype=torch.float32, device="cuda")
+    lens = torch.tensor([8], dtype=torch.int32, device="cuda")
+    kb = torch.zeros((1, 10, 128), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(K.KvattnError):
+        K.qsa_select(q_idx, w, kb, lens, n_top=0)
+    with pytest.raises(K.KvattnError):
+        K.qsa_select(q_idx, w, kb, lens, n_top=2049)
+    with pytest.raises(K.KvattnError):  # the indexer keys' length must be a multiple of 4
+        K.qsa_block_keys(torch.zeros((1, 10, 128), dtype=torch.bfloat16, device="cuda"), lens,
+                         *_tables(K, 16))
+    with pytest.raises(K.KvattnError):  # group size above 32 at head_dim 128
+        q = torch.zeros((1, 64, 128), dtype=torch.bfloat16, device="cuda")
+        kc = torch.zeros((1, 1, 16, 128), dtype=torch.bfloat16, device="cuda")
+        K.attn_decode_gqa_sparse(q, kc, kc, torch.zeros((1, 4), dtype=torch.int32, device="cuda"), 0.1)
