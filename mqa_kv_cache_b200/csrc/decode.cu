@@ -27,12 +27,13 @@
 // Attention (QSA)" ③–④: the selected tokens' full-precision K/V are fetched from
 // the cache by index and standard GQA attention runs over them): a unit's rows
 // are the listed cache rows.  GATHER_WARPS producer warps copy each 64-row tile
-// with 16-byte cp.async (a 256-byte row = 16 lanes; each warp a quarter or half
-// of the rows) into the same swizzled layout as the tiled loads, each lane arriving
-// asynchronously on the stage barrier once its copies land, and the first one
-// passes the tile's valid-row bitmask (skipped entries, the tail) along.  Row
-// gathers through the copy engine (per-row bulk copies, tile::gather4) were
-// measured slower: the engine sustains few small copies in flight per SM.
+// with 16-byte cp.async (a 256-byte row = 16 lanes; each warp its share of the
+// rows, with the row indices staged in shared memory) into the same swizzled
+// layout as the tiled loads, each lane arriving asynchronously on the stage
+// barrier once its copies land, and the first one passes the tile's valid-row
+// bitmask (skipped entries, the tail) along.  Row gathers through the copy engine
+// (per-row bulk copies, tile::gather4) were measured slower: the engine sustains
+// few small copies in flight per SM.
 #include <type_traits>
 
 #include "common.cuh"
