@@ -267,6 +267,21 @@ int attn_prefill_causal(const kvattn_bf16* q, const kvattn_bf16* k, const kvattn
                         int T, int n_head, int n_kv_head, int head_dim, float scale,
                         kvattn_bf16* out, float* lse, void* stream);
 
+/* ---- merge of decode results over disjoint key sets ---------------------------
+ * The softmax over a union of key sets from the softmax over each set: with
+ * LSE = ln sum_j exp(lse_j), out = sum_j exp(lse_j - LSE) o_j and lse = LSE (the
+ * split/merge identity the split-K decode uses inside one call).  This is the last
+ * step of a sequence-sharded decode: each GPU (or each call) runs attn_decode_gqa
+ * over one slice of a long cache, the slices' (out, lse) are exchanged once
+ * (all-gather), and every rank merges them.  A part with no keys (lse = -inf)
+ * has weight 0; if every part is empty, out = 0 and lse = -inf.
+ * o_parts [n_parts][B][n_head][head_dim] bf16 (16-byte aligned); lse_parts
+ * [n_parts][B][n_head] fp32; out [B][n_head][head_dim] bf16; lse [B][n_head] fp32
+ * or NULL.  Supported: head_dim in {64, 128}.
+ */
+int attn_merge_lse(const kvattn_bf16* o_parts, const float* lse_parts, int n_parts, int B, int n_head, int head_dim,
+                   kvattn_bf16* out, float* lse, void* stream);
+
 /*
  * attn_prefill_causal with a sliding window and attention sinks (the band
  * mask of the "attention" page, "Agentic RL 入门3" §1 sinks): query row i sees

@@ -391,6 +391,23 @@ int attn_decode_gqa_rope_window(const kvattn_bf16* q, const int32_t* q_pos, cons
                        T_max, scale, out, lse, workspace, workspace_bytes, dev_status, stream, &r, n_sink + window);
 }
 
+int attn_merge_lse(const kvattn_bf16* o_parts, const float* lse_parts, int n_parts, int B, int n_head, int head_dim,
+                   kvattn_bf16* out, float* lse, void* stream)
+{
+    if (!o_parts || !lse_parts || !out) return fail(KVATTN_ERR_NULL, "attn_merge_lse: NULL argument");
+    if (head_dim != 64 && head_dim != 128)
+        return fail(KVATTN_ERR_UNSUPPORTED, "attn_merge_lse: head_dim %d", head_dim);
+    if (n_parts < 1 || B < 1 || n_head < 1)
+        return fail(KVATTN_ERR_SHAPE, "attn_merge_lse: n_parts %d, B %d, n_head %d", n_parts, B, n_head);
+    if (static_cast<long long>(n_parts) * B * n_head * head_dim > (1ll << 40))
+        return fail(KVATTN_ERR_SHAPE, "attn_merge_lse: too large");
+    if (!aligned16(o_parts) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse_parts) & 3) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+        return fail(KVATTN_ERR_ALIGN, "attn_merge_lse: tensors must be aligned (16 bytes; 4 for lse)");
+    kvattn::MergeArgs a{o_parts, lse_parts, out, lse, n_parts, B, n_head, head_dim};
+    return cuda_status(kvattn::launch_merge_lse(a, static_cast<cudaStream_t>(stream)), "attn_merge_lse launch");
+}
+
 size_t attn_decode_gqa_sparse_workspace_bytes(int B, int n_head, int n_kv_head, int head_dim, int n_idx)
 {
     return attn_decode_gqa_workspace_bytes(B, n_head, n_kv_head, head_dim, n_idx);

@@ -113,6 +113,16 @@ cudaError_t launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tm_q, const
                              const CUtensorMap& tm_v, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeArgs& a, cudaStream_t stream);
 
+// ---- merge of decode results over disjoint key sets ----
+struct MergeArgs {
+    const kvattn_bf16* o_parts;  // [n][B][H][d]
+    const float* lse_parts;      // [n][B][H]
+    kvattn_bf16* out;            // [B][H][d]
+    float* lse;                  // [B][H] or null
+    int n, B, H, d;
+};
+cudaError_t launch_merge_lse(const MergeArgs& a, cudaStream_t stream);
+
 // ---- lightning indexer + top-k ----
 struct DsaIndexArgs {
     const float* w;

@@ -68,6 +68,7 @@ _lib.attn_decode_gqa_sparse_workspace_bytes.argtypes = [_i32, _i32, _i32, _i32, 
 _lib.attn_decode_gqa_sparse_workspace_bytes.restype = _sz
 _lib.attn_decode_gqa_sparse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp,
                                         _vp, _sz, _vp, _vp]
+_lib.attn_merge_lse.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
 
 ROPE_NONE, ROPE_PI, ROPE_NTK, ROPE_YARN, ROPE_DYN_NTK = 0, 1, 2, 3, 4
 STATUS_BAD_POSITION, STATUS_BAD_LENGTH, STATUS_BAD_INDEX, STATUS_NAN_SCORE, STATUS_TIMEOUT = 1, 2, 4, 8, 16
@@ -497,4 +498,22 @@ def attn_decode_gqa_sparse(q, k_cache, v_cache, tok_idx, scale, tok_count=None, 
     _check(_lib.attn_decode_gqa_sparse(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(tok_idx), _ptr(tok_count), n_idx, B,
                                        H, Hk, d, T_max, float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                        _ptr(dev_status), _stream()))
+    return out, lse
+
+
+def attn_merge_lse(o_parts, lse_parts, out=None, lse=None, want_lse=True):
+    """o_parts [n, B, H, d] bf16, lse_parts [n, B, H] fp32 (decode results over disjoint
+    key sets) -> (out [B, H, d] bf16, lse [B, H] fp32 or None) over their union."""
+    _need(o_parts, torch.bfloat16, "o_parts")
+    _need(lse_parts, torch.float32, "lse_parts")
+    _contig(o_parts, "o_parts")
+    _contig(lse_parts, "lse_parts")
+    n, B, H, d = o_parts.shape
+    if lse_parts.shape != (n, B, H):
+        raise ValueError("lse_parts must be [n, B, H]")
+    if out is None:
+        out = torch.empty((B, H, d), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H), dtype=torch.float32, device=o_parts.device)
+    _check(_lib.attn_merge_lse(_ptr(o_parts), _ptr(lse_parts), n, B, H, d, _ptr(out), _ptr(lse), _stream()))
     return out, lse
