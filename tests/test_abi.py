@@ -88,3 +88,30 @@ def test_rope_table_rejects_bad_params(lib):
     assert lib.rope_table_build(ctypes.byref(p), 16, fake, fake, None) == -4
     p = P(64, 1, 0, 0, 10000.0, 0.5, 0.0, 1.0, 32.0, 0.0)  # PI with s < 1
     assert lib.rope_table_build(ctypes.byref(p), 16, fake, fake, None) == -3
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host(lib):
+    vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    fake = vp(1 << 20)  # never dereferenced: validation fails first
+    # qsa_block_keys: NULL, width other than 128, L_max not a multiple of 4
+    lib.qsa_block_keys.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, vp, i32, i32, f32, vp, vp, vp]
+    assert lib.qsa_block_keys(None, fake, None, 0, 1, 128, 64, fake, fake, 64, 0, 1e-6, fake, None, None) == -1
+    assert lib.qsa_block_keys(fake, fake, None, 0, 1, 64, 64, fake, fake, 64, 0, 1e-6, fake, None, None) == -4
+    assert lib.qsa_block_keys(fake, fake, None, 0, 1, 128, 66, fake, fake, 64, 0, 1e-6, fake, None, None) == -3
+    assert "multiple of 4" in _err(lib)
+    # qsa_select: n_top outside 1..2048, wrong indexer shape, misaligned output
+    lib.qsa_select.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, vp, vp, vp, vp, sz, vp, vp]
+    assert lib.qsa_select(fake, fake, fake, fake, 1, 64, 128, 64, 0, fake, fake, None, fake, 1 << 20, None, None) == -3
+    assert lib.qsa_select(fake, fake, fake, fake, 1, 32, 128, 64, 8, fake, fake, None, fake, 1 << 20, None, None) == -4
+    assert lib.qsa_select(fake, fake, fake, fake, 1, 64, 128, 64, 8, vp((1 << 20) + 4), fake, None, fake, 1 << 20,
+                          None, None) == -2
+    # attn_decode_gqa_sparse: NULL list, group above 32 at head_dim 128
+    lib.attn_decode_gqa_sparse.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp, vp]
+    assert lib.attn_decode_gqa_sparse(fake, fake, fake, None, None, 8, 1, 8, 2, 128, 64, 0.1, fake, None, fake,
+                                      1 << 20, None, None) == -1
+    assert lib.attn_decode_gqa_sparse(fake, fake, fake, fake, None, 8, 1, 64, 1, 128, 64, 0.1, fake, None, fake,
+                                      1 << 20, None, None) == -4
+    # attn_merge_lse: no parts, unsupported head_dim
+    lib.attn_merge_lse.argtypes = [vp, vp, i32, i32, i32, i32, vp, vp, vp]
+    assert lib.attn_merge_lse(fake, fake, 0, 1, 8, 128, fake, None, None) == -3
+    assert lib.attn_merge_lse(fake, fake, 2, 1, 8, 96, fake, None, None) == -4
