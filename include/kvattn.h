@@ -116,7 +116,8 @@ int rope_table_build(const kvattn_rope_params* params, int max_pos, float* cos_o
  * For pair (a, b) with table entries (c, s): (x_a, x_b) ->
  * (x_a c - x_b s, x_a s + x_b c), computed in fp32, stored as bf16 (RNE).
  * A position outside [0, max_pos) leaves that vector unchanged and sets
- * KVATTN_STATUS_BAD_POSITION.  head_dim: multiple of 16, <= 256.
+ * KVATTN_STATUS_BAD_POSITION.  head_dim: multiple of 16, <= 256; each of q and k
+ * fewer than 2^31 chunks of 8 elements (KVATTN_ERR_SHAPE otherwise).
  */
 int rope_apply_qk(kvattn_bf16* q, int q_nb, int q_nt, int q_nh, int64_t q_sb, int64_t q_st,
                   int64_t q_sh, const int32_t* q_pos, kvattn_bf16* k, int k_nb, int k_nt, int k_nh,

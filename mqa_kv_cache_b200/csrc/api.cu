@@ -210,8 +210,8 @@ int rope_apply_qk(kvattn_bf16* q, int q_nb, int q_nt, int q_nh, int64_t q_sb, in
         if (!aligned16(v.x)) return fail(KVATTN_ERR_ALIGN, "rope_apply_qk: %s not 16-byte aligned", v.name);
         if (v.sb % 8 || v.st % 8 || v.sh % 8 || v.sb < 0 || v.st < 0 || v.sh < 0)
             return fail(KVATTN_ERR_ALIGN, "rope_apply_qk: %s strides must be non-negative multiples of 8", v.name);
-        if (static_cast<long long>(v.nb) * v.nt * v.nh > (1ll << 40))
-            return fail(KVATTN_ERR_SHAPE, "rope_apply_qk: %s too large", v.name);
+        if (static_cast<long long>(v.nb) * v.nt * v.nh * (head_dim / 8) >= (1ll << 31))
+            return fail(KVATTN_ERR_SHAPE, "rope_apply_qk: %s has 2^31 or more 16-byte chunks", v.name);
     }
     int sms = 0;
     if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "rope_apply_qk: no CUDA device");

@@ -99,6 +99,9 @@ __device__ __forceinline__ void rotate_chunk(__nv_bfloat16* vec, int chunk, int 
     }
 }
 
+// grid (x: blocks over the tensor's chunks, y: 0 = q, 1 = k).  Index arithmetic in
+// 32-bit unsigned (the host checks that every view has fewer than 2^31 chunks):
+// the three divisions per chunk are the kernel's main ALU cost.
 template <int PAIR_STYLE>
 __global__ void rope_apply_kernel(RopeView qv, RopeView kv, const float* __restrict__ cos_tab,
                                   const float* __restrict__ sin_tab, int max_pos, int head_dim,
@@ -106,29 +109,27 @@ __global__ void rope_apply_kernel(RopeView qv, RopeView kv, const float* __restr
 {
     pdl_wait();
     pdl_trigger();
+    const RopeView v = blockIdx.y == 0 ? qv : kv;
     const int half = head_dim / 2;
     // threads per head vector: one per chunk of 8 elements (adjacent pairs) or
     // per chunk of the first half (half-split pairs)
-    const int per_vec = PAIR_STYLE == 0 ? head_dim / 8 : head_dim / 16;
-    const long long q_threads = qv.n_vec * per_vec;
-    const long long total = q_threads + kv.n_vec * per_vec;
-    for (long long tid = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; tid < total;
-         tid += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const bool is_q = tid < q_threads;
-        const RopeView& v = is_q ? qv : kv;
-        const long long local = is_q ? tid : tid - q_threads;
-        const long long vec = local / per_vec;
-        const int chunk = static_cast<int>(local - vec * per_vec);
-        const int h = static_cast<int>(vec % v.nh);
-        const long long bt = vec / v.nh;
-        const int t = static_cast<int>(bt % v.nt);
-        const long long b = bt / v.nt;
+    const unsigned per_vec = PAIR_STYLE == 0 ? head_dim / 8 : head_dim / 16;
+    const unsigned total = static_cast<unsigned>(v.n_vec) * per_vec;
+    const unsigned nh = static_cast<unsigned>(v.nh), nt = static_cast<unsigned>(v.nt);
+    for (unsigned tid = blockIdx.x * blockDim.x + threadIdx.x; tid < total; tid += gridDim.x * blockDim.x) {
+        const unsigned vec = tid / per_vec;
+        const int chunk = static_cast<int>(tid - vec * per_vec);
+        const unsigned bt = vec / nh;
+        const int h = static_cast<int>(vec - bt * nh);
+        const unsigned b = bt / nt;
+        const int t = static_cast<int>(bt - b * nt);
         const int m = v.pos[bt];
         if (m < 0 || m >= max_pos) {
             if (chunk == 0) report_status(dev_status, KVATTN_STATUS_BAD_POSITION);
             continue;
         }
-        __nv_bfloat16* base = v.x + b * v.sb + static_cast<long long>(t) * v.st + static_cast<long long>(h) * v.sh;
+        __nv_bfloat16* base = v.x + static_cast<long long>(b) * v.sb + static_cast<long long>(t) * v.st +
+                              static_cast<long long>(h) * v.sh;
         rotate_chunk<PAIR_STYLE>(base, chunk, half, cos_tab + static_cast<long long>(m) * half,
                                  sin_tab + static_cast<long long>(m) * half);
     }
@@ -192,14 +193,15 @@ cudaError_t launch_rope_apply(const RopeApplyArgs& a, cudaStream_t stream)
                 a.k ? static_cast<long long>(a.k_nb) * a.k_nt * a.k_nh : 0, a.k_nt > 0 ? a.k_nt : 1,
                 a.k_nh > 0 ? a.k_nh : 1, a.k_sb, a.k_st, a.k_sh};
     const int per_vec = a.pair_style == 0 ? a.head_dim / 8 : a.head_dim / 16;
-    const long long total = (qv.n_vec + kv.n_vec) * per_vec;
-    if (total == 0) return cudaSuccess;
+    const long long most = (qv.n_vec > kv.n_vec ? qv.n_vec : kv.n_vec) * per_vec;
+    if (most == 0) return cudaSuccess;
+    if (most >= (1ll << 31)) return cudaErrorInvalidValue;  // the kernel indexes chunks in 32 bits
     const int threads = 256;
-    long long blocks = (total + threads - 1) / threads;
-    const long long cap = static_cast<long long>(a.num_sms) * 16;
+    long long blocks = (most + threads - 1) / threads;
+    const long long cap = static_cast<long long>(a.num_sms) * 8;  // 8 x 256 threads resident per SM
     if (blocks > cap) blocks = cap;
     auto kern = a.pair_style == 0 ? rope_apply_kernel<0> : rope_apply_kernel<1>;
-    return launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, qv, kv, a.cos_tab,
+    return launch_pdl(kern, dim3(static_cast<unsigned>(blocks), 2), dim3(threads), 0, stream, qv, kv, a.cos_tab,
                       a.sin_tab, a.max_pos, a.head_dim, a.dev_status);
 }
 
