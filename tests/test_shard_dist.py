@@ -68,3 +68,18 @@ def test_two_ranks_gather_and_merge(tmp_path):
             o, l = oracle.softmax_merge(parts[0][:, b, h], lses[0][:, b, h])
             np.testing.assert_allclose(o, full_o[b, h], rtol=1e-12, atol=1e-12)
             np.testing.assert_allclose(l, full_l[b, h], rtol=1e-12)
+
+
+def test_shard_lengths_partition_every_row():
+    """The slices' lengths add up to the row's length (capped at the slices' total) and
+    each slice's rows are a prefix of it."""
+    from mqa_kv_cache_b200 import shard
+    lens = torch.tensor([0, 1, 99, 100, 101, 250, 400], dtype=torch.int32)
+    S, n = 100, 4
+    parts = torch.stack([shard.shard_lengths(lens, r, S) for r in range(n)])
+    assert parts.dtype == torch.int32
+    assert torch.equal(parts.sum(0), lens.clamp(max=S * n))
+    assert torch.all((parts >= 0) & (parts <= S))
+    # a slice is full before the next one holds anything
+    for r in range(n - 1):
+        assert torch.all((parts[r + 1] == 0) | (parts[r] == S))
