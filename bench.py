@@ -34,11 +34,55 @@ sys.path.insert(0, ROOT)
 from mqa_kv_cache_b200 import workloads as W  # noqa: E402
 
 METRIC = "decode-attn effective HBM GB/s (% of peak) & tok/s; prefill TFLOP/s"
-# DRAM bytes (read + write) of one decode_kernel launch on the headline workload, from an ncu
-# capture of the current kernel (dram__bytes_read.sum + dram__bytes_write.sum); None once the
-# kernel changes after that capture.
-DECODE_TRAFFIC_BYTES = 295_056_640 + 4_192_768
 L2_FLUSH_BYTES = 256 << 20
+# The committed ncu summary of the headline decode kernel records its DRAM traffic per
+# launch (dram__bytes_read.sum + dram__bytes_write.sum) together with a hash of the kernel
+# sources it was captured from; the traffic is reported only while the sources still match.
+DECODE_PROFILE = os.path.join(ROOT, "profiles", "decode_kernel_llama3_8b_ragged_B16_H32_Hk8.md")
+DECODE_SOURCES = ["decode.cu", "decode_plan.cuh", "common.cuh", "kernels.h"]
+
+
+def kernel_sources_sha256(names):
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "mqa_kv_cache_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def profile_traffic(path, sources):
+    """(bytes per launch, note): the traffic a committed ncu summary records, or None
+    when the summary is missing or the kernel sources changed since its capture."""
+    import re
+    try:
+        text = open(path).read()
+    except OSError:
+        return None, "no committed ncu summary"
+    t = re.search(r"traffic_bytes_per_launch:\s*(\d+)", text)
+    h = re.search(r"sources_sha256:\s*([0-9a-f]{64})", text)
+    if not t or not h:
+        return None, "the ncu summary records no traffic"
+    if h.group(1) != kernel_sources_sha256(sources):
+        return None, "kernel sources changed since the committed ncu capture"
+    return int(t.group(1)), "ncu capture of the current kernel sources (" + os.path.basename(path) + ")"
+
+
+def measure_read_stream(device, nbytes=4 << 30, reps=5):
+    """Best read-only streaming rate (GB/s) of a plain reduction over nbytes: the
+    read-side counterpart of the copy figure (which moves read + write bytes)."""
+    x = torch.ones(nbytes // 4, dtype=torch.float32, device=device)
+    best = float("inf")
+    for _ in range(reps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        torch.sum(x)
+        b.record()
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b))
+    del x
+    torch.cuda.empty_cache()
+    return nbytes / (best * 1e-3) / 1e9
 
 
 def load_peaks():
@@ -277,6 +321,8 @@ def run_gpu(args, rank, world, device):
 
     gbs = total_bytes / (ms * 1e-3) / 1e9
     attn_gbs = job.bytes / (attn_ms * 1e-3) / 1e9
+    traffic, traffic_note = profile_traffic(DECODE_PROFILE, DECODE_SOURCES)
+    read_gbs = measure_read_stream(device)
     line = {
         "metric": METRIC,
         "value": round(gbs, 2),
@@ -303,8 +349,11 @@ def run_gpu(args, rank, world, device):
         "roofline": {"kernel": "decode_kernel (attn_decode_gqa_rope: RoPE of q, split-K decode, merge)",
                      "bound": "hbm",
                      "achieved": round(attn_gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(attn_gbs / peaks["hbm_gbs"], 4), "traffic": DECODE_TRAFFIC_BYTES,
-                     "peak_source": peaks["source"], "algorithmic_bytes": job.bytes},
+                     "frac": round(attn_gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
+                     "traffic_source": traffic_note,
+                     "peak_source": peaks["source"], "algorithmic_bytes": job.bytes,
+                     "read_stream_gbs": round(read_gbs, 1), "frac_of_read_stream": round(attn_gbs / read_gbs, 4),
+                     "frac_of_nominal_8tbs": round(attn_gbs / 8000.0, 4)},
         "e2e": {"value": round(total_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": job.launches_per_step * args.steps,
@@ -334,7 +383,9 @@ def measure_decode_config(K, w, device, steps, flush, peaks):
            "attn_ms": round(attn_ms, 5), "algorithmic_bytes": job.bytes,
            "GB_s": round(job.bytes / (ms * 1e-3) / 1e9, 1),
            "pct_of_hbm_peak": round(100 * job.bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 1),
+           "pct_of_nominal_8tbs": round(100 * job.bytes / (ms * 1e-3) / 1e9 / 8000.0, 1),
            "attn_pct_of_hbm_peak": round(100 * job.bytes / (attn_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 1),
+           "attn_pct_of_nominal_8tbs": round(100 * job.bytes / (attn_ms * 1e-3) / 1e9 / 8000.0, 1),
            "tok_per_s": round(w.B / (ms * 1e-3), 1)}
     del job
     torch.cuda.empty_cache()
@@ -533,6 +584,7 @@ def measure_window(K, device, steps, flush, peaks):
             "ms_per_step": round(ms, 5), "algorithmic_bytes": nbytes,
             "GB_s": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "pct_of_hbm_peak": round(100 * nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 1),
+            "pct_of_nominal_8tbs": round(100 * nbytes / (ms * 1e-3) / 1e9 / 8000.0, 1),
             "tok_per_s": round(w.B / (ms * 1e-3), 1)}
 
 

@@ -67,6 +67,26 @@ const char* kvattn_last_error_string(void);
 /* Library version string. */
 const char* kvattn_version(void);
 
+/*
+ * Failure-detection testing.  The pages have no counterpart: this hook exists
+ * so that a test can make a pipeline wait run out on the GPU without a fault.
+ * Every wait inside the kernels is bounded (about a second of %globaltimer);
+ * when one runs out the kernel stops using its pipeline, ORs
+ * KVATTN_STATUS_TIMEOUT into *dev_status and returns, and the CUDA context
+ * stays usable.  After this call, decode calls made by the calling thread
+ * (attn_decode_gqa, attn_decode_gqa_rope, attn_decode_gqa_rope_window) whose
+ * group size is at most 32, or whose head_dim is 64, bound each pipeline wait
+ * by wait_limit_ns instead (0 = the default), and, when drop_tile >= 0, the
+ * first persistent CTA never issues the loads of its tile number drop_tile,
+ * so the waits for that tile run out: the call then reports
+ * KVATTN_STATUS_TIMEOUT, its outputs are invalid, and the workspace's counter
+ * region must be cleared before the workspace is used again.  Nothing is
+ * loaded and abandoned; every copy issued completes before the kernel returns.
+ * kvattn_test_decode_stall(-1, 0) restores normal operation.
+ * Errors: KVATTN_ERR_SHAPE (drop_tile < -1, or a limit outside 0 .. 10 s).
+ */
+int kvattn_test_decode_stall(int drop_tile, long long wait_limit_ns);
+
 /* ---- RoPE ----------------------------------------------------------------
  * "Agentic RL 入门3：transformer 架构" §1.1 (rotation R(m, theta_i),
  * theta_i = base^(-2i/d)), §1.2 ① PI, ② NTK-aware, ③ YaRN (NTK-by-parts
@@ -246,11 +266,22 @@ int attn_decode_gqa_rope_window(const kvattn_bf16* q, const int32_t* q_pos, cons
  * address up (cudaGetSymbolAddress); make that first call before any stream
  * capture.  All calls on a device share the one array: it starts zeroed, as
  * the counter region at its start requires, and every call leaves that region
- * zero (after a KVATTN_STATUS_TIMEOUT the results of later calls on the device
- * are undefined).  Calls that can overlap on the GPU -- different streams, or
- * graphs replayed concurrently -- race and corrupt each other's results.
+ * zero, except one that reports KVATTN_STATUS_TIMEOUT: after it, call
+ * attn_decode_gqa_noalloc_reset before the next call on that device.  Calls
+ * that can overlap on the GPU -- different streams, or graphs replayed
+ * concurrently -- race and corrupt each other's results.
  */
 #define KVATTN_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * Zero the counter region (the first KVATTN_DECODE_WS_ZERO_BYTES) of the
+ * static array that attn_decode_gqa_noalloc uses, on the current device, as an
+ * asynchronous memset on `stream`; it allocates nothing.  Needed only after a
+ * call that reported KVATTN_STATUS_TIMEOUT.  The array's device address is
+ * looked up once per device and kept for the life of the process, so neither
+ * entry point may be used on a device after cudaDeviceReset.
+ */
+int attn_decode_gqa_noalloc_reset(void* stream);
 
 int attn_decode_gqa_noalloc(const kvattn_bf16* q, const kvattn_bf16* k_cache, const kvattn_bf16* v_cache,
                             const int32_t* seq_lens, int B, int n_head, int n_kv_head, int head_dim,

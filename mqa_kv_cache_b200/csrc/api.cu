@@ -77,21 +77,80 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
+// Encoded tensor maps, kept per (device, rank, base address, extents, box): a map
+// holds nothing but those, so a cached one is the map a fresh encode would give.
+// Decode steps call with the same cache pointers every step; the cache saves the
+// host-side encodes on each call.  Replacement is round-robin.
+struct MapKey {
+    int dev, rank;
+    const void* base;
+    uint64_t dims[4];
+    uint32_t box;
+    bool operator==(const MapKey& o) const
+    {
+        return dev == o.dev && rank == o.rank && base == o.base && box == o.box && dims[0] == o.dims[0] &&
+               dims[1] == o.dims[1] && dims[2] == o.dims[2] && dims[3] == o.dims[3];
+    }
+};
+constexpr int kMapSlots = 64;
+struct MapCache {
+    std::mutex mu;
+    MapKey key[kMapSlots];
+    CUtensorMap map[kMapSlots];
+    bool used[kMapSlots] = {};
+    int next = 0;
+};
+MapCache& map_cache()
+{
+    static MapCache c;
+    return c;
+}
+
+// bf16 tensor map of rank 3 ([z][y][x], box {64, box, 1}) or 4 ([w][z][y][x], box
+// {64, 1, box, 1}), 128-byte swizzle, zero fill out of range; from the cache when present.
+int make_map(CUtensorMap* map, int rank, const void* base, const uint64_t (&d)[4], uint32_t box_rows)
+{
+    MapKey key{};
+    if (cudaGetDevice(&key.dev) != cudaSuccess) return fail(KVATTN_ERR_CUDA, "no CUDA device");
+    key.rank = rank;
+    key.base = base;
+    for (int i = 0; i < 4; ++i) key.dims[i] = i < rank ? d[i] : 0;
+    key.box = box_rows;
+    MapCache& c = map_cache();
+    {
+        std::lock_guard<std::mutex> lk(c.mu);
+        for (int i = 0; i < kMapSlots; ++i)
+            if (c.used[i] && c.key[i] == key) {
+                *map = c.map[i];
+                return KVATTN_OK;
+            }
+    }
+    auto fn = encode_fn();
+    if (!fn) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint64_t dims[4] = {d[0], d[1], d[2], d[3]};
+    cuuint64_t strides[3] = {d[0] * 2, d[0] * d[1] * 2, d[0] * d[1] * d[2] * 2};
+    cuuint32_t box3[3] = {64, box_rows, 1};
+    cuuint32_t box4[4] = {64, 1, box_rows, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+                    rank == 3 ? box3 : box4, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    std::lock_guard<std::mutex> lk(c.mu);
+    const int i = c.next;
+    c.next = (c.next + 1) % kMapSlots;
+    c.key[i] = key;
+    c.map[i] = *map;
+    c.used[i] = true;
+    return KVATTN_OK;
+}
+
 // 3-D bf16 tensor map over [z][y][x] (x innermost) with a {64, box_y, 1} box and
 // 128-byte swizzle; out-of-range rows read as zero.
 int make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint32_t box_y)
 {
-    auto fn = encode_fn();
-    if (!fn) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    cuuint64_t dims[3] = {x, y, z};
-    cuuint64_t strides[2] = {x * 2, x * y * 2};
-    cuuint32_t box[3] = {64, box_y, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return KVATTN_OK;
+    const uint64_t d[4] = {x, y, z, 0};
+    return make_map(map, 3, base, d, box_y);
 }
 
 // 4-D bf16 tensor map over [w][z][y][x] with a {64, 1, box_z, 1} box and
@@ -99,17 +158,8 @@ int make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint
 int make_map_4d_rows(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z, uint64_t w,
                      uint32_t box_z)
 {
-    auto fn = encode_fn();
-    if (!fn) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    cuuint64_t dims[4] = {x, y, z, w};
-    cuuint64_t strides[3] = {x * 2, x * y * 2, x * y * z * 2};
-    cuuint32_t box[4] = {64, 1, box_z, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return KVATTN_OK;
+    const uint64_t d[4] = {x, y, z, w};
+    return make_map(map, 4, base, d, box_z);
 }
 
 int cuda_status(cudaError_t e, const char* what)
@@ -119,6 +169,10 @@ int cuda_status(cudaError_t e, const char* what)
 }
 
 bool g_supported(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16 || g == 32 || g == 64; }
+
+// Failure-detection test settings of the calling thread (kvattn_test_decode_stall).
+thread_local int g_test_drop_tile = -1;
+thread_local unsigned long long g_test_wait_ns = 0;
 
 // Decode workspace layout for a given grid.
 // [0, KVATTN_DECODE_WS_ZERO_BYTES): per-unit piece counters (zero between calls, at a
@@ -154,7 +208,18 @@ extern "C" {
 
 const char* kvattn_last_error_string(void) { return g_err; }
 
-const char* kvattn_version(void) { return "kvattn 0.1.0 (sm_100a)"; }
+const char* kvattn_version(void) { return "kvattn 0.2.0 (sm_100a)"; }
+
+int kvattn_test_decode_stall(int drop_tile, long long wait_limit_ns)
+{
+    if (drop_tile < -1) return fail(KVATTN_ERR_SHAPE, "kvattn_test_decode_stall: drop_tile %d < -1", drop_tile);
+    if (wait_limit_ns < 0 || wait_limit_ns > 10000000000ll)
+        return fail(KVATTN_ERR_SHAPE, "kvattn_test_decode_stall: wait limit %lld ns outside 0 .. 10 s",
+                    wait_limit_ns);
+    g_test_drop_tile = drop_tile;
+    g_test_wait_ns = static_cast<unsigned long long>(wait_limit_ns);
+    return ok();
+}
 
 // ---------------------------------------------------------------------------
 int rope_table_build(const kvattn_rope_params* p, int max_pos, float* cos_out, float* sin_out, void* stream)
@@ -352,6 +417,8 @@ static int decode_call(const char* name, const kvattn_bf16* q, const kvattn_bf16
     a.T_max = T_max;
     a.scale = scale;
     a.grid = grid;
+    a.wait_ns = g_test_wait_ns;
+    a.drop_it = g_test_drop_tile;
     return cuda_status(kvattn::launch_decode(a, tm_q, tm_k, tm_v, static_cast<cudaStream_t>(stream)),
                        name);
 }

@@ -83,13 +83,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 
 // Wait for the phase with the given parity to complete.  Returns false when
 // the time limit ran out (the caller must then stop using the pipeline).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          unsigned long long limit_ns = WAIT_LIMIT_NS)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) return false;
+        if (global_timer_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -97,12 +98,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity)
 // every lane waits (so every lane gets the barrier's memory ordering), and the
 // warp proceeds only if all lanes saw the phase complete and no abort had been
 // raised.  On a timeout the shared abort flag is set.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = WAIT_LIMIT_NS)
 {
     int go = *abort_flag == 0;
     go = __shfl_sync(0xffffffffu, go, 0);
     if (!go) return false;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, parity, limit_ns));
     if (!ok) *abort_flag = 1;
     return ok;
 }

@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
     int* s_idx = reinterpret_cast<int*>(smem + C::OFF_IDX);  // staged row indices, per producer warp (gather)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned long long wlim = a.wait_ns ? a.wait_ns : WAIT_LIMIT_NS;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
             // gather mode: every producer lane arrives once its copies land, plus the mask arrival
@@ -295,8 +296,8 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
             const int z = w.b * a.Hk + w.kvh;
             // the piece's g query rows (contiguous), once the consumers hold the previous ones
             if (np > 0 && pw == 0) {
-                const bool got = GATHER ? warp_wait(q_empty, (np - 1) & 1, s_abort)
-                                        : (!*s_abort && mbar_wait(q_empty, (np - 1) & 1));
+                const bool got = GATHER ? warp_wait(q_empty, (np - 1) & 1, s_abort, wlim)
+                                        : (!*s_abort && mbar_wait(q_empty, (np - 1) & 1, wlim));
                 if (!got) {
                     ok = false;
                     break;
@@ -338,8 +339,8 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
                 const int s = it % C::STAGES;
                 const uint32_t ph = (it / C::STAGES) & 1;
                 if (it >= C::STAGES) {
-                    const bool got = GATHER ? warp_wait(&empty[s], ph ^ 1, s_abort)
-                                            : (!*s_abort && mbar_wait(&empty[s], ph ^ 1));
+                    const bool got = GATHER ? warp_wait(&empty[s], ph ^ 1, s_abort, wlim)
+                                            : (!*s_abort && mbar_wait(&empty[s], ph ^ 1, wlim));
                     if (!got) {
                         ok = false;
                         break;
@@ -348,6 +349,7 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
                 uint8_t* kd = smem + s * C::STAGE_BYTES;
                 uint8_t* vd = kd + C::TILE_BYTES;
                 if constexpr (!GATHER) {
+                    if (blockIdx.x == 0 && it == a.drop_it) continue;  // testing: a tile never loaded
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
 #pragma unroll
                     for (int h = 0; h < C::HALVES; ++h) {
@@ -399,8 +401,8 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
         if (GATHER) cp_async_wait<0>();
         if (lane == 0 && pw == 0) {
             for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
-                mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
-            if (np > 0) mbar_wait(q_full, (np - 1) & 1);
+                mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1, wlim);
+            if (np > 0) mbar_wait(q_full, (np - 1) & 1, wlim);
         }
         return;
     }
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
         // query fragments (A operand) from the prefetched rows: heads of the group, zero beyond g
         uint32_t qa[KS][4];
         {
-            const bool have_q = warp_wait(q_full, piece & 1, s_abort);
+            const bool have_q = warp_wait(q_full, piece & 1, s_abort, wlim);
             const uint8_t* qg = sQ;
             if (rope) {
                 // rotate the piece's g query rows in place (bad positions: flagged, left as given)
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
         for (long long t = tb; t < te; ++t, ++it) {
             const int s = it % C::STAGES;
             const uint32_t ph = (it / C::STAGES) & 1;
-            const bool have = warp_wait(&full[s], ph, s_abort);
+            const bool have = warp_wait(&full[s], ph, s_abort, wlim);
             if (!have && lane == 0) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
             if (have) {
                 const uint32_t sK = smem_u32(smem + s * C::STAGE_BYTES);

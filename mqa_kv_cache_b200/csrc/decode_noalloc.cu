@@ -16,8 +16,15 @@
 //  - every call on a device uses the same array: calls that may run at the
 //    same time on the GPU (different streams, or graphs replayed
 //    concurrently) race and corrupt each other's results;
-//  - the array keeps whatever the previous call left; the decode kernels
-//    write every scratch entry before they read it, so nothing needs clearing;
+//  - the array keeps whatever the previous call left.  Its first
+//    KVATTN_DECODE_WS_ZERO_BYTES hold the per-(batch, KV head) piece counters
+//    that the split-K merge counts on: they start zero because the array is
+//    zero-initialised when the module loads, and every call leaves them zero
+//    again -- except a call that reports KVATTN_STATUS_TIMEOUT, after which
+//    attn_decode_gqa_noalloc_reset must clear them.  The rest of the array
+//    (partial outputs and their max/sum) is written before it is read;
+//  - the array's device address is looked up once per device and kept, so
+//    the entry points may not be used on a device after cudaDeviceReset;
 //  - every GPU that loads this library holds the array until the process
 //    exits.
 #include <mutex>
@@ -71,6 +78,19 @@ int attn_decode_gqa_noalloc(const kvattn_bf16* q, const kvattn_bf16* k_cache, co
     // need == 0 means the shape is invalid: attn_decode_gqa reports why.
     return attn_decode_gqa(q, k_cache, v_cache, seq_lens, B, n_head, n_kv_head, head_dim, T_max, scale, out, lse,
                            scratch, KVATTN_NOALLOC_SCRATCH_BYTES, dev_status, stream);
+}
+
+int attn_decode_gqa_noalloc_reset(void* stream)
+{
+    void* scratch = nullptr;
+    if (scratch_address(&scratch) != 0)
+        return kvattn::record_error(KVATTN_ERR_CUDA,
+                                    "attn_decode_gqa_noalloc_reset: cudaGetSymbolAddress of the static scratch failed");
+    const cudaError_t e =
+        cudaMemsetAsync(scratch, 0, KVATTN_DECODE_WS_ZERO_BYTES, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return kvattn::record_error(KVATTN_ERR_CUDA, "attn_decode_gqa_noalloc_reset: %s", cudaGetErrorString(e));
+    return kvattn::record_error(KVATTN_OK, "%s", "");
 }
 
 }  // extern "C"

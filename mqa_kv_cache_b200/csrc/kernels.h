@@ -99,6 +99,11 @@ struct DecodeArgs {
     int B, H, Hk, g, d, T_max;
     float scale;
     int grid;        // persistent CTAs (also the number of tile ranges)
+    // Failure-detection testing (mma.sync kernel, tensor-map mode): each pipeline wait
+    // gives up after wait_ns (0: WAIT_LIMIT_NS), and CTA 0 issues no loads for its
+    // tile number drop_it (-1: none), so that its consumers' waits run out.
+    unsigned long long wait_ns = 0;
+    int drop_it = -1;
 };
 // Number of partial slots the decode kernel may write for a given grid.
 long long decode_max_slots(int B, int Hk, int grid);

@@ -69,6 +69,8 @@ _lib.attn_decode_gqa_sparse_workspace_bytes.restype = _sz
 _lib.attn_decode_gqa_sparse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp,
                                         _vp, _sz, _vp, _vp]
 _lib.attn_merge_lse.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.kvattn_test_decode_stall.argtypes = [_i32, ctypes.c_longlong]
+_lib.attn_decode_gqa_noalloc_reset.argtypes = [_vp]
 
 ROPE_NONE, ROPE_PI, ROPE_NTK, ROPE_YARN, ROPE_DYN_NTK = 0, 1, 2, 3, 4
 STATUS_BAD_POSITION, STATUS_BAD_LENGTH, STATUS_BAD_INDEX, STATUS_NAN_SCORE, STATUS_TIMEOUT = 1, 2, 4, 8, 16
@@ -78,6 +80,18 @@ class KvattnError(RuntimeError):
     def __init__(self, code: int, msg: str):
         super().__init__(f"kvattn error {code}: {msg}")
         self.code = code
+
+
+def kvattn_test_decode_stall(drop_tile: int = -1, wait_limit_ns: int = 0):
+    """kvattn_test_decode_stall: failure-detection testing only (see the header).
+    (-1, 0) restores normal operation."""
+    _check(_lib.kvattn_test_decode_stall(int(drop_tile), int(wait_limit_ns)))
+
+
+def attn_decode_gqa_noalloc_reset():
+    """Zero the counter region of the allocation-free decode's static scratch
+    (on the current stream); needed only after a call that timed out."""
+    _check(_lib.attn_decode_gqa_noalloc_reset(_stream()))
 
 
 def library():

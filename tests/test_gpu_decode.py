@@ -155,6 +155,53 @@ def test_llama2_70b_32k_sampled_heads(K, wl):
         assert_attn_close(out[b:b + 1, h:h + 1], ro, lse[b:b + 1, h:h + 1], rl, f"{wl.name} b={b} h={h}")
 
 
+@pytest.mark.parametrize("wl", [W.LLAMA2_70B_GQA_32K, W.LLAMA2_70B_MQA_32K, W.LLAMA2_70B_MHA_32K],
+                         ids=["gqa", "mqa", "mha"])
+def test_llama2_70b_32k_yarn_chain_full_size(K, wl):
+    """The 32K shapes as the bench times them: raw keys rotated at positions
+    0..32767 with the YaRN s = 4 table (cos/sin carrying 0.1 ln 4 + 1), then
+    attn_decode_gqa_rope with the raw queries rotated at position 32768 inside
+    the decode kernel (the tcgen05 kernel for MQA).  Sampled (batch, head)
+    outputs are checked against the oracle's fp64 chain (RoPE then attention),
+    and against the oracle's attention on the GPU's own rotated q and k with the
+    plain lse tolerance."""
+    dev = torch.device("cuda")
+    T = wl.T_max
+    gen = W.generator(W.SEED_BASE + wl.index + 200, dev)
+    q = W.normal_bf16((wl.B, wl.H, wl.d), gen, dev)
+    k = W.normal_bf16((wl.B, wl.Hk, T, wl.d), gen, dev)
+    v = W.normal_bf16((wl.B, wl.Hk, T, wl.d), gen, dev)
+    rng = np.random.default_rng(wl.index + 7)
+    picks = [(int(rng.integers(wl.B)), int(rng.integers(wl.H))) for _ in range(10)]
+    picks += [(0, 0), (wl.B - 1, wl.H - 1)]
+    raw_k = {(b, h // wl.g): k[b:b + 1, h // wl.g:h // wl.g + 1].cpu() for b, h in picks}
+    r = wl.rope
+    p = K.rope_params(wl.d, base=r.base, scaling=r.scaling, s=r.s, L_train=r.L_train, alpha=r.alpha, beta=r.beta)
+    cos, sin = K.rope_table_build(p, T + 1)
+    K.rope_apply_qk(None, None, k, torch.arange(T, dtype=torch.int32, device=dev).repeat(wl.B, 1), cos, sin,
+                    k_layout="bhtd")
+    lens = torch.full((wl.B,), T, dtype=torch.int32, device=dev)
+    out, lse = K.attn_decode_gqa_rope(q, lens, cos, sin, k, v, lens, wl.scale)
+    q_rot = q.clone()
+    K.rope_apply_qk(q_rot, lens.view(wl.B, 1), None, None, cos, sin, q_layout="bhd")
+    torch.cuda.synchronize()
+    c, s = oracle.rope_table(wl.d, r.base, T + 1, r.scaling, s=r.s, L_train=r.L_train, alpha=r.alpha, beta=r.beta)
+    kpos = np.arange(T, dtype=np.int32)[None, :]
+    one = np.array([T], np.int32)
+    for b, h in picks:
+        kvh = h // wl.g
+        qr = oracle.rope_apply(W.bf16_bits(q[b:b + 1, h:h + 1].cpu())[:, None], np.array([[T]], np.int32), c, s)[:, 0]
+        kr = oracle.rope_apply(W.bf16_bits(raw_k[(b, kvh)]), kpos, c, s, layout="bhtd")
+        vb = W.bf16_bits(v[b:b + 1, kvh:kvh + 1].cpu())
+        ro, rl = oracle.attn_decode(qr, kr, oracle.bf16_bits_to_f64(vb), one, wl.scale)
+        tol = chain_lse_tol(np.linalg.norm(qr, axis=-1), np.linalg.norm(kr, axis=-1).max(axis=-1), wl.scale)
+        o_bh, l_bh = out[b:b + 1, h:h + 1], lse[b:b + 1, h:h + 1]
+        assert_attn_close(o_bh, ro, l_bh, rl, f"{wl.name} yarn chain b={b} h={h}", lse_tol=tol)
+        ro2, rl2 = oracle.attn_decode(W.bf16_bits(q_rot[b:b + 1, h:h + 1].cpu()),
+                                      W.bf16_bits(k[b:b + 1, kvh:kvh + 1].cpu()), vb, one, wl.scale)
+        assert_attn_close(o_bh, ro2, l_bh, rl2, f"{wl.name} b={b} h={h} on the GPU-rotated q/k")
+
+
 @pytest.mark.parametrize("wl,T_max", [(W.TINY_GQA, 256), (W.LLAMA3_8B_DECODE, 1500),
                                       (W.LLAMA2_70B_GQA_32K, 2048)], ids=["tiny", "llama3", "yarn"])
 def test_chain_rope_then_decode(K, wl, T_max):
@@ -179,6 +226,11 @@ def test_chain_rope_then_decode(K, wl, T_max):
     kmax = np.linalg.norm(kr, axis=-1).max(axis=-1)        # [B, Hk] (rows past the length included: an upper bound)
     kmax_h = np.repeat(kmax, wl.g, axis=1)
     assert_attn_close(out, ro, lse, rl, f"chain {wl.name}", lse_tol=chain_lse_tol(qn, kmax_h, wl.scale))
+    # the attention step alone, on the q and k the GPU rotated (its bf16 roundings
+    # included): the plain lse tolerance applies
+    ro2, rl2 = oracle.attn_decode(W.bf16_bits(qg.cpu()), W.bf16_bits(kg.cpu()), W.bf16_bits(inp["v"]),
+                                  inp["seq_lens"].numpy(), wl.scale)
+    assert_attn_close(out, ro2, lse, rl2, f"chain {wl.name} on the GPU-rotated q/k")
 
 
 ZERO_BYTES = 64 << 10  # KVATTN_DECODE_WS_ZERO_BYTES: the per-unit counters at the start of the workspace

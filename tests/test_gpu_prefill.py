@@ -102,6 +102,9 @@ def test_chain_rope_then_prefill(K):
     kmax = np.linalg.norm(kr, axis=-1).max(axis=-1)       # [B, Hk]
     kmax_h = np.repeat(kmax, wl.H // wl.Hk, axis=1)[:, :, None]
     assert_attn_close(out, ro, lse, rl, "chain prefill", lse_tol=chain_lse_tol(qn, kmax_h, wl.scale))
+    # the attention step alone on the GPU-rotated q and k: the plain lse tolerance
+    ro2, rl2 = oracle.attn_prefill(W.bf16_bits(qg.cpu()), W.bf16_bits(kg.cpu()), W.bf16_bits(inp["v"]), wl.scale)
+    assert_attn_close(out, ro2, lse, rl2, "chain prefill on the GPU-rotated q/k")
 
 
 def test_deterministic(K):

@@ -49,6 +49,27 @@ def test_fused_equals_rope_then_decode(K, pair_style, B, H, Hk, d, T_max):
     assert torch.equal(out_f, out_u) and torch.equal(lse_f, lse_u)
 
 
+@pytest.mark.parametrize("B,H,Hk,d,T_max", [(3, 16, 2, 128, 2100), (2, 64, 1, 128, 2100), (2, 8, 8, 64, 900)])
+def test_fused_equals_rope_then_decode_yarn(K, B, H, Hk, d, T_max):
+    """As above with the YaRN s = 4 table, whose cos/sin carry the temperature
+    factor 0.1 ln 4 + 1 (rows of magnitude other than 1)."""
+    gen = W.generator(57 + H + d)
+    q = W.normal_bf16((B, H, d), gen).cuda()
+    k = W.normal_bf16((B, Hk, T_max, d), gen).cuda()
+    v = W.normal_bf16((B, Hk, T_max, d), gen).cuda()
+    lens = torch.randint(1, T_max + 1, (B,), generator=torch.Generator().manual_seed(T_max + H), dtype=torch.int32)
+    lens = lens.cuda()
+    p = K.rope_params(d, base=10000.0, scaling=K.ROPE_YARN, s=4.0, L_train=512.0, alpha=1.0, beta=32.0)
+    cos, sin = K.rope_table_build(p, T_max + 1, device="cuda")
+    assert abs(float(torch.hypot(cos[7], sin[7]).mean()) - (0.1 * np.log(4.0) + 1.0)) < 1e-5
+    out_f, lse_f = K.attn_decode_gqa_rope(q, lens, cos, sin, k, v, lens, d ** -0.5)
+    q_rot = q.clone()
+    K.rope_apply_qk(q_rot, lens.view(B, 1), None, None, cos, sin, q_layout="bhd")
+    out_u, lse_u = K.attn_decode_gqa(q_rot, k, v, lens, d ** -0.5)
+    torch.cuda.synchronize()
+    assert torch.equal(out_f, out_u) and torch.equal(lse_f, lse_u)
+
+
 def test_fused_chain_against_oracle(K):
     wl = W.LLAMA3_8B_DECODE
     inp = W.decode_inputs(wl, B=4, T_max=3000, seed=77)
@@ -69,6 +90,14 @@ def test_fused_chain_against_oracle(K):
     qn = np.linalg.norm(qr, axis=-1)
     kmax = np.repeat(np.linalg.norm(kr, axis=-1).max(axis=-1), wl.g, axis=1)
     assert_attn_close(out, ro, lse, rl, "fused chain", lse_tol=chain_lse_tol(qn, kmax, wl.scale))
+    # on the GPU's own rotated q (rope_apply_qk rotates bit-identically to the fused
+    # prologue) and rotated cache: the plain lse tolerance
+    q_rot = inp["q"].cuda()
+    K.rope_apply_qk(q_rot, inp["q_pos"].view(B, 1).cuda(), None, None, cos, sin, q_layout="bhd")
+    torch.cuda.synchronize()
+    ro2, rl2 = oracle.attn_decode(W.bf16_bits(q_rot.cpu()), W.bf16_bits(k.cpu()), W.bf16_bits(inp["v"]),
+                                  inp["seq_lens"].numpy(), wl.scale)
+    assert_attn_close(out, ro2, lse, rl2, "fused chain on the GPU-rotated q/k")
 
 
 @pytest.mark.parametrize("H,Hk", [(8, 2), (64, 1)])

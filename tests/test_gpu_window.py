@@ -67,6 +67,14 @@ def test_ring_append_then_window_decode(K, H, Hk, n_sink, window):
     qn = np.linalg.norm(qr, axis=-1)
     kmax = np.repeat(np.linalg.norm(kr, axis=-1).max(axis=-1), H // Hk, axis=1)
     assert_attn_close(out, ro, lse, rl, f"window s={n_sink} w={window}", lse_tol=chain_lse_tol(qn, kmax, scale))
+    # on the GPU-rotated q (rope_apply_qk, bit-identical to the fused prologue) and keys:
+    # the plain lse tolerance
+    q_rot = q_raw.cuda()
+    K.rope_apply_qk(q_rot, lens_t.view(B, 1), None, None, cos, sin, q_layout="bhd")
+    torch.cuda.synchronize()
+    ro2, rl2 = oracle.attn_decode_window(W.bf16_bits(q_rot.cpu()), W.bf16_bits(k_rot.cpu()), W.bf16_bits(v_raw),
+                                         np.array(lens, np.int32), scale, n_sink, window)
+    assert_attn_close(out, ro2, lse, rl2, f"window s={n_sink} w={window} on the GPU-rotated q/k")
 
 
 def test_window_arguments_are_checked(K):
