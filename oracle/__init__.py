@@ -48,6 +48,16 @@ def lib():
         L.oracle_latent_cache_bytes_per_token.argtypes = [i32, i32, i32, i32]
         L.oracle_latent_cache_bytes_per_token.restype = i64
         L.oracle_max_threads.restype = i32
+        L.oracle_e4m3_value.argtypes = [vp, i64, vp]
+        L.oracle_e4m3_round.argtypes = [vp, i64, vp]
+        L.oracle_quant_fp8_groups.argtypes = [vp, i64, i32, vp, vp]
+        L.oracle_dequant_fp8_groups.argtypes = [vp, vp, i64, i32, vp]
+        L.oracle_latent_pack_fp8.argtypes = [vp, i64, vp]
+        L.oracle_latent_unpack_fp8.argtypes = [vp, i64, vp]
+        L.oracle_latent_fp8_row_bytes.restype = i32
+        L.oracle_idx_key_fp8_bytes.argtypes = [i32]
+        L.oracle_idx_key_fp8_bytes.restype = i32
+        L.oracle_dsa_scores_fp8.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, i32]
         _lib = L
     return _lib
 
@@ -402,3 +412,100 @@ def attn_decode_gqa_sparse(q, k, v, tok_idx, tok_count, scale):
                            np.array([n], np.int32), scale)
         out[b], lse[b] = o[0], l[0]
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) latent cache and indexer keys ("稀疏注意力：省了什么，没省什么",
+# 改进一: 656 bytes per token and layer = FP8 latent + scales + bf16 RoPE part,
+# and an indexer key of about 132 bytes).  Reading: one fp32 scale per group of
+# 128 values, s = absmax / 448, code = E4M3 round-to-nearest-even of x / s in
+# fp32, saturating; the 64 RoPE values of a latent row stay bf16.  See oracle.c.
+# ---------------------------------------------------------------------------
+LATENT_FP8_ROW_BYTES = 656
+FP8_GROUP = 128
+
+
+def e4m3_value(codes):
+    """E4M3 codes (uint8) -> their values (fp64; NaN for the NaN codes)."""
+    c = np.ascontiguousarray(codes, np.uint8)
+    out = np.zeros(c.shape, np.float64)
+    _check(lib().oracle_e4m3_value(_p(c), c.size, _p(out)), "oracle_e4m3_value")
+    return out
+
+
+def e4m3_round(y):
+    """fp32 values -> E4M3 codes (round to nearest even, saturating)."""
+    y = np.ascontiguousarray(y, np.float32)
+    out = np.zeros(y.shape, np.uint8)
+    _check(lib().oracle_e4m3_round(_p(y), y.size, _p(out)), "oracle_e4m3_round")
+    return out
+
+
+def quant_fp8(x_bits, group=FP8_GROUP):
+    """bf16 bits [..., n] (n a multiple of group) -> (codes uint8 [..., n],
+    scales float32 [..., n // group])."""
+    x = np.ascontiguousarray(x_bits, np.uint16)
+    n = x.shape[-1]
+    if n % group:
+        raise ValueError("last dimension must be a multiple of the group")
+    codes = np.zeros(x.shape, np.uint8)
+    scales = np.zeros(x.shape[:-1] + (n // group,), np.float32)
+    _check(lib().oracle_quant_fp8_groups(_p(x), x.size // group, group, _p(codes), _p(scales)),
+           "oracle_quant_fp8_groups")
+    return codes, scales
+
+
+def dequant_fp8(codes, scales, group=FP8_GROUP):
+    """(codes [..., n], scales [..., n // group]) -> values fp64 [..., n]."""
+    c = np.ascontiguousarray(codes, np.uint8)
+    sc = np.ascontiguousarray(scales, np.float32)
+    out = np.zeros(c.shape, np.float64)
+    _check(lib().oracle_dequant_fp8_groups(_p(c), _p(sc), c.size // group, group, _p(out)),
+           "oracle_dequant_fp8_groups")
+    return out
+
+
+def latent_pack_fp8(latent_bits):
+    """Latent rows [..., 576] (bf16 bits) -> packed FP8 rows [..., 656] uint8."""
+    x = np.ascontiguousarray(latent_bits, np.uint16)
+    if x.shape[-1] != 576:
+        raise ValueError("latent rows are 576 wide")
+    n = x.size // 576
+    out = np.zeros(x.shape[:-1] + (LATENT_FP8_ROW_BYTES,), np.uint8)
+    _check(lib().oracle_latent_pack_fp8(_p(x), n, _p(out)), "oracle_latent_pack_fp8")
+    return out
+
+
+def latent_unpack_fp8(packed):
+    """Packed FP8 rows [..., 656] -> dequantised latent rows [..., 576] fp64."""
+    p = np.ascontiguousarray(packed, np.uint8)
+    if p.shape[-1] != LATENT_FP8_ROW_BYTES:
+        raise ValueError("packed rows are 656 bytes")
+    n = p.size // LATENT_FP8_ROW_BYTES
+    out = np.zeros(p.shape[:-1] + (576,), np.float64)
+    _check(lib().oracle_latent_unpack_fp8(_p(p), n, _p(out)), "oracle_latent_unpack_fp8")
+    return out
+
+
+def latent_fp8_row_bytes():
+    return int(lib().oracle_latent_fp8_row_bytes())
+
+
+def idx_key_fp8_bytes(d_I=128):
+    return int(lib().oracle_idx_key_fp8_bytes(d_I))
+
+
+def dsa_scores_fp8(q_idx, w, codes, kscale, lens, nthreads=0):
+    """Indexer scores on FP8 keys: q_idx [B,H_I,d_I] uint16, w [B,H_I] float32,
+    codes [B,L_max,d_I] uint8, kscale [B,L_max] float32 -> scores [B, L_max] fp64."""
+    q_idx = np.ascontiguousarray(q_idx, np.uint16)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    kscale = np.ascontiguousarray(kscale, np.float32)
+    w = np.ascontiguousarray(w, np.float32)
+    B, HI, dI = q_idx.shape
+    L_max = codes.shape[1]
+    lens = np.ascontiguousarray(lens, np.int32)
+    sc = np.zeros((B, L_max), np.float64)
+    _check(lib().oracle_dsa_scores_fp8(_p(q_idx), _p(w), _p(codes), _p(kscale), _p(lens), B, HI, dI, L_max,
+                                       _p(sc), nthreads), "oracle_dsa_scores_fp8")
+    return sc

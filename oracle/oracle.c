@@ -554,3 +554,187 @@ int64_t oracle_latent_cache_bytes_per_token(int n_layer, int d_c, int d_rope, in
 {
     return (int64_t)n_layer * (d_c + d_rope) * bytes_per_elem;
 }
+
+/* ------------------------------------------------------------------------ */
+/* FP8 (E4M3) latent cache and indexer keys                                 */
+/* ------------------------------------------------------------------------ */
+/*
+ * [P4] "改进一: DSA" (the paragraph after the selection chain): V3.2 stores,
+ * per token and layer, 656 bytes -- the FP8 latent, its scales and the bf16
+ * RoPE part -- plus an indexer key of about 132 bytes; [P1] §2.2 (1): the
+ * indexer runs stably in fp8.  The pages give the byte budget but no rounding
+ * rule.  Reading taken here (the plainest one the budget supports):
+ *   - latent row (576 = 512 + 64): the 512 latent values in 4 groups of 128,
+ *     each group one fp32 scale and 128 E4M3 codes; the 64 RoPE values kept as
+ *     bf16: 4 * 128 * 1 + 4 * 4 + 64 * 2 = 656 bytes, stored in that order;
+ *   - indexer key (128 values): one group: 128 codes + one fp32 scale = 132 B;
+ *   - scale s = absmax / 448 (448 = the largest finite E4M3 value) in fp32,
+ *     code = E4M3 round-to-nearest-even of x / s (fp32 division), saturating
+ *     to +-448; an all-zero group has s = 0 and codes 0;
+ *   - dequantised value = value(code) * s (exact in fp64).
+ * E4M3 (the OCP 8-bit "E4M3FN" format): sign, 4 exponent bits (bias 7),
+ * 3 mantissa bits; exponent field 0 is subnormal (m/8 * 2^-6); no infinities;
+ * S.1111.111 is NaN, so the largest finite magnitude is 1.75 * 2^8 = 448.
+ */
+
+/* Value of an E4M3 code (NaN for S.1111.111). */
+static double e4m3_value(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+int oracle_e4m3_value(const uint8_t* codes, int64_t n, double* out)
+{
+    if (n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(codes[i]);
+    return 0;
+}
+
+/* Round an fp32 value to E4M3: the nearest of the 127 finite magnitudes
+ * (codes 0x00 .. 0x7E, searched one by one), a tie going to the even code
+ * (mantissa LSB 0); magnitudes above 448 saturate to 448; the sign (including
+ * that of -0) is kept; NaN gives the NaN code. */
+static uint8_t e4m3_round_sat(float y)
+{
+    if (y != y) return 0x7F;
+    double a = fabs((double)y);
+    uint8_t sgn = signbit(y) ? 0x80 : 0x00;
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double d = fabs(e4m3_value((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    if (a > 448.0) best = 0x7E;
+    return (uint8_t)(sgn | best);
+}
+
+int oracle_e4m3_round(const float* y, int64_t n, uint8_t* codes)
+{
+    if (n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) codes[i] = e4m3_round_sat(y[i]);
+    return 0;
+}
+
+/* Quantise n_groups groups of `group` bf16 values (x: bf16 bits, group after
+ * group) to E4M3 codes with one fp32 scale per group, as read above. */
+int oracle_quant_fp8_groups(const uint16_t* x, int64_t n_groups, int group, uint8_t* codes, float* scales)
+{
+    if (n_groups < 0 || group <= 0) return -1;
+    for (int64_t gi = 0; gi < n_groups; ++gi) {
+        const uint16_t* xg = x + gi * group;
+        float amax = 0.0f;
+        for (int i = 0; i < group; ++i) {
+            float a = fabsf((float)bf16_bits_to_f64(xg[i]));
+            if (a > amax) amax = a;
+        }
+        volatile float s = amax / 448.0f; /* fp32 division, as stored */
+        scales[gi] = s;
+        for (int i = 0; i < group; ++i) {
+            if (s == 0.0f) {
+                codes[gi * group + i] = 0;
+                continue;
+            }
+            volatile float yv = (float)bf16_bits_to_f64(xg[i]) / s; /* fp32 division */
+            codes[gi * group + i] = e4m3_round_sat(yv);
+        }
+    }
+    return 0;
+}
+
+/* value(code) * scale for n_groups groups of `group` codes. */
+int oracle_dequant_fp8_groups(const uint8_t* codes, const float* scales, int64_t n_groups, int group, double* out)
+{
+    if (n_groups < 0 || group <= 0) return -1;
+    for (int64_t gi = 0; gi < n_groups; ++gi)
+        for (int i = 0; i < group; ++i)
+            out[gi * group + i] = e4m3_value(codes[gi * group + i]) * (double)scales[gi];
+    return 0;
+}
+
+#define ORC_LAT_DIM 576
+#define ORC_LAT_NOPE 512
+#define ORC_LAT_GROUP 128
+#define ORC_LAT_ROW_BYTES 656
+
+/* Latent rows [n][576] bf16 -> packed FP8 rows [n][656]: 512 codes, 4 fp32
+ * scales (little-endian), 64 bf16 RoPE values. */
+int oracle_latent_pack_fp8(const uint16_t* latent, int64_t n_rows, uint8_t* packed)
+{
+    if (n_rows < 0) return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint16_t* x = latent + r * ORC_LAT_DIM;
+        uint8_t* p = packed + r * ORC_LAT_ROW_BYTES;
+        float sc[ORC_LAT_NOPE / ORC_LAT_GROUP];
+        oracle_quant_fp8_groups(x, ORC_LAT_NOPE / ORC_LAT_GROUP, ORC_LAT_GROUP, p, sc);
+        memcpy(p + ORC_LAT_NOPE, sc, sizeof sc);
+        memcpy(p + ORC_LAT_NOPE + sizeof sc, x + ORC_LAT_NOPE, (ORC_LAT_DIM - ORC_LAT_NOPE) * sizeof(uint16_t));
+    }
+    return 0;
+}
+
+/* Packed FP8 rows [n][656] -> dequantised latent rows [n][576] (fp64). */
+int oracle_latent_unpack_fp8(const uint8_t* packed, int64_t n_rows, double* latent)
+{
+    if (n_rows < 0) return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint8_t* p = packed + r * ORC_LAT_ROW_BYTES;
+        double* y = latent + r * ORC_LAT_DIM;
+        float sc[ORC_LAT_NOPE / ORC_LAT_GROUP];
+        uint16_t rope[ORC_LAT_DIM - ORC_LAT_NOPE];
+        memcpy(sc, p + ORC_LAT_NOPE, sizeof sc);
+        memcpy(rope, p + ORC_LAT_NOPE + sizeof sc, sizeof rope);
+        oracle_dequant_fp8_groups(p, sc, ORC_LAT_NOPE / ORC_LAT_GROUP, ORC_LAT_GROUP, y);
+        for (int i = 0; i < ORC_LAT_DIM - ORC_LAT_NOPE; ++i) y[ORC_LAT_NOPE + i] = bf16_bits_to_f64(rope[i]);
+    }
+    return 0;
+}
+
+/* Bytes of one packed latent row and of one FP8 indexer key (codes + scale). */
+int oracle_latent_fp8_row_bytes(void) { return ORC_LAT_NOPE + (ORC_LAT_NOPE / ORC_LAT_GROUP) * 4 + (ORC_LAT_DIM - ORC_LAT_NOPE) * 2; }
+int oracle_idx_key_fp8_bytes(int d_I) { return d_I + 4; }
+
+/*
+ * Indexer scores on FP8 keys ([P1] §2.2 (1) on the dequantised keys):
+ *   s_{b,t} = sum_j w_{b,j} * ReLU(q^I_{b,j} . khat_{b,t}),  khat = value(code) * scale.
+ * codes [B][L_max][d_I], scales [B][L_max] fp32; otherwise as oracle_dsa_scores.
+ */
+int oracle_dsa_scores_fp8(const uint16_t* qI, const float* w, const uint8_t* codes, const float* kscale,
+                          const int32_t* lens, int B, int HI, int dI, int L_max, double* scores, int nthreads)
+{
+    if (B < 0 || HI <= 0 || dI <= 0 || L_max < 0) return -1;
+    for (int b = 0; b < B; ++b)
+        if (lens[b] < 0 || lens[b] > L_max) return -2;
+    src_t Q = {qI, 0};
+    int nt = set_threads(nthreads);
+    int64_t n_units = (int64_t)B * L_max;
+#pragma omp parallel for num_threads(nt) schedule(static)
+    for (int64_t u = 0; u < n_units; ++u) {
+        int b = (int)(u / L_max);
+        int t = (int)(u % L_max);
+        if (t >= lens[b]) {
+            scores[u] = -INFINITY;
+            continue;
+        }
+        double acc = 0.0;
+        for (int j = 0; j < HI; ++j) {
+            double dot = 0.0;
+            for (int i = 0; i < dI; ++i)
+                dot += ld(Q, ((int64_t)b * HI + j) * dI + i) * (e4m3_value(codes[u * dI + i]) * (double)kscale[u]);
+            double relu = dot > 0.0 ? dot : 0.0;
+            acc += (double)w[(int64_t)b * HI + j] * relu;
+        }
+        scores[u] = acc;
+    }
+    return 0;
+}
