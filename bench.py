@@ -490,11 +490,47 @@ def measure_dsa(K, device, steps, flush, peaks):
     idx_bytes = w.B * w.L * w.dI * 2
     sp_bytes = w.B * w.k * w.Dk * 2
     sp_flops = 2.0 * w.B * w.Hq * w.k * (w.Dk + w.Dv)
+
+    # the same step on the FP8 cache: keys of 128 codes + one scale (132 B per token), latent
+    # rows of 656 B (512 codes, 4 scales, the bf16 RoPE part); quantised once, untimed
+    codes, kscales = K.idx_key_quant_fp8(k_idx)
+    packed = K.latent_quant_fp8(latent)
+    del k_idx, latent
+    torch.cuda.empty_cache()
+
+    def index8():
+        K.dsa_index_topk_fp8(q_idx, wt, codes, kscales, w.k, topk_idx=idx, scores_out=scores, ws=ws1)
+
+    def sparse8():
+        K.attn_decode_sparse_fp8(q, packed, idx, w.Dv, w.sparse_scale, out=out, lse=lse, ws=ws2)
+
+    def step8():
+        index8()
+        sparse8()
+
+    index8_ms = _graph_ms(index8, n, flush)
+    sparse8_ms = _graph_ms(sparse8, n, flush)
+    step8_ms = _graph_ms(step8, n, flush)
+    idx8_bytes = w.B * w.L * (w.dI + 4)
+    sp8_bytes = w.B * w.k * 656
+
+    def bound_ms(nbytes, flops):
+        return max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12)) * 1e3
+
     return {"workload": w.name, "step_ms": round(step_ms, 4), "tok_per_s": round(w.B / (step_ms * 1e-3), 1),
             "index_topk_ms": round(index_ms, 4),
             "indexer_GB_s_incl_topk": round(idx_bytes / (index_ms * 1e-3) / 1e9, 1),
             "sparse_ms": round(sparse_ms, 4), "sparse_TFLOP_s": round(sp_flops / (sparse_ms * 1e-3) / 1e12, 1),
-            "sparse_gathered_bytes": sp_bytes}
+            "sparse_gathered_bytes": sp_bytes,
+            "sparse_roofline_ms": round(bound_ms(sp_bytes, sp_flops), 5),
+            "sparse_frac_of_roofline": round(bound_ms(sp_bytes, sp_flops) / sparse_ms, 3),
+            "fp8": {"step_ms": round(step8_ms, 4), "tok_per_s": round(w.B / (step8_ms * 1e-3), 1),
+                    "index_topk_ms": round(index8_ms, 4), "indexer_key_bytes": idx8_bytes,
+                    "indexer_GB_s_incl_topk": round(idx8_bytes / (index8_ms * 1e-3) / 1e9, 1),
+                    "sparse_ms": round(sparse8_ms, 4), "sparse_gathered_bytes": sp8_bytes,
+                    "sparse_TFLOP_s": round(sp_flops / (sparse8_ms * 1e-3) / 1e12, 1),
+                    "sparse_roofline_ms": round(bound_ms(sp8_bytes, sp_flops), 5),
+                    "sparse_frac_of_roofline": round(bound_ms(sp8_bytes, sp_flops) / sparse8_ms, 3)}}
 
 
 def measure_qsa(K, device, steps, flush, peaks, B=None):

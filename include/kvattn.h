@@ -345,6 +345,34 @@ int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* 
                    int32_t* topk_idx, float* scores_out, void* workspace, size_t workspace_bytes,
                    int32_t* dev_status, void* stream);
 
+/* ---- the lightning indexer sharded over L ------------------------------------------
+ * "稀疏注意力：省了什么，没省什么" (改进一: the indexer still scores every earlier token,
+ * O(L) per query -- the part of DSA that grows with the context) and "Agentic RL 入门3"
+ * §2.2 (2) (S = TopK(s)).  With the keys of a row cut into slices, slice p holding
+ * global positions [p * S, p * S + L_slice), each slice keeps its own top-k
+ * (dsa_index_topk over its keys) and the global top-k is the top-k of the union of
+ * those candidates: an element of the global top-k is beaten by fewer than k keys of
+ * its own slice.  The scores of a token do not depend on the slicing, so the merged
+ * selection is the one dsa_index_topk makes over the whole row, ties included.
+ *
+ * dsa_topk_candidates: one slice's selection as (score, global index) pairs:
+ * scores [B][L_slice] (that call's scores_out), topk_idx [B][k] (its selection, local
+ * indices) -> cand_scores [B][k] = scores[b][topk_idx], cand_idx [B][k] = topk_idx +
+ * idx_offset; -1 entries give (-inf, -1).
+ * dsa_topk_merge: cand_scores, cand_idx [n_parts][B][k] (the slices' candidates in
+ * slice order, as an all-gather concatenates them) -> topk_idx [B][k]: the k best
+ * valid candidates of each row under (score descending, index ascending), listed in
+ * increasing index order, -1 padded -- exactly dsa_index_topk's output format.  The
+ * parts must come in increasing slice order, each part's indices in increasing order
+ * (as dsa_index_topk emits them).  NaN scores are never selected (KVATTN_STATUS_NAN_SCORE).
+ * Limits: 1 <= k <= 2048, n_parts * k <= 49152.
+ */
+int dsa_topk_candidates(const float* scores, const int32_t* topk_idx, int B, int L_slice, int k, int idx_offset,
+                        float* cand_scores, int32_t* cand_idx, void* stream);
+
+int dsa_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_parts, int B, int k,
+                   int32_t* topk_idx, int32_t* dev_status, void* stream);
+
 /* ---- sparse latent-row decode -------------------------------------------------
  * "Agentic RL 入门3" §2.2 (2) o = MLA(q, {k_j, v_j : j in S}); "attention"
  * DSA ② (after weight absorption every query head reads the same single-head
@@ -363,6 +391,60 @@ int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const in
                        int B, int Hq, int Dk, int Dv, int L_max, int k, float scale,
                        kvattn_bf16* out, float* lse, void* workspace, size_t workspace_bytes,
                        int32_t* dev_status, void* stream);
+
+/* ---- FP8 (E4M3) latent cache and indexer keys -----------------------------------
+ * "稀疏注意力：省了什么，没省什么", 改进一: a DeepSeek-V3.2 cache keeps per token and
+ * layer 656 bytes -- FP8 latent + scale + the bf16 RoPE part -- plus an indexer
+ * key of about 132 bytes; "Agentic RL 入门3" §2.2 (1): the indexer runs stably in
+ * fp8.  The pages give the byte budget and no rounding rule; the reading taken:
+ * each group of 128 values gets one fp32 scale s = absmax / 448 (448 = the
+ * largest finite E4M3 value) and codes E4M3(x / s) -- IEEE fp32 division,
+ * round-to-nearest-even, saturating at +-448, the sign of zero kept; an all-zero
+ * group has s = 0 and codes 0.  E4M3 = the OCP 8-bit format with 4 exponent bits
+ * (bias 7), 3 mantissa bits, no infinities.
+ *
+ * Packed latent row (656 bytes, 16-byte aligned rows): bytes 0..511 the codes of
+ * latent[0..511] (groups 0..3 of 128), bytes 512..527 the 4 fp32 scales
+ * (little-endian), bytes 528..655 latent[512..575] as bf16, unchanged.
+ * FP8 indexer key: 128 codes in codes[t][0..127] plus one fp32 scale scales[t]
+ * (132 bytes per token, kept as two arrays so that the codes stay TMA-aligned).
+ *
+ * latent_quant_fp8: latent [n_rows][576] bf16 -> packed [n_rows][656] uint8.
+ * idx_key_quant_fp8: k_idx [n_rows][128] bf16 -> codes [n_rows][128] uint8 and
+ * scales [n_rows] fp32.  Both quantise row by row (a cache built once, or the new
+ * token's row appended at each step: pass pointers to that row, n_rows = 1).
+ * Non-finite inputs are not supported.  Errors: KVATTN_ERR_NULL, _SHAPE
+ * (n_rows < 0), _ALIGN (16 bytes; scales 4).
+ *
+ * attn_decode_sparse_fp8: attn_decode_sparse over packed FP8 latent rows
+ * latent_fp8 [B][L_max][656]: key row j = the dequantised row
+ * (value(code) * scale, rounded to bf16, then the RoPE part), value row j its
+ * first 512 entries.  Arguments, limits, workspace
+ * (attn_decode_sparse_workspace_bytes) and results otherwise as
+ * attn_decode_sparse.
+ */
+int latent_quant_fp8(const kvattn_bf16* latent, long long n_rows, uint8_t* packed, void* stream);
+
+/*
+ * dsa_index_topk on FP8 indexer keys (idx_key_quant_fp8): k_codes [B][L_max][128]
+ * uint8, k_scales [B][L_max] fp32.  The scores are s_{b,t} = k_scales[b][t] *
+ * sum_j w[b][j] * ReLU(q_idx[b][j] . value(k_codes[b][t])) -- the indexer formula
+ * on the dequantised keys, since ReLU commutes with the non-negative scale -- in
+ * fp32; the codes are converted to bf16 exactly for the tensor cores.  HBM bytes per
+ * token: 132 instead of 256.  Everything else (selection, order, -1 padding,
+ * scores_out, workspace, limits) as dsa_index_topk.
+ */
+int dsa_index_topk_fp8(const kvattn_bf16* q_idx, const float* w, const uint8_t* k_codes,
+                       const float* k_scales, const int32_t* seq_lens, int B, int n_idx_head,
+                       int idx_dim, int L_max, int k, int32_t* topk_idx, float* scores_out,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+int idx_key_quant_fp8(const kvattn_bf16* k_idx, long long n_rows, uint8_t* codes, float* scales, void* stream);
+
+int attn_decode_sparse_fp8(const kvattn_bf16* q, const uint8_t* latent_fp8, const int32_t* topk_idx, int B,
+                           int Hq, int Dk, int Dv, int L_max, int k, float scale, kvattn_bf16* out,
+                           float* lse, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                           void* stream);
 
 /* ---- block-level indexer over 4-token groups ----------------------------------
  * "attention" page, "Qwen Sparse Attention (QSA)" §3 ①–④: the visible prefix is

@@ -82,14 +82,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 // Decode steps call with the same cache pointers every step; the cache saves the
 // host-side encodes on each call.  Replacement is round-robin.
 struct MapKey {
-    int dev, rank;
+    int dev, rank, u8;
     const void* base;
     uint64_t dims[4];
     uint32_t box;
     bool operator==(const MapKey& o) const
     {
-        return dev == o.dev && rank == o.rank && base == o.base && box == o.box && dims[0] == o.dims[0] &&
-               dims[1] == o.dims[1] && dims[2] == o.dims[2] && dims[3] == o.dims[3];
+        return dev == o.dev && rank == o.rank && u8 == o.u8 && base == o.base && box == o.box &&
+               dims[0] == o.dims[0] && dims[1] == o.dims[1] && dims[2] == o.dims[2] && dims[3] == o.dims[3];
     }
 };
 constexpr int kMapSlots = 64;
@@ -106,13 +106,16 @@ MapCache& map_cache()
     return c;
 }
 
-// bf16 tensor map of rank 3 ([z][y][x], box {64, box, 1}) or 4 ([w][z][y][x], box
-// {64, 1, box, 1}), 128-byte swizzle, zero fill out of range; from the cache when present.
-int make_map(CUtensorMap* map, int rank, const void* base, const uint64_t (&d)[4], uint32_t box_rows)
+// Tensor map of rank 3 ([z][y][x], box {128 bytes of x, box, 1}) or 4 ([w][z][y][x], box
+// {128 bytes of x, 1, box, 1}) over bf16 (or, with u8, bytes), 128-byte swizzle, zero fill
+// out of range; from the cache when present.
+int make_map(CUtensorMap* map, int rank, const void* base, const uint64_t (&d)[4], uint32_t box_rows,
+             bool u8 = false)
 {
     MapKey key{};
     if (cudaGetDevice(&key.dev) != cudaSuccess) return fail(KVATTN_ERR_CUDA, "no CUDA device");
     key.rank = rank;
+    key.u8 = u8;
     key.base = base;
     for (int i = 0; i < 4; ++i) key.dims[i] = i < rank ? d[i] : 0;
     key.box = box_rows;
@@ -127,12 +130,15 @@ int make_map(CUtensorMap* map, int rank, const void* base, const uint64_t (&d)[4
     }
     auto fn = encode_fn();
     if (!fn) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const uint64_t es = u8 ? 1 : 2;          // element bytes
+    const cuuint32_t bx = u8 ? 128 : 64;     // 128 bytes of x per box row
     cuuint64_t dims[4] = {d[0], d[1], d[2], d[3]};
-    cuuint64_t strides[3] = {d[0] * 2, d[0] * d[1] * 2, d[0] * d[1] * d[2] * 2};
-    cuuint32_t box3[3] = {64, box_rows, 1};
-    cuuint32_t box4[4] = {64, 1, box_rows, 1};
+    cuuint64_t strides[3] = {d[0] * es, d[0] * d[1] * es, d[0] * d[1] * d[2] * es};
+    cuuint32_t box3[3] = {bx, box_rows, 1};
+    cuuint32_t box4[4] = {bx, 1, box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+    CUresult r = fn(map, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                    const_cast<void*>(base), dims, strides,
                     rank == 3 ? box3 : box4, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(KVATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -622,6 +628,78 @@ int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* 
                        "dsa_index_topk launch");
 }
 
+int dsa_index_topk_fp8(const kvattn_bf16* q_idx, const float* w, const uint8_t* k_codes, const float* k_scales,
+                       const int32_t* seq_lens, int B, int n_idx_head, int idx_dim, int L_max, int k, int32_t* topk_idx,
+                       float* scores_out, void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    if (!q_idx || !w || !k_codes || !k_scales || !topk_idx)
+        return fail(KVATTN_ERR_NULL, "dsa_index_topk_fp8: NULL argument");
+    if (n_idx_head != 64 || idx_dim != 128)
+        return fail(KVATTN_ERR_UNSUPPORTED, "dsa_index_topk_fp8: needs 64 indexer heads of width 128 (got %d x %d)",
+                    n_idx_head, idx_dim);
+    if (B < 1 || L_max < 1 || k < 1 || k > 2048)
+        return fail(KVATTN_ERR_SHAPE, "dsa_index_topk_fp8: B %d, L_max %d, k %d (k must be 1..2048)", B, L_max, k);
+    if (L_max > 131072) return fail(KVATTN_ERR_UNSUPPORTED, "dsa_index_topk_fp8: L_max %d above 131072", L_max);
+    if (static_cast<long long>(B) * L_max > (1ll << 31))
+        return fail(KVATTN_ERR_SHAPE, "dsa_index_topk_fp8: B * L_max too large");
+    if (!aligned16(q_idx) || !aligned16(k_codes) || !aligned16(w) || !aligned16(topk_idx) ||
+        (reinterpret_cast<uintptr_t>(k_scales) & 3) || (scores_out && !aligned16(scores_out)))
+        return fail(KVATTN_ERR_ALIGN, "dsa_index_topk_fp8: tensors must be 16-byte aligned (scales 4)");
+    float* scores = scores_out;
+    if (!scores) {
+        const size_t need = align_up(kvattn::dsa_scores_bytes(B, L_max));
+        if (!workspace || workspace_bytes < need)
+            return fail(KVATTN_ERR_WORKSPACE, "dsa_index_topk_fp8: workspace needs %zu bytes when scores_out is NULL",
+                        need);
+        if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
+            return fail(KVATTN_ERR_ALIGN, "dsa_index_topk_fp8: workspace must be 256-byte aligned");
+        scores = static_cast<float*>(workspace);
+    }
+    int sms = 0;
+    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "dsa_index_topk_fp8: no CUDA device");
+    CUtensorMap tm_k, tm_q;
+    const uint64_t dk[4] = {128, static_cast<uint64_t>(L_max), static_cast<uint64_t>(B), 0};
+    if (make_map(&tm_k, 3, k_codes, dk, 128, true) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map_3d(&tm_q, q_idx, 128, 64, B, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    kvattn::DsaIndexArgs a{w, seq_lens, scores, topk_idx, dev_status, B, L_max, k, sms};
+    a.kscale = k_scales;
+    return cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, static_cast<cudaStream_t>(stream)),
+                       "dsa_index_topk_fp8 launch");
+}
+
+int dsa_topk_candidates(const float* scores, const int32_t* topk_idx, int B, int L_slice, int k, int idx_offset,
+                        float* cand_scores, int32_t* cand_idx, void* stream)
+{
+    if (!scores || !topk_idx || !cand_scores || !cand_idx) return fail(KVATTN_ERR_NULL, "dsa_topk_candidates: NULL");
+    if (B < 1 || L_slice < 1 || k < 1 || k > 2048 || idx_offset < 0 ||
+        static_cast<long long>(idx_offset) + L_slice > (1ll << 31) - 1 || static_cast<long long>(B) * L_slice > (1ll << 31))
+        return fail(KVATTN_ERR_SHAPE, "dsa_topk_candidates: B %d, L_slice %d, k %d, offset %d", B, L_slice, k,
+                    idx_offset);
+    if ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(topk_idx) |
+         reinterpret_cast<uintptr_t>(cand_scores) | reinterpret_cast<uintptr_t>(cand_idx)) & 3)
+        return fail(KVATTN_ERR_ALIGN, "dsa_topk_candidates: 4-byte alignment");
+    return cuda_status(kvattn::launch_topk_candidates(scores, topk_idx, B, L_slice, k, idx_offset, cand_scores,
+                                                      cand_idx, static_cast<cudaStream_t>(stream)),
+                       "dsa_topk_candidates launch");
+}
+
+int dsa_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_parts, int B, int k, int32_t* topk_idx,
+                   int32_t* dev_status, void* stream)
+{
+    if (!cand_scores || !cand_idx || !topk_idx) return fail(KVATTN_ERR_NULL, "dsa_topk_merge: NULL");
+    if (n_parts < 1 || B < 1 || k < 1 || k > 2048 || B > 65535)
+        return fail(KVATTN_ERR_SHAPE, "dsa_topk_merge: n_parts %d, B %d, k %d", n_parts, B, k);
+    if (static_cast<long long>(n_parts) * k > kvattn::TOPK_MERGE_MAX)
+        return fail(KVATTN_ERR_UNSUPPORTED, "dsa_topk_merge: n_parts * k = %lld above %d",
+                    static_cast<long long>(n_parts) * k, kvattn::TOPK_MERGE_MAX);
+    if ((reinterpret_cast<uintptr_t>(cand_scores) | reinterpret_cast<uintptr_t>(cand_idx) |
+         reinterpret_cast<uintptr_t>(topk_idx)) & 3)
+        return fail(KVATTN_ERR_ALIGN, "dsa_topk_merge: 4-byte alignment");
+    return cuda_status(kvattn::launch_topk_merge(cand_scores, cand_idx, n_parts, B, k, topk_idx, dev_status,
+                                                 static_cast<cudaStream_t>(stream)),
+                       "dsa_topk_merge launch");
+}
+
 // ---------------------------------------------------------------------------
 int qsa_block_keys(const kvattn_bf16* k_idx, const int32_t* seq_lens, const int32_t* block_from, int max_new, int B,
                    int idx_dim, int L_max, const float* cos_tab, const float* sin_tab, int max_pos, int pair_style,
@@ -709,32 +787,77 @@ size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k)
     return align_up(kvattn::sparse_partial_bytes(B, Hq, k));
 }
 
+// Shared by attn_decode_sparse (bf16 latent rows) and attn_decode_sparse_fp8 (packed rows).
+static int sparse_call(const char* name, const kvattn_bf16* q, const void* latent, bool fp8, const int32_t* topk_idx,
+                       int B, int Hq, int Dk, int Dv, int L_max, int k, float scale, kvattn_bf16* out, float* lse,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    if (!q || !latent || !topk_idx || !out) return fail(KVATTN_ERR_NULL, "%s: NULL argument", name);
+    if (Dk != 576 || Dv != 512)
+        return fail(KVATTN_ERR_UNSUPPORTED, "%s: needs Dk 576, Dv 512 (got %d, %d)", name, Dk, Dv);
+    if (Hq != 64 && Hq != 128) return fail(KVATTN_ERR_UNSUPPORTED, "%s: Hq must be 64 or 128 (got %d)", name, Hq);
+    if (B < 1 || L_max < 1 || k < 1 || k > 2048)
+        return fail(KVATTN_ERR_SHAPE, "%s: B %d, L_max %d, k %d (k must be 1..2048)", name, B, L_max, k);
+    if (B > 65535) return fail(KVATTN_ERR_SHAPE, "%s: B %d above 65535", name, B);
+    if (!(scale > 0.0f) || !std::isfinite(scale)) return fail(KVATTN_ERR_SHAPE, "%s: scale must be finite > 0", name);
+    if (!aligned16(q) || !aligned16(latent) || !aligned16(out) || !aligned16(topk_idx) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)))
+        return fail(KVATTN_ERR_ALIGN, "%s: tensors must be 16-byte aligned", name);
+    const size_t need = align_up(kvattn::sparse_partial_bytes(B, Hq, k));
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return fail(KVATTN_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, need);
+    if (need > 0 && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
+        return fail(KVATTN_ERR_ALIGN, "%s: workspace must be 256-byte aligned", name);
+    const int chunks = kvattn::sparse_chunks(k);
+    CUtensorMap tm_q, tm_o;
+    if (make_map_3d(&tm_q, q, Dk, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (chunks == 1) {
+        if (make_map_3d(&tm_o, out, Dv, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    } else {
+        if (make_map_3d(&tm_o, workspace, Dv, Hq, static_cast<uint64_t>(B) * chunks, Hq) != KVATTN_OK)
+            return KVATTN_ERR_CUDA;
+    }
+    kvattn::SparseLaunch l{q, latent, topk_idx, out, lse, need > 0 ? workspace : nullptr, dev_status, B, Hq, L_max,
+                           k, scale, fp8};
+    return cuda_status(kvattn::launch_sparse_attn(l, tm_q, tm_o, static_cast<cudaStream_t>(stream)), name);
+}
+
 int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const int32_t* topk_idx, int B, int Hq, int Dk,
                        int Dv, int L_max, int k, float scale, kvattn_bf16* out, float* lse, void* workspace,
                        size_t workspace_bytes, int32_t* dev_status, void* stream)
 {
-    if (!q || !latent || !topk_idx || !out) return fail(KVATTN_ERR_NULL, "attn_decode_sparse: NULL argument");
-    if (Dk != 576 || Dv != 512)
-        return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_sparse: needs Dk 576, Dv 512 (got %d, %d)", Dk, Dv);
-    if (Hq != 64 && Hq != 128)
-        return fail(KVATTN_ERR_UNSUPPORTED, "attn_decode_sparse: Hq must be 64 or 128 (got %d)", Hq);
-    if (B < 1 || L_max < 1 || k < 1 || k > 2048)
-        return fail(KVATTN_ERR_SHAPE, "attn_decode_sparse: B %d, L_max %d, k %d (k must be 1..2048)", B, L_max, k);
-    if (!(scale > 0.0f) || !std::isfinite(scale))
-        return fail(KVATTN_ERR_SHAPE, "attn_decode_sparse: scale must be finite > 0");
-    if (!aligned16(q) || !aligned16(latent) || !aligned16(out) || !aligned16(topk_idx))
-        return fail(KVATTN_ERR_ALIGN, "attn_decode_sparse: tensors must be 16-byte aligned");
-    const size_t need = align_up(kvattn::sparse_partial_bytes(B, Hq, k));
-    if (need > 0 && (!workspace || workspace_bytes < need))
-        return fail(KVATTN_ERR_WORKSPACE, "attn_decode_sparse: workspace needs %zu bytes", need);
-    if (need > 0 && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
-        return fail(KVATTN_ERR_ALIGN, "attn_decode_sparse: workspace must be 256-byte aligned");
-    CUtensorMap tm_q;
-    if (make_map_3d(&tm_q, q, Dk, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
-    kvattn::SparseLaunch l{q, latent, topk_idx, out, lse, need > 0 ? static_cast<float*>(workspace) : nullptr,
-                           dev_status, B, Hq, L_max, k, scale};
-    return cuda_status(kvattn::launch_sparse_attn(l, tm_q, static_cast<cudaStream_t>(stream)),
-                       "attn_decode_sparse launch");
+    return sparse_call("attn_decode_sparse", q, latent, false, topk_idx, B, Hq, Dk, Dv, L_max, k, scale, out, lse,
+                       workspace, workspace_bytes, dev_status, stream);
+}
+
+int attn_decode_sparse_fp8(const kvattn_bf16* q, const uint8_t* latent_fp8, const int32_t* topk_idx, int B, int Hq,
+                           int Dk, int Dv, int L_max, int k, float scale, kvattn_bf16* out, float* lse, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream)
+{
+    return sparse_call("attn_decode_sparse_fp8", q, latent_fp8, true, topk_idx, B, Hq, Dk, Dv, L_max, k, scale, out,
+                       lse, workspace, workspace_bytes, dev_status, stream);
+}
+
+// ---------------------------------------------------------------------------
+int latent_quant_fp8(const kvattn_bf16* latent, long long n_rows, uint8_t* packed, void* stream)
+{
+    if ((!latent || !packed) && n_rows > 0) return fail(KVATTN_ERR_NULL, "latent_quant_fp8: NULL argument");
+    if (n_rows < 0 || n_rows > (1ll << 34)) return fail(KVATTN_ERR_SHAPE, "latent_quant_fp8: n_rows %lld", n_rows);
+    if (!aligned16(latent) || !aligned16(packed))
+        return fail(KVATTN_ERR_ALIGN, "latent_quant_fp8: tensors must be 16-byte aligned");
+    return cuda_status(kvattn::launch_latent_quant_fp8(latent, n_rows, packed, static_cast<cudaStream_t>(stream)),
+                       "latent_quant_fp8 launch");
+}
+
+int idx_key_quant_fp8(const kvattn_bf16* k_idx, long long n_rows, uint8_t* codes, float* scales, void* stream)
+{
+    if ((!k_idx || !codes || !scales) && n_rows > 0) return fail(KVATTN_ERR_NULL, "idx_key_quant_fp8: NULL argument");
+    if (n_rows < 0 || n_rows > (1ll << 34)) return fail(KVATTN_ERR_SHAPE, "idx_key_quant_fp8: n_rows %lld", n_rows);
+    if (!aligned16(k_idx) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3))
+        return fail(KVATTN_ERR_ALIGN, "idx_key_quant_fp8: k_idx and codes 16-byte aligned, scales 4-byte aligned");
+    return cuda_status(
+        kvattn::launch_idx_key_quant_fp8(k_idx, n_rows, codes, scales, static_cast<cudaStream_t>(stream)),
+        "idx_key_quant_fp8 launch");
 }
 
 }  // extern "C"

@@ -17,6 +17,7 @@
 // shared memory and finds the digit itself.  An ordered compaction then writes
 // the selected indices straight out in increasing index order.
 #include <cooperative_groups.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -52,6 +53,7 @@ constexpr int IX_SMEM = IX_OFF_MISC + 32 + 1024;
 struct IndexerArgs {
     const float* w;
     const int32_t* seq_lens;
+    const float* kscale;  // FP8 keys: [B][L_max] fp32 scales (indexer_fp8_kernel only)
     float* scores;
     int32_t* dev_status;
     int B, L_max, tiles_per_b, chunks_per_b;
@@ -222,6 +224,257 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc = fmaf(s_w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), acc);
                 const int tok = t * IX_TOK + row;
+                if (acc != acc) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
+                if (tok < a.L_max) out[tok] = tok < len ? acc : -INFINITY;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, IX_TMEM_COLS);
+    }
+}
+
+// ---- indexer on FP8 keys -------------------------------------------------------------
+// "稀疏注意力：省了什么，没省什么", 改进一 (an indexer key of about 132 bytes: 128 E4M3
+// codes and one fp32 scale) and "Agentic RL 入门3" §2.2 (1) (the indexer runs stably in
+// fp8).  With k_t = scale_t * code_t and scale_t >= 0, ReLU(q . k_t) = scale_t *
+// ReLU(q . code_t), so s_t = scale_t * sum_j w_j ReLU(q_j . code_t): the codes enter
+// the MMA unscaled (E4M3 -> bf16 is exact) and the scale multiplies the score.
+// 320 threads: w0 TMA of 16 KB code tiles (128-byte swizzle) into a 6-slot ring,
+// w1 MMA issuer + TMEM owner, w2-5 epilogue, w6-9 convert each code tile into a
+// bf16 tile (two 64-column SW128 blocks) of a 3-slot ring.  HBM bytes per token:
+// 128 + 4 (against 256 for bf16 keys).
+constexpr int IX8_RAW = IX_TOK * 128;            // 16 KB code tile [128 tokens][128 codes]
+constexpr int IX8_RSTAGES = 6, IX8_BSTAGES = 3;
+constexpr int IX8_THREADS = 320;
+constexpr int IX8_OFF_RAW = 0;
+constexpr int IX8_OFF_BF = IX8_OFF_RAW + IX8_RSTAGES * IX8_RAW;
+constexpr int IX8_OFF_Q = IX8_OFF_BF + IX8_BSTAGES * IX_TILE;
+constexpr int IX8_OFF_W = IX8_OFF_Q + IX_QBYTES;
+constexpr int IX8_OFF_BAR = IX8_OFF_W + IX_HEADS * 4;
+// raw_full[R], raw_empty[R], bf_full[S], bf_empty[S], q_full, q_empty, acc_full[2], acc_empty[2], mma_done
+constexpr int IX8_NBAR = 2 * IX8_RSTAGES + 2 * IX8_BSTAGES + 7;
+constexpr int IX8_OFF_MISC = IX8_OFF_BAR + IX8_NBAR * 8;
+constexpr int IX8_SMEM = IX8_OFF_MISC + 32 + 1024;
+static_assert(IX8_SMEM <= 232448, "shared memory");
+
+// Sixteen E4M3 codes -> sixteen bf16 (two 16-byte chunks), exactly.
+__device__ __forceinline__ void codes16_to_bf16(uint4 c, uint4& lo, uint4& hi)
+{
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            uint32_t h2;
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(w[i] >> (16 * hf))));
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+            o[2 * i + hf] = pack_bf16x2(f.x, f.y);
+        }
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+__global__ void __launch_bounds__(IX8_THREADS, 1)
+    indexer_fp8_kernel(const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_q,
+                       IndexerArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + IX8_OFF_BAR);
+    uint64_t* raw_full = bars;
+    uint64_t* raw_empty = raw_full + IX8_RSTAGES;
+    uint64_t* bf_full = raw_empty + IX8_RSTAGES;
+    uint64_t* bf_empty = bf_full + IX8_BSTAGES;
+    uint64_t* q_full = bf_empty + IX8_BSTAGES;
+    uint64_t* q_empty = q_full + 1;
+    uint64_t* acc_full = q_full + 2;
+    uint64_t* acc_empty = q_full + 4;
+    uint64_t* mma_done = q_full + 6;
+    float* s_w = reinterpret_cast<float*>(smem + IX8_OFF_W);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + IX8_OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + IX8_OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_items = a.B * a.chunks_per_b;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < IX8_RSTAGES; ++s) {
+            mbar_init(&raw_full[s], 1);
+            mbar_init(&raw_empty[s], 4);
+        }
+        for (int s = 0; s < IX8_BSTAGES; ++s) {
+            mbar_init(&bf_full[s], 4);
+            mbar_init(&bf_empty[s], 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 4);
+        }
+        mbar_init(mma_done, 1);
+        *s_abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_k8);
+        tma_prefetch_desc(&tm_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(s_tmem, IX_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    pdl_wait();
+    pdl_trigger();
+
+    if (warp == 0) {
+        // ===== TMA producer: query, then code tiles =====
+        if (lane == 0) {
+            int it = 0, n = 0;
+            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
+                int b, t0, t1;
+                ix_item(a, item, b, t0, t1);
+                if (n > 0 && !mbar_wait(q_empty, (n - 1) & 1)) {
+                    *s_abort = 1;
+                    break;
+                }
+                mbar_arrive_expect_tx(q_full, IX_QBYTES);
+                tma_load_3d(smem + IX8_OFF_Q, &tm_q, q_full, 0, 0, b);
+                tma_load_3d(smem + IX8_OFF_Q + IX_QBOX, &tm_q, q_full, 64, 0, b);
+                for (int t = t0; t < t1; ++t, ++it) {
+                    const int s = it % IX8_RSTAGES;
+                    if (it >= IX8_RSTAGES && (*s_abort || !mbar_wait(&raw_empty[s], ((it / IX8_RSTAGES) - 1) & 1))) {
+                        *s_abort = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&raw_full[s], IX8_RAW);
+                    tma_load_3d(smem + IX8_OFF_RAW + s * IX8_RAW, &tm_k8, &raw_full[s], 0, t * IX_TOK, b);
+                }
+            }
+            if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            for (int j = it - IX8_RSTAGES > 0 ? it - IX8_RSTAGES : 0; j < it; ++j)
+                mbar_wait(&raw_full[j % IX8_RSTAGES], (j / IX8_RSTAGES) & 1);
+        }
+    } else if (warp == 1) {
+        // ===== MMA issuer (one thread) =====
+        if (lane == 0) {
+            const uint32_t q_addr = smem_u32(smem + IX8_OFF_Q);
+            int it = 0, n = 0;
+            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
+                int b, t0, t1;
+                ix_item(a, item, b, t0, t1);
+                if (!mbar_wait(q_full, n & 1)) {
+                    *s_abort = 1;
+                    break;
+                }
+                for (int t = t0; t < t1; ++t, ++it) {
+                    const int s = it % IX8_BSTAGES;
+                    const int buf = it & 1;
+                    if (*s_abort || !mbar_wait(&bf_full[s], (it / IX8_BSTAGES) & 1) ||
+                        (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1))) {
+                        *s_abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(smem + IX8_OFF_BF + s * IX_TILE);
+                    const uint32_t d_addr = tmem + buf * IX_HEADS;
+#pragma unroll
+                    for (int ks = 0; ks < IX_DIM / 16; ++ks) {
+                        const uint32_t off = (ks & 3) * 32;
+                        const uint64_t ad = umma_desc_k_sw128(k_addr + (ks >> 2) * IX_BOX + off);
+                        const uint64_t bd = umma_desc_k_sw128(q_addr + (ks >> 2) * IX_QBOX + off);
+                        tc_mma_bf16(d_addr, ad, bd, IX_IDESC, ks > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&bf_empty[s]);
+                    tc_commit(&acc_full[buf]);
+                }
+                tc_commit(q_empty);
+            }
+            tc_commit(mma_done);
+            mbar_wait(mma_done, 0);
+            if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+        }
+    } else if (warp >= 6) {
+        // ===== converters: code tile -> bf16 tile; thread r takes token row r =====
+        const int r = threadIdx.x - 192;
+        int it = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+            int b, t0, t1;
+            ix_item(a, item, b, t0, t1);
+            for (int t = t0; t < t1; ++t, ++it) {
+                const int rs = it % IX8_RSTAGES, bs = it % IX8_BSTAGES;
+                if (!warp_wait(&raw_full[rs], (it / IX8_RSTAGES) & 1, s_abort)) continue;
+                const uint8_t* src = smem + IX8_OFF_RAW + rs * IX8_RAW + r * 128;
+                uint4 c[8];
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    c[ch] = *reinterpret_cast<const uint4*>(src + ((ch ^ (r & 7)) << 4));  // TMA 128-byte swizzle
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&raw_empty[rs]);
+                if (it >= IX8_BSTAGES && !warp_wait(&bf_empty[bs], ((it / IX8_BSTAGES) - 1) & 1, s_abort)) continue;
+                uint8_t* dst = smem + IX8_OFF_BF + bs * IX_TILE;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {  // codes 16 ch .. 16 ch + 15 = bf16 chunks 2 ch, 2 ch + 1
+                    uint4 lo, hi;
+                    codes16_to_bf16(c[ch], lo, hi);
+                    uint8_t* blk = dst + (ch >> 2) * IX_BOX;
+                    *reinterpret_cast<uint4*>(blk + swz128(r, (2 * ch) & 7)) = lo;
+                    *reinterpret_cast<uint4*>(blk + swz128(r, (2 * ch + 1) & 7)) = hi;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bf_full[bs]);
+            }
+        }
+    } else {
+        // ===== epilogue: TMEM -> ReLU, weight, sum over heads, times the key's scale =====
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int ep = threadIdx.x - 64;
+        int tc = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+            int b, t0, t1;
+            ix_item(a, item, b, t0, t1);
+            const int len_raw = a.seq_lens ? (a.seq_lens[b] >> a.len_shift) : a.L_max;
+            const int len = min(max(len_raw, 0), a.L_max);
+            if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
+            named_bar_sync(2, 128);
+            if (ep < IX_HEADS) s_w[ep] = a.w[static_cast<long long>(b) * IX_HEADS + ep];
+            named_bar_sync(2, 128);
+            float* out = a.scores + static_cast<long long>(b) * a.L_max;
+            const float* ks = a.kscale + static_cast<long long>(b) * a.L_max;
+            for (int t = t0; t < t1; ++t, ++tc) {
+                const int buf = tc & 1;
+                const int tok = t * IX_TOK + row;
+                const float kscale = tok < a.L_max ? __ldg(ks + tok) : 0.f;
+                if (!warp_wait(&acc_full[buf], (tc >> 1) & 1, s_abort)) continue;
+                tc_fence_after();
+                const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_HEADS;
+                uint32_t v0[32], v1[32];
+                tmem_ld32(taddr, v0);
+                tmem_ld32(taddr + 32, v1);
+                tmem_wait_ld();
+                tmem_regs_ready(v0);
+                tmem_regs_ready(v1);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[buf]);
+                float acc = 0.f;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[j], fmaxf(__uint_as_float(v0[j]), 0.f), acc);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), acc);
+                acc *= kscale;
                 if (acc != acc) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
                 if (tok < a.L_max) out[tok] = tok < len ? acc : -INFINITY;
             }
@@ -456,6 +709,134 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     cluster.sync();  // no CTA leaves while others may still read its shared memory
 }
 
+// ---- top-k over the candidates of several key slices -----------------------------------
+// Sharding the indexer over L ("稀疏注意力：省了什么，没省什么": the indexer stays O(L) per
+// query, the cost that grows with the context): part p scores keys [p S, (p + 1) S) and
+// keeps its own top-k.  Every element of the global top-k is in its part's top-k (fewer
+// than k keys of its part beat it), so the top-k of the union of the parts' candidates is
+// the global top-k, and with the same order (score desc, index asc) it is the same set.
+
+// (score, global index) pairs of one part's selection: cand_idx = local index + offset.
+__global__ void topk_candidates_kernel(const float* scores, const int32_t* idx, int B, int L_slice, int k, int offset,
+                                       float* cand_score, int32_t* cand_idx)
+{
+    const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= static_cast<long long>(B) * k) return;
+    const int b = static_cast<int>(i / k);
+    const int j = idx[i];
+    const bool ok = j >= 0 && j < L_slice;
+    cand_score[i] = ok ? scores[static_cast<long long>(b) * L_slice + j] : -INFINITY;
+    cand_idx[i] = ok ? j + offset : -1;
+}
+
+struct MergeTopkArgs {
+    const float* cand_score;  // [n_parts][B][k]
+    const int32_t* cand_idx;  // [n_parts][B][k]; -1 = no candidate
+    int32_t* out;             // [B][k]
+    int32_t* dev_status;
+    int n_parts, B, k;
+};
+
+// One CTA per batch row: the row's n_parts * k candidates, in part order (part p's
+// indices all below part p + 1's, each part's in increasing order), as keys in shared
+// memory; an exact 3-digit radix select of the k-th largest key among the valid ones,
+// then an ordered compaction that takes the keys above it and the lowest-index keys
+// equal to it, written in increasing index order.
+__global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(MergeTopkArgs a)
+{
+    extern __shared__ uint32_t s_ck[];  // [n] keys (0: no candidate, or a NaN score)
+    __shared__ uint32_t hist[2048];
+    __shared__ int s_warp[32];
+    __shared__ uint32_t s_sel[2];
+    __shared__ int s_n;
+    const int row = blockIdx.x, tid = threadIdx.x;
+    const int n = a.n_parts * a.k;
+    pdl_wait();
+    pdl_trigger();
+    int n_valid_mine = 0;
+    bool nan = false;
+    for (int i = tid; i < n; i += TK_THREADS) {
+        const int p = i / a.k, j = i - p * a.k;
+        const long long off = (static_cast<long long>(p) * a.B + row) * a.k + j;
+        const int ci = a.cand_idx[off];
+        uint32_t key = 0u;
+        if (ci >= 0) {
+            key = score_key(a.cand_score[off], nan);  // 0 only for NaN: never selected
+            n_valid_mine += key != 0u;
+        }
+        s_ck[i] = key;
+    }
+    if (tid == 0) s_n = 0;
+    __syncthreads();
+    atomicAdd(&s_n, n_valid_mine);
+    __syncthreads();
+    const int n_valid = s_n;
+    const int kk = min(a.k, n_valid);
+    uint32_t prefix = 0u, known = 0u;
+    int k_rem = kk;
+    if (n_valid > a.k) {
+        const int shifts[3] = {21, 10, 0};
+        const int widths[3] = {11, 11, 10};
+        for (int pass = 0; pass < 3; ++pass) {
+            const int sh = shifts[pass], nb = 1 << widths[pass];
+            for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
+            __syncthreads();
+            for (int i = tid; i < n; i += TK_THREADS) {
+                const uint32_t key = s_ck[i];
+                if (key != 0u && (key & known) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1u);
+            }
+            __syncthreads();
+            // thread t owns digits nb-1-2t and nb-2-2t (largest first)
+            const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
+            const int c0 = d0 >= 0 ? static_cast<int>(hist[d0]) : 0, c1 = d1 >= 0 ? static_cast<int>(hist[d1]) : 0;
+            const int incl = block_incl_scan(c0 + c1, s_warp);
+            const int before = incl - c0 - c1;
+            if (d0 >= 0 && before < k_rem && before + c0 >= k_rem) {
+                s_sel[0] = static_cast<uint32_t>(d0);
+                s_sel[1] = static_cast<uint32_t>(k_rem - before);
+            } else if (d1 >= 0 && before + c0 < k_rem && before + c0 + c1 >= k_rem) {
+                s_sel[0] = static_cast<uint32_t>(d1);
+                s_sel[1] = static_cast<uint32_t>(k_rem - before - c0);
+            }
+            __syncthreads();
+            prefix |= s_sel[0] << sh;
+            k_rem = static_cast<int>(s_sel[1]);
+            known |= static_cast<uint32_t>(nb - 1) << sh;
+            __syncthreads();
+        }
+    }
+    // with n_valid <= k every valid candidate is taken
+    const uint32_t T = prefix;
+    const int take_eq = n_valid > a.k ? k_rem : 0;
+    const int run = (n + TK_THREADS - 1) / TK_THREADS;
+    const int r0 = min(tid * run, n), r1 = min(r0 + run, n);
+    int n_gt = 0, n_eq = 0;
+    for (int i = r0; i < r1; ++i) {
+        const uint32_t key = s_ck[i];
+        n_gt += n_valid > a.k ? key > T : key != 0u;
+        n_eq += n_valid > a.k && key == T;
+    }
+    const int inc_gt = block_incl_scan(n_gt, s_warp);
+    const int inc_eq = block_incl_scan(n_eq, s_warp);
+    int e_rank = inc_eq - n_eq;
+    int pos = (inc_gt - n_gt) + min(e_rank, take_eq);
+    int32_t* out = a.out + static_cast<long long>(row) * a.k;
+    for (int i = r0; i < r1; ++i) {
+        const uint32_t key = s_ck[i];
+        bool take = n_valid > a.k ? key > T : key != 0u;
+        if (n_valid > a.k && key == T) {
+            take = e_rank < take_eq;
+            ++e_rank;
+        }
+        if (take) {
+            const int p = i / a.k, j = i - p * a.k;
+            out[pos++] = a.cand_idx[(static_cast<long long>(p) * a.B + row) * a.k + j];
+        }
+    }
+    for (int j = kk + tid; j < a.k; j += TK_THREADS) out[j] = -1;
+    if (nan) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
+}
+
 }  // namespace
 
 size_t dsa_scores_bytes(int B, int L_max) { return static_cast<size_t>(B) * L_max * sizeof(float); }
@@ -470,9 +851,12 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     if (dev < 64 && !attr_set[dev]) {
         e = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX_SMEM);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(indexer_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX8_SMEM);
+        if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
     IndexerArgs ia{};
+    ia.kscale = a.kscale;
     ia.w = a.w;
     ia.seq_lens = a.seq_lens;
     ia.scores = a.scores;
@@ -488,7 +872,8 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     ia.chunks_per_b = chunks;
     const int items = a.B * chunks;
     const int grid = items < a.num_sms ? items : a.num_sms;
-    e = launch_pdl(indexer_kernel, dim3(grid), dim3(IX_THREADS), IX_SMEM, stream, tm_k, tm_q, ia);
+    e = a.kscale ? launch_pdl(indexer_fp8_kernel, dim3(grid), dim3(IX8_THREADS), IX8_SMEM, stream, tm_k, tm_q, ia)
+                 : launch_pdl(indexer_kernel, dim3(grid), dim3(IX_THREADS), IX_SMEM, stream, tm_k, tm_q, ia);
     if (e != cudaSuccess) return e;
 
     TopkArgs ta{a.scores, a.seq_lens, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k, a.len_shift,
@@ -517,6 +902,36 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, topk_kernel, ta);
+}
+
+}  // namespace kvattn
+
+namespace kvattn {
+
+cudaError_t launch_topk_candidates(const float* scores, const int32_t* idx, int B, int L_slice, int k, int offset,
+                                   float* cand_score, int32_t* cand_idx, cudaStream_t stream)
+{
+    const long long n = static_cast<long long>(B) * k;
+    topk_candidates_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(scores, idx, B, L_slice, k,
+                                                                                         offset, cand_score, cand_idx);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk_merge(const float* cand_score, const int32_t* cand_idx, int n_parts, int B, int k,
+                              int32_t* topk_idx, int32_t* dev_status, cudaStream_t stream)
+{
+    const size_t smem = static_cast<size_t>(n_parts) * k * sizeof(uint32_t);
+    static bool attr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && !attr[dev]) {
+        e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+        attr[dev] = true;
+    }
+    MergeTopkArgs a{cand_score, cand_idx, topk_idx, dev_status, n_parts, B, k};
+    return launch_pdl(topk_merge_kernel, dim3(B), dim3(TK_THREADS), smem, stream, a);
 }
 
 }  // namespace kvattn

@@ -144,10 +144,20 @@ struct DsaIndexArgs {
     int32_t* tok_idx = nullptr;
     int32_t* tok_count = nullptr;
     int L_tok = 0;  // token capacity of a row (seq_lens beyond it are clamped and flagged)
+    // FP8 keys (kscale non-null): tm_k maps the codes [B][L_max][128] uint8 with a {128, 128, 1}
+    // box and 128-byte swizzle; kscale [B][L_max] fp32 holds each key's scale.
+    const float* kscale = nullptr;
 };
 size_t dsa_scores_bytes(int B, int L_max);
 cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                                   cudaStream_t stream);
+
+// ---- top-k over the candidates of several key slices (sharded indexer) ----
+constexpr int TOPK_MERGE_MAX = 48 * 1024;  // candidates per row (n_parts * k) held in shared memory
+cudaError_t launch_topk_candidates(const float* scores, const int32_t* idx, int B, int L_slice, int k, int offset,
+                                   float* cand_score, int32_t* cand_idx, cudaStream_t stream);
+cudaError_t launch_topk_merge(const float* cand_score, const int32_t* cand_idx, int n_parts, int B, int k,
+                              int32_t* topk_idx, int32_t* dev_status, cudaStream_t stream);
 
 // ---- block-level indexer (4-token groups) ----
 constexpr int QSA_BLOCK = 4;
@@ -167,19 +177,29 @@ cudaError_t launch_qsa_block_keys(const QsaKeysArgs& a, cudaStream_t stream);
 // ---- sparse latent attention ----
 struct SparseLaunch {
     const kvattn_bf16* q;
-    const kvattn_bf16* latent;
+    const void* latent;  // bf16 [B][L_max][576], or packed FP8 rows [B][L_max][656] when fp8
     const int32_t* idx;
     kvattn_bf16* out;
     float* lse;
-    float* workspace;  // chunk partials (null when one chunk)
+    void* workspace;     // chunk parts: bf16 [B][chunks][Hq][512], then fp32 lse [B][chunks][Hq] (null when one chunk)
     int32_t* dev_status;
     int B, Hq, L_max, k;
     float scale;
+    bool fp8 = false;
 };
 int sparse_chunks(int k);
+size_t sparse_part_o_bytes(int B, int Hq, int k);
 size_t sparse_partial_bytes(int B, int Hq, int k);
 // tm_q: 3-D map over q [B][Hq][576] with a {64, Hq, 1} box (128-byte swizzle).
-cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, cudaStream_t stream);
+// tm_o: 3-D map with a {64, Hq, 1} box over the output [B][Hq][512] when k <= 128
+// (one chunk), else over the workspace's bf16 parts [B * chunks][Hq][512].
+cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_o,
+                               cudaStream_t stream);
+
+// ---- FP8 (E4M3) quantisation of latent rows and indexer keys ----
+cudaError_t launch_latent_quant_fp8(const kvattn_bf16* src, long long n_rows, uint8_t* dst, cudaStream_t stream);
+cudaError_t launch_idx_key_quant_fp8(const kvattn_bf16* src, long long n_rows, uint8_t* codes, float* scales,
+                                     cudaStream_t stream);
 
 // ---- causal prefill ----
 constexpr int PREFILL_Q_ROWS = 128;  // rows of a Q tile (box height of tm_q)

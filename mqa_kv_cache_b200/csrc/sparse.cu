@@ -7,25 +7,35 @@
 // row as key and its first 512 columns as value (§2.3.3, §2.3.5).
 //
 // Kernel (tcgen05): one CTA per (batch row, chunk of 128 selected rows), all
-// query heads as the M = 128 rows of both MMAs.
-//   - warps 0-3 gather the chunk's 128 latent rows (cp.async, 16 bytes at a
-//     time, eight lanes per 128-byte line so that every warp request covers
-//     four whole lines) into nine 64-column blocks laid out as the tensor cores
-//     read them (128-byte rows, 128-byte swizzle); each block is signalled as it
-//     lands.  Invalid indices are zero-filled and their columns masked.
-//   - warp 4 streams the queries through a four-slot TMA ring, 64 columns at a
-//     time; warp 5 issues S = Q C^T (M = 128 heads, N = 128 rows, K = 576) into
-//     TMEM, block by block as the gather lands.
-//   - warps 0-3 (thread = head = TMEM lane) take the row softmax of S in base 2
-//     and write P as bf16 into shared memory (over two query slots, free once S
-//     is complete); warp 5 then issues O = P V with
-//     V = the same resident rows read as an MN-major operand, N = 256 twice,
-//     into all 512 TMEM columns (S's columns are free by then).
-//   - warps 0-3 write O (normalised when the row has one chunk, else the
-//     unnormalised partial with its running max and sum, stored column-major
-//     [column][head] so that a warp's 32 heads fill one 128-byte line); the
-//     first half is written while the second half's MMAs run.
-// Chunks of one row are merged by a second kernel (the split-softmax identity).
+// query heads as the M = 128 rows of both MMAs.  320 threads:
+//   - warps 0-7 gather the chunk's 128 latent rows with 16-byte cp.async into
+//     nine 64-column blocks laid out as the tensor cores read them (128-byte
+//     rows, 128-byte swizzle); each block is signalled as it lands.  Invalid
+//     indices are zero-filled and their columns masked.  In the FP8 variant
+//     (rows of 656 bytes: 512 E4M3 codes, 4 fp32 scales, 64 bf16 RoPE values;
+//     "稀疏注意力：省了什么，没省什么", 改进一) the RoPE part lands directly in block
+//     8, the codes land in the space of blocks 4-7 and are dequantised there,
+//     block by block, into bf16 (value(code) * scale, rounded to bf16): blocks
+//     0-3 while the rest is still in flight, blocks 4-7 from registers once every
+//     code has been read.
+//   - warp 8 streams the queries through a four-slot TMA ring, 64 columns at a
+//     time, in the order the blocks land; warp 9 issues S = Q C^T (M = 128
+//     heads, N = 128 rows, K = 576) into TMEM block by block.
+//   - warps 0-7 take the row softmax of S in base 2: warp w reads head row
+//     32 (w % 4) + lane (its TMEM lane), the first four warps key columns 0-63,
+//     the other four 64-127; the two halves exchange their maxima and sums
+//     through shared memory.  P is written as bf16 over two free query slots.
+//   - warp 9 issues O = P V with V = the resident rows read as an MN-major
+//     operand, N = 256 twice, into all 512 TMEM columns (S's columns are free by
+//     then).
+//   - warps 0-3 write O columns 0-255, warps 4-7 columns 256-511: normalised by
+//     the chunk's own softmax sum, rounded to bf16 into shared memory (over the
+//     blocks whose values that half has consumed), then stored by TMA.  A row
+//     with one chunk is written to the output directly; otherwise each chunk
+//     leaves its normalised bf16 part and its log-sum-exp, and a second kernel
+//     merges the parts (out = sum_c 2^(lse_c - LSE) o_c).
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -40,38 +50,56 @@ constexpr int SP_M = 128;                      // query heads per MMA (rows past
 constexpr int SP_KB = SP_DK / 64;              // 64-column blocks of a latent row (9)
 constexpr int SP_BLOCK = SP_ROWS * 128;        // 16 KB: 128 rows x 64 columns
 constexpr int SP_QBLOCK = SP_M * 128;          // 16 KB: 128 heads x 64 columns
-constexpr int SP_THREADS = 192;                // w0-3 gather/softmax/epilogue, w4 TMA, w5 MMA + TMEM
-constexpr int SP_OFF_C = 0;                              // 9 blocks of gathered rows
-constexpr int SP_QS = 4;                                 // query slots
-constexpr int SP_OFF_Q = SP_OFF_C + SP_KB * SP_BLOCK;    // SP_QS query slots
-constexpr int SP_OFF_P = SP_OFF_Q;                       // P: 2 blocks of 64 rows, over slots 0-1 after S
-constexpr int SP_OFF_VALID = SP_OFF_Q + SP_QS * SP_QBLOCK;  // [4] bit masks: slot row holds a valid index
-constexpr int SP_OFF_ROW = SP_OFF_VALID + 16;            // [128] latent row of each slot (-1: none)
+constexpr int SP_GW = 8;                       // gather / softmax / epilogue warps
+constexpr int SP_GT = SP_GW * 32;
+constexpr int SP_THREADS = SP_GT + 64;         // + TMA warp + MMA warp
+constexpr int SP_TMA_WARP = SP_GW, SP_MMA_WARP = SP_GW + 1;
+constexpr int SP_QS = 4;                       // query slots
+constexpr int SP_OFF_C = 0;                                  // 9 blocks of gathered rows
+constexpr int SP_OFF_RAW = SP_OFF_C + 4 * SP_BLOCK;          // FP8: codes [8 blocks][128 rows][64 B] (blocks 4-7)
+constexpr int SP_RAW_BLOCK = SP_ROWS * 64;
+constexpr int SP_OFF_Q = SP_OFF_C + SP_KB * SP_BLOCK;        // SP_QS query slots
+constexpr int SP_OFF_P = SP_OFF_Q;                           // P: 2 blocks of 64 keys, over slots 0-1 after S
+constexpr int SP_OFF_SCL = SP_OFF_Q + SP_QS * SP_QBLOCK;     // FP8: [128 rows][4] fp32 scales
+constexpr int SP_OFF_RED = SP_OFF_SCL + SP_ROWS * 16;        // [2][128] row maxima, [2][128] row sums
+constexpr int SP_OFF_VALID = SP_OFF_RED + 4 * SP_M * 4;      // [4] bit masks: slot row holds a valid index
+constexpr int SP_OFF_ROW = SP_OFF_VALID + 16;                // [128] latent row of each slot (-1: none)
 constexpr int SP_OFF_BAR = SP_OFF_ROW + SP_ROWS * 4;
 // c_full[9], q_full[4], q_empty[4], s_full, p_full, o_full[2], done
 constexpr int SP_NBAR = SP_KB + SP_QS + SP_QS + 1 + 1 + 2 + 1;
 constexpr int SP_OFF_MISC = SP_OFF_BAR + SP_NBAR * 8;
 constexpr int SP_SMEM = SP_OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(SP_SMEM <= 232448, "shared memory");
+static_assert(SP_OFF_RAW + 8 * SP_RAW_BLOCK == SP_OFF_C + 8 * SP_BLOCK, "codes fill blocks 4-7 exactly");
+constexpr int SP_FP8_ROW = 656;                // packed row: 512 codes, 4 fp32 scales, 64 bf16
+constexpr int SP_FP8_SCL = 512, SP_FP8_ROPE = 528;
 constexpr uint32_t SP_IDESC_S = umma_idesc_bf16(SP_M, SP_ROWS);              // Q x C^T, both K-major
 constexpr uint32_t SP_IDESC_O = umma_idesc_bf16(SP_M, 256, false, true);     // P x V, V MN-major
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
 struct SparseArgs {
-    const kvattn_bf16* latent;  // [B][L_max][576]
+    const void* latent;         // bf16 [B][L_max][576], or packed FP8 [B][L_max][656]
     const int32_t* idx;         // [B][k]
     kvattn_bf16* out;           // [B][Hq][512]
     float* lse;                 // [B][Hq] or null
-    float* part_o;              // [B][chunks][512][Hq] (head fastest)
-    float* part_ml;             // [B][chunks][Hq][2]
+    kvattn_bf16* part_o;        // [B][chunks][Hq][512] bf16, each chunk normalised by its own sum
+    float* part_lse;            // [B][chunks][Hq], log2 units (-inf: the chunk has no valid row)
     int32_t* dev_status;
     int B, Hq, L_max, k, chunks;
     float scale;
 };
 
+// The order in which the latent blocks are consumed: the FP8 variant's RoPE block
+// lands first (with the scales), the bf16 variant's blocks in column order.
+template <bool FP8>
+__device__ __forceinline__ int block_at(int i)
+{
+    return FP8 ? (i == 0 ? SP_KB - 1 : i - 1) : i;
+}
+
 // cp.async groups still pending after block kb's group may be at most 8 - kb.
-__device__ __forceinline__ void wait_block_groups(int kb)
+__device__ __forceinline__ void wait_groups_upto(int kb)
 {
     switch (kb) {
     case 0: cp_async_wait<8>(); break;
@@ -86,19 +114,61 @@ __device__ __forceinline__ void wait_block_groups(int kb)
     }
 }
 
+// Eight E4M3 codes (two 32-bit words) times a scale -> eight bf16 (one 16-byte
+// chunk).  E4M3 -> f16 is exact; the product is rounded to fp32, then to bf16.
+__device__ __forceinline__ uint4 dequant8(uint32_t w0, uint32_t w1, float s)
+{
+    uint32_t h[4];
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[0]) : "h"(static_cast<uint16_t>(w0 & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[1]) : "h"(static_cast<uint16_t>(w0 >> 16)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[2]) : "h"(static_cast<uint16_t>(w1 & 0xffffu)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h[3]) : "h"(static_cast<uint16_t>(w1 >> 16)));
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+        o[i] = pack_bf16x2(f.x * s, f.y * s);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 32 codes of one row (two 16-byte words) -> chunks 4 hh .. 4 hh + 3 of that row
+// of a swizzled bf16 block.
+__device__ __forceinline__ void dequant_store(uint8_t* blk, int r, int hh, uint4 c0, uint4 c1, float s)
+{
+    *reinterpret_cast<uint4*>(blk + swz128(r, 4 * hh + 0)) = dequant8(c0.x, c0.y, s);
+    *reinterpret_cast<uint4*>(blk + swz128(r, 4 * hh + 1)) = dequant8(c0.z, c0.w, s);
+    *reinterpret_cast<uint4*>(blk + swz128(r, 4 * hh + 2)) = dequant8(c1.x, c1.y, s);
+    *reinterpret_cast<uint4*>(blk + swz128(r, 4 * hh + 3)) = dequant8(c1.z, c1.w, s);
+}
+
+// Tiled shared -> global store through the tensor map (bulk-group completion).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+template <bool FP8>
 __global__ void __launch_bounds__(SP_THREADS, 1)
-    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, SparseArgs a)
+    sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+                       SparseArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint32_t* s_vmask = reinterpret_cast<uint32_t*>(smem + SP_OFF_VALID);
     int* s_row = reinterpret_cast<int*>(smem + SP_OFF_ROW);
+    float* s_scl = reinterpret_cast<float*>(smem + SP_OFF_SCL);
+    float* s_max = reinterpret_cast<float*>(smem + SP_OFF_RED);
+    float* s_sum = s_max + 2 * SP_M;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SP_OFF_BAR);
-    uint64_t* c_full = bars;                 // [9]: block kb of the rows landed (128 arrivals)
+    uint64_t* c_full = bars;                 // [9]: block kb of the rows ready (SP_GT arrivals)
     uint64_t* q_full = c_full + SP_KB;       // [SP_QS]
     uint64_t* q_empty = q_full + SP_QS;      // [SP_QS]
     uint64_t* s_full = q_empty + SP_QS;      // S complete in TMEM
-    uint64_t* p_full = s_full + 1;           // P written (S read), 128 arrivals
+    uint64_t* p_full = s_full + 1;           // P written (S read), SP_GT arrivals
     uint64_t* o_full = p_full + 1;           // [2]: O columns 0-255 / 256-511 complete
     uint64_t* done = o_full + 2;             // every MMA finished
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SP_OFF_MISC);
@@ -107,20 +177,23 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     const int chunk = blockIdx.x, b = blockIdx.y;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int i = 0; i < SP_KB; ++i) mbar_init(&c_full[i], 128);
+        for (int i = 0; i < SP_KB; ++i) mbar_init(&c_full[i], SP_GT);
         for (int i = 0; i < SP_QS; ++i) {
             mbar_init(&q_full[i], 1);
             mbar_init(&q_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) mbar_init(&o_full[i], 1);
         mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, SP_GT);
         mbar_init(done, 1);
         *s_abort = 0;
         fence_barrier_init();
     }
-    if (warp == 4 && lane == 0) tma_prefetch_desc(&tm_q);
-    if (warp == 5) {
+    if (warp == SP_TMA_WARP && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_o);
+    }
+    if (warp == SP_MMA_WARP) {
         tmem_alloc(s_tmem, 512);
         tmem_relinquish();
     }
@@ -131,10 +204,10 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     pdl_wait();
     pdl_trigger();
 
-    if (warp < 4) {
-        // ===== gather: the chunk's selected rows, block by block =====
+    if (warp < SP_GW) {
         const int t = tid;
-        {
+        // ===== the chunk's row indices =====
+        if (t < SP_ROWS) {
             const int slot = chunk * SP_ROWS + t;
             int j = slot < a.k ? a.idx[static_cast<long long>(b) * a.k + slot] : -1;
             if (j < -1 || j >= a.L_max) {
@@ -145,61 +218,137 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             if (lane == 0) s_vmask[warp] = vm;
             s_row[t] = j;
         }
-        named_bar_sync(1, 128);  // every slot's row is known
-        // copy job i of a block: row i / 8, 16-byte chunk i % 8 (eight lanes per line)
-        const kvattn_bf16* lat = a.latent + static_cast<long long>(b) * a.L_max * SP_DK;
+        named_bar_sync(1, SP_GT);  // every slot's row is known
         const uint32_t c0 = smem_u32(smem + SP_OFF_C);
-        int jr[8];
+        if constexpr (!FP8) {
+            // ===== gather: block kb of row r, 16-byte chunk ch: thread (r % 32) * 8 + ch =====
+            const kvattn_bf16* lat = static_cast<const kvattn_bf16*>(a.latent) + static_cast<long long>(b) * a.L_max * SP_DK;
+            const int ch = t & 7;
+            int jr[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) jr[u] = s_row[(t >> 3) + 16 * u];
+            for (int u = 0; u < 4; ++u) jr[u] = s_row[(t >> 3) + 32 * u];
 #pragma unroll
-        for (int kb = 0; kb < SP_KB; ++kb) {
+            for (int kb = 0; kb < SP_KB; ++kb) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int r = (t >> 3) + 16 * u, ch = t & 7;
-                const int j = jr[u];
-                cp_async16(c0 + kb * SP_BLOCK + swz128(r, ch),
-                           lat + static_cast<long long>(j < 0 ? 0 : j) * SP_DK + kb * 64 + ch * 8, j < 0 ? 0u : 16u);
+                for (int u = 0; u < 4; ++u) {
+                    const int r = (t >> 3) + 32 * u;
+                    const int j = jr[u];
+                    cp_async16(c0 + kb * SP_BLOCK + swz128(r, ch),
+                               lat + static_cast<long long>(j < 0 ? 0 : j) * SP_DK + kb * 64 + ch * 8, j < 0 ? 0u : 16u);
+                }
+                cp_async_commit();
+            }
+#pragma unroll
+            for (int kb = 0; kb < SP_KB; ++kb) {
+                wait_groups_upto(kb);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(&c_full[kb]);
+            }
+        } else {
+            // ===== gather of packed FP8 rows: group 0 = scales + the RoPE block, groups 1-8 = code blocks =====
+            const uint8_t* lat = static_cast<const uint8_t*>(a.latent) + static_cast<long long>(b) * a.L_max * SP_FP8_ROW;
+            auto row_ptr = [&](int j) { return lat + static_cast<long long>(j < 0 ? 0 : j) * SP_FP8_ROW; };
+            if (t < SP_ROWS) {
+                const int j = s_row[t];
+                cp_async16(smem_u32(s_scl + t * 4), row_ptr(j) + SP_FP8_SCL, j < 0 ? 0u : 16u);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int r = (t >> 3) + 32 * u, ch = t & 7;
+                const int j = s_row[r];
+                cp_async16(c0 + (SP_KB - 1) * SP_BLOCK + swz128(r, ch), row_ptr(j) + SP_FP8_ROPE + ch * 16,
+                           j < 0 ? 0u : 16u);
             }
             cp_async_commit();
-        }
+            const uint32_t raw0 = smem_u32(smem + SP_OFF_RAW);
 #pragma unroll
-        for (int kb = 0; kb < SP_KB; ++kb) {
-            wait_block_groups(kb);
+            for (int jb = 0; jb < 8; ++jb) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int r = (t >> 2) + 64 * u, ch = t & 3;
+                    const int j = s_row[r];
+                    cp_async16(raw0 + jb * SP_RAW_BLOCK + r * 64 + ch * 16, row_ptr(j) + jb * 64 + ch * 16,
+                               j < 0 ? 0u : 16u);
+                }
+                cp_async_commit();
+            }
+            // the RoPE block is ready as it lands
+            cp_async_wait<8>();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&c_full[kb]);
+            mbar_arrive(&c_full[SP_KB - 1]);
+            // dequantisation: thread t takes row t / 2, codes 32 (t % 2) .. + 31 of each block
+            const int r = t >> 1, hh = t & 1;
+            const uint8_t* raw = smem + SP_OFF_RAW;
+            // blocks 0-3: their codes sit in blocks 4-5's space, their output in blocks 0-3
+#pragma unroll
+            for (int jb = 0; jb < 4; ++jb) {
+                wait_groups_upto(jb + 1);
+                named_bar_sync(1, SP_GT);  // every thread's copies of the block (and the scales) are visible
+                const uint8_t* src = raw + jb * SP_RAW_BLOCK + r * 64 + hh * 32;
+                dequant_store(smem + SP_OFF_C + jb * SP_BLOCK, r, hh, *reinterpret_cast<const uint4*>(src),
+                              *reinterpret_cast<const uint4*>(src + 16), s_scl[r * 4 + (jb >> 1)]);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(&c_full[jb]);
+            }
+            // blocks 4-7 overwrite the space the codes occupy: read every code first
+            cp_async_wait<0>();
+            named_bar_sync(1, SP_GT);
+            uint4 cr[4][2];
+#pragma unroll
+            for (int jb = 4; jb < 8; ++jb) {
+                const uint8_t* src = raw + jb * SP_RAW_BLOCK + r * 64 + hh * 32;
+                cr[jb - 4][0] = *reinterpret_cast<const uint4*>(src);
+                cr[jb - 4][1] = *reinterpret_cast<const uint4*>(src + 16);
+            }
+            named_bar_sync(1, SP_GT);
+#pragma unroll
+            for (int jb = 4; jb < 8; ++jb) {
+                dequant_store(smem + SP_OFF_C + jb * SP_BLOCK, r, hh, cr[jb - 4][0], cr[jb - 4][1],
+                              s_scl[r * 4 + (jb >> 1)]);
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                mbar_arrive(&c_full[jb]);
+            }
         }
 
-        // ===== softmax of head row t (TMEM lane t) =====
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const bool live = t < a.Hq;
+        // ===== softmax of head row h over key columns 64 g .. 64 g + 63 =====
+        const int g = warp >> 2, quarter = warp & 3;
+        const int h = quarter * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const bool live = h < a.Hq;
         const float sl2 = a.scale * kLog2e;
-        float m = -INFINITY, l = 0.f;
-        if (warp_wait(s_full, 0, s_abort)) {
+        uint32_t sv[2][32];
+        float mx = -INFINITY;
+        const bool have_s = warp_wait(s_full, 0, s_abort);
+        if (have_s) {
             tc_fence_after();
-            uint32_t sv[4][32];
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) tmem_ld32(tmem + lane_off + cc * 32, sv[cc]);
+            tmem_ld32(tmem + lane_off + 64 * g, sv[0]);
+            tmem_ld32(tmem + lane_off + 64 * g + 32, sv[1]);
             tmem_wait_ld();
-            float mx = -INFINITY;
+            tmem_regs_ready(sv[0]);
+            tmem_regs_ready(sv[1]);
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                const uint32_t vm = s_vmask[cc];
+            for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t vm = s_vmask[2 * g + cc];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     if (!((vm >> i) & 1u)) sv[cc][i] = 0xff800000u;  // -inf: not a selected row
                     mx = fmaxf(mx, __uint_as_float(sv[cc][i]));
                 }
             }
-            m = mx * sl2;
-            const float mu = m == -INFINITY ? 0.f : m;
+        }
+        s_max[g * SP_M + h] = mx;
+        named_bar_sync(2, SP_GT);
+        const float m = fmaxf(s_max[h], s_max[SP_M + h]) * sl2;
+        const float mu = m == -INFINITY ? 0.f : m;
+        float l_half = 0.f;
+        if (have_s) {
             const float2 sc2 = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
             float2 acc = make_float2(0.f, 0.f);
-            uint8_t* prow = smem + SP_OFF_P;
+            uint8_t* pblk = smem + SP_OFF_P + g * SP_BLOCK;
 #pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {  // 8-row chunk (16 bytes of P) q of this 32-row group
+                for (int q = 0; q < 4; ++q) {  // 8-key chunk (16 bytes of P) q of this 32-key group
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -217,78 +366,77 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                         acc = __fadd2_rn(acc, p);
                         pk[e] = pack_bf16x2(p.x, p.y);
                     }
-                    const int col = cc * 32 + q * 8;  // first selected row of the 16-byte chunk
-                    *reinterpret_cast<uint4*>(prow + (col >> 6) * SP_BLOCK + swz128(t, (col & 63) >> 3)) =
-                        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(pblk + swz128(h, cc * 4 + q)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
-            l = acc.x + acc.y;
+            l_half = acc.x + acc.y;
         }
         // S is read and P is written: the P V MMAs may reuse S's columns
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         tc_fence_before();
         mbar_arrive(p_full);
+        s_sum[g * SP_M + h] = l_half;
+        named_bar_sync(2, SP_GT);
+        const float l = s_sum[h] + s_sum[SP_M + h];
 
-        // ===== epilogue: O row t, half by half =====
+        // ===== epilogue: O columns 256 g .. 256 g + 255 of head row h =====
         const bool one = a.chunks == 1;
-        const long long bh = static_cast<long long>(b) * a.Hq + t;
-        const long long pc = (static_cast<long long>(b) * a.chunks + chunk) * SP_DV;  // partial column 0
         const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-            if (!warp_wait(&o_full[half], 0, s_abort)) break;
+        uint8_t* stg = smem + SP_OFF_C + 4 * g * SP_BLOCK;  // the blocks this half's P V has consumed
+        const bool have_o = warp_wait(&o_full[g], 0, s_abort);
+        if (have_o) {
             tc_fence_after();
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
                 uint32_t ov[32];
-                tmem_ld32(tmem + lane_off + half * 256 + cc * 32, ov);
+                tmem_ld32(tmem + lane_off + 256 * g + 32 * cc, ov);
                 tmem_wait_ld();
-                if (!live) continue;
-                const int col = half * 256 + cc * 32;
-                if (one) {
-                    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + bh * SP_DV + col;
+                tmem_regs_ready(ov);
+                uint8_t* box = stg + (cc >> 1) * SP_BLOCK;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8)
-                        *reinterpret_cast<uint4*>(o + i) = make_uint4(
-                            pack_bf16x2(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv),
-                            pack_bf16x2(__uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv),
-                            pack_bf16x2(__uint_as_float(ov[i + 4]) * inv, __uint_as_float(ov[i + 5]) * inv),
-                            pack_bf16x2(__uint_as_float(ov[i + 6]) * inv, __uint_as_float(ov[i + 7]) * inv));
-                } else {
-                    // [column][head]: the warp's 32 heads of one column are one 128-byte line
-                    float* po = a.part_o + (pc + col) * a.Hq + t;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) po[static_cast<long long>(i) * a.Hq] = __uint_as_float(ov[i]);
+                for (int i = 0; i < 4; ++i) {
+                    const float* f = reinterpret_cast<const float*>(ov) + 8 * i;
+                    *reinterpret_cast<uint4*>(box + swz128(h, (cc & 1) * 4 + i)) =
+                        make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
+                                   pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
                 }
             }
         }
-        if (live) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        named_bar_sync(3 + g, 128);
+        if (quarter == 0 && lane == 0 && have_o && !*s_abort) {
+            const int z = one ? b : b * a.chunks + chunk;
+#pragma unroll
+            for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tm_o, stg + bx * SP_BLOCK, 256 * g + 64 * bx, 0, z);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // shared memory read before exit
+        }
+        if (g == 0 && live) {
+            const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
             if (one) {
-                if (a.lse) a.lse[bh] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+                if (a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = lse2 * kLn2;
             } else {
-                const long long pr = (static_cast<long long>(b) * a.chunks + chunk) * a.Hq + t;
-                a.part_ml[pr * 2] = m;  // log2 units; -inf when the chunk holds no valid row
-                a.part_ml[pr * 2 + 1] = l;
+                a.part_lse[(static_cast<long long>(b) * a.chunks + chunk) * a.Hq + h] = lse2;
             }
         }
-    } else if (warp == 4) {
-        // ===== queries: 64 columns at a time through SP_QS slots =====
+    } else if (warp == SP_TMA_WARP) {
+        // ===== queries: 64 columns at a time through SP_QS slots, in the blocks' order =====
         if (lane == 0) {
             bool ok = true;
             const uint32_t q_bytes = static_cast<uint32_t>(a.Hq) * 128;
-            int kb = 0;
-            for (; kb < SP_KB; ++kb) {
-                const int s = kb % SP_QS;
-                if (kb >= SP_QS && !(ok = mbar_wait(&q_empty[s], ((kb / SP_QS) - 1) & 1))) break;
+            int i = 0;
+            for (; i < SP_KB; ++i) {
+                const int s = i % SP_QS;
+                if (i >= SP_QS && !(ok = mbar_wait(&q_empty[s], ((i / SP_QS) - 1) & 1))) break;
                 mbar_arrive_expect_tx(&q_full[s], q_bytes);
-                tma_load_3d(smem + SP_OFF_Q + s * SP_QBLOCK, &tm_q, &q_full[s], kb * 64, 0, b);
+                tma_load_3d(smem + SP_OFF_Q + s * SP_QBLOCK, &tm_q, &q_full[s], block_at<FP8>(i) * 64, 0, b);
             }
             if (!ok) {
                 *s_abort = 1;
                 report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
             }
             // copies in flight complete before the CTA leaves (bounded waits)
-            for (int j = kb - SP_QS > 0 ? kb - SP_QS : 0; j < kb; ++j) mbar_wait(&q_full[j % SP_QS], (j / SP_QS) & 1);
+            for (int j = i - SP_QS > 0 ? i - SP_QS : 0; j < i; ++j) mbar_wait(&q_full[j % SP_QS], (j / SP_QS) & 1);
         }
     } else {
         // ===== MMA issuer =====
@@ -296,16 +444,17 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             bool ok = true;
             const uint32_t c0 = smem_u32(smem + SP_OFF_C), q0 = smem_u32(smem + SP_OFF_Q);
             const uint32_t p0 = smem_u32(smem + SP_OFF_P);
-            for (int kb = 0; kb < SP_KB && ok; ++kb) {
+            for (int i = 0; i < SP_KB && ok; ++i) {
+                const int kb = block_at<FP8>(i);
                 if (!(ok = mbar_wait(&c_full[kb], 0))) break;
-                if (!(ok = mbar_wait(&q_full[kb % SP_QS], (kb / SP_QS) & 1))) break;
+                if (!(ok = mbar_wait(&q_full[i % SP_QS], (i / SP_QS) & 1))) break;
                 tc_fence_after();
-                const uint32_t qs = q0 + (kb % SP_QS) * SP_QBLOCK, cs = c0 + kb * SP_BLOCK;
+                const uint32_t qs = q0 + (i % SP_QS) * SP_QBLOCK, cs = c0 + kb * SP_BLOCK;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     tc_mma_bf16(tmem, umma_desc_k_sw128(qs + kk * 32), umma_desc_k_sw128(cs + kk * 32), SP_IDESC_S,
-                                (kb | kk) ? 1u : 0u);
-                tc_commit(&q_empty[kb % SP_QS]);
+                                (i | kk) ? 1u : 0u);
+                tc_commit(&q_empty[i % SP_QS]);
             }
             if (ok) {
                 tc_commit(s_full);
@@ -335,95 +484,107 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == SP_MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
 }
 
-// ---- merge of the chunk partials ------------------------------------------------
-// CTA = (batch row, 32 heads, 32 value columns), 256 threads: lane = head, warp w
-// = columns 4w .. 4w+3.  Every thread derives its head's chunk weights from the
-// (m, l) pairs and requests all chunks' values at once (one round trip); the
-// 32 x 32 result is transposed through shared memory so that each head's 32
-// columns are written as one 64-byte run.
+// ---- merge of the chunk parts ------------------------------------------------------
+// CTA = (batch row, 4 heads), 64 threads per head, one 16-byte chunk (8 columns)
+// each.  A thread loads every chunk's lse and its 16 bytes of every part at
+// once (one round trip), then out = sum_c 2^(lse_c - LSE) o_c and
+// LSE = log2 sum_c 2^lse_c (all in log2 units; lse is written in natural log).
 constexpr int SPM_MAX_CHUNKS = 16;  // k <= 2048 in chunks of 128
-constexpr int SPM_HEADS = 32, SPM_COLS = 32;
+constexpr int SPM_HEADS = 4;
 
-__global__ void __launch_bounds__(256) sparse_merge_kernel(SparseArgs a)
+__global__ void __launch_bounds__(SPM_HEADS * 64) sparse_merge_kernel(SparseArgs a)
 {
-    __shared__ float s_o[SPM_HEADS][SPM_COLS + 1];
-    __shared__ float s_lse[SPM_HEADS];
     pdl_wait();
     pdl_trigger();
     const int C = a.chunks;
-    const int col0 = blockIdx.x * SPM_COLS, h0 = blockIdx.y * SPM_HEADS, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = h0 + lane;
-    const long long mlrow = static_cast<long long>(b) * C * a.Hq + h;  // (m, l) row of chunk 0
-    float2 ml[SPM_MAX_CHUNKS];
-    float ov[SPM_MAX_CHUNKS][4];
+    const int b = blockIdx.y;
+    const int h = blockIdx.x * SPM_HEADS + (threadIdx.x >> 6);
+    const int j = threadIdx.x & 63;
+    if (h >= a.Hq) return;
+    float ls[SPM_MAX_CHUNKS];
+    uint4 ov[SPM_MAX_CHUNKS];
 #pragma unroll
     for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
         if (c < C) {
-            ml[c] = __ldcg(reinterpret_cast<const float2*>(a.part_ml) + mlrow + static_cast<long long>(c) * a.Hq);
-            const float* po = a.part_o + ((static_cast<long long>(b) * C + c) * SP_DV + col0 + 4 * warp) * a.Hq + h;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) ov[c][i] = __ldcg(po + static_cast<long long>(i) * a.Hq);
+            const long long row = (static_cast<long long>(b) * C + c) * a.Hq + h;
+            ls[c] = __ldcg(a.part_lse + row);
+            ov[c] = __ldcg(reinterpret_cast<const uint4*>(a.part_o + row * SP_DV) + j);
         }
     }
     float M = -INFINITY;
 #pragma unroll
     for (int c = 0; c < SPM_MAX_CHUNKS; ++c)
-        if (c < C) M = fmaxf(M, ml[c].x);
+        if (c < C) M = fmaxf(M, ls[c]);
     const float Mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float L = 0.f;
+    float wgt[SPM_MAX_CHUNKS];
+#pragma unroll
+    for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
+        wgt[c] = c < C ? fast_exp2(ls[c] - Mu) : 0.f;
+        L += wgt[c];
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
         if (c < C) {
-            const float w = fast_exp2(ml[c].x - Mu);
-            L += w * ml[c].y;
+            const float wc = wgt[c] * inv;
+            const uint32_t w4[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[i] += w * ov[c][i];
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = fmaf(wc, bf16_lo(w4[i]), acc[2 * i]);
+                acc[2 * i + 1] = fmaf(wc, bf16_hi(w4[i]), acc[2 * i + 1]);
+            }
         }
     }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) s_o[lane][4 * warp + i] = acc[i] * inv;
-    if (warp == 0) s_lse[lane] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
-    __syncthreads();
-    // thread -> (head tid / 8, columns 4 (tid % 8) .. +3): eight threads per head's 64 bytes
-    const int hh = threadIdx.x >> 3, cc = (threadIdx.x & 7) * 4;
-    __nv_bfloat16* out =
-        reinterpret_cast<__nv_bfloat16*>(a.out) + (static_cast<long long>(b) * a.Hq + h0 + hh) * SP_DV + col0 + cc;
-    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(s_o[hh][cc], s_o[hh][cc + 1]),
-                                                pack_bf16x2(s_o[hh][cc + 2], s_o[hh][cc + 3]));
-    if (blockIdx.x == 0 && threadIdx.x < SPM_HEADS && a.lse)
-        a.lse[static_cast<long long>(b) * a.Hq + h0 + threadIdx.x] = s_lse[threadIdx.x];
+    const long long ob = (static_cast<long long>(b) * a.Hq + h) * SP_DV;
+    reinterpret_cast<uint4*>(a.out + ob)[j] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                         pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    if (j == 0 && a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+}
+
+template <bool FP8>
+cudaError_t set_smem_attr_once()
+{
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && attr_set[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(sparse_attn_kernel<FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SP_SMEM);
+    if (e == cudaSuccess && dev < 64) attr_set[dev] = true;
+    return e;
 }
 
 }  // namespace
 
 int sparse_chunks(int k) { return (k + SP_ROWS - 1) / SP_ROWS; }
 
+size_t sparse_part_o_bytes(int B, int Hq, int k)
+{
+    const int c = sparse_chunks(k);
+    if (c <= 1) return 0;
+    return static_cast<size_t>(B) * c * Hq * SP_DV * sizeof(kvattn_bf16);
+}
+
 size_t sparse_partial_bytes(int B, int Hq, int k)
 {
     const int c = sparse_chunks(k);
     if (c <= 1) return 0;
-    return static_cast<size_t>(B) * c * Hq * (SP_DV + 2) * sizeof(float);
+    return sparse_part_o_bytes(B, Hq, k) + static_cast<size_t>(B) * c * Hq * sizeof(float);
 }
 
-cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, cudaStream_t stream)
+cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_o,
+                               cudaStream_t stream)
 {
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = l.fp8 ? set_smem_attr_once<true>() : set_smem_attr_once<false>();
     if (e != cudaSuccess) return e;
-    if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SP_SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
     SparseArgs a{};
     a.latent = l.latent;
     a.idx = l.idx;
@@ -436,11 +597,17 @@ cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, c
     a.chunks = sparse_chunks(l.k);
     a.scale = l.scale;
     a.dev_status = l.dev_status;
-    a.part_o = l.workspace;
-    a.part_ml = l.workspace ? l.workspace + static_cast<size_t>(l.B) * a.chunks * l.Hq * SP_DV : nullptr;
-    e = launch_pdl(sparse_attn_kernel, dim3(a.chunks, l.B), dim3(SP_THREADS), SP_SMEM, stream, tm_q, a);
+    if (a.chunks > 1) {
+        a.part_o = static_cast<kvattn_bf16*>(l.workspace);
+        a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(l.workspace) + sparse_part_o_bytes(l.B, l.Hq, l.k));
+    }
+    e = l.fp8 ? launch_pdl(sparse_attn_kernel<true>, dim3(a.chunks, l.B), dim3(SP_THREADS), SP_SMEM, stream, tm_q,
+                           tm_o, a)
+              : launch_pdl(sparse_attn_kernel<false>, dim3(a.chunks, l.B), dim3(SP_THREADS), SP_SMEM, stream, tm_q,
+                           tm_o, a);
     if (e != cudaSuccess || a.chunks == 1) return e;
-    return launch_pdl(sparse_merge_kernel, dim3(SP_DV / SPM_COLS, l.Hq / SPM_HEADS, l.B), dim3(256), 0, stream, a);
+    return launch_pdl(sparse_merge_kernel, dim3((l.Hq + SPM_HEADS - 1) / SPM_HEADS, l.B), dim3(SPM_HEADS * 64), 0,
+                      stream, a);
 }
 
 }  // namespace kvattn

@@ -69,6 +69,14 @@ _lib.attn_decode_gqa_sparse_workspace_bytes.restype = _sz
 _lib.attn_decode_gqa_sparse.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp,
                                         _vp, _sz, _vp, _vp]
 _lib.attn_merge_lse.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.attn_decode_sparse_fp8.argtypes = [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz,
+                                        _vp, _vp]
+_lib.latent_quant_fp8.argtypes = [_vp, ctypes.c_longlong, _vp, _vp]
+_lib.dsa_topk_candidates.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.dsa_topk_merge.argtypes = [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]
+_lib.dsa_index_topk_fp8.argtypes = [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp,
+                                    _vp]
+_lib.idx_key_quant_fp8.argtypes = [_vp, ctypes.c_longlong, _vp, _vp, _vp]
 _lib.kvattn_test_decode_stall.argtypes = [_i32, ctypes.c_longlong]
 _lib.attn_decode_gqa_noalloc_reset.argtypes = [_vp]
 
@@ -401,6 +409,70 @@ def dsa_index_topk(q_idx, w, k_idx, k, seq_lens=None, topk_idx=None, scores_out=
     return topk_idx, scores_out
 
 
+def dsa_index_topk_fp8(q_idx, w, k_codes, k_scales, k, seq_lens=None, topk_idx=None, scores_out=None, ws=None,
+                       dev_status=None, want_scores=True):
+    """q_idx [B, 64, 128] bf16, w [B, 64] fp32, k_codes [B, L_max, 128] uint8 and
+    k_scales [B, L_max] fp32 (idx_key_quant_fp8) -> (topk_idx int32 [B, k],
+    scores fp32 [B, L_max] or None)."""
+    _need(q_idx, torch.bfloat16, "q_idx")
+    _need(k_codes, torch.uint8, "k_codes")
+    _need(k_scales, torch.float32, "k_scales")
+    _need(w, torch.float32, "w")
+    for t, n in ((q_idx, "q_idx"), (k_codes, "k_codes"), (k_scales, "k_scales"), (w, "w")):
+        _contig(t, n)
+    B, HI, dI = q_idx.shape
+    L_max = k_codes.shape[1]
+    if tuple(k_scales.shape) != (B, L_max):
+        raise ValueError("k_scales must be [B, L_max]")
+    if seq_lens is not None:
+        _need(seq_lens, torch.int32, "seq_lens")
+    if topk_idx is None:
+        topk_idx = torch.empty((B, k), dtype=torch.int32, device=q_idx.device)
+    if scores_out is None and want_scores:
+        scores_out = torch.empty((B, L_max), dtype=torch.float32, device=q_idx.device)
+    if ws is None:
+        ws = workspace(dsa_index_topk_workspace_bytes(B, L_max, k), q_idx.device)
+    _check(_lib.dsa_index_topk_fp8(_ptr(q_idx), _ptr(w), _ptr(k_codes), _ptr(k_scales), _ptr(seq_lens), B, HI, dI,
+                                   L_max, k, _ptr(topk_idx), _ptr(scores_out), _ptr(ws), ws.numel(),
+                                   _ptr(dev_status), _stream()))
+    return topk_idx, scores_out
+
+
+def dsa_topk_candidates(scores, topk_idx, idx_offset, cand_scores=None, cand_idx=None):
+    """One key slice's selection as (score, global index) pairs: scores [B, L_slice] fp32,
+    topk_idx int32 [B, k] (local indices) -> (cand_scores fp32 [B, k], cand_idx int32 [B, k])."""
+    _need(scores, torch.float32, "scores")
+    _need(topk_idx, torch.int32, "topk_idx")
+    _contig(scores, "scores")
+    _contig(topk_idx, "topk_idx")
+    B, L_slice = scores.shape
+    k = topk_idx.shape[1]
+    if cand_scores is None:
+        cand_scores = torch.empty((B, k), dtype=torch.float32, device=scores.device)
+    if cand_idx is None:
+        cand_idx = torch.empty((B, k), dtype=torch.int32, device=scores.device)
+    _check(_lib.dsa_topk_candidates(_ptr(scores), _ptr(topk_idx), B, L_slice, k, int(idx_offset), _ptr(cand_scores),
+                                    _ptr(cand_idx), _stream()))
+    return cand_scores, cand_idx
+
+
+def dsa_topk_merge(cand_scores, cand_idx, topk_idx=None, dev_status=None):
+    """The slices' candidates [n_parts, B, k] (slice order) -> topk_idx int32 [B, k]: the
+    k best under (score desc, index asc), increasing index order, -1 padded."""
+    _need(cand_scores, torch.float32, "cand_scores")
+    _need(cand_idx, torch.int32, "cand_idx")
+    _contig(cand_scores, "cand_scores")
+    _contig(cand_idx, "cand_idx")
+    n, B, k = cand_idx.shape
+    if tuple(cand_scores.shape) != (n, B, k):
+        raise ValueError("cand_scores and cand_idx shapes differ")
+    if topk_idx is None:
+        topk_idx = torch.empty((B, k), dtype=torch.int32, device=cand_idx.device)
+    _check(_lib.dsa_topk_merge(_ptr(cand_scores), _ptr(cand_idx), n, B, k, _ptr(topk_idx), _ptr(dev_status),
+                               _stream()))
+    return topk_idx
+
+
 def attn_decode_sparse_workspace_bytes(B, Hq, Dv, k) -> int:
     return int(_lib.attn_decode_sparse_workspace_bytes(B, Hq, Dv, k))
 
@@ -426,6 +498,72 @@ def attn_decode_sparse(q, latent, topk_idx, Dv, scale, out=None, lse=None, ws=No
     _check(_lib.attn_decode_sparse(_ptr(q), _ptr(latent), _ptr(topk_idx), B, Hq, Dk, Dv, L_max, k, float(scale),
                                    _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status), _stream()))
     return out, lse
+
+
+def attn_decode_sparse_fp8(q, latent_fp8, topk_idx, Dv, scale, out=None, lse=None, ws=None, dev_status=None,
+                           want_lse=True):
+    """q [B, Hq, 576] bf16, latent_fp8 [B, L_max, 656] uint8 (latent_quant_fp8 rows),
+    topk_idx int32 [B, k] -> (out [B, Hq, Dv] bf16, lse [B, Hq] fp32)."""
+    _need(q, torch.bfloat16, "q")
+    _need(latent_fp8, torch.uint8, "latent_fp8")
+    _need(topk_idx, torch.int32, "topk_idx")
+    for t, n in ((q, "q"), (latent_fp8, "latent_fp8"), (topk_idx, "topk_idx")):
+        _contig(t, n)
+    B, Hq, Dk = q.shape
+    if latent_fp8.dim() != 3 or latent_fp8.shape[0] != B or latent_fp8.shape[2] != LATENT_FP8_ROW_BYTES:
+        raise ValueError("latent_fp8 must be [B, L_max, 656]")
+    L_max = latent_fp8.shape[1]
+    k = topk_idx.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, Dv), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(attn_decode_sparse_workspace_bytes(B, Hq, Dv, k), q.device)
+    _check(_lib.attn_decode_sparse_fp8(_ptr(q), _ptr(latent_fp8), _ptr(topk_idx), B, Hq, Dk, Dv, L_max, k,
+                                       float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(dev_status),
+                                       _stream()))
+    return out, lse
+
+
+LATENT_FP8_ROW_BYTES = 656
+
+
+def latent_quant_fp8(latent, packed=None):
+    """latent [..., 576] bf16 (contiguous) -> packed FP8 rows [..., 656] uint8."""
+    _need(latent, torch.bfloat16, "latent")
+    _contig(latent, "latent")
+    if latent.shape[-1] != 576:
+        raise ValueError("latent rows are 576 wide")
+    n = latent.numel() // 576
+    if packed is None:
+        packed = torch.empty(tuple(latent.shape[:-1]) + (LATENT_FP8_ROW_BYTES,), dtype=torch.uint8,
+                             device=latent.device)
+    _need(packed, torch.uint8, "packed")
+    _contig(packed, "packed")
+    if packed.numel() != n * LATENT_FP8_ROW_BYTES:
+        raise ValueError("packed must hold 656 bytes per row")
+    _check(_lib.latent_quant_fp8(_ptr(latent), n, _ptr(packed), _stream()))
+    return packed
+
+
+def idx_key_quant_fp8(k_idx, codes=None, scales=None):
+    """k_idx [..., 128] bf16 (contiguous) -> (codes [..., 128] uint8, scales [...] fp32)."""
+    _need(k_idx, torch.bfloat16, "k_idx")
+    _contig(k_idx, "k_idx")
+    if k_idx.shape[-1] != 128:
+        raise ValueError("indexer keys are 128 wide")
+    n = k_idx.numel() // 128
+    if codes is None:
+        codes = torch.empty(k_idx.shape, dtype=torch.uint8, device=k_idx.device)
+    if scales is None:
+        scales = torch.empty(k_idx.shape[:-1], dtype=torch.float32, device=k_idx.device)
+    _need(codes, torch.uint8, "codes")
+    _need(scales, torch.float32, "scales")
+    if codes.numel() != n * 128 or scales.numel() != n:
+        raise ValueError("codes / scales sizes")
+    _check(_lib.idx_key_quant_fp8(_ptr(k_idx), n, _ptr(codes), _ptr(scales), _stream()))
+    return codes, scales
 
 
 QSA_BLOCK = 4

@@ -83,3 +83,63 @@ def test_shard_lengths_partition_every_row():
     # a slice is full before the next one holds anything
     for r in range(n - 1):
         assert torch.all((parts[r + 1] == 0) | (parts[r] == S))
+
+
+def _index_inputs():
+    rng = np.random.default_rng(9)
+    B, HI, dI, L = 3, 8, 16, 96
+    q = rng.standard_normal((B, HI, dI))
+    w = rng.uniform(0, 1, (B, HI)).astype(np.float32)
+    kk = rng.standard_normal((B, L, dI))
+    kk[:, 50:60] = kk[:, 10:20]       # equal scores on both sides of the slice boundary (48)
+    lens = np.array([96, 30, 61], np.int32)
+    to_bits = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.uint16).numpy()
+    return to_bits(q), w, to_bits(kk), lens
+
+
+def _index_worker(rank, world, port, out_dir, k):
+    sys.path.insert(0, ROOT)
+    import oracle
+    from mqa_kv_cache_b200 import shard
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=timedelta(seconds=60))
+    try:
+        q, w, kk, lens = _index_inputs()
+        S = kk.shape[1] // world
+        my = shard.shard_lengths(torch.from_numpy(lens), rank, S).numpy()
+        sc = oracle.dsa_scores(q, w, np.ascontiguousarray(kk[:, rank * S:(rank + 1) * S]), my)
+        loc = oracle.topk(sc, k, lens=my)                                   # [B, k] local, -1 padded
+        cs = np.where(loc >= 0, np.take_along_axis(sc, np.maximum(loc, 0), 1), -np.inf).astype(np.float32)
+        ci = np.where(loc >= 0, loc + rank * S, -1).astype(np.int32)
+        cs_all, ci_all = shard.gather_candidates(torch.from_numpy(cs), torch.from_numpy(ci))
+        np.save(os.path.join(out_dir, f"cs{rank}.npy"), cs_all.numpy())
+        np.save(os.path.join(out_dir, f"ci{rank}.npy"), ci_all.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_indexer_candidates_give_the_global_topk(tmp_path):
+    """Each rank keeps the top-k of its key slice; the union of the gathered candidates
+    holds the global top-k, ties across the slice boundary included."""
+    import oracle
+    world, k = 2, 12
+    mp.start_processes(_index_worker, args=(world, _free_port(), str(tmp_path), k), nprocs=world, join=True,
+                       start_method="spawn")
+    q, w, kk, lens = _index_inputs()
+    cs = [np.load(tmp_path / f"cs{r}.npy") for r in range(world)]
+    ci = [np.load(tmp_path / f"ci{r}.npy") for r in range(world)]
+    assert np.array_equal(cs[0], cs[1]) and np.array_equal(ci[0], ci[1])
+    assert cs[0].shape == (world, 3, k)
+    full = oracle.dsa_scores(q, w, kk, lens)
+    want = oracle.topk(full, k, lens=lens)
+    B, L = full.shape
+    for b in range(B):
+        union = np.full(L, -np.inf)
+        for p in range(world):
+            sel = ci[0][p, b] >= 0
+            assert np.all(ci[0][p, b][sel] // (L // world) == p)            # part p holds slice p's indices
+            union[ci[0][p, b][sel]] = cs[0][p, b][sel]
+        n_valid = int(lens[b])
+        got = oracle.topk(union[None], k, lens=np.array([L], np.int32))[0]
+        got = got[:min(k, n_valid)]
+        np.testing.assert_array_equal(got, want[b][:min(k, n_valid)])
