@@ -496,8 +496,10 @@ def idx_key_fp8_bytes(d_I=128):
 
 
 def dsa_scores_fp8(q_idx, w, codes, kscale, lens, nthreads=0):
-    """Indexer scores on FP8 keys: q_idx [B,H_I,d_I] uint16, w [B,H_I] float32,
-    codes [B,L_max,d_I] uint8, kscale [B,L_max] float32 -> scores [B, L_max] fp64."""
+    """Indexer scores in fp8: the query heads q_idx [B,H_I,d_I] (bf16 bits) are quantised
+    to E4M3 like the keys, and s = sum_j w_j ReLU(qhat_j . khat_t) on the dequantised
+    operands.  w [B,H_I] float32, codes [B,L_max,d_I] uint8, kscale [B,L_max] float32
+    -> scores [B, L_max] fp64."""
     q_idx = np.ascontiguousarray(q_idx, np.uint16)
     codes = np.ascontiguousarray(codes, np.uint8)
     kscale = np.ascontiguousarray(kscale, np.float32)

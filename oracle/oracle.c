@@ -705,9 +705,12 @@ int oracle_latent_fp8_row_bytes(void) { return ORC_LAT_NOPE + (ORC_LAT_NOPE / OR
 int oracle_idx_key_fp8_bytes(int d_I) { return d_I + 4; }
 
 /*
- * Indexer scores on FP8 keys ([P1] §2.2 (1) on the dequantised keys):
- *   s_{b,t} = sum_j w_{b,j} * ReLU(q^I_{b,j} . khat_{b,t}),  khat = value(code) * scale.
- * codes [B][L_max][d_I], scales [B][L_max] fp32; otherwise as oracle_dsa_scores.
+ * Indexer scores in fp8 ([P1] §2.2 (1): the indexer runs stably in fp8, read as its
+ * product running on E4M3 operands): each indexer query head q^I_{b,j} (bf16, d_I
+ * values, one group) and each key are quantised with the rule above, and
+ *   s_{b,t} = sum_j w_{b,j} * ReLU(qhat_{b,j} . khat_{b,t}),  hat = value(code) * scale.
+ * qI [B][H_I][d_I] bf16 (quantised here), codes [B][L_max][d_I], scales [B][L_max]
+ * fp32; otherwise as oracle_dsa_scores.
  */
 int oracle_dsa_scores_fp8(const uint16_t* qI, const float* w, const uint8_t* codes, const float* kscale,
                           const int32_t* lens, int B, int HI, int dI, int L_max, double* scores, int nthreads)
@@ -715,7 +718,19 @@ int oracle_dsa_scores_fp8(const uint16_t* qI, const float* w, const uint8_t* cod
     if (B < 0 || HI <= 0 || dI <= 0 || L_max < 0) return -1;
     for (int b = 0; b < B; ++b)
         if (lens[b] < 0 || lens[b] > L_max) return -2;
-    src_t Q = {qI, 0};
+    int64_t nq = (int64_t)B * HI;
+    uint8_t* qc = (uint8_t*)malloc((size_t)(nq * dI > 0 ? nq * dI : 1));
+    float* qs = (float*)malloc(sizeof(float) * (size_t)(nq > 0 ? nq : 1));
+    double* qd = (double*)malloc(sizeof(double) * (size_t)(nq * dI > 0 ? nq * dI : 1));
+    if (!qc || !qs || !qd) {
+        free(qc);
+        free(qs);
+        free(qd);
+        return -3;
+    }
+    oracle_quant_fp8_groups(qI, nq, dI, qc, qs);
+    oracle_dequant_fp8_groups(qc, qs, nq, dI, qd);
+    src_t Q = {qd, 1};
     int nt = set_threads(nthreads);
     int64_t n_units = (int64_t)B * L_max;
 #pragma omp parallel for num_threads(nt) schedule(static)
@@ -736,5 +751,8 @@ int oracle_dsa_scores_fp8(const uint16_t* qI, const float* w, const uint8_t* cod
         }
         scores[u] = acc;
     }
+    free(qc);
+    free(qs);
+    free(qd);
     return 0;
 }

@@ -16,9 +16,9 @@ quantiser to things other than itself:
   * the error bound: |dequant - x| <= (half an E4M3 spacing at x/s + the fp32
     division's rounding) * s;
   * the absmax element mapping to +-448, an all-zero group giving scale 0;
-  * the FP8 indexer scores equal the bf16 indexer formula on the dequantised
-    keys (through the separate fp64 key path), and with lossless keys equal the
-    bf16 oracle's scores exactly.
+  * the FP8 indexer scores equal the indexer formula on the dequantised query
+    heads and keys (the indexer's product runs on E4M3 operands), and with
+    lossless operands equal the bf16 oracle's scores exactly.
 """
 import os
 
@@ -152,7 +152,7 @@ def test_zero_group_and_layout():
     assert np.array_equal(un[:, :512], oracle.dequant_fp8(codes, scales))
 
 
-def test_fp8_indexer_scores_are_the_indexer_on_dequantised_keys():
+def test_fp8_indexer_scores_are_the_indexer_on_dequantised_operands():
     rng = np.random.default_rng(17)
     B, HI, dI, L = 2, 8, 128, 40
     q = _to_bf16_bits(rng.standard_normal((B, HI, dI)))
@@ -161,17 +161,24 @@ def test_fp8_indexer_scores_are_the_indexer_on_dequantised_keys():
     lens = np.array([L, 23], np.int32)
     codes, ks = oracle.quant_fp8(k)
     got = oracle.dsa_scores_fp8(q, w, codes, ks[..., 0], lens)
-    # the same formula in numpy on the dequantised keys
+    # the same formula in numpy, on the dequantised keys and the dequantised query heads
     kd = oracle.dequant_fp8(codes, ks)
-    qd = oracle.bf16_bits_to_f64(q)
+    qc, qs = oracle.quant_fp8(q)
+    qd = oracle.dequant_fp8(qc, qs)
     ref = np.einsum("bj,btj->bt", w.astype(np.float64), np.maximum(np.einsum("bjd,btd->btj", qd, kd), 0.0))
     for b in range(B):
         assert np.allclose(got[b, :lens[b]], ref[b, :lens[b]], rtol=1e-12, atol=1e-12)
         assert np.all(np.isneginf(got[b, lens[b]:]))
-    # lossless keys (E4M3 values times a power of two): the bf16 oracle's scores exactly
+    # the query is quantised: with its bf16 values the scores differ
+    ref_bf16_q = np.einsum("bj,btj->bt", w.astype(np.float64),
+                           np.maximum(np.einsum("bjd,btd->btj", oracle.bf16_bits_to_f64(q), kd), 0.0))
+    assert not np.allclose(got[0], ref_bf16_q[0], rtol=1e-6)
+    # lossless operands (E4M3 values times a power of two): the bf16 oracle's scores exactly
     kc = rng.integers(0, 0x7F, size=(B, L, dI)).astype(np.uint8)
     kc[..., 0] = 0x7E
-    kx = (oracle.e4m3_value(kc) * 2.0 ** -4).astype(np.float32)
-    kb = _bits(kx)
+    kb = _bits((oracle.e4m3_value(kc) * 2.0 ** -4).astype(np.float32))
+    qcl = rng.integers(0, 0xFF, size=(B, HI, dI)).astype(np.uint8) & 0xF7  # no NaN codes
+    qcl[..., 5] = 0x7E
+    qb = _bits((oracle.e4m3_value(qcl) * 2.0 ** 3).astype(np.float32))
     c2, s2 = oracle.quant_fp8(kb)
-    assert np.array_equal(oracle.dsa_scores_fp8(q, w, c2, s2[..., 0], lens), oracle.dsa_scores(q, w, kb, lens))
+    assert np.array_equal(oracle.dsa_scores_fp8(qb, w, c2, s2[..., 0], lens), oracle.dsa_scores(qb, w, kb, lens))
