@@ -336,6 +336,13 @@ int attn_prefill_causal_window(const kvattn_bf16* q, const kvattn_bf16* k, const
  * listed in increasing index order; min(k, len) entries, then -1.  The
  * selection is made on the fp32 scores the kernel computed; scores_out
  * [B][L_max] fp32 receives them (-inf past each length) when non-NULL.
+ * workspace: dsa_index_topk_workspace_bytes(...) bytes, 256-byte aligned, always
+ * required.  Its first 8 KiB per row (B * 2048 counters, the histogram of the top-k's
+ * first radix digit, which the indexer fills as it scores and the top-k reads instead
+ * of a pass of its own) must be zero before the first call on the workspace
+ * (cudaMemsetAsync once); every call leaves them zero, except one that sets
+ * KVATTN_STATUS_TIMEOUT.  The rest (the scores, when scores_out is NULL) needs no
+ * initialisation.  Calls that share a workspace must be ordered.
  * Supported: H_I = 64, d_I = 128, 1 <= k <= 2048, 1 <= L_max <= 131072.
  */
 size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k);
@@ -383,7 +390,12 @@ int dsa_topk_merge(const float* cand_scores, const int32_t* cand_idx, int n_part
  * (-1 = unused slot; other values outside [0, L_max) are skipped and set
  * KVATTN_STATUS_BAD_INDEX).  out [B][Hq][Dv] bf16; lse [B][Hq] fp32 or NULL.
  * A row with no valid index gives out = 0, lse = -inf.
- * Supported: Dk = 576, Dv = 512, Hq in {64, 128}, 1 <= k <= 2048.
+ * workspace: attn_decode_sparse_workspace_bytes(...) bytes (0 when k <= 128),
+ * 256-byte aligned; its first 8 * B bytes hold per-row counters that must be zero
+ * before the first call on the workspace (cudaMemsetAsync once) -- every call leaves
+ * them zero, except one that sets KVATTN_STATUS_TIMEOUT -- and the rest needs no
+ * initialisation.  Calls that share a workspace must be ordered.
+ * Supported: Dk = 576, Dv = 512, Hq in {64, 128}, 1 <= k <= 2048, B <= 65535.
  */
 size_t attn_decode_sparse_workspace_bytes(int B, int Hq, int Dv, int k);
 
@@ -426,13 +438,15 @@ int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const in
 int latent_quant_fp8(const kvattn_bf16* latent, long long n_rows, uint8_t* packed, void* stream);
 
 /*
- * dsa_index_topk on FP8 indexer keys (idx_key_quant_fp8): k_codes [B][L_max][128]
- * uint8, k_scales [B][L_max] fp32.  The scores are s_{b,t} = k_scales[b][t] *
- * sum_j w[b][j] * ReLU(q_idx[b][j] . value(k_codes[b][t])) -- the indexer formula
- * on the dequantised keys, since ReLU commutes with the non-negative scale -- in
- * fp32; the codes are converted to bf16 exactly for the tensor cores.  HBM bytes per
- * token: 132 instead of 256.  Everything else (selection, order, -1 padding,
- * scores_out, workspace, limits) as dsa_index_topk.
+ * dsa_index_topk in fp8 ("Agentic RL 入门3" §2.2 (1): the indexer runs stably in fp8;
+ * its product runs on E4M3 operands): k_codes [B][L_max][128] uint8 and k_scales
+ * [B][L_max] fp32 are the keys (idx_key_quant_fp8); each 128-wide query head
+ * q_idx[b][j] (bf16) is quantised inside the call with the same rule (scale qs_j =
+ * absmax / 448).  The scores are the indexer formula on the dequantised operands,
+ * s_{b,t} = sum_j w[b][j] * ReLU(qhat_j . khat_t) = ks_t * sum_j (w_j qs_j) *
+ * ReLU(qcode_j . kcode_t) (the scales are >= 0), the code products exact and summed
+ * in fp32 on the tensor cores.  HBM bytes per token: 132 instead of 256.  Everything
+ * else (selection, order, -1 padding, scores_out, workspace, limits) as dsa_index_topk.
  */
 int dsa_index_topk_fp8(const kvattn_bf16* q_idx, const float* w, const uint8_t* k_codes,
                        const float* k_scales, const int32_t* seq_lens, int B, int n_idx_head,
@@ -486,7 +500,8 @@ int qsa_block_keys(const kvattn_bf16* k_idx, const int32_t* seq_lens, const int3
  * selected token positions in increasing order, -1 padded; tok_count [B] int32:
  * how many (4 min(L / 4, n_top) + L mod 4).  scores_out [B][L_max / 4] fp32 (the
  * group scores, -inf past each row's groups) or NULL.  workspace:
- * qsa_select_workspace_bytes(...) bytes, 256-byte aligned, no initialisation.
+ * qsa_select_workspace_bytes(...) bytes, 256-byte aligned, with the zero-between-calls
+ * histogram region of dsa_index_topk at its start (zero before the first call).
  * Supported: 64 indexer heads of width 128, L_max a multiple of 4 with
  * L_max / 4 <= 131072, 1 <= n_top <= 2048.
  */

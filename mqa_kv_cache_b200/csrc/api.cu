@@ -584,11 +584,28 @@ int attn_prefill_causal_window(const kvattn_bf16* q, const kvattn_bf16* k, const
                         n_sink, window, stream);
 }
 
+// DSA / QSA selection workspace: [0, hist) the per-row first-digit counts of the top-k
+// (zero between calls), then the scores when the caller keeps none.
+static size_t dsa_ws_hist(int B) { return align_up(kvattn::dsa_hist_bytes(B)); }
+
 size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k)
 {
     (void)k;
     if (B < 1 || L_max < 1) return 0;
-    return align_up(kvattn::dsa_scores_bytes(B, L_max));
+    return dsa_ws_hist(B) + align_up(kvattn::dsa_scores_bytes(B, L_max));
+}
+
+// Checks the selection workspace; on success sets the histogram and the scores buffer.
+static int dsa_ws(const char* name, int B, int L_max, float* scores_out, void* workspace, size_t workspace_bytes,
+                  uint32_t** hist, float** scores)
+{
+    const size_t need = dsa_ws_hist(B) + (scores_out ? 0 : align_up(kvattn::dsa_scores_bytes(B, L_max)));
+    if (!workspace || workspace_bytes < need) return fail(KVATTN_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, need);
+    if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
+        return fail(KVATTN_ERR_ALIGN, "%s: workspace must be 256-byte aligned", name);
+    *hist = static_cast<uint32_t*>(workspace);
+    *scores = scores_out ? scores_out : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dsa_ws_hist(B));
+    return KVATTN_OK;
 }
 
 int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* k_idx, const int32_t* seq_lens, int B,
@@ -608,22 +625,17 @@ int dsa_index_topk(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* 
     if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(topk_idx) ||
         (scores_out && !aligned16(scores_out)))
         return fail(KVATTN_ERR_ALIGN, "dsa_index_topk: tensors must be 16-byte aligned");
-    float* scores = scores_out;
-    if (!scores) {
-        const size_t need = align_up(kvattn::dsa_scores_bytes(B, L_max));
-        if (!workspace || workspace_bytes < need)
-            return fail(KVATTN_ERR_WORKSPACE, "dsa_index_topk: workspace needs %zu bytes when scores_out is NULL",
-                        need);
-        if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
-            return fail(KVATTN_ERR_ALIGN, "dsa_index_topk: workspace must be 256-byte aligned");
-        scores = static_cast<float*>(workspace);
-    }
+    float* scores = nullptr;
+    uint32_t* hist = nullptr;
+    const int ws_rc = dsa_ws("dsa_index_topk", B, L_max, scores_out, workspace, workspace_bytes, &hist, &scores);
+    if (ws_rc != KVATTN_OK) return ws_rc;
     int sms = 0;
     if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "dsa_index_topk: no CUDA device");
     CUtensorMap tm_k, tm_q;
     if (make_map_3d(&tm_k, k_idx, 128, L_max, B, 128) != KVATTN_OK) return KVATTN_ERR_CUDA;
     if (make_map_3d(&tm_q, q_idx, 128, 64, B, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
     kvattn::DsaIndexArgs a{w, seq_lens, scores, topk_idx, dev_status, B, L_max, k, sms};
+    a.hist = hist;
     return cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, static_cast<cudaStream_t>(stream)),
                        "dsa_index_topk launch");
 }
@@ -645,16 +657,10 @@ int dsa_index_topk_fp8(const kvattn_bf16* q_idx, const float* w, const uint8_t* 
     if (!aligned16(q_idx) || !aligned16(k_codes) || !aligned16(w) || !aligned16(topk_idx) ||
         (reinterpret_cast<uintptr_t>(k_scales) & 3) || (scores_out && !aligned16(scores_out)))
         return fail(KVATTN_ERR_ALIGN, "dsa_index_topk_fp8: tensors must be 16-byte aligned (scales 4)");
-    float* scores = scores_out;
-    if (!scores) {
-        const size_t need = align_up(kvattn::dsa_scores_bytes(B, L_max));
-        if (!workspace || workspace_bytes < need)
-            return fail(KVATTN_ERR_WORKSPACE, "dsa_index_topk_fp8: workspace needs %zu bytes when scores_out is NULL",
-                        need);
-        if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
-            return fail(KVATTN_ERR_ALIGN, "dsa_index_topk_fp8: workspace must be 256-byte aligned");
-        scores = static_cast<float*>(workspace);
-    }
+    float* scores = nullptr;
+    uint32_t* hist = nullptr;
+    const int ws_rc = dsa_ws("dsa_index_topk_fp8", B, L_max, scores_out, workspace, workspace_bytes, &hist, &scores);
+    if (ws_rc != KVATTN_OK) return ws_rc;
     int sms = 0;
     if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "dsa_index_topk_fp8: no CUDA device");
     CUtensorMap tm_k, tm_q;
@@ -663,6 +669,8 @@ int dsa_index_topk_fp8(const kvattn_bf16* q_idx, const float* w, const uint8_t* 
     if (make_map_3d(&tm_q, q_idx, 128, 64, B, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
     kvattn::DsaIndexArgs a{w, seq_lens, scores, topk_idx, dev_status, B, L_max, k, sms};
     a.kscale = k_scales;
+    a.q_idx = q_idx;
+    a.hist = hist;
     return cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, static_cast<cudaStream_t>(stream)),
                        "dsa_index_topk_fp8 launch");
 }
@@ -733,12 +741,11 @@ int qsa_block_keys(const kvattn_bf16* k_idx, const int32_t* seq_lens, const int3
     return cuda_status(kvattn::launch_qsa_block_keys(a, static_cast<cudaStream_t>(stream)), "qsa_block_keys launch");
 }
 
-static size_t qsa_scores_bytes(int B, int L_max) { return align_up(kvattn::dsa_scores_bytes(B, L_max / kvattn::QSA_BLOCK)); }
 size_t qsa_select_workspace_bytes(int B, int L_max, int n_top)
 {
     if (B < 1 || L_max < kvattn::QSA_BLOCK || n_top < 1) return 0;
     (void)n_top;
-    return qsa_scores_bytes(B, L_max);
+    return dsa_ws_hist(B) + align_up(kvattn::dsa_scores_bytes(B, L_max / kvattn::QSA_BLOCK));
 }
 
 int qsa_select(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* block_keys, const int32_t* seq_lens, int B,
@@ -759,13 +766,10 @@ int qsa_select(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* bloc
     if (!aligned16(q_idx) || !aligned16(block_keys) || !aligned16(w) || !aligned16(tok_idx) ||
         (scores_out && !aligned16(scores_out)))
         return fail(KVATTN_ERR_ALIGN, "qsa_select: tensors must be 16-byte aligned");
-    const size_t need = qsa_select_workspace_bytes(B, L_max, n_top);
-    if (!workspace || workspace_bytes < need)
-        return fail(KVATTN_ERR_WORKSPACE, "qsa_select: workspace needs %zu bytes", need);
-    if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
-        return fail(KVATTN_ERR_ALIGN, "qsa_select: workspace must be 256-byte aligned");
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
-    float* scores = scores_out ? scores_out : reinterpret_cast<float*>(ws);
+    float* scores = nullptr;
+    uint32_t* hist = nullptr;
+    const int ws_rc = dsa_ws("qsa_select", B, nb_max, scores_out, workspace, workspace_bytes, &hist, &scores);
+    if (ws_rc != KVATTN_OK) return ws_rc;
     int sms = 0;
     if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "qsa_select: no CUDA device");
     CUtensorMap tm_k, tm_q;
@@ -774,6 +778,7 @@ int qsa_select(const kvattn_bf16* q_idx, const float* w, const kvattn_bf16* bloc
     kvattn::DsaIndexArgs a{w, seq_lens, scores, nullptr, dev_status, B, nb_max, n_top, sms};
     static_assert(kvattn::QSA_BLOCK == 4, "len_shift below is log2 of the group size");
     a.len_shift = 2;  // a row of L tokens has L / 4 complete groups
+    a.hist = hist;
     a.tok_idx = tok_idx;  // the top-k writes the groups' tokens and the tail directly
     a.tok_count = tok_count;
     a.L_tok = L_max;
@@ -809,16 +814,19 @@ static int sparse_call(const char* name, const kvattn_bf16* q, const void* laten
     if (need > 0 && reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
         return fail(KVATTN_ERR_ALIGN, "%s: workspace must be 256-byte aligned", name);
     const int chunks = kvattn::sparse_chunks(k);
+    int sms = 0;
+    if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "%s: no CUDA device", name);
     CUtensorMap tm_q, tm_o;
     if (make_map_3d(&tm_q, q, Dk, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
     if (chunks == 1) {
         if (make_map_3d(&tm_o, out, Dv, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
     } else {
-        if (make_map_3d(&tm_o, workspace, Dv, Hq, static_cast<uint64_t>(B) * chunks, Hq) != KVATTN_OK)
+        const void* parts = static_cast<const uint8_t*>(workspace) + kvattn::sparse_counter_bytes(B);
+        if (make_map_3d(&tm_o, parts, Dv, Hq, static_cast<uint64_t>(B) * chunks, Hq) != KVATTN_OK)
             return KVATTN_ERR_CUDA;
     }
     kvattn::SparseLaunch l{q, latent, topk_idx, out, lse, need > 0 ? workspace : nullptr, dev_status, B, Hq, L_max,
-                           k, scale, fp8};
+                           k, scale, fp8, sms};
     return cuda_status(kvattn::launch_sparse_attn(l, tm_q, tm_o, static_cast<cudaStream_t>(stream)), name);
 }
 

@@ -6,8 +6,8 @@
 // is a [L x 128] x [128 x 64] contraction followed by a ReLU-weighted reduction
 // over the 64 heads, so it runs on the tensor cores: tcgen05.mma with the 128
 // tokens of a tile as M, the 64 heads as N and K = 128, the fp32 accumulator
-// in TMEM (two 64-column buffers so the epilogue of one tile overlaps the MMA
-// of the next), and the head reduction fused into the TMEM read-out.  It is
+// in TMEM (four 64-column buffers so the epilogue of one tile overlaps the MMAs
+// of the next ones), and the head reduction fused into the TMEM read-out.  It is
 // bound by the one read of k_idx from HBM (intensity ~63 FLOP/byte).
 //
 // Top-k (§2.2 (2): S = TopK_t(s_t), ties to the lower index): one cluster of
@@ -30,6 +30,28 @@ namespace {
 
 // ---- indexer ------------------------------------------------------------------
 
+// Order-preserving 32-bit key of an fp32 score (larger score, larger key);
+// -0 is first made +0 so that it ties with +0; NaN maps to 0 (never selected
+// ahead of a number) and is reported.
+__device__ __forceinline__ uint32_t score_key(float f, bool& nan)
+{
+    uint32_t u = __float_as_uint(f);
+    if ((u & 0x7fffffffu) > 0x7f800000u) {
+        nan = true;
+        return 0u;
+    }
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The first radix digit of the top-k (the key's top 11 bits).  The indexers count the
+// digits of every row's valid scores as they produce them (a shared-memory histogram per
+// work item, flushed into a per-row histogram in global memory), so that the top-k starts
+// at its second digit.
+constexpr int TK_DIGITS0 = 2048;
+constexpr int TK_SHIFT0 = 21;
+
+
 constexpr int IX_TOK = 128;   // tokens per tile (MMA M)
 constexpr int IX_HEADS = 64;  // indexer heads (MMA N)
 constexpr int IX_DIM = 128;   // key width (MMA K)
@@ -39,22 +61,28 @@ constexpr int IX_TILE = 2 * IX_BOX;           // k tile [128 x 128] bf16
 constexpr int IX_QBOX = IX_HEADS * 128;       // one 64-column box of q [64 x 64]
 constexpr int IX_QBYTES = 2 * IX_QBOX;
 constexpr int IX_THREADS = 192;               // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 epilogue
-constexpr int IX_TMEM_COLS = 128;             // two 64-column accumulators
+constexpr int IX_NACC = 4;                    // 64-column accumulators in flight (the MMA-to-epilogue
+                                              // round trip is ~1 us: two buffers capped a CTA at a tile
+                                              // per ~0.5 us)
+constexpr int IX_TMEM_COLS = IX_NACC * 64;
 constexpr uint32_t IX_IDESC = umma_idesc_bf16(IX_TOK, IX_HEADS);
 
 constexpr int IX_OFF_Q = IX_STAGES * IX_TILE;
 constexpr int IX_OFF_W = IX_OFF_Q + IX_QBYTES;
-constexpr int IX_OFF_BAR = IX_OFF_W + IX_HEADS * 4;
-// full[S], empty[S], q_full, q_empty, acc_full[2], acc_empty[2], mma_done
-constexpr int IX_NBAR = 2 * IX_STAGES + 7;
+constexpr int IX_OFF_HIST = IX_OFF_W + IX_HEADS * 4;   // [2048] digit counts of the current work item
+constexpr int IX_OFF_BAR = IX_OFF_HIST + 2048 * 4;
+// full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done
+constexpr int IX_NBAR = 2 * IX_STAGES + 3 + 2 * IX_NACC;
 constexpr int IX_OFF_MISC = IX_OFF_BAR + IX_NBAR * 8;
 constexpr int IX_SMEM = IX_OFF_MISC + 32 + 1024;
+static_assert(IX_SMEM <= 232448, "shared memory");
 
 struct IndexerArgs {
     const float* w;
     const int32_t* seq_lens;
     const float* kscale;  // FP8 keys: [B][L_max] fp32 scales (indexer_fp8_kernel only)
     float* scores;
+    uint32_t* hist;       // [B][2048] first-digit counts of the valid scores (added to; zero on entry)
     int32_t* dev_status;
     int B, L_max, tiles_per_b, chunks_per_b;
     int len_shift;  // row b scores seq_lens[b] >> len_shift keys (2: 4-token groups)
@@ -79,9 +107,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     uint64_t* q_full = bars + 2 * IX_STAGES;
     uint64_t* q_empty = q_full + 1;
     uint64_t* acc_full = q_full + 2;
-    uint64_t* acc_empty = q_full + 4;
-    uint64_t* mma_done = q_full + 6;
+    uint64_t* acc_empty = acc_full + IX_NACC;
+    uint64_t* mma_done = acc_empty + IX_NACC;
     float* s_w = reinterpret_cast<float*>(smem + IX_OFF_W);
+    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + IX_OFF_HIST);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + IX_OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + IX_OFF_MISC + 4);
 
@@ -95,7 +124,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         }
         mbar_init(q_full, 1);
         mbar_init(q_empty, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < IX_NACC; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 4);
         }
@@ -162,9 +191,9 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 }
                 for (int t = t0; t < t1; ++t, ++it, ++tc) {
                     const int s = it % IX_STAGES;
-                    const int buf = tc & 1;
+                    const int buf = tc % IX_NACC;
                     if (*s_abort || !mbar_wait(&full[s], (it / IX_STAGES) & 1) ||
-                        (tc >= 2 && !mbar_wait(&acc_empty[buf], ((tc >> 1) - 1) & 1))) {
+                        (tc >= IX_NACC && !mbar_wait(&acc_empty[buf], ((tc / IX_NACC) - 1) & 1))) {
                         *s_abort = 1;
                         break;
                     }
@@ -193,6 +222,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         const int quarter = warp & 3;  // TMEM lanes this warp may read
         const int row = quarter * 32 + lane;
         const int ep = threadIdx.x - 64;
+        for (int i = ep; i < TK_DIGITS0; i += 128) s_hist[i] = 0u;  // ordered by the item's first barrier
         int tc = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
             int b, t0, t1;
@@ -205,10 +235,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
             named_bar_sync(2, 128);
             float* out = a.scores + static_cast<long long>(b) * a.L_max;
             for (int t = t0; t < t1; ++t, ++tc) {
-                const int buf = tc & 1;
+                const int buf = tc % IX_NACC;
                 // on an abort the loops still run to the end (without waiting or
                 // working) so that all four warps meet at the same named barriers
-                if (!warp_wait(&acc_full[buf], (tc >> 1) & 1, s_abort)) continue;
+                if (!warp_wait(&acc_full[buf], (tc / IX_NACC) & 1, s_abort)) continue;
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_HEADS;
                 uint32_t v0[32], v1[32];
@@ -226,6 +256,23 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 const int tok = t * IX_TOK + row;
                 if (acc != acc) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
                 if (tok < a.L_max) out[tok] = tok < len ? acc : -INFINITY;
+                // the score's first top-k digit, counted once per warp and digit
+                const bool in = a.hist != nullptr && tok < len;
+                bool nan_key = false;
+                const uint32_t digit = in ? score_key(acc, nan_key) >> TK_SHIFT0 : 0xffffffffu;
+                const uint32_t same = __match_any_sync(0xffffffffu, digit);
+                if (in && lane == __ffs(same) - 1) atomicAdd(&s_hist[digit], static_cast<uint32_t>(__popc(same)));
+            }
+            if (a.hist) {  // the item's counts into the row's histogram; the shared one back to zero
+                named_bar_sync(2, 128);
+                uint32_t* gh = a.hist + static_cast<long long>(b) * TK_DIGITS0;
+                for (int i = ep; i < TK_DIGITS0; i += 128) {
+                    const uint32_t v = s_hist[i];
+                    if (v) {
+                        atomicAdd(gh + i, v);
+                        s_hist[i] = 0u;
+                    }
+                }
             }
         }
     }
@@ -237,66 +284,66 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     }
 }
 
-// ---- indexer on FP8 keys -------------------------------------------------------------
+// ---- indexer in fp8 ------------------------------------------------------------------
 // "稀疏注意力：省了什么，没省什么", 改进一 (an indexer key of about 132 bytes: 128 E4M3
 // codes and one fp32 scale) and "Agentic RL 入门3" §2.2 (1) (the indexer runs stably in
-// fp8).  With k_t = scale_t * code_t and scale_t >= 0, ReLU(q . k_t) = scale_t *
-// ReLU(q . code_t), so s_t = scale_t * sum_j w_j ReLU(q_j . code_t): the codes enter
-// the MMA unscaled (E4M3 -> bf16 is exact) and the scale multiplies the score.
-// 320 threads: w0 TMA of 16 KB code tiles (128-byte swizzle) into a 6-slot ring,
-// w1 MMA issuer + TMEM owner, w2-5 epilogue, w6-9 convert each code tile into a
-// bf16 tile (two 64-column SW128 blocks) of a 3-slot ring.  HBM bytes per token:
-// 128 + 4 (against 256 for bf16 keys).
-constexpr int IX8_RAW = IX_TOK * 128;            // 16 KB code tile [128 tokens][128 codes]
-constexpr int IX8_RSTAGES = 6, IX8_BSTAGES = 3;
-constexpr int IX8_THREADS = 320;
-constexpr int IX8_OFF_RAW = 0;
-constexpr int IX8_OFF_BF = IX8_OFF_RAW + IX8_RSTAGES * IX8_RAW;
-constexpr int IX8_OFF_Q = IX8_OFF_BF + IX8_BSTAGES * IX_TILE;
-constexpr int IX8_OFF_W = IX8_OFF_Q + IX_QBYTES;
-constexpr int IX8_OFF_BAR = IX8_OFF_W + IX_HEADS * 4;
-// raw_full[R], raw_empty[R], bf_full[S], bf_empty[S], q_full, q_empty, acc_full[2], acc_empty[2], mma_done
-constexpr int IX8_NBAR = 2 * IX8_RSTAGES + 2 * IX8_BSTAGES + 7;
+// fp8): the product runs on E4M3 operands.  The 64 query heads of a row are quantised
+// here with the keys' rule (one fp32 scale per 128-wide head, RNE, saturating) into the
+// MMA's B operand; the code tiles land by TMA in the A operand's layout and go to
+// tcgen05.mma kind::f8f6f4 unconverted (M = 128 tokens, N = 64 heads, K = 128 in four
+// K = 32 steps, exact products, fp32 accumulation).  With scales >= 0, ReLU(qhat .
+// khat) = qs_j ks_t ReLU(qc_j . kc_t), so the epilogue folds the head scale into the
+// head weight and multiplies the sum by the key's scale.  HBM bytes per token: 128 + 4.
+constexpr int IX8_TILE = IX_TOK * 128;           // 16 KB code tile [128 tokens][128 codes]
+constexpr int IX8_STAGES = 12;
+constexpr int IX8_QBYTES = IX_HEADS * 128;        // [64 heads][128 codes]
+constexpr int IX8_OFF_Q = IX8_STAGES * IX8_TILE;
+constexpr int IX8_OFF_W = IX8_OFF_Q + IX8_QBYTES;
+constexpr int IX8_OFF_HIST = IX8_OFF_W + IX_HEADS * 4;
+constexpr int IX8_OFF_BAR = IX8_OFF_HIST + 2048 * 4;
+// full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done
+constexpr int IX8_NBAR = 2 * IX8_STAGES + 3 + 2 * IX_NACC;
 constexpr int IX8_OFF_MISC = IX8_OFF_BAR + IX8_NBAR * 8;
 constexpr int IX8_SMEM = IX8_OFF_MISC + 32 + 1024;
 static_assert(IX8_SMEM <= 232448, "shared memory");
+// D fp32, A and B E4M3 (format 0 of kind::f8f6f4), both K-major, M x N
+constexpr uint32_t IX8_IDESC = (1u << 4) | (static_cast<uint32_t>(IX_HEADS >> 3) << 17) |
+                               (static_cast<uint32_t>(IX_TOK >> 4) << 24);
 
-// Sixteen E4M3 codes -> sixteen bf16 (two 16-byte chunks), exactly.
-__device__ __forceinline__ void codes16_to_bf16(uint4 c, uint4& lo, uint4& hi)
+__device__ __forceinline__ void tc_mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
 {
-    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            uint32_t h2;
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(w[i] >> (16 * hf))));
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
-            o[2 * i + hf] = pack_bf16x2(f.x, f.y);
-        }
-    }
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
-__global__ void __launch_bounds__(IX8_THREADS, 1)
-    indexer_fp8_kernel(const __grid_constant__ CUtensorMap tm_k8, const __grid_constant__ CUtensorMap tm_q,
+// Two fp32 -> two E4M3 codes (lo in the low byte), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t ix_e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__global__ void __launch_bounds__(IX_THREADS, 1)
+    indexer_fp8_kernel(const __grid_constant__ CUtensorMap tm_k8, const kvattn_bf16* __restrict__ q_idx,
                        IndexerArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + IX8_OFF_BAR);
-    uint64_t* raw_full = bars;
-    uint64_t* raw_empty = raw_full + IX8_RSTAGES;
-    uint64_t* bf_full = raw_empty + IX8_RSTAGES;
-    uint64_t* bf_empty = bf_full + IX8_BSTAGES;
-    uint64_t* q_full = bf_empty + IX8_BSTAGES;
+    uint64_t* full = bars;
+    uint64_t* empty = bars + IX8_STAGES;
+    uint64_t* q_full = bars + 2 * IX8_STAGES;
     uint64_t* q_empty = q_full + 1;
     uint64_t* acc_full = q_full + 2;
-    uint64_t* acc_empty = q_full + 4;
-    uint64_t* mma_done = q_full + 6;
+    uint64_t* acc_empty = acc_full + IX_NACC;
+    uint64_t* mma_done = acc_empty + IX_NACC;
     float* s_w = reinterpret_cast<float*>(smem + IX8_OFF_W);
+    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + IX8_OFF_HIST);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + IX8_OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + IX8_OFF_MISC + 4);
 
@@ -304,17 +351,13 @@ __global__ void __launch_bounds__(IX8_THREADS, 1)
     const int n_items = a.B * a.chunks_per_b;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < IX8_RSTAGES; ++s) {
-            mbar_init(&raw_full[s], 1);
-            mbar_init(&raw_empty[s], 4);
+        for (int s = 0; s < IX8_STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
-        for (int s = 0; s < IX8_BSTAGES; ++s) {
-            mbar_init(&bf_full[s], 4);
-            mbar_init(&bf_empty[s], 1);
-        }
-        mbar_init(q_full, 1);
+        mbar_init(q_full, 4);
         mbar_init(q_empty, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < IX_NACC; ++i) {
             mbar_init(&acc_full[i], 1);
             mbar_init(&acc_empty[i], 4);
         }
@@ -322,10 +365,7 @@ __global__ void __launch_bounds__(IX8_THREADS, 1)
         *s_abort = 0;
         fence_barrier_init();
     }
-    if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tm_k8);
-        tma_prefetch_desc(&tm_q);
-    }
+    if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_k8);
     if (warp == 1) {
         tmem_alloc(s_tmem, IX_TMEM_COLS);
         tmem_relinquish();
@@ -338,32 +378,25 @@ __global__ void __launch_bounds__(IX8_THREADS, 1)
     pdl_trigger();
 
     if (warp == 0) {
-        // ===== TMA producer: query, then code tiles =====
+        // ===== TMA producer: code tiles =====
         if (lane == 0) {
-            int it = 0, n = 0;
-            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
+            int it = 0;
+            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x) {
                 int b, t0, t1;
                 ix_item(a, item, b, t0, t1);
-                if (n > 0 && !mbar_wait(q_empty, (n - 1) & 1)) {
-                    *s_abort = 1;
-                    break;
-                }
-                mbar_arrive_expect_tx(q_full, IX_QBYTES);
-                tma_load_3d(smem + IX8_OFF_Q, &tm_q, q_full, 0, 0, b);
-                tma_load_3d(smem + IX8_OFF_Q + IX_QBOX, &tm_q, q_full, 64, 0, b);
                 for (int t = t0; t < t1; ++t, ++it) {
-                    const int s = it % IX8_RSTAGES;
-                    if (it >= IX8_RSTAGES && (*s_abort || !mbar_wait(&raw_empty[s], ((it / IX8_RSTAGES) - 1) & 1))) {
+                    const int s = it % IX8_STAGES;
+                    if (it >= IX8_STAGES && (*s_abort || !mbar_wait(&empty[s], ((it / IX8_STAGES) - 1) & 1))) {
                         *s_abort = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(&raw_full[s], IX8_RAW);
-                    tma_load_3d(smem + IX8_OFF_RAW + s * IX8_RAW, &tm_k8, &raw_full[s], 0, t * IX_TOK, b);
+                    mbar_arrive_expect_tx(&full[s], IX8_TILE);
+                    tma_load_3d(smem + s * IX8_TILE, &tm_k8, &full[s], 0, t * IX_TOK, b);
                 }
             }
             if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
-            for (int j = it - IX8_RSTAGES > 0 ? it - IX8_RSTAGES : 0; j < it; ++j)
-                mbar_wait(&raw_full[j % IX8_RSTAGES], (j / IX8_RSTAGES) & 1);
+            for (int j = it - IX8_STAGES > 0 ? it - IX8_STAGES : 0; j < it; ++j)
+                mbar_wait(&full[j % IX8_STAGES], (j / IX8_STAGES) & 1);
         }
     } else if (warp == 1) {
         // ===== MMA issuer (one thread) =====
@@ -378,24 +411,21 @@ __global__ void __launch_bounds__(IX8_THREADS, 1)
                     break;
                 }
                 for (int t = t0; t < t1; ++t, ++it) {
-                    const int s = it % IX8_BSTAGES;
-                    const int buf = it & 1;
-                    if (*s_abort || !mbar_wait(&bf_full[s], (it / IX8_BSTAGES) & 1) ||
-                        (it >= 2 && !mbar_wait(&acc_empty[buf], ((it >> 1) - 1) & 1))) {
+                    const int s = it % IX8_STAGES;
+                    const int buf = it % IX_NACC;
+                    if (*s_abort || !mbar_wait(&full[s], (it / IX8_STAGES) & 1) ||
+                        (it >= IX_NACC && !mbar_wait(&acc_empty[buf], ((it / IX_NACC) - 1) & 1))) {
                         *s_abort = 1;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + IX8_OFF_BF + s * IX_TILE);
+                    const uint32_t k_addr = smem_u32(smem + s * IX8_TILE);
                     const uint32_t d_addr = tmem + buf * IX_HEADS;
 #pragma unroll
-                    for (int ks = 0; ks < IX_DIM / 16; ++ks) {
-                        const uint32_t off = (ks & 3) * 32;
-                        const uint64_t ad = umma_desc_k_sw128(k_addr + (ks >> 2) * IX_BOX + off);
-                        const uint64_t bd = umma_desc_k_sw128(q_addr + (ks >> 2) * IX_QBOX + off);
-                        tc_mma_bf16(d_addr, ad, bd, IX_IDESC, ks > 0 ? 1u : 0u);
-                    }
-                    tc_commit(&bf_empty[s]);
+                    for (int ks = 0; ks < 4; ++ks)  // K = 32 codes (32 bytes of the 128-byte row) per step
+                        tc_mma_f8(d_addr, umma_desc_k_sw128(k_addr + ks * 32), umma_desc_k_sw128(q_addr + ks * 32),
+                                  IX8_IDESC, ks > 0 ? 1u : 0u);
+                    tc_commit(&empty[s]);
                     tc_commit(&acc_full[buf]);
                 }
                 tc_commit(q_empty);
@@ -404,60 +434,75 @@ __global__ void __launch_bounds__(IX8_THREADS, 1)
             mbar_wait(mma_done, 0);
             if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
         }
-    } else if (warp >= 6) {
-        // ===== converters: code tile -> bf16 tile; thread r takes token row r =====
-        const int r = threadIdx.x - 192;
-        int it = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-            int b, t0, t1;
-            ix_item(a, item, b, t0, t1);
-            for (int t = t0; t < t1; ++t, ++it) {
-                const int rs = it % IX8_RSTAGES, bs = it % IX8_BSTAGES;
-                if (!warp_wait(&raw_full[rs], (it / IX8_RSTAGES) & 1, s_abort)) continue;
-                const uint8_t* src = smem + IX8_OFF_RAW + rs * IX8_RAW + r * 128;
-                uint4 c[8];
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    c[ch] = *reinterpret_cast<const uint4*>(src + ((ch ^ (r & 7)) << 4));  // TMA 128-byte swizzle
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&raw_empty[rs]);
-                if (it >= IX8_BSTAGES && !warp_wait(&bf_empty[bs], ((it / IX8_BSTAGES) - 1) & 1, s_abort)) continue;
-                uint8_t* dst = smem + IX8_OFF_BF + bs * IX_TILE;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {  // codes 16 ch .. 16 ch + 15 = bf16 chunks 2 ch, 2 ch + 1
-                    uint4 lo, hi;
-                    codes16_to_bf16(c[ch], lo, hi);
-                    uint8_t* blk = dst + (ch >> 2) * IX_BOX;
-                    *reinterpret_cast<uint4*>(blk + swz128(r, (2 * ch) & 7)) = lo;
-                    *reinterpret_cast<uint4*>(blk + swz128(r, (2 * ch + 1) & 7)) = hi;
-                }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bf_full[bs]);
-            }
-        }
     } else {
-        // ===== epilogue: TMEM -> ReLU, weight, sum over heads, times the key's scale =====
+        // ===== epilogue (and, per item, the query heads' quantisation) =====
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
         const int ep = threadIdx.x - 64;
-        int tc = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int qh = ep >> 1, qhalf = ep & 1;  // quantisation: head qh, values 64 qhalf .. + 63
+        for (int i = ep; i < TK_DIGITS0; i += 128) s_hist[i] = 0u;  // ordered by the item's first barrier
+        int tc = 0, n = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
             int b, t0, t1;
             ix_item(a, item, b, t0, t1);
             const int len_raw = a.seq_lens ? (a.seq_lens[b] >> a.len_shift) : a.L_max;
             const int len = min(max(len_raw, 0), a.L_max);
             if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
-            named_bar_sync(2, 128);
-            if (ep < IX_HEADS) s_w[ep] = a.w[static_cast<long long>(b) * IX_HEADS + ep];
-            named_bar_sync(2, 128);
+            named_bar_sync(2, 128);  // the previous item's epilogue has read s_w
+            // the previous item's MMAs have read the query tile
+            const bool q_free = n == 0 || warp_wait(q_empty, (n - 1) & 1, s_abort);
+            {
+                const uint4* src = reinterpret_cast<const uint4*>(q_idx + (static_cast<long long>(b) * IX_HEADS + qh) * IX_DIM +
+                                                                  64 * qhalf);
+                uint4 x[8];
+                float amax = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    x[i] = __ldg(src + i);
+                    const uint32_t w4[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w4[e])), fabsf(bf16_hi(w4[e]))));
+                }
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+                const float qs = __fdiv_rn(amax, 448.f);
+                uint8_t* qrow = smem + IX8_OFF_Q;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {  // 16 codes = one 16-byte chunk of the head's 128-byte row
+                    uint32_t wd[4];
+#pragma unroll
+                    for (int hw = 0; hw < 2; ++hw) {
+                        const uint4 v = x[2 * c + hw];
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                        uint32_t pk[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const uint32_t lo = qs == 0.f ? 0u
+                                                          : ix_e4m3x2(__fdiv_rn(bf16_lo(w4[2 * e]), qs),
+                                                                      __fdiv_rn(bf16_hi(w4[2 * e]), qs));
+                            const uint32_t hi = qs == 0.f ? 0u
+                                                          : ix_e4m3x2(__fdiv_rn(bf16_lo(w4[2 * e + 1]), qs),
+                                                                      __fdiv_rn(bf16_hi(w4[2 * e + 1]), qs));
+                            pk[e] = lo | (hi << 16);
+                        }
+                        wd[2 * hw] = pk[0];
+                        wd[2 * hw + 1] = pk[1];
+                    }
+                    if (q_free)
+                        *reinterpret_cast<uint4*>(qrow + swz128(qh, 4 * qhalf + c)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+                }
+                if (qhalf == 0) s_w[qh] = a.w[static_cast<long long>(b) * IX_HEADS + qh] * qs;
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0 && q_free) mbar_arrive(q_full);
+            named_bar_sync(2, 128);  // s_w complete
             float* out = a.scores + static_cast<long long>(b) * a.L_max;
             const float* ks = a.kscale + static_cast<long long>(b) * a.L_max;
             for (int t = t0; t < t1; ++t, ++tc) {
-                const int buf = tc & 1;
+                const int buf = tc % IX_NACC;
                 const int tok = t * IX_TOK + row;
                 const float kscale = tok < a.L_max ? __ldg(ks + tok) : 0.f;
-                if (!warp_wait(&acc_full[buf], (tc >> 1) & 1, s_abort)) continue;
+                if (!warp_wait(&acc_full[buf], (tc / IX_NACC) & 1, s_abort)) continue;
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_HEADS;
                 uint32_t v0[32], v1[32];
@@ -477,6 +522,23 @@ __global__ void __launch_bounds__(IX8_THREADS, 1)
                 acc *= kscale;
                 if (acc != acc) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
                 if (tok < a.L_max) out[tok] = tok < len ? acc : -INFINITY;
+                // the score's first top-k digit, counted once per warp and digit
+                const bool in = a.hist != nullptr && tok < len;
+                bool nan_key = false;
+                const uint32_t digit = in ? score_key(acc, nan_key) >> TK_SHIFT0 : 0xffffffffu;
+                const uint32_t same = __match_any_sync(0xffffffffu, digit);
+                if (in && lane == __ffs(same) - 1) atomicAdd(&s_hist[digit], static_cast<uint32_t>(__popc(same)));
+            }
+            if (a.hist) {  // the item's counts into the row's histogram; the shared one back to zero
+                named_bar_sync(2, 128);
+                uint32_t* gh = a.hist + static_cast<long long>(b) * TK_DIGITS0;
+                for (int i = ep; i < TK_DIGITS0; i += 128) {
+                    const uint32_t v = s_hist[i];
+                    if (v) {
+                        atomicAdd(gh + i, v);
+                        s_hist[i] = 0u;
+                    }
+                }
             }
         }
     }
@@ -492,20 +554,6 @@ __global__ void __launch_bounds__(IX8_THREADS, 1)
 
 constexpr int TK_CL = 8;  // CTAs per batch row (one cluster)
 constexpr int TK_THREADS = 1024;
-
-// Order-preserving 32-bit key of an fp32 score (larger score, larger key);
-// -0 is first made +0 so that it ties with +0; NaN maps to 0 (never selected
-// ahead of a number) and is reported.
-__device__ __forceinline__ uint32_t score_key(float f, bool& nan)
-{
-    uint32_t u = __float_as_uint(f);
-    if ((u & 0x7fffffffu) > 0x7f800000u) {
-        nan = true;
-        return 0u;
-    }
-    if (u == 0x80000000u) u = 0u;
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // Block-wide inclusive scan (sum) of one value per thread; TK_THREADS threads.
 __device__ __forceinline__ int block_incl_scan(int v, int* s_warp)
@@ -536,6 +584,7 @@ __device__ __forceinline__ int block_incl_scan(int v, int* s_warp)
 struct TopkArgs {
     const float* scores;
     const int32_t* seq_lens;
+    uint32_t* hist;      // [B][2048] first-digit counts from the indexer (zeroed here after use), or null
     int32_t* out;
     int32_t* dev_status;
     int L_max, k;
@@ -594,28 +643,36 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
             // pass p - 2, before they reached pass p - 1's cluster barrier, which this CTA has passed:
             // one cluster barrier per pass suffices.
             uint32_t* hist = hist2[p & 1];
-            for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
-            __syncthreads();
-            // scores bunch into few top digits: lanes with equal digits add once per warp
-            for (int base = 0; base < n_mine; base += TK_THREADS) {
-                const int i = base + tid;
-                const uint32_t key = i < n_mine ? s_keys[kpad(i)] : 0u;
-                const bool in = i < n_mine && (key & known) == prefix;
-                const uint32_t digit = in ? (key >> sh) & (nb - 1) : 0xffffffffu;
-                const uint32_t same = __match_any_sync(0xffffffffu, digit);
-                if (in && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[digit], static_cast<uint32_t>(__popc(same)));
-            }
-            cluster.sync();
-            // every CTA sums the cluster's histograms and finds the digit itself:
-            // thread t owns digits nb-1-2t and nb-2-2t (largest first)
             const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
             int c0 = 0, c1 = 0;
-            if (d0 >= 0) {
+            if (p == 0 && a.hist) {
+                // the indexer counted the first digits of the row: every CTA reads them
+                const uint32_t* gh = a.hist + static_cast<long long>(row) * TK_DIGITS0;
+                if (d0 >= 0) c0 = static_cast<int>(__ldcg(gh + d0));
+                if (d1 >= 0) c1 = static_cast<int>(__ldcg(gh + d1));
+            } else {
+                for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
+                __syncthreads();
+                // scores bunch into few top digits: lanes with equal digits add once per warp
+                for (int base = 0; base < n_mine; base += TK_THREADS) {
+                    const int i = base + tid;
+                    const uint32_t key = i < n_mine ? s_keys[kpad(i)] : 0u;
+                    const bool in = i < n_mine && (key & known) == prefix;
+                    const uint32_t digit = in ? (key >> sh) & (nb - 1) : 0xffffffffu;
+                    const uint32_t same = __match_any_sync(0xffffffffu, digit);
+                    if (in && (tid & 31) == __ffs(same) - 1)
+                        atomicAdd(&hist[digit], static_cast<uint32_t>(__popc(same)));
+                }
+                cluster.sync();
+                // every CTA sums the cluster's histograms and finds the digit itself:
+                // thread t owns digits nb-1-2t and nb-2-2t (largest first)
+                if (d0 >= 0) {
 #pragma unroll
-                for (int q = 0; q < TK_CL; ++q) {
-                    const uint32_t* hq = cluster.map_shared_rank(hist, q);
-                    c0 += static_cast<int>(hq[d0]);
-                    if (d1 >= 0) c1 += static_cast<int>(hq[d1]);
+                    for (int q = 0; q < TK_CL; ++q) {
+                        const uint32_t* hq = cluster.map_shared_rank(hist, q);
+                        c0 += static_cast<int>(hq[d0]);
+                        if (d1 >= 0) c1 += static_cast<int>(hq[d1]);
+                    }
                 }
             }
             const int incl = block_incl_scan(c0 + c1, s_warp);
@@ -707,6 +764,10 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     __syncthreads();
     if (s_nan && tid == 0) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
     cluster.sync();  // no CTA leaves while others may still read its shared memory
+    // every CTA has read the row's first-digit counts (before its first cluster barrier):
+    // leave them zero for the next call
+    if (a.hist && rank == 0)
+        for (int i = tid; i < TK_DIGITS0; i += TK_THREADS) a.hist[static_cast<long long>(row) * TK_DIGITS0 + i] = 0u;
 }
 
 // ---- top-k over the candidates of several key slices -----------------------------------
@@ -841,6 +902,8 @@ __global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(MergeTopkArgs a)
 
 size_t dsa_scores_bytes(int B, int L_max) { return static_cast<size_t>(B) * L_max * sizeof(float); }
 
+size_t dsa_hist_bytes(int B) { return static_cast<size_t>(B) * TK_DIGITS0 * sizeof(uint32_t); }
+
 cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                                   cudaStream_t stream)
 {
@@ -856,6 +919,7 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
         attr_set[dev] = true;
     }
     IndexerArgs ia{};
+    ia.hist = a.hist;
     ia.kscale = a.kscale;
     ia.w = a.w;
     ia.seq_lens = a.seq_lens;
@@ -872,12 +936,12 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     ia.chunks_per_b = chunks;
     const int items = a.B * chunks;
     const int grid = items < a.num_sms ? items : a.num_sms;
-    e = a.kscale ? launch_pdl(indexer_fp8_kernel, dim3(grid), dim3(IX8_THREADS), IX8_SMEM, stream, tm_k, tm_q, ia)
+    e = a.kscale ? launch_pdl(indexer_fp8_kernel, dim3(grid), dim3(IX_THREADS), IX8_SMEM, stream, tm_k, a.q_idx, ia)
                  : launch_pdl(indexer_kernel, dim3(grid), dim3(IX_THREADS), IX_SMEM, stream, tm_k, tm_q, ia);
     if (e != cudaSuccess) return e;
 
-    TopkArgs ta{a.scores, a.seq_lens, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k, a.len_shift,
-                a.tok_idx, a.tok_count, a.L_tok};
+    TopkArgs ta{a.scores, a.seq_lens, a.hist, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k,
+                a.len_shift, a.tok_idx, a.tok_count, a.L_tok};
     const int slice_max = (a.L_max + TK_CL - 1) / TK_CL;
     const size_t key_bytes = static_cast<size_t>(slice_max + (slice_max >> 4) + 1) * sizeof(uint32_t);
     static bool tk_attr[64] = {};

@@ -144,11 +144,17 @@ struct DsaIndexArgs {
     int32_t* tok_idx = nullptr;
     int32_t* tok_count = nullptr;
     int L_tok = 0;  // token capacity of a row (seq_lens beyond it are clamped and flagged)
-    // FP8 keys (kscale non-null): tm_k maps the codes [B][L_max][128] uint8 with a {128, 128, 1}
-    // box and 128-byte swizzle; kscale [B][L_max] fp32 holds each key's scale.
+    // FP8 (kscale non-null): tm_k maps the key codes [B][L_max][128] uint8 with a {128, 128, 1}
+    // box and 128-byte swizzle; kscale [B][L_max] fp32 holds each key's scale; the kernel
+    // quantises the query heads q_idx [B][64][128] bf16 itself (tm_q is not used).
     const float* kscale = nullptr;
+    const kvattn_bf16* q_idx = nullptr;
+    // [B][2048] first-digit counts of the top-k: zero on entry, the indexer adds to them, the
+    // top-k reads them instead of its first pass and leaves them zero; null = the top-k counts
+    uint32_t* hist = nullptr;
 };
 size_t dsa_scores_bytes(int B, int L_max);
+size_t dsa_hist_bytes(int B);  // the [B][2048] first-digit counts
 cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                                   cudaStream_t stream);
 
@@ -181,18 +187,22 @@ struct SparseLaunch {
     const int32_t* idx;
     kvattn_bf16* out;
     float* lse;
-    void* workspace;     // chunk parts: bf16 [B][chunks][Hq][512], then fp32 lse [B][chunks][Hq] (null when one chunk)
+    void* workspace;     // several chunks: per-row counters (zero between calls), bf16 parts
+                         // [B][chunks][Hq][512], their fp32 lse [B][chunks][Hq]; null for one chunk
     int32_t* dev_status;
     int B, Hq, L_max, k;
     float scale;
     bool fp8 = false;
+    int num_sms = 0;     // the grid merges its parts itself when B * chunks <= num_sms
 };
 int sparse_chunks(int k);
 size_t sparse_part_o_bytes(int B, int Hq, int k);
 size_t sparse_partial_bytes(int B, int Hq, int k);
 // tm_q: 3-D map over q [B][Hq][576] with a {64, Hq, 1} box (128-byte swizzle).
 // tm_o: 3-D map with a {64, Hq, 1} box over the output [B][Hq][512] when k <= 128
-// (one chunk), else over the workspace's bf16 parts [B * chunks][Hq][512].
+// (one chunk), else over the workspace's bf16 parts [B * chunks][Hq][512]
+// (sparse_counter_bytes(B) bytes into the workspace).
+size_t sparse_counter_bytes(int B);
 cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_o,
                                cudaStream_t stream);
 

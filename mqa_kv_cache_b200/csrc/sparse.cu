@@ -32,8 +32,12 @@
 //     the chunk's own softmax sum, rounded to bf16 into shared memory (over the
 //     blocks whose values that half has consumed), then stored by TMA.  A row
 //     with one chunk is written to the output directly; otherwise each chunk
-//     leaves its normalised bf16 part and its log-sum-exp, and a second kernel
-//     merges the parts (out = sum_c 2^(lse_c - LSE) o_c).
+//     leaves its normalised bf16 part and its log-sum-exp, and the parts are
+//     merged (out = sum_c 2^(lse_c - LSE) o_c): when the whole grid fits on the
+//     GPU at once (one CTA per SM), it is launched cooperatively and the CTAs of
+//     a row merge its parts themselves -- each announces its part on a per-row
+//     counter, waits (bounded) for the others, and merges a 1/chunks slice of the
+//     columns; otherwise a second kernel merges them.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -86,7 +90,10 @@ struct SparseArgs {
     kvattn_bf16* part_o;        // [B][chunks][Hq][512] bf16, each chunk normalised by its own sum
     float* part_lse;            // [B][chunks][Hq], log2 units (-inf: the chunk has no valid row)
     int32_t* dev_status;
+    int* row_arrive;            // [B] parts of the row written so far (merge in the kernel; zero between calls)
+    int* row_done;              // [B] CTAs of the row done merging (zero between calls)
     int B, Hq, L_max, k, chunks;
+    int fused_merge;            // 1: the row's CTAs merge its parts themselves (cooperative launch)
     float scale;
 };
 
@@ -149,6 +156,61 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                      reinterpret_cast<uint64_t>(map)),
                  "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
                  : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// One (head, 16-byte column chunk) of the merge of a row's C parts: out = sum_c
+// 2^(lse_c - LSE) o_c, LSE = log2 sum_c 2^lse_c (log2 units; lse written in natural log).
+__device__ __forceinline__ void merge_one(const SparseArgs& a, int b, int h, int j)
+{
+    constexpr int MAXC = 16;  // k <= 2048 in chunks of 128
+    const int C = a.chunks;
+    float ls[MAXC];
+    uint4 ov[MAXC];
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+        if (c < C) {
+            const long long row = (static_cast<long long>(b) * C + c) * a.Hq + h;
+            ls[c] = __ldcg(a.part_lse + row);
+            ov[c] = __ldcg(reinterpret_cast<const uint4*>(a.part_o + row * SP_DV) + j);
+        }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c)
+        if (c < C) M = fmaxf(M, ls[c]);
+    const float Mu = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    float wgt[MAXC];
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+        wgt[c] = c < C ? fast_exp2(ls[c] - Mu) : 0.f;
+        L += wgt[c];
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+        if (c < C) {
+            const float wc = wgt[c] * inv;
+            const uint32_t w4[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = fmaf(wc, bf16_lo(w4[i]), acc[2 * i]);
+                acc[2 * i + 1] = fmaf(wc, bf16_hi(w4[i]), acc[2 * i + 1]);
+            }
+        }
+    }
+    const long long ob = (static_cast<long long>(b) * a.Hq + h) * SP_DV;
+    reinterpret_cast<uint4*>(a.out + ob)[j] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                         pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    if (j == 0 && a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
 }
 
 template <bool FP8>
@@ -404,12 +466,19 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         named_bar_sync(3 + g, 128);
+        const bool fused = !one && a.fused_merge;
         if (quarter == 0 && lane == 0 && have_o && !*s_abort) {
             const int z = one ? b : b * a.chunks + chunk;
 #pragma unroll
             for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tm_o, stg + bx * SP_BLOCK, 256 * g + 64 * bx, 0, z);
             asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // shared memory read before exit
+            if (fused) {
+                // the part is in global memory before the row's counter says so
+                asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            } else {
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // shared memory read before exit
+            }
         }
         if (g == 0 && live) {
             const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
@@ -417,6 +486,41 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                 if (a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = lse2 * kLn2;
             } else {
                 a.part_lse[(static_cast<long long>(b) * a.chunks + chunk) * a.Hq + h] = lse2;
+            }
+        }
+        if (fused) {
+            // ===== merge in the kernel: every CTA of the row (all resident: cooperative
+            // launch) announces its part, waits for the others, then merges a column slice =====
+            __threadfence();           // this thread's part stores (lse, the TMA stores it waited for)
+            named_bar_sync(1, SP_GT);  // both halves stored, every part lse written
+            if (t == 0) {
+                if (!*s_abort) {
+                    __threadfence();
+                    atomicAdd(a.row_arrive + b, 1);
+                    const unsigned long long t0 = global_timer_ns();
+                    while (ld_acquire_gpu(a.row_arrive + b) < a.chunks) {
+                        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+                            *s_abort = 1;
+                            report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+            }
+            named_bar_sync(1, SP_GT);
+            if (!*s_abort) {
+                const int j0 = chunk * (SP_DV / 8) / a.chunks, j1 = (chunk + 1) * (SP_DV / 8) / a.chunks;
+                const int nj = j1 - j0;
+                for (int it = t; it < a.Hq * nj; it += SP_GT) merge_one(a, b, it / nj, j0 + it % nj);
+                named_bar_sync(1, SP_GT);  // this CTA's reads of the parts are done
+                if (t == 0) {
+                    __threadfence();
+                    if (atomicAdd(a.row_done + b, 1) == a.chunks - 1) {  // the row's last: leave the counters zero
+                        a.row_arrive[b] = 0;
+                        a.row_done[b] = 0;
+                    }
+                }
             }
         }
     } else if (warp == SP_TMA_WARP) {
@@ -495,58 +599,15 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
 // each.  A thread loads every chunk's lse and its 16 bytes of every part at
 // once (one round trip), then out = sum_c 2^(lse_c - LSE) o_c and
 // LSE = log2 sum_c 2^lse_c (all in log2 units; lse is written in natural log).
-constexpr int SPM_MAX_CHUNKS = 16;  // k <= 2048 in chunks of 128
 constexpr int SPM_HEADS = 4;
 
 __global__ void __launch_bounds__(SPM_HEADS * 64) sparse_merge_kernel(SparseArgs a)
 {
     pdl_wait();
     pdl_trigger();
-    const int C = a.chunks;
     const int b = blockIdx.y;
     const int h = blockIdx.x * SPM_HEADS + (threadIdx.x >> 6);
-    const int j = threadIdx.x & 63;
-    if (h >= a.Hq) return;
-    float ls[SPM_MAX_CHUNKS];
-    uint4 ov[SPM_MAX_CHUNKS];
-#pragma unroll
-    for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
-        if (c < C) {
-            const long long row = (static_cast<long long>(b) * C + c) * a.Hq + h;
-            ls[c] = __ldcg(a.part_lse + row);
-            ov[c] = __ldcg(reinterpret_cast<const uint4*>(a.part_o + row * SP_DV) + j);
-        }
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < SPM_MAX_CHUNKS; ++c)
-        if (c < C) M = fmaxf(M, ls[c]);
-    const float Mu = M == -INFINITY ? 0.f : M;
-    float L = 0.f;
-    float wgt[SPM_MAX_CHUNKS];
-#pragma unroll
-    for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
-        wgt[c] = c < C ? fast_exp2(ls[c] - Mu) : 0.f;
-        L += wgt[c];
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int c = 0; c < SPM_MAX_CHUNKS; ++c) {
-        if (c < C) {
-            const float wc = wgt[c] * inv;
-            const uint32_t w4[4] = {ov[c].x, ov[c].y, ov[c].z, ov[c].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[2 * i] = fmaf(wc, bf16_lo(w4[i]), acc[2 * i]);
-                acc[2 * i + 1] = fmaf(wc, bf16_hi(w4[i]), acc[2 * i + 1]);
-            }
-        }
-    }
-    const long long ob = (static_cast<long long>(b) * a.Hq + h) * SP_DV;
-    reinterpret_cast<uint4*>(a.out + ob)[j] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                                         pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-    if (j == 0 && a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+    if (h < a.Hq) merge_one(a, b, h, threadIdx.x & 63);
 }
 
 template <bool FP8>
@@ -566,6 +627,10 @@ cudaError_t set_smem_attr_once()
 
 int sparse_chunks(int k) { return (k + SP_ROWS - 1) / SP_ROWS; }
 
+// Workspace (several chunks): [0, 256 * ceil(8 B / 256)) the per-row counters, then the
+// bf16 parts [B][chunks][Hq][512], then their lse [B][chunks][Hq].
+size_t sparse_counter_bytes(int B) { return (static_cast<size_t>(B) * 2 * sizeof(int) + 255) / 256 * 256; }
+
 size_t sparse_part_o_bytes(int B, int Hq, int k)
 {
     const int c = sparse_chunks(k);
@@ -577,7 +642,7 @@ size_t sparse_partial_bytes(int B, int Hq, int k)
 {
     const int c = sparse_chunks(k);
     if (c <= 1) return 0;
-    return sparse_part_o_bytes(B, Hq, k) + static_cast<size_t>(B) * c * Hq * sizeof(float);
+    return sparse_counter_bytes(B) + sparse_part_o_bytes(B, Hq, k) + static_cast<size_t>(B) * c * Hq * sizeof(float);
 }
 
 cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_o,
@@ -598,13 +663,32 @@ cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, c
     a.scale = l.scale;
     a.dev_status = l.dev_status;
     if (a.chunks > 1) {
-        a.part_o = static_cast<kvattn_bf16*>(l.workspace);
-        a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(l.workspace) + sparse_part_o_bytes(l.B, l.Hq, l.k));
+        uint8_t* ws = static_cast<uint8_t*>(l.workspace);
+        a.row_arrive = reinterpret_cast<int*>(ws);
+        a.row_done = a.row_arrive + l.B;
+        a.part_o = reinterpret_cast<kvattn_bf16*>(ws + sparse_counter_bytes(l.B));
+        a.part_lse = reinterpret_cast<float*>(ws + sparse_counter_bytes(l.B) + sparse_part_o_bytes(l.B, l.Hq, l.k));
+        // one CTA per SM (its shared memory): the row's CTAs can wait for each other only
+        // when the whole grid is resident at once
+        a.fused_merge = static_cast<long long>(l.B) * a.chunks <= l.num_sms ? 1 : 0;
     }
-    e = l.fp8 ? launch_pdl(sparse_attn_kernel<true>, dim3(a.chunks, l.B), dim3(SP_THREADS), SP_SMEM, stream, tm_q,
-                           tm_o, a)
-              : launch_pdl(sparse_attn_kernel<false>, dim3(a.chunks, l.B), dim3(SP_THREADS), SP_SMEM, stream, tm_q,
-                           tm_o, a);
+    const dim3 grid(a.chunks, l.B);
+    if (a.fused_merge) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = grid;
+        cfg.blockDim = dim3(SP_THREADS);
+        cfg.dynamicSmemBytes = SP_SMEM;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return l.fp8 ? cudaLaunchKernelEx(&cfg, sparse_attn_kernel<true>, tm_q, tm_o, a)
+                     : cudaLaunchKernelEx(&cfg, sparse_attn_kernel<false>, tm_q, tm_o, a);
+    }
+    e = l.fp8 ? launch_pdl(sparse_attn_kernel<true>, grid, dim3(SP_THREADS), SP_SMEM, stream, tm_q, tm_o, a)
+              : launch_pdl(sparse_attn_kernel<false>, grid, dim3(SP_THREADS), SP_SMEM, stream, tm_q, tm_o, a);
     if (e != cudaSuccess || a.chunks == 1) return e;
     return launch_pdl(sparse_merge_kernel, dim3((l.Hq + SPM_HEADS - 1) / SPM_HEADS, l.B), dim3(SPM_HEADS * 64), 0,
                       stream, a);

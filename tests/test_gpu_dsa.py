@@ -206,3 +206,62 @@ def test_sparse_row_without_valid_index(K):
     assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
     ro, rl = _sparse_ref(q[1:], lat[1:], idx[1:], wl.Dv, wl.sparse_scale)
     assert_attn_close(out[1:], ro, lse[1:], rl, "row 1 next to an empty row")
+
+
+@pytest.mark.parametrize("B", [2, 10])
+def test_sparse_merge_paths_and_workspace_counters(K, B):
+    """B * 16 chunks <= the SM count: the kernel merges the chunk parts itself (cooperative
+    launch, per-row counters in the workspace); B = 10 (160 CTAs): the merge kernel does.
+    Both against the oracle; the counters are zero after each call, and a second call on
+    the same workspace gives the same bits."""
+    wl = W.DSA_128K
+    Hq, L, k = 64, 3000, 2048
+    gen = W.generator(2100 + B)
+    q = W.normal_bf16((B, Hq, wl.Dk), gen)
+    lat = W.normal_bf16((B, L, wl.Dk), gen)
+    idx = torch.stack([torch.randperm(L, generator=gen)[:k] for _ in range(B)]).to(torch.int32)
+    idx[0, 100:300] = -1
+    ws = K.workspace(K.attn_decode_sparse_workspace_bytes(B, Hq, wl.Dv, k))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out1, lse1 = K.attn_decode_sparse(q.cuda(), lat.cuda(), idx.cuda(), wl.Dv, wl.sparse_scale, ws=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert int(ws[:8 * B].count_nonzero()) == 0
+    out2, lse2 = K.attn_decode_sparse(q.cuda(), lat.cuda(), idx.cuda(), wl.Dv, wl.sparse_scale, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+    ro, rl = _sparse_ref(q, lat, idx, wl.Dv, wl.sparse_scale)
+    assert_attn_close(out1, ro, lse1, rl, f"sparse merge path B={B}")
+
+
+def test_selection_workspace_counts_are_left_zero(K):
+    """The indexers count the top-k's first digit into the workspace's histogram region
+    and the top-k clears it: zero after every call, and calls on a reused workspace give
+    the same selection (bf16 indexer, FP8 indexer, group selection)."""
+    wl = W.DSA_128K
+    B, L, k = 3, 6000, 2048
+    inp = W.dsa_inputs(wl, B=B, L=L, seed=88, with_latent=False)
+    q_idx, w, k_idx = inp["q_idx"].cuda(), inp["w"].cuda(), inp["k_idx"].cuda()
+    lens = torch.tensor([6000, 2500, 1000], dtype=torch.int32).cuda()
+    hist_bytes = B * 2048 * 4
+    ws = K.workspace(K.dsa_index_topk_workspace_bytes(B, L, k))
+    first = K.dsa_index_topk(q_idx, w, k_idx, k, seq_lens=lens, ws=ws)[0].clone()
+    torch.cuda.synchronize()
+    assert int(ws[:hist_bytes].count_nonzero()) == 0
+    again = K.dsa_index_topk(q_idx, w, k_idx, k, seq_lens=lens, ws=ws)[0]
+    torch.cuda.synchronize()
+    assert torch.equal(first, again) and int(ws[:hist_bytes].count_nonzero()) == 0
+    codes, sc = K.idx_key_quant_fp8(k_idx)
+    f8 = K.dsa_index_topk_fp8(q_idx, w, codes, sc, k, seq_lens=lens, ws=ws)[0].clone()
+    f8b = K.dsa_index_topk_fp8(q_idx, w, codes, sc, k, seq_lens=lens, ws=ws)[0]
+    torch.cuda.synchronize()
+    assert torch.equal(f8, f8b) and int(ws[:hist_bytes].count_nonzero()) == 0
+    # group selection over 4-token group keys
+    cos, sin = K.rope_table_build(K.rope_params(128, base=500000.0), L)
+    kb = K.qsa_block_keys(k_idx, lens, cos, sin)
+    ws2 = K.workspace(K.qsa_select_workspace_bytes(B, L, 512))
+    t1, c1, _ = K.qsa_select(q_idx, w, kb, lens, n_top=512, ws=ws2)
+    t1 = t1.clone()
+    t2, c2, _ = K.qsa_select(q_idx, w, kb, lens, n_top=512, ws=ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(t1, t2) and int(ws2[:hist_bytes].count_nonzero()) == 0

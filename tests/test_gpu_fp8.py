@@ -142,13 +142,15 @@ def test_sparse_fp8_bad_index_and_empty_row(K):
     _check_fp8_sparse(out[1:], lse[1:], q[1:], packed[1:].cpu().numpy(), ok, wl.Dv, wl.sparse_scale, "fp8 bad index")
 
 
-# ---- the lightning indexer on FP8 keys ------------------------------------------------
+# ---- the lightning indexer in fp8 (query heads and keys as E4M3) ------------------------
 
 def _fp8_score_bound(q_bits, w, kd):
-    """fp32 error bound of the kernel's scores: the 128-term dot of exact code values
-    in fp32, then the 64-term weighted head sum and the scale (|d| <= 2^-16 * sum_j w_j
-    * sum_i |q_ji khat_ti|, as for bf16 keys, plus the product's rounding)."""
-    q = oracle.bf16_bits_to_f64(q_bits)
+    """fp32 error bound of the kernel's scores: exact products of the codes, the
+    128-term dot in fp32, the 64-term weighted head sum and the scales (|d| <= 2^-16 *
+    sum_j w_j * sum_i |qhat_ji khat_ti|, as for bf16 operands, plus the products'
+    rounding); qhat = the query heads as the kernel quantises them."""
+    qc, qs = oracle.quant_fp8(q_bits)
+    q = oracle.dequant_fp8(qc, qs)
     absdot = np.einsum("bji,bti->btj", np.abs(q), np.abs(kd))
     return 2.0 ** -16 * np.einsum("btj,bj->bt", absdot, w.astype(np.float64)) + 1e-30
 
