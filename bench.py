@@ -802,6 +802,13 @@ def main():
         from mqa_kv_cache_b200 import kvattn as K
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
         line["other_configs"] = measure_others(K, device, args.steps, flush, load_peaks())
+        # the read side of the denominator: the best read-only streaming rate seen in this run
+        # (a plain reduction, or a decode kernel that only reads K and V)
+        rates = [line["roofline"]["read_stream_gbs"]] + [v["GB_s"] for v in line["other_configs"].values()
+                                                          if isinstance(v, dict) and "GB_s" in v]
+        rp = max(rates)
+        line["roofline"]["read_peak_gbs"] = round(rp, 1)
+        line["roofline"]["frac_of_read_peak"] = round(line["roofline"]["achieved"] / rp, 4)
     if world > 1:
         torch.distributed.destroy_process_group()
     # the oracle on the host cores: rank 0 of a single-GPU run only

@@ -586,25 +586,34 @@ int attn_prefill_causal_window(const kvattn_bf16* q, const kvattn_bf16* k, const
 
 // DSA / QSA selection workspace: [0, hist) the per-row first-digit counts of the top-k
 // (zero between calls), then the scores when the caller keeps none.
+// ... then (FP8 calls) the quantised query heads: codes [B][64][128] and scales [B][64].
 static size_t dsa_ws_hist(int B) { return align_up(kvattn::dsa_hist_bytes(B)); }
+static size_t dsa_ws_q8(int B) { return align_up(static_cast<size_t>(B) * 64 * 128) + align_up(static_cast<size_t>(B) * 64 * 4); }
 
 size_t dsa_index_topk_workspace_bytes(int B, int L_max, int k)
 {
     (void)k;
     if (B < 1 || L_max < 1) return 0;
-    return dsa_ws_hist(B) + align_up(kvattn::dsa_scores_bytes(B, L_max));
+    return dsa_ws_hist(B) + dsa_ws_q8(B) + align_up(kvattn::dsa_scores_bytes(B, L_max));
 }
 
-// Checks the selection workspace; on success sets the histogram and the scores buffer.
+// Checks the selection workspace; on success sets the histogram, the scores buffer and
+// (with q8 non-null) the quantised query heads.
 static int dsa_ws(const char* name, int B, int L_max, float* scores_out, void* workspace, size_t workspace_bytes,
-                  uint32_t** hist, float** scores)
+                  uint32_t** hist, float** scores, uint8_t** q8 = nullptr, float** q8_scale = nullptr)
 {
-    const size_t need = dsa_ws_hist(B) + (scores_out ? 0 : align_up(kvattn::dsa_scores_bytes(B, L_max)));
+    const size_t q8b = q8 ? dsa_ws_q8(B) : 0;
+    const size_t need = dsa_ws_hist(B) + q8b + (scores_out ? 0 : align_up(kvattn::dsa_scores_bytes(B, L_max)));
     if (!workspace || workspace_bytes < need) return fail(KVATTN_ERR_WORKSPACE, "%s: workspace needs %zu bytes", name, need);
     if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign)
         return fail(KVATTN_ERR_ALIGN, "%s: workspace must be 256-byte aligned", name);
-    *hist = static_cast<uint32_t*>(workspace);
-    *scores = scores_out ? scores_out : reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + dsa_ws_hist(B));
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    *hist = reinterpret_cast<uint32_t*>(w);
+    if (q8) {
+        *q8 = w + dsa_ws_hist(B);
+        *q8_scale = reinterpret_cast<float*>(w + dsa_ws_hist(B) + align_up(static_cast<size_t>(B) * 64 * 128));
+    }
+    *scores = scores_out ? scores_out : reinterpret_cast<float*>(w + dsa_ws_hist(B) + q8b);
     return KVATTN_OK;
 }
 
@@ -659,17 +668,23 @@ int dsa_index_topk_fp8(const kvattn_bf16* q_idx, const float* w, const uint8_t* 
         return fail(KVATTN_ERR_ALIGN, "dsa_index_topk_fp8: tensors must be 16-byte aligned (scales 4)");
     float* scores = nullptr;
     uint32_t* hist = nullptr;
-    const int ws_rc = dsa_ws("dsa_index_topk_fp8", B, L_max, scores_out, workspace, workspace_bytes, &hist, &scores);
+    uint8_t* q8 = nullptr;
+    float* q8_scale = nullptr;
+    const int ws_rc = dsa_ws("dsa_index_topk_fp8", B, L_max, scores_out, workspace, workspace_bytes, &hist, &scores,
+                             &q8, &q8_scale);
     if (ws_rc != KVATTN_OK) return ws_rc;
     int sms = 0;
     if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "dsa_index_topk_fp8: no CUDA device");
     CUtensorMap tm_k, tm_q;
     const uint64_t dk[4] = {128, static_cast<uint64_t>(L_max), static_cast<uint64_t>(B), 0};
+    const uint64_t dq[4] = {128, 64, static_cast<uint64_t>(B), 0};
     if (make_map(&tm_k, 3, k_codes, dk, 128, true) != KVATTN_OK) return KVATTN_ERR_CUDA;
-    if (make_map_3d(&tm_q, q_idx, 128, 64, B, 64) != KVATTN_OK) return KVATTN_ERR_CUDA;
+    if (make_map(&tm_q, 3, q8, dq, 64, true) != KVATTN_OK) return KVATTN_ERR_CUDA;
     kvattn::DsaIndexArgs a{w, seq_lens, scores, topk_idx, dev_status, B, L_max, k, sms};
     a.kscale = k_scales;
     a.q_idx = q_idx;
+    a.q8 = q8;
+    a.q8_scale = q8_scale;
     a.hist = hist;
     return cuda_status(kvattn::launch_dsa_index_topk(a, tm_k, tm_q, static_cast<cudaStream_t>(stream)),
                        "dsa_index_topk_fp8 launch");

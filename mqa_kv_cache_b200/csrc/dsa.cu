@@ -55,32 +55,46 @@ constexpr int TK_SHIFT0 = 21;
 constexpr int IX_TOK = 128;   // tokens per tile (MMA M)
 constexpr int IX_HEADS = 64;  // indexer heads (MMA N)
 constexpr int IX_DIM = 128;   // key width (MMA K)
-constexpr int IX_STAGES = 6;
-constexpr int IX_BOX = IX_TOK * 128;          // one 64-column SW128 box of a k tile (bytes)
-constexpr int IX_TILE = 2 * IX_BOX;           // k tile [128 x 128] bf16
-constexpr int IX_QBOX = IX_HEADS * 128;       // one 64-column box of q [64 x 64]
-constexpr int IX_QBYTES = 2 * IX_QBOX;
-constexpr int IX_THREADS = 192;               // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 epilogue
+constexpr int IX_BOX = IX_TOK * 128;          // one 128-byte-wide SW128 box of a key tile (16 KB)
+constexpr int IX_QBOX = IX_HEADS * 128;       // one 128-byte-wide box of the query heads (8 KB)
+constexpr int IX_THREADS = 320;               // warp 0 TMA, warp 1 MMA + TMEM, warps 2..9 epilogue
+constexpr int IX_EPI = 256;                   // two groups of four warps, alternate tiles
 constexpr int IX_NACC = 4;                    // 64-column accumulators in flight (the MMA-to-epilogue
-                                              // round trip is ~1 us: two buffers capped a CTA at a tile
-                                              // per ~0.5 us)
+                                              // round trip is ~1 us)
 constexpr int IX_TMEM_COLS = IX_NACC * 64;
-constexpr uint32_t IX_IDESC = umma_idesc_bf16(IX_TOK, IX_HEADS);
 
-constexpr int IX_OFF_Q = IX_STAGES * IX_TILE;
-constexpr int IX_OFF_W = IX_OFF_Q + IX_QBYTES;
-constexpr int IX_OFF_HIST = IX_OFF_W + IX_HEADS * 4;   // [2048] digit counts of the current work item
-constexpr int IX_OFF_BAR = IX_OFF_HIST + 2048 * 4;
-// full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done
-constexpr int IX_NBAR = 2 * IX_STAGES + 3 + 2 * IX_NACC;
-constexpr int IX_OFF_MISC = IX_OFF_BAR + IX_NBAR * 8;
-constexpr int IX_SMEM = IX_OFF_MISC + 32 + 1024;
-static_assert(IX_SMEM <= 232448, "shared memory");
+// bf16 keys: a tile is two 64-column boxes, 6 in flight, K = 128 in eight K = 16 steps
+// (kind::f16); FP8 ("the indexer runs stably in fp8", "Agentic RL 入门3" §2.2 (1)): the
+// query heads and keys are E4M3 codes, a tile is one 128-code box, 12 in flight, K = 128
+// in four K = 32 steps on kind::f8f6f4 (exact code products, fp32 sums); the query head's
+// scale is folded into its weight and the key's scale multiplies the score, which is
+// exact algebra since ReLU(qs ks x) = qs ks ReLU(x) for scales >= 0.
+template <bool FP8>
+struct IxCfg {
+    static constexpr int KBOX = FP8 ? 1 : 2;            // boxes per key tile (and per query)
+    static constexpr int TILE = KBOX * IX_BOX;
+    static constexpr int STAGES = FP8 ? 12 : 6;
+    static constexpr int QBYTES = KBOX * IX_QBOX;
+    static constexpr int KSTEPS = FP8 ? 4 : 8;
+    static constexpr int OFF_Q = STAGES * TILE;
+    static constexpr int OFF_W = OFF_Q + QBYTES;
+    static constexpr int OFF_HIST = OFF_W + IX_HEADS * 4;   // [2048] digit counts of the current work item
+    static constexpr int OFF_BAR = OFF_HIST + 2048 * 4;
+    // full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done
+    static constexpr int NBAR = 2 * STAGES + 3 + 2 * IX_NACC;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 32 + 1024;
+    static_assert(SMEM <= 232448, "shared memory");
+    static constexpr uint32_t IDESC = FP8 ? ((1u << 4) | (static_cast<uint32_t>(IX_HEADS >> 3) << 17) |
+                                             (static_cast<uint32_t>(IX_TOK >> 4) << 24))  // E4M3 x E4M3 -> fp32
+                                          : umma_idesc_bf16(IX_TOK, IX_HEADS);
+};
 
 struct IndexerArgs {
     const float* w;
     const int32_t* seq_lens;
-    const float* kscale;  // FP8 keys: [B][L_max] fp32 scales (indexer_fp8_kernel only)
+    const float* kscale;  // FP8: [B][L_max] key scales
+    const float* qscale;  // FP8: [B][64] query-head scales
     float* scores;
     uint32_t* hist;       // [B][2048] first-digit counts of the valid scores (added to; zero on entry)
     int32_t* dev_status;
@@ -96,29 +110,41 @@ __device__ __forceinline__ void ix_item(const IndexerArgs& a, int item, int& b, 
     t1 = static_cast<int>(static_cast<long long>(c + 1) * a.tiles_per_b / a.chunks_per_b);
 }
 
+__device__ __forceinline__ void tc_mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+template <bool FP8>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q, IndexerArgs a)
 {
+    using C = IxCfg<FP8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + IX_OFF_BAR);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* full = bars;
-    uint64_t* empty = bars + IX_STAGES;
-    uint64_t* q_full = bars + 2 * IX_STAGES;
+    uint64_t* empty = bars + C::STAGES;
+    uint64_t* q_full = bars + 2 * C::STAGES;
     uint64_t* q_empty = q_full + 1;
     uint64_t* acc_full = q_full + 2;
     uint64_t* acc_empty = acc_full + IX_NACC;
     uint64_t* mma_done = acc_empty + IX_NACC;
-    float* s_w = reinterpret_cast<float*>(smem + IX_OFF_W);
-    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + IX_OFF_HIST);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + IX_OFF_MISC);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + IX_OFF_MISC + 4);
+    float* s_w = reinterpret_cast<float*>(smem + C::OFF_W);
+    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = a.B * a.chunks_per_b;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < IX_STAGES; ++s) {
+        for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -148,7 +174,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     pdl_trigger();
 
     if (warp == 0) {
-        // ===== TMA producer =====
+        // ===== TMA producer: each item's query heads, then its key tiles =====
         if (lane == 0) {
             int it = 0, n = 0;
             for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
@@ -158,30 +184,30 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                     *s_abort = 1;
                     break;
                 }
-                mbar_arrive_expect_tx(q_full, IX_QBYTES);
-                tma_load_3d(smem + IX_OFF_Q, &tm_q, q_full, 0, 0, b);
-                tma_load_3d(smem + IX_OFF_Q + IX_QBOX, &tm_q, q_full, 64, 0, b);
+                mbar_arrive_expect_tx(q_full, C::QBYTES);
+#pragma unroll
+                for (int i = 0; i < C::KBOX; ++i) tma_load_3d(smem + C::OFF_Q + i * IX_QBOX, &tm_q, q_full, 64 * i, 0, b);
                 for (int t = t0; t < t1; ++t, ++it) {
-                    const int s = it % IX_STAGES;
-                    if (it >= IX_STAGES && (*s_abort || !mbar_wait(&empty[s], ((it / IX_STAGES) - 1) & 1))) {
+                    const int s = it % C::STAGES;
+                    if (it >= C::STAGES && (*s_abort || !mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1))) {
                         *s_abort = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[s], IX_TILE);
-                    uint8_t* dst = smem + s * IX_TILE;
-                    tma_load_3d(dst, &tm_k, &full[s], 0, t * IX_TOK, b);
-                    tma_load_3d(dst + IX_BOX, &tm_k, &full[s], 64, t * IX_TOK, b);
+                    mbar_arrive_expect_tx(&full[s], C::TILE);
+                    uint8_t* dst = smem + s * C::TILE;
+#pragma unroll
+                    for (int i = 0; i < C::KBOX; ++i) tma_load_3d(dst + i * IX_BOX, &tm_k, &full[s], 64 * i, t * IX_TOK, b);
                 }
             }
             if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
-            for (int j = it - IX_STAGES > 0 ? it - IX_STAGES : 0; j < it; ++j)
-                mbar_wait(&full[j % IX_STAGES], (j / IX_STAGES) & 1);
+            for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
+                mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
         }
     } else if (warp == 1) {
         // ===== MMA issuer (one thread) =====
         if (lane == 0) {
-            const uint32_t q_addr = smem_u32(smem + IX_OFF_Q);
-            int it = 0, tc = 0, n = 0;
+            const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
+            int it = 0, n = 0;
             for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
                 int b, t0, t1;
                 ix_item(a, item, b, t0, t1);
@@ -189,23 +215,27 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                     *s_abort = 1;
                     break;
                 }
-                for (int t = t0; t < t1; ++t, ++it, ++tc) {
-                    const int s = it % IX_STAGES;
-                    const int buf = tc % IX_NACC;
-                    if (*s_abort || !mbar_wait(&full[s], (it / IX_STAGES) & 1) ||
-                        (tc >= IX_NACC && !mbar_wait(&acc_empty[buf], ((tc / IX_NACC) - 1) & 1))) {
+                for (int t = t0; t < t1; ++t, ++it) {
+                    const int s = it % C::STAGES;
+                    const int buf = it % IX_NACC;
+                    if (*s_abort || !mbar_wait(&full[s], (it / C::STAGES) & 1) ||
+                        (it >= IX_NACC && !mbar_wait(&acc_empty[buf], ((it / IX_NACC) - 1) & 1))) {
                         *s_abort = 1;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + s * IX_TILE);
+                    const uint32_t k_addr = smem_u32(smem + s * C::TILE);
                     const uint32_t d_addr = tmem + buf * IX_HEADS;
 #pragma unroll
-                    for (int ks = 0; ks < IX_DIM / 16; ++ks) {
-                        const uint32_t off = (ks & 3) * 32;
-                        const uint64_t ad = umma_desc_k_sw128(k_addr + (ks >> 2) * IX_BOX + off);
-                        const uint64_t bd = umma_desc_k_sw128(q_addr + (ks >> 2) * IX_QBOX + off);
-                        tc_mma_bf16(d_addr, ad, bd, IX_IDESC, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < C::KSTEPS; ++ks) {
+                        // 32 bytes of K per step (16 bf16 or 32 codes) of a 128-byte row
+                        const uint32_t off = (ks >> 2) * IX_BOX + (ks & 3) * 32;
+                        const uint64_t ad = umma_desc_k_sw128(k_addr + off);
+                        const uint64_t bd = umma_desc_k_sw128(q_addr + (ks >> 2) * IX_QBOX + (ks & 3) * 32);
+                        if constexpr (FP8)
+                            tc_mma_f8(d_addr, ad, bd, C::IDESC, ks > 0 ? 1u : 0u);
+                        else
+                            tc_mma_bf16(d_addr, ad, bd, C::IDESC, ks > 0 ? 1u : 0u);
                     }
                     tc_commit(&empty[s]);
                     tc_commit(&acc_full[buf]);
@@ -218,11 +248,13 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
             if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
         }
     } else {
-        // ===== epilogue: TMEM -> ReLU, weight, sum over heads -> scores =====
+        // ===== epilogue: TMEM -> ReLU, weight, sum over heads -> scores; two groups of
+        // four warps take alternate tiles (a tile's read-out and sums are serial work) =====
         const int quarter = warp & 3;  // TMEM lanes this warp may read
+        const int grp = (warp - 2) >> 2;
         const int row = quarter * 32 + lane;
         const int ep = threadIdx.x - 64;
-        for (int i = ep; i < TK_DIGITS0; i += 128) s_hist[i] = 0u;  // ordered by the item's first barrier
+        for (int i = ep; i < TK_DIGITS0; i += IX_EPI) s_hist[i] = 0u;  // ordered by the item's first barrier
         int tc = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
             int b, t0, t1;
@@ -230,278 +262,20 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
             const int len_raw = a.seq_lens ? (a.seq_lens[b] >> a.len_shift) : a.L_max;
             const int len = min(max(len_raw, 0), a.L_max);
             if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
-            named_bar_sync(2, 128);
-            if (ep < IX_HEADS) s_w[ep] = a.w[static_cast<long long>(b) * IX_HEADS + ep];
-            named_bar_sync(2, 128);
+            named_bar_sync(2, IX_EPI);
+            if (ep < IX_HEADS) {
+                const long long wi = static_cast<long long>(b) * IX_HEADS + ep;
+                s_w[ep] = FP8 ? a.w[wi] * a.qscale[wi] : a.w[wi];
+            }
+            named_bar_sync(2, IX_EPI);
             float* out = a.scores + static_cast<long long>(b) * a.L_max;
             for (int t = t0; t < t1; ++t, ++tc) {
+                if ((tc & 1) != grp) continue;
                 const int buf = tc % IX_NACC;
+                const int tok = t * IX_TOK + row;
+                const float kscale = FP8 && tok < a.L_max ? __ldg(a.kscale + static_cast<long long>(b) * a.L_max + tok) : 1.f;
                 // on an abort the loops still run to the end (without waiting or
                 // working) so that all four warps meet at the same named barriers
-                if (!warp_wait(&acc_full[buf], (tc / IX_NACC) & 1, s_abort)) continue;
-                tc_fence_after();
-                const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_HEADS;
-                uint32_t v0[32], v1[32];
-                tmem_ld32(taddr, v0);
-                tmem_ld32(taddr + 32, v1);
-                tmem_wait_ld();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[buf]);
-                float acc = 0.f;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[j], fmaxf(__uint_as_float(v0[j]), 0.f), acc);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), acc);
-                const int tok = t * IX_TOK + row;
-                if (acc != acc) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
-                if (tok < a.L_max) out[tok] = tok < len ? acc : -INFINITY;
-                // the score's first top-k digit, counted once per warp and digit
-                const bool in = a.hist != nullptr && tok < len;
-                bool nan_key = false;
-                const uint32_t digit = in ? score_key(acc, nan_key) >> TK_SHIFT0 : 0xffffffffu;
-                const uint32_t same = __match_any_sync(0xffffffffu, digit);
-                if (in && lane == __ffs(same) - 1) atomicAdd(&s_hist[digit], static_cast<uint32_t>(__popc(same)));
-            }
-            if (a.hist) {  // the item's counts into the row's histogram; the shared one back to zero
-                named_bar_sync(2, 128);
-                uint32_t* gh = a.hist + static_cast<long long>(b) * TK_DIGITS0;
-                for (int i = ep; i < TK_DIGITS0; i += 128) {
-                    const uint32_t v = s_hist[i];
-                    if (v) {
-                        atomicAdd(gh + i, v);
-                        s_hist[i] = 0u;
-                    }
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, IX_TMEM_COLS);
-    }
-}
-
-// ---- indexer in fp8 ------------------------------------------------------------------
-// "稀疏注意力：省了什么，没省什么", 改进一 (an indexer key of about 132 bytes: 128 E4M3
-// codes and one fp32 scale) and "Agentic RL 入门3" §2.2 (1) (the indexer runs stably in
-// fp8): the product runs on E4M3 operands.  The 64 query heads of a row are quantised
-// here with the keys' rule (one fp32 scale per 128-wide head, RNE, saturating) into the
-// MMA's B operand; the code tiles land by TMA in the A operand's layout and go to
-// tcgen05.mma kind::f8f6f4 unconverted (M = 128 tokens, N = 64 heads, K = 128 in four
-// K = 32 steps, exact products, fp32 accumulation).  With scales >= 0, ReLU(qhat .
-// khat) = qs_j ks_t ReLU(qc_j . kc_t), so the epilogue folds the head scale into the
-// head weight and multiplies the sum by the key's scale.  HBM bytes per token: 128 + 4.
-constexpr int IX8_TILE = IX_TOK * 128;           // 16 KB code tile [128 tokens][128 codes]
-constexpr int IX8_STAGES = 12;
-constexpr int IX8_QBYTES = IX_HEADS * 128;        // [64 heads][128 codes]
-constexpr int IX8_OFF_Q = IX8_STAGES * IX8_TILE;
-constexpr int IX8_OFF_W = IX8_OFF_Q + IX8_QBYTES;
-constexpr int IX8_OFF_HIST = IX8_OFF_W + IX_HEADS * 4;
-constexpr int IX8_OFF_BAR = IX8_OFF_HIST + 2048 * 4;
-// full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done
-constexpr int IX8_NBAR = 2 * IX8_STAGES + 3 + 2 * IX_NACC;
-constexpr int IX8_OFF_MISC = IX8_OFF_BAR + IX8_NBAR * 8;
-constexpr int IX8_SMEM = IX8_OFF_MISC + 32 + 1024;
-static_assert(IX8_SMEM <= 232448, "shared memory");
-// D fp32, A and B E4M3 (format 0 of kind::f8f6f4), both K-major, M x N
-constexpr uint32_t IX8_IDESC = (1u << 4) | (static_cast<uint32_t>(IX_HEADS >> 3) << 17) |
-                               (static_cast<uint32_t>(IX_TOK >> 4) << 24);
-
-__device__ __forceinline__ void tc_mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Two fp32 -> two E4M3 codes (lo in the low byte), round to nearest even, saturating.
-__device__ __forceinline__ uint32_t ix_e4m3x2(float lo, float hi)
-{
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    return r;
-}
-
-__global__ void __launch_bounds__(IX_THREADS, 1)
-    indexer_fp8_kernel(const __grid_constant__ CUtensorMap tm_k8, const kvattn_bf16* __restrict__ q_idx,
-                       IndexerArgs a)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + IX8_OFF_BAR);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + IX8_STAGES;
-    uint64_t* q_full = bars + 2 * IX8_STAGES;
-    uint64_t* q_empty = q_full + 1;
-    uint64_t* acc_full = q_full + 2;
-    uint64_t* acc_empty = acc_full + IX_NACC;
-    uint64_t* mma_done = acc_empty + IX_NACC;
-    float* s_w = reinterpret_cast<float*>(smem + IX8_OFF_W);
-    uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + IX8_OFF_HIST);
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + IX8_OFF_MISC);
-    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + IX8_OFF_MISC + 4);
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = a.B * a.chunks_per_b;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < IX8_STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(q_full, 4);
-        mbar_init(q_empty, 1);
-        for (int i = 0; i < IX_NACC; ++i) {
-            mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);
-        }
-        mbar_init(mma_done, 1);
-        *s_abort = 0;
-        fence_barrier_init();
-    }
-    if (warp == 0 && lane == 0) tma_prefetch_desc(&tm_k8);
-    if (warp == 1) {
-        tmem_alloc(s_tmem, IX_TMEM_COLS);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-    pdl_wait();
-    pdl_trigger();
-
-    if (warp == 0) {
-        // ===== TMA producer: code tiles =====
-        if (lane == 0) {
-            int it = 0;
-            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x) {
-                int b, t0, t1;
-                ix_item(a, item, b, t0, t1);
-                for (int t = t0; t < t1; ++t, ++it) {
-                    const int s = it % IX8_STAGES;
-                    if (it >= IX8_STAGES && (*s_abort || !mbar_wait(&empty[s], ((it / IX8_STAGES) - 1) & 1))) {
-                        *s_abort = 1;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&full[s], IX8_TILE);
-                    tma_load_3d(smem + s * IX8_TILE, &tm_k8, &full[s], 0, t * IX_TOK, b);
-                }
-            }
-            if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
-            for (int j = it - IX8_STAGES > 0 ? it - IX8_STAGES : 0; j < it; ++j)
-                mbar_wait(&full[j % IX8_STAGES], (j / IX8_STAGES) & 1);
-        }
-    } else if (warp == 1) {
-        // ===== MMA issuer (one thread) =====
-        if (lane == 0) {
-            const uint32_t q_addr = smem_u32(smem + IX8_OFF_Q);
-            int it = 0, n = 0;
-            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
-                int b, t0, t1;
-                ix_item(a, item, b, t0, t1);
-                if (!mbar_wait(q_full, n & 1)) {
-                    *s_abort = 1;
-                    break;
-                }
-                for (int t = t0; t < t1; ++t, ++it) {
-                    const int s = it % IX8_STAGES;
-                    const int buf = it % IX_NACC;
-                    if (*s_abort || !mbar_wait(&full[s], (it / IX8_STAGES) & 1) ||
-                        (it >= IX_NACC && !mbar_wait(&acc_empty[buf], ((it / IX_NACC) - 1) & 1))) {
-                        *s_abort = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + s * IX8_TILE);
-                    const uint32_t d_addr = tmem + buf * IX_HEADS;
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)  // K = 32 codes (32 bytes of the 128-byte row) per step
-                        tc_mma_f8(d_addr, umma_desc_k_sw128(k_addr + ks * 32), umma_desc_k_sw128(q_addr + ks * 32),
-                                  IX8_IDESC, ks > 0 ? 1u : 0u);
-                    tc_commit(&empty[s]);
-                    tc_commit(&acc_full[buf]);
-                }
-                tc_commit(q_empty);
-            }
-            tc_commit(mma_done);
-            mbar_wait(mma_done, 0);
-            if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
-        }
-    } else {
-        // ===== epilogue (and, per item, the query heads' quantisation) =====
-        const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;
-        const int ep = threadIdx.x - 64;
-        const int qh = ep >> 1, qhalf = ep & 1;  // quantisation: head qh, values 64 qhalf .. + 63
-        for (int i = ep; i < TK_DIGITS0; i += 128) s_hist[i] = 0u;  // ordered by the item's first barrier
-        int tc = 0, n = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++n) {
-            int b, t0, t1;
-            ix_item(a, item, b, t0, t1);
-            const int len_raw = a.seq_lens ? (a.seq_lens[b] >> a.len_shift) : a.L_max;
-            const int len = min(max(len_raw, 0), a.L_max);
-            if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
-            named_bar_sync(2, 128);  // the previous item's epilogue has read s_w
-            // the previous item's MMAs have read the query tile
-            const bool q_free = n == 0 || warp_wait(q_empty, (n - 1) & 1, s_abort);
-            {
-                const uint4* src = reinterpret_cast<const uint4*>(q_idx + (static_cast<long long>(b) * IX_HEADS + qh) * IX_DIM +
-                                                                  64 * qhalf);
-                uint4 x[8];
-                float amax = 0.f;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    x[i] = __ldg(src + i);
-                    const uint32_t w4[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w4[e])), fabsf(bf16_hi(w4[e]))));
-                }
-                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-                const float qs = __fdiv_rn(amax, 448.f);
-                uint8_t* qrow = smem + IX8_OFF_Q;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {  // 16 codes = one 16-byte chunk of the head's 128-byte row
-                    uint32_t wd[4];
-#pragma unroll
-                    for (int hw = 0; hw < 2; ++hw) {
-                        const uint4 v = x[2 * c + hw];
-                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                        uint32_t pk[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const uint32_t lo = qs == 0.f ? 0u
-                                                          : ix_e4m3x2(__fdiv_rn(bf16_lo(w4[2 * e]), qs),
-                                                                      __fdiv_rn(bf16_hi(w4[2 * e]), qs));
-                            const uint32_t hi = qs == 0.f ? 0u
-                                                          : ix_e4m3x2(__fdiv_rn(bf16_lo(w4[2 * e + 1]), qs),
-                                                                      __fdiv_rn(bf16_hi(w4[2 * e + 1]), qs));
-                            pk[e] = lo | (hi << 16);
-                        }
-                        wd[2 * hw] = pk[0];
-                        wd[2 * hw + 1] = pk[1];
-                    }
-                    if (q_free)
-                        *reinterpret_cast<uint4*>(qrow + swz128(qh, 4 * qhalf + c)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-                }
-                if (qhalf == 0) s_w[qh] = a.w[static_cast<long long>(b) * IX_HEADS + qh] * qs;
-            }
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncwarp();
-            if (lane == 0 && q_free) mbar_arrive(q_full);
-            named_bar_sync(2, 128);  // s_w complete
-            float* out = a.scores + static_cast<long long>(b) * a.L_max;
-            const float* ks = a.kscale + static_cast<long long>(b) * a.L_max;
-            for (int t = t0; t < t1; ++t, ++tc) {
-                const int buf = tc % IX_NACC;
-                const int tok = t * IX_TOK + row;
-                const float kscale = tok < a.L_max ? __ldg(ks + tok) : 0.f;
                 if (!warp_wait(&acc_full[buf], (tc / IX_NACC) & 1, s_abort)) continue;
                 tc_fence_after();
                 const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * IX_HEADS;
@@ -514,12 +288,15 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acc_empty[buf]);
-                float acc = 0.f;
+                // four independent chains over the heads (a 64-deep chain is latency-bound)
+                float accs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[j], fmaxf(__uint_as_float(v0[j]), 0.f), acc);
+                for (int j = 0; j < 32; ++j) accs[j & 3] = fmaf(s_w[j], fmaxf(__uint_as_float(v0[j]), 0.f), accs[j & 3]);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) acc = fmaf(s_w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), acc);
-                acc *= kscale;
+                for (int j = 0; j < 32; ++j)
+                    accs[j & 3] = fmaf(s_w[32 + j], fmaxf(__uint_as_float(v1[j]), 0.f), accs[j & 3]);
+                float acc = (accs[0] + accs[1]) + (accs[2] + accs[3]);
+                if (FP8) acc *= kscale;
                 if (acc != acc) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
                 if (tok < a.L_max) out[tok] = tok < len ? acc : -INFINITY;
                 // the score's first top-k digit, counted once per warp and digit
@@ -530,9 +307,9 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 if (in && lane == __ffs(same) - 1) atomicAdd(&s_hist[digit], static_cast<uint32_t>(__popc(same)));
             }
             if (a.hist) {  // the item's counts into the row's histogram; the shared one back to zero
-                named_bar_sync(2, 128);
+                named_bar_sync(2, IX_EPI);
                 uint32_t* gh = a.hist + static_cast<long long>(b) * TK_DIGITS0;
-                for (int i = ep; i < TK_DIGITS0; i += 128) {
+                for (int i = ep; i < TK_DIGITS0; i += IX_EPI) {
                     const uint32_t v = s_hist[i];
                     if (v) {
                         atomicAdd(gh + i, v);
@@ -912,15 +689,22 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 64 && !attr_set[dev]) {
-        e = cudaFuncSetAttribute(indexer_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX_SMEM);
+        e = cudaFuncSetAttribute(indexer_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, IxCfg<false>::SMEM);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(indexer_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, IX8_SMEM);
+        e = cudaFuncSetAttribute(indexer_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, IxCfg<true>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
+    }
+    const bool fp8 = a.kscale != nullptr;
+    if (fp8) {
+        // the query heads as E4M3 codes and scales, with the keys' rule, once per call
+        e = launch_idx_key_quant_fp8(a.q_idx, static_cast<long long>(a.B) * IX_HEADS, a.q8, a.q8_scale, stream);
+        if (e != cudaSuccess) return e;
     }
     IndexerArgs ia{};
     ia.hist = a.hist;
     ia.kscale = a.kscale;
+    ia.qscale = a.q8_scale;
     ia.w = a.w;
     ia.seq_lens = a.seq_lens;
     ia.scores = a.scores;
@@ -936,8 +720,8 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     ia.chunks_per_b = chunks;
     const int items = a.B * chunks;
     const int grid = items < a.num_sms ? items : a.num_sms;
-    e = a.kscale ? launch_pdl(indexer_fp8_kernel, dim3(grid), dim3(IX_THREADS), IX8_SMEM, stream, tm_k, a.q_idx, ia)
-                 : launch_pdl(indexer_kernel, dim3(grid), dim3(IX_THREADS), IX_SMEM, stream, tm_k, tm_q, ia);
+    e = fp8 ? launch_pdl(indexer_kernel<true>, dim3(grid), dim3(IX_THREADS), IxCfg<true>::SMEM, stream, tm_k, tm_q, ia)
+            : launch_pdl(indexer_kernel<false>, dim3(grid), dim3(IX_THREADS), IxCfg<false>::SMEM, stream, tm_k, tm_q, ia);
     if (e != cudaSuccess) return e;
 
     TopkArgs ta{a.scores, a.seq_lens, a.hist, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k,

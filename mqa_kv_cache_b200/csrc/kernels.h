@@ -145,10 +145,12 @@ struct DsaIndexArgs {
     int32_t* tok_count = nullptr;
     int L_tok = 0;  // token capacity of a row (seq_lens beyond it are clamped and flagged)
     // FP8 (kscale non-null): tm_k maps the key codes [B][L_max][128] uint8 with a {128, 128, 1}
-    // box and 128-byte swizzle; kscale [B][L_max] fp32 holds each key's scale; the kernel
-    // quantises the query heads q_idx [B][64][128] bf16 itself (tm_q is not used).
+    // box and 128-byte swizzle, kscale [B][L_max] fp32 holds each key's scale; the launch
+    // first quantises the query heads into q8 / q8_scale, which tm_q maps ({128, 64, 1} box).
     const float* kscale = nullptr;
-    const kvattn_bf16* q_idx = nullptr;
+    const kvattn_bf16* q_idx = nullptr;  // FP8: the bf16 query heads [B][64][128], quantised into q8 / q8_scale
+    uint8_t* q8 = nullptr;               // FP8: [B][64][128] codes (tm_q maps them)
+    float* q8_scale = nullptr;           // FP8: [B][64]
     // [B][2048] first-digit counts of the top-k: zero on entry, the indexer adds to them, the
     // top-k reads them instead of its first pass and leaves them zero; null = the top-k counts
     uint32_t* hist = nullptr;

@@ -80,6 +80,7 @@ __global__ void __launch_bounds__(LQ_WARPS * 32) latent_quant_kernel(const kvatt
 __global__ void __launch_bounds__(256) idx_key_quant_kernel(const kvattn_bf16* src, long long n_rows, uint8_t* codes,
                                                             float* scales)
 {
+    pdl_trigger();  // a following kernel launched with programmatic serialisation may set up early
     const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
     const int l = threadIdx.x & 15;
     const unsigned half = 0xffffu << (threadIdx.x & 16);
