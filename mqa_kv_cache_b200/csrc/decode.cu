@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
         int it = 0, np = 0;
         bool ok = true;
         const uint32_t q_bytes = static_cast<uint32_t>(a.g) * D * 2;
+        const uint64_t pol = l2_evict_first_policy();  // K and V are read once
         for (; ok && w.U < hi && w.b < a.B; walk_next(w, a.B, a.Hk, s_n, N, G)) {
             long long tb, te;
             if (!piece_tiles(w, s_n[w.b], lo, hi, tb, te)) continue;
@@ -353,8 +354,10 @@ __global__ void __launch_bounds__(threads_of(GATHER), 1)
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
 #pragma unroll
                     for (int h = 0; h < C::HALVES; ++h) {
-                        tma_load_3d(kd + h * (TILE * 128), &tm_k, &full[s], h * 64, static_cast<int>(t * TILE), z);
-                        tma_load_3d(vd + h * (TILE * 128), &tm_v, &full[s], h * 64, static_cast<int>(t * TILE), z);
+                        tma_load_3d_hint(kd + h * (TILE * 128), &tm_k, &full[s], h * 64, static_cast<int>(t * TILE), z,
+                                         pol);
+                        tma_load_3d_hint(vd + h * (TILE * 128), &tm_v, &full[s], h * 64, static_cast<int>(t * TILE), z,
+                                         pol);
                     }
                 } else {
                     const int rb = static_cast<int>(t - chunk_t0) * TILE;

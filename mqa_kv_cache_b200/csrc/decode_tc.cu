@@ -211,6 +211,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (active && warp == 0) {
         // ===== TMA producer: Q of each piece, then K and V of each tile =====
         if (lane == 0) {
+            const uint64_t pol = l2_evict_first_policy();  // K and V are read once
             Walk w = w_start;
             int it = 0, np = 0;
             bool ok = true;
@@ -241,16 +242,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     }
                     mbar_arrive_expect_tx(&kfull[ks], TC_TILE);
                     uint8_t* kd = smem + TC_OFF_K + ks * TC_TILE;
-                    tma_load_3d(kd, &tm_k, &kfull[ks], 0, row, z);
-                    tma_load_3d(kd + TC_BOX, &tm_k, &kfull[ks], 64, row, z);
+                    tma_load_3d_hint(kd, &tm_k, &kfull[ks], 0, row, z, pol);
+                    tma_load_3d_hint(kd + TC_BOX, &tm_k, &kfull[ks], 64, row, z, pol);
                     if (it >= TC_VS && (*s_abort || !mbar_wait(&vempty[vs], ((it / TC_VS) - 1) & 1))) {
                         ok = false;
                         break;
                     }
                     mbar_arrive_expect_tx(&vfull[vs], TC_TILE);
                     uint8_t* vd = smem + TC_OFF_V + vs * TC_TILE;
-                    tma_load_3d(vd, &tm_v, &vfull[vs], 0, row, z);
-                    tma_load_3d(vd + TC_BOX, &tm_v, &vfull[vs], 64, row, z);
+                    tma_load_3d_hint(vd, &tm_v, &vfull[vs], 0, row, z, pol);
+                    tma_load_3d_hint(vd + TC_BOX, &tm_v, &vfull[vs], 64, row, z, pol);
                 }
                 ++np;
             }

@@ -158,13 +158,6 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                  : "memory");
 }
 
-__device__ __forceinline__ int ld_acquire_gpu(const int* p)
-{
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 // One (head, 16-byte column chunk) of the merge of a row's C parts: out = sum_c
 // 2^(lse_c - LSE) o_c, LSE = log2 sum_c 2^lse_c (log2 units; lse written in natural log).
 __device__ __forceinline__ void merge_one(const SparseArgs& a, int b, int h, int j)

@@ -53,17 +53,32 @@ def test_group_sizes(K, d, g, Hk):
     assert_attn_close(out, ro, lse, rl, f"g={g} Hk={Hk} d={d}")
 
 
-def test_edge_lengths_and_empty(K):
-    lens = torch.tensor([0, 1, 63, 64, 65, 127, 128, 129, 1000, 999, 2], dtype=torch.int32)
-    B, H, Hk, d, T_max = len(lens), 8, 2, 128, 1000
-    gen = W.generator(42)
+@pytest.mark.parametrize("H,Hk", [(8, 2), (64, 1), (128, 2)])
+def test_edge_lengths_and_empty(K, H, Hk):
+    # 64 query heads per KV head: the tcgen05 kernel, whose combine pass also writes
+    # the empty sequences
+    lens = torch.tensor([0, 1, 63, 64, 65, 127, 128, 129, 1000, 999, 0, 2], dtype=torch.int32)
+    B, d, T_max = len(lens), 128, 1000
+    gen = W.generator(42 + H)
     q = W.normal_bf16((B, H, d), gen)
     k = W.normal_bf16((B, Hk, T_max, d), gen)
     v = W.normal_bf16((B, Hk, T_max, d), gen)
     out, lse = _run(K, q, k, v, lens, d ** -0.5)
     ro, rl = _oracle(q, k, v, lens, d ** -0.5)
-    assert torch.all(out[0].float() == 0) and torch.all(torch.isneginf(lse[0]))
+    for b in (0, 10):
+        assert torch.all(out[b].float() == 0) and torch.all(torch.isneginf(lse[b]))
     assert_attn_close(out, ro, lse, rl, "edge lengths")
+
+
+@pytest.mark.parametrize("H,Hk", [(8, 2), (64, 1)])
+def test_all_sequences_empty(K, H, Hk):
+    B, d, T_max = 5, 128, 256
+    gen = W.generator(43)
+    q = W.normal_bf16((B, H, d), gen)
+    k = W.normal_bf16((B, Hk, T_max, d), gen)
+    v = W.normal_bf16((B, Hk, T_max, d), gen)
+    out, lse = _run(K, q, k, v, torch.zeros(B, dtype=torch.int32), d ** -0.5)
+    assert torch.all(out.float() == 0) and torch.all(torch.isneginf(lse))
 
 
 @pytest.mark.parametrize("H,Hk", [(16, 2), (64, 1)])
