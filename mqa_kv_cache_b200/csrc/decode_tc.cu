@@ -8,15 +8,17 @@
 // which is the tcgen05 rate, not the mma.sync one.
 //
 // Per 64-key tile: S = Q K^T with M = 64 heads (rows in TMEM lanes 0-15 of
-// each 32-lane quarter), N = 64 keys, K = 128, double-buffered in TMEM so the
-// next tile's scores are computed while this one's softmax runs; the
+// each 32-lane quarter), N = 64 keys, K = 128, in one of three TMEM buffers so
+// that the next tiles' scores are computed while this one's softmax runs; the
 // softmax (four warps reading their 16 lanes with the 16x256b shape, so that
 // all 32 threads work: a head's keys spread over a lane quad, two heads per
-// thread) writes P as bf16 into a swizzled shared-memory tile and O += P V runs as a second MMA into a
-// 128-column TMEM accumulator.  Warp 0 streams Q (per piece) and the K and V
-// tiles through separate TMA rings (a K slot is released as soon as its S MMA
-// is done, a V slot after its P V); warp 1 issues the S MMAs (and owns TMEM),
-// warp 6 the P V MMAs, so neither waits for the other's operands.
+// thread) writes P as bf16 into a swizzled shared-memory tile and O += P V runs
+// as a second MMA into a 128-column TMEM accumulator.  Warp 0 streams Q (per
+// piece) and the K tiles, warp 7 the V tiles, through separate TMA rings (a K
+// slot is released as soon as its S MMA is done, a V slot after its P V, one
+// tile later: with one producer for both, a full V ring would hold back K);
+// warp 1 issues the S MMAs (and owns TMEM), warp 6 the P V MMAs, so neither
+// waits for the other's operands.
 #include "common.cuh"
 #include "decode_plan.cuh"
 #include "kernels.h"
@@ -28,15 +30,15 @@ namespace {
 constexpr int TC_T = DEC_TILE;            // keys per tile (64)
 constexpr int TC_D = 128;                 // head dim
 constexpr int TC_M = 64;                  // query heads per MMA
-constexpr int TC_KS = 4;                  // K ring slots
-constexpr int TC_VS = 6;                  // V ring slots
+constexpr int TC_KS = 5;                  // K ring slots
+constexpr int TC_VS = 5;                  // V ring slots
 constexpr int TC_BOX = TC_T * 128;        // 8 KB: 64 rows x one 64-wide d block
 constexpr int TC_TILE = 2 * TC_BOX;       // 16 KB: a K or V tile [64 x 128]
 constexpr int TC_QBOX = TC_M * 128;       // 8 KB
 constexpr int TC_PBYTES = TC_M * 128;     // 8 KB: P tile [64 heads x 64 keys] bf16
-constexpr int TC_THREADS = 224;           // w0 TMA, w1 S MMAs + TMEM, w2-5 softmax, w6 P V MMAs
-constexpr int TC_NB = 2;                  // S and P buffers (a third one measured no faster)
-constexpr int TC_TMEM_COLS = 256;         // S0 | S1 (64 columns each) | O (128)
+constexpr int TC_THREADS = 256;           // w0 Q + K loads, w1 S MMAs + TMEM, w2-5 softmax, w6 P V MMAs, w7 V loads
+constexpr int TC_NB = 3;                  // S and P buffers
+constexpr int TC_TMEM_COLS = 512;         // S0 | S1 | S2 (64 columns each) | O (128), rounded up to a power of 2
 constexpr int TC_OCOL = TC_NB * TC_T;
 constexpr uint32_t TC_IDESC_S = umma_idesc_bf16(TC_M, TC_T);             // Q x K^T
 constexpr uint32_t TC_IDESC_O = umma_idesc_bf16(TC_M, TC_D, false, true);  // P x V (V MN-major)
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     bulk_load(sSin, a.sin_tab + static_cast<long long>(qp) * (TC_D / 2), TC_D * 2, q_full);
                 }
                 for (long long t = tb; t < te; ++t, ++it) {
-                    const int ks = it % TC_KS, vs = it % TC_VS;
+                    const int ks = it % TC_KS;
                     const int row = static_cast<int>(t * TC_T);
                     if (it >= TC_KS && (*s_abort || !mbar_wait(&kempty[ks], ((it / TC_KS) - 1) & 1))) {
                         ok = false;
@@ -244,14 +246,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     uint8_t* kd = smem + TC_OFF_K + ks * TC_TILE;
                     tma_load_3d_hint(kd, &tm_k, &kfull[ks], 0, row, z, pol);
                     tma_load_3d_hint(kd + TC_BOX, &tm_k, &kfull[ks], 64, row, z, pol);
-                    if (it >= TC_VS && (*s_abort || !mbar_wait(&vempty[vs], ((it / TC_VS) - 1) & 1))) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&vfull[vs], TC_TILE);
-                    uint8_t* vd = smem + TC_OFF_V + vs * TC_TILE;
-                    tma_load_3d_hint(vd, &tm_v, &vfull[vs], 0, row, z, pol);
-                    tma_load_3d_hint(vd + TC_BOX, &tm_v, &vfull[vs], 64, row, z, pol);
                 }
                 ++np;
             }
@@ -261,6 +255,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             // copies still in flight complete before the CTA leaves (bounded waits)
             for (int j = it - TC_KS > 0 ? it - TC_KS : 0; j < it; ++j) mbar_wait(&kfull[j % TC_KS], (j / TC_KS) & 1);
+        }
+    } else if (active && warp == 7) {
+        // ===== V loads: their own ring and pace (a V slot frees one tile later than a K slot,
+        // after the P V; tied to the K loads, V would hold back K) =====
+        if (lane == 0) {
+            const uint64_t pol = l2_evict_first_policy();
+            TileStream ts{w_start};
+            bool ok = true, first = false;
+            int it = 0;
+            for (; ts.next(lo, hi, a.B, a.Hk, s_n, N, G, first); ++it) {
+                const int vs = it % TC_VS;
+                if (it >= TC_VS && (*s_abort || !mbar_wait(&vempty[vs], ((it / TC_VS) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                const int z = ts.w.b * a.Hk + ts.w.kvh;
+                const int row = static_cast<int>((ts.t_cur - 1) * TC_T);
+                mbar_arrive_expect_tx(&vfull[vs], TC_TILE);
+                uint8_t* vd = smem + TC_OFF_V + vs * TC_TILE;
+                tma_load_3d_hint(vd, &tm_v, &vfull[vs], 0, row, z, pol);
+                tma_load_3d_hint(vd + TC_BOX, &tm_v, &vfull[vs], 64, row, z, pol);
+            }
+            if (!ok) {
+                *s_abort = 1;
+                report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            }
             for (int j = it - TC_VS > 0 ? it - TC_VS : 0; j < it; ++j) mbar_wait(&vfull[j % TC_VS], (j / TC_VS) & 1);
         }
     } else if (active && warp == 1) {
