@@ -358,6 +358,56 @@ __device__ __forceinline__ int block_incl_scan(int v, int* s_warp)
     return r;
 }
 
+// An exact block-wide (TK_THREADS threads) selection among n values x_i = v[i] (~v[i]
+// with invert), of those with f[i] == fval when f is given and with x_i & known == prefix:
+// the need-th largest, its digits below `known` found by passes of 11 bits from bit
+// `top` down (the last pass takes what is left).  Returns it; *left = how many values
+// equal to it are still needed, *n_eq = how many equal it.
+__device__ uint32_t block_select(const uint32_t* v, bool invert, const uint32_t* f, uint32_t fval, int n,
+                                 uint32_t prefix, uint32_t known, int need, int top, uint32_t* hist, int* s_warp,
+                                 uint32_t* s_sel, int* left, int* n_eq)
+{
+    const int tid = threadIdx.x;
+    int eq = 0;
+    for (int sh = top; sh > -11; sh -= 11) {
+        const int lo_bit = sh < 0 ? 0 : sh;
+        const int nb = 1 << (sh < 0 ? 11 + sh : 11);
+        const uint32_t mask = static_cast<uint32_t>(nb - 1);
+        for (int i = tid; i < nb; i += TK_THREADS) hist[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < n; i += TK_THREADS) {
+            const uint32_t x = invert ? ~v[i] : v[i];
+            if ((x & known) == prefix && (f == nullptr || f[i] == fval)) atomicAdd(&hist[(x >> lo_bit) & mask], 1u);
+        }
+        __syncthreads();
+        const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
+        const int c0 = d0 >= 0 ? static_cast<int>(hist[d0]) : 0, c1 = d1 >= 0 ? static_cast<int>(hist[d1]) : 0;
+        const int incl = block_incl_scan(c0 + c1, s_warp);
+        const int before = incl - c0 - c1;
+        if (d0 >= 0 && before < need && before + c0 >= need) {
+            s_sel[0] = static_cast<uint32_t>(d0);
+            s_sel[1] = static_cast<uint32_t>(need - before);
+        } else if (d1 >= 0 && before + c0 < need && before + c0 + c1 >= need) {
+            s_sel[0] = static_cast<uint32_t>(d1);
+            s_sel[1] = static_cast<uint32_t>(need - before - c0);
+        }
+        __syncthreads();
+        prefix |= s_sel[0] << lo_bit;
+        known |= mask << lo_bit;
+        need = static_cast<int>(s_sel[1]);
+        eq = static_cast<int>(hist[s_sel[0]]);
+        __syncthreads();  // hist is cleared by the next pass
+        if (lo_bit == 0) break;
+    }
+    *left = need;
+    *n_eq = eq;
+    return prefix;
+}
+
+struct TopkArgs;
+__device__ void write_tail(const TopkArgs& a, int row, int rank, int len, int n_sel, int32_t* out, int32_t* tout,
+                           int width, int gs);
+
 struct TopkArgs {
     const float* scores;
     const int32_t* seq_lens;
@@ -372,17 +422,46 @@ struct TopkArgs {
 };
 
 constexpr int TK_SLICE_MAX = 16384;  // keys per CTA held in shared memory
+// Keys of the row whose first digit is the threshold's, gathered into rank 0's shared
+// memory (key, index) for the rest of the selection; more than this many take the
+// cluster-wide passes instead.
+constexpr int TK_CAND_MAX = 16384;
 // Key i of the slice sits at word i + i / 16: a thread's run of 16 keys then
 // starts in its own bank, so the runs of a warp are read without conflicts.
 __device__ __forceinline__ int kpad(int i) { return i + (i >> 4); }
 constexpr int TK_SLICE_WORDS = TK_SLICE_MAX + TK_SLICE_MAX / 16;
+
+// Words of a CTA's key slice (kpad layout) for rows of L_max scores.
+__host__ __device__ constexpr int slice_words(int L_max)
+{
+    return (L_max + TK_CL - 1) / TK_CL + ((L_max + TK_CL - 1) / TK_CL >> 4) + 1;
+}
+
+// After the n_sel selected entries of a row: -1 (fewer than k only when NaN scores were
+// skipped); in groups mode the row's trailing tokens come first.  Rank 0 writes it.
+__device__ void write_tail(const TopkArgs& a, int row, int rank, int len, int n_sel, int32_t* out, int32_t* tout,
+                           int width, int gs)
+{
+    if (rank != 0) return;
+    const int tid = threadIdx.x;
+    if (tout) {
+        const int tok_raw = a.seq_lens[row];
+        const int tok_len = min(max(tok_raw, 0), a.L_tok);
+        if (tok_len != tok_raw && tid == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
+        const int tail0 = len * gs, n_tail = max(tok_len - tail0, 0), first = n_sel * gs;
+        for (int j = first + tid; j < width; j += TK_THREADS) tout[j] = j - first < n_tail ? tail0 + (j - first) : -1;
+        if (tid == 0) a.tok_count[row] = first + n_tail;
+    } else {
+        for (int j = n_sel + tid; j < a.k; j += TK_THREADS) out[j] = -1;
+    }
+}
 
 __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
 {
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
     const int row = blockIdx.x / TK_CL;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
 
     extern __shared__ uint32_t s_keys[];  // this CTA's slice as keys (TK_SLICE_MAX at most), kpad layout
     __shared__ uint32_t hist2[2][2048];  // per-pass histograms, alternating (see below)
@@ -404,9 +483,31 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     const float* sc = a.scores + static_cast<long long>(row) * a.L_max;
     if (tid == 0) s_nan = 0;
     bool nan = false;
-    // keys of the slice -> shared memory (one read of the scores)
-    for (int i = tid; i < n_mine; i += TK_THREADS) s_keys[kpad(i)] = score_key(sc[lo + i], nan);
+    // the candidate counter in rank 0 is zero before any CTA of the cluster counts into it
+    __shared__ int s_cand_n;
+    __shared__ int s_gt1[TK_CL];       // rank 0: per rank, its keys above the threshold's first digit
+    __shared__ int s_rsel[TK_CL];      // rank 0: per rank, its selected candidates
+    __shared__ uint32_t s_bcast[4];    // from rank 0: T, last index taken among keys == T, first position, total
+    if (tid == 0) s_cand_n = 0;
     __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    // keys of the slice -> shared memory (one read of the scores, 16 loads in flight per thread)
+    constexpr int TK_U = 16;
+    for (int base = 0; base < n_mine; base += TK_THREADS * TK_U) {
+        float v[TK_U];
+#pragma unroll
+        for (int u = 0; u < TK_U; ++u) {
+            const int i = base + u * TK_THREADS + tid;
+            v[u] = i < n_mine ? __ldcg(sc + lo + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < TK_U; ++u) {
+            const int i = base + u * TK_THREADS + tid;
+            if (i < n_mine) s_keys[kpad(i)] = score_key(v[u], nan);
+        }
+    }
+    __syncthreads();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 
     // ---- radix select: the (k)-th largest key T, and how many keys equal to T to take ----
     uint32_t prefix = 0u, known = 0u;
@@ -465,6 +566,111 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
             prefix |= s_sel[0] << sh;
             k_rem = static_cast<int>(s_sel[1]);
             known |= static_cast<uint32_t>(nb - 1) << sh;
+            if (p == 0) {
+                // ---- the keys with the threshold's first digit, (key, index), into rank 0 ----
+                const uint32_t b1 = prefix >> TK_SHIFT0;
+                const int key_words = slice_words(a.L_max);
+                uint32_t* cand_key = s_keys + key_words;
+                uint32_t* cand_idx = cand_key + TK_CAND_MAX;
+                int* cnt0 = cluster.map_shared_rank(&s_cand_n, 0);
+                uint32_t* ck0 = cluster.map_shared_rank(cand_key, 0);
+                uint32_t* ci0 = cluster.map_shared_rank(cand_idx, 0);
+                int n_gt1 = 0;
+                for (int base = 0; base < n_mine; base += TK_THREADS) {
+                    const int i = base + tid;
+                    const uint32_t key = i < n_mine ? s_keys[kpad(i)] : 0u;
+                    const uint32_t d = key >> TK_SHIFT0;
+                    n_gt1 += i < n_mine && d > b1;
+                    const bool in = i < n_mine && d == b1;
+                    const uint32_t m = __ballot_sync(0xffffffffu, in);
+                    if (m) {
+                        const int leader = __ffs(m) - 1;
+                        int off = 0;
+                        if (lane == leader) off = atomicAdd(cnt0, __popc(m));
+                        off = __shfl_sync(0xffffffffu, off, leader);
+                        const int pos = off + __popc(m & ((1u << lane) - 1u));
+                        if (in && pos < TK_CAND_MAX) {
+                            ck0[pos] = key;
+                            ci0[pos] = static_cast<uint32_t>(lo + i);
+                        }
+                    }
+                }
+                const int gt_all = block_incl_scan(n_gt1, s_warp);
+                if (tid == TK_THREADS - 1) *cluster.map_shared_rank(&s_gt1[rank], 0) = gt_all;
+                cluster.sync();
+                const int n_c = *cnt0;
+                if (n_c <= TK_CAND_MAX) {
+                    // every CTA has read the row's first-digit counts: leave them zero
+                    if (a.hist && rank == 0)
+                        for (int i = tid; i < TK_DIGITS0; i += TK_THREADS)
+                            a.hist[static_cast<long long>(row) * TK_DIGITS0 + i] = 0u;
+                    if (rank == 0) {
+                        // T = the k_rem-th largest candidate; among the candidates equal to T
+                        // (T != 0: NaN keys are 0 and never taken) the `left` lowest indices
+                        int left = 0, n_eq = 0, l2 = 0, e2 = 0;
+                        const uint32_t T = block_select(cand_key, false, nullptr, 0u, n_c, prefix, known, k_rem,
+                                                        TK_SHIFT0 - 11, hist2[0], s_warp, s_sel, &left, &n_eq);
+                        uint32_t cut = 0x7fffffffu;  // last index taken among the keys equal to T
+                        if (T != 0u && left < n_eq)
+                            cut = ~block_select(cand_idx, true, cand_key, T, n_c, 0x80000000u, 0x80000000u, left, 20,
+                                                hist2[1], s_warp, s_sel, &l2, &e2);
+                        if (tid < TK_CL) s_rsel[tid] = 0;
+                        __syncthreads();
+                        for (int i = tid; i < n_c; i += TK_THREADS) {
+                            const uint32_t key = cand_key[i], idx = cand_idx[i];
+                            if (key > T || (T != 0u && key == T && idx <= cut))
+                                atomicAdd(&s_rsel[static_cast<int>(idx) / slice], 1);
+                        }
+                        __syncthreads();
+                        if (tid == 0) {
+                            uint32_t first = 0u;
+                            for (int q = 0; q < TK_CL; ++q) first += static_cast<uint32_t>(s_gt1[q] + s_rsel[q]);
+                            const uint32_t total = first;
+                            first = 0u;
+                            for (int q = 0; q < TK_CL; ++q) {
+                                uint32_t* bq = cluster.map_shared_rank(s_bcast, q);
+                                bq[0] = T;
+                                bq[1] = cut;
+                                bq[2] = first;
+                                bq[3] = total;
+                                first += static_cast<uint32_t>(s_gt1[q] + s_rsel[q]);
+                            }
+                        }
+                    }
+                    cluster.sync();
+                    // ---- ordered compaction: each thread owns a contiguous run of the slice ----
+                    const uint32_t Tf = s_bcast[0], cut = s_bcast[1];
+                    const int run = (n_mine + TK_THREADS - 1) / TK_THREADS;
+                    const int r0 = min(tid * run, n_mine), r1 = min(r0 + run, n_mine);
+                    int n_take = 0;
+                    for (int i = r0; i < r1; ++i) {
+                        const uint32_t key = s_keys[kpad(i)];
+                        n_take += key > Tf || (Tf != 0u && key == Tf && static_cast<uint32_t>(lo + i) <= cut);
+                    }
+                    const int inc = block_incl_scan(n_take, s_warp);
+                    int pos = static_cast<int>(s_bcast[2]) + inc - n_take;
+                    const int gs = 1 << a.len_shift;
+                    const int width = a.k * gs + gs - 1;
+                    int32_t* out = a.out ? a.out + static_cast<long long>(row) * a.k : nullptr;
+                    int32_t* tout = a.tok_out ? a.tok_out + static_cast<long long>(row) * width : nullptr;
+                    for (int i = r0; i < r1; ++i) {
+                        const uint32_t key = s_keys[kpad(i)];
+                        if (key > Tf || (Tf != 0u && key == Tf && static_cast<uint32_t>(lo + i) <= cut)) {
+                            if (tout) {
+                                for (int r = 0; r < gs; ++r) tout[pos * gs + r] = (lo + i) * gs + r;
+                            } else {
+                                out[pos] = lo + i;
+                            }
+                            ++pos;
+                        }
+                    }
+                    write_tail(a, row, rank, len, static_cast<int>(s_bcast[3]), out, tout, width, gs);
+                    if (nan) s_nan = 1;
+                    __syncthreads();
+                    if (s_nan && tid == 0) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
+                    return;
+                }
+            }
         }
     }
     // With len <= k everything is taken: T = 0 selects every number (NaN keys are 0).
@@ -522,21 +728,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
             ++pos;
         }
     }
-    // -1 after the selected entries (fewer than kk only when NaN scores were skipped);
-    // in groups mode the row's trailing tokens come first
-    const int n_sel = gt_total + min(max(take_eq, 0), eq_total);
-    if (rank == 0) {
-        if (tout) {
-            const int tok_raw = a.seq_lens[row];
-            const int tok_len = min(max(tok_raw, 0), a.L_tok);
-            if (tok_len != tok_raw && tid == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
-            const int tail0 = len * gs, n_tail = max(tok_len - tail0, 0), first = n_sel * gs;
-            for (int j = first + tid; j < width; j += TK_THREADS) tout[j] = j - first < n_tail ? tail0 + (j - first) : -1;
-            if (tid == 0) a.tok_count[row] = first + n_tail;
-        } else {
-            for (int j = n_sel + tid; j < a.k; j += TK_THREADS) out[j] = -1;
-        }
-    }
+    write_tail(a, row, rank, len, gt_total + min(max(take_eq, 0), eq_total), out, tout, width, gs);
     if (nan) s_nan = 1;
     __syncthreads();
     if (s_nan && tid == 0) report_status(a.dev_status, KVATTN_STATUS_NAN_SCORE);
@@ -726,12 +918,11 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
 
     TopkArgs ta{a.scores, a.seq_lens, a.hist, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k,
                 a.len_shift, a.tok_idx, a.tok_count, a.L_tok};
-    const int slice_max = (a.L_max + TK_CL - 1) / TK_CL;
-    const size_t key_bytes = static_cast<size_t>(slice_max + (slice_max >> 4) + 1) * sizeof(uint32_t);
+    const size_t key_bytes = static_cast<size_t>(slice_words(a.L_max) + 2 * TK_CAND_MAX) * sizeof(uint32_t);
     static bool tk_attr[64] = {};
     if (dev < 64 && !tk_attr[dev]) {
         e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (TK_SLICE_WORDS + 1) * static_cast<int>(sizeof(uint32_t)));
+                                 (TK_SLICE_WORDS + 1 + 2 * TK_CAND_MAX) * static_cast<int>(sizeof(uint32_t)));
         if (e != cudaSuccess) return e;
         tk_attr[dev] = true;
     }
