@@ -575,25 +575,29 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
                 int* cnt0 = cluster.map_shared_rank(&s_cand_n, 0);
                 uint32_t* ck0 = cluster.map_shared_rank(cand_key, 0);
                 uint32_t* ci0 = cluster.map_shared_rank(cand_idx, 0);
-                int n_gt1 = 0;
+                // two passes over the slice: count per warp, one remote add per warp for its
+                // place in rank 0's list, then the stores
+                int n_gt1 = 0, w_total = 0;
                 for (int base = 0; base < n_mine; base += TK_THREADS) {
                     const int i = base + tid;
-                    const uint32_t key = i < n_mine ? s_keys[kpad(i)] : 0u;
-                    const uint32_t d = key >> TK_SHIFT0;
+                    const uint32_t d = i < n_mine ? s_keys[kpad(i)] >> TK_SHIFT0 : 0u;
                     n_gt1 += i < n_mine && d > b1;
-                    const bool in = i < n_mine && d == b1;
+                    w_total += __popc(__ballot_sync(0xffffffffu, i < n_mine && d == b1));
+                }
+                int w_pos = 0;
+                if (lane == 0 && w_total > 0) w_pos = atomicAdd(cnt0, w_total);
+                w_pos = __shfl_sync(0xffffffffu, w_pos, 0);
+                for (int base = 0; base < n_mine && w_total > 0; base += TK_THREADS) {
+                    const int i = base + tid;
+                    const uint32_t key = i < n_mine ? s_keys[kpad(i)] : 0u;
+                    const bool in = i < n_mine && (key >> TK_SHIFT0) == b1;
                     const uint32_t m = __ballot_sync(0xffffffffu, in);
-                    if (m) {
-                        const int leader = __ffs(m) - 1;
-                        int off = 0;
-                        if (lane == leader) off = atomicAdd(cnt0, __popc(m));
-                        off = __shfl_sync(0xffffffffu, off, leader);
-                        const int pos = off + __popc(m & ((1u << lane) - 1u));
-                        if (in && pos < TK_CAND_MAX) {
-                            ck0[pos] = key;
-                            ci0[pos] = static_cast<uint32_t>(lo + i);
-                        }
+                    const int pos = w_pos + __popc(m & ((1u << lane) - 1u));
+                    if (in && pos < TK_CAND_MAX) {
+                        ck0[pos] = key;
+                        ci0[pos] = static_cast<uint32_t>(lo + i);
                     }
+                    w_pos += __popc(m);
                 }
                 const int gt_all = block_incl_scan(n_gt1, s_warp);
                 if (tid == TK_THREADS - 1) *cluster.map_shared_rank(&s_gt1[rank], 0) = gt_all;
