@@ -343,7 +343,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const int kbase = j * PF_BN;
                 // Pass 1: row max of the raw scores (scale > 0 commutes with the max): the four
                 // 32-column loads are in flight together, one wait.
-                float mx = -INFINITY;
+                float mxc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
                 {
                     uint32_t sv[4][32];
 #pragma unroll
@@ -369,10 +369,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         }
 #pragma unroll
                         for (int i = 0; i < 32; i += 2)
-                            mx = fmax3(mx, __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
+                            mxc[c] = fmax3(mxc[c], __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
                     }
                 }
-                mx *= sl2;
+                float mx = fmaxf(fmaxf(mxc[0], mxc[1]), fmaxf(mxc[2], mxc[3])) * sl2;
                 // Move this row's reference max only when it grows by more than 2^8.
                 // The O rescale uses warp-collective TMEM loads/stores, so the
                 // warp takes that path together (alpha = 1 for rows that keep
@@ -396,7 +396,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 m_run = m_new;
                 const float mu = m_run == -INFINITY ? 0.f : m_run;
                 const float2 sc2 = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
-                float2 acc = make_float2(0.f, 0.f);
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f)};  // four independent sums
                 // Pass 2: p = 2^(s * scale * log2 e - m) -> bf16 P over the first 64 S
                 // columns (chunk c's P lands in columns 16c..16c+15, all already read).
                 // Chunk c + 1 is loaded while chunk c is processed.
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                             pr.x = fast_exp2(x.x);
                             pr.y = fast_exp2(x.y);
                         }
-                        acc = __fadd2_rn(acc, pr);
+                        acc[i & 3] = __fadd2_rn(acc[i & 3], pr);
                         pk[i] = pack_bf16x2(pr.x, pr.y);
                     }
                     asm volatile(
@@ -450,7 +451,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         tmem_regs_ready(sb[(c + 1) & 1]);
                     }
                 }
-                const float ls = acc.x + acc.y;
+                const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
+                const float ls = (a01.x + a01.y) + (a23.x + a23.y);
                 l_run += ls;
                 tmem_wait_st();
                 tc_fence_before();
