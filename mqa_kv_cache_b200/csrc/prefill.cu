@@ -11,9 +11,12 @@
 // CTA = (batch, query head, block of 256 query rows) = two 128-row Q tiles that
 // share every K/V tile, so the softmax of one tile overlaps the MMAs of the
 // other.  Warps 0-3 / 4-7: softmax of Q tile 0 / 1, one thread per query row
-// (a full score row per thread: row max and sum need no shuffles); warp 8: the
-// single MMA-issuing thread; warp 9: TMA loads (Q once, then K_j, V_j through a
-// 4-slot ring).  TMEM (512 columns): S0 | S1 | O0 | O1, 128 columns each.
+// (a full score row per thread, all 128 scores in registers: row max and sum need
+// no shuffles and the scores are read from TMEM once); warp 8: the single
+// MMA-issuing thread; warp 9: TMA loads (Q once, then K_j, V_j through a 4-slot
+// ring); warps 10-11 idle, so that warps 8-11 form a warpgroup that hands its
+// registers to the softmax warpgroups (setmaxnreg).  TMEM (512 columns):
+// S0 | S1 | O0 | O1, 128 columns each.
 // The softmax writes P (bf16, two per 32-bit column) over the first 64 columns
 // of its S buffer and the P V product takes P straight from TMEM.  The running
 // max is only moved (and O rescaled) when it grows by more than 2^8, so most
@@ -30,7 +33,7 @@ constexpr int PF_BM = 128;    // query rows per Q tile
 constexpr int PF_BN = 128;    // keys per K/V tile
 static_assert(PF_BM == PREFILL_Q_ROWS && PF_BN == PREFILL_KV_ROWS, "tensor map boxes");
 constexpr int PF_SLOTS = 4;   // K/V ring slots (one tile each)
-constexpr int PF_THREADS = 320;
+constexpr int PF_THREADS = 384;  // w0-7 softmax, w8 MMA, w9 TMA, w10-11 idle (a whole warpgroup for setmaxnreg)
 constexpr int PF_TILE = PF_BN * PF_D * 2;  // 32 KB: one K or V tile, two 64-column SW128 boxes
 constexpr int PF_BOX = PF_BN * 128;        // 16 KB
 constexpr int PF_OFF_Q = 0;                // two Q tiles
@@ -132,7 +135,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     pdl_wait();
     pdl_trigger();
 
+    // registers: the softmax warpgroups take 216 each thread, the MMA / TMA warpgroup keeps 56
+    // (2 x 128 x 216 + 128 x 56 = 62464 of the 384 x 168 the block is launched with)
     if (warp == 9) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
         // ===== TMA loads =====
         if (lane == 0) {
             mbar_arrive_expect_tx(q_full, n_qt * PF_TILE);
@@ -181,6 +187,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 mbar_wait(&kv_full[x % PF_SLOTS], (x / PF_SLOTS) & 1);
         }
     } else if (warp == 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
         // ===== MMA issue (one thread) =====
         if (lane == 0) {
             const uint32_t sq = smem_u32(smem + PF_OFF_Q);
@@ -318,7 +325,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             tc_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
-    } else {
+    } else if (warp < 8) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 216;" ::: "memory");
         // ===== softmax + epilogue: warps 0-3 -> Q tile 0, warps 4-7 -> Q tile 1 =====
         const int t = warp >> 2;
         const int quarter = warp & 3;
@@ -341,36 +349,35 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const bool diag = j == dg;  // keys j*128 .. : the diagonal tile
                 const bool band = WINDOW && j * PF_BN <= band_top;
                 const int kbase = j * PF_BN;
-                // Pass 1: row max of the raw scores (scale > 0 commutes with the max): the four
-                // 32-column loads are in flight together, one wait.
+                // The row's 128 raw scores in registers (four 32-column loads in flight, one wait):
+                // the row max (scale > 0 commutes with the max), then the exponentials from the
+                // same registers.
+                uint32_t sv[4][32];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sv[c]);
+                tmem_wait_ld();
                 float mxc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
-                {
-                    uint32_t sv[4][32];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, sv[c]);
-                    tmem_wait_ld();
+                for (int c = 0; c < 4; ++c) {
+                    tmem_regs_ready(sv[c]);
+                    if constexpr (WINDOW) {
+                        if (diag || band) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        tmem_regs_ready(sv[c]);
-                        if constexpr (WINDOW) {
-                            if (diag || band) {
-#pragma unroll
-                                for (int i = 0; i < 32; ++i) {
-                                    const int key = kbase + c * 32 + i;
-                                    // -inf: key after the query, or below its band and not a sink
-                                    if (key > qrow || (band && key <= qrow - a.window && key >= a.n_sink))
-                                        sv[c][i] = 0xff800000u;
-                                }
+                            for (int i = 0; i < 32; ++i) {
+                                const int key = kbase + c * 32 + i;
+                                // -inf: key after the query, or below its band and not a sink
+                                if (key > qrow || (band && key <= qrow - a.window && key >= a.n_sink))
+                                    sv[c][i] = 0xff800000u;
                             }
-                        } else if (diag) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (c * 32 + i > row) sv[c][i] = 0xff800000u;  // -inf: key after the query
                         }
+                    } else if (diag) {
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2)
-                            mxc[c] = fmax3(mxc[c], __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
+                        for (int i = 0; i < 32; ++i)
+                            if (c * 32 + i > row) sv[c][i] = 0xff800000u;  // -inf: key after the query
                     }
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2)
+                        mxc[c] = fmax3(mxc[c], __uint_as_float(sv[c][i]), __uint_as_float(sv[c][i + 1]));
                 }
                 float mx = fmaxf(fmaxf(mxc[0], mxc[1]), fmaxf(mxc[2], mxc[3])) * sl2;
                 // Move this row's reference max only when it grows by more than 2^8.
@@ -383,7 +390,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 if (__any_sync(0xffffffffu, rescale)) {
                     const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.f;
                     l_run *= alpha;
-#pragma unroll
+#pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t ov[32];
                         tmem_ld32(o_addr + c * 32, ov);
@@ -398,36 +405,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 const float2 sc2 = make_float2(sl2, sl2), nmu = make_float2(-mu, -mu);
                 float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                                  make_float2(0.f, 0.f)};  // four independent sums
-                // Pass 2: p = 2^(s * scale * log2 e - m) -> bf16 P over the first 64 S
-                // columns (chunk c's P lands in columns 16c..16c+15, all already read).
-                // Chunk c + 1 is loaded while chunk c is processed.
-                uint32_t sb[2][32];
-                tmem_ld32(s_addr, sb[0]);
-                tmem_wait_ld();
-                tmem_regs_ready(sb[0]);
+                // p = 2^(s * scale * log2 e - m) -> bf16 P over the first 64 S columns (chunk c's
+                // P lands in columns 16c..16c+15; every score is already in registers)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    uint32_t (&sv)[32] = sb[c & 1];
-                    if (c < 3) tmem_ld32(s_addr + (c + 1) * 32, sb[(c + 1) & 1]);
-                    if constexpr (WINDOW) {
-                        if (diag || band) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) {
-                                const int key = kbase + c * 32 + i;
-                                if (key > qrow || (band && key <= qrow - a.window && key >= a.n_sink))
-                                    sv[i] = 0xff800000u;
-                            }
-                        }
-                    } else if (diag) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (c * 32 + i > row) sv[i] = 0xff800000u;
-                    }
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float2 x =
-                            __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sc2, nmu);
+                        const float2 x = __ffma2_rn(
+                            make_float2(__uint_as_float(sv[c][2 * i]), __uint_as_float(sv[c][2 * i + 1])), sc2, nmu);
                         float2 pr;
                         if ((i & 3) == 0) {
                             pr = exp2_fma2(x);  // a quarter of the exponentials off the MUFU pipe
@@ -446,10 +432,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         "r"(pk[7]), "r"(pk[8]), "r"(pk[9]), "r"(pk[10]), "r"(pk[11]), "r"(pk[12]), "r"(pk[13]),
                         "r"(pk[14]), "r"(pk[15])
                         : "memory");
-                    if (c < 3) {
-                        tmem_wait_ld();
-                        tmem_regs_ready(sb[(c + 1) & 1]);
-                    }
                 }
                 const float2 a01 = __fadd2_rn(acc[0], acc[1]), a23 = __fadd2_rn(acc[2], acc[3]);
                 const float ls = (a01.x + a01.y) + (a23.x + a23.y);
@@ -487,6 +469,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
             }
         }
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");  // warps 10-11: idle
     }
     tc_fence_before();
     __syncthreads();
