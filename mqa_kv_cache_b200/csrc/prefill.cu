@@ -285,37 +285,42 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     if (n_qt > 1) issue_s(1, ka);
                     tc_commit(&kv_empty[kslot]);
                 }
+                // Per key tile j: each Q tile's P V, then at once its next scores (S_t shares its
+                // columns with P_t, so the scores wait for that P V), so that Q tile 0's next
+                // scores never wait for Q tile 1's softmax.
                 for (int j = 0; j < n_kv && ok; ++j) {
                     const int vslot = u % PF_SLOTS;
                     ok = mbar_wait(&kv_full[vslot], (u / PF_SLOTS) & 1);
                     ++u;
                     if (!ok) break;
                     const uint32_t va = skv + vslot * PF_TILE;
+                    const bool more = j + 1 < n_kv;
+                    uint32_t ka = 0;
                     for (int t = 0; t < n_qt && ok; ++t) {
-                        if (j >= n_kv0 + t) continue;  // Q tile 0 stops one tile earlier
-                        ok = mbar_wait(&p_full[t], j & 1);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(t, j > 0, va);
-                    }
-                    if (!ok) break;
-                    tc_commit(&kv_empty[vslot]);
-                    if (j + 1 < n_kv) {
-                        kslot = u % PF_SLOTS;
-                        ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
-                        ++u;
-                        if (!ok) break;
-                        const uint32_t ka = skv + kslot * PF_TILE;
-                        for (int t = 0; t < n_qt && ok; ++t) {
-                            if (j + 1 >= n_kv0 + t) continue;
+                        if (j < n_kv0 + t) {  // Q tile 0 stops one tile earlier
+                            ok = mbar_wait(&p_full[t], j & 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(t, j > 0, va);
+                        }
+                        if (more && t == 0) {
+                            kslot = u % PF_SLOTS;
+                            ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
+                            ++u;
+                            if (!ok) break;
+                            ka = skv + kslot * PF_TILE;
+                        }
+                        if (more && j + 1 < n_kv0 + t) {
                             // P_t (read by the P V just issued) shares columns with S_t: wait for it
                             ok = mbar_wait(&pv_done[t], j & 1);
                             if (!ok) break;
                             tc_fence_after();
                             issue_s(t, ka);
                         }
-                        tc_commit(&kv_empty[kslot]);
                     }
+                    if (!ok) break;
+                    tc_commit(&kv_empty[vslot]);
+                    if (more) tc_commit(&kv_empty[kslot]);
                 }
             }
             if (!ok) {
