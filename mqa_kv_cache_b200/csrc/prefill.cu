@@ -135,10 +135,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     pdl_wait();
     pdl_trigger();
 
-    // registers: the softmax warpgroups take 216 each thread, the MMA / TMA warpgroup keeps 56
-    // (2 x 128 x 216 + 128 x 56 = 62464 of the 384 x 168 the block is launched with)
+    // registers: the softmax warpgroups take 216 each thread, the MMA / TMA warpgroup keeps 64
+    // (2 x 128 x 216 + 128 x 64 = 63488 of the 384 x 168 = 64512 the block is launched with;
+    // per SM sub-partition 2 x 32 x 216 + 32 x 64 = 15872 of 16384)
     if (warp == 9) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
         // ===== TMA loads =====
         if (lane == 0) {
             mbar_arrive_expect_tx(q_full, n_qt * PF_TILE);
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                 mbar_wait(&kv_full[x % PF_SLOTS], (x / PF_SLOTS) & 1);
         }
     } else if (warp == 8) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
         // ===== MMA issue (one thread) =====
         if (lane == 0) {
             const uint32_t sq = smem_u32(smem + PF_OFF_Q);
@@ -233,6 +234,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                         if (in_t(t, j)) issue_s(t, ka);
                     tc_commit(&kv_empty[kslot]);
                 }
+                // per key tile: each Q tile's P V, then at once its next scores (as in the plain loop)
                 for (; j <= d_u && ok;) {
                     const int jn = next_in(lo_u, j);
                     const int vslot = u % PF_SLOTS;
@@ -240,24 +242,24 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                     ++u;
                     if (!ok) break;
                     const uint32_t va = skv + vslot * PF_TILE;
+                    const bool more = jn <= d_u;
+                    uint32_t ka = 0;
                     for (int t = 0; t < 2 && ok; ++t) {
-                        if (!in_t(t, j)) continue;
-                        ok = mbar_wait(&p_full[t], cnt[t] & 1);
-                        if (!ok) break;
-                        tc_fence_after();
-                        issue_pv(t, cnt[t] > 0, va);
-                        ++cnt[t];
-                    }
-                    if (!ok) break;
-                    tc_commit(&kv_empty[vslot]);
-                    if (jn <= d_u) {
-                        kslot = u % PF_SLOTS;
-                        ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
-                        ++u;
-                        if (!ok) break;
-                        const uint32_t ka = skv + kslot * PF_TILE;
-                        for (int t = 0; t < 2 && ok; ++t) {
-                            if (!in_t(t, jn)) continue;
+                        if (in_t(t, j)) {
+                            ok = mbar_wait(&p_full[t], cnt[t] & 1);
+                            if (!ok) break;
+                            tc_fence_after();
+                            issue_pv(t, cnt[t] > 0, va);
+                            ++cnt[t];
+                        }
+                        if (more && t == 0) {
+                            kslot = u % PF_SLOTS;
+                            ok = mbar_wait(&kv_full[kslot], (u / PF_SLOTS) & 1);
+                            ++u;
+                            if (!ok) break;
+                            ka = skv + kslot * PF_TILE;
+                        }
+                        if (more && in_t(t, jn)) {
                             // P_t (read by this Q tile's last P V) shares columns with S_t: wait for it
                             if (cnt[t] > 0) {
                                 ok = mbar_wait(&pv_done[t], (cnt[t] - 1) & 1);
@@ -266,8 +268,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
                             }
                             issue_s(t, ka);
                         }
-                        tc_commit(&kv_empty[kslot]);
                     }
+                    if (!ok) break;
+                    tc_commit(&kv_empty[vslot]);
+                    if (more) tc_commit(&kv_empty[kslot]);
                     j = jn;
                 }
             } else {
@@ -475,7 +479,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             }
         }
     } else {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");  // warps 10-11: idle
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");  // warps 10-11: idle
     }
     tc_fence_before();
     __syncthreads();
