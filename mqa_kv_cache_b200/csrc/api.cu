@@ -831,18 +831,23 @@ static int sparse_call(const char* name, const kvattn_bf16* q, const void* laten
     const int chunks = kvattn::sparse_chunks(k);
     int sms = 0;
     if (num_sms_current(&sms) != 0) return fail(KVATTN_ERR_CUDA, "%s: no CUDA device", name);
-    CUtensorMap tm_q, tm_o;
+    CUtensorMap tm_q, tm_o, tm_pm;
     if (make_map_3d(&tm_q, q, Dk, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
     if (chunks == 1) {
         if (make_map_3d(&tm_o, out, Dv, Hq, B, Hq) != KVATTN_OK) return KVATTN_ERR_CUDA;
+        tm_pm = tm_o;  // no merge
     } else {
+        // the chunk parts: stored by their CTAs ({64 columns, Hq heads} boxes), read back by the
+        // in-kernel merge in tiles of 64 columns x 64 heads
         const void* parts = static_cast<const uint8_t*>(workspace) + kvattn::sparse_counter_bytes(B);
         if (make_map_3d(&tm_o, parts, Dv, Hq, static_cast<uint64_t>(B) * chunks, Hq) != KVATTN_OK)
+            return KVATTN_ERR_CUDA;
+        if (make_map_3d(&tm_pm, parts, Dv, Hq, static_cast<uint64_t>(B) * chunks, 64) != KVATTN_OK)
             return KVATTN_ERR_CUDA;
     }
     kvattn::SparseLaunch l{q, latent, topk_idx, out, lse, need > 0 ? workspace : nullptr, dev_status, B, Hq, L_max,
                            k, scale, fp8, sms};
-    return cuda_status(kvattn::launch_sparse_attn(l, tm_q, tm_o, static_cast<cudaStream_t>(stream)), name);
+    return cuda_status(kvattn::launch_sparse_attn(l, tm_q, tm_o, tm_pm, static_cast<cudaStream_t>(stream)), name);
 }
 
 int attn_decode_sparse(const kvattn_bf16* q, const kvattn_bf16* latent, const int32_t* topk_idx, int B, int Hq, int Dk,

@@ -206,7 +206,7 @@ size_t sparse_partial_bytes(int B, int Hq, int k);
 // (sparse_counter_bytes(B) bytes into the workspace).
 size_t sparse_counter_bytes(int B);
 cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_o,
-                               cudaStream_t stream);
+                               const CUtensorMap& tm_pm, cudaStream_t stream);
 
 // ---- FP8 (E4M3) quantisation of latent rows and indexer keys ----
 cudaError_t launch_latent_quant_fp8(const kvattn_bf16* src, long long n_rows, uint8_t* dst, cudaStream_t stream);

@@ -70,7 +70,7 @@ constexpr int SP_OFF_VALID = SP_OFF_RED + 4 * SP_M * 4;      // [4] bit masks: s
 constexpr int SP_OFF_ROW = SP_OFF_VALID + 16;                // [128] latent row of each slot (-1: none)
 constexpr int SP_OFF_BAR = SP_OFF_ROW + SP_ROWS * 4;
 // c_full[9], q_full[4], q_empty[4], s_full, p_full, o_full[2], done
-constexpr int SP_NBAR = SP_KB + SP_QS + SP_QS + 1 + 1 + 2 + 1;
+constexpr int SP_NBAR = SP_KB + SP_QS + SP_QS + 1 + 1 + 2 + 1 + 1;  // + m_full (merge tiles)
 constexpr int SP_OFF_MISC = SP_OFF_BAR + SP_NBAR * 8;
 constexpr int SP_SMEM = SP_OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(SP_SMEM <= 232448, "shared memory");
@@ -206,10 +206,11 @@ __device__ __forceinline__ void merge_one(const SparseArgs& a, int b, int h, int
     if (j == 0 && a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
 }
 
+
 template <bool FP8>
 __global__ void __launch_bounds__(SP_THREADS, 1)
     sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
-                       SparseArgs a)
+                       const __grid_constant__ CUtensorMap tm_pm, SparseArgs a)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -226,6 +227,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     uint64_t* p_full = s_full + 1;           // P written (S read), SP_GT arrivals
     uint64_t* o_full = p_full + 1;           // [2]: O columns 0-255 / 256-511 complete
     uint64_t* done = o_full + 2;             // every MMA finished
+    uint64_t* m_full = done + 1;             // in-kernel merge: a tile of every part landed
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + SP_OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + SP_OFF_MISC + 4);
 
@@ -241,6 +243,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
         mbar_init(s_full, 1);
         mbar_init(p_full, SP_GT);
         mbar_init(done, 1);
+        mbar_init(m_full, 1);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -433,6 +436,14 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
         s_sum[g * SP_M + h] = l_half;
         named_bar_sync(2, SP_GT);
         const float l = s_sum[h] + s_sum[SP_M + h];
+        if (g == 0 && live) {  // early: its stores are done by the time the part is announced
+            const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
+            if (a.chunks == 1) {
+                if (a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = lse2 * kLn2;
+            } else {
+                a.part_lse[(static_cast<long long>(b) * a.chunks + chunk) * a.Hq + h] = lse2;
+            }
+        }
 
         // ===== epilogue: O columns 256 g .. 256 g + 255 of head row h =====
         const bool one = a.chunks == 1;
@@ -473,14 +484,6 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // shared memory read before exit
             }
         }
-        if (g == 0 && live) {
-            const float lse2 = l > 0.f ? m + __log2f(l) : -INFINITY;
-            if (one) {
-                if (a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = lse2 * kLn2;
-            } else {
-                a.part_lse[(static_cast<long long>(b) * a.chunks + chunk) * a.Hq + h] = lse2;
-            }
-        }
         if (fused) {
             // ===== merge in the kernel: every CTA of the row (all resident: cooperative
             // launch) announces its part, waits for the others, then merges a column slice =====
@@ -503,9 +506,57 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
             }
             named_bar_sync(1, SP_GT);
             if (!*s_abort) {
-                const int j0 = chunk * (SP_DV / 8) / a.chunks, j1 = (chunk + 1) * (SP_DV / 8) / a.chunks;
-                const int nj = j1 - j0;
-                for (int it = t; it < a.Hq * nj; it += SP_GT) merge_one(a, b, it / nj, j0 + it % nj);
+                const int C = a.chunks;
+                // The row's merge as tiles of 64 columns x 64 heads (8 per 64 heads); this CTA's
+                // tiles are chunk, chunk + C, ...  Every part's 8 KB of a tile comes in by TMA
+                // (one round trip for all of them), the parts' lse by plain loads meanwhile.
+                uint8_t* mbuf = smem + SP_OFF_C;                               // [C][64 heads][128 B]
+                float* mlse = reinterpret_cast<float*>(smem + SP_OFF_C + 16 * 8192);  // [C][64]
+                const int n_tiles = 8 * ((a.Hq + 63) / 64);
+                if (t == 0) asm volatile("fence.proxy.async.global;" ::: "memory");  // the parts, seen through the counter
+                int n_t = 0;
+                for (int wt = chunk; wt < n_tiles; wt += C, ++n_t) {
+                    const int cb = wt & 7, hb = wt >> 3;
+                    if (t == 0) {
+                        mbar_arrive_expect_tx(m_full, static_cast<uint32_t>(C) * 8192u);
+                        for (int c = 0; c < C; ++c)
+                            tma_load_3d(mbuf + c * 8192, &tm_pm, m_full, 64 * cb, 64 * hb, b * C + c);
+                    }
+                    for (int x = t; x < C * 64; x += SP_GT) {
+                        const int c = x >> 6, hh = 64 * hb + (x & 63);
+                        mlse[x] = hh < a.Hq ? __ldcg(a.part_lse + (static_cast<long long>(b) * C + c) * a.Hq + hh) : 0.f;
+                    }
+                    named_bar_sync(1, SP_GT);  // mlse written
+                    if (!warp_wait(m_full, n_t & 1, s_abort)) break;
+                    for (int it = t; it < 64 * 8; it += SP_GT) {
+                        const int hh = it >> 3, ch = it & 7, hq = 64 * hb + hh;
+                        if (hq >= a.Hq) continue;
+                        float M = -INFINITY;
+                        for (int c = 0; c < C; ++c) M = fmaxf(M, mlse[c * 64 + hh]);
+                        const float Mu = M == -INFINITY ? 0.f : M;
+                        float L = 0.f;
+                        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        for (int c = 0; c < C; ++c) {
+                            const float wc = fast_exp2(mlse[c * 64 + hh] - Mu);
+                            L += wc;
+                            const uint4 o = *reinterpret_cast<const uint4*>(mbuf + c * 8192 + swz128(hh, ch));
+                            const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                acc[2 * i] = fmaf(wc, bf16_lo(w4[i]), acc[2 * i]);
+                                acc[2 * i + 1] = fmaf(wc, bf16_hi(w4[i]), acc[2 * i + 1]);
+                            }
+                        }
+                        const float inv = L > 0.f ? 1.f / L : 0.f;
+                        const long long ob = (static_cast<long long>(b) * a.Hq + hq) * SP_DV + 64 * cb + 8 * ch;
+                        *reinterpret_cast<uint4*>(a.out + ob) =
+                            make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                                       pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+                        if (cb == 0 && ch == 0 && a.lse)
+                            a.lse[static_cast<long long>(b) * a.Hq + hq] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+                    }
+                    named_bar_sync(1, SP_GT);  // the buffers are read before the next tile's loads
+                }
                 named_bar_sync(1, SP_GT);  // this CTA's reads of the parts are done
                 if (t == 0) {
                     __threadfence();
@@ -639,6 +690,7 @@ size_t sparse_partial_bytes(int B, int Hq, int k)
 }
 
 cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, const CUtensorMap& tm_o,
+                               const CUtensorMap& tm_pm,
                                cudaStream_t stream)
 {
     cudaError_t e = l.fp8 ? set_smem_attr_once<true>() : set_smem_attr_once<false>();
@@ -677,11 +729,11 @@ cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, c
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        return l.fp8 ? cudaLaunchKernelEx(&cfg, sparse_attn_kernel<true>, tm_q, tm_o, a)
-                     : cudaLaunchKernelEx(&cfg, sparse_attn_kernel<false>, tm_q, tm_o, a);
+        return l.fp8 ? cudaLaunchKernelEx(&cfg, sparse_attn_kernel<true>, tm_q, tm_o, tm_pm, a)
+                     : cudaLaunchKernelEx(&cfg, sparse_attn_kernel<false>, tm_q, tm_o, tm_pm, a);
     }
-    e = l.fp8 ? launch_pdl(sparse_attn_kernel<true>, grid, dim3(SP_THREADS), SP_SMEM, stream, tm_q, tm_o, a)
-              : launch_pdl(sparse_attn_kernel<false>, grid, dim3(SP_THREADS), SP_SMEM, stream, tm_q, tm_o, a);
+    e = l.fp8 ? launch_pdl(sparse_attn_kernel<true>, grid, dim3(SP_THREADS), SP_SMEM, stream, tm_q, tm_o, tm_pm, a)
+              : launch_pdl(sparse_attn_kernel<false>, grid, dim3(SP_THREADS), SP_SMEM, stream, tm_q, tm_o, tm_pm, a);
     if (e != cudaSuccess || a.chunks == 1) return e;
     return launch_pdl(sparse_merge_kernel, dim3((l.Hq + SPM_HEADS - 1) / SPM_HEADS, l.B), dim3(SPM_HEADS * 64), 0,
                       stream, a);
