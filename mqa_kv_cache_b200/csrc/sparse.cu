@@ -36,8 +36,9 @@
 //     merged (out = sum_c 2^(lse_c - LSE) o_c): when the whole grid fits on the
 //     GPU at once (one CTA per SM), it is launched cooperatively and the CTAs of
 //     a row merge its parts themselves -- each announces its part on a per-row
-//     counter, waits (bounded) for the others, and merges a 1/chunks slice of the
-//     columns; otherwise a second kernel merges them.
+//     counter, waits (bounded) for the others, and merges its share of the row's
+//     tiles of 64 columns x 64 heads, every part's tile brought in by TMA;
+//     otherwise a second kernel merges them.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -486,7 +487,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
         }
         if (fused) {
             // ===== merge in the kernel: every CTA of the row (all resident: cooperative
-            // launch) announces its part, waits for the others, then merges a column slice =====
+            // launch) announces its part, waits for the others, then merges its tiles of the row =====
             __threadfence();           // this thread's part stores (lse, the TMA stores it waited for)
             named_bar_sync(1, SP_GT);  // both halves stored, every part lse written
             if (t == 0) {
