@@ -339,9 +339,10 @@ int attn_prefill_causal_window(const kvattn_bf16* q, const kvattn_bf16* k, const
  * workspace: dsa_index_topk_workspace_bytes(...) bytes, 256-byte aligned, always
  * required.  Its first 8 KiB per row (B * 2048 counters, the histogram of the top-k's
  * first radix digit, which the indexer fills as it scores and the top-k reads instead
- * of a pass of its own) must be zero before the first call on the workspace
- * (cudaMemsetAsync once); every call leaves them zero, except one that sets
- * KVATTN_STATUS_TIMEOUT.  The rest (the scores, when scores_out is NULL) needs no
+ * of a pass of its own) and the B counters after them (rounded up to 256 bytes: the key
+ * tiles of each row the indexer's CTAs have claimed) must be zero before the first call
+ * on the workspace (cudaMemsetAsync once); every call leaves them zero, except one that
+ * sets KVATTN_STATUS_TIMEOUT.  The rest (the scores, when scores_out is NULL) needs no
  * initialisation.  Calls that share a workspace must be ordered.
  * Supported: H_I = 64, d_I = 128, 1 <= k <= 2048, 1 <= L_max <= 131072.
  */

@@ -62,6 +62,8 @@ constexpr int IX_EPI = 256;                   // two groups of four warps, alter
 constexpr int IX_NACC = 4;                    // 64-column accumulators in flight (the MMA-to-epilogue
                                               // round trip is ~1 us)
 constexpr int IX_TMEM_COLS = IX_NACC * 64;
+constexpr int IX_IQ = 4;     // work items in the producer's hand-out ring
+constexpr int IX_CLAIM = 4;  // key tiles per claim
 
 // bf16 keys: a tile is two 64-column boxes, 6 in flight, K = 128 in eight K = 16 steps
 // (kind::f16); FP8 ("the indexer runs stably in fp8", "Agentic RL 入门3" §2.2 (1)): the
@@ -79,9 +81,10 @@ struct IxCfg {
     static constexpr int OFF_Q = STAGES * TILE;
     static constexpr int OFF_W = OFF_Q + QBYTES;
     static constexpr int OFF_HIST = OFF_W + IX_HEADS * 4;   // [2048] digit counts of the current work item
-    static constexpr int OFF_BAR = OFF_HIST + 2048 * 4;
-    // full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done
-    static constexpr int NBAR = 2 * STAGES + 3 + 2 * IX_NACC;
+    static constexpr int OFF_ITEMS = OFF_HIST + 2048 * 4;     // [IX_IQ][3] (row, first tile, end tile); [3] the epilogue's
+    static constexpr int OFF_BAR = OFF_ITEMS + (IX_IQ + 1) * 3 * 4 + 4;
+    // full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done, item_full[IQ], item_empty[IQ]
+    static constexpr int NBAR = 2 * STAGES + 3 + 2 * IX_NACC + 2 * IX_IQ;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 32 + 1024;
     static_assert(SMEM <= 232448, "shared memory");
@@ -97,18 +100,20 @@ struct IndexerArgs {
     const float* qscale;  // FP8: [B][64] query-head scales
     float* scores;
     uint32_t* hist;       // [B][2048] first-digit counts of the valid scores (added to; zero on entry)
+    int* row_ctr;         // [B] key tiles of each row claimed so far (zero on entry; the top-k clears them)
     int32_t* dev_status;
-    int B, L_max, tiles_per_b, chunks_per_b;
+    int B, L_max, tiles_per_b;
     int len_shift;  // row b scores seq_lens[b] >> len_shift keys (2: 4-token groups)
 };
 
-__device__ __forceinline__ void ix_item(const IndexerArgs& a, int item, int& b, int& t0, int& t1)
+// Rows served by CTA c of G: with G >= B the CTAs are split over the rows (row c B / G),
+// each row's tiles claimed IX_CLAIM at a time from its counter by whichever of its CTAs
+// is ready, so that faster CTAs take more; with G < B, rows c, c + G, ...
+__device__ __forceinline__ int ix_first_row(int c, int G, int B)
 {
-    b = item / a.chunks_per_b;
-    const int c = item - b * a.chunks_per_b;
-    t0 = static_cast<int>(static_cast<long long>(c) * a.tiles_per_b / a.chunks_per_b);
-    t1 = static_cast<int>(static_cast<long long>(c + 1) * a.tiles_per_b / a.chunks_per_b);
+    return G >= B ? static_cast<int>(static_cast<long long>(c) * B / G) : c;
 }
+__device__ __forceinline__ int ix_next_row(int c, int G, int B, int b) { return G >= B ? B : b + G; }
 
 __device__ __forceinline__ void tc_mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate)
@@ -135,13 +140,19 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     uint64_t* acc_full = q_full + 2;
     uint64_t* acc_empty = acc_full + IX_NACC;
     uint64_t* mma_done = acc_empty + IX_NACC;
+    // The producer hands out work items (row b, key tiles [t0, t1)) through a ring; an item
+    // with t0 == t1 closes row b, and b < 0 ends the stream.
+    uint64_t* item_full = mma_done + 1;        // [IQ]
+    uint64_t* item_empty = item_full + IX_IQ;  // [IQ]: read by the MMA thread and the epilogue
+    int* s_items = reinterpret_cast<int*>(smem + C::OFF_ITEMS);
+    volatile int* s_cur = reinterpret_cast<volatile int*>(s_items + IX_IQ * 3);  // the epilogue's current item
     float* s_w = reinterpret_cast<float*>(smem + C::OFF_W);
     uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = a.B * a.chunks_per_b;
+    const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -155,6 +166,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
             mbar_init(&acc_empty[i], 4);
         }
         mbar_init(mma_done, 1);
+        for (int i = 0; i < IX_IQ; ++i) {
+            mbar_init(&item_full[i], 1);
+            mbar_init(&item_empty[i], 2);
+        }
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -174,31 +189,51 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     pdl_trigger();
 
     if (warp == 0) {
-        // ===== TMA producer: each item's query heads, then its key tiles =====
+        // ===== TMA producer: each row's query heads, then the key tiles it claims =====
         if (lane == 0) {
-            int it = 0, n = 0;
-            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
-                int b, t0, t1;
-                ix_item(a, item, b, t0, t1);
-                if (n > 0 && !mbar_wait(q_empty, (n - 1) & 1)) {
-                    *s_abort = 1;
+            int it = 0, n = 0, nq = 0;
+            auto push = [&](int b, int t0, int t1) {
+                const int slot = n % IX_IQ;
+                if (n >= IX_IQ && !mbar_wait(&item_empty[slot], ((n / IX_IQ) - 1) & 1)) return false;
+                s_items[3 * slot] = b;
+                s_items[3 * slot + 1] = t0;
+                s_items[3 * slot + 2] = t1;
+                mbar_arrive(&item_full[slot]);
+                ++n;
+                return true;
+            };
+            bool ok = true;
+            for (int b = ix_first_row(cta, G, a.B); ok && b < a.B && !*s_abort; b = ix_next_row(cta, G, a.B, b)) {
+                // the row's query heads, once the S MMAs of the previous row are done with its own
+                if (nq > 0 && !mbar_wait(q_empty, (nq - 1) & 1)) {
+                    ok = false;
                     break;
                 }
                 mbar_arrive_expect_tx(q_full, C::QBYTES);
 #pragma unroll
                 for (int i = 0; i < C::KBOX; ++i) tma_load_3d(smem + C::OFF_Q + i * IX_QBOX, &tm_q, q_full, 64 * i, 0, b);
-                for (int t = t0; t < t1; ++t, ++it) {
-                    const int s = it % C::STAGES;
-                    if (it >= C::STAGES && (*s_abort || !mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1))) {
-                        *s_abort = 1;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&full[s], C::TILE);
-                    uint8_t* dst = smem + s * C::TILE;
+                ++nq;
+                while (ok) {
+                    const int t0 = atomicAdd(a.row_ctr + b, IX_CLAIM);
+                    if (t0 >= a.tiles_per_b) break;
+                    const int t1 = min(t0 + IX_CLAIM, a.tiles_per_b);
+                    if (!(ok = push(b, t0, t1))) break;
+                    for (int t = t0; t < t1; ++t, ++it) {
+                        const int s = it % C::STAGES;
+                        if (it >= C::STAGES && (*s_abort || !mbar_wait(&empty[s], ((it / C::STAGES) - 1) & 1))) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[s], C::TILE);
+                        uint8_t* dst = smem + s * C::TILE;
 #pragma unroll
-                    for (int i = 0; i < C::KBOX; ++i) tma_load_3d(dst + i * IX_BOX, &tm_k, &full[s], 64 * i, t * IX_TOK, b);
+                        for (int i = 0; i < C::KBOX; ++i) tma_load_3d(dst + i * IX_BOX, &tm_k, &full[s], 64 * i, t * IX_TOK, b);
+                    }
                 }
+                if (ok) ok = push(b, 0, 0);  // row b closed
             }
+            if (!ok) *s_abort = 1;
+            push(-1, 0, 0);  // the end (bounded wait; after a timeout the consumers' own waits end them)
             if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
             for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
                 mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
@@ -207,13 +242,28 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         // ===== MMA issuer (one thread) =====
         if (lane == 0) {
             const uint32_t q_addr = smem_u32(smem + C::OFF_Q);
-            int it = 0, n = 0;
-            for (int item = blockIdx.x; item < n_items && !*s_abort; item += gridDim.x, ++n) {
-                int b, t0, t1;
-                ix_item(a, item, b, t0, t1);
-                if (!mbar_wait(q_full, n & 1)) {
+            int it = 0, nq = 0, cur_b = -1;
+            for (int n = 0; !*s_abort; ++n) {
+                const int slot = n % IX_IQ;
+                if (!mbar_wait(&item_full[slot], (n / IX_IQ) & 1)) {
                     *s_abort = 1;
                     break;
+                }
+                const int b = s_items[3 * slot], t0 = s_items[3 * slot + 1], t1 = s_items[3 * slot + 2];
+                mbar_arrive(&item_empty[slot]);
+                if (b < 0) break;
+                if (t0 == t1) {  // row b closed: every S of it is issued, its query heads may go
+                    tc_commit(q_empty);
+                    cur_b = -1;
+                    continue;
+                }
+                if (b != cur_b) {  // the row's query heads have landed
+                    if (!mbar_wait(q_full, nq & 1)) {
+                        *s_abort = 1;
+                        break;
+                    }
+                    ++nq;
+                    cur_b = b;
                 }
                 for (int t = t0; t < t1; ++t, ++it) {
                     const int s = it % C::STAGES;
@@ -240,7 +290,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                     tc_commit(&empty[s]);
                     tc_commit(&acc_full[buf]);
                 }
-                tc_commit(q_empty);
             }
             // every issued MMA has finished before the accumulators are released
             tc_commit(mma_done);
@@ -255,19 +304,51 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         const int row = quarter * 32 + lane;
         const int ep = threadIdx.x - 64;
         for (int i = ep; i < TK_DIGITS0; i += IX_EPI) s_hist[i] = 0u;  // ordered by the item's first barrier
-        int tc = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
-            int b, t0, t1;
-            ix_item(a, item, b, t0, t1);
-            const int len_raw = a.seq_lens ? (a.seq_lens[b] >> a.len_shift) : a.L_max;
-            const int len = min(max(len_raw, 0), a.L_max);
-            if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
-            named_bar_sync(2, IX_EPI);
-            if (ep < IX_HEADS) {
-                const long long wi = static_cast<long long>(b) * IX_HEADS + ep;
-                s_w[ep] = FP8 ? a.w[wi] * a.qscale[wi] : a.w[wi];
+        int tc = 0, cur_b = -1, len = 0;
+        for (int n = 0;; ++n) {
+            // one thread takes the item from the ring (bounded wait; b < 0 ends) and every
+            // epilogue thread reads it between two barriers, so that all meet the same barriers
+            if (ep == 0) {
+                const int slot = n % IX_IQ;
+                if (!*s_abort && mbar_wait(&item_full[slot], (n / IX_IQ) & 1)) {
+                    s_cur[0] = s_items[3 * slot];
+                    s_cur[1] = s_items[3 * slot + 1];
+                    s_cur[2] = s_items[3 * slot + 2];
+                } else {
+                    *s_abort = 1;
+                    s_cur[0] = -1;
+                }
+                mbar_arrive(&item_empty[slot]);
             }
             named_bar_sync(2, IX_EPI);
+            const int b = s_cur[0], t0 = s_cur[1], t1 = s_cur[2];
+            named_bar_sync(2, IX_EPI);
+            if (b < 0) break;
+            if (t0 == t1) {  // row b closed: its counts into the row's histogram, the shared one back to zero
+                if (a.hist) {
+                    uint32_t* gh = a.hist + static_cast<long long>(b) * TK_DIGITS0;
+                    for (int i = ep; i < TK_DIGITS0; i += IX_EPI) {
+                        const uint32_t v = s_hist[i];
+                        if (v) {
+                            atomicAdd(gh + i, v);
+                            s_hist[i] = 0u;
+                        }
+                    }
+                }
+                cur_b = -1;
+                continue;  // the next item's barriers order these before any new count
+            }
+            if (b != cur_b) {
+                const int len_raw = a.seq_lens ? (a.seq_lens[b] >> a.len_shift) : a.L_max;
+                len = min(max(len_raw, 0), a.L_max);
+                if (len != len_raw && ep == 0) report_status(a.dev_status, KVATTN_STATUS_BAD_LENGTH);
+                if (ep < IX_HEADS) {
+                    const long long wi = static_cast<long long>(b) * IX_HEADS + ep;
+                    s_w[ep] = FP8 ? a.w[wi] * a.qscale[wi] : a.w[wi];
+                }
+                named_bar_sync(2, IX_EPI);
+                cur_b = b;
+            }
             float* out = a.scores + static_cast<long long>(b) * a.L_max;
             for (int t = t0; t < t1; ++t, ++tc) {
                 if ((tc & 1) != grp) continue;
@@ -305,17 +386,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 const uint32_t digit = in ? score_key(acc, nan_key) >> TK_SHIFT0 : 0xffffffffu;
                 const uint32_t same = __match_any_sync(0xffffffffu, digit);
                 if (in && lane == __ffs(same) - 1) atomicAdd(&s_hist[digit], static_cast<uint32_t>(__popc(same)));
-            }
-            if (a.hist) {  // the item's counts into the row's histogram; the shared one back to zero
-                named_bar_sync(2, IX_EPI);
-                uint32_t* gh = a.hist + static_cast<long long>(b) * TK_DIGITS0;
-                for (int i = ep; i < TK_DIGITS0; i += IX_EPI) {
-                    const uint32_t v = s_hist[i];
-                    if (v) {
-                        atomicAdd(gh + i, v);
-                        s_hist[i] = 0u;
-                    }
-                }
             }
         }
     }
@@ -419,6 +489,7 @@ struct TopkArgs {
     int32_t* tok_out;    // groups mode (see DsaIndexArgs), else null
     int32_t* tok_count;
     int L_tok;
+    int* row_ctr;        // [B] the indexer's claim counters: cleared here for the next call (null: none)
 };
 
 constexpr int TK_SLICE_MAX = 16384;  // keys per CTA held in shared memory
@@ -472,6 +543,7 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
 
     pdl_wait();
     pdl_trigger();
+    if (a.row_ctr && rank == 0 && tid == 0) a.row_ctr[row] = 0;  // the indexer is done with it
 
     const int len_raw = a.seq_lens ? (a.seq_lens[row] >> a.len_shift) : a.L_max;
     const int len = min(max(len_raw, 0), a.L_max);
@@ -875,7 +947,11 @@ __global__ void __launch_bounds__(TK_THREADS) topk_merge_kernel(MergeTopkArgs a)
 
 size_t dsa_scores_bytes(int B, int L_max) { return static_cast<size_t>(B) * L_max * sizeof(float); }
 
-size_t dsa_hist_bytes(int B) { return static_cast<size_t>(B) * TK_DIGITS0 * sizeof(uint32_t); }
+// [B][2048] first-digit counts, then [B] claim counters of the indexer's rows
+size_t dsa_hist_bytes(int B)
+{
+    return static_cast<size_t>(B) * TK_DIGITS0 * sizeof(uint32_t) + (static_cast<size_t>(B) * 4 + 255) / 256 * 256;
+}
 
 cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
                                   cudaStream_t stream)
@@ -897,6 +973,7 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
         e = launch_idx_key_quant_fp8(a.q_idx, static_cast<long long>(a.B) * IX_HEADS, a.q8, a.q8_scale, stream);
         if (e != cudaSuccess) return e;
     }
+    if (!a.hist) return cudaErrorInvalidValue;  // the workspace's zero region holds the claim counters
     IndexerArgs ia{};
     ia.hist = a.hist;
     ia.kscale = a.kscale;
@@ -909,19 +986,16 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     ia.L_max = a.L_max;
     ia.len_shift = a.len_shift;
     ia.tiles_per_b = (a.L_max + IX_TOK - 1) / IX_TOK;
-    // about two contiguous chunks per CTA, never more chunks than tiles
-    int chunks = (2 * a.num_sms + a.B - 1) / a.B;
-    if (chunks > ia.tiles_per_b) chunks = ia.tiles_per_b;
-    if (chunks < 1) chunks = 1;
-    ia.chunks_per_b = chunks;
-    const int items = a.B * chunks;
-    const int grid = items < a.num_sms ? items : a.num_sms;
+    ia.row_ctr = reinterpret_cast<int*>(a.hist + static_cast<size_t>(a.B) * TK_DIGITS0);
+    // every SM, but no more CTAs than claims
+    const long long claims = static_cast<long long>(a.B) * ((ia.tiles_per_b + IX_CLAIM - 1) / IX_CLAIM);
+    const int grid = claims < a.num_sms ? static_cast<int>(claims) : a.num_sms;
     e = fp8 ? launch_pdl(indexer_kernel<true>, dim3(grid), dim3(IX_THREADS), IxCfg<true>::SMEM, stream, tm_k, tm_q, ia)
             : launch_pdl(indexer_kernel<false>, dim3(grid), dim3(IX_THREADS), IxCfg<false>::SMEM, stream, tm_k, tm_q, ia);
     if (e != cudaSuccess) return e;
 
     TopkArgs ta{a.scores, a.seq_lens, a.hist, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k,
-                a.len_shift, a.tok_idx, a.tok_count, a.L_tok};
+                a.len_shift, a.tok_idx, a.tok_count, a.L_tok, ia.row_ctr};
     const size_t key_bytes = static_cast<size_t>(slice_words(a.L_max) + 2 * TK_CAND_MAX) * sizeof(uint32_t);
     static bool tk_attr[64] = {};
     if (dev < 64 && !tk_attr[dev]) {

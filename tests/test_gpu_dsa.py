@@ -243,7 +243,7 @@ def test_selection_workspace_counts_are_left_zero(K):
     inp = W.dsa_inputs(wl, B=B, L=L, seed=88, with_latent=False)
     q_idx, w, k_idx = inp["q_idx"].cuda(), inp["w"].cuda(), inp["k_idx"].cuda()
     lens = torch.tensor([6000, 2500, 1000], dtype=torch.int32).cuda()
-    hist_bytes = B * 2048 * 4
+    hist_bytes = B * 2048 * 4 + B * 4  # first-digit counts, then the indexer's per-row claim counters
     ws = K.workspace(K.dsa_index_topk_workspace_bytes(B, L, k))
     first = K.dsa_index_topk(q_idx, w, k_idx, k, seq_lens=lens, ws=ws)[0].clone()
     torch.cuda.synchronize()
