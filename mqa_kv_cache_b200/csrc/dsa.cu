@@ -108,12 +108,13 @@ struct IndexerArgs {
 
 // Rows served by CTA c of G: with G >= B the CTAs are split over the rows (row c B / G),
 // each row's tiles claimed IX_CLAIM at a time from its counter by whichever of its CTAs
-// is ready, so that faster CTAs take more; with G < B, rows c, c + G, ...
-__device__ __forceinline__ int ix_first_row(int c, int G, int B)
+// is ready, so that faster CTAs take more (going on to other rows once a row is done
+// was measured slower); with G < B, rows c, c + G, ...
+__device__ __forceinline__ int ix_rows(int c, int G, int B) { return G >= B ? 1 : (B - c + G - 1) / G; }
+__device__ __forceinline__ int ix_row(int c, int G, int B, int r)
 {
-    return G >= B ? static_cast<int>(static_cast<long long>(c) * B / G) : c;
+    return G >= B ? static_cast<int>(static_cast<long long>(c) * B / G) : c + r * G;
 }
-__device__ __forceinline__ int ix_next_row(int c, int G, int B, int b) { return G >= B ? B : b + G; }
 
 __device__ __forceinline__ void tc_mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate)
@@ -203,7 +204,14 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 return true;
             };
             bool ok = true;
-            for (int b = ix_first_row(cta, G, a.B); ok && b < a.B && !*s_abort; b = ix_next_row(cta, G, a.B, b)) {
+            const int n_rows = ix_rows(cta, G, a.B);
+            for (int r = 0; ok && r < n_rows && !*s_abort; ++r) {
+                const int b = ix_row(cta, G, a.B, r);
+                if (r > 0 && __ldcg(a.row_ctr + b) >= a.tiles_per_b) continue;  // nothing left there
+                // the first claim comes before the row's query heads: a row this CTA gets no tiles of
+                // loads nothing and hands out nothing (every query load is waited for by the MMA)
+                int t0 = atomicAdd(a.row_ctr + b, IX_CLAIM);
+                if (t0 >= a.tiles_per_b) continue;
                 // the row's query heads, once the S MMAs of the previous row are done with its own
                 if (nq > 0 && !mbar_wait(q_empty, (nq - 1) & 1)) {
                     ok = false;
@@ -214,8 +222,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 for (int i = 0; i < C::KBOX; ++i) tma_load_3d(smem + C::OFF_Q + i * IX_QBOX, &tm_q, q_full, 64 * i, 0, b);
                 ++nq;
                 while (ok) {
-                    const int t0 = atomicAdd(a.row_ctr + b, IX_CLAIM);
-                    if (t0 >= a.tiles_per_b) break;
                     const int t1 = min(t0 + IX_CLAIM, a.tiles_per_b);
                     if (!(ok = push(b, t0, t1))) break;
                     for (int t = t0; t < t1; ++t, ++it) {
@@ -229,12 +235,17 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
 #pragma unroll
                         for (int i = 0; i < C::KBOX; ++i) tma_load_3d(dst + i * IX_BOX, &tm_k, &full[s], 64 * i, t * IX_TOK, b);
                     }
+                    if (!ok) break;
+                    t0 = atomicAdd(a.row_ctr + b, IX_CLAIM);
+                    if (t0 >= a.tiles_per_b) break;
                 }
                 if (ok) ok = push(b, 0, 0);  // row b closed
             }
             if (!ok) *s_abort = 1;
             push(-1, 0, 0);  // the end (bounded wait; after a timeout the consumers' own waits end them)
             if (*s_abort) report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+            // copies still in flight complete before the CTA leaves (bounded waits)
+            if (nq > 0) mbar_wait(q_full, (nq - 1) & 1);
             for (int j = it - C::STAGES > 0 ? it - C::STAGES : 0; j < it; ++j)
                 mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1);
         }
