@@ -77,6 +77,30 @@ def test_indexer_and_topk_small(K, L, k, lens):
     np.testing.assert_array_equal(idx, _index_order(ref_idx))
 
 
+@pytest.mark.parametrize("B,L,k", [(160, 512, 64), (2, 700, 100), (5, 128, 16)])
+def test_indexer_work_claims(K, B, L, k):
+    """The indexer's CTAs claim each row's key tiles from a per-row counter: more rows
+    than CTAs (a CTA serves several rows in turn), and rows of a few tiles shared by
+    several CTAs (some of which may find the row already taken).  Scores and selection
+    against the oracle, twice on the same workspace (the counters are left zero)."""
+    wl = W.DSA_128K
+    inp = W.dsa_inputs(wl, B=B, L=L, seed=71 + B + L, with_latent=False)
+    lens = torch.randint(1, L + 1, (B,), generator=torch.Generator().manual_seed(B + L), dtype=torch.int32)
+    q_idx, w, k_idx = inp["q_idx"].cuda(), inp["w"].cuda(), inp["k_idx"].cuda()
+    ws = K.workspace(K.dsa_index_topk_workspace_bytes(B, L, k))
+    qb, kb, wn = W.bf16_bits(inp["q_idx"]), W.bf16_bits(inp["k_idx"]), inp["w"].numpy()
+    for call in range(2):
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        idx, scores = K.dsa_index_topk(q_idx, w, k_idx, k, seq_lens=lens.cuda(), ws=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0, call
+        assert int(ws[:B * 2048 * 4 + B * 4].count_nonzero()) == 0, call
+        scores = scores.cpu().numpy()
+        _check_scores(scores, qb, wn, kb, lens.numpy())
+        ref_idx = oracle.topk(scores, k, lens=lens.numpy())
+        np.testing.assert_array_equal(idx.cpu().numpy(), _index_order(ref_idx))
+
+
 def test_topk_ties_go_to_the_lower_index(K):
     # duplicated key rows give bit-identical scores; all-zero rows give exact 0 scores
     B, L, k = 2, 3000, 500
