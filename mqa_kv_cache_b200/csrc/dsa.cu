@@ -46,8 +46,8 @@ __device__ __forceinline__ uint32_t score_key(float f, bool& nan)
 
 // The first radix digit of the top-k (the key's top 11 bits).  The indexers count the
 // digits of every row's valid scores as they produce them (a shared-memory histogram per
-// work item, flushed into a per-row histogram in global memory), so that the top-k starts
-// at its second digit.
+// CTA and row, flushed into the row's histogram in global memory when the CTA is done with
+// the row), so that the top-k starts at its second digit.
 constexpr int TK_DIGITS0 = 2048;
 constexpr int TK_SHIFT0 = 21;
 
@@ -80,7 +80,7 @@ struct IxCfg {
     static constexpr int KSTEPS = FP8 ? 4 : 8;
     static constexpr int OFF_Q = STAGES * TILE;
     static constexpr int OFF_W = OFF_Q + QBYTES;
-    static constexpr int OFF_HIST = OFF_W + IX_HEADS * 4;   // [2048] digit counts of the current work item
+    static constexpr int OFF_HIST = OFF_W + IX_HEADS * 4;   // [2048] digit counts of the current row
     static constexpr int OFF_ITEMS = OFF_HIST + 2048 * 4;     // [IX_IQ][3] (row, first tile, end tile); [3] the epilogue's
     static constexpr int OFF_BAR = OFF_ITEMS + (IX_IQ + 1) * 3 * 4 + 4;
     // full[S], empty[S], q_full, q_empty, acc_full[NACC], acc_empty[NACC], mma_done, item_full[IQ], item_empty[IQ]
