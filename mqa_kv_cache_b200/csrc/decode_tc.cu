@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     w_start.S = S0;
 
     if (active && warp == 0) {
-        // ===== TMA producer: Q of each piece, then K and V of each tile =====
+        // ===== TMA producer: Q of each piece, then K of each tile (warp 7 loads V) =====
         if (lane == 0) {
             const uint64_t pol = l2_evict_first_policy();  // K and V are read once
             Walk w = w_start;
