@@ -28,17 +28,21 @@
 //   - warp 9 issues O = P V with V = the resident rows read as an MN-major
 //     operand, N = 256 twice, into all 512 TMEM columns (S's columns are free by
 //     then).
-//   - warps 0-3 write O columns 0-255, warps 4-7 columns 256-511: normalised by
-//     the chunk's own softmax sum, rounded to bf16 into shared memory (over the
-//     blocks whose values that half has consumed), then stored by TMA.  A row
-//     with one chunk is written to the output directly; otherwise each chunk
-//     leaves its normalised bf16 part and its log-sum-exp, and the parts are
-//     merged (out = sum_c 2^(lse_c - LSE) o_c): when the whole grid fits on the
-//     GPU at once (one CTA per SM), it is launched cooperatively and the CTAs of
-//     a row merge its parts themselves -- each announces its part on a per-row
-//     counter, waits (bounded) for the others, and merges its share of the row's
-//     tiles of 64 columns x 64 heads, every part's tile brought in by TMA;
-//     otherwise a second kernel merges them.
+//   - the epilogue writes O in boxes of 64 columns, normalised by the chunk's own
+//     softmax sum and rounded to bf16 into shared memory (over the row blocks
+//     that half's P V has consumed), each box stored by TMA as soon as it is
+//     staged; warps 0-3 take boxes 0-1 and warps 4-7 boxes 2-3 of each half, so
+//     both groups start on a half as soon as its P V is done.  A row with one
+//     chunk is written to the output directly; otherwise each chunk leaves its
+//     normalised bf16 part and its log-sum-exp, and the parts are merged
+//     (out = sum_c 2^(lse_c - LSE) o_c): when the whole grid fits on the GPU at
+//     once (one CTA per SM), it is launched cooperatively and the CTAs of a row
+//     merge its parts themselves -- each warp group counts its stored boxes on a
+//     per-row counter (a release add), every CTA waits (bounded) for the row's
+//     2 x chunks counts, then merges its share of the row's tiles of 64 columns
+//     x 64 heads: every part's tile comes in by TMA, and meanwhile the parts'
+//     lse give each head's weights once (four threads per head); otherwise a
+//     second kernel merges them.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -60,6 +64,8 @@ constexpr int SP_GT = SP_GW * 32;
 constexpr int SP_THREADS = SP_GT + 64;         // + TMA warp + MMA warp
 constexpr int SP_TMA_WARP = SP_GW, SP_MMA_WARP = SP_GW + 1;
 constexpr int SP_QS = 4;                       // query slots
+constexpr int SP_K_MAX = 2048;                 // selected rows per batch row (the entry points' limit)
+constexpr int SP_MAXC = SP_K_MAX / SP_ROWS;    // chunks per batch row (16)
 constexpr int SP_OFF_C = 0;                                  // 9 blocks of gathered rows
 constexpr int SP_OFF_RAW = SP_OFF_C + 4 * SP_BLOCK;          // FP8: codes [8 blocks][128 rows][64 B] (blocks 4-7)
 constexpr int SP_RAW_BLOCK = SP_ROWS * 64;
@@ -76,6 +82,7 @@ constexpr int SP_OFF_MISC = SP_OFF_BAR + SP_NBAR * 8;
 constexpr int SP_SMEM = SP_OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(SP_SMEM <= 232448, "shared memory");
 static_assert(SP_OFF_RAW + 8 * SP_RAW_BLOCK == SP_OFF_C + 8 * SP_BLOCK, "codes fill blocks 4-7 exactly");
+static_assert(SP_MAXC * (8192 + 64 * 4) <= SP_KB * SP_BLOCK, "a merge tile of every part and its weights fit in the row blocks");
 constexpr int SP_FP8_ROW = 656;                // packed row: 512 codes, 4 fp32 scales, 64 bf16
 constexpr int SP_FP8_SCL = 512, SP_FP8_ROPE = 528;
 constexpr uint32_t SP_IDESC_S = umma_idesc_bf16(SP_M, SP_ROWS);              // Q x C^T, both K-major
@@ -159,11 +166,18 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                  : "memory");
 }
 
+// Add with release semantics at GPU scope: what this thread wrote or saw before is visible
+// to a thread that reads the sum with acquire.
+__device__ __forceinline__ void red_release_add(int* p, int v)
+{
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // One (head, 16-byte column chunk) of the merge of a row's C parts: out = sum_c
 // 2^(lse_c - LSE) o_c, LSE = log2 sum_c 2^lse_c (log2 units; lse written in natural log).
 __device__ __forceinline__ void merge_one(const SparseArgs& a, int b, int h, int j)
 {
-    constexpr int MAXC = 16;  // k <= 2048 in chunks of 128
+    constexpr int MAXC = SP_MAXC;
     const int C = a.chunks;
     float ls[MAXC];
     uint4 ov[MAXC];
@@ -251,6 +265,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
     if (warp == SP_TMA_WARP && lane == 0) {
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_o);
+        tma_prefetch_desc(&tm_pm);
     }
     if (warp == SP_MMA_WARP) {
         tmem_alloc(s_tmem, 512);
@@ -443,128 +458,157 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                 if (a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = lse2 * kLn2;
             } else {
                 a.part_lse[(static_cast<long long>(b) * a.chunks + chunk) * a.Hq + h] = lse2;
+                __threadfence();  // before half 0 counts itself on the row's counter
             }
         }
 
-        // ===== epilogue: O columns 256 g .. 256 g + 255 of head row h =====
+        // ===== epilogue: O of head row h, normalised, as bf16 boxes of 64 columns; warps 0-3 take
+        // boxes 0-1 and warps 4-7 boxes 2-3 of each 256-column half, so that both groups work on
+        // a half as soon as its P V is done =====
         const bool one = a.chunks == 1;
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint8_t* stg = smem + SP_OFF_C + 4 * g * SP_BLOCK;  // the blocks this half's P V has consumed
-        const bool have_o = warp_wait(&o_full[g], 0, s_abort);
-        if (have_o) {
+        const bool fused = !one && a.fused_merge;
+        const bool store = quarter == 0 && lane == 0;
+        const int z = one ? b : b * a.chunks + chunk;
+        bool have_o = true;
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+            if (!(have_o = warp_wait(&o_full[hf], 0, s_abort))) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int cc = 0; cc < 8; ++cc) {
-                uint32_t ov[32];
-                tmem_ld32(tmem + lane_off + 256 * g + 32 * cc, ov);
+            for (int j = 0; j < 2; ++j) {
+                // box bx = O columns 64 bx .. 64 bx + 63, staged in row block bx (read by this half's P V)
+                const int bx = 4 * hf + 2 * g + j;
+                uint32_t ov[2][32];
+                tmem_ld32(tmem + lane_off + 64 * bx, ov[0]);
+                tmem_ld32(tmem + lane_off + 64 * bx + 32, ov[1]);
                 tmem_wait_ld();
-                tmem_regs_ready(ov);
-                uint8_t* box = stg + (cc >> 1) * SP_BLOCK;
+                tmem_regs_ready(ov[0]);
+                tmem_regs_ready(ov[1]);
+                uint8_t* box = smem + SP_OFF_C + bx * SP_BLOCK;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float* f = reinterpret_cast<const float*>(ov) + 8 * i;
-                    *reinterpret_cast<uint4*>(box + swz128(h, (cc & 1) * 4 + i)) =
+                for (int i = 0; i < 8; ++i) {
+                    const float* f = reinterpret_cast<const float*>(ov[i >> 2]) + 8 * (i & 3);
+                    *reinterpret_cast<uint4*>(box + swz128(h, i)) =
                         make_uint4(pack_bf16x2(f[0] * inv, f[1] * inv), pack_bf16x2(f[2] * inv, f[3] * inv),
                                    pack_bf16x2(f[4] * inv, f[5] * inv), pack_bf16x2(f[6] * inv, f[7] * inv));
                 }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                named_bar_sync(3 + g, 128);
+                if (store && !*s_abort) {
+                    tma_store_3d(&tm_o, box, 64 * bx, 0, z);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
             }
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        named_bar_sync(3 + g, 128);
-        const bool fused = !one && a.fused_merge;
-        if (quarter == 0 && lane == 0 && have_o && !*s_abort) {
-            const int z = one ? b : b * a.chunks + chunk;
-#pragma unroll
-            for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tm_o, stg + bx * SP_BLOCK, 256 * g + 64 * bx, 0, z);
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            if (fused) {
-                // the part is in global memory before the row's counter says so
+        if (store) {
+            if (fused && have_o) {
+                // the group's boxes are in global memory before the row's counter says so: each
+                // group counts itself (the lse, written by warps 0-3, was fenced before their barriers)
                 asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
                 asm volatile("fence.proxy.async.global;" ::: "memory");
+                if (!*s_abort) red_release_add(a.row_arrive + b, 1);
             } else {
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // shared memory read before exit
             }
         }
         if (fused) {
             // ===== merge in the kernel: every CTA of the row (all resident: cooperative
-            // launch) announces its part, waits for the others, then merges its tiles of the row =====
-            __threadfence();           // this thread's part stores (lse, the TMA stores it waited for)
-            named_bar_sync(1, SP_GT);  // both halves stored, every part lse written
-            if (t == 0) {
-                if (!*s_abort) {
-                    __threadfence();
-                    atomicAdd(a.row_arrive + b, 1);
-                    const unsigned long long t0 = global_timer_ns();
-                    while (ld_acquire_gpu(a.row_arrive + b) < a.chunks) {
-                        if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
-                            *s_abort = 1;
-                            report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
-                            break;
-                        }
-                        __nanosleep(64);
+            // launch) waits for the row's 2 x chunks counts, then merges its tiles of the row =====
+            if (t == 0 && !*s_abort) {
+                const unsigned long long t0 = global_timer_ns();
+                while (ld_acquire_gpu(a.row_arrive + b) < 2 * a.chunks) {
+                    if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+                        *s_abort = 1;
+                        report_status(a.dev_status, KVATTN_STATUS_TIMEOUT);
+                        break;
                     }
+                    __nanosleep(64);
                 }
             }
             named_bar_sync(1, SP_GT);
             if (!*s_abort) {
-                const int C = a.chunks;
+                const int C = a.chunks;  // <= SP_K_MAX / SP_ROWS
+                // this CTA is past the wait: the row's last one to get here leaves the counters zero
+                // (nobody reads them any more); the atomic's answer is needed only at the end
+                const int past = t == 32 ? atomicAdd(a.row_done + b, 1) : 0;
                 // The row's merge as tiles of 64 columns x 64 heads (8 per 64 heads); this CTA's
                 // tiles are chunk, chunk + C, ...  Every part's 8 KB of a tile comes in by TMA
-                // (one round trip for all of them), the parts' lse by plain loads meanwhile.
-                uint8_t* mbuf = smem + SP_OFF_C;                               // [C][64 heads][128 B]
-                float* mlse = reinterpret_cast<float*>(smem + SP_OFF_C + 16 * 8192);  // [C][64]
+                // (one round trip for all of them); meanwhile the parts' lse give each head's
+                // weights 2^(lse_c - LSE), computed once per head: thread (head t / 4, t % 4) takes
+                // parts t % 4, t % 4 + 4, ...
+                uint8_t* mbuf = smem + SP_OFF_C;                                   // [C][64 heads][128 B]
+                float* mw = reinterpret_cast<float*>(smem + SP_OFF_C + SP_MAXC * 8192);  // [C][64] weights
                 const int n_tiles = 8 * ((a.Hq + 63) / 64);
-                if (t == 0) asm volatile("fence.proxy.async.global;" ::: "memory");  // the parts, seen through the counter
+                const int wh = t >> 2, wq = t & 3;
                 int n_t = 0;
                 for (int wt = chunk; wt < n_tiles; wt += C, ++n_t) {
                     const int cb = wt & 7, hb = wt >> 3;
-                    if (t == 0) {
-                        mbar_arrive_expect_tx(m_full, static_cast<uint32_t>(C) * 8192u);
-                        for (int c = 0; c < C; ++c)
+                    const int whq = 64 * hb + wh;
+                    float lv[SP_MAXC / 4];
+#pragma unroll
+                    for (int i = 0; i < SP_MAXC / 4; ++i) {
+                        const int c = wq + 4 * i;
+                        lv[i] = c < C && whq < a.Hq
+                                    ? __ldcg(a.part_lse + (static_cast<long long>(b) * C + c) * a.Hq + whq)
+                                    : -INFINITY;
+                    }
+                    if (lane == 0) {  // lane 0 of warp w loads parts w, w + 8
+                        asm volatile("fence.proxy.async.global;" ::: "memory");  // the parts, seen through the counter
+                        if (warp == 0) mbar_arrive_expect_tx(m_full, static_cast<uint32_t>(C) * 8192u);
+                        for (int c = warp; c < C; c += SP_GW)
                             tma_load_3d(mbuf + c * 8192, &tm_pm, m_full, 64 * cb, 64 * hb, b * C + c);
                     }
-                    for (int x = t; x < C * 64; x += SP_GT) {
-                        const int c = x >> 6, hh = 64 * hb + (x & 63);
-                        mlse[x] = hh < a.Hq ? __ldcg(a.part_lse + (static_cast<long long>(b) * C + c) * a.Hq + hh) : 0.f;
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < SP_MAXC / 4; ++i) M = fmaxf(M, lv[i]);
+                    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 1));
+                    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 2));
+                    const float Mu = M == -INFINITY ? 0.f : M;
+                    float L = 0.f;
+#pragma unroll
+                    for (int i = 0; i < SP_MAXC / 4; ++i) {
+                        lv[i] = fast_exp2(lv[i] - Mu);
+                        L += lv[i];
                     }
-                    named_bar_sync(1, SP_GT);  // mlse written
+                    L += __shfl_xor_sync(0xffffffffu, L, 1);
+                    L += __shfl_xor_sync(0xffffffffu, L, 2);
+                    const float winv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+                    for (int i = 0; i < SP_MAXC / 4; ++i)
+                        if (wq + 4 * i < C) mw[(wq + 4 * i) * 64 + wh] = lv[i] * winv;
+                    if (cb == 0 && wq == 0 && whq < a.Hq && a.lse)
+                        a.lse[static_cast<long long>(b) * a.Hq + whq] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+                    named_bar_sync(1, SP_GT);  // the weights are written
                     if (!warp_wait(m_full, n_t & 1, s_abort)) break;
                     for (int it = t; it < 64 * 8; it += SP_GT) {
                         const int hh = it >> 3, ch = it & 7, hq = 64 * hb + hh;
                         if (hq >= a.Hq) continue;
-                        float M = -INFINITY;
-                        for (int c = 0; c < C; ++c) M = fmaxf(M, mlse[c * 64 + hh]);
-                        const float Mu = M == -INFINITY ? 0.f : M;
-                        float L = 0.f;
                         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
                         for (int c = 0; c < C; ++c) {
-                            const float wc = fast_exp2(mlse[c * 64 + hh] - Mu);
-                            L += wc;
+                            const float wc = mw[c * 64 + hh];
+                            const float2 w2 = make_float2(wc, wc);
                             const uint4 o = *reinterpret_cast<const uint4*>(mbuf + c * 8192 + swz128(hh, ch));
                             const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                acc[2 * i] = fmaf(wc, bf16_lo(w4[i]), acc[2 * i]);
-                                acc[2 * i + 1] = fmaf(wc, bf16_hi(w4[i]), acc[2 * i + 1]);
+                                const float2 r = __ffma2_rn(w2, make_float2(bf16_lo(w4[i]), bf16_hi(w4[i])),
+                                                            make_float2(acc[2 * i], acc[2 * i + 1]));
+                                acc[2 * i] = r.x;
+                                acc[2 * i + 1] = r.y;
                             }
                         }
-                        const float inv = L > 0.f ? 1.f / L : 0.f;
                         const long long ob = (static_cast<long long>(b) * a.Hq + hq) * SP_DV + 64 * cb + 8 * ch;
                         *reinterpret_cast<uint4*>(a.out + ob) =
-                            make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
-                                       pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
-                        if (cb == 0 && ch == 0 && a.lse)
-                            a.lse[static_cast<long long>(b) * a.Hq + hq] = L > 0.f ? (Mu + __log2f(L)) * kLn2 : -INFINITY;
+                            make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
                     }
                     named_bar_sync(1, SP_GT);  // the buffers are read before the next tile's loads
                 }
-                named_bar_sync(1, SP_GT);  // this CTA's reads of the parts are done
-                if (t == 0) {
-                    __threadfence();
-                    if (atomicAdd(a.row_done + b, 1) == a.chunks - 1) {  // the row's last: leave the counters zero
-                        a.row_arrive[b] = 0;
-                        a.row_done[b] = 0;
-                    }
+                if (t == 32 && past == C - 1) {
+                    a.row_arrive[b] = 0;
+                    a.row_done[b] = 0;
                 }
             }
         }
