@@ -596,10 +596,9 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     uint32_t prefix = 0u, known = 0u;
     int k_rem = kk;
     if (len > a.k) {
-        const int shifts[3] = {21, 10, 0};
-        const int widths[3] = {11, 11, 10};
         for (int p = 0; p < 3; ++p) {
-            const int sh = shifts[p], nb = 1 << widths[p];
+            // digits of 11, 11 and 10 bits from the top
+            const int sh = p == 0 ? 21 : (p == 1 ? 10 : 0), nb = p == 2 ? 1024 : 2048;
             // Pass p clears and fills buffer p & 1.  Buffer p & 1 was last read by the other CTAs in
             // pass p - 2, before they reached pass p - 1's cluster barrier, which this CTA has passed:
             // one cluster barrier per pass suffices.
