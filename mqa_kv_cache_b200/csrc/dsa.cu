@@ -204,6 +204,9 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 return true;
             };
             bool ok = true;
+            // the keys are read once: evict them from L2 first, so that the scores (and their
+            // histograms) this kernel writes are still there for the top-k
+            const uint64_t k_pol = l2_evict_first_policy();
             const int n_rows = ix_rows(cta, G, a.B);
             for (int r = 0; ok && r < n_rows && !*s_abort; ++r) {
                 const int b = ix_row(cta, G, a.B, r);
@@ -233,7 +236,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                         mbar_arrive_expect_tx(&full[s], C::TILE);
                         uint8_t* dst = smem + s * C::TILE;
 #pragma unroll
-                        for (int i = 0; i < C::KBOX; ++i) tma_load_3d(dst + i * IX_BOX, &tm_k, &full[s], 64 * i, t * IX_TOK, b);
+                        for (int i = 0; i < C::KBOX; ++i)
+                            tma_load_3d_hint(dst + i * IX_BOX, &tm_k, &full[s], 64 * i, t * IX_TOK, b, k_pol);
                     }
                     if (!ok) break;
                     t0 = atomicAdd(a.row_ctr + b, IX_CLAIM);
