@@ -458,7 +458,7 @@ __global__ void __launch_bounds__(SP_THREADS, 1)
                 if (a.lse) a.lse[static_cast<long long>(b) * a.Hq + h] = lse2 * kLn2;
             } else {
                 a.part_lse[(static_cast<long long>(b) * a.chunks + chunk) * a.Hq + h] = lse2;
-                __threadfence();  // before half 0 counts itself on the row's counter
+                __threadfence();  // before warps 0-3 count their boxes on the row's counter
             }
         }
 
