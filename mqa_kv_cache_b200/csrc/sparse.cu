@@ -769,11 +769,15 @@ cudaError_t launch_sparse_attn(const SparseLaunch& l, const CUtensorMap& tm_q, c
         cfg.blockDim = dim3(SP_THREADS);
         cfg.dynamicSmemBytes = SP_SMEM;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
+        // cooperative (the row's CTAs wait for each other) and, like the other kernels, a
+        // programmatic dependent of the previous launch (its prologue overlaps that one's tail)
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeCooperative;
         attr[0].val.cooperative = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         return l.fp8 ? cudaLaunchKernelEx(&cfg, sparse_attn_kernel<true>, tm_q, tm_o, tm_pm, a)
                      : cudaLaunchKernelEx(&cfg, sparse_attn_kernel<false>, tm_q, tm_o, tm_pm, a);
     }
