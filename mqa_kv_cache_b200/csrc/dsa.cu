@@ -210,11 +210,14 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
             const int n_rows = ix_rows(cta, G, a.B);
             for (int r = 0; ok && r < n_rows && !*s_abort; ++r) {
                 const int b = ix_row(cta, G, a.B, r);
-                if (r > 0 && __ldcg(a.row_ctr + b) >= a.tiles_per_b) continue;  // nothing left there
+                // the row's tiles up to its length (the epilogue writes -inf past it within the last)
+                const int len_raw = a.seq_lens ? (__ldg(a.seq_lens + b) >> a.len_shift) : a.L_max;
+                const int T = (min(max(len_raw, 0), a.L_max) + IX_TOK - 1) / IX_TOK;
+                if (r > 0 && __ldcg(a.row_ctr + b) >= T) continue;  // nothing left there
                 // the first claim comes before the row's query heads: a row this CTA gets no tiles of
                 // loads nothing and hands out nothing (every query load is waited for by the MMA)
                 int t0 = atomicAdd(a.row_ctr + b, IX_CLAIM);
-                if (t0 >= a.tiles_per_b) continue;
+                if (t0 >= T) continue;
                 // the row's query heads, once the S MMAs of the previous row are done with its own
                 if (nq > 0 && !mbar_wait(q_empty, (nq - 1) & 1)) {
                     ok = false;
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                 for (int i = 0; i < C::KBOX; ++i) tma_load_3d(smem + C::OFF_Q + i * IX_QBOX, &tm_q, q_full, 64 * i, 0, b);
                 ++nq;
                 while (ok) {
-                    const int t1 = min(t0 + IX_CLAIM, a.tiles_per_b);
+                    const int t1 = min(t0 + IX_CLAIM, T);
                     if (!(ok = push(b, t0, t1))) break;
                     for (int t = t0; t < t1; ++t, ++it) {
                         const int s = it % C::STAGES;
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
                     }
                     if (!ok) break;
                     t0 = atomicAdd(a.row_ctr + b, IX_CLAIM);
-                    if (t0 >= a.tiles_per_b) break;
+                    if (t0 >= T) break;
                 }
                 if (ok) ok = push(b, 0, 0);  // row b closed
             }
@@ -505,6 +508,7 @@ struct TopkArgs {
     int32_t* tok_count;
     int L_tok;
     int* row_ctr;        // [B] the indexer's claim counters: cleared here for the next call (null: none)
+    float* fill;         // scores, writable: -inf is written past each row's length (null: none)
 };
 
 constexpr int TK_SLICE_MAX = 16384;  // keys per CTA held in shared memory
@@ -568,6 +572,12 @@ __global__ void __launch_bounds__(TK_THREADS, 1) topk_kernel(TopkArgs a)
     const int lo = min(rank * slice, len), hi = min(lo + slice, len);
     const int n_mine = hi - lo;
     const float* sc = a.scores + static_cast<long long>(row) * a.L_max;
+    if (a.fill) {
+        // the indexer scored whole tiles up to the length only: the rest of the row is -inf (in
+        // the workspace nothing reads it; a caller's scores_out gets -inf past the length)
+        float* f = a.fill + static_cast<long long>(row) * a.L_max;
+        for (int i = len + rank * TK_THREADS + tid; i < a.L_max; i += TK_CL * TK_THREADS) f[i] = -INFINITY;
+    }
     if (tid == 0) s_nan = 0;
     bool nan = false;
     // the candidate counter in rank 0 is zero before any CTA of the cluster counts into it
@@ -1009,7 +1019,7 @@ cudaError_t launch_dsa_index_topk(const DsaIndexArgs& a, const CUtensorMap& tm_k
     if (e != cudaSuccess) return e;
 
     TopkArgs ta{a.scores, a.seq_lens, a.hist, a.tok_idx ? nullptr : a.topk_idx, a.dev_status, a.L_max, a.k,
-                a.len_shift, a.tok_idx, a.tok_count, a.L_tok, ia.row_ctr};
+                a.len_shift, a.tok_idx, a.tok_count, a.L_tok, ia.row_ctr, a.scores};
     const size_t key_bytes = static_cast<size_t>(slice_words(a.L_max) + 2 * TK_CAND_MAX) * sizeof(uint32_t);
     static bool tk_attr[64] = {};
     if (dev < 64 && !tk_attr[dev]) {
