@@ -102,14 +102,14 @@ struct IndexerArgs {
     uint32_t* hist;       // [B][2048] first-digit counts of the valid scores (added to; zero on entry)
     int* row_ctr;         // [B] key tiles of each row claimed so far (zero on entry; the top-k clears them)
     int32_t* dev_status;
-    int B, L_max, tiles_per_b;
+    int B, L_max, tiles_per_b;  // tiles_per_b: tiles of a full row (L_max); a row's claims stop at its length
     int len_shift;  // row b scores seq_lens[b] >> len_shift keys (2: 4-token groups)
 };
 
 // Rows served by CTA c of G: with G >= B the CTAs are split over the rows (row c B / G),
-// each row's tiles claimed IX_CLAIM at a time from its counter by whichever of its CTAs
-// is ready, so that faster CTAs take more (going on to other rows once a row is done
-// was measured slower); with G < B, rows c, c + G, ...
+// each row's tiles (up to its length) claimed IX_CLAIM at a time from its counter by
+// whichever of its CTAs is ready, so that faster CTAs take more (going on to other rows
+// once a row is done was measured slower); with G < B, rows c, c + G, ...
 __device__ __forceinline__ int ix_rows(int c, int G, int B) { return G >= B ? 1 : (B - c + G - 1) / G; }
 __device__ __forceinline__ int ix_row(int c, int G, int B, int r)
 {
