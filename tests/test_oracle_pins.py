@@ -412,6 +412,45 @@ def test_prefill_row_equals_decode_over_prefix():
     np.testing.assert_array_equal(o[1], out[0, 0, 0])
 
 
+def _textbook_attention(q, k, v, scale, mask):
+    """A second, independent statement of grouped-query attention in fp64 torch
+    ("注意力变体与 MoE", attention(); "attention", GroupQueryAttention): K/V heads
+    repeated g times along the head axis (query head h reads KV head h // g),
+    scores = scale q k^T, masked entries -inf, softmax over keys, weights @ V.
+    q [B, H, Tq, d]; k, v [B, Hk, Tk, d]; mask [B, Tq, Tk] True = hidden.
+    A cross-check of the C oracle on tiny shapes, not a pin."""
+    g = q.shape[1] // k.shape[1]
+    kr = torch.repeat_interleave(k, g, dim=1)
+    vr = torch.repeat_interleave(v, g, dim=1)
+    s = torch.einsum("bhqd,bhkd->bhqk", q, kr) * scale
+    s = s.masked_fill(mask[:, None], float("-inf"))
+    lse = torch.logsumexp(s, dim=-1)
+    return torch.einsum("bhqk,bhkd->bhqd", torch.softmax(s, dim=-1), vr), lse
+
+
+def test_decode_matches_a_textbook_statement():
+    B, H, Hk, T, d = 3, 8, 2, 40, 16
+    q, k, v = _bf16_bits((B, H, d), 11), _bf16_bits((B, Hk, T, d), 12), _bf16_bits((B, Hk, T, d), 13)
+    lens = np.array([40, 17, 1], np.int32)
+    out, lse = oracle.attn_decode(q, k, v, lens, 0.25)
+    f = lambda bits: torch.from_numpy(oracle.bf16_bits_to_f64(bits))
+    mask = torch.arange(T)[None, None, :] >= torch.from_numpy(lens)[:, None, None]
+    ro, rl = _textbook_attention(f(q)[:, :, None], f(k), f(v), 0.25, mask)
+    np.testing.assert_allclose(out, ro[:, :, 0].numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl[:, :, 0].numpy(), rtol=0, atol=1e-12)
+
+
+def test_prefill_matches_a_textbook_statement():
+    B, T, H, Hk, d = 2, 24, 4, 1, 8
+    q, k, v = _bf16_bits((B, T, H, d), 14), _bf16_bits((B, Hk, T, d), 15), _bf16_bits((B, Hk, T, d), 16)
+    out, lse = oracle.attn_prefill(q, k, v, 0.3)
+    f = lambda bits: torch.from_numpy(oracle.bf16_bits_to_f64(bits))
+    causal = torch.triu(torch.ones(T, T, dtype=torch.bool), diagonal=1).expand(B, T, T)
+    ro, rl = _textbook_attention(f(q).permute(0, 2, 1, 3), f(k), f(v), 0.3, causal)
+    np.testing.assert_allclose(out, ro.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, rl.numpy(), rtol=0, atol=1e-12)
+
+
 # --------------------------------------------------------------------------
 # Lightning indexer and top-k ("Agentic RL 入门3" §2.2 (1)(2); "attention" DSA ①)
 # --------------------------------------------------------------------------
